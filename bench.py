@@ -1,0 +1,381 @@
+#!/usr/bin/env python
+"""Batch-1 decode benchmark of the persistent megakernel on B200.
+
+One "step" is one decode step (one token) of the configured workload: the
+Llama-3.2-1B-shaped random-init model with its KV cache pre-filled to 1024
+positions, decoding positions 1024..1151 (cycled when more steps are timed).
+Prints ONE JSON line (rank 0):
+  value            device-timed µs/token (CUDA events around K back-to-back
+                   launches on the launching stream, token fed on the device),
+                   whole job: max-over-ranks time / (K * ranks)
+  e2e              the same metric through the C ABI with a host round trip
+                   per step (token in by value, next token + status read back
+                   from device to pinned host memory, synchronised)
+  roofline         algorithmic bytes per token / mean launch duration vs the
+                   measured HBM copy bandwidth
+  cpu_baseline     the fp64 oracle on this host's cores, bounded sample
+  baselines        the plain multi-kernel path of the same opcodes, stream
+                   launches and a CUDA graph
+`--impl reference` times the fp64 oracle instead (rank 0 only).
+Multi-GPU (torchrun): independent replicas, one per GPU, no collective on the
+data path ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "batch-1 decode µs/token and achieved HBM GB/s vs ~8 TB/s roofline (1×B200)"
+UNIT = "µs/token"
+ROOFLINE_NOMINAL_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1280)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="llama1b")
+    ap.add_argument("--mode", default="megakernel", choices=["megakernel", "multi_kernel", "multi_kernel_graph"])
+    ap.add_argument("--layers", type=int, default=0, help="override n_layers (profiling small cases only)")
+    ap.add_argument("--l2-prefetch", type=int, default=-1)
+    ap.add_argument("--ring-stages", type=int, default=0)
+    ap.add_argument("--stage-bytes", type=int, default=0)
+    ap.add_argument("--kv-splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-baselines", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ---- process group (replicas) ---------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- clocks during the timed region ---------------------------------------------------------------
+
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if not self.proc:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit()),
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows
+                                                          if r[3].replace(".", "").isdigit()),
+                "reasons": reasons}
+
+
+# ---- measured peaks and committed ncu traffic ---------------------------------------------------------
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        v = float(json.load(open(p))["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "decode_persistent_block_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(f.encode())
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(config: str, mode: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(p))
+        e = d[f"{mode}:{config}"]
+        if e.get("kernel_hash") == kernel_source_hash():
+            return e["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+# ---- workload ---------------------------------------------------------------------------------------
+
+def workload(args):
+    from synth import configs
+    cfg = configs.get(args.config)
+    if args.layers:
+        cfg = cfg.with_(name=f"{cfg.name}_L{args.layers}", n_layers=args.layers)
+    p0 = cfg.prefill + cfg.prompt_len
+    positions = [p0 + (i % cfg.steps) for i in range(max(args.steps, args.warmup) + 1)]
+    return cfg, p0, positions
+
+
+def oracle_steps(cfg, seconds: float, max_steps: int | None = None):
+    """Time the fp64 oracle on consecutive decode positions for about `seconds`."""
+    import oracle
+    import synth
+    W = synth.make_model(cfg)
+    kc, vc = synth.make_kv_cache(cfg)
+    orc = oracle.Model(cfg, W, kc, vc)
+    p0 = cfg.prefill + cfg.prompt_len
+    tok = int(synth.prompt_tokens(cfg)[0])
+    times = []
+    t_start = time.perf_counter()
+    i = 0
+    while True:
+        t0 = time.perf_counter()
+        tok = orc.step(tok, p0 + (i % cfg.steps), want_hidden=False)["next"]
+        times.append(time.perf_counter() - t0)
+        i += 1
+        if max_steps is not None and i >= max_steps:
+            break
+        if max_steps is None and time.perf_counter() - t_start >= seconds and i >= 2:
+            break
+    return times, oracle.num_threads()
+
+
+def bytes_per_token(cfg, positions):
+    return cfg.weight_bytes_per_token() + statistics.fmean(cfg.kv_bytes_per_token(p) for p in positions)
+
+
+# ---- our arm --------------------------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local):
+    import numpy as np
+    import torch
+
+    import synth
+    from decode_persistent_block_b200 import Decoder, to_device
+    torch.cuda.set_device(local)
+    cfg, p0, positions = workload(args)
+    W = synth.make_model(cfg)
+    kc, vc = synth.make_kv_cache(cfg)
+    dW = to_device(W)
+    dk = torch.from_numpy(kc.view(np.int16)).cuda()
+    dv = torch.from_numpy(vc.view(np.int16)).cuda()
+    first = int(synth.prompt_tokens(cfg)[0])
+    mode = {"megakernel": 0, "multi_kernel": 1, "multi_kernel_graph": 2}[args.mode]
+    opts = dict(mode=mode, l2_prefetch=args.l2_prefetch, ring_stages=args.ring_stages,
+                stage_bytes=args.stage_bytes, kv_splits=args.kv_splits)
+    dec = Decoder(cfg, dW, dk, dv, **opts)
+    K, Wm = args.steps, args.warmup
+
+    def timed(d, k, warm):
+        d.step(first, positions[0])
+        for i in range(1, warm):
+            d.step(-1, positions[i], sync=False)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(k):
+            evs[i][0].record(stream)
+            d.step(-1, positions[i % len(positions)], sync=False)
+            evs[i][1].record(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        st = d.status()
+        if st["code"] != 0:
+            raise RuntimeError(f"device status after timed steps: {st}")
+        return e0.elapsed_time(e1), [a.elapsed_time(b) for a, b in evs]
+
+    clocks = Clocks(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
+                    if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local)
+    clocks.start()
+    total_ms, per_launch = timed(dec, K, Wm)
+    clk = clocks.stop()
+    total_ms = reduce_max(total_ms, world)
+    us_per_token = total_ms * 1000.0 / (K * world)
+    launch_ms = statistics.fmean(per_launch)
+    bpt = bytes_per_token(cfg, [positions[i % len(positions)] for i in range(K)])
+    peak, peak_kind = hbm_peak()
+    achieved = bpt / (launch_ms * 1e-3) / 1e9
+
+    # e2e through the C ABI: token in by value, next token + status back to pinned host memory, per step
+    e2e = None
+    if not args.no_e2e:
+        tok = dec.step(first, positions[0])
+        torch.cuda.synchronize()
+        barrier(world)
+        t0 = time.perf_counter()
+        for i in range(K):
+            tok = dec.step(tok, positions[i % len(positions)])
+        t1 = time.perf_counter()
+        e2e_s = reduce_max(t1 - t0, world)
+        e2e = {"value": round(e2e_s * 1e6 / (K * world), 3), "unit": UNIT, "h2d_bytes_per_step": 4,
+               "d2h_bytes_per_step": 64}
+
+    baselines = {}
+    if not args.no_baselines and args.mode == "megakernel":
+        for name, m in (("multi_kernel", 1), ("multi_kernel_graph", 2)):
+            with Decoder(cfg, dW, dk, dv, mode=m) as b:
+                kb = min(K, 128)
+                tms, _ = timed(b, kb, 3)
+                baselines[name] = round(reduce_max(tms, world) * 1000.0 / (kb * world), 3)
+    dec.close()
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        times, cores = oracle_steps(cfg, args.cpu_seconds)
+        cpu = {"value": round(statistics.fmean(times) * 1e6, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{len(times)} fp64 oracle decode steps of {cfg.name} at positions {p0}..",
+               "ms_per_token": round(statistics.fmean(times) * 1e3, 2)}
+
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": round(us_per_token, 3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": round(us_per_token * world / 1000.0, 6), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 weights/KV, fp32 accumulate",
+        "data": "synthetic random-init weights and KV prefill (seeded generator)",
+        "config": {"workload": f"{cfg.name}: batch-1 greedy decode, KV pre-filled to {cfg.prefill}, positions "
+                               f"{p0}..{p0 + cfg.steps - 1}", "layers": cfg.n_layers, "hidden": cfg.hidden,
+                   "vocab": cfg.vocab, "mode": args.mode, "parallelism": f"replicas x{world}",
+                   "l2": f"no flush: {bpt / 1e9:.2f} GB streamed per token > 126 MB L2"},
+        "tokens_per_s": round(1e6 / us_per_token, 1),
+        "hbm_gbs": round(achieved, 1),
+        "frac_of_8tbs": round(achieved / ROOFLINE_NOMINAL_GBS, 4),
+        "bytes_per_token": int(bpt),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+                     "traffic": committed_traffic(cfg.name, args.mode), "launch_us": round(launch_ms * 1000, 2)},
+        "e2e": e2e,
+        "gpu_launches": K if args.mode == "megakernel" else None,
+        "baselines": baselines,
+        "cpu_baseline": cpu,
+        "clocks": clk,
+    }
+    if args.mode != "megakernel":
+        per_step = 6 * cfg.n_layers + 3 + (cfg.n_layers * cfg.top_k if cfg.n_experts else 0)
+        line["gpu_launches"] = K * (per_step + 1)
+    return line
+
+
+# ---- reference arm: the fp64 oracle on the host cores ---------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cfg, p0, positions = workload(args)
+    times, cores = oracle_steps(cfg, 0, max_steps=args.warmup + args.steps)
+    t = times[args.warmup:]
+    v = statistics.fmean(t) * 1e6
+    sample = f"{len(t)} fp64 oracle decode steps of {cfg.name} at positions {p0}.. after {args.warmup} warm-up"
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v / 1000.0, 3),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic random-init weights and KV prefill (seeded generator)",
+            "config": {"workload": f"{cfg.name}: batch-1 greedy decode, KV pre-filled to {cfg.prefill}, positions "
+                                   f"{p0}..{p0 + cfg.steps - 1}", "layers": cfg.n_layers, "hidden": cfg.hidden,
+                       "vocab": cfg.vocab, "mode": "fp64 CPU oracle"},
+            "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_ours(args, rank, world, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,499 @@
+// mk_api.cu -- the C ABI (include/mk.h): handle lifetime, device buffers,
+// schedule upload, the step launch with a host-side watchdog, fault injection
+// and the debug getters.
+#include <cuda_runtime.h>
+
+#include <chrono>
+#include <cmath>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#include "mk_internal.h"
+#include "mk_kernels.h"
+#include "mk_plan.h"
+
+struct mk_handle {
+    mk_config cfg;
+    mk_options opt;
+    cudaStream_t stream = nullptr;
+    int device = 0;
+    int n_sm = 0;
+    mk::DevParams p;
+    std::vector<const uint16_t*> wt_host;
+    std::vector<void*> allocs;
+    mk::Planned plan;
+    bool scheduled = false;
+    uint32_t epoch = 0;
+    mk::StepBuf* stepbuf = nullptr;
+    mk::DevStatus* status_pinned = nullptr;
+    cudaEvent_t ev0 = nullptr, ev1 = nullptr, ev_done = nullptr;
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t graph_exec = nullptr;
+    int lm_slots = 0;
+    int last_cuda = 0;
+    int last_error = MK_OK;
+};
+
+namespace {
+
+int cuda_fail(mk_handle* h, cudaError_t e) {
+    if (h) h->last_cuda = (int)e;
+    return MK_ERR_CUDA;
+}
+
+#define CK(expr)                                   \
+    do {                                           \
+        cudaError_t e_ = (expr);                   \
+        if (e_ != cudaSuccess) return cuda_fail(h, e_); \
+    } while (0)
+
+template <class T>
+int dalloc(mk_handle* h, T** out, size_t count) {
+    void* ptr = nullptr;
+    const size_t bytes = count * sizeof(T) > 0 ? count * sizeof(T) : 16;
+    cudaError_t e = cudaMalloc(&ptr, bytes);
+    if (e != cudaSuccess) return cuda_fail(h, e);
+    e = cudaMemset(ptr, 0, bytes);
+    if (e != cudaSuccess) {
+        cudaFree(ptr);
+        return cuda_fail(h, e);
+    }
+    h->allocs.push_back(ptr);
+    *out = static_cast<T*>(ptr);
+    return MK_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_weights(const mk_config& c, const mk_weights* w) {
+    if (!w || !w->embed || !w->lm_head || !w->final_norm || !w->k_cache || !w->v_cache) return MK_ERR_INVALID_ARG;
+    if (!aligned16(w->embed) || !aligned16(w->lm_head) || !aligned16(w->final_norm) || !aligned16(w->k_cache) ||
+        !aligned16(w->v_cache))
+        return MK_ERR_INVALID_ARG;
+    const int L = c.n_layers;
+    const int ne = c.n_experts > 0 ? L * c.n_experts : L;
+    const void* const* per_layer[] = {w->attn_norm, w->wq, w->wk, w->wv, w->wo, w->ffn_norm};
+    for (auto arr : per_layer) {
+        if (L > 0 && !arr) return MK_ERR_INVALID_ARG;
+        for (int l = 0; l < L; ++l)
+            if (!arr[l] || !aligned16(arr[l])) return MK_ERR_INVALID_ARG;
+    }
+    const void* const* per_expert[] = {w->w_gate, w->w_up, w->w_down};
+    for (auto arr : per_expert) {
+        if (ne > 0 && !arr) return MK_ERR_INVALID_ARG;
+        for (int i = 0; i < ne; ++i)
+            if (!arr[i] || !aligned16(arr[i])) return MK_ERR_INVALID_ARG;
+    }
+    if (c.n_experts > 0) {
+        if (L > 0 && !w->router) return MK_ERR_INVALID_ARG;
+        for (int l = 0; l < L; ++l)
+            if (!w->router[l] || !aligned16(w->router[l])) return MK_ERR_INVALID_ARG;
+    }
+    return MK_OK;
+}
+
+int upload_schedule(mk_handle* h) {
+    CK(cudaMemcpy(const_cast<int32_t*>(h->p.instr), h->plan.words.data(), h->plan.words.size() * sizeof(int32_t),
+                  cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(const_cast<int32_t*>(h->p.n_instr), h->plan.n_instr.data(), h->plan.n_instr.size() * sizeof(int32_t),
+                  cudaMemcpyHostToDevice));
+    return MK_OK;
+}
+
+// Wait for the step's completion event with a deadline (host-side watchdog,
+// the backstop behind the kernel's own bounded waits).
+int wait_event(mk_handle* h, cudaEvent_t ev) {
+    const double limit_s = std::max(10.0, 4.0 * (double)h->opt.spin_limit_ns * 1e-9);
+    const auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+        const cudaError_t e = cudaEventQuery(ev);
+        if (e == cudaSuccess) return MK_OK;
+        if (e != cudaErrorNotReady) return cuda_fail(h, e);
+        if (std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count() > limit_s)
+            return MK_ERR_TIMEOUT;
+        std::this_thread::yield();
+    }
+}
+
+int read_status(mk_handle* h, mk::DevStatus* out) {
+    CK(cudaMemcpyAsync(h->status_pinned, h->p.status, sizeof(mk::DevStatus), cudaMemcpyDeviceToHost, h->stream));
+    CK(cudaEventRecord(h->ev_done, h->stream));
+    int rc = wait_event(h, h->ev_done);
+    if (rc) return rc;
+    *out = *h->status_pinned;
+    return MK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void mk_default_options(mk_options* o) {
+    if (!o) return;
+    std::memset(o, 0, sizeof(*o));
+    o->l2_prefetch = -1;
+    o->mode = MK_MODE_MEGAKERNEL;
+}
+
+const char* mk_strerror(int code) {
+    switch (code) {
+        case MK_OK: return "ok";
+        case MK_ERR_INVALID_ARG: return "invalid argument";
+        case MK_ERR_CUDA: return "CUDA runtime error";
+        case MK_ERR_NOT_RESIDENT: return "persistent grid cannot be co-resident";
+        case MK_ERR_TIMEOUT: return "bounded device wait timed out";
+        case MK_ERR_BAD_INSTR: return "bad instruction or index";
+        case MK_ERR_SCHEDULE: return "schedule rejected by the validator";
+        case MK_ERR_STOPPED: return "stop word set";
+        case MK_ERR_NO_SCHEDULE: return "no schedule built";
+        case MK_ERR_CAPACITY: return "buffer too small";
+        case MK_ERR_UNSUPPORTED: return "unsupported shape";
+    }
+    return "unknown error";
+}
+
+int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, void* cuda_stream, mk_handle** out) {
+    if (!cfg || !out) return MK_ERR_INVALID_ARG;
+    *out = nullptr;
+    int rc = mk::check_config(*cfg);
+    if (rc) return rc;
+    rc = check_weights(*cfg, w);
+    if (rc) return rc;
+    mk_options o;
+    if (opt) o = *opt; else mk_default_options(&o);
+    mk::fill_defaults(&o);
+    rc = mk::check_options(*cfg, o);
+    if (rc) return rc;
+
+    mk_handle* h = new mk_handle();
+    h->cfg = *cfg;
+    h->opt = o;
+    h->stream = static_cast<cudaStream_t>(cuda_stream);
+    auto fail = [&](int code) {
+        mk_destroy(h);
+        return code;
+    };
+    cudaError_t e = cudaGetDevice(&h->device);
+    if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
+    int dev_sms = 0, coop = 0;
+    cudaDeviceGetAttribute(&dev_sms, cudaDevAttrMultiProcessorCount, h->device);
+    cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, h->device);
+    if (dev_sms <= 0) return fail(MK_ERR_CUDA);
+    h->n_sm = (o.n_sm > 0 && o.n_sm < dev_sms) ? o.n_sm : dev_sms;
+
+    const mk_config& c = *cfg;
+    const int L = c.n_layers, H = c.hidden, d = c.head_dim, nq = c.n_q_heads, nkv = c.n_kv_heads;
+    const int S = o.kv_splits > 0 ? o.kv_splits : mk::default_kv_splits(c, h->n_sm);
+    const int E = c.n_experts, topk = E > 0 ? c.top_k : 1;
+    mk::DevParams& p = h->p;
+    std::memset(&p, 0, sizeof(p));
+    p.L = L; p.H = H; p.nq = nq; p.nkv = nkv; p.d = d; p.F = c.ffn; p.V = c.vocab; p.E = E;
+    p.topk = E > 0 ? c.top_k : 0; p.max_seq = c.max_seq; p.eps = c.rms_eps; p.kv_splits = S;
+    p.n_ctr = mk::n_counters(L, nkv);
+    p.embed = static_cast<const uint16_t*>(w->embed);
+    p.lm_head = static_cast<const uint16_t*>(w->lm_head);
+    p.final_norm = static_cast<const uint16_t*>(w->final_norm);
+    p.kcache = static_cast<uint16_t*>(w->k_cache);
+    p.vcache = static_cast<uint16_t*>(w->v_cache);
+    p.ring_stages = o.ring_stages;
+    p.stage_bytes = o.stage_bytes;
+    p.l2_prefetch = o.l2_prefetch;
+    p.spin_limit_ns = o.spin_limit_ns;
+
+    // weight pointer table
+    const int stride = mk::wt_stride(E);
+    h->wt_host.assign((size_t)std::max(L, 1) * stride, nullptr);
+    for (int l = 0; l < L; ++l) {
+        const uint16_t** t = &h->wt_host[(size_t)l * stride];
+        t[mk::WT_ATTN_NORM] = static_cast<const uint16_t*>(w->attn_norm[l]);
+        t[mk::WT_Q] = static_cast<const uint16_t*>(w->wq[l]);
+        t[mk::WT_K] = static_cast<const uint16_t*>(w->wk[l]);
+        t[mk::WT_V] = static_cast<const uint16_t*>(w->wv[l]);
+        t[mk::WT_O] = static_cast<const uint16_t*>(w->wo[l]);
+        t[mk::WT_FFN_NORM] = static_cast<const uint16_t*>(w->ffn_norm[l]);
+        t[mk::WT_ROUTER] = E > 0 ? static_cast<const uint16_t*>(w->router[l]) : nullptr;
+        const int ne = E > 0 ? E : 1;
+        for (int x = 0; x < ne; ++x) {
+            const size_t src = E > 0 ? (size_t)l * E + x : (size_t)l;
+            t[mk::wt_gate(x)] = static_cast<const uint16_t*>(w->w_gate[src]);
+            t[mk::wt_up(x, E)] = static_cast<const uint16_t*>(w->w_up[src]);
+            t[mk::wt_down(x, E)] = static_cast<const uint16_t*>(w->w_down[src]);
+        }
+    }
+    const uint16_t** wt_dev = nullptr;
+    const int lm_slots = std::max(h->n_sm + c.vocab / mk::kMaxRows + 1, mk::baseline_lm_blocks(p, h->n_sm));
+    h->lm_slots = lm_slots;
+    if ((rc = dalloc(h, &wt_dev, h->wt_host.size()))) return fail(rc);
+    if ((rc = dalloc(h, &p.counters, (size_t)p.n_ctr))) return fail(rc);
+    if ((rc = dalloc(h, &p.status, 1))) return fail(rc);
+    if ((rc = dalloc(h, &p.x, (size_t)H))) return fail(rc);
+    if ((rc = dalloc(h, &p.qkv, (size_t)(nq + 2 * nkv) * d))) return fail(rc);
+    if ((rc = dalloc(h, &p.attn, (size_t)nq * d))) return fail(rc);
+    if ((rc = dalloc(h, &p.part_o, (size_t)nq * S * d))) return fail(rc);
+    if ((rc = dalloc(h, &p.part_ml, (size_t)nq * S * 2))) return fail(rc);
+    if ((rc = dalloc(h, &p.hbuf, (size_t)topk * c.ffn))) return fail(rc);
+    if ((rc = dalloc(h, &p.logits, (size_t)c.vocab))) return fail(rc);
+    if ((rc = dalloc(h, &p.lm_part, (size_t)lm_slots * 2))) return fail(rc);
+    if ((rc = dalloc(h, &p.router_idx, (size_t)std::max(L, 1) * mk::kMaxTopK))) return fail(rc);
+    if ((rc = dalloc(h, &p.router_w, (size_t)std::max(L, 1) * mk::kMaxTopK))) return fail(rc);
+    if (o.snapshots && (rc = dalloc(h, &p.snap, (size_t)(L + 1) * H))) return fail(rc);
+    float2* rope = nullptr;
+    if ((rc = dalloc(h, &rope, (size_t)c.max_seq * (d / 2)))) return fail(rc);
+    if ((rc = dalloc(h, &h->stepbuf, 1))) return fail(rc);
+    p.wt = wt_dev;
+    p.rope = rope;
+    e = cudaMemcpy(wt_dev, h->wt_host.data(), h->wt_host.size() * sizeof(void*), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
+
+    // RoPE table: angle = pos * theta^(-2i/d), evaluated in double
+    {
+        std::vector<float2> tab((size_t)c.max_seq * (d / 2));
+        for (int pos = 0; pos < c.max_seq; ++pos)
+            for (int i = 0; i < d / 2; ++i) {
+                const double a = (double)pos * std::pow((double)c.rope_theta, -2.0 * i / d);
+                tab[(size_t)pos * (d / 2) + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+            }
+        e = cudaMemcpy(rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
+    }
+
+    e = cudaMallocHost(&h->status_pinned, sizeof(mk::DevStatus));
+    if (e != cudaSuccess) { h->last_cuda = e; h->status_pinned = nullptr; return fail(MK_ERR_CUDA); }
+    if (cudaEventCreate(&h->ev0) || cudaEventCreate(&h->ev1) ||
+        cudaEventCreateWithFlags(&h->ev_done, cudaEventDisableTiming))
+        return fail(MK_ERR_CUDA);
+
+    if (o.mode == MK_MODE_MEGAKERNEL) {
+        int per_sm = 0;
+        e = mk::prepare_megakernel(o.ring_stages, o.stage_bytes, &per_sm);
+        if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
+        if (!coop || per_sm < 1) return fail(MK_ERR_NOT_RESIDENT);
+    } else {
+        e = mk::prepare_baseline();
+        if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
+    }
+    *out = h;
+    return MK_OK;
+}
+
+int mk_build_schedule(mk_handle* h) {
+    if (!h) return MK_ERR_INVALID_ARG;
+    mk::Planned plan;
+    int rc = mk::plan_schedule(h->cfg, h->opt, h->n_sm, &plan);
+    if (rc) return rc;
+    if (plan.kv_splits != h->p.kv_splits) return MK_ERR_SCHEDULE;
+    if (plan.n_lm > h->lm_slots) return MK_ERR_SCHEDULE;
+    h->plan = plan;
+    int32_t* words = nullptr;
+    int32_t* n_instr = nullptr;
+    if ((rc = dalloc(h, &words, plan.words.size()))) return rc;
+    if ((rc = dalloc(h, &n_instr, (size_t)plan.n_sm))) return rc;
+    h->p.instr = words;
+    h->p.n_instr = n_instr;
+    h->p.max_instr = plan.max_instr;
+    if (h->opt.trace) {
+        unsigned long long* tr = nullptr;
+        if ((rc = dalloc(h, &tr, (size_t)plan.n_sm * plan.max_instr * 4))) return rc;
+        h->p.trace = tr;
+    }
+    if ((rc = upload_schedule(h))) return rc;
+    h->scheduled = true;
+    return MK_OK;
+}
+
+int mk_get_schedule(mk_handle* h, int32_t* buf, size_t cap, size_t* n_words, int* n_sm, int* max_instr) {
+    if (!h) return MK_ERR_INVALID_ARG;
+    if (!h->scheduled) return MK_ERR_NO_SCHEDULE;
+    if (n_words) *n_words = h->plan.words.size();
+    if (n_sm) *n_sm = h->plan.n_sm;
+    if (max_instr) *max_instr = h->plan.max_instr;
+    if (!buf) return MK_OK;
+    if (cap < h->plan.words.size()) return MK_ERR_CAPACITY;
+    std::memcpy(buf, h->plan.words.data(), h->plan.words.size() * sizeof(int32_t));
+    return MK_OK;
+}
+
+int mk_decode_step(mk_handle* h, int32_t token, int32_t pos, float* logits_dev, int32_t* next_token_host) {
+    if (!h) return MK_ERR_INVALID_ARG;
+    if (token >= h->cfg.vocab || pos < 0 || pos >= h->cfg.max_seq) return MK_ERR_INVALID_ARG;
+    if (!h->scheduled) return MK_ERR_NO_SCHEDULE;
+    if (token < 0) token = -1;
+    h->epoch++;
+    mk::DevParams& p = h->p;
+    if (h->opt.mode == MK_MODE_MEGAKERNEL) {
+        mk::StepArgs a;
+        a.token = token;
+        a.pos = pos;
+        a.epoch = h->epoch;
+        a.logits = logits_dev ? logits_dev : p.logits;
+        CK(cudaEventRecord(h->ev0, h->stream));
+        CK(mk::launch_megakernel(p, a, h->n_sm, h->stream));
+        CK(cudaEventRecord(h->ev1, h->stream));
+    } else {
+        mk::BaselineShape bs{h->n_sm, mk::baseline_lm_blocks(p, h->n_sm)};
+        CK(mk::launch_baseline_set_step(p, h->stepbuf, token, pos, h->stream));
+        CK(cudaEventRecord(h->ev0, h->stream));
+        if (h->opt.mode == MK_MODE_MULTI_KERNEL_GRAPH) {
+            if (!h->graph_exec) {
+                cudaStream_t cap = nullptr;
+                CK(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
+                cudaError_t e = cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal);
+                if (e == cudaSuccess) {
+                    mk::launch_baseline_layers(p, h->wt_host.data(), h->stepbuf, bs, p.logits, cap);
+                    e = cudaStreamEndCapture(cap, &h->graph);
+                }
+                if (e == cudaSuccess) e = cudaGraphInstantiate(&h->graph_exec, h->graph, 0);
+                cudaStreamDestroy(cap);
+                if (e != cudaSuccess) return cuda_fail(h, e);
+            }
+            CK(cudaGraphLaunch(h->graph_exec, h->stream));
+        } else {
+            CK(mk::launch_baseline_layers(p, h->wt_host.data(), h->stepbuf, bs, p.logits, h->stream));
+        }
+        CK(cudaEventRecord(h->ev1, h->stream));
+        if (logits_dev)
+            CK(cudaMemcpyAsync(logits_dev, p.logits, sizeof(float) * h->cfg.vocab, cudaMemcpyDeviceToDevice,
+                               h->stream));
+    }
+    if (next_token_host) {
+        mk::DevStatus st;
+        int rc = read_status(h, &st);
+        if (rc) return rc;
+        if (st.code != MK_OK) return st.code;
+        *next_token_host = st.next_token;
+    }
+    return MK_OK;
+}
+
+int mk_get_hidden(mk_handle* h, int layer, float* out_host) {
+    if (!h || !out_host || layer < 0 || layer > h->cfg.n_layers || !h->p.snap) return MK_ERR_INVALID_ARG;
+    CK(cudaStreamSynchronize(h->stream));
+    CK(cudaMemcpy(out_host, h->p.snap + (size_t)layer * h->cfg.hidden, sizeof(float) * h->cfg.hidden,
+                  cudaMemcpyDeviceToHost));
+    return MK_OK;
+}
+
+int mk_get_router(mk_handle* h, int layer, int32_t* idx, float* wts) {
+    if (!h || !idx || !wts || h->cfg.n_experts <= 0 || layer < 0 || layer >= h->cfg.n_layers)
+        return MK_ERR_INVALID_ARG;
+    CK(cudaStreamSynchronize(h->stream));
+    CK(cudaMemcpy(idx, h->p.router_idx + (size_t)layer * mk::kMaxTopK, sizeof(int32_t) * h->cfg.top_k,
+                  cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(wts, h->p.router_w + (size_t)layer * mk::kMaxTopK, sizeof(float) * h->cfg.top_k,
+                  cudaMemcpyDeviceToHost));
+    return MK_OK;
+}
+
+int mk_get_counters(mk_handle* h, uint32_t* out, size_t cap, size_t* n) {
+    if (!h) return MK_ERR_INVALID_ARG;
+    if (n) *n = (size_t)h->p.n_ctr;
+    if (!out) return MK_OK;
+    if (cap < (size_t)h->p.n_ctr) return MK_ERR_CAPACITY;
+    CK(cudaStreamSynchronize(h->stream));
+    CK(cudaMemcpy(out, h->p.counters, sizeof(uint32_t) * h->p.n_ctr, cudaMemcpyDeviceToHost));
+    return MK_OK;
+}
+
+int mk_get_counter_increments(mk_handle* h, uint32_t* out, size_t cap, size_t* n) {
+    if (!h) return MK_ERR_INVALID_ARG;
+    if (!h->scheduled) return MK_ERR_NO_SCHEDULE;
+    if (n) *n = h->plan.ctr_inc.size();
+    if (!out) return MK_OK;
+    if (cap < h->plan.ctr_inc.size()) return MK_ERR_CAPACITY;
+    std::memcpy(out, h->plan.ctr_inc.data(), h->plan.ctr_inc.size() * sizeof(uint32_t));
+    return MK_OK;
+}
+
+int mk_get_status(mk_handle* h, mk_status* out) {
+    if (!h || !out) return MK_ERR_INVALID_ARG;
+    mk::DevStatus st;
+    int rc = read_status(h, &st);
+    if (rc) return rc;
+    out->code = st.code;
+    out->sm = st.sm;
+    out->instr = st.instr;
+    out->opcode = st.opcode;
+    out->counter = st.counter;
+    out->observed = st.observed;
+    out->expected = st.expected;
+    out->cuda_error = h->last_cuda;
+    return MK_OK;
+}
+
+int mk_get_trace(mk_handle* h, uint64_t* out, size_t cap, size_t* n) {
+    if (!h || !h->p.trace) return MK_ERR_INVALID_ARG;
+    const size_t cnt = (size_t)h->plan.n_sm * h->plan.max_instr * 4;
+    if (n) *n = cnt;
+    if (!out) return MK_OK;
+    if (cap < cnt) return MK_ERR_CAPACITY;
+    CK(cudaStreamSynchronize(h->stream));
+    CK(cudaMemcpy(out, h->p.trace, cnt * sizeof(uint64_t), cudaMemcpyDeviceToHost));
+    return MK_OK;
+}
+
+int mk_reset(mk_handle* h) {
+    if (!h) return MK_ERR_INVALID_ARG;
+    CK(cudaStreamSynchronize(h->stream));
+    CK(cudaMemset(h->p.counters, 0, sizeof(uint32_t) * h->p.n_ctr));
+    CK(cudaMemset(h->p.status, 0, sizeof(mk::DevStatus)));
+    if (h->p.trace) CK(cudaMemset(h->p.trace, 0, sizeof(uint64_t) * h->plan.n_sm * h->plan.max_instr * 4));
+    h->epoch = 0;
+    if (h->scheduled) return upload_schedule(h);
+    return MK_OK;
+}
+
+int mk_inject_fault(mk_handle* h, int kind, int arg) {
+    if (!h) return MK_ERR_INVALID_ARG;
+    if (kind == MK_FAULT_NONE) return mk_reset(h);
+    if (kind == MK_FAULT_PRESET_STOP) {
+        const int one = 1;
+        CK(cudaStreamSynchronize(h->stream));
+        CK(cudaMemcpy(&h->p.status->stop, &one, sizeof(int), cudaMemcpyHostToDevice));
+        return MK_OK;
+    }
+    if (!h->scheduled) return MK_ERR_NO_SCHEDULE;
+    if (kind != MK_FAULT_UNREACHABLE_WAIT && kind != MK_FAULT_BAD_OPCODE) return MK_ERR_INVALID_ARG;
+    std::vector<int32_t> words = h->plan.words;
+    const int sm = ((arg % h->plan.n_sm) + h->plan.n_sm) % h->plan.n_sm;
+    bool done = false;
+    for (int i = 0; i < h->plan.n_instr[sm] && !done; ++i) {
+        int32_t* w = &words[((size_t)sm * h->plan.max_instr + i) * mk::W_NWORDS];
+        if (kind == MK_FAULT_BAD_OPCODE) {
+            w[mk::W_OP] = 99;
+            done = true;
+        } else if (w[mk::W_WAIT_CTR] >= 0) {
+            w[mk::W_WAIT_INC] += 1000000;  // a target no step reaches
+            done = true;
+        }
+    }
+    if (!done) return MK_ERR_INVALID_ARG;
+    CK(cudaStreamSynchronize(h->stream));
+    CK(cudaMemcpy(const_cast<int32_t*>(h->p.instr), words.data(), words.size() * sizeof(int32_t),
+                  cudaMemcpyHostToDevice));
+    return MK_OK;
+}
+
+int mk_last_step_ns(mk_handle* h, double* ns) {
+    if (!h || !ns) return MK_ERR_INVALID_ARG;
+    CK(cudaEventSynchronize(h->ev1));
+    float ms = 0.f;
+    CK(cudaEventElapsedTime(&ms, h->ev0, h->ev1));
+    *ns = (double)ms * 1e6;
+    return MK_OK;
+}
+
+void mk_destroy(mk_handle* h) {
+    if (!h) return;
+    cudaStreamSynchronize(h->stream);
+    if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+    if (h->graph) cudaGraphDestroy(h->graph);
+    for (void* ptr : h->allocs) cudaFree(ptr);
+    if (h->status_pinned) cudaFreeHost(h->status_pinned);
+    if (h->ev0) cudaEventDestroy(h->ev0);
+    if (h->ev1) cudaEventDestroy(h->ev1);
+    if (h->ev_done) cudaEventDestroy(h->ev_done);
+    delete h;
+}
+
+}  // extern "C"

@@ -1,0 +1,172 @@
+// mk_device.cuh -- sm_100a device helpers: mbarriers, TMA bulk copies, L2
+// prefetch, acquire/release counter ops, globaltimer, bf16 unpacking and
+// warp reductions.  Inline PTX written for this library.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mk_internal.h"
+
+namespace mk {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarriers ----------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// One probe of phase `parity`; true when that phase has completed.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+// ---- TMA bulk copy (1D, no tensor map) and L2 prefetch --------------------------
+// dst/src 16-byte aligned, bytes a multiple of 16.  Completion is reported as
+// transaction bytes on `bar`.  Never the multicast form.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// ---- global-memory counters -------------------------------------------------------
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ int ld_relaxed_s32(const int* p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---- bf16 ------------------------------------------------------------------------
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ void unpack8(const uint4 w, float* f) {
+    f[0] = bf_lo(w.x); f[1] = bf_hi(w.x);
+    f[2] = bf_lo(w.y); f[3] = bf_hi(w.y);
+    f[4] = bf_lo(w.z); f[5] = bf_hi(w.z);
+    f[6] = bf_lo(w.w); f[7] = bf_hi(w.w);
+}
+// sum_k bf16(w)_k * v_k, fp32, ascending k
+__device__ __forceinline__ float dot8(const uint4 w, const float* v, float acc) {
+    acc = fmaf(bf_lo(w.x), v[0], acc);
+    acc = fmaf(bf_hi(w.x), v[1], acc);
+    acc = fmaf(bf_lo(w.y), v[2], acc);
+    acc = fmaf(bf_hi(w.y), v[3], acc);
+    acc = fmaf(bf_lo(w.z), v[4], acc);
+    acc = fmaf(bf_hi(w.z), v[5], acc);
+    acc = fmaf(bf_lo(w.w), v[6], acc);
+    acc = fmaf(bf_hi(w.w), v[7], acc);
+    return acc;
+}
+// fp32 -> bf16 bits, round to nearest even
+__device__ __forceinline__ uint32_t f2bf(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (u >> 16) | 0x40u;
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return u >> 16;
+}
+
+// ---- warp reductions ----------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+// (value, index) max with ties to the lower index
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        const int oi = __shfl_xor_sync(0xFFFFFFFFu, i, o);
+        if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
+    }
+}
+// Transpose-reduce of RG per-lane partials (one per row, RG in {1,2,4,8})
+// across the warp: log2(RG) halving rounds exchange half of the values, then
+// 5 - log2(RG) butterfly rounds finish the sum (RG - 1 + 5 - log2(RG) shuffles
+// instead of 5 * RG).  On return every lane holds the full sum of row
+// lane >> (5 - log2(RG)).
+template <int RG>
+__device__ __forceinline__ float reduce_rows(float (&a)[RG], int lane) {
+#pragma unroll
+    for (int n = RG, off = 16; n > 1; n >>= 1, off >>= 1) {
+        const bool up = lane & off;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = up ? a[i] : a[i + n / 2];
+            const float keep = up ? a[i + n / 2] : a[i];
+            a[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
+        }
+    }
+    constexpr int first = RG == 8 ? 2 : RG == 4 ? 4 : RG == 2 ? 8 : 16;
+    float e = a[0];
+#pragma unroll
+    for (int off = first; off > 0; off >>= 1) e += __shfl_xor_sync(0xFFFFFFFFu, e, off);
+    return e;
+}
+template <int RG>
+__device__ __forceinline__ int reduce_rows_lane_row(int lane) {
+    return RG == 8 ? lane >> 2 : RG == 4 ? lane >> 3 : RG == 2 ? lane >> 4 : 0;
+}
+template <int RG>
+__device__ __forceinline__ bool reduce_rows_writer(int lane) {
+    return (lane & (32 / RG - 1)) == 0;
+}
+
+// ---- status -------------------------------------------------------------------------
+__device__ __forceinline__ void record_error(DevStatus* st, int code, int sm, int instr, int op, int ctr,
+                                             uint32_t observed, uint32_t expected) {
+    if (atomicCAS(&st->code, 0, code) == 0) {
+        st->sm = sm;
+        st->instr = instr;
+        st->opcode = op;
+        st->counter = ctr;
+        st->observed = observed;
+        st->expected = expected;
+    }
+    __threadfence();
+    atomicExch(&st->stop, 1);
+}
+
+}  // namespace mk

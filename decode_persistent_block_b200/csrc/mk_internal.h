@@ -1,0 +1,132 @@
+// mk_internal.h -- instruction format, counter layout and the device parameter
+// block shared by the host scheduler, the persistent kernel and the baseline.
+#pragma once
+#include <stddef.h>
+#include <stdint.h>
+
+#include <vector_types.h>
+
+#include "../../include/mk.h"
+
+#if defined(__CUDACC__)
+#define MK_HD __host__ __device__
+#else
+#define MK_HD
+#endif
+
+namespace mk {
+
+// Opcodes: "simple kernels become opcodes" dispatched inside the persistent
+// interpreter (Kittens VM summary page, "Method").  The set is the batch-1
+// Llama/Mixtral decode step (epic-kernel README, "3B model support", "Mixtral
+// 8x7B MoE for batch-1 inference").
+enum Opcode : int32_t {
+    OP_NOP = 0,
+    OP_RMS_QKV = 1,          // xn = rmsnorm(x) * w_attn; rows of [Wq; Wk; Wv] xn (raw, pre-RoPE)
+    OP_ATTN = 2,             // RoPE + KV append + one split of GQA decode attention; last split merges
+    OP_OPROJ_RES = 3,        // x[rows] = x[rows] + Wo[rows] attn   (layer 0: embed row + ...)
+    OP_RMS_UPGATE_SILU = 4,  // h[rows] = silu(Wg[rows] xn) * (Wu[rows] xn), xn = rmsnorm(x) * w_ffn
+    OP_DOWN_RES = 5,         // x[rows] += Wd[rows] h
+    OP_LMHEAD_ARGMAX = 6,    // logits[rows] = Wlm[rows] rmsnorm(x) * w_final; last instruction reduces argmax
+    OP_MOE_UPGATE = 7,       // router + top-k in prologue; h_slot[rows] for the selected expert of `slot`
+    OP_MOE_DOWN2_RES = 8,    // x[rows] += sum_slot w_slot * Wd_{e_slot}[rows] h_slot  (all slots, one instr)
+    OP_COUNT = 9
+};
+
+// Instruction words (int32 each, MK_INSTR_WORDS per instruction).
+enum Word : int {
+    W_OP = 0,
+    W_LAYER = 1,
+    W_SUB = 2,        // QKV: 0 q / 1 k / 2 v; ATTN: kv head; MOE_UPGATE: expert slot
+    W_BEGIN = 3,      // first row (GEMV) or split index (ATTN)
+    W_END = 4,        // one past the last row (GEMV) or number of splits (ATTN)
+    W_WAIT_CTR = 5,   // counter waited on before reading activations (-1: none)
+    W_WAIT_INC = 6,   // its per-step increment (target = epoch * inc)
+    W_SIGNAL_CTR = 7, // counter incremented once when the instruction's outputs are visible (-1: none)
+    W_AUX_CTR = 8,    // ATTN: per-head-group arrival counter; LMHEAD: arrival counter
+    W_AUX_INC = 9,    // its per-step increment
+    W_SEQ = 10,       // LMHEAD: slot of this instruction's partial argmax; ATTN: unused
+    W_NWORDS = MK_INSTR_WORDS
+};
+
+constexpr int kMaxRows = 1024;       // rows per GEMV instruction (smem accumulators)
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kThreads = kConsumerThreads + 32;  // + one loader warp
+constexpr int kMaxGroup = 4;         // query heads per kv head
+constexpr int kMaxHeadDim = 128;
+constexpr int kMaxTopK = 2;
+
+// Counter ids: per layer [QKV, ATTN_DONE, OPROJ, FFN1, FFN2, GROUP_0..GROUP_{nkv-1}], then LM.
+enum CtrSlot : int { C_QKV = 0, C_ATTN = 1, C_OPROJ = 2, C_FFN1 = 3, C_FFN2 = 4, C_GROUP0 = 5 };
+MK_HD inline int counters_per_layer(int n_kv) { return C_GROUP0 + n_kv; }
+MK_HD inline int ctr_id(int layer, int slot, int n_kv) { return layer * counters_per_layer(n_kv) + slot; }
+MK_HD inline int ctr_lm(int n_layers, int n_kv) { return n_layers * counters_per_layer(n_kv); }
+MK_HD inline int n_counters(int n_layers, int n_kv) { return n_layers * counters_per_layer(n_kv) + 1; }
+
+// Weight pointer table: per layer kLayerFixed entries, then gate/up/down per expert.
+enum WSlot : int { WT_ATTN_NORM = 0, WT_Q, WT_K, WT_V, WT_O, WT_FFN_NORM, WT_ROUTER, kLayerFixed };
+MK_HD inline int wt_stride(int n_experts) { return kLayerFixed + 3 * (n_experts > 0 ? n_experts : 1); }
+MK_HD inline int wt_gate(int e) { return kLayerFixed + e; }
+MK_HD inline int wt_up(int e, int n_experts) { return kLayerFixed + (n_experts > 0 ? n_experts : 1) + e; }
+MK_HD inline int wt_down(int e, int n_experts) { return kLayerFixed + 2 * (n_experts > 0 ? n_experts : 1) + e; }
+
+struct DevStatus {
+    int code, sm, instr, opcode, counter;
+    unsigned int observed, expected;
+    int cuda_error;
+    int stop;        // stop word: nonzero makes every block leave at its next wait
+    int next_token;  // argmax of the last completed step
+    int pad[6];
+};
+
+// Everything the kernels read that stays fixed for a handle (device memory).
+struct DevParams {
+    // model
+    int L, H, nq, nkv, d, F, V, E, topk, max_seq;
+    float eps;
+    int kv_splits;
+    // schedule
+    const int32_t* instr;    // [n_sm][max_instr][W_NWORDS]
+    const int32_t* n_instr;  // [n_sm]
+    int max_instr;
+    int n_ctr;
+    uint32_t* counters;
+    DevStatus* status;
+    // weights (bf16 as raw uint16)
+    const uint16_t* embed;
+    const uint16_t* lm_head;
+    const uint16_t* final_norm;
+    const uint16_t* const* wt;  // [L][wt_stride]
+    uint16_t* kcache;
+    uint16_t* vcache;
+    const float2* rope;      // [max_seq][d/2] (cos, sin)
+    // activations (fp32)
+    float* x;          // [H]
+    float* qkv;        // [(nq + 2 nkv) d]  raw projections, pre-RoPE
+    float* attn;       // [nq d]
+    float* part_o;     // [nq][kv_splits][d]
+    float* part_ml;    // [nq][kv_splits][2]
+    float* hbuf;       // [max(topk,1)][F]
+    float* logits;     // [V] (internal; a caller buffer overrides per step)
+    float* lm_part;    // [n_lm][2] (value, index bits)
+    float* snap;       // [(L+1)][H] or null
+    int32_t* router_idx;  // [L][kMaxTopK]
+    float* router_w;      // [L][kMaxTopK]
+    unsigned long long* trace;  // [n_sm][max_instr][4] or null
+    // kernel knobs
+    int ring_stages;
+    int stage_bytes;
+    int l2_prefetch;
+    unsigned long long spin_limit_ns;
+};
+
+// Per-launch arguments (passed by value).
+struct StepArgs {
+    int token;        // < 0: use *next_token from the previous step
+    int pos;
+    uint32_t epoch;   // 1-based step count since the last reset
+    float* logits;    // output logits (device)
+};
+
+}  // namespace mk

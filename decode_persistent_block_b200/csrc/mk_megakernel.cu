@@ -1,0 +1,1105 @@
+// mk_megakernel.cu -- the persistent batch-1 decode kernel for sm_100a.
+//
+// One block per SM, launched cooperatively so that every block is resident;
+// each block interprets its queue of the host-built instruction tensor and
+// never returns to the host inside a step ("a single persistent CUDA kernel
+// that occupies the entire GPU and reads an instruction tensor at runtime":
+// Kittens VM summary page, "Method"; "Launch one kernel with one block per SM
+// ... Never let the blocks exit ... synchronize with each other on the
+// device": Hyperkernel teardown, "What a megakernel buys").
+//
+// Block = 8 consumer warps + 1 loader warp (warp-specialised roles: epic-kernel
+// README, "Fence removal and barrier reduction"):
+//  * the loader (one elected lane) walks the block's queue and streams every
+//    instruction's bf16 weight rows (or KV-cache rows) into a ring of
+//    shared-memory stages with TMA bulk copies completed on mbarriers.  Weight
+//    loads do not depend on activations, so the loader runs ahead across the
+//    consumers' dependency waits ("tiles of the next layer's weights can be
+//    loaded while the current layer still computes": Hyperkernel teardown,
+//    "What a megakernel buys").  After each stage it keeps a configurable
+//    number of bytes of the following stages, across instruction boundaries,
+//    prefetched into L2 (epic-kernel README, "L2 prefetching overlapped with
+//    prior instructions").
+//  * the consumers wait on the instruction's global dependency counter (one
+//    acquiring lane, bounded), build the fp32 input vector in registers, run
+//    the fp32-accumulate dot products from the ring, reduce across the warp
+//    with shuffles and across warps with shared-memory atomics, and in the
+//    epilogue act as the storer: write outputs, then release-increment the
+//    signal counter.
+// Every wait is bounded by a spin limit; on expiry the block records where it
+// gave up in the status block, sets the stop word (every other block leaves at
+// its next wait), drains its in-flight copies and returns (Hyperkernel
+// teardown, "Hardware fault detection and replanning": watchdog word, stop
+// word, bounds flags).
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "mk_device.cuh"
+#include "mk_internal.h"
+#include "mk_kernels.h"
+
+namespace mk {
+
+// ---------------------------------------------------------------------------
+// shared memory layout
+// ---------------------------------------------------------------------------
+constexpr int kScratchBytes = 17408;  // max(acc 2*kMaxRows*4, attention merge 8*512*4 + 8*8*2*4, router 8*64*4)
+
+struct Misc {
+    float red[kConsumerWarps * 2];
+    int redi[kConsumerWarps];
+    int abort_flag;
+    int router_layer;  // layer whose routing is in eidx/ew (-1: none)
+    int eidx[kMaxTopK];
+    float ew[kMaxTopK];
+    int is_last;
+    int pad[3];
+};
+
+__host__ __device__ inline size_t smem_bars_off(int ns, int sb) { return (size_t)ns * sb; }
+__host__ __device__ inline size_t smem_scratch_off(int ns, int sb) {
+    return (smem_bars_off(ns, sb) + 16 * (size_t)ns + 127) & ~(size_t)127;
+}
+__host__ __device__ inline size_t smem_misc_off(int ns, int sb) { return smem_scratch_off(ns, sb) + kScratchBytes; }
+size_t megakernel_smem_bytes(int ns, int sb) { return smem_misc_off(ns, sb) + sizeof(Misc); }
+
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ int vload(const int* p) { return *(volatile const int*)p; }
+__device__ __forceinline__ void vstore(int* p, int v) { *(volatile int*)p = v; }
+
+// ---------------------------------------------------------------------------
+// bounded waits
+// ---------------------------------------------------------------------------
+__device__ bool wait_counter(const DevParams& p, Misc& m, int ctr, uint32_t target, int ii, int op) {
+    const uint32_t* addr = p.counters + ctr;
+    uint32_t v = ld_acquire_u32(addr);
+    if ((int32_t)(v - target) >= 0) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        v = ld_acquire_u32(addr);
+        if ((int32_t)(v - target) >= 0) return true;
+        if ((it & 31u) == 0) {
+            if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
+            if (globaltimer_ns() - t0 > p.spin_limit_ns) {
+                record_error(p.status, MK_ERR_TIMEOUT, blockIdx.x, ii, op, ctr, v, target);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const DevParams& p, Misc& m, int ii, int op) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0) {
+            if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
+            if (globaltimer_ns() - t0 > p.spin_limit_ns) {
+                record_error(p.status, MK_ERR_TIMEOUT, blockIdx.x, ii, op, -1, parity, 0);
+                return false;
+            }
+        }
+    }
+}
+
+// Warp-uniform wait for a full ring stage: lane 0 waits (bounded), the result
+// is broadcast, then every lane takes its own acquire of the completed phase.
+__device__ bool warp_wait_full(uint64_t* bar, uint32_t parity, const DevParams& p, Misc& m, int ii, int op) {
+    const int lane = threadIdx.x & 31;
+    int ok = 1;
+    if (lane == 0) ok = wait_mbar(bar, parity, p, m, ii, op) ? 1 : 0;
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    if (ok) {
+        for (int k = 0; k < 64 && !mbar_try_wait(bar, parity); ++k) {
+        }
+    }
+    return ok != 0;
+}
+
+// ---------------------------------------------------------------------------
+// instruction checks and the stage plan shared by loader and consumers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int op_rows(const DevParams& p, int op, int sub) {
+    switch (op) {
+        case OP_RMS_QKV: return sub == 0 ? p.nq * p.d : p.nkv * p.d;
+        case OP_OPROJ_RES:
+        case OP_DOWN_RES:
+        case OP_MOE_DOWN2_RES: return p.H;
+        case OP_RMS_UPGATE_SILU:
+        case OP_MOE_UPGATE: return p.F;
+        case OP_LMHEAD_ARGMAX: return p.V;
+    }
+    return 0;
+}
+
+// Bounds flags: every index an instruction carries is checked before use.
+__device__ bool instr_ok(const DevParams& p, const int32_t* w) {
+    const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], e = w[W_END];
+    if (op <= OP_NOP || op >= OP_COUNT) return false;
+    const bool moe_op = op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES;
+    if ((p.E > 0) != moe_op && (moe_op || op == OP_RMS_UPGATE_SILU || op == OP_DOWN_RES)) return false;
+    if (op == OP_LMHEAD_ARGMAX ? l != p.L : (l < 0 || l >= p.L)) return false;
+    if (w[W_WAIT_CTR] < -1 || w[W_WAIT_CTR] >= p.n_ctr || w[W_SIGNAL_CTR] < -1 || w[W_SIGNAL_CTR] >= p.n_ctr ||
+        w[W_AUX_CTR] < -1 || w[W_AUX_CTR] >= p.n_ctr)
+        return false;
+    if (w[W_WAIT_CTR] >= 0 && w[W_WAIT_INC] <= 0) return false;
+    if (op == OP_ATTN) {
+        if (sub < 0 || sub >= p.nkv || e != p.kv_splits || b < 0 || b >= e) return false;
+        return w[W_AUX_CTR] >= 0 && w[W_SIGNAL_CTR] >= 0 && w[W_AUX_INC] > 0;
+    }
+    if (op == OP_RMS_QKV && (sub < 0 || sub > 2)) return false;
+    if (op == OP_MOE_UPGATE && (sub < 0 || sub >= p.topk)) return false;
+    if (b < 0 || b >= e || e > op_rows(p, op, sub) || e - b > kMaxRows) return false;
+    if (op == OP_LMHEAD_ARGMAX) return w[W_AUX_CTR] >= 0 && w[W_AUX_INC] > 0 && w[W_SEQ] >= 0 && w[W_SEQ] < w[W_AUX_INC];
+    return w[W_SIGNAL_CTR] >= 0;
+}
+
+// Column parts: rows wider than kMaxPartK columns are streamed and reduced in
+// column parts (one phase per part) so that each thread's slice of the input
+// vector stays within 4 chunks of 8 in registers.
+constexpr int kMaxPartK = 8 * kConsumerThreads * 4;  // 8192
+
+__host__ __device__ __forceinline__ int kparts_of(int K) { return (K + kMaxPartK - 1) / kMaxPartK; }
+
+struct Plan {
+    int n_stages;   // stages of the whole instruction
+    int nphase;     // slots * kparts (slots: top_k for the fused expert down-projection, else 1)
+    int kparts;     // column parts per row
+    int nspan;      // spans per stage (gate+up, K+V: 2)
+    int rows;       // rows of the instruction
+    int rps;        // rows per stage
+    int spp;        // stages per phase
+    uint32_t row_bytes;   // bytes of one row part in shared memory
+    uint32_t src_stride;  // bytes between consecutive rows in global memory
+    const unsigned char* src[kMaxTopK][2];  // [slot][span]: row 0 of the instruction, column 0
+};
+
+struct AttnRange {
+    int jb, je, ncached;
+    bool has_new;
+};
+__device__ __forceinline__ AttnRange attn_range(int pos, int split, int S) {
+    const long long npos = (long long)pos + 1;
+    AttnRange r;
+    r.jb = (int)(npos * split / S);
+    r.je = (int)(npos * (split + 1) / S);
+    const int jce = r.je < pos ? r.je : pos;
+    r.ncached = jce > r.jb ? jce - r.jb : 0;
+    r.has_new = (r.je == npos);
+    return r;
+}
+
+// eidx: the routed experts of the instruction's layer (MoE ops only).
+__device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const int* eidx, Plan& pl) {
+    const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], e = w[W_END];
+    const uint16_t* const* wt = p.wt + (size_t)(l < p.L ? l : 0) * wt_stride(p.E);
+    const uint32_t SB = (uint32_t)p.stage_bytes;
+    int nslot = 1;
+    pl.nspan = 1;
+    pl.kparts = 1;
+    pl.src[0][1] = pl.src[1][0] = pl.src[1][1] = nullptr;
+    int K = p.H;
+    const uint16_t* s0 = nullptr;
+    const uint16_t* s1 = nullptr;
+    const uint16_t* s2 = nullptr;  // second slot's matrix (fused expert down-projection)
+    switch (op) {
+        case OP_ATTN: {
+            const AttnRange r = attn_range(pos, b, e);
+            pl.nphase = 1;
+            pl.nspan = 2;
+            pl.rows = r.ncached;
+            pl.row_bytes = pl.src_stride = (uint32_t)p.d * 2u;
+            pl.rps = (int)(SB / (2u * pl.row_bytes));
+            pl.spp = (pl.rows + pl.rps - 1) / pl.rps;
+            pl.n_stages = pl.spp;
+            const size_t base = (((size_t)l * p.nkv + sub) * (size_t)p.max_seq + (size_t)r.jb) * (size_t)p.d;
+            pl.src[0][0] = (const unsigned char*)(p.kcache + base);
+            pl.src[0][1] = (const unsigned char*)(p.vcache + base);
+            return;
+        }
+        case OP_RMS_QKV: s0 = wt[WT_Q + sub]; break;
+        case OP_OPROJ_RES: K = p.nq * p.d; s0 = wt[WT_O]; break;
+        case OP_RMS_UPGATE_SILU: pl.nspan = 2; s0 = wt[wt_gate(0)]; s1 = wt[wt_up(0, p.E)]; break;
+        case OP_DOWN_RES: K = p.F; s0 = wt[wt_down(0, p.E)]; break;
+        case OP_LMHEAD_ARGMAX: s0 = p.lm_head; break;
+        case OP_MOE_UPGATE:
+            pl.nspan = 2;
+            s0 = wt[wt_gate(eidx[sub])];
+            s1 = wt[wt_up(eidx[sub], p.E)];
+            break;
+        case OP_MOE_DOWN2_RES:
+            K = p.F;
+            nslot = p.topk;
+            s0 = wt[wt_down(eidx[0], p.E)];
+            if (p.topk > 1) s2 = wt[wt_down(eidx[1], p.E)];
+            break;
+    }
+    pl.kparts = kparts_of(K);
+    pl.nphase = nslot * pl.kparts;
+    pl.rows = e - b;
+    pl.src_stride = (uint32_t)K * 2u;
+    pl.row_bytes = pl.src_stride / (uint32_t)pl.kparts;
+    const int rps = (int)(SB / ((uint32_t)pl.nspan * pl.row_bytes));
+    pl.rps = rps < pl.rows ? rps : pl.rows;
+    pl.spp = (pl.rows + pl.rps - 1) / pl.rps;
+    pl.n_stages = pl.spp * pl.nphase;
+    pl.src[0][0] = (const unsigned char*)(s0 + (size_t)b * K);
+    if (s1) pl.src[0][1] = (const unsigned char*)(s1 + (size_t)b * K);
+    if (s2) pl.src[1][0] = (const unsigned char*)(s2 + (size_t)b * K);
+}
+
+__device__ __forceinline__ bool needs_routing(int op) { return op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES; }
+
+// ---------------------------------------------------------------------------
+// loader warp (one lane)
+// ---------------------------------------------------------------------------
+__device__ void issue_stage(const Plan& pl, int st, unsigned char* dst_stage, uint64_t* bar) {
+    const int ph = st / pl.spp, sst = st % pl.spp;
+    const int slot = ph / pl.kparts, part = ph % pl.kparts;
+    const int r0 = sst * pl.rps;
+    const int nr = (pl.rows - r0) < pl.rps ? (pl.rows - r0) : pl.rps;
+    const uint32_t bytes = (uint32_t)nr * pl.row_bytes;
+    mbar_arrive_expect_tx(bar, bytes * (uint32_t)pl.nspan);
+    for (int s = 0; s < pl.nspan; ++s) {
+        const unsigned char* src = pl.src[slot][s] + (size_t)r0 * pl.src_stride + (size_t)part * pl.row_bytes;
+        unsigned char* dst = dst_stage + (size_t)s * pl.rps * pl.row_bytes;
+        if (pl.kparts == 1) {
+            bulk_g2s(dst, src, bytes, bar);
+        } else {
+            for (int r = 0; r < nr; ++r)
+                bulk_g2s(dst + (size_t)r * pl.row_bytes, src + (size_t)r * pl.src_stride, pl.row_bytes, bar);
+        }
+    }
+}
+
+__device__ void prefetch_stage(const Plan& pl, int st) {
+    const int ph = st / pl.spp, sst = st % pl.spp;
+    const int slot = ph / pl.kparts, part = ph % pl.kparts;
+    const int r0 = sst * pl.rps;
+    const int nr = (pl.rows - r0) < pl.rps ? (pl.rows - r0) : pl.rps;
+    for (int s = 0; s < pl.nspan; ++s) {
+        const unsigned char* src = pl.src[slot][s] + (size_t)r0 * pl.src_stride + (size_t)part * pl.row_bytes;
+        if (pl.kparts == 1) {
+            prefetch_l2(src, (uint32_t)nr * pl.row_bytes);
+        } else {
+            for (int r = 0; r < nr; ++r) prefetch_l2(src + (size_t)r * pl.src_stride, pl.row_bytes);
+        }
+    }
+}
+
+// Plan instruction i for the loader; for MoE ops wait (bounded) until the
+// consumers have routed the layer, unless `block` is false.
+__device__ bool loader_plan(const DevParams& p, const StepArgs& a, const int32_t* w, Misc& m, Plan& pl, bool block,
+                            int ii) {
+    if (!instr_ok(p, w)) {
+        pl.n_stages = 0;
+        return true;
+    }
+    if (needs_routing(w[W_OP])) {
+        const int l = w[W_LAYER];
+        if (vload(&m.router_layer) != l) {
+            if (!block) return false;
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t it = 1; vload(&m.router_layer) != l; ++it) {
+                if ((it & 63u) == 0) {
+                    if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
+                    if (globaltimer_ns() - t0 > p.spin_limit_ns) {
+                        record_error(p.status, MK_ERR_TIMEOUT, blockIdx.x, ii, w[W_OP], -1, 0, 0);
+                        return false;
+                    }
+                }
+            }
+        }
+        __threadfence_block();
+        int eidx[kMaxTopK];
+        for (int k = 0; k < kMaxTopK; ++k) eidx[k] = vload(&m.eidx[k]);
+        make_plan(p, a.pos, w, eidx, pl);
+        return true;
+    }
+    make_plan(p, a.pos, w, nullptr, pl);
+    return true;
+}
+
+__device__ void loader(const DevParams& p, const StepArgs& a, const int32_t* q, int n, unsigned char* ring,
+                       uint64_t* full, uint64_t* empty, Misc& m) {
+    const int NS = p.ring_stages;
+    const uint32_t SB = (uint32_t)p.stage_bytes;
+    const int pf_stages = p.l2_prefetch > 0 ? (int)((uint32_t)p.l2_prefetch / SB) : 0;
+    int slot = 0;
+    uint32_t phase = 0;
+    uint32_t used = 0, last_parity = 0;
+    // L2 prefetch cursor: next (instruction, stage) to prefetch and its global stage index
+    int pf_i = 0, pf_st = 0;
+    long long pf_g = 0, g = 0;
+    Plan pf_plan;
+    pf_plan.n_stages = 0;
+    bool pf_stalled = false;
+
+    for (int i = 0; i < n; ++i) {
+        const int32_t* w = q + (size_t)i * W_NWORDS;
+        Plan pl;
+        if (!loader_plan(p, a, w, m, pl, true, i)) break;
+        bool ok = true;
+        for (int st = 0; st < pl.n_stages; ++st, ++g) {
+            if (!wait_mbar(&empty[slot], phase ^ 1u, p, m, i, w[W_OP])) {
+                ok = false;
+                break;
+            }
+            issue_stage(pl, st, ring + (size_t)slot * SB, &full[slot]);
+            used |= 1u << slot;
+            last_parity = (last_parity & ~(1u << slot)) | (phase << slot);
+            if (++slot == NS) {
+                slot = 0;
+                phase ^= 1u;
+            }
+            if (pf_stages > 0) {
+                if (pf_g <= g) {  // cursor caught up: restart right after this stage
+                    pf_i = i;
+                    pf_st = st + 1;
+                    pf_g = g + 1;
+                    pf_plan = pl;
+                    pf_stalled = false;
+                }
+                while (pf_g <= g + pf_stages && !pf_stalled) {
+                    if (pf_st >= pf_plan.n_stages) {
+                        if (pf_i + 1 >= n) {
+                            pf_stalled = true;
+                            break;
+                        }
+                        Plan np;
+                        if (!loader_plan(p, a, q + (size_t)(pf_i + 1) * W_NWORDS, m, np, false, pf_i + 1)) break;
+                        pf_i++;
+                        pf_plan = np;
+                        pf_st = 0;
+                        continue;
+                    }
+                    prefetch_stage(pf_plan, pf_st);
+                    pf_st++;
+                    pf_g++;
+                }
+            }
+        }
+        if (!ok) break;
+    }
+    // drain: wait for the last copy issued into every used slot
+    for (int s = 0; s < NS; ++s) {
+        if (!((used >> s) & 1u)) continue;
+        const uint32_t par = (last_parity >> s) & 1u;
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&full[s], par)) {
+            if (globaltimer_ns() - t0 > p.spin_limit_ns) break;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// consumers: GEMV-type instructions
+// ---------------------------------------------------------------------------
+enum VecKind { VK_RMS, VK_ATTN, VK_H };
+
+// Fill v[j][0..8) with the input vector slice of this thread (chunks
+// c = tid + 256 j of 8 elements; zero outside [0, K)).
+template <int J>
+__device__ __forceinline__ void load_vec(const float* __restrict__ src, int K, float (&v)[J][8]) {
+    const int tid = threadIdx.x, nch = K >> 3;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int c = tid + kConsumerThreads * j;
+        if (c < nch) {
+            const float4 a0 = __ldcg(reinterpret_cast<const float4*>(src) + 2 * c);
+            const float4 a1 = __ldcg(reinterpret_cast<const float4*>(src) + 2 * c + 1);
+            v[j][0] = a0.x; v[j][1] = a0.y; v[j][2] = a0.z; v[j][3] = a0.w;
+            v[j][4] = a1.x; v[j][5] = a1.y; v[j][6] = a1.z; v[j][7] = a1.w;
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
+        }
+    }
+}
+
+// v = rmsnorm(x) * w for x fp32 (or the bf16 embedding row), all threads.
+template <int J>
+__device__ void load_rms(const DevParams& p, Misc& m, const float* x32, const uint16_t* x16, const uint16_t* nw,
+                         float (&v)[J][8]) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.H, nch = K >> 3;
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int c = tid + kConsumerThreads * j;
+        if (c < nch) {
+            if (x16) {
+                const uint4 r = __ldg(reinterpret_cast<const uint4*>(x16) + c);
+                unpack8(r, v[j]);
+            } else {
+                const float4 a0 = __ldcg(reinterpret_cast<const float4*>(x32) + 2 * c);
+                const float4 a1 = __ldcg(reinterpret_cast<const float4*>(x32) + 2 * c + 1);
+                v[j][0] = a0.x; v[j][1] = a0.y; v[j][2] = a0.z; v[j][3] = a0.w;
+                v[j][4] = a1.x; v[j][5] = a1.y; v[j][6] = a1.z; v[j][7] = a1.w;
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) ss = fmaf(v[j][k], v[j][k], ss);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
+        }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) m.red[warp] = ss;
+    cbar();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) tot += m.red[w];
+    const float rs = 1.0f / sqrtf(tot / (float)K + p.eps);
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int c = tid + kConsumerThreads * j;
+        if (c < nch) {
+            float wf[8];
+            unpack8(__ldg(reinterpret_cast<const uint4*>(nw) + c), wf);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[j][k] = v[j][k] * rs * wf[k];
+        }
+    }
+    cbar();  // m.red free again
+}
+
+// Router of a MoE layer from xn (this thread's slice in v): logits of all
+// experts, top-k (ties to the lower index), softmax over the selected.
+template <int J>
+__device__ void route(const DevParams& p, Misc& m, float* scratch, const uint16_t* wr, int layer, bool publish,
+                      float (&v)[J][8]) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.H, nch = K >> 3, E = p.E;
+    for (int e0 = 0; e0 < E; e0 += 8) {
+        float a[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            a[r] = 0.f;
+            if (e0 + r < E) {
+#pragma unroll
+                for (int j = 0; j < J; ++j) {
+                    const int c = tid + kConsumerThreads * j;
+                    if (c < nch) a[r] = dot8(__ldg(reinterpret_cast<const uint4*>(wr + (size_t)(e0 + r) * K) + c), v[j], a[r]);
+                }
+            }
+        }
+        const float s = reduce_rows<8>(a, lane);
+        const int r = reduce_rows_lane_row<8>(lane);
+        if (reduce_rows_writer<8>(lane) && e0 + r < E) scratch[warp * 64 + e0 + r] = s;
+    }
+    cbar();
+    if (tid == 0) {
+        float logit[64];
+        for (int e = 0; e < E; ++e) {
+            float t = 0.f;
+            for (int w = 0; w < kConsumerWarps; ++w) t += scratch[w * 64 + e];
+            logit[e] = t;
+        }
+        int idx[kMaxTopK];
+        unsigned long long taken = 0;
+        for (int k = 0; k < p.topk; ++k) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if ((taken >> e) & 1ull) continue;
+                if (best < 0 || logit[e] > logit[best]) best = e;
+            }
+            taken |= 1ull << best;
+            idx[k] = best;
+        }
+        float mx = logit[idx[0]], z = 0.f, ex[kMaxTopK];
+        for (int k = 0; k < p.topk; ++k) {
+            ex[k] = expf(logit[idx[k]] - mx);
+            z += ex[k];
+        }
+        for (int k = 0; k < p.topk; ++k) {
+            m.eidx[k] = idx[k];
+            m.ew[k] = ex[k] / z;
+            if (publish) {
+                p.router_idx[layer * kMaxTopK + k] = idx[k];
+                p.router_w[layer * kMaxTopK + k] = ex[k] / z;
+            }
+        }
+        __threadfence_block();
+        vstore(&m.router_layer, layer);
+    }
+    cbar();
+}
+
+template <int J>
+__device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
+                           uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase,
+                           int token) {
+    // rows reduced together: keeps the live 128-bit weight loads at RG * J <= 8
+    constexpr int RG = J == 1 ? 8 : J == 2 ? 4 : J <= 4 ? 2 : 1;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], rows = w[W_END] - b;
+    const uint32_t SB = (uint32_t)p.stage_bytes;
+    float* acc = scratch;  // [2][kMaxRows]
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * 4 : nullptr;
+
+    // 1. dependency, zero accumulators
+    if (tid == 0) {
+        if (w[W_WAIT_CTR] >= 0 &&
+            !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op))
+            vstore(&m.abort_flag, 1);
+        if (tr) tr[1] = globaltimer_ns();
+    }
+    for (int r = tid; r < rows; r += kConsumerThreads) {
+        acc[r] = 0.f;
+        acc[kMaxRows + r] = 0.f;
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+
+    // 2. input vector (first column part)
+    float v[J][8];
+    const uint16_t* const* wt = p.wt + (size_t)(l < p.L ? l : 0) * wt_stride(p.E);
+    int K = p.H;
+    const float* vsrc = nullptr;  // fp32 input for OPROJ / DOWN (all column parts)
+    switch (op) {
+        case OP_RMS_QKV:
+            load_rms<J>(p, m, p.x, l == 0 ? p.embed + (size_t)token * p.H : nullptr, wt[WT_ATTN_NORM], v);
+            break;
+        case OP_RMS_UPGATE_SILU:
+        case OP_MOE_UPGATE:
+            load_rms<J>(p, m, p.x, nullptr, wt[WT_FFN_NORM], v);
+            break;
+        case OP_LMHEAD_ARGMAX:
+            load_rms<J>(p, m, p.x, p.L == 0 ? p.embed + (size_t)token * p.H : nullptr, p.final_norm, v);
+            break;
+        case OP_OPROJ_RES:
+            K = p.nq * p.d;
+            vsrc = p.attn;
+            break;
+        case OP_DOWN_RES:
+        case OP_MOE_DOWN2_RES:
+            K = p.F;
+            vsrc = p.hbuf;
+            break;
+    }
+    const int kp = K / kparts_of(K);  // columns per part
+    if (vsrc) load_vec<J>(vsrc, kp, v);
+    // 3. routing (once per layer per block; the loader waits for it)
+    if (op == OP_MOE_UPGATE && vload(&m.router_layer) != l)
+        route<J>(p, m, scratch + 2 * kMaxRows, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
+
+    int eidx[kMaxTopK];
+    for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
+    Plan pl;
+    make_plan(p, a.pos, w, eidx, pl);
+
+    // 4. stages: every warp covers its column slice of every row of the stage
+    const int nch = kp >> 3;
+    for (int ph = 0; ph < pl.nphase; ++ph) {
+        const int vslot = ph / pl.kparts, part = ph % pl.kparts;
+        if (ph > 0) load_vec<J>(vsrc + (size_t)vslot * p.F + (size_t)part * kp, kp, v);
+        for (int sst = 0; sst < pl.spp; ++sst) {
+            const int r0 = sst * pl.rps;
+            const int nr = (rows - r0) < pl.rps ? (rows - r0) : pl.rps;
+            const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, op);
+            if (tr && tid == 0 && ph == 0 && sst == 0) tr[2] = globaltimer_ns();
+            if (ok) {
+                const uint32_t stage = smem_u32(ring) + slot * SB;
+                for (int s = 0; s < pl.nspan; ++s) {
+                    const uint32_t W0 = stage + (uint32_t)(s * pl.rps) * pl.row_bytes;
+                    float* A = acc + (vslot + s) * kMaxRows + r0;
+                    for (int rg = 0; rg < nr; rg += RG) {
+                        float part[RG];
+#pragma unroll
+                        for (int r = 0; r < RG; ++r) {
+                            part[r] = 0.f;
+                            if (rg + r < nr) {
+                                const uint32_t row = W0 + (uint32_t)(rg + r) * pl.row_bytes;
+#pragma unroll
+                                for (int j = 0; j < J; ++j) {
+                                    const int c = tid + kConsumerThreads * j;
+                                    if (c < nch) part[r] = dot8(lds128(row + 16u * c), v[j], part[r]);
+                                }
+                            }
+                        }
+                        const float s_row = reduce_rows<RG>(part, lane);
+                        const int rr = rg + reduce_rows_lane_row<RG>(lane);
+                        if (reduce_rows_writer<RG>(lane) && rr < nr) atomicAdd(&A[rr], s_row);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[slot]);
+            } else if (tid == 0) {
+                vstore(&m.abort_flag, 1);
+            }
+            if (++slot == p.ring_stages) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+
+    // 5. epilogue (storer role)
+    switch (op) {
+        case OP_RMS_QKV: {
+            const int off = sub == 0 ? 0 : (sub == 1 ? p.nq * p.d : (p.nq + p.nkv) * p.d);
+            for (int r = tid; r < rows; r += kConsumerThreads) p.qkv[off + b + r] = acc[r];
+            break;
+        }
+        case OP_OPROJ_RES:
+            for (int r = tid; r < rows; r += kConsumerThreads) {
+                float base;
+                if (l == 0) {
+                    const uint16_t e = p.embed[(size_t)token * p.H + b + r];
+                    base = __uint_as_float((uint32_t)e << 16);
+                    if (p.snap) p.snap[b + r] = base;
+                } else {
+                    base = __ldcg(p.x + b + r);
+                }
+                p.x[b + r] = base + acc[r];
+            }
+            break;
+        case OP_RMS_UPGATE_SILU:
+        case OP_MOE_UPGATE: {
+            float* h = p.hbuf + (op == OP_MOE_UPGATE ? (size_t)sub * p.F : 0);
+            for (int r = tid; r < rows; r += kConsumerThreads) {
+                const float g = acc[r], u = acc[kMaxRows + r];
+                h[b + r] = g / (1.0f + expf(-g)) * u;
+            }
+            break;
+        }
+        case OP_DOWN_RES:
+        case OP_MOE_DOWN2_RES:
+            for (int r = tid; r < rows; r += kConsumerThreads) {
+                float add = acc[r];
+                if (op == OP_MOE_DOWN2_RES) {
+                    add = m.ew[0] * acc[r];
+                    if (p.topk > 1) add += m.ew[1] * acc[kMaxRows + r];
+                }
+                const float nx = __ldcg(p.x + b + r) + add;
+                p.x[b + r] = nx;
+                if (p.snap) p.snap[(size_t)(l + 1) * p.H + b + r] = nx;
+            }
+            break;
+        case OP_LMHEAD_ARGMAX: {
+            float bv = -CUDART_INF_F;
+            int bi = 0x7FFFFFFF;
+            for (int r = tid; r < rows; r += kConsumerThreads) {
+                const float val = acc[r];
+                a.logits[b + r] = val;
+                if (val > bv || (val == bv && b + r < bi)) {
+                    bv = val;
+                    bi = b + r;
+                }
+            }
+            warp_argmax(bv, bi);
+            const int warp = tid >> 5;
+            if (lane == 0) {
+                m.red[warp] = bv;
+                m.redi[warp] = bi;
+            }
+            cbar();
+            if (tid == 0) {
+                for (int k = 1; k < kConsumerWarps; ++k)
+                    if (m.red[k] > bv || (m.red[k] == bv && m.redi[k] < bi)) {
+                        bv = m.red[k];
+                        bi = m.redi[k];
+                    }
+                // lanes other than 0 of warp 0 keep their own partial; only tid 0 writes
+                p.lm_part[2 * w[W_SEQ]] = bv;
+                p.lm_part[2 * w[W_SEQ] + 1] = __int_as_float(bi);
+                __threadfence();
+                const uint32_t old = atomicAdd(p.counters + w[W_AUX_CTR], 1u);
+                m.is_last = (old + 1u == a.epoch * (uint32_t)w[W_AUX_INC]) ? 1 : 0;
+            }
+            cbar();
+            if (m.is_last) {
+                __threadfence();
+                const int n_lm = w[W_AUX_INC];
+                float cv = -CUDART_INF_F;
+                int ci = 0x7FFFFFFF;
+                for (int k = tid; k < n_lm; k += kConsumerThreads) {
+                    const float val = __ldcg(p.lm_part + 2 * k);
+                    const int idx = __float_as_int(__ldcg(p.lm_part + 2 * k + 1));
+                    if (val > cv || (val == cv && idx < ci)) {
+                        cv = val;
+                        ci = idx;
+                    }
+                }
+                warp_argmax(cv, ci);
+                cbar();
+                if (lane == 0) {
+                    m.red[warp] = cv;
+                    m.redi[warp] = ci;
+                }
+                cbar();
+                if (tid == 0) {
+                    for (int k = 1; k < kConsumerWarps; ++k)
+                        if (m.red[k] > cv || (m.red[k] == cv && m.redi[k] < ci)) {
+                            cv = m.red[k];
+                            ci = m.redi[k];
+                        }
+                    p.status->next_token = ci;
+                }
+            }
+            break;
+        }
+    }
+    cbar();
+    if (tid == 0 && w[W_SIGNAL_CTR] >= 0 && op != OP_LMHEAD_ARGMAX) {
+        __threadfence();
+        atomicAdd(p.counters + w[W_SIGNAL_CTR], 1u);
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------------
+// consumers: attention (RoPE + append + one split of GQA decode attention)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ml_combine(float& m, float& l, float* o, float m2, float l2, const float* o2) {
+    const float M = fmaxf(m, m2);
+    if (M == -CUDART_INF_F) return;
+    const float a = exp2f(m - M), b = exp2f(m2 - M);
+    l = a * l + b * l2;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o[k] = a * o[k] + b * o2[k];
+    m = M;
+}
+
+template <int D, int G>
+__device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
+                           uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
+    constexpr int LPR = D / 8;                     // lanes per K/V row
+    constexpr int RGN = kConsumerThreads / LPR;    // rows per pass over the block
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int l = w[W_LAYER], g = w[W_SUB], c = w[W_BEGIN], S = w[W_END], pos = a.pos;
+    const uint32_t SB = (uint32_t)p.stage_bytes;
+    const AttnRange rg = attn_range(pos, c, S);
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * 4 : nullptr;
+
+    if (tid == 0) {
+        if (!wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, OP_ATTN))
+            vstore(&m.abort_flag, 1);
+        if (tr) tr[1] = globaltimer_ns();
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+
+    // q of the group's heads, rotated (rotate-half pairing) and pre-scaled by log2(e)/sqrt(D)
+    const int col0 = (tid % LPR) * 8;
+    const int pcol = col0 ^ (D / 2);
+    const float2* rp = p.rope + (size_t)pos * (D / 2) + (col0 & (D / 2 - 1));
+    float cs[8], sn[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float2 t = __ldg(rp + k);
+        cs[k] = t.x;
+        sn[k] = t.y;
+    }
+    const bool first_half = col0 < D / 2;
+    const float qscale = 1.4426950408889634f / sqrtf((float)D);
+    float q[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        const float* src = p.qkv + (size_t)(g * G + h) * D;
+        float x[8], y[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            x[k] = __ldcg(src + col0 + k);
+            y[k] = __ldcg(src + pcol + k);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            q[h][k] = (first_half ? x[k] * cs[k] - y[k] * sn[k] : x[k] * cs[k] + y[k] * sn[k]) * qscale;
+    }
+
+    // the new position: rotated k and v rounded to bf16 (the cache format),
+    // appended by the split that holds it (threads of row group 0)
+    float kn[8], vn[8];
+    if (rg.has_new && tid < LPR) {
+        const float* ks = p.qkv + (size_t)p.nq * D + (size_t)g * D;
+        const float* vs = p.qkv + (size_t)(p.nq + p.nkv) * D + (size_t)g * D;
+        uint32_t kb[8], vb[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float x = __ldcg(ks + col0 + k), y = __ldcg(ks + pcol + k);
+            const float r = first_half ? x * cs[k] - y * sn[k] : x * cs[k] + y * sn[k];
+            kb[k] = f2bf(r);
+            vb[k] = f2bf(__ldcg(vs + col0 + k));
+            kn[k] = __uint_as_float(kb[k] << 16);
+            vn[k] = __uint_as_float(vb[k] << 16);
+        }
+        const size_t off = (((size_t)l * p.nkv + g) * (size_t)p.max_seq + (size_t)pos) * D + col0;
+        uint4 ku, vu;
+        ku.x = kb[0] | (kb[1] << 16); ku.y = kb[2] | (kb[3] << 16); ku.z = kb[4] | (kb[5] << 16); ku.w = kb[6] | (kb[7] << 16);
+        vu.x = vb[0] | (vb[1] << 16); vu.y = vb[2] | (vb[3] << 16); vu.z = vb[4] | (vb[5] << 16); vu.w = vb[6] | (vb[7] << 16);
+        *reinterpret_cast<uint4*>(p.kcache + off) = ku;
+        *reinterpret_cast<uint4*>(p.vcache + off) = vu;
+    }
+
+    // online softmax over the cached positions streamed through the ring
+    float mx[G], ls[G], o[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        mx[h] = -CUDART_INF_F;
+        ls[h] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[h][k] = 0.f;
+    }
+    auto row_update = [&](const float* kf, const float* vf, bool valid) {
+        float s[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float t = 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t = fmaf(q[h][k], kf[k], t);
+            s[h] = t;
+        }
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1)
+#pragma unroll
+            for (int h = 0; h < G; ++h) s[h] += __shfl_xor_sync(0xFFFFFFFFu, s[h], off);
+        if (valid) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float mn = fmaxf(mx[h], s[h]);
+                const float al = exp2f(mx[h] - mn), pr = exp2f(s[h] - mn);
+                ls[h] = ls[h] * al + pr;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) o[h][k] = fmaf(pr, vf[k], o[h][k] * al);
+                mx[h] = mn;
+            }
+        }
+    };
+
+    Plan pl;
+    make_plan(p, pos, w, nullptr, pl);
+    for (int st = 0; st < pl.n_stages; ++st) {
+        const int r0 = st * pl.rps;
+        const int nr = (pl.rows - r0) < pl.rps ? (pl.rows - r0) : pl.rps;
+        const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, OP_ATTN);
+        if (tr && tid == 0 && st == 0) tr[2] = globaltimer_ns();
+        if (ok) {
+            const uint32_t Ks = smem_u32(ring) + slot * SB;
+            const uint32_t Vs = Ks + (uint32_t)pl.rps * D * 2u;
+            for (int base = 0; base < nr; base += RGN) {
+                const int r = base + tid / LPR;
+                const bool valid = r < nr;
+                float kf[8], vf[8];
+                if (valid) {
+                    unpack8(lds128(Ks + (uint32_t)(r * D + col0) * 2u), kf);
+                    unpack8(lds128(Vs + (uint32_t)(r * D + col0) * 2u), vf);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) kf[k] = vf[k] = 0.f;
+                }
+                row_update(kf, vf, valid);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        } else if (tid == 0) {
+            vstore(&m.abort_flag, 1);
+        }
+        if (++slot == p.ring_stages) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    if (rg.has_new && warp == 0) row_update(kn, vn, lane < LPR);
+
+    // merge row groups within the warp, then warps through shared memory
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float m2 = __shfl_xor_sync(0xFFFFFFFFu, mx[h], off);
+            const float l2 = __shfl_xor_sync(0xFFFFFFFFu, ls[h], off);
+            float o2[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o2[k] = __shfl_xor_sync(0xFFFFFFFFu, o[h][k], off);
+            ml_combine(mx[h], ls[h], o[h], m2, l2, o2);
+        }
+    }
+    float* sm_o = scratch;                                 // [8 warps][G][D], G*D <= 512
+    float* sm_ml = scratch + kConsumerWarps * 512;         // [8 warps][G][2]
+    cbar();  // the accumulator region may still be read by nobody, but keep the union ordered
+    if (lane < LPR) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) sm_o[(warp * G + h) * D + col0 + k] = o[h][k];
+            if (lane == 0) {
+                sm_ml[(warp * G + h) * 2] = mx[h];
+                sm_ml[(warp * G + h) * 2 + 1] = ls[h];
+            }
+        }
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+    for (int idx = tid; idx < G * D; idx += kConsumerThreads) {
+        const int h = idx / D, col = idx % D;
+        float M = -CUDART_INF_F;
+        for (int wv = 0; wv < kConsumerWarps; ++wv) M = fmaxf(M, sm_ml[(wv * G + h) * 2]);
+        float O = 0.f, Ls = 0.f;
+        if (M != -CUDART_INF_F) {
+            for (int wv = 0; wv < kConsumerWarps; ++wv) {
+                const float f = exp2f(sm_ml[(wv * G + h) * 2] - M);
+                O += f * sm_o[(wv * G + h) * D + col];
+                Ls += f * sm_ml[(wv * G + h) * 2 + 1];
+            }
+        }
+        const size_t part = (size_t)(g * G + h) * S + c;
+        p.part_o[part * D + col] = O;
+        if (col == 0) {
+            p.part_ml[part * 2] = M;
+            p.part_ml[part * 2 + 1] = Ls;
+        }
+    }
+    cbar();
+    if (tid == 0) {
+        __threadfence();
+        const uint32_t old = atomicAdd(p.counters + w[W_AUX_CTR], 1u);
+        m.is_last = (old + 1u == a.epoch * (uint32_t)w[W_AUX_INC]) ? 1 : 0;
+    }
+    cbar();
+    if (m.is_last) {
+        // last split of this kv head: merge all splits' partials into attn
+        __threadfence();
+        for (int idx = tid; idx < G * D; idx += kConsumerThreads) {
+            const int h = idx / D, col = idx % D;
+            const size_t base = (size_t)(g * G + h) * S;
+            float M = -CUDART_INF_F;
+            for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(p.part_ml + (base + s) * 2));
+            float num = 0.f, den = 0.f;
+            for (int s = 0; s < S; ++s) {
+                const float ms = __ldcg(p.part_ml + (base + s) * 2);
+                const float f = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
+                num += f * __ldcg(p.part_o + (base + s) * D + col);
+                den += f * __ldcg(p.part_ml + (base + s) * 2 + 1);
+            }
+            p.attn[(size_t)(g * G + h) * D + col] = num / den;
+        }
+        cbar();
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(p.counters + w[W_SIGNAL_CTR], 1u);
+        }
+    }
+    return true;
+}
+
+template <int D>
+__device__ bool attn_dispatch_g(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
+                                uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
+    switch (p.nq / p.nkv) {
+        case 1: return attn_instr<D, 1>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+        case 2: return attn_instr<D, 2>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+        case 3: return attn_instr<D, 3>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+        case 4: return attn_instr<D, 4>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+    }
+    return false;
+}
+
+__device__ __forceinline__ int gemv_k(const DevParams& p, int op) {
+    switch (op) {
+        case OP_OPROJ_RES: return p.nq * p.d;
+        case OP_DOWN_RES:
+        case OP_MOE_DOWN2_RES: return p.F;
+    }
+    return p.H;
+}
+
+__device__ bool gemv_dispatch(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
+                              uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase,
+                              int token) {
+    const int K = gemv_k(p, w[W_OP]);
+    const int kp = K / kparts_of(K);
+    const int J = ((kp >> 3) + kConsumerThreads - 1) / kConsumerThreads;
+    switch (J) {
+        case 1: return gemv_instr<1>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+        case 2: return gemv_instr<2>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+        case 3: return gemv_instr<3>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+        case 4: return gemv_instr<4>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+    }
+    return false;
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ DevParams p, const StepArgs a) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int NS = p.ring_stages, SB = p.stage_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + smem_bars_off(NS, SB));
+    uint64_t* empty = full + NS;
+    float* scratch = reinterpret_cast<float*>(smem + smem_scratch_off(NS, SB));
+    Misc& m = *reinterpret_cast<Misc*>(smem + smem_misc_off(NS, SB));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        m.router_layer = -1;
+        m.is_last = 0;
+        m.abort_flag = ld_relaxed_s32(&p.status->stop) ? 1 : 0;
+        if (m.abort_flag && atomicCAS(&p.status->code, 0, MK_ERR_STOPPED) == 0) p.status->sm = blockIdx.x;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (m.abort_flag) return;
+
+    const int n = p.n_instr[blockIdx.x];
+    const int32_t* q = p.instr + (size_t)blockIdx.x * p.max_instr * W_NWORDS;
+    if (warp == kConsumerWarps) {
+        if (lane == 0) loader(p, a, q, n, smem, full, empty, m);
+        return;
+    }
+
+    const int token = a.token >= 0 ? a.token : __ldcg(&p.status->next_token);
+    int slot = 0;
+    uint32_t phase = 0;
+    for (int i = 0; i < n; ++i) {
+        const int32_t* w = q + (size_t)i * W_NWORDS;
+        if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * 4] = globaltimer_ns();
+        bool ok;
+        if (!instr_ok(p, w) || token < 0 || token >= p.V) {
+            if (tid == 0) {
+                record_error(p.status, MK_ERR_BAD_INSTR, blockIdx.x, i, w[W_OP], -1, (uint32_t)token, 0);
+                vstore(&m.abort_flag, 1);
+            }
+            ok = false;
+        } else if (w[W_OP] == OP_ATTN) {
+            ok = p.d == 64 ? attn_dispatch_g<64>(p, a, w, i, smem, full, empty, scratch, m, slot, phase)
+                           : attn_dispatch_g<128>(p, a, w, i, smem, full, empty, scratch, m, slot, phase);
+        } else {
+            ok = gemv_dispatch(p, a, w, i, smem, full, empty, scratch, m, slot, phase, token);
+        }
+        if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * 4 + 3] = globaltimer_ns();
+        if (!ok) break;
+    }
+    if (tid == 0) vstore(&m.abort_flag, 1);  // lets the loader stop early if it is still waiting
+}
+
+cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, cudaStream_t stream) {
+    const size_t smem = megakernel_smem_bytes(p.ring_stages, p.stage_bytes);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_sm);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, megakernel, p, a);
+}
+
+cudaError_t prepare_megakernel(int ring_stages, int stage_bytes, int* max_blocks_per_sm) {
+    const size_t smem = megakernel_smem_bytes(ring_stages, stage_bytes);
+    cudaError_t e = cudaFuncSetAttribute(megakernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(max_blocks_per_sm, megakernel, kThreads, smem);
+}
+
+}  // namespace mk

@@ -1,0 +1,29 @@
+// mk_plan.h -- host-side schedule planning (no CUDA dependency).
+#pragma once
+#include <cstdint>
+#include <vector>
+
+#include "mk_internal.h"
+
+namespace mk {
+
+struct Planned {
+    int n_sm = 0;
+    int max_instr = 0;
+    int kv_splits = 1;
+    int n_lm = 0;                  // LM-head instructions (partial argmax slots)
+    std::vector<int32_t> words;    // [n_sm][max_instr][W_NWORDS]
+    std::vector<int32_t> n_instr;  // [n_sm]
+    std::vector<uint32_t> ctr_inc; // per-step increment of every counter
+};
+
+int check_config(const mk_config& c);
+int check_options(const mk_config& c, const mk_options& o);
+void fill_defaults(mk_options* o);
+int default_kv_splits(const mk_config& c, int n_sm);
+int plan_schedule(const mk_config& c, const mk_options& o, int n_sm, Planned* out);
+int validate(const mk_config& c, const Planned& p);
+int simulate(const int32_t* words, int n_sm, int max_instr, const int32_t* n_instr, const uint32_t* ctr_inc,
+             int nctr, int steps, uint64_t seed, long long* executed);
+
+}  // namespace mk

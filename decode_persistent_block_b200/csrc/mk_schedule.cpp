@@ -1,0 +1,443 @@
+// mk_schedule.cpp -- host scheduler: splits every op of one decode step into
+// instructions, assigns them to per-SM queues, sets the dependency counters,
+// validates the result and can execute it on the host under random
+// interleavings.
+//
+// The pages name the hard parts of a megakernel schedule: "a barrier that does
+// not deadlock, a schedule that keeps every SM busy when layers have different
+// shapes, and correctness checks" (Hyperkernel teardown, "What a megakernel
+// buys").  Here:
+//  - every SM queue is sorted by global op index and every wait targets a
+//    counter signalled only by strictly earlier ops, so some instruction is
+//    always runnable (checked by validate() and exercised by simulate());
+//  - every GEMV op is split into one contiguous row range per SM of equal
+//    bytes (+-1 row), so each op spans all SMs whatever its shape;
+//  - attention is split along the sequence (split-KV) into kv_heads * splits
+//    instructions so that the low-occupancy op still covers ~all SMs
+//    (epic-kernel README, "Speculative expert prediction": attention "has low
+//    SM occupancy").
+#include <algorithm>
+#include <array>
+#include <cstdint>
+#include <cstring>
+#include <random>
+#include <vector>
+
+#include "mk_internal.h"
+#include "mk_plan.h"
+
+namespace mk {
+
+namespace {
+
+using Instr = std::array<int32_t, W_NWORDS>;
+
+Instr blank() {
+    Instr w;
+    w.fill(0);
+    w[W_WAIT_CTR] = -1;
+    w[W_SIGNAL_CTR] = -1;
+    w[W_AUX_CTR] = -1;
+    return w;
+}
+
+struct Segment {
+    int sub;   // tensor / slot selector stored in W_SUB
+    int rows;
+};
+
+// Split the virtual concatenation of `segs` into one contiguous range per SM,
+// cut at segment boundaries and at `cap` rows.  Calls emit(sm, sub, begin, end).
+template <class F>
+void split_rows(const std::vector<Segment>& segs, int n_sm, int cap, F emit) {
+    long long total = 0;
+    for (auto& s : segs) total += s.rows;
+    for (int sm = 0; sm < n_sm; ++sm) {
+        long long a = total * sm / n_sm, b = total * (sm + 1) / n_sm;
+        long long base = 0;
+        for (auto& s : segs) {
+            long long lo = std::max(a, base), hi = std::min(b, base + s.rows);
+            for (long long r = lo; r < hi; r += cap) {
+                long long e = std::min(hi, r + cap);
+                emit(sm, s.sub, (int)(r - base), (int)(e - base));
+            }
+            base += s.rows;
+        }
+    }
+}
+
+}  // namespace
+
+int default_kv_splits(const mk_config& c, int n_sm) {
+    int s = std::max(1, n_sm / std::max(1, c.n_kv_heads));
+    int cap = std::max(1, (c.max_seq + 31) / 32);
+    return std::min(s, cap);
+}
+
+int check_config(const mk_config& c) {
+    if (c.n_layers < 0 || c.hidden <= 0 || c.n_q_heads <= 0 || c.n_kv_heads <= 0 || c.head_dim <= 0 ||
+        c.ffn <= 0 || c.vocab <= 0 || c.max_seq <= 0 || c.n_experts < 0)
+        return MK_ERR_INVALID_ARG;
+    if (!(c.rms_eps >= 0.f) || !(c.rope_theta > 0.f)) return MK_ERR_INVALID_ARG;
+    if (c.head_dim != 64 && c.head_dim != 128) return MK_ERR_UNSUPPORTED;
+    if (c.n_q_heads % c.n_kv_heads) return MK_ERR_UNSUPPORTED;
+    {
+        const int g = c.n_q_heads / c.n_kv_heads;  // query heads per kv head (attention kernel instances)
+        if (g < 1 || g > 4) return MK_ERR_UNSUPPORTED;  // attention kernel instances
+    }
+    const int qd = c.n_q_heads * c.head_dim;
+    for (int k : {c.hidden, c.ffn, qd}) {
+        if (k % 8 || k > 16384) return MK_ERR_UNSUPPORTED;
+        // rows wider than 8192 columns are reduced in equal column parts of whole 8-element chunks
+        const int parts = (k + 8191) / 8192;
+        if (k % (8 * parts)) return MK_ERR_UNSUPPORTED;
+    }
+    if (c.hidden > 8192) return MK_ERR_UNSUPPORTED;  // RMSNorm inputs are never split
+    if (c.n_experts > 0 && (c.top_k < 1 || c.top_k > kMaxTopK || c.top_k > c.n_experts || c.n_experts > 64))
+        return MK_ERR_UNSUPPORTED;
+    return MK_OK;
+}
+
+void fill_defaults(mk_options* o) {
+    if (o->ring_stages <= 0) o->ring_stages = 6;
+    if (o->stage_bytes <= 0) o->stage_bytes = 32768;
+    if (o->rows_per_instr <= 0 || o->rows_per_instr > kMaxRows) o->rows_per_instr = kMaxRows;
+    if (o->l2_prefetch < 0) o->l2_prefetch = 0;
+    if (o->spin_limit_ns == 0) o->spin_limit_ns = 2000000000ull;
+}
+
+int check_options(const mk_config& c, const mk_options& o) {
+    if (o.stage_bytes % 1024 || o.stage_bytes < 4096 || o.ring_stages < 2 || o.ring_stages > 32)
+        return MK_ERR_INVALID_ARG;
+    // one GEMV stage holds at least one row of every span: up/gate pairs of
+    // hidden-wide rows, and one ffn-wide (down) or heads*dim-wide (o) row.
+    const long long sb = o.stage_bytes;
+    auto part_bytes = [](long long k) { return 2LL * (k / ((k + 8191) / 8192)); };
+    if (2LL * 2 * c.hidden > sb || part_bytes(c.ffn) > sb || part_bytes((long long)c.n_q_heads * c.head_dim) > sb)
+        return MK_ERR_UNSUPPORTED;
+    if (2LL * 2 * c.head_dim > sb) return MK_ERR_UNSUPPORTED;
+    if (o.mode < MK_MODE_MEGAKERNEL || o.mode > MK_MODE_MULTI_KERNEL_GRAPH) return MK_ERR_INVALID_ARG;
+    return MK_OK;
+}
+
+int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned* out) {
+    int rc = check_config(c);
+    if (rc) return rc;
+    if (n_sm <= 0) return MK_ERR_INVALID_ARG;
+    mk_options o = o_in;
+    fill_defaults(&o);
+    const int L = c.n_layers, nkv = c.n_kv_heads, d = c.head_dim, H = c.hidden, F = c.ffn;
+    const int S = o.kv_splits > 0 ? o.kv_splits : default_kv_splits(c, n_sm);
+    const int cap = o.rows_per_instr;
+    const bool moe = c.n_experts > 0;
+
+    std::vector<std::vector<Instr>> q(n_sm);
+    std::vector<uint32_t> inc(n_counters(L, nkv), 0);
+
+    auto add = [&](int sm, Instr w) {
+        q[sm].push_back(w);
+        if (w[W_SIGNAL_CTR] >= 0 && w[W_OP] != OP_ATTN) inc[w[W_SIGNAL_CTR]]++;
+        if (w[W_AUX_CTR] >= 0) inc[w[W_AUX_CTR]]++;
+    };
+    auto gemv_op = [&](int op, int layer, const std::vector<Segment>& segs, int wait, int signal) {
+        split_rows(segs, n_sm, cap, [&](int sm, int sub, int b, int e) {
+            Instr w = blank();
+            w[W_OP] = op;
+            w[W_LAYER] = layer;
+            w[W_SUB] = sub;
+            w[W_BEGIN] = b;
+            w[W_END] = e;
+            w[W_WAIT_CTR] = wait;
+            w[W_SIGNAL_CTR] = signal;
+            add(sm, w);
+        });
+    };
+
+    for (int l = 0; l < L; ++l) {
+        const int prev_down = l > 0 ? ctr_id(l - 1, C_FFN2, nkv) : -1;
+        gemv_op(OP_RMS_QKV, l, {{0, c.n_q_heads * d}, {1, nkv * d}, {2, nkv * d}}, prev_down,
+                ctr_id(l, C_QKV, nkv));
+        // attention: kv head g, split s -> instruction k = g * S + s, rotated per layer
+        const int total = nkv * S;
+        for (int k = 0; k < total; ++k) {
+            Instr w = blank();
+            w[W_OP] = OP_ATTN;
+            w[W_LAYER] = l;
+            w[W_SUB] = k / S;
+            w[W_BEGIN] = k % S;
+            w[W_END] = S;
+            w[W_WAIT_CTR] = ctr_id(l, C_QKV, nkv);
+            w[W_SIGNAL_CTR] = ctr_id(l, C_ATTN, nkv);
+            w[W_AUX_CTR] = ctr_id(l, C_GROUP0 + k / S, nkv);
+            int sm = (int)(((long long)k + (long long)l * total) % n_sm);
+            add(sm, w);
+        }
+        inc[ctr_id(l, C_ATTN, nkv)] = nkv;  // one signal per kv head, by its last-arriving split
+        gemv_op(OP_OPROJ_RES, l, {{0, H}}, ctr_id(l, C_ATTN, nkv), ctr_id(l, C_OPROJ, nkv));
+        if (!moe) {
+            gemv_op(OP_RMS_UPGATE_SILU, l, {{0, F}}, ctr_id(l, C_OPROJ, nkv), ctr_id(l, C_FFN1, nkv));
+            gemv_op(OP_DOWN_RES, l, {{0, H}}, ctr_id(l, C_FFN1, nkv), ctr_id(l, C_FFN2, nkv));
+        } else {
+            std::vector<Segment> slots;
+            for (int s = 0; s < c.top_k; ++s) slots.push_back({s, F});
+            gemv_op(OP_MOE_UPGATE, l, slots, ctr_id(l, C_OPROJ, nkv), ctr_id(l, C_FFN1, nkv));
+            gemv_op(OP_MOE_DOWN2_RES, l, {{0, H}}, ctr_id(l, C_FFN1, nkv), ctr_id(l, C_FFN2, nkv));
+        }
+    }
+    // LM head + argmax: partial slots numbered in emission order
+    {
+        int seq = 0;
+        const int wait = L > 0 ? ctr_id(L - 1, C_FFN2, nkv) : -1;
+        split_rows({{0, c.vocab}}, n_sm, cap, [&](int sm, int, int b, int e) {
+            Instr w = blank();
+            w[W_OP] = OP_LMHEAD_ARGMAX;
+            w[W_LAYER] = L;
+            w[W_BEGIN] = b;
+            w[W_END] = e;
+            w[W_WAIT_CTR] = wait;
+            w[W_AUX_CTR] = ctr_lm(L, nkv);
+            w[W_SEQ] = seq++;
+            add(sm, w);
+        });
+    }
+    // fill wait increments and aux increments
+    for (auto& qs : q)
+        for (auto& w : qs) {
+            w[W_WAIT_INC] = w[W_WAIT_CTR] >= 0 ? (int32_t)inc[w[W_WAIT_CTR]] : 0;
+            w[W_AUX_INC] = w[W_AUX_CTR] >= 0 ? (int32_t)inc[w[W_AUX_CTR]] : 0;
+        }
+
+    int max_instr = 1;
+    for (auto& qs : q) max_instr = std::max<int>(max_instr, (int)qs.size());
+    out->n_sm = n_sm;
+    out->max_instr = max_instr;
+    out->kv_splits = S;
+    out->n_lm = (int)inc[ctr_lm(L, nkv)];
+    out->words.assign((size_t)n_sm * max_instr * W_NWORDS, 0);
+    out->n_instr.assign(n_sm, 0);
+    for (int sm = 0; sm < n_sm; ++sm) {
+        out->n_instr[sm] = (int32_t)q[sm].size();
+        for (size_t i = 0; i < q[sm].size(); ++i)
+            std::memcpy(&out->words[((size_t)sm * max_instr + i) * W_NWORDS], q[sm][i].data(),
+                        sizeof(int32_t) * W_NWORDS);
+    }
+    out->ctr_inc = inc;
+    return validate(c, *out);
+}
+
+// Global op index of an instruction: 5 ops per layer, LM head last.
+static int op_index(const int32_t* w) {
+    int slot = 0;
+    switch (w[W_OP]) {
+        case OP_RMS_QKV: slot = 0; break;
+        case OP_ATTN: slot = 1; break;
+        case OP_OPROJ_RES: slot = 2; break;
+        case OP_RMS_UPGATE_SILU:
+        case OP_MOE_UPGATE: slot = 3; break;
+        case OP_DOWN_RES:
+        case OP_MOE_DOWN2_RES: slot = 4; break;
+        case OP_LMHEAD_ARGMAX: slot = 0; break;
+        default: return -1;
+    }
+    return w[W_LAYER] * 5 + slot;
+}
+
+// Op index of the op that signals counter `ctr` (LM arrival counter: n_layers*5).
+static int producer_op(int ctr, int L, int nkv) {
+    if (ctr == ctr_lm(L, nkv)) return L * 5;
+    const int per = counters_per_layer(nkv);
+    const int l = ctr / per, slot = ctr % per;
+    switch (slot) {
+        case C_QKV: return l * 5 + 0;
+        case C_ATTN: return l * 5 + 1;
+        case C_OPROJ: return l * 5 + 2;
+        case C_FFN1: return l * 5 + 3;
+        case C_FFN2: return l * 5 + 4;
+        default: return l * 5 + 1;  // head-group arrival counters belong to attention
+    }
+}
+
+int validate(const mk_config& c, const Planned& p) {
+    const int L = c.n_layers, nkv = c.n_kv_heads, d = c.head_dim;
+    const int nctr = n_counters(L, nkv);
+    if ((int)p.ctr_inc.size() != nctr) return MK_ERR_SCHEDULE;
+    const bool moe = c.n_experts > 0;
+    // coverage bitmaps: per (layer, op, sub) rows covered exactly once
+    std::vector<std::vector<uint8_t>> cov;
+    auto cov_key = [&](int l, int op, int sub) { return ((size_t)l * OP_COUNT + op) * 4 + sub; };
+    cov.resize((size_t)(L + 1) * OP_COUNT * 4);
+    auto rows_of = [&](int op, int sub) -> int {
+        switch (op) {
+            case OP_RMS_QKV: return sub == 0 ? c.n_q_heads * d : nkv * d;
+            case OP_OPROJ_RES: case OP_DOWN_RES: case OP_MOE_DOWN2_RES: return c.hidden;
+            case OP_RMS_UPGATE_SILU: case OP_MOE_UPGATE: return c.ffn;
+            case OP_LMHEAD_ARGMAX: return c.vocab;
+        }
+        return -1;
+    };
+    std::vector<uint32_t> signals(nctr, 0);
+    std::vector<std::vector<uint8_t>> attn_seen((size_t)std::max(L, 1) * nkv, std::vector<uint8_t>(p.kv_splits, 0));
+    std::vector<uint8_t> lm_seq(std::max(p.n_lm, 1), 0);
+    for (int sm = 0; sm < p.n_sm; ++sm) {
+        int last_op = -1;
+        std::vector<uint8_t> had_moe_ug(std::max(L, 1), 0);
+        if (p.n_instr[sm] < 0 || p.n_instr[sm] > p.max_instr) return MK_ERR_SCHEDULE;
+        for (int i = 0; i < p.n_instr[sm]; ++i) {
+            const int32_t* w = &p.words[((size_t)sm * p.max_instr + i) * W_NWORDS];
+            const int op = w[W_OP], l = w[W_LAYER];
+            if (op <= OP_NOP || op >= OP_COUNT) return MK_ERR_SCHEDULE;
+            if (moe != (op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES) &&
+                (op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES || op == OP_RMS_UPGATE_SILU || op == OP_DOWN_RES))
+                return MK_ERR_SCHEDULE;
+            if (op == OP_LMHEAD_ARGMAX ? l != L : (l < 0 || l >= L)) return MK_ERR_SCHEDULE;
+            const int oi = op_index(w);
+            if (oi < last_op) return MK_ERR_SCHEDULE;  // queue sorted by global op order
+            last_op = oi;
+            // waits only on counters produced by strictly earlier ops, with the planned increment
+            if (w[W_WAIT_CTR] >= 0) {
+                if (w[W_WAIT_CTR] >= nctr) return MK_ERR_SCHEDULE;
+                if (producer_op(w[W_WAIT_CTR], L, nkv) >= oi) return MK_ERR_SCHEDULE;
+                if ((uint32_t)w[W_WAIT_INC] != p.ctr_inc[w[W_WAIT_CTR]] || w[W_WAIT_INC] <= 0) return MK_ERR_SCHEDULE;
+            } else if (!(op == OP_RMS_QKV && l == 0) && !(op == OP_LMHEAD_ARGMAX && L == 0)) {
+                return MK_ERR_SCHEDULE;  // everything but the first op depends on something
+            }
+            if (w[W_SIGNAL_CTR] >= nctr || w[W_AUX_CTR] >= nctr) return MK_ERR_SCHEDULE;
+            if (w[W_AUX_CTR] >= 0 && (uint32_t)w[W_AUX_INC] != p.ctr_inc[w[W_AUX_CTR]]) return MK_ERR_SCHEDULE;
+            if (op == OP_ATTN) {
+                const int g = w[W_SUB], s = w[W_BEGIN];
+                if (g < 0 || g >= nkv || s < 0 || s >= p.kv_splits || w[W_END] != p.kv_splits) return MK_ERR_SCHEDULE;
+                if (w[W_AUX_CTR] != ctr_id(l, C_GROUP0 + g, nkv) || w[W_SIGNAL_CTR] != ctr_id(l, C_ATTN, nkv))
+                    return MK_ERR_SCHEDULE;
+                if (attn_seen[(size_t)l * nkv + g][s]++) return MK_ERR_SCHEDULE;
+                signals[w[W_AUX_CTR]]++;
+                continue;
+            }
+            if (op == OP_MOE_UPGATE) had_moe_ug[l] = 1;
+            if (op == OP_MOE_DOWN2_RES && !had_moe_ug[l]) return MK_ERR_SCHEDULE;  // routing known on this SM
+            const int sub = w[W_SUB];
+            const int R = rows_of(op, op == OP_RMS_QKV ? sub : 0);
+            if (op == OP_RMS_QKV && (sub < 0 || sub > 2)) return MK_ERR_SCHEDULE;
+            if (op == OP_MOE_UPGATE && (sub < 0 || sub >= c.top_k)) return MK_ERR_SCHEDULE;
+            if (op != OP_RMS_QKV && op != OP_MOE_UPGATE && sub != 0) return MK_ERR_SCHEDULE;
+            const int b = w[W_BEGIN], e = w[W_END];
+            if (b < 0 || e > R || b >= e || e - b > kMaxRows) return MK_ERR_SCHEDULE;
+            auto& hits = cov[cov_key(l, op, sub)];
+            if (hits.empty()) hits.assign(R, 0);
+            for (int r = b; r < e; ++r)
+                if (hits[r]++) return MK_ERR_SCHEDULE;
+            if (op == OP_LMHEAD_ARGMAX) {
+                if (w[W_AUX_CTR] != ctr_lm(L, nkv) || w[W_SEQ] < 0 || w[W_SEQ] >= p.n_lm || lm_seq[w[W_SEQ]]++)
+                    return MK_ERR_SCHEDULE;
+                signals[w[W_AUX_CTR]]++;
+            } else {
+                if (w[W_SIGNAL_CTR] < 0) return MK_ERR_SCHEDULE;
+                signals[w[W_SIGNAL_CTR]]++;
+            }
+        }
+    }
+    // every op fully covered
+    for (int l = 0; l <= L; ++l)
+        for (int op = 1; op < OP_COUNT; ++op)
+            for (int sub = 0; sub < 4; ++sub) {
+                auto& hits = cov[cov_key(l, op, sub)];
+                for (auto h : hits)
+                    if (h != 1) return MK_ERR_SCHEDULE;
+            }
+    for (int l = 0; l < L; ++l) {
+        for (int g = 0; g < nkv; ++g)
+            for (int s = 0; s < p.kv_splits; ++s)
+                if (attn_seen[(size_t)l * nkv + g][s] != 1) return MK_ERR_SCHEDULE;
+        for (int op : {OP_RMS_QKV, OP_OPROJ_RES, moe ? OP_MOE_UPGATE : OP_RMS_UPGATE_SILU,
+                       moe ? OP_MOE_DOWN2_RES : OP_DOWN_RES})
+            if (cov[cov_key(l, op, 0)].empty()) return MK_ERR_SCHEDULE;
+        signals[ctr_id(l, C_ATTN, nkv)] = nkv;  // emitted by the merging split of each head group
+    }
+    if (cov[cov_key(L, OP_LMHEAD_ARGMAX, 0)].empty()) return MK_ERR_SCHEDULE;
+    for (int i = 0; i < nctr; ++i)
+        if (signals[i] != p.ctr_inc[i]) return MK_ERR_SCHEDULE;
+    return MK_OK;
+}
+
+int simulate(const int32_t* words, int n_sm, int max_instr, const int32_t* n_instr, const uint32_t* ctr_inc,
+             int nctr, int steps, uint64_t seed, long long* executed) {
+    std::vector<uint64_t> ctr(nctr, 0);
+    std::mt19937_64 rng(seed);
+    long long done = 0;
+    for (int e = 1; e <= steps; ++e) {
+        std::vector<int> pc(n_sm, 0);
+        long long remaining = 0;
+        for (int sm = 0; sm < n_sm; ++sm) remaining += n_instr[sm];
+        std::vector<int> ready;
+        while (remaining > 0) {
+            ready.clear();
+            for (int sm = 0; sm < n_sm; ++sm) {
+                if (pc[sm] >= n_instr[sm]) continue;
+                const int32_t* w = words + ((size_t)sm * max_instr + pc[sm]) * W_NWORDS;
+                const int wc = w[W_WAIT_CTR];
+                if (wc < 0 || ctr[wc] >= (uint64_t)e * (uint32_t)w[W_WAIT_INC]) ready.push_back(sm);
+            }
+            if (ready.empty()) {
+                if (executed) *executed = done;
+                return MK_ERR_SCHEDULE;  // deadlock
+            }
+            const int sm = ready[rng() % ready.size()];
+            const int32_t* w = words + ((size_t)sm * max_instr + pc[sm]) * W_NWORDS;
+            if (w[W_OP] == OP_ATTN) {
+                const uint64_t now = ++ctr[w[W_AUX_CTR]];
+                if (now == (uint64_t)e * (uint32_t)w[W_AUX_INC]) ctr[w[W_SIGNAL_CTR]]++;  // last split merges
+            } else {
+                if (w[W_AUX_CTR] >= 0) ctr[w[W_AUX_CTR]]++;
+                if (w[W_SIGNAL_CTR] >= 0) ctr[w[W_SIGNAL_CTR]]++;
+            }
+            pc[sm]++;
+            remaining--;
+            done++;
+        }
+    }
+    if (executed) *executed = done;
+    for (int i = 0; i < nctr; ++i)
+        if (ctr[i] != (uint64_t)steps * ctr_inc[i]) return MK_ERR_SCHEDULE;
+    return MK_OK;
+}
+
+}  // namespace mk
+
+extern "C" int mk_plan(const mk_config* cfg, const mk_options* opt, int n_sm, int32_t* buf, size_t cap,
+                       int* max_instr, int32_t* n_instr, uint32_t* ctr_inc, size_t ctr_cap, int* n_ctr) {
+    if (!cfg || n_sm <= 0) return MK_ERR_INVALID_ARG;
+    mk_options o;
+    if (opt) o = *opt; else mk_default_options(&o);
+    mk::fill_defaults(&o);
+    int rc = mk::check_config(*cfg);
+    if (rc) return rc;
+    rc = mk::check_options(*cfg, o);
+    if (rc) return rc;
+    mk::Planned p;
+    rc = mk::plan_schedule(*cfg, o, n_sm, &p);
+    if (rc) return rc;
+    if (max_instr) *max_instr = p.max_instr;
+    if (n_ctr) *n_ctr = (int)p.ctr_inc.size();
+    if (!buf || cap < p.words.size() || !n_instr || (ctr_inc && ctr_cap < p.ctr_inc.size())) return MK_ERR_CAPACITY;
+    std::memcpy(buf, p.words.data(), p.words.size() * sizeof(int32_t));
+    std::memcpy(n_instr, p.n_instr.data(), sizeof(int32_t) * n_sm);
+    if (ctr_inc) std::memcpy(ctr_inc, p.ctr_inc.data(), p.ctr_inc.size() * sizeof(uint32_t));
+    return MK_OK;
+}
+
+extern "C" int mk_simulate(const int32_t* buf, int n_sm, int max_instr, const int32_t* n_instr,
+                           const uint32_t* ctr_inc, int n_counters, int steps, uint64_t seed, long long* executed) {
+    if (!buf || !n_instr || !ctr_inc || n_sm <= 0 || max_instr <= 0 || n_counters <= 0 || steps < 0)
+        return MK_ERR_INVALID_ARG;
+    // reject out-of-range counter ids before touching them
+    for (int sm = 0; sm < n_sm; ++sm) {
+        if (n_instr[sm] < 0 || n_instr[sm] > max_instr) return MK_ERR_INVALID_ARG;
+        for (int i = 0; i < n_instr[sm]; ++i) {
+            const int32_t* w = buf + ((size_t)sm * max_instr + i) * mk::W_NWORDS;
+            for (int k : {mk::W_WAIT_CTR, mk::W_SIGNAL_CTR, mk::W_AUX_CTR})
+                if (w[k] >= n_counters || w[k] < -1) return MK_ERR_INVALID_ARG;
+            if (w[mk::W_OP] == mk::OP_ATTN && (w[mk::W_AUX_CTR] < 0 || w[mk::W_SIGNAL_CTR] < 0))
+                return MK_ERR_INVALID_ARG;
+        }
+    }
+    return mk::simulate(buf, n_sm, max_instr, n_instr, ctr_inc, n_counters, steps, seed, executed);
+}

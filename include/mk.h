@@ -1,0 +1,219 @@
+/*
+ * mk.h -- C ABI of the persistent batch-1 decode megakernel for one B200 (sm_100a).
+ *
+ * What the library computes: one greedy decode step of a Llama-style decoder
+ * (optionally with a top-k MoE FFN) for a single sequence, as ONE persistent
+ * kernel with one block per SM whose blocks never exit mid-step and read, at
+ * run time, a host-built instruction tensor that tells each block which
+ * operation to run next ("a single persistent CUDA kernel that occupies the
+ * entire GPU and reads an instruction tensor at runtime to decide what work
+ * each SM does next": Kittens VM summary page, "Method"; "Launch one kernel
+ * with one block per SM ... Never let the blocks exit ... synchronize with each
+ * other on the device": Hyperkernel teardown, "What a megakernel buys").
+ * Dependencies between instructions are global-memory counters.  Weight tiles
+ * stream through a multi-stage shared-memory ring fed by TMA bulk copies, with
+ * an L2 prefetch of the following weights (epic-kernel README, "Pipelining for
+ * B200 bandwidth", "L2 prefetching overlapped with prior instructions").
+ *
+ * Conventions for every function:
+ *  - Return value: MK_OK (0) or a negative MK_ERR_* code; nothing here calls
+ *    exit() or abort().  mk_strerror() names a code.
+ *  - Pointers documented as "device" are CUDA device addresses on the device
+ *    that was current at mk_create(); "host" pointers are ordinary CPU memory.
+ *  - A handle is not thread-safe: one call at a time per handle.
+ *
+ * Data layout (all row-major, the nn.Linear [out, in] convention):
+ *   bf16 weights: embed/lm_head [vocab, hidden]; wq [n_q_heads*head_dim, hidden];
+ *   wk, wv [n_kv_heads*head_dim, hidden]; wo [hidden, n_q_heads*head_dim];
+ *   w_gate, w_up [ffn, hidden]; w_down [hidden, ffn]; router [n_experts, hidden];
+ *   norm weights [hidden].
+ *   KV cache (bf16, caller-owned): k_cache, v_cache [n_layers][n_kv_heads][max_seq][head_dim].
+ *   Activations inside the library are fp32; logits are fp32 [vocab].
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ----------------------------------------------------------- */
+#define MK_OK 0
+#define MK_ERR_INVALID_ARG (-1)   /* bad config, null pointer, pos >= max_seq, token outside [0, vocab) */
+#define MK_ERR_CUDA (-2)          /* a CUDA runtime call failed; mk_status.cuda_error holds the cudaError_t */
+#define MK_ERR_NOT_RESIDENT (-3)  /* the one-block-per-SM cooperative grid cannot be co-resident */
+#define MK_ERR_TIMEOUT (-4)       /* a bounded device wait ran out (dependency counter or smem ring) */
+#define MK_ERR_BAD_INSTR (-5)     /* the device met an opcode or index outside the valid range */
+#define MK_ERR_SCHEDULE (-6)      /* the host validator rejected the schedule */
+#define MK_ERR_STOPPED (-7)       /* the stop word was set before or during the step */
+#define MK_ERR_NO_SCHEDULE (-8)   /* mk_decode_step before mk_build_schedule */
+#define MK_ERR_CAPACITY (-9)      /* a caller buffer is too small */
+#define MK_ERR_UNSUPPORTED (-10)  /* shape outside what the kernels handle (see mk_create) */
+
+/* ---- execution modes -------------------------------------------------------- */
+#define MK_MODE_MEGAKERNEL 0        /* one persistent cooperative launch per step */
+#define MK_MODE_MULTI_KERNEL 1      /* baseline: one plain launch per op and layer */
+#define MK_MODE_MULTI_KERNEL_GRAPH 2/* baseline launches replayed from a CUDA graph */
+
+/* ---- fault injection (host side; see mk_inject_fault) ------------------------ */
+#define MK_FAULT_NONE 0
+#define MK_FAULT_UNREACHABLE_WAIT 1 /* one instruction waits for a counter value no step reaches */
+#define MK_FAULT_BAD_OPCODE 2       /* one instruction carries an opcode outside the table */
+#define MK_FAULT_PRESET_STOP 3      /* the stop word is set before the launch */
+
+/* Model shape.  n_experts = 0 selects the dense SiLU-gated FFN; otherwise each
+ * layer's FFN is a top_k-of-n_experts MoE (top_k in {1, 2}, n_experts <= 64).
+ * Supported (else MK_ERR_UNSUPPORTED): head_dim in {64, 128}; 1 to 4 query
+ * heads per kv head; hidden <= 8192; hidden, ffn and n_q_heads*head_dim
+ * multiples of 8 and at most 16384, and a width above 8192 must split into 2
+ * equal parts of whole 8-element chunks.  tied_embeddings: lm_head may equal
+ * embed (informational). */
+typedef struct {
+    int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+    int n_experts, top_k;
+    float rms_eps, rope_theta;
+    int max_seq;
+    int tied_embeddings;
+} mk_config;
+
+/* Device pointers to bf16 weights and the bf16 KV caches; all caller-owned and
+ * kept alive for the handle's lifetime (the library reads them, and writes the
+ * KV caches at the decoded position).  Per-layer arrays are HOST arrays of
+ * n_layers device pointers; for MoE, w_gate/w_up/w_down have
+ * n_layers * n_experts entries ([layer * n_experts + expert]) and router has
+ * n_layers entries.  router may be NULL for dense models.  All device
+ * pointers must be 16-byte aligned. */
+typedef struct {
+    const void *embed, *lm_head, *final_norm;
+    const void *const *attn_norm, *const *wq, *const *wk, *const *wv, *const *wo, *const *ffn_norm;
+    const void *const *w_gate, *const *w_up, *const *w_down;
+    const void *const *router;
+    void *k_cache, *v_cache;
+} mk_weights;
+
+/* Schedule and kernel knobs.  Zero selects the default for every field except
+ * l2_prefetch (-1 = default, 0 = off). */
+typedef struct {
+    int ring_stages;      /* shared-memory weight ring depth (default 6) */
+    int stage_bytes;      /* bytes per ring stage, multiple of 1024 (default 32768) */
+    int rows_per_instr;   /* cap on GEMV rows per instruction (default and max 1024) */
+    int kv_splits;        /* split-KV chunks per kv head (default: SMs / n_kv_heads, capped by max_seq/32) */
+    int l2_prefetch;      /* bytes kept prefetched into L2 ahead of the TMA stream (-1 default) */
+    int trace;            /* 1: record per-instruction globaltimer stamps (mk_get_trace) */
+    int snapshots;        /* 1: record the residual stream after every layer (mk_get_hidden) */
+    unsigned long long spin_limit_ns; /* bound on every device-side wait (default 2 s) */
+    int mode;             /* MK_MODE_* */
+    int n_sm;             /* blocks of the persistent grid (default: all SMs) */
+} mk_options;
+
+/* Device status block, copied out by mk_get_status.  On a device-side error
+ * the first failing wait records where it gave up. */
+typedef struct {
+    int code;             /* MK_OK or MK_ERR_TIMEOUT / MK_ERR_BAD_INSTR / MK_ERR_STOPPED / MK_ERR_CUDA */
+    int sm;               /* block index that recorded the error */
+    int instr;            /* index of the instruction in that block's queue */
+    int opcode;
+    int counter;          /* counter id waited on (-1: the shared-memory ring) */
+    unsigned int observed, expected;
+    int cuda_error;       /* cudaError_t for MK_ERR_CUDA */
+} mk_status;
+
+typedef struct mk_handle mk_handle;
+
+/* Fill *out with the defaults described in mk_options. */
+void mk_default_options(mk_options *out);
+
+/* Create a handle: validates the config and pointers, allocates the library's
+ * device buffers (instruction tensor, counters, fp32 activations, status) on
+ * the current device and binds `cuda_stream` (a cudaStream_t, NULL = legacy
+ * default stream).  Errors: MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_CUDA. */
+int mk_create(const mk_config *cfg, const mk_weights *w, const mk_options *opt, void *cuda_stream,
+              mk_handle **out);
+
+/* Build, validate and upload the instruction schedule (host work, done once).
+ * Deterministic: the instruction words depend only on (config, options, SMs).
+ * Errors: MK_ERR_SCHEDULE (validator), MK_ERR_CUDA. */
+int mk_build_schedule(mk_handle *h);
+
+/* Copy the instruction tensor ([n_sm][max_instr][MK_INSTR_WORDS] int32, unused
+ * slots zero) to host `buf` of `cap` words.  *n_words receives the size. */
+#define MK_INSTR_WORDS 16
+int mk_get_schedule(mk_handle *h, int32_t *buf, size_t cap, size_t *n_words, int *n_sm, int *max_instr);
+
+/* One decode step: embeds `token` (or, if token < 0, the previous step's
+ * on-device argmax), runs every layer at position `pos` (appending K/V at pos
+ * and attending over 0..pos), writes fp32 logits to `logits_dev` (device,
+ * [vocab], may be NULL) and, if `next_token_host` is not NULL, waits for the
+ * step and stores the argmax there (lowest index on ties).  With
+ * next_token_host == NULL the call only enqueues on the handle's stream, and
+ * device-side errors surface at the next synchronous call or mk_get_status.
+ * Positions must be stepped in order: pos reads cache entries 0..pos-1.
+ * Errors: MK_ERR_INVALID_ARG, MK_ERR_NO_SCHEDULE, MK_ERR_TIMEOUT,
+ * MK_ERR_BAD_INSTR, MK_ERR_STOPPED, MK_ERR_CUDA. */
+int mk_decode_step(mk_handle *h, int32_t token, int32_t pos, float *logits_dev, int32_t *next_token_host);
+
+/* Residual stream after layer `layer` of the last step (0 = embedding,
+ * n_layers = after the last layer) as fp32 [hidden] into host `out_host`.
+ * Needs options.snapshots = 1.  Synchronises the stream. */
+int mk_get_hidden(mk_handle *h, int layer, float *out_host);
+
+/* MoE routing of `layer` in the last step: top_k expert ids and weights
+ * (host arrays of top_k entries).  MK_ERR_INVALID_ARG for dense models. */
+int mk_get_router(mk_handle *h, int layer, int32_t *idx, float *w);
+
+/* Dependency counters (uint32, monotone across steps) into host `out`. */
+int mk_get_counters(mk_handle *h, uint32_t *out, size_t cap, size_t *n);
+
+/* Per-counter increment per step, as planned by the scheduler (host `out`). */
+int mk_get_counter_increments(mk_handle *h, uint32_t *out, size_t cap, size_t *n);
+
+/* Copy the device status block (synchronises the stream). */
+int mk_get_status(mk_handle *h, mk_status *out);
+
+/* Trace stamps of the last step: [n_sm][max_instr][4] uint64 globaltimer ns
+ * (instruction start, dependency satisfied, first weight stage ready, end;
+ * zero where not reached).  Needs options.trace = 1. */
+int mk_get_trace(mk_handle *h, uint64_t *out, size_t cap, size_t *n);
+
+/* Clear counters, epoch, status and stop word and re-upload the schedule
+ * (undoes mk_inject_fault).  Use after any failed step. */
+int mk_reset(mk_handle *h);
+
+/* Host-side fault injection for tests: MK_FAULT_* (see above).  The fault
+ * applies from the next step until mk_reset.  `arg` selects the block for
+ * instruction faults. */
+int mk_inject_fault(mk_handle *h, int kind, int arg);
+
+/* Device-side step time of the last megakernel launch in ns (CUDA events on
+ * the handle's stream); synchronises. */
+int mk_last_step_ns(mk_handle *h, double *ns);
+
+const char *mk_strerror(int code);
+void mk_destroy(mk_handle *h);
+
+/* ---- host-only planning (no GPU needed) ---------------------------------------- */
+
+/* Plan the schedule for `n_sm` blocks without a device: writes the instruction
+ * tensor ([n_sm][max_instr][MK_INSTR_WORDS]) to `buf` (cap words), the
+ * per-SM instruction counts to `n_instr` (n_sm entries) and the per-step
+ * increment of every counter to `ctr_inc` (ctr_cap entries).  Runs the
+ * validator.  Errors: MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_CAPACITY,
+ * MK_ERR_SCHEDULE. */
+int mk_plan(const mk_config *cfg, const mk_options *opt, int n_sm, int32_t *buf, size_t cap, int *max_instr,
+            int32_t *n_instr, uint32_t *ctr_inc, size_t ctr_cap, int *n_counters);
+
+/* Execute a planned schedule on the host under a seeded random interleaving of
+ * the blocks (an instruction may run once its counter has reached its target)
+ * for `steps` steps.  Returns MK_OK when every instruction ran and every
+ * counter ends at steps * its increment, MK_ERR_SCHEDULE on a deadlock or a
+ * count mismatch.  *executed receives the number of instructions run. */
+int mk_simulate(const int32_t *buf, int n_sm, int max_instr, const int32_t *n_instr, const uint32_t *ctr_inc,
+                int n_counters, int steps, uint64_t seed, long long *executed);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H */

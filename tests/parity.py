@@ -1,0 +1,114 @@
+"""Shared parity harness: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Both sides get the identical bf16 weights and pre-filled KV cache from the
+seeded generator.  Multi-step runs are teacher-forced: both consume the
+oracle's greedy token each step, so a near-tie never makes the two chains
+incomparable.  Tolerances (per layer snapshot rel-L2 <= 1e-2, logits max-abs <=
+5e-2, greedy token equal where the oracle's top-1/top-2 margin > 0.1) are the
+workload's stated bar.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import synth
+
+HIDDEN_RTOL = 1e-2
+LOGIT_ATOL = 5e-2
+MARGIN = 0.1
+ROUTER_MARGIN = 1e-2
+
+
+def schedule(cfg, steps: int | None = None):
+    """(pos, token or None) pairs; None = the oracle's previous greedy token."""
+    out = []
+    if cfg.prompt_len:
+        toks = synth.prompt_tokens(cfg)
+        out += [(i, int(t)) for i, t in enumerate(toks)]
+        out += [(cfg.prompt_len + i, None) for i in range(cfg.steps)]
+    else:
+        first = int(synth.prompt_tokens(cfg)[0])
+        out += [(cfg.prefill, first)] + [(cfg.prefill + i, None) for i in range(1, cfg.steps)]
+    return out if steps is None else out[:steps]
+
+
+class Setup:
+    """Weights and caches for one config on both sides."""
+
+    def __init__(self, cfg, weights: dict | None = None):
+        import torch
+        from decode_persistent_block_b200 import to_device
+        self.cfg = cfg
+        self.W = weights if weights is not None else synth.make_model(cfg)
+        self.kc, self.vc = synth.make_kv_cache(cfg)
+        self.dW = to_device(self.W)
+        self.dk = torch.from_numpy(self.kc.view(np.int16)).cuda()
+        self.dv = torch.from_numpy(self.vc.view(np.int16)).cuda()
+
+    def fresh_caches(self):
+        """Reset the device caches to the pre-filled state."""
+        import torch
+        self.dk.copy_(torch.from_numpy(self.kc.view(np.int16)))
+        self.dv.copy_(torch.from_numpy(self.vc.view(np.int16)))
+
+    def oracle(self):
+        return oracle.Model(self.cfg, self.W, self.kc.copy(), self.vc.copy())
+
+    def decoder(self, **opts):
+        from decode_persistent_block_b200 import Decoder
+        opts.setdefault("snapshots", 1)
+        return Decoder(self.cfg, self.dW, self.dk, self.dv, **opts)
+
+
+def compare_step(cfg, dec, logits_gpu, o, gpu_next) -> dict:
+    lo = o["logits"]
+    lg = logits_gpu.astype(np.float64)
+    srt = np.sort(lo)
+    margin = float(srt[-1] - srt[-2]) if lo.size > 1 else np.inf
+    r = {"logit_err": float(np.max(np.abs(lg - lo))), "margin": margin, "next_orc": o["next"], "next_gpu": gpu_next}
+    if dec.options.snapshots:
+        hg = dec.hidden_all().astype(np.float64)
+        ho = o["hidden"]
+        r["hidden_rel"] = (np.linalg.norm(hg - ho, axis=1) / np.maximum(np.linalg.norm(ho, axis=1), 1e-30)).tolist()
+    if cfg.n_experts:
+        r["router"] = []
+        for l in range(cfg.n_layers):
+            gi, gw = dec.router(l)
+            r["router"].append((gi.tolist(), o["router_idx"][l].tolist(), gw.tolist(), o["router_w"][l].tolist()))
+    return r
+
+
+def run(setup: Setup, steps: int | None = None, orc=None, **opts) -> list[dict]:
+    """Teacher-forced run of `steps` positions; returns one report per step."""
+    import torch
+    cfg = setup.cfg
+    orc = orc or setup.oracle()
+    setup.fresh_caches()
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    reports = []
+    nxt = None
+    with setup.decoder(**opts) as dec:
+        for pos, tok in schedule(cfg, steps):
+            t = tok if tok is not None else nxt
+            gpu_next = dec.step(t, pos, logits=logits)
+            o = orc.step(t, pos)
+            r = compare_step(cfg, dec, logits.cpu().numpy(), o, gpu_next)
+            r["pos"] = pos
+            reports.append(r)
+            nxt = o["next"]
+    return reports
+
+
+def assert_parity(reports: list[dict], cfg=None):
+    worst_h = max((max(r["hidden_rel"]) for r in reports if "hidden_rel" in r), default=0.0)
+    worst_l = max(r["logit_err"] for r in reports)
+    assert worst_h <= HIDDEN_RTOL, f"hidden rel-L2 {worst_h}"
+    assert worst_l <= LOGIT_ATOL, f"logits max-abs {worst_l}"
+    for r in reports:
+        if r["margin"] > MARGIN:
+            assert r["next_gpu"] == r["next_orc"], r
+        for gi, oi, gw, ow in r.get("router", []):
+            assert gi == oi, (r["pos"], gi, oi)
+            assert np.allclose(gw, ow, atol=1e-4), (gw, ow)
+    return worst_h, worst_l

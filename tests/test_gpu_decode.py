@@ -1,0 +1,161 @@
+"""GPU parity of the decode step (through the C ABI) against the fp64 oracle.
+
+Small configs run every step of their workload on both execution modes; the
+full-size configs (Llama-1B/3B shapes, the KV-length sweep, Mixtral-shaped
+MoE) run a teacher-forced subset of their decode positions in the same launch
+configuration the benchmark times (set MK_FULL_PARITY=1 for every step).
+"""
+import os
+
+import numpy as np
+import pytest
+
+from synth import configs
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+FULL = os.environ.get("MK_FULL_PARITY") == "1"
+MODES = {"megakernel": 0, "multi_kernel": 1, "multi_kernel_graph": 2}
+
+
+@pytest.fixture(scope="module")
+def tiny(cuda):
+    return parity.Setup(configs.TINY)
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+def test_tiny_all_steps(tiny, mode):
+    reps = parity.run(tiny, mode=MODES[mode])
+    assert len(reps) == configs.TINY.prompt_len + configs.TINY.steps
+    h, l = parity.assert_parity(reps)
+    assert h < 1e-4 and l < 1e-3  # fp32 vs fp64 on identical bf16 bytes: far inside the bar
+
+
+@pytest.mark.parametrize("opts", [
+    dict(n_sm=7), dict(n_sm=1), dict(kv_splits=1), dict(kv_splits=40), dict(ring_stages=2),
+    dict(stage_bytes=4096), dict(stage_bytes=4096, ring_stages=3, l2_prefetch=16384), dict(rows_per_instr=3),
+    dict(l2_prefetch=65536),
+], ids=lambda o: ",".join(f"{k}={v}" for k, v in o.items()))
+def test_tiny_schedule_options(tiny, opts):
+    parity.assert_parity(parity.run(tiny, **opts))
+
+
+@pytest.mark.parametrize("E,k", [(4, 2), (2, 1), (8, 2)])
+@pytest.mark.parametrize("mode", ["megakernel", "multi_kernel"])
+def test_tiny_moe(cuda, E, k, mode):
+    cfg = configs.TINY.with_(name=f"tiny_moe{E}_{k}", n_experts=E, top_k=k)
+    parity.assert_parity(parity.run(parity.Setup(cfg), mode=MODES[mode]), cfg)
+
+
+def test_no_layers_is_lm_head_of_embedding(cuda):
+    cfg = configs.TINY.with_(n_layers=0, steps=2)
+    parity.assert_parity(parity.run(parity.Setup(cfg)))
+
+
+def test_head_dim_128_group_3(cuda):
+    cfg = configs.TINY.with_(name="tiny_d128", n_heads=6, n_kv_heads=2, head_dim=128, hidden=384, ffn=1024)
+    parity.assert_parity(parity.run(parity.Setup(cfg)))
+
+
+def test_group_1_and_wide_rows(cuda):
+    # n_heads == n_kv_heads, and an ffn wider than 8192 columns (column-part phases)
+    cfg = configs.TINY.with_(name="tiny_wide", n_heads=2, n_kv_heads=2, ffn=9216, steps=3)
+    for mode in (0, 1):
+        parity.assert_parity(parity.run(parity.Setup(cfg), mode=mode))
+
+
+def test_counters_are_exact_multiples_after_steps(tiny):
+    tiny.fresh_caches()
+    with tiny.decoder() as dec:
+        inc = dec.counter_increments()
+        for s, (pos, tok) in enumerate(parity.schedule(configs.TINY)):
+            dec.step(tok if tok is not None else 1, pos)
+            assert np.array_equal(dec.counters(), (s + 1) * inc.astype(np.uint64)), s
+        dec.reset()
+        assert not dec.counters().any()
+
+
+def test_determinism_bitwise(tiny):
+    import torch
+    outs = []
+    for _ in range(2):
+        tiny.fresh_caches()
+        lg = torch.empty(configs.TINY.vocab, device="cuda")
+        with tiny.decoder() as dec:
+            for pos, tok in parity.schedule(configs.TINY, 20):
+                dec.step(tok if tok is not None else 7, pos, logits=lg)
+            outs.append((lg.cpu().numpy().copy(), tiny.dk.cpu().numpy().copy()))
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+
+
+def test_on_device_token_feed_matches_host_feed(tiny):
+    import torch
+    res = []
+    for feed in ("host", "device"):
+        tiny.fresh_caches()
+        lg = torch.empty(configs.TINY.vocab, device="cuda")
+        with tiny.decoder() as dec:
+            nxt = dec.step(5, 0)
+            for pos in range(1, 6):
+                if feed == "host":
+                    nxt = dec.step(nxt, pos, logits=lg)
+                else:
+                    dec.step(-1, pos, logits=lg, sync=False)
+            res.append(lg.cpu().numpy().copy())
+    assert np.array_equal(res[0], res[1])
+
+
+def test_kv_append_matches_oracle_cache(tiny):
+    orc = tiny.oracle()
+    reps = parity.run(tiny, orc=orc)
+    parity.assert_parity(reps)
+    g = tiny.dk.cpu().numpy().view(np.uint16)
+    o = orc.k
+    n = configs.TINY.prompt_len + configs.TINY.steps
+    a = (g[:, :, :n].astype(np.uint32) << 16).view(np.float32)
+    b = (o[:, :, :n].astype(np.uint32) << 16).view(np.float32)
+    # identical bf16 bits except where fp32 vs fp64 rounding straddles a bf16 tie (at most one ulp)
+    assert np.all(np.abs(a - b) <= np.abs(b) * 2.0 ** -7 + 1e-30)
+    assert np.mean(a == b) > 0.99
+
+
+def test_argument_errors(tiny):
+    from decode_persistent_block_b200 import MkError
+    with tiny.decoder() as dec:
+        for tok, pos in ((configs.TINY.vocab, 0), (0, configs.TINY.max_seq), (0, -1)):
+            with pytest.raises(MkError) as e:
+                dec.step(tok, pos)
+            assert e.value.name == "MK_ERR_INVALID_ARG"
+        with pytest.raises(MkError):
+            dec.router(0)  # dense model
+
+
+# ---- full-size configs -----------------------------------------------------------------
+
+def _full(cfg, steps, mode=0, **opts):
+    s = parity.Setup(cfg)
+    reps = parity.run(s, steps=None if FULL else steps, mode=mode, **opts)
+    h, l = parity.assert_parity(reps, cfg)
+    return reps
+
+
+def test_llama1b(cuda):
+    _full(configs.LLAMA_1B, 4)
+
+
+def test_llama1b_multi_kernel(cuda):
+    _full(configs.LLAMA_1B, 2, mode=1)
+
+
+def test_llama3b(cuda):
+    _full(configs.LLAMA_3B, 3)
+
+
+@pytest.mark.parametrize("prefill", configs.SWEEP_PREFILLS)
+def test_llama1b_kv_sweep(cuda, prefill):
+    _full(configs.llama1b_sweep(prefill), 2)
+
+
+def test_mixtral8l(cuda):
+    _full(configs.MIXTRAL_8L, 3)

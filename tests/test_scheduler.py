@@ -1,0 +1,175 @@
+"""Host scheduler: bit-exact integer checks, no GPU needed.
+
+The schedule must cover every output row of every op exactly once, order each
+block's queue by op so that no wait can deadlock, and give every dependency
+counter a per-step increment equal to the number of instructions that signal
+it (after S steps on the device every counter must read exactly S times that).
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+import decode_persistent_block_b200 as dpb
+from decode_persistent_block_b200 import mk
+from synth import configs
+
+OP = dict(RMS_QKV=1, ATTN=2, OPROJ=3, UG=4, DOWN=5, LM=6, MOE_UG=7, MOE_DOWN=8)
+W_OP, W_LAYER, W_SUB, W_BEGIN, W_END, W_WAIT, W_WINC, W_SIG, W_AUX, W_AINC, W_SEQ = range(11)
+
+CFGS = [configs.TINY, configs.LLAMA_1B, configs.LLAMA_3B, configs.MIXTRAL_8L, configs.llama1b_sweep(16384),
+        configs.TINY.with_(name="tiny_moe", n_experts=4, top_k=2),
+        configs.TINY.with_(name="tiny_moe1", n_experts=2, top_k=1),
+        configs.TINY.with_(name="tiny_l0", n_layers=0)]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    dpb.build()
+
+
+def instrs(words, n_instr):
+    for sm in range(words.shape[0]):
+        for i in range(n_instr[sm]):
+            yield sm, i, words[sm, i]
+
+
+def n_ctr_per_layer(cfg):
+    return 5 + cfg.n_kv_heads
+
+
+@pytest.mark.parametrize("cfg", CFGS, ids=lambda c: c.name)
+@pytest.mark.parametrize("n_sm", [148, 37, 1])
+def test_plan_covers_rows_and_counts_signals(cfg, n_sm):
+    words, n_instr, inc = dpb.plan(cfg, n_sm)
+    L, nkv, d = cfg.n_layers, cfg.n_kv_heads, cfg.head_dim
+    per = n_ctr_per_layer(cfg)
+    assert inc.size == L * per + 1
+    rows = {OP["RMS_QKV"]: {0: cfg.n_heads * d, 1: nkv * d, 2: nkv * d}, OP["OPROJ"]: {0: cfg.hidden},
+            OP["UG"]: {0: cfg.ffn}, OP["DOWN"]: {0: cfg.hidden}, OP["LM"]: {0: cfg.vocab},
+            OP["MOE_UG"]: {s: cfg.ffn for s in range(max(cfg.top_k, 1))}, OP["MOE_DOWN"]: {0: cfg.hidden}}
+    cover = {}
+    signals = np.zeros_like(inc)
+    splits = None
+    attn_seen = set()
+    for sm, i, w in instrs(words, n_instr):
+        op, l = int(w[W_OP]), int(w[W_LAYER])
+        if op == OP["ATTN"]:
+            splits = int(w[W_END])
+            key = (l, int(w[W_SUB]), int(w[W_BEGIN]))
+            assert key not in attn_seen
+            attn_seen.add(key)
+            assert w[W_AUX] == l * per + 5 + w[W_SUB]
+            signals[w[W_AUX]] += 1
+            continue
+        key = (l, op, int(w[W_SUB]))
+        hit = cover.setdefault(key, np.zeros(rows[op][int(w[W_SUB])], dtype=np.int32))
+        hit[w[W_BEGIN]:w[W_END]] += 1
+        assert 0 < w[W_END] - w[W_BEGIN] <= 1024
+        signals[w[W_AUX] if op == OP["LM"] else w[W_SIG]] += 1
+    for key, hit in cover.items():
+        assert np.all(hit == 1), key
+    moe = cfg.n_experts > 0
+    ffn_ops = (OP["MOE_UG"], OP["MOE_DOWN"]) if moe else (OP["UG"], OP["DOWN"])
+    for l in range(L):
+        for op in (OP["RMS_QKV"], OP["OPROJ"]) + ffn_ops:
+            assert (l, op, 0) in cover
+        signals[l * per + 1] = nkv  # ATTN_DONE: one per kv head from its last split
+    assert (L, OP["LM"], 0) in cover
+    assert np.array_equal(signals, inc)
+    if L:
+        assert len(attn_seen) == L * nkv * splits
+        # closed forms: one signal per kv head, `splits` per head group
+        for l in range(L):
+            assert inc[l * per + 1] == nkv
+            assert np.all(inc[l * per + 5: l * per + 5 + nkv] == splits)
+
+
+def _ranges(total, n_sm):
+    return [(total * s // n_sm, total * (s + 1) // n_sm) for s in range(n_sm)]
+
+
+@pytest.mark.parametrize("n_sm", [148, 132, 64])
+def test_increment_closed_forms_llama1b(n_sm):
+    cfg = configs.LLAMA_1B
+    words, n_instr, inc = dpb.plan(cfg, n_sm)
+    per = n_ctr_per_layer(cfg)
+    # QKV: one instruction per block range, plus one for every q/k/v boundary strictly inside a range
+    qkv_rows = cfg.qkv_rows
+    bounds = [cfg.n_heads * cfg.head_dim, (cfg.n_heads + cfg.n_kv_heads) * cfg.head_dim]
+    n_qkv = sum(1 for a, b in _ranges(qkv_rows, n_sm) if b > a) + \
+        sum(1 for a, b in _ranges(qkv_rows, n_sm) for x in bounds if a < x < b)
+    lm = sum(-(-(b - a) // 1024) for a, b in _ranges(cfg.vocab, n_sm))
+    for l in range(cfg.n_layers):
+        assert inc[l * per + 0] == n_qkv
+        assert inc[l * per + 2] == n_sm      # O-proj: hidden >= n_sm rows, <= 1024 per block
+        assert inc[l * per + 3] == n_sm      # up/gate
+        assert inc[l * per + 4] == n_sm      # down
+    assert inc[-1] == lm
+    # every block's queue is sorted by (layer, op slot)
+    order = {OP["RMS_QKV"]: 0, OP["ATTN"]: 1, OP["OPROJ"]: 2, OP["UG"]: 3, OP["DOWN"]: 4, OP["LM"]: 0}
+    for sm in range(n_sm):
+        keys = [int(w[W_LAYER]) * 5 + order[int(w[W_OP])] for w in words[sm, :n_instr[sm]]]
+        assert keys == sorted(keys)
+
+
+def test_plan_is_deterministic():
+    a = dpb.plan(configs.LLAMA_3B, 148)
+    b = dpb.plan(configs.LLAMA_3B, 148)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+@pytest.mark.parametrize("cfg", CFGS, ids=lambda c: c.name)
+def test_simulated_interleavings_complete_and_counters_match(cfg):
+    words, n_instr, inc = dpb.plan(cfg, 148 if cfg.hidden > 256 else 23)
+    for seed in range(3):
+        rc, done = dpb.simulate(words, n_instr, inc, steps=3, seed=seed)
+        assert rc == mk.MK_OK
+        assert done == 3 * int(n_instr.sum())
+
+
+def test_simulator_detects_deadlock_and_count_mismatch():
+    cfg = configs.TINY
+    words, n_instr, inc = dpb.plan(cfg, 4)
+    # move block 0's first layer-1 QKV in front of its layer-0 down-projection
+    q = words[0, :n_instr[0]].copy()
+    i_down = next(i for i, w in enumerate(q) if w[W_OP] == OP["DOWN"] and w[W_LAYER] == 0)
+    i_qkv = next(i for i, w in enumerate(q) if w[W_OP] == OP["RMS_QKV"] and w[W_LAYER] == 1)
+    bad = words.copy()
+    bad[0, [i_down, i_qkv]] = q[[i_qkv, i_down]]
+    rc, done = dpb.simulate(bad, n_instr, inc, steps=1, seed=0)
+    assert rc == mk.CODES["MK_ERR_SCHEDULE"] and done < n_instr.sum()
+    wrong = inc.copy()
+    wrong[0] += 1
+    rc, _ = dpb.simulate(words, n_instr, wrong, steps=1, seed=0)
+    assert rc != mk.MK_OK
+
+
+def test_plan_rejects_unsupported_shapes():
+    with pytest.raises(mk.MkError) as e:
+        dpb.plan(configs.TINY.with_(head_dim=96), 148)
+    assert e.value.name == "MK_ERR_UNSUPPORTED"
+    with pytest.raises(mk.MkError) as e:
+        dpb.plan(configs.TINY.with_(n_heads=10, n_kv_heads=2), 148)  # 5 query heads per kv head
+    assert e.value.name == "MK_ERR_UNSUPPORTED"
+    with pytest.raises(mk.MkError) as e:
+        dpb.plan(configs.TINY, 0)
+    assert e.value.name == "MK_ERR_INVALID_ARG"
+    with pytest.raises(mk.MkError):
+        dpb.plan(configs.TINY, 148, stage_bytes=1000)
+
+
+@pytest.mark.parametrize("splits", [1, 3, 40])
+def test_kv_splits_option(splits):
+    words, n_instr, inc = dpb.plan(configs.TINY, 16, kv_splits=splits)
+    attn = [w for _, _, w in instrs(words, n_instr) if w[W_OP] == OP["ATTN"]]
+    assert len(attn) == configs.TINY.n_layers * configs.TINY.n_kv_heads * splits
+    assert all(w[W_END] == splits for w in attn)
+
+
+def test_rows_per_instr_cap_splits_instructions():
+    words, n_instr, inc = dpb.plan(configs.TINY, 2, rows_per_instr=64)
+    for _, _, w in instrs(words, n_instr):
+        if w[W_OP] != OP["ATTN"]:
+            assert w[W_END] - w[W_BEGIN] <= 64
