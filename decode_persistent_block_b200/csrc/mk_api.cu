@@ -67,7 +67,8 @@ int dalloc(mk_handle* h, T** out, size_t count) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_weights(const mk_config& c, const mk_weights* w) {
-    if (!w || !w->embed || !w->lm_head || !w->final_norm || !w->k_cache || !w->v_cache) return MK_ERR_INVALID_ARG;
+    if (!w || !w->embed || !w->lm_head || !w->final_norm) return MK_ERR_INVALID_ARG;
+    if (c.n_layers > 0 && (!w->k_cache || !w->v_cache)) return MK_ERR_INVALID_ARG;  // no cache without layers
     if (!aligned16(w->embed) || !aligned16(w->lm_head) || !aligned16(w->final_norm) || !aligned16(w->k_cache) ||
         !aligned16(w->v_cache))
         return MK_ERR_INVALID_ARG;
@@ -133,6 +134,7 @@ void mk_default_options(mk_options* o) {
     if (!o) return;
     std::memset(o, 0, sizeof(*o));
     o->l2_prefetch = -1;
+    o->prefetch_ahead = -1;
     o->mode = MK_MODE_MEGAKERNEL;
 }
 
@@ -199,6 +201,8 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     p.ring_stages = o.ring_stages;
     p.stage_bytes = o.stage_bytes;
     p.l2_prefetch = o.l2_prefetch;
+    p.prefetch_ahead = o.prefetch_ahead;
+    p.prefetch_max_bytes = o.prefetch_max_bytes;
     p.spin_limit_ns = o.spin_limit_ns;
 
     // weight pointer table
@@ -222,7 +226,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
         }
     }
     const uint16_t** wt_dev = nullptr;
-    const int lm_slots = std::max(h->n_sm + c.vocab / mk::kMaxRows + 1, mk::baseline_lm_blocks(p, h->n_sm));
+    const int lm_slots = std::max(h->n_sm + c.vocab / o.rows_per_instr + 1, mk::baseline_lm_blocks(p, h->n_sm));
     h->lm_slots = lm_slots;
     if ((rc = dalloc(h, &wt_dev, h->wt_host.size()))) return fail(rc);
     if ((rc = dalloc(h, &p.counters, (size_t)p.n_ctr))) return fail(rc);

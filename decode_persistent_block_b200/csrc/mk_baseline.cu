@@ -355,6 +355,8 @@ __global__ void __launch_bounds__(kBT) bl_lm_head(const __grid_constant__ DevPar
     __shared__ float red[kBW];
     __shared__ int redi[kBW];
     const uint16_t* x16 = p.L == 0 ? p.embed + (size_t)step_token(sb) * p.H : nullptr;
+    if (x16 && p.snap && blockIdx.x == 0)  // no layers: the residual stream is the embedding row
+        for (int i = threadIdx.x; i < p.H; i += kBT) p.snap[i] = __uint_as_float((uint32_t)x16[i] << 16);
     block_rmsnorm(p.x, x16, p.final_norm, p.H, p.eps, vec, red);
     __syncthreads();
     const int r0 = blockIdx.x * rpb, r1 = min(p.V, r0 + rpb);

@@ -49,7 +49,9 @@ enum Word : int {
     W_NWORDS = MK_INSTR_WORDS
 };
 
-constexpr int kMaxRows = 1024;       // rows per GEMV instruction (smem accumulators)
+constexpr int kMaxRows = 1024;       // rows per GEMV instruction
+constexpr int kRowSlots = 1024;      // rows x accumulator sets held in shared memory per instruction
+constexpr int kMaxPartK = 8192;      // widest row part reduced in one phase (4 chunks of 8 per thread)
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;  // + one loader warp
@@ -70,6 +72,21 @@ MK_HD inline int wt_stride(int n_experts) { return kLayerFixed + 3 * (n_experts 
 MK_HD inline int wt_gate(int e) { return kLayerFixed + e; }
 MK_HD inline int wt_up(int e, int n_experts) { return kLayerFixed + (n_experts > 0 ? n_experts : 1) + e; }
 MK_HD inline int wt_down(int e, int n_experts) { return kLayerFixed + 2 * (n_experts > 0 ? n_experts : 1) + e; }
+
+// Column parts of a row of width K, and the accumulator sets an op keeps per
+// row (spans x expert slots x column parts); rows per instruction are capped at
+// kRowSlots / sets so that every (set, row) has a slot per consumer warp.
+MK_HD inline int kparts_of(int K) { return (K + kMaxPartK - 1) / kMaxPartK; }
+MK_HD inline int acc_sets(int op, int H, int qd, int F, int topk) {
+    switch (op) {
+        case OP_OPROJ_RES: return kparts_of(qd);
+        case OP_RMS_UPGATE_SILU:
+        case OP_MOE_UPGATE: return 2 * kparts_of(H);
+        case OP_DOWN_RES: return kparts_of(F);
+        case OP_MOE_DOWN2_RES: return (topk > 0 ? topk : 1) * kparts_of(F);
+        default: return kparts_of(H);
+    }
+}
 
 struct DevStatus {
     int code, sm, instr, opcode, counter;
@@ -118,6 +135,8 @@ struct DevParams {
     int ring_stages;
     int stage_bytes;
     int l2_prefetch;
+    int prefetch_ahead;
+    int prefetch_max_bytes;
     unsigned long long spin_limit_ns;
 };
 

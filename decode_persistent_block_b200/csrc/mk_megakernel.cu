@@ -43,7 +43,7 @@ namespace mk {
 // ---------------------------------------------------------------------------
 // shared memory layout
 // ---------------------------------------------------------------------------
-constexpr int kScratchBytes = 17408;  // max(acc 2*kMaxRows*4, attention merge 8*512*4 + 8*8*2*4, router 8*64*4)
+constexpr int kScratchBytes = 4 * kRowSlots * kConsumerWarps;  // partial row sums; attention merge and router reuse it
 
 struct Misc {
     float red[kConsumerWarps * 2];
@@ -71,35 +71,48 @@ __device__ __forceinline__ void vstore(int* p, int v) { *(volatile int*)p = v; }
 // ---------------------------------------------------------------------------
 // bounded waits
 // ---------------------------------------------------------------------------
+// The stop word and the block's abort flag are only polled once a wait has
+// lasted kStopPollNs: a global load inside every spin iteration would put an
+// L2 round trip between a barrier completing and the waiter noticing it.
+constexpr uint64_t kStopPollNs = 20000;
+
 __device__ bool wait_counter(const DevParams& p, Misc& m, int ctr, uint32_t target, int ii, int op) {
     const uint32_t* addr = p.counters + ctr;
     uint32_t v = ld_acquire_u32(addr);
     if ((int32_t)(v - target) >= 0) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
+    uint64_t next = t0 + kStopPollNs;
+    for (;;) {
         v = ld_acquire_u32(addr);
         if ((int32_t)(v - target) >= 0) return true;
-        if ((it & 31u) == 0) {
+        const uint64_t now = globaltimer_ns();
+        if (now >= next) {
             if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
-            if (globaltimer_ns() - t0 > p.spin_limit_ns) {
+            if (now - t0 > p.spin_limit_ns) {
                 record_error(p.status, MK_ERR_TIMEOUT, blockIdx.x, ii, op, ctr, v, target);
                 return false;
             }
+            next = now + kStopPollNs;
         }
     }
 }
 
+constexpr uint32_t kSuspendHintNs = 20000;
+
 __device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const DevParams& p, Misc& m, int ii, int op) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 15u) == 0) {
+    uint64_t next = t0 + kStopPollNs;
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
+        const uint64_t now = globaltimer_ns();
+        if (now >= next) {
             if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
-            if (globaltimer_ns() - t0 > p.spin_limit_ns) {
+            if (now - t0 > p.spin_limit_ns) {
                 record_error(p.status, MK_ERR_TIMEOUT, blockIdx.x, ii, op, -1, parity, 0);
                 return false;
             }
+            next = now + kStopPollNs;
         }
     }
 }
@@ -152,6 +165,7 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
     if (op == OP_RMS_QKV && (sub < 0 || sub > 2)) return false;
     if (op == OP_MOE_UPGATE && (sub < 0 || sub >= p.topk)) return false;
     if (b < 0 || b >= e || e > op_rows(p, op, sub) || e - b > kMaxRows) return false;
+    if ((e - b) * acc_sets(op, p.H, p.nq * p.d, p.F, p.topk) > kRowSlots) return false;
     if (op == OP_LMHEAD_ARGMAX) return w[W_AUX_CTR] >= 0 && w[W_AUX_INC] > 0 && w[W_SEQ] >= 0 && w[W_SEQ] < w[W_AUX_INC];
     return w[W_SIGNAL_CTR] >= 0;
 }
@@ -159,9 +173,7 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
 // Column parts: rows wider than kMaxPartK columns are streamed and reduced in
 // column parts (one phase per part) so that each thread's slice of the input
 // vector stays within 4 chunks of 8 in registers.
-constexpr int kMaxPartK = 8 * kConsumerThreads * 4;  // 8192
-
-__host__ __device__ __forceinline__ int kparts_of(int K) { return (K + kMaxPartK - 1) / kMaxPartK; }
+static_assert(kMaxPartK == 8 * kConsumerThreads * 4, "a column part is 4 chunks of 8 per consumer thread");
 
 struct Plan {
     int n_stages;   // stages of the whole instruction
@@ -302,13 +314,16 @@ __device__ bool loader_plan(const DevParams& p, const StepArgs& a, const int32_t
         if (vload(&m.router_layer) != l) {
             if (!block) return false;
             const uint64_t t0 = globaltimer_ns();
-            for (uint32_t it = 1; vload(&m.router_layer) != l; ++it) {
-                if ((it & 63u) == 0) {
+            uint64_t next = t0 + kStopPollNs;
+            while (vload(&m.router_layer) != l) {
+                const uint64_t now = globaltimer_ns();
+                if (now >= next) {
                     if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
-                    if (globaltimer_ns() - t0 > p.spin_limit_ns) {
+                    if (now - t0 > p.spin_limit_ns) {
                         record_error(p.status, MK_ERR_TIMEOUT, blockIdx.x, ii, w[W_OP], -1, 0, 0);
                         return false;
                     }
+                    next = now + kStopPollNs;
                 }
             }
         }
@@ -420,31 +435,35 @@ __device__ __forceinline__ void load_vec(const float* __restrict__ src, int K, f
 }
 
 // v = rmsnorm(x) * w for x fp32 (or the bf16 embedding row), all threads.
+// The norm weights are loaded together with x so both round trips overlap.
 template <int J>
 __device__ void load_rms(const DevParams& p, Misc& m, const float* x32, const uint16_t* x16, const uint16_t* nw,
                          float (&v)[J][8]) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.H, nch = K >> 3;
-    float ss = 0.f;
+    uint4 wraw[J];
 #pragma unroll
     for (int j = 0; j < J; ++j) {
         const int c = tid + kConsumerThreads * j;
+        wraw[j] = c < nch ? __ldg(reinterpret_cast<const uint4*>(nw) + c) : make_uint4(0u, 0u, 0u, 0u);
         if (c < nch) {
             if (x16) {
-                const uint4 r = __ldg(reinterpret_cast<const uint4*>(x16) + c);
-                unpack8(r, v[j]);
+                unpack8(__ldg(reinterpret_cast<const uint4*>(x16) + c), v[j]);
             } else {
                 const float4 a0 = __ldcg(reinterpret_cast<const float4*>(x32) + 2 * c);
                 const float4 a1 = __ldcg(reinterpret_cast<const float4*>(x32) + 2 * c + 1);
                 v[j][0] = a0.x; v[j][1] = a0.y; v[j][2] = a0.z; v[j][3] = a0.w;
                 v[j][4] = a1.x; v[j][5] = a1.y; v[j][6] = a1.z; v[j][7] = a1.w;
             }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) ss = fmaf(v[j][k], v[j][k], ss);
         } else {
 #pragma unroll
             for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
         }
     }
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ss = fmaf(v[j][k], v[j][k], ss);
     ss = warp_sum(ss);
     if (lane == 0) m.red[warp] = ss;
     cbar();
@@ -454,15 +473,24 @@ __device__ void load_rms(const DevParams& p, Misc& m, const float* x32, const ui
     const float rs = 1.0f / sqrtf(tot / (float)K + p.eps);
 #pragma unroll
     for (int j = 0; j < J; ++j) {
-        const int c = tid + kConsumerThreads * j;
-        if (c < nch) {
-            float wf[8];
-            unpack8(__ldg(reinterpret_cast<const uint4*>(nw) + c), wf);
+        float wf[8];
+        unpack8(wraw[j], wf);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) v[j][k] = v[j][k] * rs * wf[k];
-        }
+        for (int k = 0; k < 8; ++k) v[j][k] = v[j][k] * rs * wf[k];
     }
     cbar();  // m.red free again
+}
+
+// Two interleaved fp32 chains over the 8 bf16 of w (even / odd elements).
+__device__ __forceinline__ void dot8x2(const uint4 w, const float* v, float& a0, float& a1) {
+    a0 = fmaf(bf_lo(w.x), v[0], a0);
+    a1 = fmaf(bf_hi(w.x), v[1], a1);
+    a0 = fmaf(bf_lo(w.y), v[2], a0);
+    a1 = fmaf(bf_hi(w.y), v[3], a1);
+    a0 = fmaf(bf_lo(w.z), v[4], a0);
+    a1 = fmaf(bf_hi(w.z), v[5], a1);
+    a0 = fmaf(bf_lo(w.w), v[6], a0);
+    a1 = fmaf(bf_hi(w.w), v[7], a1);
 }
 
 // Router of a MoE layer from xn (this thread's slice in v): logits of all
@@ -471,22 +499,15 @@ template <int J>
 __device__ void route(const DevParams& p, Misc& m, float* scratch, const uint16_t* wr, int layer, bool publish,
                       float (&v)[J][8]) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.H, nch = K >> 3, E = p.E;
-    for (int e0 = 0; e0 < E; e0 += 8) {
-        float a[8];
+    for (int e = 0; e < E; ++e) {  // one expert row at a time: few live registers
+        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            a[r] = 0.f;
-            if (e0 + r < E) {
-#pragma unroll
-                for (int j = 0; j < J; ++j) {
-                    const int c = tid + kConsumerThreads * j;
-                    if (c < nch) a[r] = dot8(__ldg(reinterpret_cast<const uint4*>(wr + (size_t)(e0 + r) * K) + c), v[j], a[r]);
-                }
-            }
+        for (int j = 0; j < J; ++j) {
+            const int c = tid + kConsumerThreads * j;
+            if (c < nch) dot8x2(__ldg(reinterpret_cast<const uint4*>(wr + (size_t)e * K) + c), v[j], a0, a1);
         }
-        const float s = reduce_rows<8>(a, lane);
-        const int r = reduce_rows_lane_row<8>(lane);
-        if (reduce_rows_writer<8>(lane) && e0 + r < E) scratch[warp * 64 + e0 + r] = s;
+        const float s_e = warp_sum(a0 + a1);
+        if (lane == 0) scratch[warp * 64 + e] = s_e;
     }
     cbar();
     if (tid == 0) {
@@ -526,16 +547,69 @@ __device__ void route(const DevParams& p, Misc& m, float* scratch, const uint16_
     cbar();
 }
 
+
+// RG full rows [rg, rg + RG) of a stage span: every chunk this thread owns is
+// loaded before any FMA, then each row sum is reduced across the warp and
+// stored in this warp's slot A[row * 8 + warp] (shared memory; the epilogue
+// adds the 8 warps' slots in a fixed order, so results are bitwise
+// reproducible).  jv[j]: chunk j of this thread exists.
+template <int J, int RG>
+__device__ __forceinline__ void rows_block(const uint4* __restrict__ Ws, int row16, int rg, const bool (&jv)[J],
+                                           const float (&v)[J][8], float* A, int lane) {
+    const int tid = threadIdx.x;
+    uint4 wv[RG][J];
+#pragma unroll
+    for (int r = 0; r < RG; ++r)
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+            wv[r][j] = jv[j] ? Ws[(rg + r) * row16 + tid + kConsumerThreads * j] : make_uint4(0u, 0u, 0u, 0u);
+    float part[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < J; ++j) dot8x2(wv[r][j], v[j], a0, a1);
+        part[r] = a0 + a1;
+    }
+    const float s_row = reduce_rows<RG>(part, lane);
+    if (reduce_rows_writer<RG>(lane)) A[(rg + reduce_rows_lane_row<RG>(lane)) * kConsumerWarps + (tid >> 5)] = s_row;
+}
+
+// This thread's column slice of rows [0, nr) of one span of a ring stage (Ws:
+// the span in shared memory, row16 16-byte chunks per row) dotted with its
+// slice v of the input vector, into the warp slots of rows [0, nr) of A.  Rows go in blocks of
+// RG, then RG/2, ... 1, so no row needs a guard; a chunk that lies outside
+// the row (widths that are not a multiple of 2048) is a per-thread predicate,
+// uniform across each warp for widths that are multiples of 256.
+template <int J, int RG>
+__device__ __forceinline__ void stage_rows(const uint4* __restrict__ Ws, int row16, int nr, int nch,
+                                           const float (&v)[J][8], float* A, int lane) {
+    bool jv[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) jv[j] = (int)threadIdx.x + kConsumerThreads * j < nch;
+    int rg = 0;
+    for (; rg + RG <= nr; rg += RG) rows_block<J, RG>(Ws, row16, rg, jv, v, A, lane);
+    if constexpr (RG >= 8) {
+        if (rg + 4 <= nr) { rows_block<J, 4>(Ws, row16, rg, jv, v, A, lane); rg += 4; }
+    }
+    if constexpr (RG >= 4) {
+        if (rg + 2 <= nr) { rows_block<J, 2>(Ws, row16, rg, jv, v, A, lane); rg += 2; }
+    }
+    if constexpr (RG >= 2) {
+        if (rg < nr) rows_block<J, 1>(Ws, row16, rg, jv, v, A, lane);
+    }
+}
+
 template <int J>
 __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                            uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase,
                            int token) {
-    // rows reduced together: keeps the live 128-bit weight loads at RG * J <= 8
-    constexpr int RG = J == 1 ? 8 : J == 2 ? 4 : J <= 4 ? 2 : 1;
+    // rows reduced together: keeps the live 128-bit weight loads at RG * J <= 8 (4 for J = 4)
+    constexpr int RG = J == 1 ? 8 : J == 2 ? 4 : J == 3 ? 2 : 1;
     const int tid = threadIdx.x, lane = tid & 31;
     const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], rows = w[W_END] - b;
     const uint32_t SB = (uint32_t)p.stage_bytes;
-    float* acc = scratch;  // [2][kMaxRows]
+    float* part_sums = scratch;  // [set * rows + row][8 warps]
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * 4 : nullptr;
 
     // 1. dependency, zero accumulators
@@ -544,10 +618,6 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
             !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op))
             vstore(&m.abort_flag, 1);
         if (tr) tr[1] = globaltimer_ns();
-    }
-    for (int r = tid; r < rows; r += kConsumerThreads) {
-        acc[r] = 0.f;
-        acc[kMaxRows + r] = 0.f;
     }
     cbar();
     if (vload(&m.abort_flag)) return false;
@@ -567,6 +637,9 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
             break;
         case OP_LMHEAD_ARGMAX:
             load_rms<J>(p, m, p.x, p.L == 0 ? p.embed + (size_t)token * p.H : nullptr, p.final_norm, v);
+            if (p.L == 0 && p.snap && w[W_SEQ] == 0)  // no layers: the residual stream is the embedding row
+                for (int i = tid; i < p.H; i += kConsumerThreads)
+                    p.snap[i] = __uint_as_float((uint32_t)p.embed[(size_t)token * p.H + i] << 16);
             break;
         case OP_OPROJ_RES:
             K = p.nq * p.d;
@@ -582,7 +655,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     if (vsrc) load_vec<J>(vsrc, kp, v);
     // 3. routing (once per layer per block; the loader waits for it)
     if (op == OP_MOE_UPGATE && vload(&m.router_layer) != l)
-        route<J>(p, m, scratch + 2 * kMaxRows, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
+        route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
 
     int eidx[kMaxTopK];
     for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
@@ -600,28 +673,12 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
             const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, op);
             if (tr && tid == 0 && ph == 0 && sst == 0) tr[2] = globaltimer_ns();
             if (ok) {
-                const uint32_t stage = smem_u32(ring) + slot * SB;
+                const unsigned char* stage = ring + (size_t)slot * SB;
                 for (int s = 0; s < pl.nspan; ++s) {
-                    const uint32_t W0 = stage + (uint32_t)(s * pl.rps) * pl.row_bytes;
-                    float* A = acc + (vslot + s) * kMaxRows + r0;
-                    for (int rg = 0; rg < nr; rg += RG) {
-                        float part[RG];
-#pragma unroll
-                        for (int r = 0; r < RG; ++r) {
-                            part[r] = 0.f;
-                            if (rg + r < nr) {
-                                const uint32_t row = W0 + (uint32_t)(rg + r) * pl.row_bytes;
-#pragma unroll
-                                for (int j = 0; j < J; ++j) {
-                                    const int c = tid + kConsumerThreads * j;
-                                    if (c < nch) part[r] = dot8(lds128(row + 16u * c), v[j], part[r]);
-                                }
-                            }
-                        }
-                        const float s_row = reduce_rows<RG>(part, lane);
-                        const int rr = rg + reduce_rows_lane_row<RG>(lane);
-                        if (reduce_rows_writer<RG>(lane) && rr < nr) atomicAdd(&A[rr], s_row);
-                    }
+                    const uint4* Ws = reinterpret_cast<const uint4*>(stage + (size_t)s * pl.rps * pl.row_bytes);
+                    const int set = (vslot * pl.nspan + s) * pl.kparts + part;
+                    stage_rows<J, RG>(Ws, (int)(pl.row_bytes >> 4), nr, nch, v,
+                                      part_sums + ((size_t)set * rows + r0) * kConsumerWarps, lane);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[slot]);
@@ -637,11 +694,22 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     cbar();
     if (vload(&m.abort_flag)) return false;
 
-    // 5. epilogue (storer role)
+    // 5. epilogue (storer role): row value of accumulator set k (spans x
+    // slots) = the 8 warps' partial sums of every column part, in fixed order
+    auto acc = [&](int k, int r) {
+        float t = 0.f;
+        for (int q2 = 0; q2 < pl.kparts; ++q2) {
+            const float4* ps = reinterpret_cast<const float4*>(
+                part_sums + ((size_t)(k * pl.kparts + q2) * rows + r) * kConsumerWarps);
+            const float4 x0 = ps[0], x1 = ps[1];
+            t += ((x0.x + x0.y) + (x0.z + x0.w)) + ((x1.x + x1.y) + (x1.z + x1.w));
+        }
+        return t;
+    };
     switch (op) {
         case OP_RMS_QKV: {
             const int off = sub == 0 ? 0 : (sub == 1 ? p.nq * p.d : (p.nq + p.nkv) * p.d);
-            for (int r = tid; r < rows; r += kConsumerThreads) p.qkv[off + b + r] = acc[r];
+            for (int r = tid; r < rows; r += kConsumerThreads) p.qkv[off + b + r] = acc(0, r);
             break;
         }
         case OP_OPROJ_RES:
@@ -654,14 +722,14 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
                 } else {
                     base = __ldcg(p.x + b + r);
                 }
-                p.x[b + r] = base + acc[r];
+                p.x[b + r] = base + acc(0, r);
             }
             break;
         case OP_RMS_UPGATE_SILU:
         case OP_MOE_UPGATE: {
             float* h = p.hbuf + (op == OP_MOE_UPGATE ? (size_t)sub * p.F : 0);
             for (int r = tid; r < rows; r += kConsumerThreads) {
-                const float g = acc[r], u = acc[kMaxRows + r];
+                const float g = acc(0, r), u = acc(1, r);
                 h[b + r] = g / (1.0f + expf(-g)) * u;
             }
             break;
@@ -669,10 +737,10 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
         case OP_DOWN_RES:
         case OP_MOE_DOWN2_RES:
             for (int r = tid; r < rows; r += kConsumerThreads) {
-                float add = acc[r];
+                float add = acc(0, r);
                 if (op == OP_MOE_DOWN2_RES) {
-                    add = m.ew[0] * acc[r];
-                    if (p.topk > 1) add += m.ew[1] * acc[kMaxRows + r];
+                    add = m.ew[0] * add;
+                    if (p.topk > 1) add += m.ew[1] * acc(1, r);
                 }
                 const float nx = __ldcg(p.x + b + r) + add;
                 p.x[b + r] = nx;
@@ -683,7 +751,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
             float bv = -CUDART_INF_F;
             int bi = 0x7FFFFFFF;
             for (int r = tid; r < rows; r += kConsumerThreads) {
-                const float val = acc[r];
+                const float val = acc(0, r);
                 a.logits[b + r] = val;
                 if (val > bv || (val == bv && b + r < bi)) {
                     bv = val;
@@ -764,12 +832,23 @@ __device__ __forceinline__ void ml_combine(float& m, float& l, float* o, float m
     m = M;
 }
 
-template <int D, int G>
+// Query heads are split between the two halves of the consumer warps (each
+// half owns at most 2 of the kv head's query heads and streams every K/V row of
+// the stage for them), which keeps the per-thread q and output accumulators to
+// 2 x 8 + 2 x 8 registers.
 __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                            uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
-    constexpr int LPR = D / 8;                     // lanes per K/V row
-    constexpr int RGN = kConsumerThreads / LPR;    // rows per pass over the block
+    const int D = p.d;                                  // head_dim, 64 or 128
+    const int LPR = D / 8;                              // lanes per K/V row, 8 columns each
+    constexpr int GW = 2;                               // head slots per set
+    constexpr int SET_THREADS = kConsumerThreads / 2;
+    constexpr int SET_WARPS = kConsumerWarps / 2;
+    const int RGN = SET_THREADS / LPR;                  // rows per pass of a set
+    const int G = p.nq / p.nkv;                         // query heads per kv head (1..4)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int set = warp / SET_WARPS;
+    const int stid = tid - set * SET_THREADS;
+    const int h0 = set * GW;                            // first query head (within the group) of this set
     const int l = w[W_LAYER], g = w[W_SUB], c = w[W_BEGIN], S = w[W_END], pos = a.pos;
     const uint32_t SB = (uint32_t)p.stage_bytes;
     const AttnRange rg = attn_range(pos, c, S);
@@ -783,89 +862,86 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
     cbar();
     if (vload(&m.abort_flag)) return false;
 
-    // q of the group's heads, rotated (rotate-half pairing) and pre-scaled by log2(e)/sqrt(D)
-    const int col0 = (tid % LPR) * 8;
+    // q of this set's heads, rotated (rotate-half pairing) and pre-scaled by log2(e)/sqrt(D)
+    const int col0 = (stid % LPR) * 8;
     const int pcol = col0 ^ (D / 2);
-    const float2* rp = p.rope + (size_t)pos * (D / 2) + (col0 & (D / 2 - 1));
-    float cs[8], sn[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const float2 t = __ldg(rp + k);
-        cs[k] = t.x;
-        sn[k] = t.y;
-    }
     const bool first_half = col0 < D / 2;
     const float qscale = 1.4426950408889634f / sqrtf((float)D);
-    float q[G][8];
+    const float2* rp = p.rope + (size_t)pos * (D / 2) + (col0 & (D / 2 - 1));
+    float q[GW][8];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
+    for (int hh = 0; hh < GW; ++hh) {
+        const int h = h0 + hh < G ? h0 + hh : G - 1;  // spare head slots compute a copy that is never stored
         const float* src = p.qkv + (size_t)(g * G + h) * D;
-        float x[8], y[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            x[k] = __ldcg(src + col0 + k);
-            y[k] = __ldcg(src + pcol + k);
+            const float2 cssn = __ldg(rp + k);
+            const float x = __ldcg(src + col0 + k), y = __ldcg(src + pcol + k);
+            q[hh][k] = (first_half ? x * cssn.x - y * cssn.y : x * cssn.x + y * cssn.y) * qscale;
         }
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-            q[h][k] = (first_half ? x[k] * cs[k] - y[k] * sn[k] : x[k] * cs[k] + y[k] * sn[k]) * qscale;
     }
 
-    // the new position: rotated k and v rounded to bf16 (the cache format),
-    // appended by the split that holds it (threads of row group 0)
+    // the new position: rotated k and v rounded to bf16 (the cache format); the
+    // first row group of each set holds it, set 0 appends it to the cache
     float kn[8], vn[8];
-    if (rg.has_new && tid < LPR) {
+    const bool new_rows = rg.has_new && stid < 32;  // first warp of each set
+    if (new_rows) {
         const float* ks = p.qkv + (size_t)p.nq * D + (size_t)g * D;
         const float* vs = p.qkv + (size_t)(p.nq + p.nkv) * D + (size_t)g * D;
         uint32_t kb[8], vb[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
+            const float2 cssn = __ldg(rp + k);
             const float x = __ldcg(ks + col0 + k), y = __ldcg(ks + pcol + k);
-            const float r = first_half ? x * cs[k] - y * sn[k] : x * cs[k] + y * sn[k];
-            kb[k] = f2bf(r);
+            kb[k] = f2bf(first_half ? x * cssn.x - y * cssn.y : x * cssn.x + y * cssn.y);
             vb[k] = f2bf(__ldcg(vs + col0 + k));
             kn[k] = __uint_as_float(kb[k] << 16);
             vn[k] = __uint_as_float(vb[k] << 16);
         }
-        const size_t off = (((size_t)l * p.nkv + g) * (size_t)p.max_seq + (size_t)pos) * D + col0;
-        uint4 ku, vu;
-        ku.x = kb[0] | (kb[1] << 16); ku.y = kb[2] | (kb[3] << 16); ku.z = kb[4] | (kb[5] << 16); ku.w = kb[6] | (kb[7] << 16);
-        vu.x = vb[0] | (vb[1] << 16); vu.y = vb[2] | (vb[3] << 16); vu.z = vb[4] | (vb[5] << 16); vu.w = vb[6] | (vb[7] << 16);
-        *reinterpret_cast<uint4*>(p.kcache + off) = ku;
-        *reinterpret_cast<uint4*>(p.vcache + off) = vu;
+        if (set == 0 && stid < LPR) {
+            const size_t off = (((size_t)l * p.nkv + g) * (size_t)p.max_seq + (size_t)pos) * D + col0;
+            uint4 ku, vu;
+            ku.x = kb[0] | (kb[1] << 16); ku.y = kb[2] | (kb[3] << 16); ku.z = kb[4] | (kb[5] << 16); ku.w = kb[6] | (kb[7] << 16);
+            vu.x = vb[0] | (vb[1] << 16); vu.y = vb[2] | (vb[3] << 16); vu.z = vb[4] | (vb[5] << 16); vu.w = vb[6] | (vb[7] << 16);
+            *reinterpret_cast<uint4*>(p.kcache + off) = ku;
+            *reinterpret_cast<uint4*>(p.vcache + off) = vu;
+        }
     }
 
     // online softmax over the cached positions streamed through the ring
-    float mx[G], ls[G], o[G][8];
+    float mx[GW], ls[GW], o[GW][8];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        mx[h] = -CUDART_INF_F;
-        ls[h] = 0.f;
+    for (int hh = 0; hh < GW; ++hh) {
+        mx[hh] = -CUDART_INF_F;
+        ls[hh] = 0.f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[h][k] = 0.f;
+        for (int k = 0; k < 8; ++k) o[hh][k] = 0.f;
     }
     auto row_update = [&](const float* kf, const float* vf, bool valid) {
-        float s[G];
+        float sc[GW];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float t = 0.f;
+        for (int hh = 0; hh < GW; ++hh) {
+            float t0 = 0.f, t1 = 0.f;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) t = fmaf(q[h][k], kf[k], t);
-            s[h] = t;
+            for (int k = 0; k < 8; k += 2) {
+                t0 = fmaf(q[hh][k], kf[k], t0);
+                t1 = fmaf(q[hh][k + 1], kf[k + 1], t1);
+            }
+            sc[hh] = t0 + t1;
         }
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1)
 #pragma unroll
-            for (int h = 0; h < G; ++h) s[h] += __shfl_xor_sync(0xFFFFFFFFu, s[h], off);
+            for (int hh = 0; hh < GW; ++hh) sc[hh] += __shfl_xor_sync(0xFFFFFFFFu, sc[hh], off);
         if (valid) {
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const float mn = fmaxf(mx[h], s[h]);
-                const float al = exp2f(mx[h] - mn), pr = exp2f(s[h] - mn);
-                ls[h] = ls[h] * al + pr;
+            for (int hh = 0; hh < GW; ++hh) {
+                const float mn = fmaxf(mx[hh], sc[hh]);
+                const float al = exp2f(mx[hh] - mn), pr = exp2f(sc[hh] - mn);
+                ls[hh] = ls[hh] * al + pr;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) o[h][k] = fmaf(pr, vf[k], o[h][k] * al);
-                mx[h] = mn;
+                for (int k = 0; k < 8; ++k) o[hh][k] = fmaf(pr, vf[k], o[hh][k] * al);
+                mx[hh] = mn;
             }
         }
     };
@@ -878,15 +954,15 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
         const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, OP_ATTN);
         if (tr && tid == 0 && st == 0) tr[2] = globaltimer_ns();
         if (ok) {
-            const uint32_t Ks = smem_u32(ring) + slot * SB;
-            const uint32_t Vs = Ks + (uint32_t)pl.rps * D * 2u;
+            const uint4* Ks = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
+            const uint4* Vs = Ks + (size_t)pl.rps * (D / 8);
             for (int base = 0; base < nr; base += RGN) {
-                const int r = base + tid / LPR;
+                const int r = base + stid / LPR;
                 const bool valid = r < nr;
                 float kf[8], vf[8];
                 if (valid) {
-                    unpack8(lds128(Ks + (uint32_t)(r * D + col0) * 2u), kf);
-                    unpack8(lds128(Vs + (uint32_t)(r * D + col0) * 2u), vf);
+                    unpack8(Ks[r * (D / 8) + col0 / 8], kf);
+                    unpack8(Vs[r * (D / 8) + col0 / 8], vf);
                 } else {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) kf[k] = vf[k] = 0.f;
@@ -903,32 +979,32 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
             phase ^= 1u;
         }
     }
-    if (rg.has_new && warp == 0) row_update(kn, vn, lane < LPR);
+    if (new_rows) row_update(kn, vn, lane < LPR);
 
-    // merge row groups within the warp, then warps through shared memory
+    // merge row groups within the warp, then the set's warps through shared memory
 #pragma unroll
     for (int off = LPR; off < 32; off <<= 1) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float m2 = __shfl_xor_sync(0xFFFFFFFFu, mx[h], off);
-            const float l2 = __shfl_xor_sync(0xFFFFFFFFu, ls[h], off);
+        for (int hh = 0; hh < GW; ++hh) {
+            const float m2 = __shfl_xor_sync(0xFFFFFFFFu, mx[hh], off);
+            const float l2 = __shfl_xor_sync(0xFFFFFFFFu, ls[hh], off);
             float o2[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) o2[k] = __shfl_xor_sync(0xFFFFFFFFu, o[h][k], off);
-            ml_combine(mx[h], ls[h], o[h], m2, l2, o2);
+            for (int k = 0; k < 8; ++k) o2[k] = __shfl_xor_sync(0xFFFFFFFFu, o[hh][k], off);
+            ml_combine(mx[hh], ls[hh], o[hh], m2, l2, o2);
         }
     }
-    float* sm_o = scratch;                                 // [8 warps][G][D], G*D <= 512
-    float* sm_ml = scratch + kConsumerWarps * 512;         // [8 warps][G][2]
-    cbar();  // the accumulator region may still be read by nobody, but keep the union ordered
+    float* sm_o = scratch;                          // [8 warps][GW][D]
+    float* sm_ml = scratch + kConsumerWarps * 512;  // [8 warps][GW][2]
+    cbar();
     if (lane < LPR) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int hh = 0; hh < GW; ++hh) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) sm_o[(warp * G + h) * D + col0 + k] = o[h][k];
+            for (int k = 0; k < 8; ++k) sm_o[(warp * GW + hh) * D + col0 + k] = o[hh][k];
             if (lane == 0) {
-                sm_ml[(warp * G + h) * 2] = mx[h];
-                sm_ml[(warp * G + h) * 2 + 1] = ls[h];
+                sm_ml[(warp * GW + hh) * 2] = mx[hh];
+                sm_ml[(warp * GW + hh) * 2 + 1] = ls[hh];
             }
         }
     }
@@ -936,14 +1012,15 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
     if (vload(&m.abort_flag)) return false;
     for (int idx = tid; idx < G * D; idx += kConsumerThreads) {
         const int h = idx / D, col = idx % D;
+        const int hs = h / GW, hh = h % GW;  // owning set and head slot
         float M = -CUDART_INF_F;
-        for (int wv = 0; wv < kConsumerWarps; ++wv) M = fmaxf(M, sm_ml[(wv * G + h) * 2]);
+        for (int wv = hs * SET_WARPS; wv < (hs + 1) * SET_WARPS; ++wv) M = fmaxf(M, sm_ml[(wv * GW + hh) * 2]);
         float O = 0.f, Ls = 0.f;
         if (M != -CUDART_INF_F) {
-            for (int wv = 0; wv < kConsumerWarps; ++wv) {
-                const float f = exp2f(sm_ml[(wv * G + h) * 2] - M);
-                O += f * sm_o[(wv * G + h) * D + col];
-                Ls += f * sm_ml[(wv * G + h) * 2 + 1];
+            for (int wv = hs * SET_WARPS; wv < (hs + 1) * SET_WARPS; ++wv) {
+                const float f = exp2f(sm_ml[(wv * GW + hh) * 2] - M);
+                O += f * sm_o[(wv * GW + hh) * D + col];
+                Ls += f * sm_ml[(wv * GW + hh) * 2 + 1];
             }
         }
         const size_t part = (size_t)(g * G + h) * S + c;
@@ -967,13 +1044,13 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
             const int h = idx / D, col = idx % D;
             const size_t base = (size_t)(g * G + h) * S;
             float M = -CUDART_INF_F;
-            for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(p.part_ml + (base + s) * 2));
+            for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, __ldcg(p.part_ml + (base + s2) * 2));
             float num = 0.f, den = 0.f;
-            for (int s = 0; s < S; ++s) {
-                const float ms = __ldcg(p.part_ml + (base + s) * 2);
+            for (int s2 = 0; s2 < S; ++s2) {
+                const float ms = __ldcg(p.part_ml + (base + s2) * 2);
                 const float f = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
-                num += f * __ldcg(p.part_o + (base + s) * D + col);
-                den += f * __ldcg(p.part_ml + (base + s) * 2 + 1);
+                num += f * __ldcg(p.part_o + (base + s2) * D + col);
+                den += f * __ldcg(p.part_ml + (base + s2) * 2 + 1);
             }
             p.attn[(size_t)(g * G + h) * D + col] = num / den;
         }
@@ -984,18 +1061,6 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
         }
     }
     return true;
-}
-
-template <int D>
-__device__ bool attn_dispatch_g(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
-                                uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
-    switch (p.nq / p.nkv) {
-        case 1: return attn_instr<D, 1>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-        case 2: return attn_instr<D, 2>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-        case 3: return attn_instr<D, 3>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-        case 4: return attn_instr<D, 4>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-    }
-    return false;
 }
 
 __device__ __forceinline__ int gemv_k(const DevParams& p, int op) {
@@ -1020,6 +1085,36 @@ __device__ bool gemv_dispatch(const DevParams& p, const StepArgs& a, const int32
         case 4: return gemv_instr<4>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
     }
     return false;
+}
+
+// Consumers prefetch, into L2, the weight (or KV-cache) rows of the
+// instruction `ahead` places further in their block's queue, spread over the
+// 256 consumer threads one 128-byte line each.  Issued before the dependency
+// wait of the current instruction, so the HBM keeps streaming while the block
+// waits; each instruction is prefetched once.  MoE instructions whose routing
+// is not known yet are skipped.
+__device__ void prefetch_instr(const DevParams& p, const StepArgs& a, const int32_t* w, const Misc& m) {
+    if (!instr_ok(p, w)) return;
+    int eidx[kMaxTopK] = {0, 0};
+    if (needs_routing(w[W_OP])) {
+        if (m.router_layer != w[W_LAYER]) return;
+        eidx[0] = m.eidx[0];
+        eidx[1] = m.eidx[1];
+    }
+    Plan pl;
+    make_plan(p, a.pos, w, eidx, pl);
+    const size_t cap = (size_t)p.prefetch_max_bytes;
+    size_t done = 0;
+    const int nslot = pl.nphase / pl.kparts;
+    for (int sl = 0; sl < nslot; ++sl)
+        for (int s = 0; s < pl.nspan; ++s) {
+            const unsigned char* base = pl.src[sl][s];
+            size_t bytes = (size_t)pl.rows * pl.src_stride;
+            if (done + bytes > cap) bytes = cap > done ? cap - done : 0;
+            for (size_t off = (size_t)threadIdx.x * 128; off < bytes; off += (size_t)kConsumerThreads * 128)
+                prefetch_line_l2(base + off);
+            done += bytes;
+        }
 }
 
 // ---------------------------------------------------------------------------
@@ -1061,6 +1156,8 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     for (int i = 0; i < n; ++i) {
         const int32_t* w = q + (size_t)i * W_NWORDS;
         if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * 4] = globaltimer_ns();
+        if (p.prefetch_ahead > 0 && i + p.prefetch_ahead < n)
+            prefetch_instr(p, a, q + (size_t)(i + p.prefetch_ahead) * W_NWORDS, m);
         bool ok;
         if (!instr_ok(p, w) || token < 0 || token >= p.V) {
             if (tid == 0) {
@@ -1069,8 +1166,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             }
             ok = false;
         } else if (w[W_OP] == OP_ATTN) {
-            ok = p.d == 64 ? attn_dispatch_g<64>(p, a, w, i, smem, full, empty, scratch, m, slot, phase)
-                           : attn_dispatch_g<128>(p, a, w, i, smem, full, empty, scratch, m, slot, phase);
+            ok = attn_instr(p, a, w, i, smem, full, empty, scratch, m, slot, phase);
         } else {
             ok = gemv_dispatch(p, a, w, i, smem, full, empty, scratch, m, slot, phase, token);
         }

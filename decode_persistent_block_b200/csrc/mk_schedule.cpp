@@ -99,10 +99,12 @@ int check_config(const mk_config& c) {
 }
 
 void fill_defaults(mk_options* o) {
-    if (o->ring_stages <= 0) o->ring_stages = 6;
-    if (o->stage_bytes <= 0) o->stage_bytes = 32768;
+    if (o->ring_stages <= 0) o->ring_stages = 3;
+    if (o->stage_bytes <= 0) o->stage_bytes = 65536;
     if (o->rows_per_instr <= 0 || o->rows_per_instr > kMaxRows) o->rows_per_instr = kMaxRows;
     if (o->l2_prefetch < 0) o->l2_prefetch = 0;
+    if (o->prefetch_ahead < 0) o->prefetch_ahead = 0;
+    if (o->prefetch_max_bytes <= 0) o->prefetch_max_bytes = 1 << 20;
     if (o->spin_limit_ns == 0) o->spin_limit_ns = 2000000000ull;
 }
 
@@ -117,6 +119,9 @@ int check_options(const mk_config& c, const mk_options& o) {
         return MK_ERR_UNSUPPORTED;
     if (2LL * 2 * c.head_dim > sb) return MK_ERR_UNSUPPORTED;
     if (o.mode < MK_MODE_MEGAKERNEL || o.mode > MK_MODE_MULTI_KERNEL_GRAPH) return MK_ERR_INVALID_ARG;
+    // ring + barriers + partial-sum slots + misc must fit the 227 KB per-block opt-in limit
+    if ((long long)o.ring_stages * o.stage_bytes + 16LL * o.ring_stages + 128 + 4LL * kRowSlots * 8 + 512 > 232448)
+        return MK_ERR_INVALID_ARG;
     return MK_OK;
 }
 
@@ -139,8 +144,10 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
         if (w[W_SIGNAL_CTR] >= 0 && w[W_OP] != OP_ATTN) inc[w[W_SIGNAL_CTR]]++;
         if (w[W_AUX_CTR] >= 0) inc[w[W_AUX_CTR]]++;
     };
+    const int qd = c.n_q_heads * d;
+    auto op_cap = [&](int op) { return std::min(cap, kRowSlots / acc_sets(op, H, qd, F, c.top_k)); };
     auto gemv_op = [&](int op, int layer, const std::vector<Segment>& segs, int wait, int signal) {
-        split_rows(segs, n_sm, cap, [&](int sm, int sub, int b, int e) {
+        split_rows(segs, n_sm, op_cap(op), [&](int sm, int sub, int b, int e) {
             Instr w = blank();
             w[W_OP] = op;
             w[W_LAYER] = layer;
@@ -188,7 +195,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     {
         int seq = 0;
         const int wait = L > 0 ? ctr_id(L - 1, C_FFN2, nkv) : -1;
-        split_rows({{0, c.vocab}}, n_sm, cap, [&](int sm, int, int b, int e) {
+        split_rows({{0, c.vocab}}, n_sm, op_cap(OP_LMHEAD_ARGMAX), [&](int sm, int, int b, int e) {
             Instr w = blank();
             w[W_OP] = OP_LMHEAD_ARGMAX;
             w[W_LAYER] = L;
@@ -320,7 +327,8 @@ int validate(const mk_config& c, const Planned& p) {
             if (op == OP_MOE_UPGATE && (sub < 0 || sub >= c.top_k)) return MK_ERR_SCHEDULE;
             if (op != OP_RMS_QKV && op != OP_MOE_UPGATE && sub != 0) return MK_ERR_SCHEDULE;
             const int b = w[W_BEGIN], e = w[W_END];
-            if (b < 0 || e > R || b >= e || e - b > kMaxRows) return MK_ERR_SCHEDULE;
+            const int sets = acc_sets(op, c.hidden, c.n_q_heads * d, c.ffn, c.top_k);
+            if (b < 0 || e > R || b >= e || e - b > kMaxRows || (e - b) * sets > kRowSlots) return MK_ERR_SCHEDULE;
             auto& hits = cov[cov_key(l, op, sub)];
             if (hits.empty()) hits.assign(R, 0);
             for (int r = b; r < e; ++r)

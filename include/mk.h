@@ -84,8 +84,8 @@ typedef struct {
  * KV caches at the decoded position).  Per-layer arrays are HOST arrays of
  * n_layers device pointers; for MoE, w_gate/w_up/w_down have
  * n_layers * n_experts entries ([layer * n_experts + expert]) and router has
- * n_layers entries.  router may be NULL for dense models.  All device
- * pointers must be 16-byte aligned. */
+ * n_layers entries.  router may be NULL for dense models; the KV caches may
+ * be NULL when n_layers == 0.  All device pointers must be 16-byte aligned. */
 typedef struct {
     const void *embed, *lm_head, *final_norm;
     const void *const *attn_norm, *const *wq, *const *wk, *const *wv, *const *wo, *const *ffn_norm;
@@ -95,10 +95,10 @@ typedef struct {
 } mk_weights;
 
 /* Schedule and kernel knobs.  Zero selects the default for every field except
- * l2_prefetch (-1 = default, 0 = off). */
+ * l2_prefetch and prefetch_ahead (-1 = default, 0 = off). */
 typedef struct {
-    int ring_stages;      /* shared-memory weight ring depth (default 6) */
-    int stage_bytes;      /* bytes per ring stage, multiple of 1024 (default 32768) */
+    int ring_stages;      /* shared-memory weight ring depth (default 3) */
+    int stage_bytes;      /* bytes per ring stage, multiple of 1024 (default 65536) */
     int rows_per_instr;   /* cap on GEMV rows per instruction (default and max 1024) */
     int kv_splits;        /* split-KV chunks per kv head (default: SMs / n_kv_heads, capped by max_seq/32) */
     int l2_prefetch;      /* bytes kept prefetched into L2 ahead of the TMA stream (-1 default) */
@@ -107,6 +107,9 @@ typedef struct {
     unsigned long long spin_limit_ns; /* bound on every device-side wait (default 2 s) */
     int mode;             /* MK_MODE_* */
     int n_sm;             /* blocks of the persistent grid (default: all SMs) */
+    int prefetch_ahead;   /* consumers prefetch into L2 the weights of the instruction this many
+                             places ahead in their queue (-1 default, 0 = off) */
+    int prefetch_max_bytes; /* cap on the bytes prefetched per instruction (0 = default 1 MiB) */
 } mk_options;
 
 /* Device status block, copied out by mk_get_status.  On a device-side error
