@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["mk_api.cu", "mk_megakernel.cu", "mk_baseline.cu", "mk_schedule.cpp"]
+SOURCES = ["mk_api.cu", "mk_megakernel.cu", "mk_baseline.cu", "mk_ops.cu", "mk_schedule.cpp"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -1,0 +1,207 @@
+// mk_ops.cu -- standalone opcode entry points (one plain launch per call),
+// used for per-opcode parity tests and by callers that want a single op.
+//
+// mk_attention_decode: GQA decode attention of one layer over cached
+// positions [0, n_pos), split along the sequence (split-KV) so that the
+// low-occupancy op still spreads over many SMs, then merged by the
+// log-sum-exp rule.  Query head h reads kv head floor(h / (n_q / n_kv)).
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "mk_device.cuh"
+#include "mk_internal.h"
+
+namespace mk {
+namespace {
+
+constexpr int kOpThreads = 256;
+constexpr int kOpWarps = kOpThreads / 32;
+
+struct AttnOpArgs {
+    const float* q;          // [nq][d], already rotated
+    const uint16_t* kcache;  // [nkv][max_seq][d] bf16
+    const uint16_t* vcache;
+    int nq, nkv, n_pos, max_seq, splits;
+    float* part_o;           // [nq][splits][d]
+    float* part_ml;          // [nq][splits][2] (max score in log2 units, sum of exponentials)
+    float* out;              // [nq][d]
+};
+
+// One block per (split, kv head): every query head of the group over the
+// split's positions, online softmax per thread, merged across the block.
+template <int D>
+__global__ void __launch_bounds__(kOpThreads) attn_op_split(const AttnOpArgs a) {
+    constexpr int LPR = D / 8;
+    constexpr int RGN = kOpThreads / LPR;
+    __shared__ float sq[kMaxGroup * D];
+    __shared__ float sm_o[kOpWarps * kMaxGroup * D];
+    __shared__ float sm_ml[kOpWarps * kMaxGroup * 2];
+    const int G = a.nq / a.nkv;
+    const int c = blockIdx.x, g = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int jb = (int)((long long)a.n_pos * c / a.splits), je = (int)((long long)a.n_pos * (c + 1) / a.splits);
+    const float qscale = 1.4426950408889634f / sqrtf((float)D);
+    for (int i = tid; i < G * D; i += kOpThreads) sq[i] = a.q[(size_t)g * G * D + i] * qscale;
+    __syncthreads();
+    const int col0 = (tid % LPR) * 8;
+    float q[kMaxGroup][8], mx[kMaxGroup], ls[kMaxGroup], o[kMaxGroup][8];
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+        mx[h] = -CUDART_INF_F;
+        ls[h] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            o[h][k] = 0.f;
+            q[h][k] = h < G ? sq[h * D + col0 + k] : 0.f;
+        }
+    }
+    const uint16_t* K = a.kcache + (size_t)g * a.max_seq * D;
+    const uint16_t* V = a.vcache + (size_t)g * a.max_seq * D;
+    for (int base = jb; base < je; base += RGN) {
+        const int j = base + tid / LPR;
+        const bool valid = j < je;
+        float kf[8], vf[8];
+        if (valid) {
+            unpack8(*reinterpret_cast<const uint4*>(K + (size_t)j * D + col0), kf);
+            unpack8(*reinterpret_cast<const uint4*>(V + (size_t)j * D + col0), vf);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) kf[k] = vf[k] = 0.f;
+        }
+        float s[kMaxGroup];
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) {
+            float t = 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t = fmaf(q[h][k], kf[k], t);
+            s[h] = t;
+        }
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1)
+#pragma unroll
+            for (int h = 0; h < kMaxGroup; ++h) s[h] += __shfl_xor_sync(0xFFFFFFFFu, s[h], off);
+        if (valid) {
+#pragma unroll
+            for (int h = 0; h < kMaxGroup; ++h) {
+                if (h >= G) break;
+                const float mn = fmaxf(mx[h], s[h]);
+                const float al = exp2f(mx[h] - mn), pr = exp2f(s[h] - mn);
+                ls[h] = ls[h] * al + pr;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) o[h][k] = fmaf(pr, vf[k], o[h][k] * al);
+                mx[h] = mn;
+            }
+        }
+    }
+    // merge the row groups of a warp, then the warps
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1)
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) {
+            const float m2 = __shfl_xor_sync(0xFFFFFFFFu, mx[h], off);
+            const float l2 = __shfl_xor_sync(0xFFFFFFFFu, ls[h], off);
+            float o2[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o2[k] = __shfl_xor_sync(0xFFFFFFFFu, o[h][k], off);
+            const float M = fmaxf(mx[h], m2);
+            if (M != -CUDART_INF_F) {
+                const float x = exp2f(mx[h] - M), y = exp2f(m2 - M);
+                ls[h] = x * ls[h] + y * l2;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) o[h][k] = x * o[h][k] + y * o2[k];
+                mx[h] = M;
+            }
+        }
+    if (lane < LPR)
+        for (int h = 0; h < G; ++h) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) sm_o[(warp * kMaxGroup + h) * D + col0 + k] = o[h][k];
+            if (lane == 0) {
+                sm_ml[(warp * kMaxGroup + h) * 2] = mx[h];
+                sm_ml[(warp * kMaxGroup + h) * 2 + 1] = ls[h];
+            }
+        }
+    __syncthreads();
+    for (int idx = tid; idx < G * D; idx += kOpThreads) {
+        const int h = idx / D, col = idx % D;
+        float M = -CUDART_INF_F;
+        for (int w = 0; w < kOpWarps; ++w) M = fmaxf(M, sm_ml[(w * kMaxGroup + h) * 2]);
+        float O = 0.f, L = 0.f;
+        if (M != -CUDART_INF_F)
+            for (int w = 0; w < kOpWarps; ++w) {
+                const float f = exp2f(sm_ml[(w * kMaxGroup + h) * 2] - M);
+                O += f * sm_o[(w * kMaxGroup + h) * D + col];
+                L += f * sm_ml[(w * kMaxGroup + h) * 2 + 1];
+            }
+        const size_t slot = (size_t)(g * G + h) * a.splits + c;
+        a.part_o[slot * D + col] = O;
+        if (col == 0) {
+            a.part_ml[slot * 2] = M;
+            a.part_ml[slot * 2 + 1] = L;
+        }
+    }
+}
+
+// out[h] = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) L_c; grid nq, block d.
+__global__ void attn_op_merge(const AttnOpArgs a, int D) {
+    const int h = blockIdx.x, col = threadIdx.x;
+    if (col >= D) return;
+    float M = -CUDART_INF_F;
+    for (int c = 0; c < a.splits; ++c) M = fmaxf(M, a.part_ml[((size_t)h * a.splits + c) * 2]);
+    float num = 0.f, den = 0.f;
+    for (int c = 0; c < a.splits; ++c) {
+        const float m = a.part_ml[((size_t)h * a.splits + c) * 2];
+        const float f = m == -CUDART_INF_F ? 0.f : exp2f(m - M);
+        num += f * a.part_o[((size_t)h * a.splits + c) * D + col];
+        den += f * a.part_ml[((size_t)h * a.splits + c) * 2 + 1];
+    }
+    a.out[(size_t)h * D + col] = num / den;
+}
+
+int check_attn_args(const float* q, const void* kc, const void* vc, int nq, int nkv, int d, int n_pos, int max_seq,
+                    float* out, int splits) {
+    if (!q || !kc || !vc || !out) return MK_ERR_INVALID_ARG;
+    if (nq <= 0 || nkv <= 0 || n_pos <= 0 || max_seq < n_pos || splits <= 0) return MK_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return MK_ERR_UNSUPPORTED;
+    if (nq % nkv || nq / nkv > kMaxGroup) return MK_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(kc) | reinterpret_cast<uintptr_t>(vc)) & 15u) return MK_ERR_INVALID_ARG;
+    return MK_OK;
+}
+
+int launch_attn(const AttnOpArgs& a, int d, cudaStream_t s) {
+    const dim3 grid(a.splits, a.nkv);
+    if (d == 64) attn_op_split<64><<<grid, kOpThreads, 0, s>>>(a);
+    else attn_op_split<128><<<grid, kOpThreads, 0, s>>>(a);
+    attn_op_merge<<<a.nq, d, 0, s>>>(a, d);
+    return cudaGetLastError() == cudaSuccess ? MK_OK : MK_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace mk
+
+extern "C" size_t mk_attention_workspace_bytes(int n_q_heads, int head_dim, int splits) {
+    if (n_q_heads <= 0 || head_dim <= 0 || splits <= 0) return 0;
+    return sizeof(float) * (size_t)n_q_heads * (size_t)splits * (size_t)(head_dim + 2);
+}
+
+extern "C" int mk_attention_decode(const float* q, const void* k_cache, const void* v_cache, int n_q_heads,
+                                   int n_kv_heads, int head_dim, int n_pos, int max_seq, int splits, float* out,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = mk::check_attn_args(q, k_cache, v_cache, n_q_heads, n_kv_heads, head_dim, n_pos, max_seq, out, splits);
+    if (rc) return rc;
+    const size_t need = mk_attention_workspace_bytes(n_q_heads, head_dim, splits);
+    if (!workspace || workspace_bytes < need) return MK_ERR_CAPACITY;
+    mk::AttnOpArgs a;
+    a.q = q;
+    a.kcache = static_cast<const uint16_t*>(k_cache);
+    a.vcache = static_cast<const uint16_t*>(v_cache);
+    a.nq = n_q_heads;
+    a.nkv = n_kv_heads;
+    a.n_pos = n_pos;
+    a.max_seq = max_seq;
+    a.splits = splits;
+    a.part_o = static_cast<float*>(workspace);
+    a.part_ml = a.part_o + (size_t)n_q_heads * splits * head_dim;
+    a.out = out;
+    return mk::launch_attn(a, head_dim, static_cast<cudaStream_t>(stream));
+}

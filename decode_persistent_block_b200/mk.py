@@ -77,6 +77,8 @@ SIGNATURES = {
     "mk_plan": (_I, [ctypes.POINTER(MkConfig), ctypes.POINTER(MkOptions), _I, _P, ctypes.c_size_t,
                      ctypes.POINTER(_I), _P, _P, ctypes.c_size_t, ctypes.POINTER(_I)]),
     "mk_simulate": (_I, [_P, _I, _I, _P, _P, _I, _I, ctypes.c_uint64, ctypes.POINTER(ctypes.c_longlong)]),
+    "mk_attention_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I]),
+    "mk_attention_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]),
 }
 
 _lib = None
@@ -313,6 +315,24 @@ class Decoder:
         ns = ctypes.c_double(0)
         check(self.lib.mk_last_step_ns(self.h, ctypes.byref(ns)), "mk_last_step_ns")
         return ns.value
+
+
+def attention_decode(q, kcache, vcache, n_pos: int, splits: int, out, workspace=None, stream=None):
+    """mk_attention_decode on torch CUDA tensors: q [nq, d] fp32, kcache/vcache
+    [nkv, max_seq, d] bf16 bits, out [nq, d] fp32.  Allocates the workspace
+    with torch when none is given."""
+    import torch
+    lib = load()
+    nq, d = int(q.shape[0]), int(q.shape[1])
+    nkv, max_seq = int(kcache.shape[0]), int(kcache.shape[1])
+    need = lib.mk_attention_workspace_bytes(nq, d, splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    s = stream if stream is not None else torch.cuda.current_stream()
+    check(lib.mk_attention_decode(_ptr(q), _ptr(kcache), _ptr(vcache), nq, nkv, d, n_pos, max_seq, splits, _ptr(out),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  ctypes.c_void_p(s.cuda_stream)), "mk_attention_decode")
+    return out
 
 
 def to_device(model: dict, device="cuda"):

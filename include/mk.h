@@ -197,6 +197,30 @@ int mk_last_step_ns(mk_handle *h, double *ns);
 const char *mk_strerror(int code);
 void mk_destroy(mk_handle *h);
 
+/* ---- standalone ops ------------------------------------------------------------------- */
+
+/* Bytes of workspace mk_attention_decode needs: n_q_heads * splits * (head_dim + 2) floats. */
+size_t mk_attention_workspace_bytes(int n_q_heads, int head_dim, int splits);
+
+/* GQA decode attention of one layer, as one op (two plain launches on
+ * `stream`, a cudaStream_t or NULL): for query head h and its kv head
+ * g = floor(h / (n_q_heads / n_kv_heads)),
+ *   out[h] = softmax_j(q[h] . K[g][j] / sqrt(head_dim)) V[g][j],  j in [0, n_pos)
+ * (the decode attention step of the Llama decoder the megakernel pages target;
+ * the sequence is split into `splits` chunks whose partial softmax states are
+ * merged by the log-sum-exp rule, "split-KV").
+ * q: device fp32 [n_q_heads][head_dim], already rotated.  k_cache, v_cache:
+ * device bf16 [n_kv_heads][max_seq][head_dim], 16-byte aligned.  out: device
+ * fp32 [n_q_heads][head_dim].  workspace: device, at least
+ * mk_attention_workspace_bytes(...) bytes, caller-owned, overwritten.
+ * head_dim in {64, 128}; 1..4 query heads per kv head; 1 <= n_pos <= max_seq;
+ * splits >= 1 (splits beyond n_pos leave empty chunks, which merge to
+ * nothing).  Enqueues only.  Errors: MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED,
+ * MK_ERR_CAPACITY (workspace too small), MK_ERR_CUDA. */
+int mk_attention_decode(const float *q, const void *k_cache, const void *v_cache, int n_q_heads, int n_kv_heads,
+                        int head_dim, int n_pos, int max_seq, int splits, float *out, void *workspace,
+                        size_t workspace_bytes, void *stream);
+
 /* ---- host-only planning (no GPU needed) ---------------------------------------- */
 
 /* Plan the schedule for `n_sm` blocks without a device: writes the instruction

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "mk.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return set(re.findall(r"^\s*(?:int|void|const\s+char\s*\*)\s*\*?\s*(mk_\w+)\s*\(", src, flags=re.M))
+    return set(re.findall(r"^\s*(?:int|void|size_t|const\s+char\s*\*)\s*\*?\s*(mk_\w+)\s*\(", src, flags=re.M))
 
 
 @pytest.fixture(scope="module")
