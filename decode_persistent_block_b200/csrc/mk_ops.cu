@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <mutex>
+
 #include "mk_device.cuh"
 #include "mk_internal.h"
 
@@ -202,6 +204,57 @@ extern "C" int mk_attention_decode(const float* q, const void* k_cache, const vo
     a.splits = splits;
     a.part_o = static_cast<float*>(workspace);
     a.part_ml = a.part_o + (size_t)n_q_heads * splits * head_dim;
+    a.out = out;
+    return mk::launch_attn(a, head_dim, static_cast<cudaStream_t>(stream));
+}
+
+// ---- variant without allocation -------------------------------------------------------------
+//
+// Scratch for mk_attention_decode_noalloc: the split partials live in this
+// file-scope device array instead of a caller workspace.  Every GPU that loads
+// the library holds it (MK_ATTENTION_NOALLOC_SCRATCH_BYTES) until the process
+// exits.  All calls share it and it keeps the last call's contents; the split
+// kernel writes every partial slot a call reads, so nothing needs clearing.
+static __device__ __align__(256) float g_attn_noalloc_scratch[MK_ATTENTION_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+constexpr int kMaxDevices = 64;
+float* g_scratch_addr[kMaxDevices];  // device address of the array, per device ordinal (host-side cache)
+std::mutex g_scratch_mu;
+}  // namespace
+
+extern "C" int mk_attention_decode_noalloc(const float* q, const void* k_cache, const void* v_cache, int n_q_heads,
+                                           int n_kv_heads, int head_dim, int n_pos, int max_seq, int splits,
+                                           float* out, void* stream) {
+    int rc = mk::check_attn_args(q, k_cache, v_cache, n_q_heads, n_kv_heads, head_dim, n_pos, max_seq, out, splits);
+    if (rc) return rc;
+    if (mk_attention_workspace_bytes(n_q_heads, head_dim, splits) > MK_ATTENTION_NOALLOC_SCRATCH_BYTES)
+        return MK_ERR_CAPACITY;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MK_ERR_CUDA;
+    float* scratch = nullptr;
+    {
+        // Set-up, once per device, with that device current: the array's name is a
+        // host-side stand-in, so its device address has to be looked up.
+        std::lock_guard<std::mutex> lock(g_scratch_mu);
+        if (!g_scratch_addr[dev]) {
+            void* addr = nullptr;
+            if (cudaGetSymbolAddress(&addr, g_attn_noalloc_scratch) != cudaSuccess || !addr) return MK_ERR_CUDA;
+            g_scratch_addr[dev] = static_cast<float*>(addr);
+        }
+        scratch = g_scratch_addr[dev];
+    }
+    mk::AttnOpArgs a;
+    a.q = q;
+    a.kcache = static_cast<const uint16_t*>(k_cache);
+    a.vcache = static_cast<const uint16_t*>(v_cache);
+    a.nq = n_q_heads;
+    a.nkv = n_kv_heads;
+    a.n_pos = n_pos;
+    a.max_seq = max_seq;
+    a.splits = splits;
+    a.part_o = scratch;
+    a.part_ml = scratch + (size_t)n_q_heads * splits * head_dim;
     a.out = out;
     return mk::launch_attn(a, head_dim, static_cast<cudaStream_t>(stream));
 }

@@ -79,7 +79,9 @@ SIGNATURES = {
     "mk_simulate": (_I, [_P, _I, _I, _P, _P, _I, _I, ctypes.c_uint64, ctypes.POINTER(ctypes.c_longlong)]),
     "mk_attention_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I]),
     "mk_attention_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]),
+    "mk_attention_decode_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
 }
+NOALLOC_SCRATCH_BYTES = 1 << 20  # MK_ATTENTION_NOALLOC_SCRATCH_BYTES
 
 _lib = None
 
@@ -332,6 +334,20 @@ def attention_decode(q, kcache, vcache, n_pos: int, splits: int, out, workspace=
     check(lib.mk_attention_decode(_ptr(q), _ptr(kcache), _ptr(vcache), nq, nkv, d, n_pos, max_seq, splits, _ptr(out),
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   ctypes.c_void_p(s.cuda_stream)), "mk_attention_decode")
+    return out
+
+
+def attention_decode_noalloc(q, kcache, vcache, n_pos: int, splits: int, out, stream=None):
+    """mk_attention_decode_noalloc on torch CUDA tensors (same layout as
+    attention_decode); the library uses its own fixed device scratch, so
+    nothing is allocated for the call."""
+    import torch
+    lib = load()
+    nq, d = int(q.shape[0]), int(q.shape[1])
+    nkv, max_seq = int(kcache.shape[0]), int(kcache.shape[1])
+    s = stream if stream is not None else torch.cuda.current_stream()
+    check(lib.mk_attention_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), nq, nkv, d, n_pos, max_seq, splits,
+                                          _ptr(out), ctypes.c_void_p(s.cuda_stream)), "mk_attention_decode_noalloc")
     return out
 
 

@@ -221,6 +221,32 @@ int mk_attention_decode(const float *q, const void *k_cache, const void *v_cache
                         int head_dim, int n_pos, int max_seq, int splits, float *out, void *workspace,
                         size_t workspace_bytes, void *stream);
 
+/* Size of the device-resident scratch of mk_attention_decode_noalloc: 1 MiB,
+ * i.e. n_q_heads * splits * (head_dim + 2) <= 262144 floats. */
+#define MK_ATTENTION_NOALLOC_SCRATCH_BYTES ((size_t)1 << 20)
+
+/* mk_attention_decode for callers that cannot allocate device memory: the
+ * same computation, arguments and errors, but no workspace argument.  It is
+ * for code that must not call cudaMalloc, for example a host whose device
+ * memory is owned by another allocator or pool, or a latency-critical decode
+ * loop where an allocation (and the device synchronisation it can imply) is
+ * not allowed.  This entry point calls no cudaMalloc, cudaFree or other
+ * allocating routine.  The paper has no counterpart for it.
+ *  - Its split partials live in one fixed device array of
+ *    MK_ATTENTION_NOALLOC_SCRATCH_BYTES inside the library, present on every
+ *    GPU that loads the library until the process exits; a call whose
+ *    n_q_heads * splits * (head_dim + 2) floats exceed it returns
+ *    MK_ERR_CAPACITY.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture.
+ *  - All calls share the array: calls that overlap on the GPU (for example on
+ *    two streams at once) race and give wrong results; serialise them.  Each
+ *    call writes every slot it reads, so no clearing is needed between calls. */
+int mk_attention_decode_noalloc(const float *q, const void *k_cache, const void *v_cache, int n_q_heads,
+                                int n_kv_heads, int head_dim, int n_pos, int max_seq, int splits, float *out,
+                                void *stream);
+
 /* ---- host-only planning (no GPU needed) ---------------------------------------- */
 
 /* Plan the schedule for `n_sm` blocks without a device: writes the instruction
