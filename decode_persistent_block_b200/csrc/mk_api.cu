@@ -31,6 +31,7 @@ struct mk_handle {
     cudaGraph_t graph = nullptr;
     cudaGraphExec_t graph_exec = nullptr;
     int lm_slots = 0;
+    bool down_t = false;  // transposed down-projection copies exist (fused FFN schedules)
     int last_cuda = 0;
     int last_error = MK_OK;
 };
@@ -167,6 +168,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     mk::fill_defaults(&o);
     rc = mk::check_options(*cfg, o);
     if (rc) return rc;
+    if (o.mode != MK_MODE_MEGAKERNEL) o.split_ffn = 1;  // the schedule of the plain launches is never fused
 
     mk_handle* h = new mk_handle();
     h->cfg = *cfg;
@@ -232,6 +234,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     if ((rc = dalloc(h, &p.counters, (size_t)p.n_ctr))) return fail(rc);
     if ((rc = dalloc(h, &p.status, 1))) return fail(rc);
     if ((rc = dalloc(h, &p.x, (size_t)H))) return fail(rc);
+    if ((rc = dalloc(h, &p.x2, (size_t)H))) return fail(rc);
     if ((rc = dalloc(h, &p.qkv, (size_t)(nq + 2 * nkv) * d))) return fail(rc);
     if ((rc = dalloc(h, &p.attn, (size_t)nq * d))) return fail(rc);
     if ((rc = dalloc(h, &p.part_o, (size_t)nq * S * d))) return fail(rc);
@@ -245,6 +248,23 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     float2* rope = nullptr;
     if ((rc = dalloc(h, &rope, (size_t)c.max_seq * (d / 2)))) return fail(rc);
     if ((rc = dalloc(h, &h->stepbuf, 1))) return fail(rc);
+    // The fused FFN streams the down-projection by its input index: keep a
+    // transposed copy [ffn][hidden] of every w_down (library-owned).
+    if (o.mode == MK_MODE_MEGAKERNEL && mk::ffn_fused(c, o)) {
+        const int ne = E > 0 ? E : 1;
+        for (int l = 0; l < L; ++l)
+            for (int x = 0; x < ne; ++x) {
+                const uint16_t** t = &h->wt_host[(size_t)l * stride];
+                uint16_t* dt = nullptr;
+                if ((rc = dalloc(h, &dt, (size_t)c.ffn * H))) return fail(rc);
+                e = mk::launch_transpose_bf16(t[mk::wt_down(x, E)], dt, H, c.ffn, nullptr);
+                if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
+                t[mk::wt_down_t(x, E)] = dt;
+            }
+        e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
+        h->down_t = true;
+    }
     p.wt = wt_dev;
     p.rope = rope;
     e = cudaMemcpy(wt_dev, h->wt_host.data(), h->wt_host.size() * sizeof(void*), cudaMemcpyHostToDevice);
@@ -288,6 +308,7 @@ int mk_build_schedule(mk_handle* h) {
     if (rc) return rc;
     if (plan.kv_splits != h->p.kv_splits) return MK_ERR_SCHEDULE;
     if (plan.n_lm > h->lm_slots) return MK_ERR_SCHEDULE;
+    if (plan.fused_ffn && h->cfg.n_layers > 0 && !h->down_t) return MK_ERR_SCHEDULE;
     h->plan = plan;
     int32_t* words = nullptr;
     int32_t* n_instr = nullptr;

@@ -30,7 +30,10 @@ enum Opcode : int32_t {
     OP_LMHEAD_ARGMAX = 6,    // logits[rows] = Wlm[rows] rmsnorm(x) * w_final; last instruction reduces argmax
     OP_MOE_UPGATE = 7,       // router + top-k in prologue; h_slot[rows] for the selected expert of `slot`
     OP_MOE_DOWN2_RES = 8,    // x[rows] += sum_slot w_slot * Wd_{e_slot}[rows] h_slot  (all slots, one instr)
-    OP_COUNT = 9
+    OP_FFN = 9,              // fused FFN slice: h[rows] as OP_RMS_UPGATE_SILU, then x2 += Wd[:, rows] h[rows]
+                             //   (streamed as rows of the transposed down-projection, added with atomics)
+    OP_MOE_FFN = 10,         // the same for one routed expert slot, scaled by its router weight
+    OP_COUNT = 11
 };
 
 // Instruction words (int32 each, MK_INSTR_WORDS per instruction).
@@ -67,11 +70,14 @@ MK_HD inline int ctr_lm(int n_layers, int n_kv) { return n_layers * counters_per
 MK_HD inline int n_counters(int n_layers, int n_kv) { return n_layers * counters_per_layer(n_kv) + 1; }
 
 // Weight pointer table: per layer kLayerFixed entries, then gate/up/down per expert.
+// Slot wt_down_t holds the library's transposed copy [ffn][hidden] of w_down
+// (null unless the fused FFN is used).
 enum WSlot : int { WT_ATTN_NORM = 0, WT_Q, WT_K, WT_V, WT_O, WT_FFN_NORM, WT_ROUTER, kLayerFixed };
-MK_HD inline int wt_stride(int n_experts) { return kLayerFixed + 3 * (n_experts > 0 ? n_experts : 1); }
+MK_HD inline int wt_stride(int n_experts) { return kLayerFixed + 4 * (n_experts > 0 ? n_experts : 1); }
 MK_HD inline int wt_gate(int e) { return kLayerFixed + e; }
 MK_HD inline int wt_up(int e, int n_experts) { return kLayerFixed + (n_experts > 0 ? n_experts : 1) + e; }
 MK_HD inline int wt_down(int e, int n_experts) { return kLayerFixed + 2 * (n_experts > 0 ? n_experts : 1) + e; }
+MK_HD inline int wt_down_t(int e, int n_experts) { return kLayerFixed + 3 * (n_experts > 0 ? n_experts : 1) + e; }
 
 // Column parts of a row of width K, and the accumulator sets an op keeps per
 // row (spans x expert slots x column parts); rows per instruction are capped at
@@ -81,7 +87,9 @@ MK_HD inline int acc_sets(int op, int H, int qd, int F, int topk) {
     switch (op) {
         case OP_OPROJ_RES: return kparts_of(qd);
         case OP_RMS_UPGATE_SILU:
-        case OP_MOE_UPGATE: return 2 * kparts_of(H);
+        case OP_MOE_UPGATE:
+        case OP_FFN:
+        case OP_MOE_FFN: return 2 * kparts_of(H);
         case OP_DOWN_RES: return kparts_of(F);
         case OP_MOE_DOWN2_RES: return (topk > 0 ? topk : 1) * kparts_of(F);
         default: return kparts_of(H);
@@ -119,7 +127,8 @@ struct DevParams {
     uint16_t* vcache;
     const float2* rope;      // [max_seq][d/2] (cos, sin)
     // activations (fp32)
-    float* x;          // [H]
+    float* x;          // [H] residual stream read by the FFN (written by O-proj)
+    float* x2;         // [H] residual stream after the FFN (O-proj writes it too; the FFN adds into it)
     float* qkv;        // [(nq + 2 nkv) d]  raw projections, pre-RoPE
     float* attn;       // [nq d]
     float* part_o;     // [nq][kv_splits][d]

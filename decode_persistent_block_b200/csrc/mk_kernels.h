@@ -23,6 +23,10 @@ size_t megakernel_smem_bytes(int ring_stages, int stage_bytes);
 cudaError_t prepare_megakernel(int ring_stages, int stage_bytes, int* max_blocks_per_sm);
 cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, cudaStream_t stream);
 
+// dst[c][r] = src[r][c] for a row-major bf16 matrix of rows x cols (one-time,
+// at set-up: the fused FFN streams the down-projection by its input index).
+cudaError_t launch_transpose_bf16(const uint16_t* src, uint16_t* dst, int rows, int cols, cudaStream_t stream);
+
 int baseline_lm_blocks(const DevParams& p, int n_sm);
 cudaError_t prepare_baseline();
 cudaError_t launch_baseline_set_step(const DevParams& p, StepBuf* sb, int token, int pos, cudaStream_t stream);

@@ -141,7 +141,9 @@ __device__ __forceinline__ int op_rows(const DevParams& p, int op, int sub) {
         case OP_DOWN_RES:
         case OP_MOE_DOWN2_RES: return p.H;
         case OP_RMS_UPGATE_SILU:
-        case OP_MOE_UPGATE: return p.F;
+        case OP_MOE_UPGATE:
+        case OP_FFN:
+        case OP_MOE_FFN: return p.F;
         case OP_LMHEAD_ARGMAX: return p.V;
     }
     return 0;
@@ -151,8 +153,9 @@ __device__ __forceinline__ int op_rows(const DevParams& p, int op, int sub) {
 __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
     const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], e = w[W_END];
     if (op <= OP_NOP || op >= OP_COUNT) return false;
-    const bool moe_op = op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES;
-    if ((p.E > 0) != moe_op && (moe_op || op == OP_RMS_UPGATE_SILU || op == OP_DOWN_RES)) return false;
+    const bool moe_op = op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES || op == OP_MOE_FFN;
+    if ((p.E > 0) != moe_op && (moe_op || op == OP_RMS_UPGATE_SILU || op == OP_DOWN_RES || op == OP_FFN))
+        return false;
     if (op == OP_LMHEAD_ARGMAX ? l != p.L : (l < 0 || l >= p.L)) return false;
     if (w[W_WAIT_CTR] < -1 || w[W_WAIT_CTR] >= p.n_ctr || w[W_SIGNAL_CTR] < -1 || w[W_SIGNAL_CTR] >= p.n_ctr ||
         w[W_AUX_CTR] < -1 || w[W_AUX_CTR] >= p.n_ctr)
@@ -163,7 +166,9 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
         return w[W_AUX_CTR] >= 0 && w[W_SIGNAL_CTR] >= 0 && w[W_AUX_INC] > 0;
     }
     if (op == OP_RMS_QKV && (sub < 0 || sub > 2)) return false;
-    if (op == OP_MOE_UPGATE && (sub < 0 || sub >= p.topk)) return false;
+    if ((op == OP_MOE_UPGATE || op == OP_MOE_FFN) && (sub < 0 || sub >= p.topk)) return false;
+    if (op == OP_FFN && sub != 0) return false;
+    if ((op == OP_FFN || op == OP_MOE_FFN) && (p.H > kMaxPartK || 2 * p.H > p.stage_bytes)) return false;
     if (b < 0 || b >= e || e > op_rows(p, op, sub) || e - b > kMaxRows) return false;
     if ((e - b) * acc_sets(op, p.H, p.nq * p.d, p.F, p.topk) > kRowSlots) return false;
     if (op == OP_LMHEAD_ARGMAX) return w[W_AUX_CTR] >= 0 && w[W_AUX_INC] > 0 && w[W_SEQ] >= 0 && w[W_SEQ] < w[W_AUX_INC];
@@ -186,6 +191,12 @@ struct Plan {
     uint32_t row_bytes;   // bytes of one row part in shared memory
     uint32_t src_stride;  // bytes between consecutive rows in global memory
     const unsigned char* src[kMaxTopK][2];  // [slot][span]: row 0 of the instruction, column 0
+    // fused FFN: after the main stages, `tail_spp` stages of the transposed
+    // down-projection rows (one span, whole rows of tail_row_bytes)
+    int main_stages;
+    int tail_rps, tail_spp;
+    uint32_t tail_row_bytes;
+    const unsigned char* tail_src;
 };
 
 struct AttnRange {
@@ -212,6 +223,10 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
     pl.nspan = 1;
     pl.kparts = 1;
     pl.src[0][1] = pl.src[1][0] = pl.src[1][1] = nullptr;
+    pl.tail_rps = pl.tail_spp = 0;
+    pl.tail_row_bytes = 0;
+    pl.tail_src = nullptr;
+    const uint16_t* tail = nullptr;  // transposed down-projection rows of a fused FFN
     int K = p.H;
     const uint16_t* s0 = nullptr;
     const uint16_t* s1 = nullptr;
@@ -225,7 +240,7 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
             pl.row_bytes = pl.src_stride = (uint32_t)p.d * 2u;
             pl.rps = (int)(SB / (2u * pl.row_bytes));
             pl.spp = (pl.rows + pl.rps - 1) / pl.rps;
-            pl.n_stages = pl.spp;
+            pl.n_stages = pl.main_stages = pl.spp;
             const size_t base = (((size_t)l * p.nkv + sub) * (size_t)p.max_seq + (size_t)r.jb) * (size_t)p.d;
             pl.src[0][0] = (const unsigned char*)(p.kcache + base);
             pl.src[0][1] = (const unsigned char*)(p.vcache + base);
@@ -247,6 +262,18 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
             s0 = wt[wt_down(eidx[0], p.E)];
             if (p.topk > 1) s2 = wt[wt_down(eidx[1], p.E)];
             break;
+        case OP_FFN:
+            pl.nspan = 2;
+            s0 = wt[wt_gate(0)];
+            s1 = wt[wt_up(0, p.E)];
+            tail = wt[wt_down_t(0, p.E)];
+            break;
+        case OP_MOE_FFN:
+            pl.nspan = 2;
+            s0 = wt[wt_gate(eidx[sub])];
+            s1 = wt[wt_up(eidx[sub], p.E)];
+            tail = wt[wt_down_t(eidx[sub], p.E)];
+            break;
     }
     pl.kparts = kparts_of(K);
     pl.nphase = nslot * pl.kparts;
@@ -256,18 +283,36 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
     const int rps = (int)(SB / ((uint32_t)pl.nspan * pl.row_bytes));
     pl.rps = rps < pl.rows ? rps : pl.rows;
     pl.spp = (pl.rows + pl.rps - 1) / pl.rps;
-    pl.n_stages = pl.spp * pl.nphase;
+    pl.n_stages = pl.main_stages = pl.spp * pl.nphase;
+    if (tail) {
+        pl.tail_row_bytes = (uint32_t)p.H * 2u;
+        const int trps = (int)(SB / pl.tail_row_bytes);
+        pl.tail_rps = trps < pl.rows ? trps : pl.rows;
+        pl.tail_spp = (pl.rows + pl.tail_rps - 1) / pl.tail_rps;
+        pl.tail_src = (const unsigned char*)(tail + (size_t)b * p.H);
+        pl.n_stages += pl.tail_spp;
+    }
     pl.src[0][0] = (const unsigned char*)(s0 + (size_t)b * K);
     if (s1) pl.src[0][1] = (const unsigned char*)(s1 + (size_t)b * K);
     if (s2) pl.src[1][0] = (const unsigned char*)(s2 + (size_t)b * K);
 }
 
-__device__ __forceinline__ bool needs_routing(int op) { return op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES; }
+__device__ __forceinline__ bool needs_routing(int op) {
+    return op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES || op == OP_MOE_FFN;
+}
 
 // ---------------------------------------------------------------------------
 // loader warp (one lane)
 // ---------------------------------------------------------------------------
 __device__ void issue_stage(const Plan& pl, int st, unsigned char* dst_stage, uint64_t* bar) {
+    if (st >= pl.main_stages) {  // fused FFN: transposed down-projection rows
+        const int r0 = (st - pl.main_stages) * pl.tail_rps;
+        const int nr = (pl.rows - r0) < pl.tail_rps ? (pl.rows - r0) : pl.tail_rps;
+        const uint32_t bytes = (uint32_t)nr * pl.tail_row_bytes;
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_g2s(dst_stage, pl.tail_src + (size_t)r0 * pl.tail_row_bytes, bytes, bar);
+        return;
+    }
     const int ph = st / pl.spp, sst = st % pl.spp;
     const int slot = ph / pl.kparts, part = ph % pl.kparts;
     const int r0 = sst * pl.rps;
@@ -287,6 +332,12 @@ __device__ void issue_stage(const Plan& pl, int st, unsigned char* dst_stage, ui
 }
 
 __device__ void prefetch_stage(const Plan& pl, int st) {
+    if (st >= pl.main_stages) {
+        const int r0 = (st - pl.main_stages) * pl.tail_rps;
+        const int nr = (pl.rows - r0) < pl.tail_rps ? (pl.rows - r0) : pl.tail_rps;
+        prefetch_l2(pl.tail_src + (size_t)r0 * pl.tail_row_bytes, (uint32_t)nr * pl.tail_row_bytes);
+        return;
+    }
     const int ph = st / pl.spp, sst = st % pl.spp;
     const int slot = ph / pl.kparts, part = ph % pl.kparts;
     const int r0 = sst * pl.rps;
@@ -438,7 +489,7 @@ __device__ __forceinline__ void load_vec(const float* __restrict__ src, int K, f
 // The norm weights are loaded together with x so both round trips overlap.
 template <int J>
 __device__ void load_rms(const DevParams& p, Misc& m, const float* x32, const uint16_t* x16, const uint16_t* nw,
-                         float (&v)[J][8]) {
+                         float (&v)[J][8], float* snap = nullptr) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.H, nch = K >> 3;
     uint4 wraw[J];
 #pragma unroll
@@ -457,6 +508,16 @@ __device__ void load_rms(const DevParams& p, Misc& m, const float* x32, const ui
         } else {
 #pragma unroll
             for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
+        }
+    }
+    if (snap) {  // record the residual stream the op reads (hidden-state snapshot)
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int c = tid + kConsumerThreads * j;
+            if (c < nch) {
+                reinterpret_cast<float4*>(snap)[2 * c] = make_float4(v[j][0], v[j][1], v[j][2], v[j][3]);
+                reinterpret_cast<float4*>(snap)[2 * c + 1] = make_float4(v[j][4], v[j][5], v[j][6], v[j][7]);
+            }
         }
     }
     float ss = 0.f;
@@ -629,17 +690,18 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     const float* vsrc = nullptr;  // fp32 input for OPROJ / DOWN (all column parts)
     switch (op) {
         case OP_RMS_QKV:
-            load_rms<J>(p, m, p.x, l == 0 ? p.embed + (size_t)token * p.H : nullptr, wt[WT_ATTN_NORM], v);
+            // the residual after layer l-1 (x2); one block records it as snapshot l
+            load_rms<J>(p, m, p.x2, l == 0 ? p.embed + (size_t)token * p.H : nullptr, wt[WT_ATTN_NORM], v,
+                        (p.snap && l > 0 && sub == 0 && b == 0) ? p.snap + (size_t)l * p.H : nullptr);
             break;
         case OP_RMS_UPGATE_SILU:
         case OP_MOE_UPGATE:
             load_rms<J>(p, m, p.x, nullptr, wt[WT_FFN_NORM], v);
             break;
         case OP_LMHEAD_ARGMAX:
-            load_rms<J>(p, m, p.x, p.L == 0 ? p.embed + (size_t)token * p.H : nullptr, p.final_norm, v);
-            if (p.L == 0 && p.snap && w[W_SEQ] == 0)  // no layers: the residual stream is the embedding row
-                for (int i = tid; i < p.H; i += kConsumerThreads)
-                    p.snap[i] = __uint_as_float((uint32_t)p.embed[(size_t)token * p.H + i] << 16);
+            // the residual after the last layer (or the embedding row without layers): snapshot L
+            load_rms<J>(p, m, p.x2, p.L == 0 ? p.embed + (size_t)token * p.H : nullptr, p.final_norm, v,
+                        (p.snap && w[W_SEQ] == 0) ? p.snap + (size_t)p.L * p.H : nullptr);
             break;
         case OP_OPROJ_RES:
             K = p.nq * p.d;
@@ -720,9 +782,11 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
                     base = __uint_as_float((uint32_t)e << 16);
                     if (p.snap) p.snap[b + r] = base;
                 } else {
-                    base = __ldcg(p.x + b + r);
+                    base = __ldcg(p.x2 + b + r);
                 }
-                p.x[b + r] = base + acc(0, r);
+                const float nx = base + acc(0, r);
+                p.x[b + r] = nx;   // read by the FFN's RMSNorm
+                p.x2[b + r] = nx;  // the FFN adds its output here
             }
             break;
         case OP_RMS_UPGATE_SILU:
@@ -742,9 +806,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
                     add = m.ew[0] * add;
                     if (p.topk > 1) add += m.ew[1] * acc(1, r);
                 }
-                const float nx = __ldcg(p.x + b + r) + add;
-                p.x[b + r] = nx;
-                if (p.snap) p.snap[(size_t)(l + 1) * p.H + b + r] = nx;
+                p.x2[b + r] = __ldcg(p.x2 + b + r) + add;
             }
             break;
         case OP_LMHEAD_ARGMAX: {
@@ -813,6 +875,165 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     }
     cbar();
     if (tid == 0 && w[W_SIGNAL_CTR] >= 0 && op != OP_LMHEAD_ARGMAX) {
+        __threadfence();
+        atomicAdd(p.counters + w[W_SIGNAL_CTR], 1u);
+    }
+    return true;
+}
+
+// Fused FFN slice (OP_FFN / OP_MOE_FFN).  Rows [b, e) of the up/gate
+// projections give h = silu(Wg xn) * (Wu xn) for this block's rows (MoE: of
+// its routed expert, scaled by the router weight); the block then streams the
+// same rows of the transposed down-projection, Wd^T[b..e) = Wd[:, b..e)^T, and
+// accumulates its column chunks of Wd[:, b..e) h[b..e) in registers, which are
+// added into the post-FFN residual x2 with float4 atomics.  One instruction,
+// one continuous weight stream per block: the up/gate -> down dependency stays
+// inside the block.
+template <int J>
+__device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
+                          uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
+    constexpr int RG = J == 1 ? 8 : J == 2 ? 4 : J == 3 ? 2 : 1;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], rows = w[W_END] - b;
+    const uint32_t SB = (uint32_t)p.stage_bytes;
+    float* part_sums = scratch;  // [2 * rows][8 warps] gate / up row sums, then h[rows]
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * 4 : nullptr;
+
+    if (tid == 0) {
+        if (!wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op)) vstore(&m.abort_flag, 1);
+        if (tr) tr[1] = globaltimer_ns();
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+
+    float v[J][8];
+    const uint16_t* const* wt = p.wt + (size_t)l * wt_stride(p.E);
+    load_rms<J>(p, m, p.x, nullptr, wt[WT_FFN_NORM], v);
+    if (op == OP_MOE_FFN && vload(&m.router_layer) != l)
+        route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
+    int eidx[kMaxTopK];
+    for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
+    Plan pl;
+    make_plan(p, a.pos, w, eidx, pl);
+    const int nch = p.H >> 3;
+
+    // up/gate rows
+    for (int sst = 0; sst < pl.spp; ++sst) {
+        const int r0 = sst * pl.rps;
+        const int nr = (rows - r0) < pl.rps ? (rows - r0) : pl.rps;
+        const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, op);
+        if (tr && tid == 0 && sst == 0) tr[2] = globaltimer_ns();
+        if (ok) {
+            const unsigned char* stage = ring + (size_t)slot * SB;
+            for (int s = 0; s < 2; ++s) {
+                const uint4* Ws = reinterpret_cast<const uint4*>(stage + (size_t)s * pl.rps * pl.row_bytes);
+                stage_rows<J, RG>(Ws, (int)(pl.row_bytes >> 4), nr, nch, v,
+                                  part_sums + ((size_t)s * rows + r0) * kConsumerWarps, lane);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        } else if (tid == 0) {
+            vstore(&m.abort_flag, 1);
+        }
+        if (++slot == p.ring_stages) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+
+    // h = silu(g) * u (times the router weight), then kept at the start of the scratch
+    const float wgt = op == OP_MOE_FFN ? m.ew[sub] : 1.0f;
+    float hv[2] = {0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int r = tid + kConsumerThreads * k;
+        if (r < rows) {
+            const float4* pg = reinterpret_cast<const float4*>(part_sums + (size_t)r * kConsumerWarps);
+            const float4* pu = reinterpret_cast<const float4*>(part_sums + ((size_t)rows + r) * kConsumerWarps);
+            const float4 g0 = pg[0], g1 = pg[1], u0 = pu[0], u1 = pu[1];
+            const float g = ((g0.x + g0.y) + (g0.z + g0.w)) + ((g1.x + g1.y) + (g1.z + g1.w));
+            const float u = ((u0.x + u0.y) + (u0.z + u0.w)) + ((u1.x + u1.y) + (u1.z + u1.w));
+            hv[k] = wgt * (g / (1.0f + expf(-g)) * u);
+        }
+    }
+    cbar();
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int r = tid + kConsumerThreads * k;
+        if (r < rows) scratch[r] = hv[k];
+    }
+    cbar();
+
+    // transposed down-projection rows: this thread's column chunks of Wd[:, rows] h
+    float y[J][8];
+    bool jv[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        jv[j] = tid + kConsumerThreads * j < nch;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) y[j][k] = 0.f;
+    }
+    for (int tst = 0; tst < pl.tail_spp; ++tst) {
+        const int r0 = tst * pl.tail_rps;
+        const int nr = (rows - r0) < pl.tail_rps ? (rows - r0) : pl.tail_rps;
+        const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, op);
+        if (ok) {
+            const uint4* Ws = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
+            constexpr int RQ = J <= 2 ? 4 : 2;  // rows in flight per thread
+            int r = 0;
+            for (; r + RQ <= nr; r += RQ) {
+                uint4 wv[RQ][J];
+#pragma unroll
+                for (int q = 0; q < RQ; ++q)
+#pragma unroll
+                    for (int j = 0; j < J; ++j)
+                        wv[q][j] = jv[j] ? Ws[(r + q) * nch + tid + kConsumerThreads * j] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int q = 0; q < RQ; ++q) {
+                    const float hk = scratch[r0 + r + q];
+#pragma unroll
+                    for (int j = 0; j < J; ++j) {
+                        float f[8];
+                        unpack8(wv[q][j], f);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) y[j][k] = fmaf(f[k], hk, y[j][k]);
+                    }
+                }
+            }
+            for (; r < nr; ++r) {
+                const float hk = scratch[r0 + r];
+#pragma unroll
+                for (int j = 0; j < J; ++j) {
+                    if (!jv[j]) continue;
+                    float f[8];
+                    unpack8(Ws[r * nch + tid + kConsumerThreads * j], f);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) y[j][k] = fmaf(f[k], hk, y[j][k]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        } else if (tid == 0) {
+            vstore(&m.abort_flag, 1);
+        }
+        if (++slot == p.ring_stages) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        if (!jv[j]) continue;
+        float4* dst = reinterpret_cast<float4*>(p.x2) + 2 * (tid + kConsumerThreads * j);
+        atomicAdd(dst, make_float4(y[j][0], y[j][1], y[j][2], y[j][3]));
+        atomicAdd(dst + 1, make_float4(y[j][4], y[j][5], y[j][6], y[j][7]));
+    }
+    cbar();
+    if (tid == 0) {
         __threadfence();
         atomicAdd(p.counters + w[W_SIGNAL_CTR], 1u);
     }
@@ -1078,6 +1299,15 @@ __device__ bool gemv_dispatch(const DevParams& p, const StepArgs& a, const int32
     const int K = gemv_k(p, w[W_OP]);
     const int kp = K / kparts_of(K);
     const int J = ((kp >> 3) + kConsumerThreads - 1) / kConsumerThreads;
+    if (w[W_OP] == OP_FFN || w[W_OP] == OP_MOE_FFN) {
+        switch (J) {
+            case 1: return ffn_instr<1>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 2: return ffn_instr<2>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 3: return ffn_instr<3>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 4: return ffn_instr<4>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+        }
+        return false;
+    }
     switch (J) {
         case 1: return gemv_instr<1>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
         case 2: return gemv_instr<2>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
@@ -1115,6 +1345,12 @@ __device__ void prefetch_instr(const DevParams& p, const StepArgs& a, const int3
                 prefetch_line_l2(base + off);
             done += bytes;
         }
+    if (pl.tail_src) {
+        size_t bytes = (size_t)pl.rows * pl.tail_row_bytes;
+        if (done + bytes > cap) bytes = cap > done ? cap - done : 0;
+        for (size_t off = (size_t)threadIdx.x * 128; off < bytes; off += (size_t)kConsumerThreads * 128)
+            prefetch_line_l2(pl.tail_src + off);
+    }
 }
 
 // ---------------------------------------------------------------------------

@@ -12,6 +12,7 @@
 
 #include "mk_device.cuh"
 #include "mk_internal.h"
+#include "mk_kernels.h"
 
 namespace mk {
 namespace {
@@ -258,3 +259,31 @@ extern "C" int mk_attention_decode_noalloc(const float* q, const void* k_cache, 
     a.out = out;
     return mk::launch_attn(a, head_dim, static_cast<cudaStream_t>(stream));
 }
+
+// ---------------------------------------------------------------------------
+// Set-up: bf16 transpose through a 32 x 33 shared tile (coalesced on both sides).
+namespace mk {
+namespace {
+__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, int rows,
+                                      int cols) {
+    __shared__ uint16_t tile[32][33];
+    const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int r = r0 + i, c = c0 + threadIdx.x;
+        if (r < rows && c < cols) tile[i][threadIdx.x] = src[(size_t)r * cols + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int c = c0 + i, r = r0 + threadIdx.x;
+        if (r < rows && c < cols) dst[(size_t)c * rows + r] = tile[threadIdx.x][i];
+    }
+}
+}  // namespace
+
+cudaError_t launch_transpose_bf16(const uint16_t* src, uint16_t* dst, int rows, int cols, cudaStream_t stream) {
+    if (rows <= 0 || cols <= 0) return cudaSuccess;
+    const dim3 grid((unsigned)((cols + 31) / 32), (unsigned)((rows + 31) / 32));
+    transpose_bf16_kernel<<<grid, dim3(32, 8), 0, stream>>>(src, dst, rows, cols);
+    return cudaGetLastError();
+}
+}  // namespace mk

@@ -12,6 +12,7 @@ struct Planned {
     int max_instr = 0;
     int kv_splits = 1;
     int n_lm = 0;                  // LM-head instructions (partial argmax slots)
+    bool fused_ffn = true;         // one OP_FFN / OP_MOE_FFN per layer instead of up/gate + down
     std::vector<int32_t> words;    // [n_sm][max_instr][W_NWORDS]
     std::vector<int32_t> n_instr;  // [n_sm]
     std::vector<uint32_t> ctr_inc; // per-step increment of every counter
@@ -21,6 +22,10 @@ int check_config(const mk_config& c);
 int check_options(const mk_config& c, const mk_options& o);
 void fill_defaults(mk_options* o);
 int default_kv_splits(const mk_config& c, int n_sm);
+// Whether the schedule fuses each layer's FFN into one instruction per block:
+// asked for (split_ffn == 0), the up/gate rows need no column parts, and one
+// transposed down-projection row (hidden bf16 values) fits a ring stage.
+bool ffn_fused(const mk_config& c, const mk_options& o);
 int plan_schedule(const mk_config& c, const mk_options& o, int n_sm, Planned* out);
 int validate(const mk_config& c, const Planned& p);
 int simulate(const int32_t* words, int n_sm, int max_instr, const int32_t* n_instr, const uint32_t* ctr_inc,

@@ -46,22 +46,49 @@ struct Segment {
     int rows;
 };
 
-// Split the virtual concatenation of `segs` into one contiguous range per SM,
-// cut at segment boundaries and at `cap` rows.  Calls emit(sm, sub, begin, end).
+// Split the rows of `segs` (e.g. the q, k and v row blocks) over n_sm blocks
+// so that every block gets rows of ONE segment only: blocks are given to the
+// segments in proportion to their rows (largest remainder, at least one each
+// when there are enough blocks), then each segment's rows are split evenly
+// over its blocks and cut at `cap` rows.  A block holding rows of two segments
+// would run two instructions back to back and finish last, delaying every
+// block that waits for the op.  With fewer blocks than segments the virtual
+// concatenation is split instead.  Calls emit(sm, sub, begin, end).
 template <class F>
 void split_rows(const std::vector<Segment>& segs, int n_sm, int cap, F emit) {
     long long total = 0;
     for (auto& s : segs) total += s.rows;
-    for (int sm = 0; sm < n_sm; ++sm) {
-        long long a = total * sm / n_sm, b = total * (sm + 1) / n_sm;
-        long long base = 0;
-        for (auto& s : segs) {
-            long long lo = std::max(a, base), hi = std::min(b, base + s.rows);
-            for (long long r = lo; r < hi; r += cap) {
-                long long e = std::min(hi, r + cap);
-                emit(sm, s.sub, (int)(r - base), (int)(e - base));
+    const int ns = (int)segs.size();
+    if (n_sm < ns || ns == 1) {
+        for (int sm = 0; sm < n_sm; ++sm) {
+            long long a = total * sm / n_sm, b = total * (sm + 1) / n_sm;
+            long long base = 0;
+            for (auto& s : segs) {
+                long long lo = std::max(a, base), hi = std::min(b, base + s.rows);
+                for (long long r = lo; r < hi; r += cap) emit(sm, s.sub, (int)(r - base), (int)(std::min(hi, r + cap) - base));
+                base += s.rows;
             }
-            base += s.rows;
+        }
+        return;
+    }
+    std::vector<int> blocks(ns, 1);
+    int left = n_sm - ns;
+    std::vector<std::pair<double, int>> rem;
+    for (int i = 0; i < ns; ++i) {
+        const double share = (double)segs[i].rows * n_sm / (double)total - 1.0;
+        const int extra = std::max(0, std::min(left, (int)share));
+        blocks[i] += extra;
+        left -= extra;
+        rem.push_back({share - extra, i});
+    }
+    std::sort(rem.begin(), rem.end(), [](auto& x, auto& y) { return x.first > y.first || (x.first == y.first && x.second < y.second); });
+    for (int k = 0; left > 0; k = (k + 1) % ns, --left) blocks[rem[k].second]++;
+    int sm = 0;
+    for (int i = 0; i < ns; ++i) {
+        const long long R = segs[i].rows;
+        for (int k = 0; k < blocks[i]; ++k, ++sm) {
+            const long long a = R * k / blocks[i], b = R * (k + 1) / blocks[i];
+            for (long long r = a; r < b; r += cap) emit(sm, segs[i].sub, (int)r, (int)std::min(b, r + cap));
         }
     }
 }
@@ -125,6 +152,12 @@ int check_options(const mk_config& c, const mk_options& o) {
     return MK_OK;
 }
 
+bool ffn_fused(const mk_config& c, const mk_options& o_in) {
+    mk_options o = o_in;
+    fill_defaults(&o);
+    return o.split_ffn == 0 && c.hidden <= kMaxPartK && 2LL * c.hidden <= (long long)o.stage_bytes;
+}
+
 int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned* out) {
     int rc = check_config(c);
     if (rc) return rc;
@@ -135,6 +168,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     const int S = o.kv_splits > 0 ? o.kv_splits : default_kv_splits(c, n_sm);
     const int cap = o.rows_per_instr;
     const bool moe = c.n_experts > 0;
+    const bool fused = ffn_fused(c, o);
 
     std::vector<std::vector<Instr>> q(n_sm);
     std::vector<uint32_t> inc(n_counters(L, nkv), 0);
@@ -181,12 +215,15 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
         }
         inc[ctr_id(l, C_ATTN, nkv)] = nkv;  // one signal per kv head, by its last-arriving split
         gemv_op(OP_OPROJ_RES, l, {{0, H}}, ctr_id(l, C_ATTN, nkv), ctr_id(l, C_OPROJ, nkv));
-        if (!moe) {
-            gemv_op(OP_RMS_UPGATE_SILU, l, {{0, F}}, ctr_id(l, C_OPROJ, nkv), ctr_id(l, C_FFN1, nkv));
+        std::vector<Segment> slots;
+        for (int s = 0; s < (moe ? c.top_k : 1); ++s) slots.push_back({s, F});
+        if (fused) {
+            // one instruction per block: its up/gate rows, then the matching down-projection columns
+            gemv_op(moe ? OP_MOE_FFN : OP_FFN, l, slots, ctr_id(l, C_OPROJ, nkv), ctr_id(l, C_FFN2, nkv));
+        } else if (!moe) {
+            gemv_op(OP_RMS_UPGATE_SILU, l, slots, ctr_id(l, C_OPROJ, nkv), ctr_id(l, C_FFN1, nkv));
             gemv_op(OP_DOWN_RES, l, {{0, H}}, ctr_id(l, C_FFN1, nkv), ctr_id(l, C_FFN2, nkv));
         } else {
-            std::vector<Segment> slots;
-            for (int s = 0; s < c.top_k; ++s) slots.push_back({s, F});
             gemv_op(OP_MOE_UPGATE, l, slots, ctr_id(l, C_OPROJ, nkv), ctr_id(l, C_FFN1, nkv));
             gemv_op(OP_MOE_DOWN2_RES, l, {{0, H}}, ctr_id(l, C_FFN1, nkv), ctr_id(l, C_FFN2, nkv));
         }
@@ -220,6 +257,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     out->max_instr = max_instr;
     out->kv_splits = S;
     out->n_lm = (int)inc[ctr_lm(L, nkv)];
+    out->fused_ffn = fused;
     out->words.assign((size_t)n_sm * max_instr * W_NWORDS, 0);
     out->n_instr.assign(n_sm, 0);
     for (int sm = 0; sm < n_sm; ++sm) {
@@ -240,7 +278,9 @@ static int op_index(const int32_t* w) {
         case OP_ATTN: slot = 1; break;
         case OP_OPROJ_RES: slot = 2; break;
         case OP_RMS_UPGATE_SILU:
-        case OP_MOE_UPGATE: slot = 3; break;
+        case OP_MOE_UPGATE:
+        case OP_FFN:
+        case OP_MOE_FFN: slot = 3; break;
         case OP_DOWN_RES:
         case OP_MOE_DOWN2_RES: slot = 4; break;
         case OP_LMHEAD_ARGMAX: slot = 0; break;
@@ -277,7 +317,7 @@ int validate(const mk_config& c, const Planned& p) {
         switch (op) {
             case OP_RMS_QKV: return sub == 0 ? c.n_q_heads * d : nkv * d;
             case OP_OPROJ_RES: case OP_DOWN_RES: case OP_MOE_DOWN2_RES: return c.hidden;
-            case OP_RMS_UPGATE_SILU: case OP_MOE_UPGATE: return c.ffn;
+            case OP_RMS_UPGATE_SILU: case OP_MOE_UPGATE: case OP_FFN: case OP_MOE_FFN: return c.ffn;
             case OP_LMHEAD_ARGMAX: return c.vocab;
         }
         return -1;
@@ -293,9 +333,10 @@ int validate(const mk_config& c, const Planned& p) {
             const int32_t* w = &p.words[((size_t)sm * p.max_instr + i) * W_NWORDS];
             const int op = w[W_OP], l = w[W_LAYER];
             if (op <= OP_NOP || op >= OP_COUNT) return MK_ERR_SCHEDULE;
-            if (moe != (op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES) &&
-                (op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES || op == OP_RMS_UPGATE_SILU || op == OP_DOWN_RES))
-                return MK_ERR_SCHEDULE;
+            const bool moe_op = op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES || op == OP_MOE_FFN;
+            const bool ffn_op = moe_op || op == OP_RMS_UPGATE_SILU || op == OP_DOWN_RES || op == OP_FFN;
+            if (ffn_op && moe != moe_op) return MK_ERR_SCHEDULE;
+            if (ffn_op && p.fused_ffn != (op == OP_FFN || op == OP_MOE_FFN)) return MK_ERR_SCHEDULE;
             if (op == OP_LMHEAD_ARGMAX ? l != L : (l < 0 || l >= L)) return MK_ERR_SCHEDULE;
             const int oi = op_index(w);
             if (oi < last_op) return MK_ERR_SCHEDULE;  // queue sorted by global op order
@@ -324,8 +365,8 @@ int validate(const mk_config& c, const Planned& p) {
             const int sub = w[W_SUB];
             const int R = rows_of(op, op == OP_RMS_QKV ? sub : 0);
             if (op == OP_RMS_QKV && (sub < 0 || sub > 2)) return MK_ERR_SCHEDULE;
-            if (op == OP_MOE_UPGATE && (sub < 0 || sub >= c.top_k)) return MK_ERR_SCHEDULE;
-            if (op != OP_RMS_QKV && op != OP_MOE_UPGATE && sub != 0) return MK_ERR_SCHEDULE;
+            if ((op == OP_MOE_UPGATE || op == OP_MOE_FFN) && (sub < 0 || sub >= c.top_k)) return MK_ERR_SCHEDULE;
+            if (op != OP_RMS_QKV && op != OP_MOE_UPGATE && op != OP_MOE_FFN && sub != 0) return MK_ERR_SCHEDULE;
             const int b = w[W_BEGIN], e = w[W_END];
             const int sets = acc_sets(op, c.hidden, c.n_q_heads * d, c.ffn, c.top_k);
             if (b < 0 || e > R || b >= e || e - b > kMaxRows || (e - b) * sets > kRowSlots) return MK_ERR_SCHEDULE;
@@ -355,9 +396,15 @@ int validate(const mk_config& c, const Planned& p) {
         for (int g = 0; g < nkv; ++g)
             for (int s = 0; s < p.kv_splits; ++s)
                 if (attn_seen[(size_t)l * nkv + g][s] != 1) return MK_ERR_SCHEDULE;
-        for (int op : {OP_RMS_QKV, OP_OPROJ_RES, moe ? OP_MOE_UPGATE : OP_RMS_UPGATE_SILU,
-                       moe ? OP_MOE_DOWN2_RES : OP_DOWN_RES})
+        const std::vector<int> need = p.fused_ffn
+            ? std::vector<int>{OP_RMS_QKV, OP_OPROJ_RES, moe ? OP_MOE_FFN : OP_FFN}
+            : std::vector<int>{OP_RMS_QKV, OP_OPROJ_RES, moe ? OP_MOE_UPGATE : OP_RMS_UPGATE_SILU,
+                               moe ? OP_MOE_DOWN2_RES : OP_DOWN_RES};
+        for (int op : need)
             if (cov[cov_key(l, op, 0)].empty()) return MK_ERR_SCHEDULE;
+        if (moe)  // every routed slot's rows are covered
+            for (int sl = 1; sl < c.top_k; ++sl)
+                if (cov[cov_key(l, p.fused_ffn ? OP_MOE_FFN : OP_MOE_UPGATE, sl)].empty()) return MK_ERR_SCHEDULE;
         signals[ctr_id(l, C_ATTN, nkv)] = nkv;  // emitted by the merging split of each head group
     }
     if (cov[cov_key(L, OP_LMHEAD_ARGMAX, 0)].empty()) return MK_ERR_SCHEDULE;

@@ -110,6 +110,12 @@ typedef struct {
     int prefetch_ahead;   /* consumers prefetch into L2 the weights of the instruction this many
                              places ahead in their queue (-1 default, 0 = off) */
     int prefetch_max_bytes; /* cap on the bytes prefetched per instruction (0 = default 1 MiB) */
+    int split_ffn;        /* 0 (default): each layer's FFN is one fused instruction per SM (up/gate rows,
+                             then the matching columns of w_down, streamed from a transposed copy the
+                             library keeps, added into the residual with atomics: fp32 summation order
+                             varies between runs); 1: separate up/gate and down instructions, no copy,
+                             bitwise reproducible.  The split form is also used whenever hidden > 8192
+                             or 2 * hidden > stage_bytes */
 } mk_options;
 
 /* Device status block, copied out by mk_get_status.  On a device-side error

@@ -14,7 +14,7 @@ import decode_persistent_block_b200 as dpb
 from decode_persistent_block_b200 import mk
 from synth import configs
 
-OP = dict(RMS_QKV=1, ATTN=2, OPROJ=3, UG=4, DOWN=5, LM=6, MOE_UG=7, MOE_DOWN=8)
+OP = dict(RMS_QKV=1, ATTN=2, OPROJ=3, UG=4, DOWN=5, LM=6, MOE_UG=7, MOE_DOWN=8, FFN=9, MOE_FFN=10)
 W_OP, W_LAYER, W_SUB, W_BEGIN, W_END, W_WAIT, W_WINC, W_SIG, W_AUX, W_AINC, W_SEQ = range(11)
 
 CFGS = [configs.TINY, configs.LLAMA_1B, configs.LLAMA_3B, configs.MIXTRAL_8L, configs.llama1b_sweep(16384),
@@ -38,16 +38,18 @@ def n_ctr_per_layer(cfg):
     return 5 + cfg.n_kv_heads
 
 
+@pytest.mark.parametrize("split_ffn", [0, 1], ids=["fused_ffn", "split_ffn"])
 @pytest.mark.parametrize("cfg", CFGS, ids=lambda c: c.name)
 @pytest.mark.parametrize("n_sm", [148, 37, 1])
-def test_plan_covers_rows_and_counts_signals(cfg, n_sm):
-    words, n_instr, inc = dpb.plan(cfg, n_sm)
+def test_plan_covers_rows_and_counts_signals(cfg, n_sm, split_ffn):
+    words, n_instr, inc = dpb.plan(cfg, n_sm, split_ffn=split_ffn)
     L, nkv, d = cfg.n_layers, cfg.n_kv_heads, cfg.head_dim
     per = n_ctr_per_layer(cfg)
     assert inc.size == L * per + 1
     rows = {OP["RMS_QKV"]: {0: cfg.n_heads * d, 1: nkv * d, 2: nkv * d}, OP["OPROJ"]: {0: cfg.hidden},
             OP["UG"]: {0: cfg.ffn}, OP["DOWN"]: {0: cfg.hidden}, OP["LM"]: {0: cfg.vocab},
-            OP["MOE_UG"]: {s: cfg.ffn for s in range(max(cfg.top_k, 1))}, OP["MOE_DOWN"]: {0: cfg.hidden}}
+            OP["MOE_UG"]: {s: cfg.ffn for s in range(max(cfg.top_k, 1))}, OP["MOE_DOWN"]: {0: cfg.hidden},
+            OP["FFN"]: {0: cfg.ffn}, OP["MOE_FFN"]: {s: cfg.ffn for s in range(max(cfg.top_k, 1))}}
     cover = {}
     signals = np.zeros_like(inc)
     splits = None
@@ -70,7 +72,12 @@ def test_plan_covers_rows_and_counts_signals(cfg, n_sm):
     for key, hit in cover.items():
         assert np.all(hit == 1), key
     moe = cfg.n_experts > 0
-    ffn_ops = (OP["MOE_UG"], OP["MOE_DOWN"]) if moe else (OP["UG"], OP["DOWN"])
+    if split_ffn:
+        ffn_ops = (OP["MOE_UG"], OP["MOE_DOWN"]) if moe else (OP["UG"], OP["DOWN"])
+    else:
+        ffn_ops = (OP["MOE_FFN"],) if moe else (OP["FFN"],)
+        for l in range(L):  # the fused FFN signals the post-FFN counter; the mid-FFN one is unused
+            assert inc[l * per + 3] == 0
     for l in range(L):
         for op in (OP["RMS_QKV"], OP["OPROJ"]) + ffn_ops:
             assert (l, op, 0) in cover
@@ -89,28 +96,37 @@ def _ranges(total, n_sm):
     return [(total * s // n_sm, total * (s + 1) // n_sm) for s in range(n_sm)]
 
 
+@pytest.mark.parametrize("split_ffn", [0, 1], ids=["fused_ffn", "split_ffn"])
 @pytest.mark.parametrize("n_sm", [148, 132, 64])
-def test_increment_closed_forms_llama1b(n_sm):
+def test_increment_closed_forms_llama1b(n_sm, split_ffn):
     cfg = configs.LLAMA_1B
-    words, n_instr, inc = dpb.plan(cfg, n_sm)
+    words, n_instr, inc = dpb.plan(cfg, n_sm, split_ffn=split_ffn)
     per = n_ctr_per_layer(cfg)
-    # QKV: one instruction per block range, plus one for every q/k/v boundary strictly inside a range
-    qkv_rows = cfg.qkv_rows
-    bounds = [cfg.n_heads * cfg.head_dim, (cfg.n_heads + cfg.n_kv_heads) * cfg.head_dim]
-    n_qkv = sum(1 for a, b in _ranges(qkv_rows, n_sm) if b > a) + \
-        sum(1 for a, b in _ranges(qkv_rows, n_sm) for x in bounds if a < x < b)
     lm = sum(-(-(b - a) // 1024) for a, b in _ranges(cfg.vocab, n_sm))
     for l in range(cfg.n_layers):
-        assert inc[l * per + 0] == n_qkv
+        assert inc[l * per + 0] == n_sm      # QKV: every block holds rows of exactly one of q, k, v
         assert inc[l * per + 2] == n_sm      # O-proj: hidden >= n_sm rows, <= 1024 per block
-        assert inc[l * per + 3] == n_sm      # up/gate
-        assert inc[l * per + 4] == n_sm      # down
+        assert inc[l * per + 3] == (n_sm if split_ffn else 0)  # up/gate (split FFN only)
+        assert inc[l * per + 4] == n_sm      # down, or the fused FFN slice
     assert inc[-1] == lm
     # every block's queue is sorted by (layer, op slot)
-    order = {OP["RMS_QKV"]: 0, OP["ATTN"]: 1, OP["OPROJ"]: 2, OP["UG"]: 3, OP["DOWN"]: 4, OP["LM"]: 0}
+    order = {OP["RMS_QKV"]: 0, OP["ATTN"]: 1, OP["OPROJ"]: 2, OP["UG"]: 3, OP["FFN"]: 3, OP["DOWN"]: 4,
+             OP["LM"]: 0}
     for sm in range(n_sm):
         keys = [int(w[W_LAYER]) * 5 + order[int(w[W_OP])] for w in words[sm, :n_instr[sm]]]
         assert keys == sorted(keys)
+
+
+@pytest.mark.parametrize("cfg", [configs.LLAMA_1B, configs.LLAMA_3B, configs.MIXTRAL_8L], ids=lambda c: c.name)
+def test_segments_get_blocks_in_proportion_to_rows(cfg):
+    # QKV (and the MoE expert slots): blocks are shared out by rows, so the
+    # largest per-block row count stays within one row of the even split.
+    n_sm = 148
+    words, n_instr, _ = dpb.plan(cfg, n_sm)
+    op = OP["RMS_QKV"]
+    rows = [int(w[W_END] - w[W_BEGIN]) for _, _, w in instrs(words, n_instr) if w[W_OP] == op and w[W_LAYER] == 0]
+    assert len(rows) == n_sm
+    assert max(rows) <= -(-cfg.qkv_rows // n_sm) + 1
 
 
 def test_plan_is_deterministic():
@@ -120,9 +136,10 @@ def test_plan_is_deterministic():
         assert np.array_equal(x, y)
 
 
+@pytest.mark.parametrize("split_ffn", [0, 1], ids=["fused_ffn", "split_ffn"])
 @pytest.mark.parametrize("cfg", CFGS, ids=lambda c: c.name)
-def test_simulated_interleavings_complete_and_counters_match(cfg):
-    words, n_instr, inc = dpb.plan(cfg, 148 if cfg.hidden > 256 else 23)
+def test_simulated_interleavings_complete_and_counters_match(cfg, split_ffn):
+    words, n_instr, inc = dpb.plan(cfg, 148 if cfg.hidden > 256 else 23, split_ffn=split_ffn)
     for seed in range(3):
         rc, done = dpb.simulate(words, n_instr, inc, steps=3, seed=seed)
         assert rc == mk.MK_OK
@@ -131,7 +148,7 @@ def test_simulated_interleavings_complete_and_counters_match(cfg):
 
 def test_simulator_detects_deadlock_and_count_mismatch():
     cfg = configs.TINY
-    words, n_instr, inc = dpb.plan(cfg, 4)
+    words, n_instr, inc = dpb.plan(cfg, 4, split_ffn=1)
     # move block 0's first layer-1 QKV in front of its layer-0 down-projection
     q = words[0, :n_instr[0]].copy()
     i_down = next(i for i, w in enumerate(q) if w[W_OP] == OP["DOWN"] and w[W_LAYER] == 0)
@@ -173,3 +190,11 @@ def test_rows_per_instr_cap_splits_instructions():
     for _, _, w in instrs(words, n_instr):
         if w[W_OP] != OP["ATTN"]:
             assert w[W_END] - w[W_BEGIN] <= 64
+
+
+def test_fused_ffn_is_the_default_for_every_supported_hidden_size():
+    # hidden <= 8192 and a stage holds a whole hidden row: the fused form always applies
+    ops = lambda cfg, **kw: {int(w[W_OP]) for _, _, w in instrs(*dpb.plan(cfg, 148, **kw)[:2])}
+    for cfg in (configs.LLAMA_3B, configs.TINY.with_(hidden=8192)):
+        assert OP["FFN"] in ops(cfg) and OP["UG"] not in ops(cfg)
+        assert OP["FFN"] not in ops(cfg, split_ffn=1) and {OP["UG"], OP["DOWN"]} <= ops(cfg, split_ffn=1)
