@@ -194,7 +194,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     std::memset(&p, 0, sizeof(p));
     p.L = L; p.H = H; p.nq = nq; p.nkv = nkv; p.d = d; p.F = c.ffn; p.V = c.vocab; p.E = E;
     p.topk = E > 0 ? c.top_k : 0; p.max_seq = c.max_seq; p.eps = c.rms_eps; p.kv_splits = S;
-    p.n_ctr = mk::n_counters(L, nkv);
+    p.n_ctr = mk::n_counters(L);
     p.embed = static_cast<const uint16_t*>(w->embed);
     p.lm_head = static_cast<const uint16_t*>(w->lm_head);
     p.final_norm = static_cast<const uint16_t*>(w->final_norm);
@@ -319,7 +319,7 @@ int mk_build_schedule(mk_handle* h) {
     h->p.max_instr = plan.max_instr;
     if (h->opt.trace) {
         unsigned long long* tr = nullptr;
-        if ((rc = dalloc(h, &tr, (size_t)plan.n_sm * plan.max_instr * 4))) return rc;
+        if ((rc = dalloc(h, &tr, (size_t)plan.n_sm * plan.max_instr * mk::kTraceWords))) return rc;
         h->p.trace = tr;
     }
     if ((rc = upload_schedule(h))) return rc;
@@ -448,7 +448,7 @@ int mk_get_status(mk_handle* h, mk_status* out) {
 
 int mk_get_trace(mk_handle* h, uint64_t* out, size_t cap, size_t* n) {
     if (!h || !h->p.trace) return MK_ERR_INVALID_ARG;
-    const size_t cnt = (size_t)h->plan.n_sm * h->plan.max_instr * 4;
+    const size_t cnt = (size_t)h->plan.n_sm * h->plan.max_instr * mk::kTraceWords;
     if (n) *n = cnt;
     if (!out) return MK_OK;
     if (cap < cnt) return MK_ERR_CAPACITY;
@@ -462,7 +462,7 @@ int mk_reset(mk_handle* h) {
     CK(cudaStreamSynchronize(h->stream));
     CK(cudaMemset(h->p.counters, 0, sizeof(uint32_t) * h->p.n_ctr));
     CK(cudaMemset(h->p.status, 0, sizeof(mk::DevStatus)));
-    if (h->p.trace) CK(cudaMemset(h->p.trace, 0, sizeof(uint64_t) * h->plan.n_sm * h->plan.max_instr * 4));
+    if (h->p.trace) CK(cudaMemset(h->p.trace, 0, sizeof(uint64_t) * h->plan.n_sm * h->plan.max_instr * mk::kTraceWords));
     h->epoch = 0;
     if (h->scheduled) return upload_schedule(h);
     return MK_OK;

@@ -89,6 +89,22 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+// Publish one arrival on a dependency counter: the fence orders every write
+// this block made before the preceding block barrier (cumulatively, at gpu
+// scope) ahead of the increment, which itself needs no ordering.
+__device__ __forceinline__ void signal_release(uint32_t* ctr) {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+// Arrival that also returns the previous count (last-arriver detection); the
+// caller fences again (acquire) before reading what the other arrivals wrote.
+__device__ __forceinline__ uint32_t arrive_release(uint32_t* ctr) {
+    uint32_t old;
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(ctr) : "memory");
+    return old;
+}
+__device__ __forceinline__ void fence_acquire() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ int ld_relaxed_s32(const int* p) {
     int v;
     asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

@@ -61,13 +61,20 @@ constexpr int kThreads = kConsumerThreads + 32;  // + one loader warp
 constexpr int kMaxGroup = 4;         // query heads per kv head
 constexpr int kMaxHeadDim = 128;
 constexpr int kMaxTopK = 2;
+constexpr int kMaxMergeSlots = 2048;  // query heads x kv splits merged in the O-projection prologue
 
-// Counter ids: per layer [QKV, ATTN_DONE, OPROJ, FFN1, FFN2, GROUP_0..GROUP_{nkv-1}], then LM.
-enum CtrSlot : int { C_QKV = 0, C_ATTN = 1, C_OPROJ = 2, C_FFN1 = 3, C_FFN2 = 4, C_GROUP0 = 5 };
-MK_HD inline int counters_per_layer(int n_kv) { return C_GROUP0 + n_kv; }
-MK_HD inline int ctr_id(int layer, int slot, int n_kv) { return layer * counters_per_layer(n_kv) + slot; }
-MK_HD inline int ctr_lm(int n_layers, int n_kv) { return n_layers * counters_per_layer(n_kv); }
-MK_HD inline int n_counters(int n_layers, int n_kv) { return n_layers * counters_per_layer(n_kv) + 1; }
+// Counter ids: per layer [QKV, ATTN (one signal per split), OPROJ, FFN1, FFN2], then the LM head's
+// arrival counter.
+enum CtrSlot : int { C_QKV = 0, C_ATTN = 1, C_OPROJ = 2, C_FFN1 = 3, C_FFN2 = 4, kCountersPerLayer = 5 };
+MK_HD inline int ctr_id(int layer, int slot) { return layer * kCountersPerLayer + slot; }
+MK_HD inline int ctr_lm(int n_layers) { return n_layers * kCountersPerLayer; }
+MK_HD inline int n_counters(int n_layers) { return n_layers * kCountersPerLayer + 1; }
+
+// Trace record of one instruction (options.trace): globaltimer stamps in ns,
+// zero where not reached.  Consumer side: reached, dependency satisfied,
+// input vector ready, first stage full, main stages consumed, signalled.
+// Loader side: first and last stage issued.
+enum TraceStamp : int { T_START = 0, T_DEP, T_READY, T_FIRST, T_MAIN, T_END, T_LD_FIRST, T_LD_LAST, kTraceWords };
 
 // Weight pointer table: per layer kLayerFixed entries, then gate/up/down per expert.
 // Slot wt_down_t holds the library's transposed copy [ffn][hidden] of w_down

@@ -163,7 +163,7 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
     if (w[W_WAIT_CTR] >= 0 && w[W_WAIT_INC] <= 0) return false;
     if (op == OP_ATTN) {
         if (sub < 0 || sub >= p.nkv || e != p.kv_splits || b < 0 || b >= e) return false;
-        return w[W_AUX_CTR] >= 0 && w[W_SIGNAL_CTR] >= 0 && w[W_AUX_INC] > 0;
+        return w[W_SIGNAL_CTR] >= 0;
     }
     if (op == OP_RMS_QKV && (sub < 0 || sub > 2)) return false;
     if ((op == OP_MOE_UPGATE || op == OP_MOE_FFN) && (sub < 0 || sub >= p.topk)) return false;
@@ -297,6 +297,19 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
     if (s2) pl.src[1][0] = (const unsigned char*)(s2 + (size_t)b * K);
 }
 
+// Pull this instruction's row of the weight-pointer table into L1 (one line
+// per thread of the first warp), so that make_plan's loads hit.
+__device__ __forceinline__ void prefetch_plan_l1(const DevParams& p, const int32_t* w) {
+    const int l = w[W_LAYER];
+    if (threadIdx.x >= 32 || l >= p.L) return;
+    const int stride = wt_stride(p.E);
+    const char* row = reinterpret_cast<const char*>(p.wt + (size_t)l * stride);
+    const int bytes = stride * (int)sizeof(void*);
+    const int lines = (bytes + 127) / 128 + 1;  // the row may start mid-line
+    const int off = 128 * (int)threadIdx.x < bytes ? 128 * (int)threadIdx.x : bytes - 1;
+    if ((int)threadIdx.x < lines) asm volatile("prefetch.global.L1 [%0];" ::"l"(row + off));
+}
+
 __device__ __forceinline__ bool needs_routing(int op) {
     return op == OP_MOE_UPGATE || op == OP_MOE_DOWN2_RES || op == OP_MOE_FFN;
 }
@@ -408,12 +421,15 @@ __device__ void loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
         Plan pl;
         if (!loader_plan(p, a, w, m, pl, true, i)) break;
         bool ok = true;
+        unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + i) * kTraceWords : nullptr;
         for (int st = 0; st < pl.n_stages; ++st, ++g) {
             if (!wait_mbar(&empty[slot], phase ^ 1u, p, m, i, w[W_OP])) {
                 ok = false;
                 break;
             }
             issue_stage(pl, st, ring + (size_t)slot * SB, &full[slot]);
+            if (tr && st == 0) tr[T_LD_FIRST] = globaltimer_ns();
+            if (tr && st == pl.n_stages - 1) tr[T_LD_LAST] = globaltimer_ns();
             used |= 1u << slot;
             last_parity = (last_parity & ~(1u << slot)) | (phase << slot);
             if (++slot == NS) {
@@ -482,6 +498,73 @@ __device__ __forceinline__ void load_vec(const float* __restrict__ src, int K, f
 #pragma unroll
             for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
         }
+    }
+}
+
+// Input of the O-projection, columns [col0, col0 + K): the attention output of
+// every query head, merged here from its kv splits' partials (unnormalised
+// o_s, running max m_s in the log2 domain, sum l_s):
+//   attn = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s,
+// taken B splits per round trip with an online rescale, in split order.
+template <int J>
+__device__ __forceinline__ void load_attn_merged(const DevParams& p, int col0, int K, float (&v)[J][8]) {
+    constexpr int B = 4;
+    const int tid = threadIdx.x, nch = K >> 3, S = p.kv_splits, D = p.d;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int c = tid + kConsumerThreads * j;
+        if (c >= nch) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
+            continue;
+        }
+        const int col = col0 + 8 * c, h = col / D, dc = col - h * D;
+        const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)h * S;
+        const float4* po = reinterpret_cast<const float4*>(p.part_o + (size_t)h * S * D + dc);
+        const int D4 = D >> 2;
+        float M = -CUDART_INF_F, den = 0.f, acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+        for (int s0 = 0; s0 < S; s0 += B) {
+            float2 t[B];
+            float4 o0[B], o1[B];
+#pragma unroll
+            for (int k = 0; k < B; ++k) {
+                if (s0 + k < S) {
+                    t[k] = __ldcg(ml + s0 + k);
+                    o0[k] = __ldcg(po + (size_t)(s0 + k) * D4);
+                    o1[k] = __ldcg(po + (size_t)(s0 + k) * D4 + 1);
+                } else {
+                    t[k] = make_float2(-CUDART_INF_F, 0.f);
+                    o0[k] = o1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            float bm = M;
+#pragma unroll
+            for (int k = 0; k < B; ++k) bm = fmaxf(bm, t[k].x);
+            if (bm == -CUDART_INF_F) continue;  // no position in these splits yet
+            const float r = exp2f(M - bm);
+            den *= r;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] *= r;
+#pragma unroll
+            for (int k = 0; k < B; ++k) {
+                const float f = exp2f(t[k].x - bm);
+                den = fmaf(f, t[k].y, den);
+                acc[0] = fmaf(f, o0[k].x, acc[0]);
+                acc[1] = fmaf(f, o0[k].y, acc[1]);
+                acc[2] = fmaf(f, o0[k].z, acc[2]);
+                acc[3] = fmaf(f, o0[k].w, acc[3]);
+                acc[4] = fmaf(f, o1[k].x, acc[4]);
+                acc[5] = fmaf(f, o1[k].y, acc[5]);
+                acc[6] = fmaf(f, o1[k].z, acc[6]);
+                acc[7] = fmaf(f, o1[k].w, acc[7]);
+            }
+            M = bm;
+        }
+        const float inv = 1.0f / den;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[j][k] = acc[k] * inv;
     }
 }
 
@@ -671,14 +754,15 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], rows = w[W_END] - b;
     const uint32_t SB = (uint32_t)p.stage_bytes;
     float* part_sums = scratch;  // [set * rows + row][8 warps]
-    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * 4 : nullptr;
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
 
-    // 1. dependency, zero accumulators
+    // 1. dependency (the weight-pointer table entries of the plan are fetched meanwhile)
+    prefetch_plan_l1(p, w);
     if (tid == 0) {
         if (w[W_WAIT_CTR] >= 0 &&
             !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op))
             vstore(&m.abort_flag, 1);
-        if (tr) tr[1] = globaltimer_ns();
+        if (tr) tr[T_DEP] = globaltimer_ns();
     }
     cbar();
     if (vload(&m.abort_flag)) return false;
@@ -704,8 +788,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
                         (p.snap && w[W_SEQ] == 0) ? p.snap + (size_t)p.L * p.H : nullptr);
             break;
         case OP_OPROJ_RES:
-            K = p.nq * p.d;
-            vsrc = p.attn;
+            K = p.nq * p.d;  // input: the attention output, merged from the kv splits below
             break;
         case OP_DOWN_RES:
         case OP_MOE_DOWN2_RES:
@@ -714,11 +797,12 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
             break;
     }
     const int kp = K / kparts_of(K);  // columns per part
+    if (op == OP_OPROJ_RES) load_attn_merged<J>(p, 0, kp, v);
     if (vsrc) load_vec<J>(vsrc, kp, v);
     // 3. routing (once per layer per block; the loader waits for it)
     if (op == OP_MOE_UPGATE && vload(&m.router_layer) != l)
         route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
-
+    if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
     int eidx[kMaxTopK];
     for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
     Plan pl;
@@ -728,12 +812,13 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     const int nch = kp >> 3;
     for (int ph = 0; ph < pl.nphase; ++ph) {
         const int vslot = ph / pl.kparts, part = ph % pl.kparts;
-        if (ph > 0) load_vec<J>(vsrc + (size_t)vslot * p.F + (size_t)part * kp, kp, v);
+        if (ph > 0 && op == OP_OPROJ_RES) load_attn_merged<J>(p, part * kp, kp, v);
+        else if (ph > 0) load_vec<J>(vsrc + (size_t)vslot * p.F + (size_t)part * kp, kp, v);
         for (int sst = 0; sst < pl.spp; ++sst) {
             const int r0 = sst * pl.rps;
             const int nr = (rows - r0) < pl.rps ? (rows - r0) : pl.rps;
             const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, op);
-            if (tr && tid == 0 && ph == 0 && sst == 0) tr[2] = globaltimer_ns();
+            if (tr && tid == 0 && ph == 0 && sst == 0) tr[T_FIRST] = globaltimer_ns();
             if (ok) {
                 const unsigned char* stage = ring + (size_t)slot * SB;
                 for (int s = 0; s < pl.nspan; ++s) {
@@ -755,6 +840,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     }
     cbar();
     if (vload(&m.abort_flag)) return false;
+    if (tr && tid == 0) tr[T_MAIN] = globaltimer_ns();
 
     // 5. epilogue (storer role): row value of accumulator set k (spans x
     // slots) = the 8 warps' partial sums of every column part, in fixed order
@@ -836,13 +922,12 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
                 // lanes other than 0 of warp 0 keep their own partial; only tid 0 writes
                 p.lm_part[2 * w[W_SEQ]] = bv;
                 p.lm_part[2 * w[W_SEQ] + 1] = __int_as_float(bi);
-                __threadfence();
-                const uint32_t old = atomicAdd(p.counters + w[W_AUX_CTR], 1u);
+                const uint32_t old = arrive_release(p.counters + w[W_AUX_CTR]);
                 m.is_last = (old + 1u == a.epoch * (uint32_t)w[W_AUX_INC]) ? 1 : 0;
             }
             cbar();
             if (m.is_last) {
-                __threadfence();
+                fence_acquire();
                 const int n_lm = w[W_AUX_INC];
                 float cv = -CUDART_INF_F;
                 int ci = 0x7FFFFFFF;
@@ -874,10 +959,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
         }
     }
     cbar();
-    if (tid == 0 && w[W_SIGNAL_CTR] >= 0 && op != OP_LMHEAD_ARGMAX) {
-        __threadfence();
-        atomicAdd(p.counters + w[W_SIGNAL_CTR], 1u);
-    }
+    if (tid == 0 && w[W_SIGNAL_CTR] >= 0 && op != OP_LMHEAD_ARGMAX) signal_release(p.counters + w[W_SIGNAL_CTR]);
     return true;
 }
 
@@ -897,11 +979,12 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], rows = w[W_END] - b;
     const uint32_t SB = (uint32_t)p.stage_bytes;
     float* part_sums = scratch;  // [2 * rows][8 warps] gate / up row sums, then h[rows]
-    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * 4 : nullptr;
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
+    prefetch_plan_l1(p, w);  // weight-pointer table entries, while the dependency is pending
 
     if (tid == 0) {
         if (!wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op)) vstore(&m.abort_flag, 1);
-        if (tr) tr[1] = globaltimer_ns();
+        if (tr) tr[T_DEP] = globaltimer_ns();
     }
     cbar();
     if (vload(&m.abort_flag)) return false;
@@ -911,6 +994,7 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     load_rms<J>(p, m, p.x, nullptr, wt[WT_FFN_NORM], v);
     if (op == OP_MOE_FFN && vload(&m.router_layer) != l)
         route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
+    if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
     int eidx[kMaxTopK];
     for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
     Plan pl;
@@ -922,7 +1006,7 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
         const int r0 = sst * pl.rps;
         const int nr = (rows - r0) < pl.rps ? (rows - r0) : pl.rps;
         const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, op);
-        if (tr && tid == 0 && sst == 0) tr[2] = globaltimer_ns();
+        if (tr && tid == 0 && sst == 0) tr[T_FIRST] = globaltimer_ns();
         if (ok) {
             const unsigned char* stage = ring + (size_t)slot * SB;
             for (int s = 0; s < 2; ++s) {
@@ -942,6 +1026,7 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     }
     cbar();
     if (vload(&m.abort_flag)) return false;
+    if (tr && tid == 0) tr[T_MAIN] = globaltimer_ns();
 
     // h = silu(g) * u (times the router weight), then kept at the start of the scratch
     const float wgt = op == OP_MOE_FFN ? m.ew[sub] : 1.0f;
@@ -1033,10 +1118,7 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
         atomicAdd(dst + 1, make_float4(y[j][4], y[j][5], y[j][6], y[j][7]));
     }
     cbar();
-    if (tid == 0) {
-        __threadfence();
-        atomicAdd(p.counters + w[W_SIGNAL_CTR], 1u);
-    }
+    if (tid == 0) signal_release(p.counters + w[W_SIGNAL_CTR]);
     return true;
 }
 
@@ -1073,53 +1155,83 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
     const int l = w[W_LAYER], g = w[W_SUB], c = w[W_BEGIN], S = w[W_END], pos = a.pos;
     const uint32_t SB = (uint32_t)p.stage_bytes;
     const AttnRange rg = attn_range(pos, c, S);
-    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * 4 : nullptr;
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
+    Plan pl;  // stage plan (weights only: computed while the dependency is still pending)
+    make_plan(p, pos, w, nullptr, pl);
 
     if (tid == 0) {
         if (!wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, OP_ATTN))
             vstore(&m.abort_flag, 1);
-        if (tr) tr[1] = globaltimer_ns();
+        if (tr) tr[T_DEP] = globaltimer_ns();
     }
     cbar();
     if (vload(&m.abort_flag)) return false;
 
-    // q of this set's heads, rotated (rotate-half pairing) and pre-scaled by log2(e)/sqrt(D)
+    // Prologue loads, all issued before any is used (one round trip): this
+    // thread's 8 columns (and their rotate-half partners) of q for the set's
+    // heads, of the new k and v, and the RoPE cos/sin of this position.
     const int col0 = (stid % LPR) * 8;
     const int pcol = col0 ^ (D / 2);
     const bool first_half = col0 < D / 2;
     const float qscale = 1.4426950408889634f / sqrtf((float)D);
-    const float2* rp = p.rope + (size_t)pos * (D / 2) + (col0 & (D / 2 - 1));
-    float q[GW][8];
+    const float4* rp4 = reinterpret_cast<const float4*>(p.rope + (size_t)pos * (D / 2) + (col0 & (D / 2 - 1)));
+    const float* ks = p.qkv + (size_t)p.nq * D + (size_t)g * D;
+    const float* vs = p.qkv + (size_t)(p.nq + p.nkv) * D + (size_t)g * D;
+    float4 qx[GW][2], qy[GW][2], rc[4], kx[2], ky[2], vx[2];
 #pragma unroll
     for (int hh = 0; hh < GW; ++hh) {
         const int h = h0 + hh < G ? h0 + hh : G - 1;  // spare head slots compute a copy that is never stored
-        const float* src = p.qkv + (size_t)(g * G + h) * D;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const float2 cssn = __ldg(rp + k);
-            const float x = __ldcg(src + col0 + k), y = __ldcg(src + pcol + k);
-            q[hh][k] = (first_half ? x * cssn.x - y * cssn.y : x * cssn.x + y * cssn.y) * qscale;
-        }
+        const float4* src = reinterpret_cast<const float4*>(p.qkv + (size_t)(g * G + h) * D);
+        qx[hh][0] = __ldcg(src + col0 / 4);
+        qx[hh][1] = __ldcg(src + col0 / 4 + 1);
+        qy[hh][0] = __ldcg(src + pcol / 4);
+        qy[hh][1] = __ldcg(src + pcol / 4 + 1);
     }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rc[k] = __ldg(rp4 + k);
+    kx[0] = __ldcg(reinterpret_cast<const float4*>(ks + col0));
+    kx[1] = __ldcg(reinterpret_cast<const float4*>(ks + col0) + 1);
+    ky[0] = __ldcg(reinterpret_cast<const float4*>(ks + pcol));
+    ky[1] = __ldcg(reinterpret_cast<const float4*>(ks + pcol) + 1);
+    vx[0] = __ldcg(reinterpret_cast<const float4*>(vs + col0));
+    vx[1] = __ldcg(reinterpret_cast<const float4*>(vs + col0) + 1);
+    float cs[8], sn[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        cs[2 * k] = rc[k].x;
+        sn[2 * k] = rc[k].y;
+        cs[2 * k + 1] = rc[k].z;
+        sn[2 * k + 1] = rc[k].w;
+    }
+    // rotate-half RoPE of one 8-column slice: x' = x cos - y sin (first half), x cos + y sin (second)
+    auto rope8 = [&](const float4 (&x)[2], const float4 (&y)[2], float scale, float* out) {
+        const float xv[8] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w};
+        const float yv[8] = {y[0].x, y[0].y, y[0].z, y[0].w, y[1].x, y[1].y, y[1].z, y[1].w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            out[k] = (first_half ? xv[k] * cs[k] - yv[k] * sn[k] : xv[k] * cs[k] + yv[k] * sn[k]) * scale;
+    };
+    float q[GW][8];
+#pragma unroll
+    for (int hh = 0; hh < GW; ++hh) rope8(qx[hh], qy[hh], qscale, q[hh]);
 
     // the new position: rotated k and v rounded to bf16 (the cache format); the
     // first row group of each set holds it, set 0 appends it to the cache
     float kn[8], vn[8];
     const bool new_rows = rg.has_new && stid < 32;  // first warp of each set
-    if (new_rows) {
-        const float* ks = p.qkv + (size_t)p.nq * D + (size_t)g * D;
-        const float* vs = p.qkv + (size_t)(p.nq + p.nkv) * D + (size_t)g * D;
+    {
+        float kr[8];
+        rope8(kx, ky, 1.0f, kr);
+        const float vv[8] = {vx[0].x, vx[0].y, vx[0].z, vx[0].w, vx[1].x, vx[1].y, vx[1].z, vx[1].w};
         uint32_t kb[8], vb[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            const float2 cssn = __ldg(rp + k);
-            const float x = __ldcg(ks + col0 + k), y = __ldcg(ks + pcol + k);
-            kb[k] = f2bf(first_half ? x * cssn.x - y * cssn.y : x * cssn.x + y * cssn.y);
-            vb[k] = f2bf(__ldcg(vs + col0 + k));
+            kb[k] = f2bf(kr[k]);
+            vb[k] = f2bf(vv[k]);
             kn[k] = __uint_as_float(kb[k] << 16);
             vn[k] = __uint_as_float(vb[k] << 16);
         }
-        if (set == 0 && stid < LPR) {
+        if (new_rows && set == 0 && stid < LPR) {
             const size_t off = (((size_t)l * p.nkv + g) * (size_t)p.max_seq + (size_t)pos) * D + col0;
             uint4 ku, vu;
             ku.x = kb[0] | (kb[1] << 16); ku.y = kb[2] | (kb[3] << 16); ku.z = kb[4] | (kb[5] << 16); ku.w = kb[6] | (kb[7] << 16);
@@ -1128,6 +1240,8 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
             *reinterpret_cast<uint4*>(p.vcache + off) = vu;
         }
     }
+
+    if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
 
     // online softmax over the cached positions streamed through the ring
     float mx[GW], ls[GW], o[GW][8];
@@ -1167,13 +1281,11 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
         }
     };
 
-    Plan pl;
-    make_plan(p, pos, w, nullptr, pl);
     for (int st = 0; st < pl.n_stages; ++st) {
         const int r0 = st * pl.rps;
         const int nr = (pl.rows - r0) < pl.rps ? (pl.rows - r0) : pl.rps;
         const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, OP_ATTN);
-        if (tr && tid == 0 && st == 0) tr[2] = globaltimer_ns();
+        if (tr && tid == 0 && st == 0) tr[T_FIRST] = globaltimer_ns();
         if (ok) {
             const uint4* Ks = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
             const uint4* Vs = Ks + (size_t)pl.rps * (D / 8);
@@ -1201,6 +1313,7 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
         }
     }
     if (new_rows) row_update(kn, vn, lane < LPR);
+    if (tr && tid == 0) tr[T_MAIN] = globaltimer_ns();
 
     // merge row groups within the warp, then the set's warps through shared memory
 #pragma unroll
@@ -1252,35 +1365,7 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
         }
     }
     cbar();
-    if (tid == 0) {
-        __threadfence();
-        const uint32_t old = atomicAdd(p.counters + w[W_AUX_CTR], 1u);
-        m.is_last = (old + 1u == a.epoch * (uint32_t)w[W_AUX_INC]) ? 1 : 0;
-    }
-    cbar();
-    if (m.is_last) {
-        // last split of this kv head: merge all splits' partials into attn
-        __threadfence();
-        for (int idx = tid; idx < G * D; idx += kConsumerThreads) {
-            const int h = idx / D, col = idx % D;
-            const size_t base = (size_t)(g * G + h) * S;
-            float M = -CUDART_INF_F;
-            for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, __ldcg(p.part_ml + (base + s2) * 2));
-            float num = 0.f, den = 0.f;
-            for (int s2 = 0; s2 < S; ++s2) {
-                const float ms = __ldcg(p.part_ml + (base + s2) * 2);
-                const float f = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
-                num += f * __ldcg(p.part_o + (base + s2) * D + col);
-                den += f * __ldcg(p.part_ml + (base + s2) * 2 + 1);
-            }
-            p.attn[(size_t)(g * G + h) * D + col] = num / den;
-        }
-        cbar();
-        if (tid == 0) {
-            __threadfence();
-            atomicAdd(p.counters + w[W_SIGNAL_CTR], 1u);
-        }
-    }
+    if (tid == 0) signal_release(p.counters + w[W_SIGNAL_CTR]);
     return true;
 }
 
@@ -1391,7 +1476,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     uint32_t phase = 0;
     for (int i = 0; i < n; ++i) {
         const int32_t* w = q + (size_t)i * W_NWORDS;
-        if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * 4] = globaltimer_ns();
+        if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_START] = globaltimer_ns();
         if (p.prefetch_ahead > 0 && i + p.prefetch_ahead < n)
             prefetch_instr(p, a, q + (size_t)(i + p.prefetch_ahead) * W_NWORDS, m);
         bool ok;
@@ -1406,7 +1491,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         } else {
             ok = gemv_dispatch(p, a, w, i, smem, full, empty, scratch, m, slot, phase, token);
         }
-        if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * 4 + 3] = globaltimer_ns();
+        if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_END] = globaltimer_ns();
         if (!ok) break;
     }
     if (tid == 0) vstore(&m.abort_flag, 1);  // lets the loader stop early if it is still waiting

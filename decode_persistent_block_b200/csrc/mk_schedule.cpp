@@ -95,10 +95,14 @@ void split_rows(const std::vector<Segment>& segs, int n_sm, int cap, F emit) {
 
 }  // namespace
 
+// Splits per kv head: about 128 cached positions per split at the longest
+// context, at most one split per SM, and few enough that the O-projection's
+// prologue can merge every head's splits (kMaxMergeSlots).
 int default_kv_splits(const mk_config& c, int n_sm) {
-    int s = std::max(1, n_sm / std::max(1, c.n_kv_heads));
-    int cap = std::max(1, (c.max_seq + 31) / 32);
-    return std::min(s, cap);
+    const int per_sm = std::max(1, n_sm / std::max(1, c.n_kv_heads));
+    const int by_len = std::max(1, (c.max_seq + 127) / 128);
+    const int by_merge = std::max(1, kMaxMergeSlots / std::max(1, c.n_q_heads));
+    return std::min(std::min(per_sm, by_len), by_merge);
 }
 
 int check_config(const mk_config& c) {
@@ -145,6 +149,7 @@ int check_options(const mk_config& c, const mk_options& o) {
     if (2LL * 2 * c.hidden > sb || part_bytes(c.ffn) > sb || part_bytes((long long)c.n_q_heads * c.head_dim) > sb)
         return MK_ERR_UNSUPPORTED;
     if (2LL * 2 * c.head_dim > sb) return MK_ERR_UNSUPPORTED;
+    if (o.kv_splits < 0 || (long long)o.kv_splits * c.n_q_heads > kMaxMergeSlots) return MK_ERR_INVALID_ARG;
     if (o.mode < MK_MODE_MEGAKERNEL || o.mode > MK_MODE_MULTI_KERNEL_GRAPH) return MK_ERR_INVALID_ARG;
     // ring + barriers + partial-sum slots + misc must fit the 227 KB per-block opt-in limit
     if ((long long)o.ring_stages * o.stage_bytes + 16LL * o.ring_stages + 128 + 4LL * kRowSlots * 8 + 512 > 232448)
@@ -171,11 +176,11 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     const bool fused = ffn_fused(c, o);
 
     std::vector<std::vector<Instr>> q(n_sm);
-    std::vector<uint32_t> inc(n_counters(L, nkv), 0);
+    std::vector<uint32_t> inc(n_counters(L), 0);
 
     auto add = [&](int sm, Instr w) {
         q[sm].push_back(w);
-        if (w[W_SIGNAL_CTR] >= 0 && w[W_OP] != OP_ATTN) inc[w[W_SIGNAL_CTR]]++;
+        if (w[W_SIGNAL_CTR] >= 0) inc[w[W_SIGNAL_CTR]]++;
         if (w[W_AUX_CTR] >= 0) inc[w[W_AUX_CTR]]++;
     };
     const int qd = c.n_q_heads * d;
@@ -195,9 +200,9 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     };
 
     for (int l = 0; l < L; ++l) {
-        const int prev_down = l > 0 ? ctr_id(l - 1, C_FFN2, nkv) : -1;
+        const int prev_down = l > 0 ? ctr_id(l - 1, C_FFN2) : -1;
         gemv_op(OP_RMS_QKV, l, {{0, c.n_q_heads * d}, {1, nkv * d}, {2, nkv * d}}, prev_down,
-                ctr_id(l, C_QKV, nkv));
+                ctr_id(l, C_QKV));
         // attention: kv head g, split s -> instruction k = g * S + s, rotated per layer
         const int total = nkv * S;
         for (int k = 0; k < total; ++k) {
@@ -207,31 +212,29 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
             w[W_SUB] = k / S;
             w[W_BEGIN] = k % S;
             w[W_END] = S;
-            w[W_WAIT_CTR] = ctr_id(l, C_QKV, nkv);
-            w[W_SIGNAL_CTR] = ctr_id(l, C_ATTN, nkv);
-            w[W_AUX_CTR] = ctr_id(l, C_GROUP0 + k / S, nkv);
+            w[W_WAIT_CTR] = ctr_id(l, C_QKV);
+            w[W_SIGNAL_CTR] = ctr_id(l, C_ATTN);
             int sm = (int)(((long long)k + (long long)l * total) % n_sm);
             add(sm, w);
         }
-        inc[ctr_id(l, C_ATTN, nkv)] = nkv;  // one signal per kv head, by its last-arriving split
-        gemv_op(OP_OPROJ_RES, l, {{0, H}}, ctr_id(l, C_ATTN, nkv), ctr_id(l, C_OPROJ, nkv));
+        gemv_op(OP_OPROJ_RES, l, {{0, H}}, ctr_id(l, C_ATTN), ctr_id(l, C_OPROJ));
         std::vector<Segment> slots;
         for (int s = 0; s < (moe ? c.top_k : 1); ++s) slots.push_back({s, F});
         if (fused) {
             // one instruction per block: its up/gate rows, then the matching down-projection columns
-            gemv_op(moe ? OP_MOE_FFN : OP_FFN, l, slots, ctr_id(l, C_OPROJ, nkv), ctr_id(l, C_FFN2, nkv));
+            gemv_op(moe ? OP_MOE_FFN : OP_FFN, l, slots, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN2));
         } else if (!moe) {
-            gemv_op(OP_RMS_UPGATE_SILU, l, slots, ctr_id(l, C_OPROJ, nkv), ctr_id(l, C_FFN1, nkv));
-            gemv_op(OP_DOWN_RES, l, {{0, H}}, ctr_id(l, C_FFN1, nkv), ctr_id(l, C_FFN2, nkv));
+            gemv_op(OP_RMS_UPGATE_SILU, l, slots, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN1));
+            gemv_op(OP_DOWN_RES, l, {{0, H}}, ctr_id(l, C_FFN1), ctr_id(l, C_FFN2));
         } else {
-            gemv_op(OP_MOE_UPGATE, l, slots, ctr_id(l, C_OPROJ, nkv), ctr_id(l, C_FFN1, nkv));
-            gemv_op(OP_MOE_DOWN2_RES, l, {{0, H}}, ctr_id(l, C_FFN1, nkv), ctr_id(l, C_FFN2, nkv));
+            gemv_op(OP_MOE_UPGATE, l, slots, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN1));
+            gemv_op(OP_MOE_DOWN2_RES, l, {{0, H}}, ctr_id(l, C_FFN1), ctr_id(l, C_FFN2));
         }
     }
     // LM head + argmax: partial slots numbered in emission order
     {
         int seq = 0;
-        const int wait = L > 0 ? ctr_id(L - 1, C_FFN2, nkv) : -1;
+        const int wait = L > 0 ? ctr_id(L - 1, C_FFN2) : -1;
         split_rows({{0, c.vocab}}, n_sm, op_cap(OP_LMHEAD_ARGMAX), [&](int sm, int, int b, int e) {
             Instr w = blank();
             w[W_OP] = OP_LMHEAD_ARGMAX;
@@ -239,7 +242,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
             w[W_BEGIN] = b;
             w[W_END] = e;
             w[W_WAIT_CTR] = wait;
-            w[W_AUX_CTR] = ctr_lm(L, nkv);
+            w[W_AUX_CTR] = ctr_lm(L);
             w[W_SEQ] = seq++;
             add(sm, w);
         });
@@ -256,7 +259,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     out->n_sm = n_sm;
     out->max_instr = max_instr;
     out->kv_splits = S;
-    out->n_lm = (int)inc[ctr_lm(L, nkv)];
+    out->n_lm = (int)inc[ctr_lm(L)];
     out->fused_ffn = fused;
     out->words.assign((size_t)n_sm * max_instr * W_NWORDS, 0);
     out->n_instr.assign(n_sm, 0);
@@ -290,23 +293,22 @@ static int op_index(const int32_t* w) {
 }
 
 // Op index of the op that signals counter `ctr` (LM arrival counter: n_layers*5).
-static int producer_op(int ctr, int L, int nkv) {
-    if (ctr == ctr_lm(L, nkv)) return L * 5;
-    const int per = counters_per_layer(nkv);
-    const int l = ctr / per, slot = ctr % per;
+static int producer_op(int ctr, int L) {
+    if (ctr == ctr_lm(L)) return L * 5;
+    const int l = ctr / kCountersPerLayer, slot = ctr % kCountersPerLayer;
     switch (slot) {
         case C_QKV: return l * 5 + 0;
         case C_ATTN: return l * 5 + 1;
         case C_OPROJ: return l * 5 + 2;
         case C_FFN1: return l * 5 + 3;
         case C_FFN2: return l * 5 + 4;
-        default: return l * 5 + 1;  // head-group arrival counters belong to attention
+        default: return -1;
     }
 }
 
 int validate(const mk_config& c, const Planned& p) {
     const int L = c.n_layers, nkv = c.n_kv_heads, d = c.head_dim;
-    const int nctr = n_counters(L, nkv);
+    const int nctr = n_counters(L);
     if ((int)p.ctr_inc.size() != nctr) return MK_ERR_SCHEDULE;
     const bool moe = c.n_experts > 0;
     // coverage bitmaps: per (layer, op, sub) rows covered exactly once
@@ -344,7 +346,8 @@ int validate(const mk_config& c, const Planned& p) {
             // waits only on counters produced by strictly earlier ops, with the planned increment
             if (w[W_WAIT_CTR] >= 0) {
                 if (w[W_WAIT_CTR] >= nctr) return MK_ERR_SCHEDULE;
-                if (producer_op(w[W_WAIT_CTR], L, nkv) >= oi) return MK_ERR_SCHEDULE;
+                const int po = producer_op(w[W_WAIT_CTR], L);
+                if (po < 0 || po >= oi) return MK_ERR_SCHEDULE;
                 if ((uint32_t)w[W_WAIT_INC] != p.ctr_inc[w[W_WAIT_CTR]] || w[W_WAIT_INC] <= 0) return MK_ERR_SCHEDULE;
             } else if (!(op == OP_RMS_QKV && l == 0) && !(op == OP_LMHEAD_ARGMAX && L == 0)) {
                 return MK_ERR_SCHEDULE;  // everything but the first op depends on something
@@ -354,10 +357,9 @@ int validate(const mk_config& c, const Planned& p) {
             if (op == OP_ATTN) {
                 const int g = w[W_SUB], s = w[W_BEGIN];
                 if (g < 0 || g >= nkv || s < 0 || s >= p.kv_splits || w[W_END] != p.kv_splits) return MK_ERR_SCHEDULE;
-                if (w[W_AUX_CTR] != ctr_id(l, C_GROUP0 + g, nkv) || w[W_SIGNAL_CTR] != ctr_id(l, C_ATTN, nkv))
-                    return MK_ERR_SCHEDULE;
+                if (w[W_AUX_CTR] != -1 || w[W_SIGNAL_CTR] != ctr_id(l, C_ATTN)) return MK_ERR_SCHEDULE;
                 if (attn_seen[(size_t)l * nkv + g][s]++) return MK_ERR_SCHEDULE;
-                signals[w[W_AUX_CTR]]++;
+                signals[w[W_SIGNAL_CTR]]++;
                 continue;
             }
             if (op == OP_MOE_UPGATE) had_moe_ug[l] = 1;
@@ -375,7 +377,7 @@ int validate(const mk_config& c, const Planned& p) {
             for (int r = b; r < e; ++r)
                 if (hits[r]++) return MK_ERR_SCHEDULE;
             if (op == OP_LMHEAD_ARGMAX) {
-                if (w[W_AUX_CTR] != ctr_lm(L, nkv) || w[W_SEQ] < 0 || w[W_SEQ] >= p.n_lm || lm_seq[w[W_SEQ]]++)
+                if (w[W_AUX_CTR] != ctr_lm(L) || w[W_SEQ] < 0 || w[W_SEQ] >= p.n_lm || lm_seq[w[W_SEQ]]++)
                     return MK_ERR_SCHEDULE;
                 signals[w[W_AUX_CTR]]++;
             } else {
@@ -405,7 +407,6 @@ int validate(const mk_config& c, const Planned& p) {
         if (moe)  // every routed slot's rows are covered
             for (int sl = 1; sl < c.top_k; ++sl)
                 if (cov[cov_key(l, p.fused_ffn ? OP_MOE_FFN : OP_MOE_UPGATE, sl)].empty()) return MK_ERR_SCHEDULE;
-        signals[ctr_id(l, C_ATTN, nkv)] = nkv;  // emitted by the merging split of each head group
     }
     if (cov[cov_key(L, OP_LMHEAD_ARGMAX, 0)].empty()) return MK_ERR_SCHEDULE;
     for (int i = 0; i < nctr; ++i)
@@ -437,13 +438,8 @@ int simulate(const int32_t* words, int n_sm, int max_instr, const int32_t* n_ins
             }
             const int sm = ready[rng() % ready.size()];
             const int32_t* w = words + ((size_t)sm * max_instr + pc[sm]) * W_NWORDS;
-            if (w[W_OP] == OP_ATTN) {
-                const uint64_t now = ++ctr[w[W_AUX_CTR]];
-                if (now == (uint64_t)e * (uint32_t)w[W_AUX_INC]) ctr[w[W_SIGNAL_CTR]]++;  // last split merges
-            } else {
-                if (w[W_AUX_CTR] >= 0) ctr[w[W_AUX_CTR]]++;
-                if (w[W_SIGNAL_CTR] >= 0) ctr[w[W_SIGNAL_CTR]]++;
-            }
+            if (w[W_AUX_CTR] >= 0) ctr[w[W_AUX_CTR]]++;
+            if (w[W_SIGNAL_CTR] >= 0) ctr[w[W_SIGNAL_CTR]]++;
             pc[sm]++;
             remaining--;
             done++;
@@ -490,8 +486,6 @@ extern "C" int mk_simulate(const int32_t* buf, int n_sm, int max_instr, const in
             const int32_t* w = buf + ((size_t)sm * max_instr + i) * mk::W_NWORDS;
             for (int k : {mk::W_WAIT_CTR, mk::W_SIGNAL_CTR, mk::W_AUX_CTR})
                 if (w[k] >= n_counters || w[k] < -1) return MK_ERR_INVALID_ARG;
-            if (w[mk::W_OP] == mk::OP_ATTN && (w[mk::W_AUX_CTR] < 0 || w[mk::W_SIGNAL_CTR] < 0))
-                return MK_ERR_INVALID_ARG;
         }
     }
     return mk::simulate(buf, n_sm, max_instr, n_instr, ctr_inc, n_counters, steps, seed, executed);

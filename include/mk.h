@@ -100,7 +100,8 @@ typedef struct {
     int ring_stages;      /* shared-memory weight ring depth (default 3) */
     int stage_bytes;      /* bytes per ring stage, multiple of 1024 (default 65536) */
     int rows_per_instr;   /* cap on GEMV rows per instruction (default and max 1024) */
-    int kv_splits;        /* split-KV chunks per kv head (default: SMs / n_kv_heads, capped by max_seq/32) */
+    int kv_splits;        /* split-KV chunks per kv head (0 = default: about one split per 128 positions of
+                             max_seq, at most SMs / n_kv_heads; n_q_heads * kv_splits <= 2048) */
     int l2_prefetch;      /* bytes kept prefetched into L2 ahead of the TMA stream (-1 default) */
     int trace;            /* 1: record per-instruction globaltimer stamps (mk_get_trace) */
     int snapshots;        /* 1: record the residual stream after every layer (mk_get_hidden) */
@@ -182,9 +183,11 @@ int mk_get_counter_increments(mk_handle *h, uint32_t *out, size_t cap, size_t *n
 /* Copy the device status block (synchronises the stream). */
 int mk_get_status(mk_handle *h, mk_status *out);
 
-/* Trace stamps of the last step: [n_sm][max_instr][4] uint64 globaltimer ns
- * (instruction start, dependency satisfied, first weight stage ready, end;
- * zero where not reached).  Needs options.trace = 1. */
+/* Trace stamps of the last step: [n_sm][max_instr][8] uint64 globaltimer ns,
+ * zero where not reached.  Consumer warps: 0 instruction reached, 1 dependency
+ * satisfied, 2 input vector ready, 3 first stage full, 4 main stages consumed
+ * (the fused FFN's up/gate rows), 5 done and signalled.  Loader warp: 6 first
+ * stage issued, 7 last stage issued.  Needs options.trace = 1. */
 int mk_get_trace(mk_handle *h, uint64_t *out, size_t cap, size_t *n);
 
 /* Clear counters, epoch, status and stop word and re-upload the schedule

@@ -92,9 +92,16 @@ def test_trace_stamps_are_ordered(tiny):
     with tiny.decoder(trace=1) as dec:
         dec.step(3, 0)
         sched = dec.schedule()
-        tr = dec.trace().reshape(sched.shape[0], -1, 4)
+        tr = dec.trace().reshape(sched.shape[0], -1, 8).astype(np.int64)
         n = (sched[:, :, 0] != 0).sum(1)
         for sm in range(tr.shape[0]):
             t = tr[sm, :n[sm]]
-            assert np.all(t[:, 0] > 0) and np.all(t[:, 3] >= t[:, 1]) and np.all(t[:, 1] >= t[:, 0])
-            assert np.all(np.diff(t[:, 0].astype(np.int64)) >= 0)
+            # consumer stamps: reached <= dependency <= ready <= first stage <= main done <= end
+            assert np.all(t[:, 0] > 0) and np.all(t[:, 5] >= t[:, 1]) and np.all(t[:, 1] >= t[:, 0])
+            for a, b in ((1, 2), (2, 3), (3, 4), (4, 5)):
+                hit = (t[:, a] > 0) & (t[:, b] > 0)
+                assert np.all(t[hit, b] >= t[hit, a]), (sm, a, b)
+            assert np.all(np.diff(t[:, 0]) >= 0)
+            # loader: the first stage of an instruction is issued before its consumers see it full
+            hit = (t[:, 6] > 0) & (t[:, 3] > 0)
+            assert np.all(t[hit, 3] >= t[hit, 6]) and np.all(t[t[:, 7] > 0, 7] >= t[t[:, 7] > 0, 6])

@@ -35,7 +35,7 @@ def instrs(words, n_instr):
 
 
 def n_ctr_per_layer(cfg):
-    return 5 + cfg.n_kv_heads
+    return 5  # QKV, ATTN, OPROJ, FFN1, FFN2
 
 
 @pytest.mark.parametrize("split_ffn", [0, 1], ids=["fused_ffn", "split_ffn"])
@@ -61,8 +61,8 @@ def test_plan_covers_rows_and_counts_signals(cfg, n_sm, split_ffn):
             key = (l, int(w[W_SUB]), int(w[W_BEGIN]))
             assert key not in attn_seen
             attn_seen.add(key)
-            assert w[W_AUX] == l * per + 5 + w[W_SUB]
-            signals[w[W_AUX]] += 1
+            assert w[W_AUX] == -1 and w[W_SIG] == l * per + 1 and w[W_WAIT] == l * per + 0
+            signals[w[W_SIG]] += 1
             continue
         key = (l, op, int(w[W_SUB]))
         hit = cover.setdefault(key, np.zeros(rows[op][int(w[W_SUB])], dtype=np.int32))
@@ -81,15 +81,13 @@ def test_plan_covers_rows_and_counts_signals(cfg, n_sm, split_ffn):
     for l in range(L):
         for op in (OP["RMS_QKV"], OP["OPROJ"]) + ffn_ops:
             assert (l, op, 0) in cover
-        signals[l * per + 1] = nkv  # ATTN_DONE: one per kv head from its last split
     assert (L, OP["LM"], 0) in cover
     assert np.array_equal(signals, inc)
     if L:
         assert len(attn_seen) == L * nkv * splits
-        # closed forms: one signal per kv head, `splits` per head group
+        # closed form: every split of every kv head signals; the O-projection waits for all
         for l in range(L):
-            assert inc[l * per + 1] == nkv
-            assert np.all(inc[l * per + 5: l * per + 5 + nkv] == splits)
+            assert inc[l * per + 1] == nkv * splits
 
 
 def _ranges(total, n_sm):
@@ -198,3 +196,23 @@ def test_fused_ffn_is_the_default_for_every_supported_hidden_size():
     for cfg in (configs.LLAMA_3B, configs.TINY.with_(hidden=8192)):
         assert OP["FFN"] in ops(cfg) and OP["UG"] not in ops(cfg)
         assert OP["FFN"] not in ops(cfg, split_ffn=1) and {OP["UG"], OP["DOWN"]} <= ops(cfg, split_ffn=1)
+
+
+@pytest.mark.parametrize("cfg,expect", [(configs.LLAMA_1B, 9), (configs.LLAMA_3B, 17), (configs.TINY, 1),
+                                        (configs.llama1b_sweep(16384), 18)], ids=lambda x: getattr(x, "name", x))
+def test_default_kv_splits(cfg, expect):
+    # about one split per 128 positions of the longest context, at most one per SM per kv head
+    words, n_instr, inc = dpb.plan(cfg, 148)
+    attn = [w for _, _, w in instrs(words, n_instr) if w[W_OP] == OP["ATTN"]]
+    s = int(attn[0][W_END]) if attn else 0
+    assert s == min(-(-cfg.max_seq // 128), 148 // cfg.n_kv_heads, 2048 // cfg.n_heads)
+    if expect is not None:
+        assert s == expect
+
+
+def test_kv_splits_limit_is_checked():
+    cfg = configs.LLAMA_1B  # 32 query heads: at most 64 splits merged per head
+    dpb.plan(cfg, 148, kv_splits=64)
+    with pytest.raises(mk.MkError) as e:
+        dpb.plan(cfg, 148, kv_splits=65)
+    assert e.value.name == "MK_ERR_INVALID_ARG"
