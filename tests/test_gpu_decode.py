@@ -35,7 +35,8 @@ def test_tiny_all_steps(tiny, mode):
 @pytest.mark.parametrize("opts", [
     dict(n_sm=7), dict(n_sm=1), dict(kv_splits=1), dict(kv_splits=40), dict(ring_stages=2),
     dict(stage_bytes=4096), dict(stage_bytes=4096, ring_stages=3, l2_prefetch=16384), dict(rows_per_instr=3),
-    dict(l2_prefetch=65536), dict(split_ffn=1), dict(split_ffn=1, n_sm=7),
+    dict(l2_prefetch=65536), dict(split_ffn=1), dict(split_ffn=1, n_sm=7), dict(ffn_l2_prefetch=500),
+    dict(ffn_l2_prefetch=500, n_sm=5),
 ], ids=lambda o: ",".join(f"{k}={v}" for k, v in o.items()))
 def test_tiny_schedule_options(tiny, opts):
     parity.assert_parity(parity.run(tiny, **opts))
@@ -139,8 +140,15 @@ def test_kv_append_matches_oracle_cache(tiny):
     n = configs.TINY.prompt_len + configs.TINY.steps
     a = (g[:, :, :n].astype(np.uint32) << 16).view(np.float32)
     b = (o[:, :, :n].astype(np.uint32) << 16).view(np.float32)
-    # identical bf16 bits except where fp32 vs fp64 rounding straddles a bf16 tie (at most one ulp)
-    assert np.all(np.abs(a - b) <= np.abs(b) * 2.0 ** -7 + 1e-30)
+    # identical bf16 bits except where the fp32 value and the fp64 one round to neighbouring bf16
+    # values (one ulp), or where k is the small remainder of a cancelling dot product, whose
+    # fp32 error is small against the layer's largest |k| but not against k itself
+    atol = 1e-4 * np.abs(b).max(axis=(1, 2, 3), keepdims=True)
+    bound = np.abs(b) * 2.0 ** -7 + atol
+    ratio = np.abs(a - b) / bound
+    worst = np.argsort(ratio, axis=None)[-3:]
+    detail = [(np.unravel_index(i, a.shape), float(a.flat[i]), float(b.flat[i])) for i in worst]
+    assert np.all(ratio <= 1.0), detail
     assert np.mean(a == b) > 0.99
 
 
