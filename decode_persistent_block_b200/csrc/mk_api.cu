@@ -204,7 +204,6 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     p.stage_bytes = o.stage_bytes;
     p.l2_prefetch = o.l2_prefetch;
     p.prefetch_ahead = o.prefetch_ahead;
-    p.pf_pace_ns = o.ffn_l2_prefetch > 0 ? o.ffn_l2_prefetch : 0;
     p.prefetch_max_bytes = o.prefetch_max_bytes;
     p.spin_limit_ns = o.spin_limit_ns;
 

@@ -46,12 +46,9 @@ enum Word : int {
     W_WAIT_CTR = 5,   // counter waited on before reading activations (-1: none)
     W_WAIT_INC = 6,   // its per-step increment (target = epoch * inc)
     W_SIGNAL_CTR = 7, // counter incremented once when the instruction's outputs are visible (-1: none)
-    W_AUX_CTR = 8,    // LMHEAD: arrival counter (the last arrival takes the global argmax); else -1
+    W_AUX_CTR = 8,    // ATTN: per-head-group arrival counter; LMHEAD: arrival counter
     W_AUX_INC = 9,    // its per-step increment
-    W_SEQ = 10,       // LMHEAD: slot of this instruction's partial argmax
-    W_PF_FIRST = 11,  // queue index (this block) of the first later instruction whose weight rows are
-                      // prefetched into L2 once this instruction's dependency is satisfied (-1: none)
-    W_PF_COUNT = 12,  // number of consecutive queue entries prefetched from W_PF_FIRST
+    W_SEQ = 10,       // LMHEAD: slot of this instruction's partial argmax; ATTN: unused
     W_NWORDS = MK_INSTR_WORDS
 };
 
@@ -154,7 +151,6 @@ struct DevParams {
     int ring_stages;
     int stage_bytes;
     int l2_prefetch;
-    int pf_pace_ns;    // paced L2 prefetch of the FFN weights during the attention chain (0: off)
     int prefetch_ahead;
     int prefetch_max_bytes;
     unsigned long long spin_limit_ns;

@@ -45,25 +45,6 @@ namespace mk {
 // ---------------------------------------------------------------------------
 constexpr int kScratchBytes = 4 * kRowSlots * kConsumerWarps;  // partial row sums; attention merge and router reuse it
 
-struct Plan {
-    int n_stages;   // stages of the whole instruction
-    int nphase;     // slots * kparts (slots: top_k for the fused expert down-projection, else 1)
-    int kparts;     // column parts per row
-    int nspan;      // spans per stage (gate+up, K+V: 2)
-    int rows;       // rows of the instruction
-    int rps;        // rows per stage
-    int spp;        // stages per phase
-    uint32_t row_bytes;   // bytes of one row part in shared memory
-    uint32_t src_stride;  // bytes between consecutive rows in global memory
-    const unsigned char* src[kMaxTopK][2];  // [slot][span]: row 0 of the instruction, column 0
-    // fused FFN: after the main stages, `tail_spp` stages of the transposed
-    // down-projection rows (one span, whole rows of tail_row_bytes)
-    int main_stages;
-    int tail_rps, tail_spp;
-    uint32_t tail_row_bytes;
-    const unsigned char* tail_src;
-};
-
 struct Misc {
     float red[kConsumerWarps * 2];
     int redi[kConsumerWarps];
@@ -73,14 +54,7 @@ struct Misc {
     float ew[kMaxTopK];
     int is_last;
     int pad[3];
-    Plan plan;  // stage plan of a dense instruction, made by thread 0 while it waits for the dependency
-    // Paced L2 prefetch of a later instruction's weights (thread 0, inside its dependency waits):
-    // stage pf_stage of pf_plan is asked for once the clock passes pf_next_ns.
-    Plan pf_plan;
-    int pf_stage;
-    unsigned long long pf_next_ns;
 };
-static_assert(sizeof(Misc) <= 384, "the shared-memory budget reserves 512 bytes for Misc and alignment");
 
 __host__ __device__ inline size_t smem_bars_off(int ns, int sb) { return (size_t)ns * sb; }
 __host__ __device__ inline size_t smem_scratch_off(int ns, int sb) {
@@ -102,9 +76,7 @@ __device__ __forceinline__ void vstore(int* p, int v) { *(volatile int*)p = v; }
 // L2 round trip between a barrier completing and the waiter noticing it.
 constexpr uint64_t kStopPollNs = 20000;
 
-__device__ void drip_prefetch(const DevParams& p, Misc& m, uint64_t now);
-
-__device__ __noinline__ bool wait_counter(const DevParams& p, Misc& m, int ctr, uint32_t target, int ii, int op) {
+__device__ bool wait_counter(const DevParams& p, Misc& m, int ctr, uint32_t target, int ii, int op) {
     const uint32_t* addr = p.counters + ctr;
     uint32_t v = ld_acquire_u32(addr);
     if ((int32_t)(v - target) >= 0) return true;
@@ -114,7 +86,6 @@ __device__ __noinline__ bool wait_counter(const DevParams& p, Misc& m, int ctr, 
         v = ld_acquire_u32(addr);
         if ((int32_t)(v - target) >= 0) return true;
         const uint64_t now = globaltimer_ns();
-        if (m.pf_stage < m.pf_plan.n_stages && now >= m.pf_next_ns) drip_prefetch(p, m, now);
         if (now >= next) {
             if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
             if (now - t0 > p.spin_limit_ns) {
@@ -209,6 +180,24 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
 // vector stays within 4 chunks of 8 in registers.
 static_assert(kMaxPartK == 8 * kConsumerThreads * 4, "a column part is 4 chunks of 8 per consumer thread");
 
+struct Plan {
+    int n_stages;   // stages of the whole instruction
+    int nphase;     // slots * kparts (slots: top_k for the fused expert down-projection, else 1)
+    int kparts;     // column parts per row
+    int nspan;      // spans per stage (gate+up, K+V: 2)
+    int rows;       // rows of the instruction
+    int rps;        // rows per stage
+    int spp;        // stages per phase
+    uint32_t row_bytes;   // bytes of one row part in shared memory
+    uint32_t src_stride;  // bytes between consecutive rows in global memory
+    const unsigned char* src[kMaxTopK][2];  // [slot][span]: row 0 of the instruction, column 0
+    // fused FFN: after the main stages, `tail_spp` stages of the transposed
+    // down-projection rows (one span, whole rows of tail_row_bytes)
+    int main_stages;
+    int tail_rps, tail_spp;
+    uint32_t tail_row_bytes;
+    const unsigned char* tail_src;
+};
 
 struct AttnRange {
     int jb, je, ncached;
@@ -374,31 +363,6 @@ __device__ void prefetch_stage(const Plan& pl, int st) {
             for (int r = 0; r < nr; ++r) prefetch_l2(src + (size_t)r * pl.src_stride, pl.row_bytes);
         }
     }
-}
-
-// Weights of a later instruction of this block's queue (W_PF_FIRST), asked
-// of L2 one ring stage at a time while thread 0 waits on dependency counters
-// (paced: one stage per pf_pace_ns).  The attention chain between a layer's
-// QKV and its FFN leaves HBM mostly idle; the paced stream uses that time
-// without flooding the memory system ahead of the chain's own loads.  The
-// stages the loader is about to copy itself are skipped.
-__device__ __noinline__ void start_prefetch(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, Misc& m) {
-    m.pf_plan.n_stages = 0;
-    m.pf_stage = 0;
-    const int n = p.n_instr[blockIdx.x];
-    const int f = w[W_PF_FIRST];
-    if (p.pf_pace_ns <= 0 || f <= ii || f >= n) return;
-    const int32_t* t = p.instr + ((size_t)blockIdx.x * p.max_instr + f) * W_NWORDS;
-    if (!instr_ok(p, t) || t[W_OP] == OP_ATTN || needs_routing(t[W_OP])) return;
-    make_plan(p, a.pos, t, nullptr, m.pf_plan);
-    m.pf_stage = p.ring_stages - 1 < m.pf_plan.n_stages ? p.ring_stages - 1 : m.pf_plan.n_stages;
-    m.pf_next_ns = 0;
-}
-
-__device__ void drip_prefetch(const DevParams& p, Misc& m, uint64_t now) {
-    prefetch_stage(m.pf_plan, m.pf_stage);
-    m.pf_stage++;
-    m.pf_next_ns = now + (uint64_t)p.pf_pace_ns;
 }
 
 // Plan instruction i for the loader; for MoE ops wait (bounded) until the
@@ -792,17 +756,13 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     float* part_sums = scratch;  // [set * rows + row][8 warps]
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
 
-    // 1. dependency; thread 0 plans the stages of a dense op first (the plan
-    // needs no activations), so that the plan's latency hides behind the wait
+    // 1. dependency (the weight-pointer table entries of the plan are fetched meanwhile)
     prefetch_plan_l1(p, w);
-    const bool routed = needs_routing(op);
     if (tid == 0) {
-        if (!routed) make_plan(p, a.pos, w, nullptr, m.plan);
         if (w[W_WAIT_CTR] >= 0 &&
             !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op))
             vstore(&m.abort_flag, 1);
         if (tr) tr[T_DEP] = globaltimer_ns();
-        if (w[W_PF_FIRST] >= 0) start_prefetch(p, a, w, ii, m);
     }
     cbar();
     if (vload(&m.abort_flag)) return false;
@@ -843,14 +803,10 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     if (op == OP_MOE_UPGATE && vload(&m.router_layer) != l)
         route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
     if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
+    int eidx[kMaxTopK];
+    for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
     Plan pl;
-    if (routed) {
-        int eidx[kMaxTopK];
-        for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
-        make_plan(p, a.pos, w, eidx, pl);
-    } else {
-        pl = m.plan;
-    }
+    make_plan(p, a.pos, w, eidx, pl);
 
     // 4. stages: every warp covers its column slice of every row of the stage
     const int nch = kp >> 3;
@@ -1027,9 +983,7 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     prefetch_plan_l1(p, w);  // weight-pointer table entries, while the dependency is pending
 
     if (tid == 0) {
-        if (op == OP_FFN) make_plan(p, a.pos, w, nullptr, m.plan);  // dense: planned before the wait
         if (!wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op)) vstore(&m.abort_flag, 1);
-        m.pf_plan.n_stages = 0;  // the FFN streams now: no more paced prefetch of its weights
         if (tr) tr[T_DEP] = globaltimer_ns();
     }
     cbar();
@@ -1041,14 +995,10 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     if (op == OP_MOE_FFN && vload(&m.router_layer) != l)
         route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
     if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
+    int eidx[kMaxTopK];
+    for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
     Plan pl;
-    if (op == OP_MOE_FFN) {
-        int eidx[kMaxTopK];
-        for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
-        make_plan(p, a.pos, w, eidx, pl);
-    } else {
-        pl = m.plan;
-    }
+    make_plan(p, a.pos, w, eidx, pl);
     const int nch = p.H >> 3;
 
     // up/gate rows
@@ -1506,9 +1456,6 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(&empty[s], kConsumerWarps);
         }
         m.router_layer = -1;
-        m.pf_plan.n_stages = 0;
-        m.pf_stage = 0;
-        m.pf_next_ns = 0;
         m.is_last = 0;
         m.abort_flag = ld_relaxed_s32(&p.status->stop) ? 1 : 0;
         if (m.abort_flag && atomicCAS(&p.status->code, 0, MK_ERR_STOPPED) == 0) p.status->sm = blockIdx.x;

@@ -38,7 +38,6 @@ Instr blank() {
     w[W_WAIT_CTR] = -1;
     w[W_SIGNAL_CTR] = -1;
     w[W_AUX_CTR] = -1;
-    w[W_PF_FIRST] = -1;
     return w;
 }
 
@@ -248,28 +247,6 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
             add(sm, w);
         });
     }
-    // L2 prefetch of the dense fused FFN's weight rows: each block's first QKV
-    // instruction of layer l names that block's FFN instructions of layer l.
-    // They stream after the attention chain, which leaves HBM mostly idle.
-    if (fused && !moe && o.ffn_l2_prefetch > 0) {
-        for (auto& qs : q) {
-            for (int l = 0; l < L; ++l) {
-                int first_qkv = -1, ffn0 = -1, nffn = 0;
-                for (int i = 0; i < (int)qs.size(); ++i) {
-                    if (qs[i][W_LAYER] != l) continue;
-                    if (qs[i][W_OP] == OP_RMS_QKV && first_qkv < 0) first_qkv = i;
-                    if (qs[i][W_OP] == OP_FFN) {
-                        if (ffn0 < 0) ffn0 = i;
-                        ++nffn;
-                    }
-                }
-                if (first_qkv >= 0 && ffn0 > first_qkv) {
-                    qs[first_qkv][W_PF_FIRST] = ffn0;
-                    qs[first_qkv][W_PF_COUNT] = nffn;
-                }
-            }
-        }
-    }
     // fill wait increments and aux increments
     for (auto& qs : q)
         for (auto& w : qs) {
@@ -376,14 +353,6 @@ int validate(const mk_config& c, const Planned& p) {
                 return MK_ERR_SCHEDULE;  // everything but the first op depends on something
             }
             if (w[W_SIGNAL_CTR] >= nctr || w[W_AUX_CTR] >= nctr) return MK_ERR_SCHEDULE;
-            if (w[W_PF_FIRST] != -1) {  // a later run of this block's own GEMV instructions
-                const int f = w[W_PF_FIRST], n = w[W_PF_COUNT];
-                if (f <= i || n < 1 || f + n > p.n_instr[sm]) return MK_ERR_SCHEDULE;
-                for (int k = f; k < f + n; ++k)
-                    if (p.words[((size_t)sm * p.max_instr + k) * W_NWORDS + W_OP] == OP_ATTN) return MK_ERR_SCHEDULE;
-            } else if (w[W_PF_COUNT] != 0) {
-                return MK_ERR_SCHEDULE;
-            }
             if (w[W_AUX_CTR] >= 0 && (uint32_t)w[W_AUX_INC] != p.ctr_inc[w[W_AUX_CTR]]) return MK_ERR_SCHEDULE;
             if (op == OP_ATTN) {
                 const int g = w[W_SUB], s = w[W_BEGIN];

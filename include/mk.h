@@ -111,10 +111,6 @@ typedef struct {
     int prefetch_ahead;   /* consumers prefetch into L2 the weights of the instruction this many
                              places ahead in their queue (-1 default, 0 = off) */
     int prefetch_max_bytes; /* cap on the bytes prefetched per instruction (0 = default 1 MiB) */
-    int ffn_l2_prefetch;  /* dense models, > 0: once a layer's QKV dependency is met, each block asks L2
-                             for the weight rows of its fused FFN instruction of that layer, one ring
-                             stage per this many ns while it waits on the attention chain's
-                             dependencies.  0 (default): off (measured slower on B200) */
     int split_ffn;        /* 0 (default): each layer's FFN is one fused instruction per SM (up/gate rows,
                              then the matching columns of w_down, streamed from a transposed copy the
                              library keeps, added into the residual with atomics: fp32 summation order

@@ -35,8 +35,7 @@ def test_tiny_all_steps(tiny, mode):
 @pytest.mark.parametrize("opts", [
     dict(n_sm=7), dict(n_sm=1), dict(kv_splits=1), dict(kv_splits=40), dict(ring_stages=2),
     dict(stage_bytes=4096), dict(stage_bytes=4096, ring_stages=3, l2_prefetch=16384), dict(rows_per_instr=3),
-    dict(l2_prefetch=65536), dict(split_ffn=1), dict(split_ffn=1, n_sm=7), dict(ffn_l2_prefetch=500),
-    dict(ffn_l2_prefetch=500, n_sm=5),
+    dict(l2_prefetch=65536), dict(split_ffn=1), dict(split_ffn=1, n_sm=7),
 ], ids=lambda o: ",".join(f"{k}={v}" for k, v in o.items()))
 def test_tiny_schedule_options(tiny, opts):
     parity.assert_parity(parity.run(tiny, **opts))

@@ -15,7 +15,7 @@ from decode_persistent_block_b200 import mk
 from synth import configs
 
 OP = dict(RMS_QKV=1, ATTN=2, OPROJ=3, UG=4, DOWN=5, LM=6, MOE_UG=7, MOE_DOWN=8, FFN=9, MOE_FFN=10)
-W_OP, W_LAYER, W_SUB, W_BEGIN, W_END, W_WAIT, W_WINC, W_SIG, W_AUX, W_AINC, W_SEQ, W_PF, W_PFN = range(13)
+W_OP, W_LAYER, W_SUB, W_BEGIN, W_END, W_WAIT, W_WINC, W_SIG, W_AUX, W_AINC, W_SEQ = range(11)
 
 CFGS = [configs.TINY, configs.LLAMA_1B, configs.LLAMA_3B, configs.MIXTRAL_8L, configs.llama1b_sweep(16384),
         configs.TINY.with_(name="tiny_moe", n_experts=4, top_k=2),
@@ -216,36 +216,3 @@ def test_kv_splits_limit_is_checked():
     with pytest.raises(mk.MkError) as e:
         dpb.plan(cfg, 148, kv_splits=65)
     assert e.value.name == "MK_ERR_INVALID_ARG"
-
-
-@pytest.mark.parametrize("cfg", [configs.LLAMA_1B, configs.LLAMA_3B, configs.TINY], ids=lambda c: c.name)
-def test_ffn_l2_prefetch_words(cfg):
-    # each block's first QKV of layer l names exactly that block's fused FFN instructions of layer l
-    words, n_instr, _ = dpb.plan(cfg, 148 if cfg.hidden > 256 else 9, ffn_l2_prefetch=2000)
-    seen = 0
-    for sm in range(words.shape[0]):
-        q = words[sm, :n_instr[sm]]
-        for i, w in enumerate(q):
-            if w[W_PF] < 0:
-                assert w[W_PFN] == 0
-                continue
-            assert w[W_OP] == OP["RMS_QKV"]
-            l = w[W_LAYER]
-            named = list(range(w[W_PF], w[W_PF] + w[W_PFN]))
-            ffn = [k for k, x in enumerate(q) if x[W_OP] == OP["FFN"] and x[W_LAYER] == l]
-            assert named == ffn and named[0] > i
-            assert all(x[W_OP] != OP["RMS_QKV"] or x[W_LAYER] != l for x in q[:i])  # the first QKV of l
-            seen += 1
-    assert seen == sum(1 for sm in range(words.shape[0]) for l in range(cfg.n_layers)
-                       if any(x[W_OP] == OP["FFN"] and x[W_LAYER] == l for x in words[sm, :n_instr[sm]])
-                       and any(x[W_OP] == OP["RMS_QKV"] and x[W_LAYER] == l for x in words[sm, :n_instr[sm]]))
-    for kw in (dict(), dict(ffn_l2_prefetch=2000, split_ffn=1)):
-        words, n_instr, _ = dpb.plan(cfg, 148, **kw)
-        assert np.all(words[:, :, W_PF] == -1 * (words[:, :, W_OP] != 0)) and not words[:, :, W_PFN].any()
-
-
-def test_moe_has_no_ffn_l2_prefetch():
-    words, n_instr, _ = dpb.plan(configs.MIXTRAL_8L, 148, ffn_l2_prefetch=2000)
-    used = words[:, :, W_OP] != 0
-    assert np.all(words[:, :, W_PF][used] == -1)
-
