@@ -31,6 +31,7 @@ struct mk_handle {
     cudaGraph_t graph = nullptr;
     cudaGraphExec_t graph_exec = nullptr;
     int lm_slots = 0;
+    int variant = 0;  // megakernel instantiation for the built schedule
     bool down_t = false;  // transposed down-projection copies exist (fused FFN schedules)
     int last_cuda = 0;
     int last_error = MK_OK;
@@ -310,6 +311,7 @@ int mk_build_schedule(mk_handle* h) {
     if (plan.n_lm > h->lm_slots) return MK_ERR_SCHEDULE;
     if (plan.fused_ffn && h->cfg.n_layers > 0 && !h->down_t) return MK_ERR_SCHEDULE;
     h->plan = plan;
+    h->variant = mk::megakernel_variant(h->p, plan.fused_ffn);
     int32_t* words = nullptr;
     int32_t* n_instr = nullptr;
     if ((rc = dalloc(h, &words, plan.words.size()))) return rc;
@@ -353,7 +355,7 @@ int mk_decode_step(mk_handle* h, int32_t token, int32_t pos, float* logits_dev, 
         a.epoch = h->epoch;
         a.logits = logits_dev ? logits_dev : p.logits;
         CK(cudaEventRecord(h->ev0, h->stream));
-        CK(mk::launch_megakernel(p, a, h->n_sm, h->stream));
+        CK(mk::launch_megakernel(p, a, h->n_sm, h->variant, h->stream));
         CK(cudaEventRecord(h->ev1, h->stream));
     } else {
         mk::BaselineShape bs{h->n_sm, mk::baseline_lm_blocks(p, h->n_sm)};

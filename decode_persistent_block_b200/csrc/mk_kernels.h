@@ -21,7 +21,11 @@ struct BaselineShape {
 
 size_t megakernel_smem_bytes(int ring_stages, int stage_bytes);
 cudaError_t prepare_megakernel(int ring_stages, int stage_bytes, int* max_blocks_per_sm);
-cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, cudaStream_t stream);
+// Kernel instantiation for a schedule: 1 or 2 when every GEMV-type instruction
+// has that many 8-column chunks per consumer thread (fused FFN, no optional L2
+// prefetch), else 0 (the general kernel).
+int megakernel_variant(const DevParams& p, bool fused_ffn);
+cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, int variant, cudaStream_t stream);
 
 // dst[c][r] = src[r][c] for a row-major bf16 matrix of rows x cols (one-time,
 // at set-up: the fused FFN streams the down-projection by its input index).

@@ -401,11 +401,13 @@ __device__ bool loader_plan(const DevParams& p, const StepArgs& a, const int32_t
     return true;
 }
 
+// PF: the L2 prefetch cursor (options.l2_prefetch) is compiled in.
+template <bool PF>
 __device__ void loader(const DevParams& p, const StepArgs& a, const int32_t* q, int n, unsigned char* ring,
                        uint64_t* full, uint64_t* empty, Misc& m) {
     const int NS = p.ring_stages;
     const uint32_t SB = (uint32_t)p.stage_bytes;
-    const int pf_stages = p.l2_prefetch > 0 ? (int)((uint32_t)p.l2_prefetch / SB) : 0;
+    const int pf_stages = PF && p.l2_prefetch > 0 ? (int)((uint32_t)p.l2_prefetch / SB) : 0;
     int slot = 0;
     uint32_t phase = 0;
     uint32_t used = 0, last_parity = 0;
@@ -436,7 +438,7 @@ __device__ void loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                 slot = 0;
                 phase ^= 1u;
             }
-            if (pf_stages > 0) {
+            if (PF && pf_stages > 0) {
                 if (pf_g <= g) {  // cursor caught up: restart right after this stage
                     pf_i = i;
                     pf_st = st + 1;
@@ -1144,6 +1146,7 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
     const int D = p.d;                                  // head_dim, 64 or 128
     const int LPR = D / 8;                              // lanes per K/V row, 8 columns each
     constexpr int GW = 2;                               // head slots per set
+    constexpr int AR = 4;                               // K/V rows per lane group per pass
     constexpr int SET_THREADS = kConsumerThreads / 2;
     constexpr int SET_WARPS = kConsumerWarps / 2;
     const int RGN = SET_THREADS / LPR;                  // rows per pass of a set
@@ -1289,18 +1292,68 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
         if (ok) {
             const uint4* Ks = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
             const uint4* Vs = Ks + (size_t)pl.rps * (D / 8);
-            for (int base = 0; base < nr; base += RGN) {
-                const int r = base + stid / LPR;
-                const bool valid = r < nr;
-                float kf[8], vf[8];
-                if (valid) {
-                    unpack8(Ks[r * (D / 8) + col0 / 8], kf);
-                    unpack8(Vs[r * (D / 8) + col0 / 8], vf);
-                } else {
+            // AR rows per lane group per pass: their scores are independent, and
+            // the running max / rescale is taken once per pass instead of per row
+            for (int base = 0; base < nr; base += RGN * AR) {
+                uint4 kw[AR], vw[AR];
+                bool valid[AR];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) kf[k] = vf[k] = 0.f;
+                for (int i = 0; i < AR; ++i) {
+                    const int r = base + i * RGN + stid / LPR;
+                    valid[i] = r < nr;
+                    const int rr = valid[i] ? r : 0;
+                    kw[i] = Ks[rr * (D / 8) + col0 / 8];
+                    vw[i] = Vs[rr * (D / 8) + col0 / 8];
                 }
-                row_update(kf, vf, valid);
+                float sc[AR][GW];
+#pragma unroll
+                for (int i = 0; i < AR; ++i) {
+                    float kf[8];
+                    unpack8(kw[i], kf);
+#pragma unroll
+                    for (int hh = 0; hh < GW; ++hh) {
+                        float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+                        for (int k = 0; k < 8; k += 2) {
+                            t0 = fmaf(q[hh][k], kf[k], t0);
+                            t1 = fmaf(q[hh][k + 1], kf[k + 1], t1);
+                        }
+                        sc[i][hh] = t0 + t1;
+                    }
+                }
+#pragma unroll
+                for (int off = LPR / 2; off > 0; off >>= 1)
+#pragma unroll
+                    for (int i = 0; i < AR; ++i)
+#pragma unroll
+                        for (int hh = 0; hh < GW; ++hh) sc[i][hh] += __shfl_xor_sync(0xFFFFFFFFu, sc[i][hh], off);
+#pragma unroll
+                for (int hh = 0; hh < GW; ++hh) {
+                    float mn = mx[hh];
+#pragma unroll
+                    for (int i = 0; i < AR; ++i)
+                        if (valid[i]) mn = fmaxf(mn, sc[i][hh]);
+                    if (mn == -CUDART_INF_F) continue;  // no valid row in this pass
+                    const float al = exp2f(mx[hh] - mn);
+                    float pr[AR];
+                    float psum = 0.f;
+#pragma unroll
+                    for (int i = 0; i < AR; ++i) {
+                        pr[i] = valid[i] ? exp2f(sc[i][hh] - mn) : 0.f;
+                        psum += pr[i];
+                    }
+                    ls[hh] = fmaf(ls[hh], al, psum);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) o[hh][k] *= al;
+#pragma unroll
+                    for (int i = 0; i < AR; ++i) {
+                        float vf[8];
+                        unpack8(vw[i], vf);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) o[hh][k] = fmaf(pr[i], vf[k], o[hh][k]);
+                    }
+                    mx[hh] = mn;
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
@@ -1378,9 +1431,18 @@ __device__ __forceinline__ int gemv_k(const DevParams& p, int op) {
     return p.H;
 }
 
+// JF > 0: every GEMV-type instruction of the schedule has J == JF (checked on
+// the host), so only that instantiation is compiled into the kernel; JF == 0:
+// dispatch on the instruction's J at run time.
+template <int JF>
 __device__ bool gemv_dispatch(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                               uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase,
                               int token) {
+    if constexpr (JF > 0) {
+        if (w[W_OP] == OP_FFN || w[W_OP] == OP_MOE_FFN)
+            return ffn_instr<JF>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+        return gemv_instr<JF>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+    }
     const int K = gemv_k(p, w[W_OP]);
     const int kp = K / kparts_of(K);
     const int J = ((kp >> 3) + kConsumerThreads - 1) / kConsumerThreads;
@@ -1441,6 +1503,9 @@ __device__ void prefetch_instr(const DevParams& p, const StepArgs& a, const int3
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
+// One instantiation per JF (see gemv_dispatch); the specialised ones also
+// leave out the optional L2-prefetch paths.
+template <int JF>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ DevParams p, const StepArgs a) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int NS = p.ring_stages, SB = p.stage_bytes;
@@ -1467,7 +1532,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     const int n = p.n_instr[blockIdx.x];
     const int32_t* q = p.instr + (size_t)blockIdx.x * p.max_instr * W_NWORDS;
     if (warp == kConsumerWarps) {
-        if (lane == 0) loader(p, a, q, n, smem, full, empty, m);
+        if (lane == 0) loader<JF == 0>(p, a, q, n, smem, full, empty, m);
         return;
     }
 
@@ -1477,7 +1542,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     for (int i = 0; i < n; ++i) {
         const int32_t* w = q + (size_t)i * W_NWORDS;
         if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_START] = globaltimer_ns();
-        if (p.prefetch_ahead > 0 && i + p.prefetch_ahead < n)
+        if (JF == 0 && p.prefetch_ahead > 0 && i + p.prefetch_ahead < n)
             prefetch_instr(p, a, q + (size_t)(i + p.prefetch_ahead) * W_NWORDS, m);
         bool ok;
         if (!instr_ok(p, w) || token < 0 || token >= p.V) {
@@ -1489,7 +1554,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         } else if (w[W_OP] == OP_ATTN) {
             ok = attn_instr(p, a, w, i, smem, full, empty, scratch, m, slot, phase);
         } else {
-            ok = gemv_dispatch(p, a, w, i, smem, full, empty, scratch, m, slot, phase, token);
+            ok = gemv_dispatch<JF>(p, a, w, i, smem, full, empty, scratch, m, slot, phase, token);
         }
         if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_END] = globaltimer_ns();
         if (!ok) break;
@@ -1497,7 +1562,30 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     if (tid == 0) vstore(&m.abort_flag, 1);  // lets the loader stop early if it is still waiting
 }
 
-cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, cudaStream_t stream) {
+namespace {
+using KernelFn = void (*)(DevParams, StepArgs);
+KernelFn kernel_of(int jf) {
+    switch (jf) {
+        case 1: return megakernel<1>;
+        case 2: return megakernel<2>;
+    }
+    return megakernel<0>;
+}
+// J of a GEMV over K columns (chunks of 8 per consumer thread, per column part)
+int j_of(int K) {
+    const int kp = K / kparts_of(K);
+    return ((kp >> 3) + kConsumerThreads - 1) / kConsumerThreads;
+}
+}  // namespace
+
+int megakernel_variant(const DevParams& p, bool fused_ffn) {
+    if (!fused_ffn || p.l2_prefetch > 0 || p.prefetch_ahead > 0) return 0;
+    const int jh = j_of(p.H), jo = j_of(p.nq * p.d);
+    if (jh != jo || jh > 2) return 0;
+    return jh;
+}
+
+cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, int variant, cudaStream_t stream) {
     const size_t smem = megakernel_smem_bytes(p.ring_stages, p.stage_bytes);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(n_sm);
@@ -1509,14 +1597,21 @@ cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, c
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, megakernel, p, a);
+    return cudaLaunchKernelEx(&cfg, kernel_of(variant), p, a);
 }
 
 cudaError_t prepare_megakernel(int ring_stages, int stage_bytes, int* max_blocks_per_sm) {
     const size_t smem = megakernel_smem_bytes(ring_stages, stage_bytes);
-    cudaError_t e = cudaFuncSetAttribute(megakernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(max_blocks_per_sm, megakernel, kThreads, smem);
+    *max_blocks_per_sm = 1 << 30;
+    for (int v = 0; v <= 2; ++v) {
+        cudaError_t e = cudaFuncSetAttribute(kernel_of(v), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel_of(v), kThreads, smem);
+        if (e != cudaSuccess) return e;
+        if (per_sm < *max_blocks_per_sm) *max_blocks_per_sm = per_sm;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace mk
