@@ -508,9 +508,8 @@ __device__ __forceinline__ void load_vec(const float* __restrict__ src, int K, f
 // o_s, running max m_s in the log2 domain, sum l_s):
 //   attn = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s,
 // taken B splits per round trip with an online rescale, in split order.
-template <int J>
+template <int J, int B>
 __device__ __forceinline__ void load_attn_merged(const DevParams& p, int col0, int K, float (&v)[J][8]) {
-    constexpr int B = 4;
     const int tid = threadIdx.x, nch = K >> 3, S = p.kv_splits, D = p.d;
 #pragma unroll
     for (int j = 0; j < J; ++j) {
@@ -746,7 +745,9 @@ __device__ __forceinline__ void stage_rows(const uint4* __restrict__ Ws, int row
     }
 }
 
-template <int J>
+// HOIST: dense instructions make their stage plan before the dependency wait
+// (costs registers across the wait; used by the specialised kernels).
+template <int J, bool HOIST>
 __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                            uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase,
                            int token) {
@@ -758,8 +759,12 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     float* part_sums = scratch;  // [set * rows + row][8 warps]
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
 
-    // 1. dependency (the weight-pointer table entries of the plan are fetched meanwhile)
-    prefetch_plan_l1(p, w);
+    // 1. dependency (the weight-pointer table entries of the plan are fetched meanwhile, or the
+    // plan of a dense op is made before the wait)
+    Plan pl;
+    const bool early = HOIST && !needs_routing(op);
+    if (early) make_plan(p, a.pos, w, nullptr, pl);
+    else prefetch_plan_l1(p, w);
     if (tid == 0) {
         if (w[W_WAIT_CTR] >= 0 &&
             !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op))
@@ -799,22 +804,23 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
             break;
     }
     const int kp = K / kparts_of(K);  // columns per part
-    if (op == OP_OPROJ_RES) load_attn_merged<J>(p, 0, kp, v);
+    if (op == OP_OPROJ_RES) load_attn_merged<J, HOIST ? 8 : 4>(p, 0, kp, v);
     if (vsrc) load_vec<J>(vsrc, kp, v);
     // 3. routing (once per layer per block; the loader waits for it)
     if (op == OP_MOE_UPGATE && vload(&m.router_layer) != l)
         route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
     if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
-    int eidx[kMaxTopK];
-    for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
-    Plan pl;
-    make_plan(p, a.pos, w, eidx, pl);
+    if (!early) {
+        int eidx[kMaxTopK];
+        for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
+        make_plan(p, a.pos, w, eidx, pl);
+    }
 
     // 4. stages: every warp covers its column slice of every row of the stage
     const int nch = kp >> 3;
     for (int ph = 0; ph < pl.nphase; ++ph) {
         const int vslot = ph / pl.kparts, part = ph % pl.kparts;
-        if (ph > 0 && op == OP_OPROJ_RES) load_attn_merged<J>(p, part * kp, kp, v);
+        if (ph > 0 && op == OP_OPROJ_RES) load_attn_merged<J, HOIST ? 8 : 4>(p, part * kp, kp, v);
         else if (ph > 0) load_vec<J>(vsrc + (size_t)vslot * p.F + (size_t)part * kp, kp, v);
         for (int sst = 0; sst < pl.spp; ++sst) {
             const int r0 = sst * pl.rps;
@@ -973,7 +979,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
 // added into the post-FFN residual x2 with float4 atomics.  One instruction,
 // one continuous weight stream per block: the up/gate -> down dependency stays
 // inside the block.
-template <int J>
+template <int J, bool HOIST>
 __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                           uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
     constexpr int RG = J == 1 ? 8 : J == 2 ? 4 : J == 3 ? 2 : 1;
@@ -982,7 +988,10 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     const uint32_t SB = (uint32_t)p.stage_bytes;
     float* part_sums = scratch;  // [2 * rows][8 warps] gate / up row sums, then h[rows]
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
-    prefetch_plan_l1(p, w);  // weight-pointer table entries, while the dependency is pending
+    Plan pl;
+    const bool early = HOIST && op == OP_FFN;  // dense: planned before the wait
+    if (early) make_plan(p, a.pos, w, nullptr, pl);
+    else prefetch_plan_l1(p, w);  // weight-pointer table entries, while the dependency is pending
 
     if (tid == 0) {
         if (!wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op)) vstore(&m.abort_flag, 1);
@@ -997,10 +1006,11 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     if (op == OP_MOE_FFN && vload(&m.router_layer) != l)
         route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
     if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
-    int eidx[kMaxTopK];
-    for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
-    Plan pl;
-    make_plan(p, a.pos, w, eidx, pl);
+    if (!early) {
+        int eidx[kMaxTopK];
+        for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
+        make_plan(p, a.pos, w, eidx, pl);
+    }
     const int nch = p.H >> 3;
 
     // up/gate rows
@@ -1440,26 +1450,26 @@ __device__ bool gemv_dispatch(const DevParams& p, const StepArgs& a, const int32
                               int token) {
     if constexpr (JF > 0) {
         if (w[W_OP] == OP_FFN || w[W_OP] == OP_MOE_FFN)
-            return ffn_instr<JF>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-        return gemv_instr<JF>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+            return ffn_instr<JF, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+        return gemv_instr<JF, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
     }
     const int K = gemv_k(p, w[W_OP]);
     const int kp = K / kparts_of(K);
     const int J = ((kp >> 3) + kConsumerThreads - 1) / kConsumerThreads;
     if (w[W_OP] == OP_FFN || w[W_OP] == OP_MOE_FFN) {
         switch (J) {
-            case 1: return ffn_instr<1>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-            case 2: return ffn_instr<2>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-            case 3: return ffn_instr<3>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-            case 4: return ffn_instr<4>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 1: return ffn_instr<1, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 2: return ffn_instr<2, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 3: return ffn_instr<3, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 4: return ffn_instr<4, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
         }
         return false;
     }
     switch (J) {
-        case 1: return gemv_instr<1>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
-        case 2: return gemv_instr<2>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
-        case 3: return gemv_instr<3>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
-        case 4: return gemv_instr<4>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+        case 1: return gemv_instr<1, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+        case 2: return gemv_instr<2, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+        case 3: return gemv_instr<3, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+        case 4: return gemv_instr<4, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
     }
     return false;
 }
