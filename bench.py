@@ -97,6 +97,13 @@ def reduce_max(x: float, world: int) -> float:
     return float(t.item())
 
 
+def job_us_per_token(local_ms: float, steps: int, world: int) -> float:
+    """Whole-job time per token: the slowest rank's device time over the
+    tokens all ranks decoded (each rank decodes `steps` tokens of its own
+    replica)."""
+    return reduce_max(local_ms, world) * 1000.0 / (steps * world)
+
+
 # ---- clocks during the timed region ---------------------------------------------------------------
 
 class Clocks:
@@ -195,8 +202,10 @@ def workload(args):
     return cfg, p0, positions
 
 
-def oracle_steps(cfg, seconds: float, max_steps: int | None = None):
-    """Time the fp64 oracle on consecutive decode positions for about `seconds`."""
+def oracle_steps(cfg, seconds: float, max_steps: int | None = None, min_steps: int = 2):
+    """Time the fp64 oracle on consecutive decode positions: until `max_steps`
+    steps or about `seconds` of work, whichever comes first (at least
+    `min_steps`)."""
     import oracle
     import synth
     W = synth.make_model(cfg)
@@ -214,7 +223,7 @@ def oracle_steps(cfg, seconds: float, max_steps: int | None = None):
         i += 1
         if max_steps is not None and i >= max_steps:
             break
-        if max_steps is None and time.perf_counter() - t_start >= seconds and i >= 2:
+        if time.perf_counter() - t_start >= seconds and i >= min_steps:
             break
     return times, oracle.num_threads()
 
@@ -273,8 +282,7 @@ def run_ours(args, rank, world, local):
     clocks.start()
     total_ms, per_launch = timed(dec, K, Wm)
     clk = clocks.stop()
-    total_ms = reduce_max(total_ms, world)
-    us_per_token = total_ms * 1000.0 / (K * world)
+    us_per_token = job_us_per_token(total_ms, K, world)
     launch_ms = statistics.fmean(per_launch)
     bpt = bytes_per_token(cfg, [positions[i % len(positions)] for i in range(K)])
     peak, peak_kind = hbm_peak()
@@ -342,14 +350,23 @@ def run_ours(args, rank, world, local):
 
 # ---- reference arm: the fp64 oracle on the host cores ---------------------------------------------------
 
+REFERENCE_SECONDS = 90.0  # bound on the reference arm's timed oracle work
+
+
 def run_reference(args, rank, world):
+    """The fp64 oracle on the host cores, rank 0 only: W warm-up steps (at most
+    one), then up to K timed decode steps, stopping early once about
+    REFERENCE_SECONDS of oracle work is done (each step is one whole decode step
+    of the workload; the sample says how many were timed)."""
     if rank != 0:
         return None
     cfg, p0, positions = workload(args)
-    times, cores = oracle_steps(cfg, 0, max_steps=args.warmup + args.steps)
-    t = times[args.warmup:]
+    warm = min(args.warmup, 1)
+    times, cores = oracle_steps(cfg, REFERENCE_SECONDS, max_steps=warm + args.steps, min_steps=warm + 2)
+    t = times[warm:]
     v = statistics.fmean(t) * 1e6
-    sample = f"{len(t)} fp64 oracle decode steps of {cfg.name} at positions {p0}.. after {args.warmup} warm-up"
+    sample = (f"{len(t)} of the {args.steps} requested fp64 oracle decode steps of {cfg.name} at positions "
+              f"{p0}.. (bounded to about {REFERENCE_SECONDS:.0f} s), after {warm} warm-up")
     return {"impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v / 1000.0, 3),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
