@@ -54,14 +54,28 @@ struct Segment {
 // would run two instructions back to back and finish last, delaying every
 // block that waits for the op.  With fewer blocks than segments the virtual
 // concatenation is split instead.  Calls emit(sm, sub, begin, end).
+// `weight` (optional, one entry per block, single-segment ops only) scales a
+// block's share of the rows.
 template <class F>
-void split_rows(const std::vector<Segment>& segs, int n_sm, int cap, F emit) {
+void split_rows(const std::vector<Segment>& segs, int n_sm, int cap, F emit,
+                const std::vector<double>* weight = nullptr) {
     long long total = 0;
     for (auto& s : segs) total += s.rows;
     const int ns = (int)segs.size();
+    std::vector<long long> cut(n_sm + 1);
+    if (weight && ns == 1) {
+        double sum = 0.0, acc = 0.0;
+        for (int sm = 0; sm < n_sm; ++sm) sum += (*weight)[sm];
+        for (int sm = 0; sm <= n_sm; ++sm) {
+            cut[sm] = sm == n_sm ? total : std::min(total, (long long)std::llround(total * acc / sum));
+            if (sm < n_sm) acc += (*weight)[sm];
+        }
+    } else {
+        for (int sm = 0; sm <= n_sm; ++sm) cut[sm] = total * sm / n_sm;
+    }
     if (n_sm < ns || ns == 1) {
         for (int sm = 0; sm < n_sm; ++sm) {
-            long long a = total * sm / n_sm, b = total * (sm + 1) / n_sm;
+            long long a = cut[sm], b = cut[sm + 1];
             long long base = 0;
             for (auto& s : segs) {
                 long long lo = std::max(a, base), hi = std::min(b, base + s.rows);
@@ -136,6 +150,7 @@ void fill_defaults(mk_options* o) {
     if (o->l2_prefetch < 0) o->l2_prefetch = 0;
     if (o->prefetch_ahead < 0) o->prefetch_ahead = 0;
     if (o->prefetch_max_bytes <= 0) o->prefetch_max_bytes = 1 << 20;
+    if (o->attn_sm_ffn_permille <= 0) o->attn_sm_ffn_permille = 950;
     if (o->spin_limit_ns == 0) o->spin_limit_ns = 2000000000ull;
 }
 
@@ -150,6 +165,7 @@ int check_options(const mk_config& c, const mk_options& o) {
         return MK_ERR_UNSUPPORTED;
     if (2LL * 2 * c.head_dim > sb) return MK_ERR_UNSUPPORTED;
     if (o.kv_splits < 0 || (long long)o.kv_splits * c.n_q_heads > kMaxMergeSlots) return MK_ERR_INVALID_ARG;
+    if (o.attn_sm_ffn_permille < 0 || o.attn_sm_ffn_permille > 4000) return MK_ERR_INVALID_ARG;
     if (o.mode < MK_MODE_MEGAKERNEL || o.mode > MK_MODE_MULTI_KERNEL_GRAPH) return MK_ERR_INVALID_ARG;
     // ring + barriers + partial-sum slots + misc must fit the 227 KB per-block opt-in limit
     if ((long long)o.ring_stages * o.stage_bytes + 16LL * o.ring_stages + 128 + 4LL * kRowSlots * 8 + 512 > 232448)
@@ -185,7 +201,8 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     };
     const int qd = c.n_q_heads * d;
     auto op_cap = [&](int op) { return std::min(cap, kRowSlots / acc_sets(op, H, qd, F, c.top_k)); };
-    auto gemv_op = [&](int op, int layer, const std::vector<Segment>& segs, int wait, int signal) {
+    auto gemv_op = [&](int op, int layer, const std::vector<Segment>& segs, int wait, int signal,
+                       const std::vector<double>* weight = nullptr) {
         split_rows(segs, n_sm, op_cap(op), [&](int sm, int sub, int b, int e) {
             Instr w = blank();
             w[W_OP] = op;
@@ -196,7 +213,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
             w[W_WAIT_CTR] = wait;
             w[W_SIGNAL_CTR] = signal;
             add(sm, w);
-        });
+        }, weight);
     };
 
     for (int l = 0; l < L; ++l) {
@@ -205,6 +222,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
                 ctr_id(l, C_QKV));
         // attention: kv head g, split s -> instruction k = g * S + s, rotated per layer
         const int total = nkv * S;
+        std::vector<double> ffn_weight(n_sm, 1.0);  // blocks with an attention split take fewer FFN rows
         for (int k = 0; k < total; ++k) {
             Instr w = blank();
             w[W_OP] = OP_ATTN;
@@ -216,13 +234,14 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
             w[W_SIGNAL_CTR] = ctr_id(l, C_ATTN);
             int sm = (int)(((long long)k + (long long)l * total) % n_sm);
             add(sm, w);
+            ffn_weight[sm] = o.attn_sm_ffn_permille / 1000.0;
         }
         gemv_op(OP_OPROJ_RES, l, {{0, H}}, ctr_id(l, C_ATTN), ctr_id(l, C_OPROJ));
         std::vector<Segment> slots;
         for (int s = 0; s < (moe ? c.top_k : 1); ++s) slots.push_back({s, F});
         if (fused) {
             // one instruction per block: its up/gate rows, then the matching down-projection columns
-            gemv_op(moe ? OP_MOE_FFN : OP_FFN, l, slots, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN2));
+            gemv_op(moe ? OP_MOE_FFN : OP_FFN, l, slots, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN2), &ffn_weight);
         } else if (!moe) {
             gemv_op(OP_RMS_UPGATE_SILU, l, slots, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN1));
             gemv_op(OP_DOWN_RES, l, {{0, H}}, ctr_id(l, C_FFN1), ctr_id(l, C_FFN2));

@@ -216,3 +216,18 @@ def test_kv_splits_limit_is_checked():
     with pytest.raises(mk.MkError) as e:
         dpb.plan(cfg, 148, kv_splits=65)
     assert e.value.name == "MK_ERR_INVALID_ARG"
+
+
+@pytest.mark.parametrize("permille", [950, 1000, 800])
+def test_attention_blocks_take_fewer_ffn_rows(permille):
+    cfg = configs.LLAMA_1B
+    words, n_instr, _ = dpb.plan(cfg, 148, attn_sm_ffn_permille=permille)
+    for l in (0, 1):
+        attn_sms = {sm for sm in range(148) for w in words[sm, :n_instr[sm]]
+                    if w[W_OP] == OP["ATTN"] and w[W_LAYER] == l}
+        rows = {sm: int(w[W_END] - w[W_BEGIN]) for sm in range(148) for w in words[sm, :n_instr[sm]]
+                if w[W_OP] == OP["FFN"] and w[W_LAYER] == l}
+        assert sum(rows.values()) == cfg.ffn and len(rows) == 148
+        a = np.mean([rows[s] for s in attn_sms])
+        b = np.mean([rows[s] for s in rows if s not in attn_sms])
+        assert a / b == pytest.approx(permille / 1000, abs=0.03)
