@@ -150,7 +150,7 @@ void fill_defaults(mk_options* o) {
     if (o->l2_prefetch < 0) o->l2_prefetch = 0;
     if (o->prefetch_ahead < 0) o->prefetch_ahead = 0;
     if (o->prefetch_max_bytes <= 0) o->prefetch_max_bytes = 1 << 20;
-    if (o->attn_sm_ffn_permille <= 0) o->attn_sm_ffn_permille = 950;
+    if (o->attn_sm_ffn_permille <= 0) o->attn_sm_ffn_permille = 1000;
     if (o->spin_limit_ns == 0) o->spin_limit_ns = 2000000000ull;
 }
 

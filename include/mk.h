@@ -112,7 +112,8 @@ typedef struct {
                              places ahead in their queue (-1 default, 0 = off) */
     int prefetch_max_bytes; /* cap on the bytes prefetched per instruction (0 = default 1 MiB) */
     int attn_sm_ffn_permille; /* fused-FFN rows of a block that also runs an attention split of the
-                             layer, per mille of an even share (0 = default 950; 1000 = even split) */
+                             layer, per mille of an even share (0 = default 1000: even split; 950
+                             measured slower on the Llama-1B shape) */
     int split_ffn;        /* 0 (default): each layer's FFN is one fused instruction per SM (up/gate rows,
                              then the matching columns of w_down, streamed from a transposed copy the
                              library keeps, added into the residual with atomics: fp32 summation order
