@@ -228,6 +228,23 @@ def oracle_steps(cfg, seconds: float, max_steps: int | None = None, min_steps: i
     return times, oracle.num_threads()
 
 
+def single_thread_oracle_ms(args, steps: int = 2):
+    """ms/token of the fp64 oracle on one host thread (OMP_NUM_THREADS=1, a
+    child process), over `steps` decode steps of the workload."""
+    code = ("import sys, json; sys.path.insert(0, %r); import bench, statistics; "
+            "a = bench.parse(); cfg, p0, pos = bench.workload(a); "
+            "t, c = bench.oracle_steps(cfg, 0, max_steps=%d); "
+            "print(json.dumps([statistics.fmean(t) * 1e3, c]))") % (ROOT, steps)
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    argv = [sys.executable, "-c", code, "--config", args.config] + (["--layers", str(args.layers)] if args.layers else [])
+    try:
+        out = subprocess.run(argv, env=env, capture_output=True, text=True, timeout=300)
+        ms, cores = json.loads(out.stdout.strip().splitlines()[-1])
+        return round(ms, 1) if cores == 1 else None
+    except Exception:
+        return None
+
+
 def bytes_per_token(cfg, positions):
     return cfg.weight_bytes_per_token() + statistics.fmean(cfg.kv_bytes_per_token(p) for p in positions)
 
@@ -317,6 +334,9 @@ def run_ours(args, rank, world, local):
         cpu = {"value": round(statistics.fmean(times) * 1e6, 1), "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{len(times)} fp64 oracle decode steps of {cfg.name} at positions {p0}..",
                "ms_per_token": round(statistics.fmean(times) * 1e3, 2)}
+        single = single_thread_oracle_ms(args)
+        if single is not None:
+            cpu["single_thread_ms_per_token"] = single
 
     if rank != 0:
         return None

@@ -311,7 +311,7 @@ int mk_build_schedule(mk_handle* h) {
     if (plan.n_lm > h->lm_slots) return MK_ERR_SCHEDULE;
     if (plan.fused_ffn && h->cfg.n_layers > 0 && !h->down_t) return MK_ERR_SCHEDULE;
     h->plan = plan;
-    h->variant = mk::megakernel_variant(h->p, plan.fused_ffn);
+    h->variant = h->opt.general_kernel ? 0 : mk::megakernel_variant(h->p, plan.fused_ffn);
     int32_t* words = nullptr;
     int32_t* n_instr = nullptr;
     if ((rc = dalloc(h, &words, plan.words.size()))) return rc;

@@ -44,7 +44,7 @@ class MkOptions(ctypes.Structure):
     _fields_ = [("ring_stages", _I), ("stage_bytes", _I), ("rows_per_instr", _I), ("kv_splits", _I),
                 ("l2_prefetch", _I), ("trace", _I), ("snapshots", _I), ("spin_limit_ns", ctypes.c_ulonglong),
                 ("mode", _I), ("n_sm", _I), ("prefetch_ahead", _I), ("prefetch_max_bytes", _I),
-                ("attn_sm_ffn_permille", _I), ("split_ffn", _I)]
+                ("attn_sm_ffn_permille", _I), ("general_kernel", _I), ("split_ffn", _I)]
 
 
 class MkStatus(ctypes.Structure):

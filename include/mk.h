@@ -114,6 +114,8 @@ typedef struct {
     int attn_sm_ffn_permille; /* fused-FFN rows of a block that also runs an attention split of the
                              layer, per mille of an even share (0 = default 1000: even split; 950
                              measured slower on the Llama-1B shape) */
+    int general_kernel;   /* 1: always run the general kernel instantiation (ablations; default 0 picks the
+                             specialised one when the schedule allows it) */
     int split_ffn;        /* 0 (default): each layer's FFN is one fused instruction per SM (up/gate rows,
                              then the matching columns of w_down, streamed from a transposed copy the
                              library keeps, added into the residual with atomics: fp32 summation order
