@@ -11,6 +11,8 @@ Prints ONE JSON line (rank 0):
   e2e              the same metric through the C ABI with a host round trip
                    per step (token in by value, next token + status read back
                    from device to pinned host memory, synchronised)
+  e2e_serve        the same through launch-once serving (mk_serve_step): one
+                   resident grid, each step a mailbox round trip
   roofline         algorithmic bytes per token / mean launch duration vs the
                    measured HBM copy bandwidth
   cpu_baseline     the fp64 oracle on this host's cores, bounded sample
@@ -319,6 +321,28 @@ def run_ours(args, rank, world, local):
         e2e = {"value": round(e2e_s * 1e6 / (K * world), 3), "unit": UNIT, "h2d_bytes_per_step": 4,
                "d2h_bytes_per_step": 64}
 
+    # launch-once serving through the C ABI: the grid stays resident, each step is one
+    # mailbox round trip (token and pos in, next token and status out, pinned host memory)
+    e2e_serve = None
+    if not args.no_e2e and args.mode == "megakernel":
+        torch.cuda.synchronize()
+        dec.serve_start()
+        try:
+            tok = dec.serve_step(first, positions[0])
+            barrier(world)
+            t0 = time.perf_counter()
+            for i in range(K):
+                tok = dec.serve_step(tok, positions[i % len(positions)])
+            t1 = time.perf_counter()
+        finally:
+            dec.serve_stop()
+        st = dec.status()
+        if st["code"] != 0:
+            raise RuntimeError(f"device status after served steps: {st}")
+        e2e_serve = {"value": round(reduce_max(t1 - t0, world) * 1e6 / (K * world), 3), "unit": UNIT,
+                     "h2d_bytes_per_step": 16, "d2h_bytes_per_step": 12,
+                     "path": "mk_serve_step (resident grid, pinned mailbox)"}
+
     baselines = {}
     if not args.no_baselines and args.mode == "megakernel":
         for name, m in (("multi_kernel", 1), ("multi_kernel_graph", 2)):
@@ -357,6 +381,7 @@ def run_ours(args, rank, world, local):
                      "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
                      "traffic": committed_traffic(cfg.name, args.mode), "launch_us": round(launch_ms * 1000, 2)},
         "e2e": e2e,
+        "e2e_serve": e2e_serve,
         "gpu_launches": K if args.mode == "megakernel" else None,
         "baselines": baselines,
         "cpu_baseline": cpu,

@@ -3,6 +3,7 @@
 // and the debug getters.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <chrono>
 #include <cmath>
 #include <cstring>
@@ -32,6 +33,14 @@ struct mk_handle {
     cudaGraphExec_t graph_exec = nullptr;
     int lm_slots = 0;
     int variant = 0;  // megakernel instantiation for the built schedule
+    // launch-once serving
+    mk::ServeBox* box_host = nullptr;  // pinned, mapped
+    mk::ServeBox* box_dev = nullptr;
+    mk::ServeStep* serve_step = nullptr;
+    uint32_t* serve_ctr = nullptr;
+    cudaEvent_t ev_serve = nullptr;
+    bool serving = false;
+    int32_t serve_seq = 0;  // requests answered since mk_serve_start
     bool down_t = false;  // transposed down-projection copies exist (fused FFN schedules)
     int last_cuda = 0;
     int last_error = MK_OK;
@@ -249,6 +258,8 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     float2* rope = nullptr;
     if ((rc = dalloc(h, &rope, (size_t)c.max_seq * (d / 2)))) return fail(rc);
     if ((rc = dalloc(h, &h->stepbuf, 1))) return fail(rc);
+    if ((rc = dalloc(h, &h->serve_step, 1))) return fail(rc);
+    if ((rc = dalloc(h, &h->serve_ctr, 1))) return fail(rc);
     // The fused FFN streams the down-projection by its input index: keep a
     // transposed copy [ffn][hidden] of every w_down (library-owned).
     if (o.mode == MK_MODE_MEGAKERNEL && mk::ffn_fused(c, o)) {
@@ -286,7 +297,8 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     e = cudaMallocHost(&h->status_pinned, sizeof(mk::DevStatus));
     if (e != cudaSuccess) { h->last_cuda = e; h->status_pinned = nullptr; return fail(MK_ERR_CUDA); }
     if (cudaEventCreate(&h->ev0) || cudaEventCreate(&h->ev1) ||
-        cudaEventCreateWithFlags(&h->ev_done, cudaEventDisableTiming))
+        cudaEventCreateWithFlags(&h->ev_done, cudaEventDisableTiming) ||
+        cudaEventCreateWithFlags(&h->ev_serve, cudaEventDisableTiming))
         return fail(MK_ERR_CUDA);
 
     if (o.mode == MK_MODE_MEGAKERNEL) {
@@ -303,7 +315,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
 }
 
 int mk_build_schedule(mk_handle* h) {
-    if (!h) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving) return MK_ERR_INVALID_ARG;
     mk::Planned plan;
     int rc = mk::plan_schedule(h->cfg, h->opt, h->n_sm, &plan);
     if (rc) return rc;
@@ -342,7 +354,7 @@ int mk_get_schedule(mk_handle* h, int32_t* buf, size_t cap, size_t* n_words, int
 }
 
 int mk_decode_step(mk_handle* h, int32_t token, int32_t pos, float* logits_dev, int32_t* next_token_host) {
-    if (!h) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving) return MK_ERR_INVALID_ARG;
     if (token >= h->cfg.vocab || pos < 0 || pos >= h->cfg.max_seq) return MK_ERR_INVALID_ARG;
     if (!h->scheduled) return MK_ERR_NO_SCHEDULE;
     if (token < 0) token = -1;
@@ -394,7 +406,7 @@ int mk_decode_step(mk_handle* h, int32_t token, int32_t pos, float* logits_dev, 
 }
 
 int mk_get_hidden(mk_handle* h, int layer, float* out_host) {
-    if (!h || !out_host || layer < 0 || layer > h->cfg.n_layers || !h->p.snap) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving || !out_host || layer < 0 || layer > h->cfg.n_layers || !h->p.snap) return MK_ERR_INVALID_ARG;
     CK(cudaStreamSynchronize(h->stream));
     CK(cudaMemcpy(out_host, h->p.snap + (size_t)layer * h->cfg.hidden, sizeof(float) * h->cfg.hidden,
                   cudaMemcpyDeviceToHost));
@@ -402,7 +414,7 @@ int mk_get_hidden(mk_handle* h, int layer, float* out_host) {
 }
 
 int mk_get_router(mk_handle* h, int layer, int32_t* idx, float* wts) {
-    if (!h || !idx || !wts || h->cfg.n_experts <= 0 || layer < 0 || layer >= h->cfg.n_layers)
+    if (!h || h->serving || !idx || !wts || h->cfg.n_experts <= 0 || layer < 0 || layer >= h->cfg.n_layers)
         return MK_ERR_INVALID_ARG;
     CK(cudaStreamSynchronize(h->stream));
     CK(cudaMemcpy(idx, h->p.router_idx + (size_t)layer * mk::kMaxTopK, sizeof(int32_t) * h->cfg.top_k,
@@ -413,7 +425,7 @@ int mk_get_router(mk_handle* h, int layer, int32_t* idx, float* wts) {
 }
 
 int mk_get_counters(mk_handle* h, uint32_t* out, size_t cap, size_t* n) {
-    if (!h) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving) return MK_ERR_INVALID_ARG;
     if (n) *n = (size_t)h->p.n_ctr;
     if (!out) return MK_OK;
     if (cap < (size_t)h->p.n_ctr) return MK_ERR_CAPACITY;
@@ -433,7 +445,7 @@ int mk_get_counter_increments(mk_handle* h, uint32_t* out, size_t cap, size_t* n
 }
 
 int mk_get_status(mk_handle* h, mk_status* out) {
-    if (!h || !out) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving || !out) return MK_ERR_INVALID_ARG;
     mk::DevStatus st;
     int rc = read_status(h, &st);
     if (rc) return rc;
@@ -449,7 +461,7 @@ int mk_get_status(mk_handle* h, mk_status* out) {
 }
 
 int mk_get_trace(mk_handle* h, uint64_t* out, size_t cap, size_t* n) {
-    if (!h || !h->p.trace) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving || !h->p.trace) return MK_ERR_INVALID_ARG;
     const size_t cnt = (size_t)h->plan.n_sm * h->plan.max_instr * mk::kTraceWords;
     if (n) *n = cnt;
     if (!out) return MK_OK;
@@ -460,7 +472,7 @@ int mk_get_trace(mk_handle* h, uint64_t* out, size_t cap, size_t* n) {
 }
 
 int mk_reset(mk_handle* h) {
-    if (!h) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving) return MK_ERR_INVALID_ARG;
     CK(cudaStreamSynchronize(h->stream));
     CK(cudaMemset(h->p.counters, 0, sizeof(uint32_t) * h->p.n_ctr));
     CK(cudaMemset(h->p.status, 0, sizeof(mk::DevStatus)));
@@ -471,7 +483,7 @@ int mk_reset(mk_handle* h) {
 }
 
 int mk_inject_fault(mk_handle* h, int kind, int arg) {
-    if (!h) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving) return MK_ERR_INVALID_ARG;
     if (kind == MK_FAULT_NONE) return mk_reset(h);
     if (kind == MK_FAULT_PRESET_STOP) {
         const int one = 1;
@@ -502,7 +514,7 @@ int mk_inject_fault(mk_handle* h, int kind, int arg) {
 }
 
 int mk_last_step_ns(mk_handle* h, double* ns) {
-    if (!h || !ns) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving || !ns) return MK_ERR_INVALID_ARG;
     CK(cudaEventSynchronize(h->ev1));
     float ms = 0.f;
     CK(cudaEventElapsedTime(&ms, h->ev0, h->ev1));
@@ -510,8 +522,109 @@ int mk_last_step_ns(mk_handle* h, double* ns) {
     return MK_OK;
 }
 
+// ---- launch-once serving ---------------------------------------------------------------
+namespace {
+double host_wait_limit_s(const mk_handle* h) {
+    return std::max(10.0, 4.0 * (double)h->opt.spin_limit_ns * 1e-9);
+}
+void post_request(mk_handle* h, int32_t token, int32_t pos, int32_t stop, int32_t seq) {
+    volatile mk::ServeBox* b = h->box_host;
+    b->token = token;
+    b->pos = pos;
+    b->stop = stop;
+    std::atomic_thread_fence(std::memory_order_seq_cst);
+    b->req_seq = seq;  // the grid reads the other fields after it sees this
+    std::atomic_thread_fence(std::memory_order_seq_cst);
+}
+// The serving grid has left (launch complete): collect its status.
+int serve_ended(mk_handle* h) {
+    h->serving = false;
+    mk::DevStatus st;
+    int rc = read_status(h, &st);
+    if (rc) return rc;
+    return st.code != MK_OK ? st.code : MK_ERR_STOPPED;
+}
+}  // namespace
+
+int mk_serve_start(mk_handle* h, float* logits_dev) {
+    if (!h || h->serving || h->opt.mode != MK_MODE_MEGAKERNEL) return MK_ERR_INVALID_ARG;
+    if (!h->scheduled) return MK_ERR_NO_SCHEDULE;
+    if (!h->box_host) {
+        void* ptr = nullptr;
+        cudaError_t e = cudaHostAlloc(&ptr, sizeof(mk::ServeBox), cudaHostAllocMapped);
+        if (e != cudaSuccess) return cuda_fail(h, e);
+        h->box_host = static_cast<mk::ServeBox*>(ptr);
+        void* dptr = nullptr;
+        e = cudaHostGetDevicePointer(&dptr, ptr, 0);
+        if (e != cudaSuccess) return cuda_fail(h, e);
+        h->box_dev = static_cast<mk::ServeBox*>(dptr);
+    }
+    std::memset(h->box_host, 0, sizeof(mk::ServeBox));
+    CK(cudaMemsetAsync(h->serve_ctr, 0, sizeof(uint32_t), h->stream));
+    CK(cudaMemsetAsync(h->serve_step, 0, sizeof(mk::ServeStep), h->stream));
+    mk::DevParams p = h->p;
+    p.serve_box = h->box_dev;
+    p.serve_step = h->serve_step;
+    p.serve_ctr = h->serve_ctr;
+    p.serve_idle_ns = h->opt.serve_idle_ns;
+    mk::StepArgs a;
+    a.token = 0;
+    a.pos = 0;
+    a.epoch = h->epoch;  // request k runs epoch + k
+    a.logits = logits_dev ? logits_dev : h->p.logits;
+    a.serve = 1;
+    a.seq = 0;
+    CK(mk::launch_megakernel(p, a, h->n_sm, h->variant, h->stream));
+    CK(cudaEventRecord(h->ev_serve, h->stream));
+    h->serving = true;
+    h->serve_seq = 0;
+    return MK_OK;
+}
+
+int mk_serve_step(mk_handle* h, int32_t token, int32_t pos, int32_t* next_token_host) {
+    if (!h || !h->serving) return MK_ERR_INVALID_ARG;
+    if (token >= h->cfg.vocab || pos < 0 || pos >= h->cfg.max_seq) return MK_ERR_INVALID_ARG;
+    if (token < 0) token = -1;
+    if (cudaEventQuery(h->ev_serve) != cudaErrorNotReady) return serve_ended(h);
+    const int32_t seq = h->serve_seq + 1;
+    post_request(h, token, pos, 0, seq);
+    volatile mk::ServeBox* b = h->box_host;
+    const double limit_s = host_wait_limit_s(h);
+    const auto t0 = std::chrono::steady_clock::now();
+    for (long it = 0;; ++it) {
+        if (b->resp_seq == seq) break;
+        if ((it & 1023) == 1023) {
+            if (cudaEventQuery(h->ev_serve) != cudaErrorNotReady) {
+                if (b->resp_seq == seq) break;
+                return serve_ended(h);
+            }
+            if (std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count() > limit_s)
+                return MK_ERR_TIMEOUT;
+        }
+    }
+    std::atomic_thread_fence(std::memory_order_seq_cst);
+    h->serve_seq = seq;
+    h->epoch++;
+    if (next_token_host) *next_token_host = b->next_token;
+    return b->code;
+}
+
+int mk_serve_stop(mk_handle* h) {
+    if (!h) return MK_ERR_INVALID_ARG;
+    if (!h->serving) return MK_OK;
+    post_request(h, 0, 0, 1, h->serve_seq + 1);
+    int rc = wait_event(h, h->ev_serve);
+    h->serving = false;
+    if (rc) return rc;
+    mk::DevStatus st;
+    rc = read_status(h, &st);
+    if (rc) return rc;
+    return st.code;
+}
+
 void mk_destroy(mk_handle* h) {
     if (!h) return;
+    if (h->serving) mk_serve_stop(h);
     cudaStreamSynchronize(h->stream);
     if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
     if (h->graph) cudaGraphDestroy(h->graph);
@@ -520,6 +633,8 @@ void mk_destroy(mk_handle* h) {
     if (h->ev0) cudaEventDestroy(h->ev0);
     if (h->ev1) cudaEventDestroy(h->ev1);
     if (h->ev_done) cudaEventDestroy(h->ev_done);
+    if (h->ev_serve) cudaEventDestroy(h->ev_serve);
+    if (h->box_host) cudaFreeHost(h->box_host);
     delete h;
 }
 

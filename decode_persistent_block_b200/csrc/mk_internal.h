@@ -112,6 +112,22 @@ struct DevStatus {
     int pad[6];
 };
 
+// Launch-once serving (mk_serve_*): mailbox in pinned, mapped host memory.
+struct ServeBox {
+    int32_t req_seq;    // host -> device: number of the request (1, 2, ...), written last
+    int32_t token;      // < 0: the previous step's argmax
+    int32_t pos;
+    int32_t stop;       // 1: leave the grid instead of stepping
+    int32_t resp_seq;   // device -> host: number of the last finished request, written last
+    int32_t next_token;
+    int32_t code;       // device status code after the step (MK_OK or MK_ERR_*)
+    int32_t pad;
+};
+// The step a serving grid runs next, published in device memory by block 0.
+struct ServeStep {
+    int32_t token, pos, stop, pad;
+};
+
 // Everything the kernels read that stays fixed for a handle (device memory).
 struct DevParams {
     // model
@@ -154,6 +170,11 @@ struct DevParams {
     int prefetch_ahead;
     int prefetch_max_bytes;
     unsigned long long spin_limit_ns;
+    // serving (only read when the launch's StepArgs.serve is set)
+    ServeBox* serve_box;     // device view of the pinned host mailbox
+    ServeStep* serve_step;   // [1]
+    uint32_t* serve_ctr;     // number of requests published so far in this launch
+    unsigned long long serve_idle_ns;  // block 0 leaves after this long without a request
 };
 
 // Per-launch arguments (passed by value).
@@ -162,6 +183,9 @@ struct StepArgs {
     int pos;
     uint32_t epoch;   // 1-based step count since the last reset
     float* logits;    // output logits (device)
+    int serve = 0;    // 1: launch-once serving; the step fields come from the mailbox, epoch is the
+                      // base (request k, counted from 1, runs epoch + k)
+    int seq = 0;      // serving: number of this step's request
 };
 
 }  // namespace mk

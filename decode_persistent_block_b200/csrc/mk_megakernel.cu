@@ -45,15 +45,25 @@ namespace mk {
 // ---------------------------------------------------------------------------
 constexpr int kScratchBytes = 4 * kRowSlots * kConsumerWarps;  // partial row sums; attention merge and router reuse it
 
+__device__ void serve_respond(const DevParams& p, const StepArgs& a, int next_token);
+
+// Key of one layer's routing in one step (steps share a launch when serving).
+__device__ __forceinline__ int route_key(uint32_t epoch, int layer, int n_layers) {
+    return (int)((epoch * (uint32_t)(n_layers + 1) + (uint32_t)layer) & 0x7FFFFFFFu);
+}
+
 struct Misc {
     float red[kConsumerWarps * 2];
     int redi[kConsumerWarps];
     int abort_flag;
-    int router_layer;  // layer whose routing is in eidx/ew (-1: none)
+    int router_layer;  // route_key(epoch, layer) of the routing in eidx/ew (-1: none)
     int eidx[kMaxTopK];
     float ew[kMaxTopK];
     int is_last;
     int pad[3];
+    // serving: the step block 0 published, as taken by this block's consumer thread 0
+    int s_go, s_token, s_pos, s_seq;
+    uint32_t s_epoch;
 };
 
 __host__ __device__ inline size_t smem_bars_off(int ns, int sb) { return (size_t)ns * sb; }
@@ -375,11 +385,11 @@ __device__ bool loader_plan(const DevParams& p, const StepArgs& a, const int32_t
     }
     if (needs_routing(w[W_OP])) {
         const int l = w[W_LAYER];
-        if (vload(&m.router_layer) != l) {
+        if (vload(&m.router_layer) != route_key(a.epoch, l, p.L)) {
             if (!block) return false;
             const uint64_t t0 = globaltimer_ns();
             uint64_t next = t0 + kStopPollNs;
-            while (vload(&m.router_layer) != l) {
+            while (vload(&m.router_layer) != route_key(a.epoch, l, p.L)) {
                 const uint64_t now = globaltimer_ns();
                 if (now >= next) {
                     if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
@@ -402,15 +412,24 @@ __device__ bool loader_plan(const DevParams& p, const StepArgs& a, const int32_t
 }
 
 // PF: the L2 prefetch cursor (options.l2_prefetch) is compiled in.
+// Ring position of the loader, kept across the steps of a serving launch.
+struct LoaderRing {
+    int slot = 0;
+    uint32_t phase = 0;
+    uint32_t used = 0, last_parity = 0;  // slots ever filled, parity of their last fill
+};
+
+// One step's queue; false if a wait gave up (the block is leaving).
 template <bool PF>
-__device__ void loader(const DevParams& p, const StepArgs& a, const int32_t* q, int n, unsigned char* ring,
-                       uint64_t* full, uint64_t* empty, Misc& m) {
+__device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, int n, unsigned char* ring,
+                       uint64_t* full, uint64_t* empty, Misc& m, LoaderRing& lr) {
     const int NS = p.ring_stages;
     const uint32_t SB = (uint32_t)p.stage_bytes;
     const int pf_stages = PF && p.l2_prefetch > 0 ? (int)((uint32_t)p.l2_prefetch / SB) : 0;
-    int slot = 0;
-    uint32_t phase = 0;
-    uint32_t used = 0, last_parity = 0;
+    int& slot = lr.slot;
+    uint32_t& phase = lr.phase;
+    uint32_t& used = lr.used;
+    uint32_t& last_parity = lr.last_parity;
     // L2 prefetch cursor: next (instruction, stage) to prefetch and its global stage index
     int pf_i = 0, pf_st = 0;
     long long pf_g = 0, g = 0;
@@ -465,12 +484,16 @@ __device__ void loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                 }
             }
         }
-        if (!ok) break;
+        if (!ok) return false;
     }
-    // drain: wait for the last copy issued into every used slot
-    for (int s = 0; s < NS; ++s) {
-        if (!((used >> s) & 1u)) continue;
-        const uint32_t par = (last_parity >> s) & 1u;
+    return true;
+}
+
+// Before the block leaves: wait (bounded) for the last copy issued into every used slot.
+__device__ void loader_drain(const DevParams& p, uint64_t* full, const LoaderRing& lr) {
+    for (int s = 0; s < p.ring_stages; ++s) {
+        if (!((lr.used >> s) & 1u)) continue;
+        const uint32_t par = (lr.last_parity >> s) & 1u;
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&full[s], par)) {
             if (globaltimer_ns() - t0 > p.spin_limit_ns) break;
@@ -642,7 +665,7 @@ __device__ __forceinline__ void dot8x2(const uint4 w, const float* v, float& a0,
 // experts, top-k (ties to the lower index), softmax over the selected.
 template <int J>
 __device__ void route(const DevParams& p, Misc& m, float* scratch, const uint16_t* wr, int layer, bool publish,
-                      float (&v)[J][8]) {
+                      float (&v)[J][8], uint32_t epoch) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.H, nch = K >> 3, E = p.E;
     for (int e = 0; e < E; ++e) {  // one expert row at a time: few live registers
         float a0 = 0.f, a1 = 0.f;
@@ -687,7 +710,7 @@ __device__ void route(const DevParams& p, Misc& m, float* scratch, const uint16_
             }
         }
         __threadfence_block();
-        vstore(&m.router_layer, layer);
+        vstore(&m.router_layer, route_key(epoch, layer, p.L));
     }
     cbar();
 }
@@ -807,8 +830,8 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     if (op == OP_OPROJ_RES) load_attn_merged<J, HOIST ? 8 : 4>(p, 0, kp, v);
     if (vsrc) load_vec<J>(vsrc, kp, v);
     // 3. routing (once per layer per block; the loader waits for it)
-    if (op == OP_MOE_UPGATE && vload(&m.router_layer) != l)
-        route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
+    if (op == OP_MOE_UPGATE && vload(&m.router_layer) != route_key(a.epoch, l, p.L))
+        route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v, a.epoch);
     if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
     if (!early) {
         int eidx[kMaxTopK];
@@ -961,6 +984,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
                             ci = m.redi[k];
                         }
                     p.status->next_token = ci;
+                    if (a.serve) serve_respond(p, a, ci);
                 }
             }
             break;
@@ -1003,8 +1027,8 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     float v[J][8];
     const uint16_t* const* wt = p.wt + (size_t)l * wt_stride(p.E);
     load_rms<J>(p, m, p.x, nullptr, wt[WT_FFN_NORM], v);
-    if (op == OP_MOE_FFN && vload(&m.router_layer) != l)
-        route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v);
+    if (op == OP_MOE_FFN && vload(&m.router_layer) != route_key(a.epoch, l, p.L))
+        route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v, a.epoch);
     if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
     if (!early) {
         int eidx[kMaxTopK];
@@ -1484,7 +1508,7 @@ __device__ void prefetch_instr(const DevParams& p, const StepArgs& a, const int3
     if (!instr_ok(p, w)) return;
     int eidx[kMaxTopK] = {0, 0};
     if (needs_routing(w[W_OP])) {
-        if (m.router_layer != w[W_LAYER]) return;
+        if (m.router_layer != route_key(a.epoch, w[W_LAYER], p.L)) return;
         eidx[0] = m.eidx[0];
         eidx[1] = m.eidx[1];
     }
@@ -1508,6 +1532,79 @@ __device__ void prefetch_instr(const DevParams& p, const StepArgs& a, const int3
         for (size_t off = (size_t)threadIdx.x * 128; off < bytes; off += (size_t)kConsumerThreads * 128)
             prefetch_line_l2(pl.tail_src + off);
     }
+}
+
+// ---------------------------------------------------------------------------
+// launch-once serving: the step hand-off
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int ld_sys_acquire(const int32_t* ptr) {
+    int v;
+    asm volatile("ld.acquire.sys.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+// Block 0's consumer thread 0: take request k + 1 from the host mailbox
+// (bounded by serve_idle_ns; past it the grid leaves as if stopped) and
+// publish it to every block.
+__device__ void serve_publish(const DevParams& p, Misc& m, uint32_t k) {
+    const ServeBox* box = p.serve_box;
+    int stop = 1, token = -1, pos = 0;
+    const uint64_t t0 = globaltimer_ns();
+    uint64_t next = t0 + kStopPollNs;
+    for (;;) {
+        if (ld_sys_acquire(&box->req_seq) == (int)(k + 1)) {
+            token = *(volatile const int32_t*)&box->token;
+            pos = *(volatile const int32_t*)&box->pos;
+            stop = *(volatile const int32_t*)&box->stop;
+            break;
+        }
+        const uint64_t now = globaltimer_ns();
+        if (now >= next) {
+            if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) break;
+            if (now - t0 > p.serve_idle_ns) break;  // idle: leave (stop = 1)
+            next = now + kStopPollNs;
+        }
+    }
+    p.serve_step->token = token;
+    p.serve_step->pos = pos;
+    p.serve_step->stop = stop;
+    signal_release(p.serve_ctr);
+}
+
+// Every block's consumer thread 0 and loader lane: wait (bounded) for request
+// k + 1 and fill the step's arguments; false when the grid is to leave.
+__device__ bool serve_take(const DevParams& p, Misc& m, uint32_t k, const StepArgs& a0, StepArgs& a) {
+    const uint32_t* ctr = p.serve_ctr;
+    const uint64_t t0 = globaltimer_ns();
+    uint64_t next = t0 + kStopPollNs;
+    const unsigned long long limit = p.serve_idle_ns + p.spin_limit_ns;
+    while ((int32_t)(ld_acquire_u32(ctr) - (k + 1)) < 0) {
+        const uint64_t now = globaltimer_ns();
+        if (now >= next) {
+            if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
+            if (now - t0 > limit) {
+                record_error(p.status, MK_ERR_TIMEOUT, blockIdx.x, -1, 0, -1, 0, k + 1);
+                return false;
+            }
+            next = now + kStopPollNs;
+        }
+    }
+    if (__ldcg(&p.serve_step->stop)) return false;
+    a = a0;
+    a.token = __ldcg(&p.serve_step->token);
+    a.pos = __ldcg(&p.serve_step->pos);
+    a.epoch = a0.epoch + k + 1;
+    a.seq = (int)(k + 1);
+    return a.pos >= 0 && a.pos < p.max_seq && a.token < p.V;
+}
+
+// The last LM-head arrival of a served step hands the result to the host.
+__device__ void serve_respond(const DevParams& p, const StepArgs& a, int next_token) {
+    ServeBox* box = p.serve_box;
+    *(volatile int32_t*)&box->next_token = next_token;
+    *(volatile int32_t*)&box->code = *(volatile int*)&p.status->code;
+    __threadfence_system();
+    *(volatile int32_t*)&box->resp_seq = a.seq;
 }
 
 // ---------------------------------------------------------------------------
@@ -1542,32 +1639,63 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
     const int n = p.n_instr[blockIdx.x];
     const int32_t* q = p.instr + (size_t)blockIdx.x * p.max_instr * W_NWORDS;
     if (warp == kConsumerWarps) {
-        if (lane == 0) loader<JF == 0>(p, a, q, n, smem, full, empty, m);
+        if (lane == 0) {
+            LoaderRing lr;
+            for (uint32_t k = 0;; ++k) {
+                StepArgs sa = a;
+                if (a.serve && !serve_take(p, m, k, a, sa)) break;
+                if (!loader<JF == 0>(p, sa, q, n, smem, full, empty, m, lr) || !a.serve) break;
+            }
+            loader_drain(p, full, lr);
+        }
         return;
     }
 
-    const int token = a.token >= 0 ? a.token : __ldcg(&p.status->next_token);
     int slot = 0;
     uint32_t phase = 0;
-    for (int i = 0; i < n; ++i) {
-        const int32_t* w = q + (size_t)i * W_NWORDS;
-        if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_START] = globaltimer_ns();
-        if (JF == 0 && p.prefetch_ahead > 0 && i + p.prefetch_ahead < n)
-            prefetch_instr(p, a, q + (size_t)(i + p.prefetch_ahead) * W_NWORDS, m);
-        bool ok;
-        if (!instr_ok(p, w) || token < 0 || token >= p.V) {
+    for (uint32_t k = 0;; ++k) {
+        StepArgs sa = a;
+        if (a.serve) {  // launch-once serving: one request per iteration
             if (tid == 0) {
-                record_error(p.status, MK_ERR_BAD_INSTR, blockIdx.x, i, w[W_OP], -1, (uint32_t)token, 0);
-                vstore(&m.abort_flag, 1);
+                if (blockIdx.x == 0) serve_publish(p, m, k);
+                StepArgs t = a;
+                const bool go = serve_take(p, m, k, a, t);
+                m.s_go = go ? 1 : 0;
+                m.s_token = t.token;
+                m.s_pos = t.pos;
+                m.s_seq = t.seq;
+                m.s_epoch = t.epoch;
             }
-            ok = false;
-        } else if (w[W_OP] == OP_ATTN) {
-            ok = attn_instr(p, a, w, i, smem, full, empty, scratch, m, slot, phase);
-        } else {
-            ok = gemv_dispatch<JF>(p, a, w, i, smem, full, empty, scratch, m, slot, phase, token);
+            cbar();
+            if (!m.s_go) break;
+            sa.token = m.s_token;
+            sa.pos = m.s_pos;
+            sa.seq = m.s_seq;
+            sa.epoch = m.s_epoch;
         }
-        if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_END] = globaltimer_ns();
-        if (!ok) break;
+        const int token = sa.token >= 0 ? sa.token : __ldcg(&p.status->next_token);
+        bool ok = true;
+        for (int i = 0; i < n; ++i) {
+            const int32_t* w = q + (size_t)i * W_NWORDS;
+            if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_START] = globaltimer_ns();
+            if (JF == 0 && p.prefetch_ahead > 0 && i + p.prefetch_ahead < n)
+                prefetch_instr(p, sa, q + (size_t)(i + p.prefetch_ahead) * W_NWORDS, m);
+            if (!instr_ok(p, w) || token < 0 || token >= p.V) {
+                if (tid == 0) {
+                    record_error(p.status, MK_ERR_BAD_INSTR, blockIdx.x, i, w[W_OP], -1, (uint32_t)token, 0);
+                    vstore(&m.abort_flag, 1);
+                }
+                ok = false;
+            } else if (w[W_OP] == OP_ATTN) {
+                ok = attn_instr(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
+            } else {
+                ok = gemv_dispatch<JF>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase, token);
+            }
+            if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_END] = globaltimer_ns();
+            if (!ok) break;
+        }
+        if (!ok || !a.serve) break;
+        cbar();  // every thread has read this request's fields before thread 0 takes the next
     }
     if (tid == 0) vstore(&m.abort_flag, 1);  // lets the loader stop early if it is still waiting
 }

@@ -152,6 +152,7 @@ void fill_defaults(mk_options* o) {
     if (o->prefetch_max_bytes <= 0) o->prefetch_max_bytes = 1 << 20;
     if (o->attn_sm_ffn_permille <= 0) o->attn_sm_ffn_permille = 1000;
     if (o->spin_limit_ns == 0) o->spin_limit_ns = 2000000000ull;
+    if (o->serve_idle_ns == 0) o->serve_idle_ns = 60000000000ull;
 }
 
 int check_options(const mk_config& c, const mk_options& o) {

@@ -44,7 +44,8 @@ class MkOptions(ctypes.Structure):
     _fields_ = [("ring_stages", _I), ("stage_bytes", _I), ("rows_per_instr", _I), ("kv_splits", _I),
                 ("l2_prefetch", _I), ("trace", _I), ("snapshots", _I), ("spin_limit_ns", ctypes.c_ulonglong),
                 ("mode", _I), ("n_sm", _I), ("prefetch_ahead", _I), ("prefetch_max_bytes", _I),
-                ("attn_sm_ffn_permille", _I), ("general_kernel", _I), ("split_ffn", _I)]
+                ("attn_sm_ffn_permille", _I), ("serve_idle_ns", ctypes.c_ulonglong), ("general_kernel", _I),
+                ("split_ffn", _I)]
 
 
 class MkStatus(ctypes.Structure):
@@ -78,6 +79,9 @@ SIGNATURES = {
     "mk_plan": (_I, [ctypes.POINTER(MkConfig), ctypes.POINTER(MkOptions), _I, _P, ctypes.c_size_t,
                      ctypes.POINTER(_I), _P, _P, ctypes.c_size_t, ctypes.POINTER(_I)]),
     "mk_simulate": (_I, [_P, _I, _I, _P, _P, _I, _I, ctypes.c_uint64, ctypes.POINTER(ctypes.c_longlong)]),
+    "mk_serve_start": (_I, [_P, _P]),
+    "mk_serve_step": (_I, [_P, ctypes.c_int32, ctypes.c_int32, _P]),
+    "mk_serve_stop": (_I, [_P]),
     "mk_attention_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I]),
     "mk_attention_decode": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]),
     "mk_attention_decode_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
@@ -240,6 +244,20 @@ class Decoder:
 
     def __exit__(self, *a):
         self.close()
+
+    # -- launch-once serving ---------------------------------------------------------
+    def serve_start(self, logits=None):
+        """Launch the resident grid; logits: optional CUDA fp32 tensor [vocab]."""
+        check(self.lib.mk_serve_start(self.h, _ptr(logits) if logits is not None else None), "mk_serve_start")
+
+    def serve_step(self, token: int, pos: int) -> int:
+        """Run one step on the resident grid; returns the next token."""
+        out = ctypes.c_int32(-1)
+        check(self.lib.mk_serve_step(self.h, int(token), int(pos), ctypes.byref(out)), "mk_serve_step")
+        return int(out.value)
+
+    def serve_stop(self):
+        check(self.lib.mk_serve_stop(self.h), "mk_serve_stop")
 
     # -- the step -------------------------------------------------------------------
     def step(self, token: int, pos: int, logits=None, sync: bool = True):

@@ -114,6 +114,8 @@ typedef struct {
     int attn_sm_ffn_permille; /* fused-FFN rows of a block that also runs an attention split of the
                              layer, per mille of an even share (0 = default 1000: even split; 950
                              measured slower on the Llama-1B shape) */
+    unsigned long long serve_idle_ns; /* launch-once serving: the grid leaves after this long without a
+                             request (default 60 s) */
     int general_kernel;   /* 1: always run the general kernel instantiation (ablations; default 0 picks the
                              specialised one when the schedule allows it) */
     int split_ffn;        /* 0 (default): each layer's FFN is one fused instruction per SM (up/gate rows,
@@ -198,6 +200,26 @@ int mk_get_trace(mk_handle *h, uint64_t *out, size_t cap, size_t *n);
 /* Clear counters, epoch, status and stop word and re-upload the schedule
  * (undoes mk_inject_fault).  Use after any failed step. */
 int mk_reset(mk_handle *h);
+
+/* ---- launch-once serving ---------------------------------------------------
+ * The persistent grid stays resident across decode steps: no launch per step.
+ * mk_serve_start launches it on the handle's stream (megakernel mode, schedule
+ * built).  Each mk_serve_step writes (token, pos) to a mailbox in pinned host
+ * memory and waits, bounded like mk_decode_step, until the grid has run that
+ * step and posted its next token (token < 0: the previous step's argmax).
+ * Logits go to the device buffer given at start (or the internal one); read
+ * them from another stream after mk_serve_step returns.  mk_serve_stop asks the
+ * grid to leave and waits for it.  The grid also leaves by itself after
+ * serve_idle_ns without a request; the next mk_serve_step then returns
+ * MK_ERR_STOPPED and mk_serve_start may be called again.  While serving, the
+ * calls that touch the device (step, reset, getters, fault injection, schedule
+ * rebuild) return MK_ERR_INVALID_ARG; mk_destroy stops the grid first.  Counters and KV positions continue across the serving
+ * and per-launch paths (same epoch rule).  The paper's launch-once server loop;
+ * errors: MK_ERR_INVALID_ARG, MK_ERR_STOPPED, MK_ERR_TIMEOUT, MK_ERR_BAD_INSTR,
+ * MK_ERR_CUDA. */
+int mk_serve_start(mk_handle *h, float *logits_dev);
+int mk_serve_step(mk_handle *h, int32_t token, int32_t pos, int32_t *next_token_host);
+int mk_serve_stop(mk_handle *h);
 
 /* Host-side fault injection for tests: MK_FAULT_* (see above).  The fault
  * applies from the next step until mk_reset.  `arg` selects the block for
