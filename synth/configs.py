@@ -89,8 +89,12 @@ MIXTRAL_8L = ModelConfig(name="mixtral8l", n_layers=8, hidden=4096, n_heads=32, 
                          ffn=14336, vocab=32000, n_experts=8, top_k=2, rope_theta=1000000.0,
                          prefill=1024, steps=64)
 
+# Beyond the sweep: long-context decode, the 1B shape with the cache pre-filled
+# to 32768 and 65536 positions (attention becomes a large share of the bytes).
+LONG_PREFILLS = (32768, 65536)
+
 ALL = {c.name: c for c in (TINY, LLAMA_1B, LLAMA_3B, MIXTRAL_8L)}
-for _p in SWEEP_PREFILLS:
+for _p in SWEEP_PREFILLS + LONG_PREFILLS:
     ALL[f"llama1b_kv{_p}"] = llama1b_sweep(_p)
 
 

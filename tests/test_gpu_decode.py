@@ -187,6 +187,11 @@ def test_llama3b(cuda):
     _full(configs.LLAMA_3B, 3)
 
 
+@pytest.mark.parametrize("prefill", configs.LONG_PREFILLS)
+def test_llama1b_long_context(cuda, prefill):
+    _full(configs.llama1b_sweep(prefill), 2)
+
+
 @pytest.mark.parametrize("prefill", configs.SWEEP_PREFILLS)
 def test_llama1b_kv_sweep(cuda, prefill):
     _full(configs.llama1b_sweep(prefill), 2)
