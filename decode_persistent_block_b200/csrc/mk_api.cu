@@ -10,6 +10,8 @@
 #include <thread>
 #include <vector>
 
+#include <cudaTypedefs.h>  // PFN_cuTensorMapEncodeTiled
+
 #include "mk_internal.h"
 #include "mk_kernels.h"
 #include "mk_plan.h"
@@ -101,6 +103,35 @@ int check_weights(const mk_config& c, const mk_weights* w) {
         if (L > 0 && !w->router) return MK_ERR_INVALID_ARG;
         for (int l = 0; l < L; ++l)
             if (!w->router[l] || !aligned16(w->router[l])) return MK_ERR_INVALID_ARG;
+    }
+    return MK_OK;
+}
+
+// Tensor maps over the K and V caches for the attention stages: rows of d bf16,
+// [n_layers * n_kv * max_seq] rows, boxes of 64 columns x attn_box_rows rows,
+// 128-byte swizzle.  The driver entry point is looked up through the runtime.
+int make_kv_maps(mk_handle* h, const mk_config& c, const mk_options& o, void* kcache, void* vcache) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(h, e != cudaSuccess ? e : cudaErrorNotSupported);
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const int d = c.head_dim;
+    const cuuint64_t rows = (cuuint64_t)std::max(c.n_layers, 1) * c.n_kv_heads * c.max_seq;
+    const cuuint64_t dims[2] = {(cuuint64_t)d, rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)mk::attn_box_rows(o.stage_bytes, d)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUtensorMap* maps[2] = {&h->p.kmap, &h->p.vmap};
+    void* bases[2] = {kcache, vcache};
+    for (int i = 0; i < 2; ++i) {
+        CUresult r = encode(maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, bases[i], dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return MK_ERR_UNSUPPORTED;
     }
     return MK_OK;
 }
@@ -301,6 +332,8 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
         cudaEventCreateWithFlags(&h->ev_serve, cudaEventDisableTiming))
         return fail(MK_ERR_CUDA);
 
+    if (o.mode == MK_MODE_MEGAKERNEL && L > 0 && (rc = make_kv_maps(h, c, o, w->k_cache, w->v_cache)))
+        return fail(rc);
     if (o.mode == MK_MODE_MEGAKERNEL) {
         int per_sm = 0;
         e = mk::prepare_megakernel(o.ring_stages, o.stage_bytes, &per_sm);

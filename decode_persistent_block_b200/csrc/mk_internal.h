@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <vector_types.h>
+#include <cuda.h>  // CUtensorMap (the KV-cache tensor maps travel in the kernel parameters)
 
 #include "../../include/mk.h"
 
@@ -128,8 +129,28 @@ struct ServeStep {
     int32_t token, pos, stop, pad;
 };
 
+// Rows of one attention ring stage: K and V of `rows` positions, 4 * d bytes
+// per position, at most 256, whole boxes of kAttnBoxRows rows (the tensor
+// maps' box height: a split loads only the boxes that hold its rows).
+constexpr int kAttnBoxRows = 64;
+MK_HD inline int attn_stage_rows(int stage_bytes, int d) {
+    int r = stage_bytes / (4 * d);
+    r = r >= kAttnBoxRows ? (r & ~(kAttnBoxRows - 1)) : (r & ~15);  // whole boxes, or whole 16-row tiles
+    return r < 256 ? r : 256;
+}
+// Box height of the tensor maps (at most one stage).
+MK_HD inline int attn_box_rows(int stage_bytes, int d) {
+    const int r = attn_stage_rows(stage_bytes, d);
+    return r < kAttnBoxRows ? r : kAttnBoxRows;
+}
+
 // Everything the kernels read that stays fixed for a handle (device memory).
 struct DevParams {
+    // 2-D tensor maps over the K and V caches, viewed as [n_layers * n_kv * max_seq][d] bf16
+    // rows, boxes of 64 columns x attn_box_rows rows, 128-byte swizzle (the attention
+    // stage's bank-conflict-free layout for ldmatrix)
+    CUtensorMap kmap;
+    CUtensorMap vmap;
     // model
     int L, H, nq, nkv, d, F, V, E, topk, max_seq;
     float eps;

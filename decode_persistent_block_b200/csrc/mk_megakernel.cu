@@ -207,6 +207,7 @@ struct Plan {
     int tail_rps, tail_spp;
     uint32_t tail_row_bytes;
     const unsigned char* tail_src;
+    int tma_row0;  // attention: first cache row of the split in the tensor maps' row space (-1: not attention)
 };
 
 struct AttnRange {
@@ -236,6 +237,7 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
     pl.tail_rps = pl.tail_spp = 0;
     pl.tail_row_bytes = 0;
     pl.tail_src = nullptr;
+    pl.tma_row0 = -1;
     const uint16_t* tail = nullptr;  // transposed down-projection rows of a fused FFN
     int K = p.H;
     const uint16_t* s0 = nullptr;
@@ -243,17 +245,18 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
     const uint16_t* s2 = nullptr;  // second slot's matrix (fused expert down-projection)
     switch (op) {
         case OP_ATTN: {
+            // K and V rows of the split, as tensor-map boxes (row coordinate tma_row0 + stage row)
             const AttnRange r = attn_range(pos, b, e);
             pl.nphase = 1;
             pl.nspan = 2;
             pl.rows = r.ncached;
             pl.row_bytes = pl.src_stride = (uint32_t)p.d * 2u;
-            pl.rps = (int)(SB / (2u * pl.row_bytes));
+            pl.rps = attn_stage_rows((int)SB, p.d);
             pl.spp = (pl.rows + pl.rps - 1) / pl.rps;
             pl.n_stages = pl.main_stages = pl.spp;
-            const size_t base = (((size_t)l * p.nkv + sub) * (size_t)p.max_seq + (size_t)r.jb) * (size_t)p.d;
-            pl.src[0][0] = (const unsigned char*)(p.kcache + base);
-            pl.src[0][1] = (const unsigned char*)(p.vcache + base);
+            pl.tma_row0 = (int)(((size_t)l * p.nkv + sub) * (size_t)p.max_seq + (size_t)r.jb);
+            pl.src[0][0] = (const unsigned char*)(p.kcache + (size_t)pl.tma_row0 * p.d);
+            pl.src[0][1] = (const unsigned char*)(p.vcache + (size_t)pl.tma_row0 * p.d);
             return;
         }
         case OP_RMS_QKV: s0 = wt[WT_Q + sub]; break;
@@ -327,7 +330,25 @@ __device__ __forceinline__ bool needs_routing(int op) {
 // ---------------------------------------------------------------------------
 // loader warp (one lane)
 // ---------------------------------------------------------------------------
-__device__ void issue_stage(const Plan& pl, int st, unsigned char* dst_stage, uint64_t* bar) {
+// TC: attention stages are tensor-map boxes (for attn_tc); otherwise contiguous
+// K and V spans (for attn_cc).
+template <bool TC>
+__device__ void issue_stage(const DevParams& p, const Plan& pl, int st, unsigned char* dst_stage, uint64_t* bar) {
+    if (TC && pl.tma_row0 >= 0) {  // attention: K and V in boxes of attn_box_rows rows (past the split: masked)
+        const int halves = p.d / 64, y = pl.tma_row0 + st * pl.rps;
+        const int nr = (pl.rows - st * pl.rps) < pl.rps ? (pl.rows - st * pl.rps) : pl.rps;
+        const int br = attn_box_rows(p.stage_bytes, p.d);  // divides pl.rps
+        const int nb = (nr + br - 1) / br;
+        const uint32_t half = (uint32_t)pl.rps * 128u, box = (uint32_t)br * 128u;
+        mbar_arrive_expect_tx(bar, 2u * (uint32_t)halves * (uint32_t)nb * box);
+        unsigned char* vdst = dst_stage + (size_t)pl.rps * p.d * 2;
+        for (int h = 0; h < halves; ++h)
+            for (int b = 0; b < nb; ++b) {
+                tma_load_2d(dst_stage + (size_t)h * half + (size_t)b * box, &p.kmap, 64 * h, y + b * br, bar);
+                tma_load_2d(vdst + (size_t)h * half + (size_t)b * box, &p.vmap, 64 * h, y + b * br, bar);
+            }
+        return;
+    }
     if (st >= pl.main_stages) {  // fused FFN: transposed down-projection rows
         const int r0 = (st - pl.main_stages) * pl.tail_rps;
         const int nr = (pl.rows - r0) < pl.tail_rps ? (pl.rows - r0) : pl.tail_rps;
@@ -420,7 +441,7 @@ struct LoaderRing {
 };
 
 // One step's queue; false if a wait gave up (the block is leaving).
-template <bool PF>
+template <bool PF, bool TC>
 __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, int n, unsigned char* ring,
                        uint64_t* full, uint64_t* empty, Misc& m, LoaderRing& lr) {
     const int NS = p.ring_stages;
@@ -448,7 +469,7 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                 ok = false;
                 break;
             }
-            issue_stage(pl, st, ring + (size_t)slot * SB, &full[slot]);
+            issue_stage<TC>(p, pl, st, ring + (size_t)slot * SB, &full[slot]);
             if (tr && st == 0) tr[T_LD_FIRST] = globaltimer_ns();
             if (tr && st == pl.n_stages - 1) tr[T_LD_LAST] = globaltimer_ns();
             used |= 1u << slot;
@@ -1175,7 +1196,12 @@ __device__ __forceinline__ void ml_combine(float& m, float& l, float* o, float m
 // half owns at most 2 of the kv head's query heads and streams every K/V row of
 // the stage for them), which keeps the per-thread q and output accumulators to
 // 2 x 8 + 2 x 8 registers.
-__device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
+// CUDA-core split attention (the general and head_dim-128 kernels): query
+// heads are split between the two halves of the consumer warps (each half owns
+// at most 2 of the kv head's query heads and streams every K/V row of the stage
+// for them), which keeps the per-thread q and output accumulators to 2 x 8 +
+// 2 x 8 registers.  The stage holds K then V rows, contiguous (bulk copies).
+__device__ bool attn_cc(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                            uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
     const int D = p.d;                                  // head_dim, 64 or 128
     const int LPR = D / 8;                              // lanes per K/V row, 8 columns each
@@ -1456,6 +1482,317 @@ __device__ bool attn_instr(const DevParams& p, const StepArgs& a, const int32_t*
     return true;
 }
 
+// Tensor-core split attention (the head_dim-64 kernel).  DH: head_dim fixed at
+// compile time.  The stage holds K then V rows in 128-byte-swizzled tensor-map
+// boxes.
+template <int DH>
+__device__ bool attn_tc(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
+                           uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
+    constexpr int DMAX = DH > 0 ? DH : kMaxHeadDim;
+    const int D = DH > 0 ? DH : p.d;                    // head_dim, 64 or 128
+    const int LPR = D / 8;                              // lanes per K/V row, 8 columns each
+    constexpr int GW = 2;                               // head slots per set
+    constexpr int SET_THREADS = kConsumerThreads / 2;
+    constexpr int SET_WARPS = kConsumerWarps / 2;
+    const int G = p.nq / p.nkv;                         // query heads per kv head (1..4)
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int set = warp / SET_WARPS;
+    const int stid = tid - set * SET_THREADS;
+    const int h0 = set * GW;                            // first query head (within the group) of this set
+    const int l = w[W_LAYER], g = w[W_SUB], c = w[W_BEGIN], S = w[W_END], pos = a.pos;
+    const uint32_t SB = (uint32_t)p.stage_bytes;
+    const AttnRange rg = attn_range(pos, c, S);
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
+    Plan pl;  // stage plan (weights only: computed while the dependency is still pending)
+    make_plan(p, pos, w, nullptr, pl);
+
+    if (tid == 0) {
+        if (!wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, OP_ATTN))
+            vstore(&m.abort_flag, 1);
+        if (tr) tr[T_DEP] = globaltimer_ns();
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+
+    // Prologue loads, all issued before any is used (one round trip): this
+    // thread's 8 columns (and their rotate-half partners) of q for the set's
+    // heads, of the new k and v, and the RoPE cos/sin of this position.
+    const int col0 = (stid % LPR) * 8;
+    const int pcol = col0 ^ (D / 2);
+    const bool first_half = col0 < D / 2;
+    const float qscale = 1.4426950408889634f / sqrtf((float)D);
+    const float4* rp4 = reinterpret_cast<const float4*>(p.rope + (size_t)pos * (D / 2) + (col0 & (D / 2 - 1)));
+    const float* ks = p.qkv + (size_t)p.nq * D + (size_t)g * D;
+    const float* vs = p.qkv + (size_t)(p.nq + p.nkv) * D + (size_t)g * D;
+    float4 qx[GW][2], qy[GW][2], rc[4], kx[2], ky[2], vx[2];
+#pragma unroll
+    for (int hh = 0; hh < GW; ++hh) {
+        const int h = h0 + hh < G ? h0 + hh : G - 1;  // spare head slots compute a copy that is never stored
+        const float4* src = reinterpret_cast<const float4*>(p.qkv + (size_t)(g * G + h) * D);
+        qx[hh][0] = __ldcg(src + col0 / 4);
+        qx[hh][1] = __ldcg(src + col0 / 4 + 1);
+        qy[hh][0] = __ldcg(src + pcol / 4);
+        qy[hh][1] = __ldcg(src + pcol / 4 + 1);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rc[k] = __ldg(rp4 + k);
+    kx[0] = __ldcg(reinterpret_cast<const float4*>(ks + col0));
+    kx[1] = __ldcg(reinterpret_cast<const float4*>(ks + col0) + 1);
+    ky[0] = __ldcg(reinterpret_cast<const float4*>(ks + pcol));
+    ky[1] = __ldcg(reinterpret_cast<const float4*>(ks + pcol) + 1);
+    vx[0] = __ldcg(reinterpret_cast<const float4*>(vs + col0));
+    vx[1] = __ldcg(reinterpret_cast<const float4*>(vs + col0) + 1);
+    float cs[8], sn[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        cs[2 * k] = rc[k].x;
+        sn[2 * k] = rc[k].y;
+        cs[2 * k + 1] = rc[k].z;
+        sn[2 * k + 1] = rc[k].w;
+    }
+    // rotate-half RoPE of one 8-column slice: x' = x cos - y sin (first half), x cos + y sin (second)
+    auto rope8 = [&](const float4 (&x)[2], const float4 (&y)[2], float scale, float* out) {
+        const float xv[8] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w};
+        const float yv[8] = {y[0].x, y[0].y, y[0].z, y[0].w, y[1].x, y[1].y, y[1].z, y[1].w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            out[k] = (first_half ? xv[k] * cs[k] - yv[k] * sn[k] : xv[k] * cs[k] + yv[k] * sn[k]) * scale;
+    };
+    float q[GW][8];
+#pragma unroll
+    for (int hh = 0; hh < GW; ++hh) rope8(qx[hh], qy[hh], qscale, q[hh]);
+
+    // the new position: rotated k and v rounded to bf16 (the cache format); the
+    // first row group of each set holds it, set 0 appends it to the cache
+    float kn[8], vn[8];
+    const bool new_rows = rg.has_new && stid < 32;  // first warp of each set
+    {
+        float kr[8];
+        rope8(kx, ky, 1.0f, kr);
+        const float vv[8] = {vx[0].x, vx[0].y, vx[0].z, vx[0].w, vx[1].x, vx[1].y, vx[1].z, vx[1].w};
+        uint32_t kb[8], vb[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            kb[k] = f2bf(kr[k]);
+            vb[k] = f2bf(vv[k]);
+            kn[k] = __uint_as_float(kb[k] << 16);
+            vn[k] = __uint_as_float(vb[k] << 16);
+        }
+        if (new_rows && set == 0 && stid < LPR) {
+            const size_t off = (((size_t)l * p.nkv + g) * (size_t)p.max_seq + (size_t)pos) * D + col0;
+            uint4 ku, vu;
+            ku.x = kb[0] | (kb[1] << 16); ku.y = kb[2] | (kb[3] << 16); ku.z = kb[4] | (kb[5] << 16); ku.w = kb[6] | (kb[7] << 16);
+            vu.x = vb[0] | (vb[1] << 16); vu.y = vb[2] | (vb[3] << 16); vu.z = vb[4] | (vb[5] << 16); vu.w = vb[6] | (vb[7] << 16);
+            *reinterpret_cast<uint4*>(p.kcache + off) = ku;
+            *reinterpret_cast<uint4*>(p.vcache + off) = vu;
+        }
+    }
+
+    // q (rotated, scaled) of every head of the group and the new k, v to shared
+    // memory: the tensor-core loop below takes its fragments from there
+    float* sm_o = scratch;                           // [8 warps][4][D]  per-warp outputs
+    float* sm_ml = scratch + kConsumerWarps * 512;   // [8 warps][4][2]  per-warp (max, sum)
+    float* sm_q = scratch + kConsumerWarps * 512 + 256;  // [4][D]
+    float* sm_kv = sm_q + 4 * kMaxHeadDim;               // [2][D] new k, v (bf16 values)
+    if (stid < LPR) {
+#pragma unroll
+        for (int hh = 0; hh < GW; ++hh)
+            if (h0 + hh < G)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) sm_q[(h0 + hh) * D + col0 + k] = q[hh][k];
+        if (set == 0)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                sm_kv[col0 + k] = kn[k];
+                sm_kv[D + col0 + k] = vn[k];
+            }
+    }
+    cbar();
+    if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
+
+    // Tensor-core split attention (mma m16n8k16, bf16 operands, fp32 accumulate).
+    // Row r = lane/4 of the 16-row operand is head r & 3, the high (r < 4) or low
+    // (r >= 4) bf16 part of q or of the probabilities, so hi + lo keeps fp32
+    // accuracy; rows 8..15 are zero.  Each warp takes 16-position tiles w, w+8, ...
+    // of every stage with its own online softmax (log2 domain); warps merge at the end.
+    const int g4 = lane >> 2, t4 = lane & 3;
+    const int hrow = g4 & 3;
+    const bool lo_row = g4 >= 4, real = hrow < G;
+    const int KS = D / 16, NT = D / 8;
+    uint32_t qa[DMAX / 16][2];
+#pragma unroll
+    for (int kk = 0; kk < DMAX / 16; ++kk) {
+        qa[kk][0] = qa[kk][1] = 0u;
+        if (kk < KS && real) {
+            float x[4];
+            const float* qr = sm_q + hrow * D + kk * 16 + 2 * t4;
+            x[0] = qr[0]; x[1] = qr[1]; x[2] = qr[8]; x[3] = qr[9];
+            uint32_t h16[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t hi = f2bf(x[k]);
+                h16[k] = lo_row ? f2bf(x[k] - __uint_as_float(hi << 16)) : hi;
+            }
+            qa[kk][0] = h16[0] | (h16[1] << 16);
+            qa[kk][1] = h16[2] | (h16[3] << 16);
+        }
+    }
+    float m_run = -CUDART_INF_F, l_run = 0.f;
+    float oacc[DMAX / 8][2];  // rows 0..7 of each 8-column output tile (this lane: row g4, 2 columns)
+#pragma unroll
+    for (int nt = 0; nt < DMAX / 8; ++nt) oacc[nt][0] = oacc[nt][1] = 0.f;
+
+    const int lm_i = lane >> 3, lm_j = lane & 7;  // ldmatrix: matrix index, row within it
+    for (int st = 0; st < pl.n_stages; ++st) {
+        const int r0 = st * pl.rps;
+        const int nr = (pl.rows - r0) < pl.rps ? (pl.rows - r0) : pl.rps;
+        const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, OP_ATTN);
+        if (tr && tid == 0 && st == 0) tr[T_FIRST] = globaltimer_ns();
+        if (ok) {
+            const uint32_t kbase = smem_u32(ring + (size_t)slot * SB);
+            const uint32_t vbase = kbase + (uint32_t)pl.rps * D * 2;
+            const uint32_t half_bytes = (uint32_t)pl.rps * 128u;
+            // byte offset of (row, column) in a 128-byte-swizzled stage: 16-byte chunk c of row r sits at c ^ (r & 7)
+            auto swz = [&](int row, int col) -> uint32_t {
+                return (uint32_t)(col >> 6) * half_bytes + (uint32_t)row * 128u +
+                       ((((uint32_t)(col & 63) >> 3) ^ ((uint32_t)row & 7u)) << 4);
+            };
+            const int ntiles = (nr + 15) >> 4;
+            for (int tile = warp; tile < ntiles; tile += kConsumerWarps) {
+                const int tb = tile * 16;
+                // scores: S[16 x 16 positions] = Q . K^T, two n-halves of 8 positions
+                float sc0[2] = {0.f, 0.f}, sc1[2] = {0.f, 0.f};
+#pragma unroll
+                for (int kk = 0; kk < DMAX / 16; ++kk) {
+                    if (kk >= KS) break;
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kbase + swz(tb + ((lm_i >> 1) << 3) + lm_j, kk * 16 + ((lm_i & 1) << 3)), b0, b1, b2, b3);
+                    mma_bf16_top(sc0[0], sc0[1], qa[kk][0], qa[kk][1], b0, b1);
+                    mma_bf16_top(sc1[0], sc1[1], qa[kk][0], qa[kk][1], b2, b3);
+                }
+                // this lane's 4 positions of row g4: tb + 2t4, +1, tb + 8 + 2t4, +1; hi + lo rows
+                float sv[4] = {sc0[0], sc0[1], sc1[0], sc1[1]};
+                const int pp[4] = {tb + 2 * t4, tb + 2 * t4 + 1, tb + 8 + 2 * t4, tb + 9 + 2 * t4};
+                float tmax = -CUDART_INF_F;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    sv[k] += __shfl_xor_sync(0xFFFFFFFFu, sv[k], 16);
+                    if (pp[k] >= nr) sv[k] = -CUDART_INF_F;
+                    tmax = fmaxf(tmax, sv[k]);
+                }
+                tmax = fmaxf(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, 1));
+                tmax = fmaxf(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, 2));
+                const float mn = fmaxf(m_run, tmax);  // finite: every tile has a valid position
+                const float al = exp2f(m_run - mn);
+                float pv[4], psum = 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    pv[k] = pp[k] < nr ? exp2f(sv[k] - mn) : 0.f;
+                    psum += pv[k];
+                }
+                psum += __shfl_xor_sync(0xFFFFFFFFu, psum, 1);
+                psum += __shfl_xor_sync(0xFFFFFFFFu, psum, 2);
+                l_run = fmaf(l_run, al, psum);
+                m_run = mn;
+                uint32_t ph[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t hi = f2bf(pv[k]);
+                    ph[k] = lo_row ? f2bf(pv[k] - __uint_as_float(hi << 16)) : hi;
+                }
+                const uint32_t pa0 = ph[0] | (ph[1] << 16), pa2 = ph[2] | (ph[3] << 16);
+#pragma unroll
+                for (int nt = 0; nt < DMAX / 8; ++nt) {
+                    oacc[nt][0] *= al;
+                    oacc[nt][1] *= al;
+                }
+                // O += P . V, two 8-column tiles per ldmatrix
+#pragma unroll
+                for (int n2 = 0; n2 < DMAX / 16; ++n2) {
+                    if (n2 >= KS) break;
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_trans(vbase + swz(tb + ((lm_i & 1) << 3) + lm_j, (2 * n2 + (lm_i >> 1)) * 8), b0, b1, b2, b3);
+                    mma_bf16_top(oacc[2 * n2][0], oacc[2 * n2][1], pa0, pa2, b0, b1);
+                    mma_bf16_top(oacc[2 * n2 + 1][0], oacc[2 * n2 + 1][1], pa0, pa2, b2, b3);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        } else if (tid == 0) {
+            vstore(&m.abort_flag, 1);
+        }
+        if (++slot == p.ring_stages) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    // the new position (its k, v are not in the cache stream): warp 0 adds it
+    if (warp == 0 && rg.has_new) {
+        float part = 0.f;
+        const int dq = D / 4;
+        for (int k = t4 * dq; k < (t4 + 1) * dq; ++k) part = fmaf(sm_q[(real ? hrow : 0) * D + k], sm_kv[k], part);
+        part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
+        part += __shfl_xor_sync(0xFFFFFFFFu, part, 2);
+        const float mn = fmaxf(m_run, part);
+        const float al = exp2f(m_run - mn), pr = exp2f(part - mn);
+        l_run = fmaf(l_run, al, pr);
+        m_run = mn;
+#pragma unroll
+        for (int nt = 0; nt < DMAX / 8; ++nt) {
+            if (nt >= NT) break;
+            const int col = nt * 8 + 2 * t4;
+            const float add0 = lo_row ? 0.f : pr * sm_kv[D + col], add1 = lo_row ? 0.f : pr * sm_kv[D + col + 1];
+            oacc[nt][0] = fmaf(oacc[nt][0], al, add0);
+            oacc[nt][1] = fmaf(oacc[nt][1], al, add1);
+        }
+    }
+    if (tr && tid == 0) tr[T_MAIN] = globaltimer_ns();
+
+    // hi + lo rows, then each warp's (max, sum, output) of every head to shared memory
+#pragma unroll
+    for (int nt = 0; nt < DMAX / 8; ++nt) {
+        oacc[nt][0] += __shfl_xor_sync(0xFFFFFFFFu, oacc[nt][0], 16);
+        oacc[nt][1] += __shfl_xor_sync(0xFFFFFFFFu, oacc[nt][1], 16);
+    }
+    cbar();  // the scratch held q and the new k, v until every warp was done with them
+    if (lane < 16 && real) {
+#pragma unroll
+        for (int nt = 0; nt < DMAX / 8; ++nt) {
+            if (nt >= NT) break;
+            sm_o[(warp * 4 + hrow) * D + nt * 8 + 2 * t4] = oacc[nt][0];
+            sm_o[(warp * 4 + hrow) * D + nt * 8 + 2 * t4 + 1] = oacc[nt][1];
+        }
+        if (t4 == 0) {
+            sm_ml[(warp * 4 + hrow) * 2] = m_run;
+            sm_ml[(warp * 4 + hrow) * 2 + 1] = l_run;
+        }
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+    for (int idx = tid; idx < G * D; idx += kConsumerThreads) {
+        const int h = idx / D, col = idx % D;
+        float M = -CUDART_INF_F;
+        for (int wv = 0; wv < kConsumerWarps; ++wv) M = fmaxf(M, sm_ml[(wv * 4 + h) * 2]);
+        float O = 0.f, Ls = 0.f;
+        if (M != -CUDART_INF_F) {
+            for (int wv = 0; wv < kConsumerWarps; ++wv) {
+                const float f = exp2f(sm_ml[(wv * 4 + h) * 2] - M);
+                O += f * sm_o[(wv * 4 + h) * D + col];
+                Ls += f * sm_ml[(wv * 4 + h) * 2 + 1];
+            }
+        }
+        const size_t part = (size_t)(g * G + h) * S + c;
+        p.part_o[part * D + col] = O;
+        if (col == 0) {
+            p.part_ml[part * 2] = M;
+            p.part_ml[part * 2 + 1] = Ls;
+        }
+    }
+    cbar();
+    if (tid == 0) signal_release(p.counters + w[W_SIGNAL_CTR]);
+    return true;
+}
+
 __device__ __forceinline__ int gemv_k(const DevParams& p, int op) {
     switch (op) {
         case OP_OPROJ_RES: return p.nq * p.d;
@@ -1612,7 +1949,7 @@ __device__ void serve_respond(const DevParams& p, const StepArgs& a, int next_to
 // ---------------------------------------------------------------------------
 // One instantiation per JF (see gemv_dispatch); the specialised ones also
 // leave out the optional L2-prefetch paths.
-template <int JF>
+template <int JF, int DH>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ DevParams p, const StepArgs a) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int NS = p.ring_stages, SB = p.stage_bytes;
@@ -1644,7 +1981,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             for (uint32_t k = 0;; ++k) {
                 StepArgs sa = a;
                 if (a.serve && !serve_take(p, m, k, a, sa)) break;
-                if (!loader<JF == 0>(p, sa, q, n, smem, full, empty, m, lr) || !a.serve) break;
+                if (!loader<JF == 0, DH == 64>(p, sa, q, n, smem, full, empty, m, lr) || !a.serve) break;
             }
             loader_drain(p, full, lr);
         }
@@ -1687,7 +2024,10 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
                 }
                 ok = false;
             } else if (w[W_OP] == OP_ATTN) {
-                ok = attn_instr(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
+                if constexpr (DH == 64)
+                    ok = attn_tc<64>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
+                else
+                    ok = attn_cc(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
             } else {
                 ok = gemv_dispatch<JF>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase, token);
             }
@@ -1702,12 +2042,12 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
 
 namespace {
 using KernelFn = void (*)(DevParams, StepArgs);
-KernelFn kernel_of(int jf) {
-    switch (jf) {
-        case 1: return megakernel<1>;
-        case 2: return megakernel<2>;
+KernelFn kernel_of(int variant) {
+    switch (variant) {
+        case 1: return megakernel<1, 64>;
+        case 2: return megakernel<2, 128>;
     }
-    return megakernel<0>;
+    return megakernel<0, 0>;
 }
 // J of a GEMV over K columns (chunks of 8 per consumer thread, per column part)
 int j_of(int K) {
@@ -1719,8 +2059,9 @@ int j_of(int K) {
 int megakernel_variant(const DevParams& p, bool fused_ffn) {
     if (!fused_ffn || p.l2_prefetch > 0 || p.prefetch_ahead > 0) return 0;
     const int jh = j_of(p.H), jo = j_of(p.nq * p.d);
-    if (jh != jo || jh > 2) return 0;
-    return jh;
+    if (jh == 1 && jo == 1 && p.d == 64) return 1;
+    if (jh == 2 && jo == 2 && p.d == 128) return 2;
+    return 0;
 }
 
 cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, int variant, cudaStream_t stream) {

@@ -165,6 +165,7 @@ int check_options(const mk_config& c, const mk_options& o) {
     if (2LL * 2 * c.hidden > sb || part_bytes(c.ffn) > sb || part_bytes((long long)c.n_q_heads * c.head_dim) > sb)
         return MK_ERR_UNSUPPORTED;
     if (2LL * 2 * c.head_dim > sb) return MK_ERR_UNSUPPORTED;
+    if (attn_stage_rows(o.stage_bytes, c.head_dim) < 16) return MK_ERR_UNSUPPORTED;  // 16-row attention tiles
     if (o.kv_splits < 0 || (long long)o.kv_splits * c.n_q_heads > kMaxMergeSlots) return MK_ERR_INVALID_ARG;
     if (o.attn_sm_ffn_permille < 0 || o.attn_sm_ffn_permille > 4000) return MK_ERR_INVALID_ARG;
     if (o.mode < MK_MODE_MEGAKERNEL || o.mode > MK_MODE_MULTI_KERNEL_GRAPH) return MK_ERR_INVALID_ARG;
