@@ -28,6 +28,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -169,12 +170,19 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+_COMMENT = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
+
+
 def kernel_source_hash() -> str:
+    """Hash of the library sources with comments and whitespace removed, so a
+    profile summary stays attached to the code it measured across comment-only
+    edits."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "decode_persistent_block_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
+        code = _COMMENT.sub(" ", open(os.path.join(csrc, f), encoding="utf-8").read())
         h.update(f.encode())
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        h.update(" ".join(code.split()).encode())
     return h.hexdigest()[:16]
 
 

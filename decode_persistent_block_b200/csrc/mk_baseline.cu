@@ -3,10 +3,9 @@
 // One ordinary launch per op and layer (about 5 per layer plus the LM head and
 // the argmax), each kernel reading its weights straight from global memory
 // with 128-bit loads, one warp per output row.  Between launches every kernel
-// starts cold, which is the cost the persistent kernel removes ("each kernel
-// starts cold: it loads its operands, computes, writes its result to HBM and
-// exits, and the next kernel reads it back": Hyperkernel teardown, "What a
-// megakernel buys").  Step parameters come from a small device buffer so the
+// starts cold: its operands come in from memory, its result goes back out, and
+// the next launch reads that result again.  That round trip is the cost the
+// persistent kernel removes (Hyperkernel teardown, "What a megakernel buys").  Step parameters come from a small device buffer so the
 // launch sequence can be replayed from a CUDA graph.
 #include <cuda_runtime.h>
 #include <math_constants.h>

@@ -17,14 +17,15 @@
 
 namespace mk {
 
-// Opcodes: "simple kernels become opcodes" dispatched inside the persistent
-// interpreter (Kittens VM summary page, "Method").  The set is the batch-1
+// Opcodes: each op that would otherwise be its own kernel launch is an opcode
+// dispatched inside the persistent interpreter (Kittens VM summary page,
+// "Method").  The set is the batch-1
 // Llama/Mixtral decode step (epic-kernel README, "3B model support", "Mixtral
 // 8x7B MoE for batch-1 inference").
 enum Opcode : int32_t {
     OP_NOP = 0,
     OP_RMS_QKV = 1,          // xn = rmsnorm(x) * w_attn; rows of [Wq; Wk; Wv] xn (raw, pre-RoPE)
-    OP_ATTN = 2,             // RoPE + KV append + one split of GQA decode attention; last split merges
+    OP_ATTN = 2,             // RoPE + KV append + one split of GQA decode attention (partial o, m, l)
     OP_OPROJ_RES = 3,        // x[rows] = x[rows] + Wo[rows] attn   (layer 0: embed row + ...)
     OP_RMS_UPGATE_SILU = 4,  // h[rows] = silu(Wg[rows] xn) * (Wu[rows] xn), xn = rmsnorm(x) * w_ffn
     OP_DOWN_RES = 5,         // x[rows] += Wd[rows] h

@@ -2,11 +2,11 @@
 //
 // One block per SM, launched cooperatively so that every block is resident;
 // each block interprets its queue of the host-built instruction tensor and
-// never returns to the host inside a step ("a single persistent CUDA kernel
-// that occupies the entire GPU and reads an instruction tensor at runtime":
-// Kittens VM summary page, "Method"; "Launch one kernel with one block per SM
-// ... Never let the blocks exit ... synchronize with each other on the
-// device": Hyperkernel teardown, "What a megakernel buys").
+// never returns to the host inside a step.  This is the megakernel shape the
+// pages describe: one resident kernel that owns every SM and learns its work
+// from a tensor read at run time, with the blocks synchronising among
+// themselves on the device instead of through kernel boundaries (Kittens VM
+// summary page, "Method"; Hyperkernel teardown, "What a megakernel buys").
 //
 // Block = 8 consumer warps + 1 loader warp (warp-specialised roles: epic-kernel
 // README, "Fence removal and barrier reduction"):
@@ -14,9 +14,9 @@
 //    instruction's bf16 weight rows (or KV-cache rows) into a ring of
 //    shared-memory stages with TMA bulk copies completed on mbarriers.  Weight
 //    loads do not depend on activations, so the loader runs ahead across the
-//    consumers' dependency waits ("tiles of the next layer's weights can be
-//    loaded while the current layer still computes": Hyperkernel teardown,
-//    "What a megakernel buys").  After each stage it keeps a configurable
+//    consumers' dependency waits, overlapping the next op's weight traffic
+//    with the current op's compute (Hyperkernel teardown, "What a megakernel
+//    buys").  After each stage it keeps a configurable
 //    number of bytes of the following stages, across instruction boundaries,
 //    prefetched into L2 (epic-kernel README, "L2 prefetching overlapped with
 //    prior instructions").

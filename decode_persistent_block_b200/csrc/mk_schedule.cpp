@@ -3,9 +3,9 @@
 // validates the result and can execute it on the host under random
 // interleavings.
 //
-// The pages name the hard parts of a megakernel schedule: "a barrier that does
-// not deadlock, a schedule that keeps every SM busy when layers have different
-// shapes, and correctness checks" (Hyperkernel teardown, "What a megakernel
+// The pages list what makes a megakernel schedule hard: grid-wide waits must
+// never deadlock, every SM must stay busy although the ops differ in shape,
+// and the result must be checkable (Hyperkernel teardown, "What a megakernel
 // buys").  Here:
 //  - every SM queue is sorted by global op index and every wait targets a
 //    counter signalled only by strictly earlier ops, so some instruction is
@@ -13,9 +13,9 @@
 //  - every GEMV op is split into one contiguous row range per SM of equal
 //    bytes (+-1 row), so each op spans all SMs whatever its shape;
 //  - attention is split along the sequence (split-KV) into kv_heads * splits
-//    instructions so that the low-occupancy op still covers ~all SMs
-//    (epic-kernel README, "Speculative expert prediction": attention "has low
-//    SM occupancy").
+//    instructions so that attention, which on its own would occupy few SMs,
+//    still covers ~all of them (epic-kernel README, "Speculative expert
+//    prediction", which notes the idle SMs during attention).
 #include <algorithm>
 #include <array>
 #include <cstdint>
@@ -109,12 +109,16 @@ void split_rows(const std::vector<Segment>& segs, int n_sm, int cap, F emit,
 
 }  // namespace
 
-// Splits per kv head: about 128 cached positions per split at the longest
-// context, at most one split per SM, and few enough that the O-projection's
+// Splits per kv head.  A split takes about `span` cached positions of the
+// longest context: 192 at head_dim 64, where the attention runs on tensor cores
+// and a split's fixed costs (prologue, partial write, its share of the merge)
+// outweigh its per-row work, and 128 at head_dim 128 (CUDA-core attention).
+// At most one split per SM per kv head, and few enough that the O-projection's
 // prologue can merge every head's splits (kMaxMergeSlots).
 int default_kv_splits(const mk_config& c, int n_sm) {
+    const int span = c.head_dim == 64 ? 192 : 128;
     const int per_sm = std::max(1, n_sm / std::max(1, c.n_kv_heads));
-    const int by_len = std::max(1, (c.max_seq + 127) / 128);
+    const int by_len = std::max(1, (c.max_seq + span - 1) / span);
     const int by_merge = std::max(1, kMaxMergeSlots / std::max(1, c.n_q_heads));
     return std::min(std::min(per_sm, by_len), by_merge);
 }

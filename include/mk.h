@@ -5,11 +5,9 @@
  * (optionally with a top-k MoE FFN) for a single sequence, as ONE persistent
  * kernel with one block per SM whose blocks never exit mid-step and read, at
  * run time, a host-built instruction tensor that tells each block which
- * operation to run next ("a single persistent CUDA kernel that occupies the
- * entire GPU and reads an instruction tensor at runtime to decide what work
- * each SM does next": Kittens VM summary page, "Method"; "Launch one kernel
- * with one block per SM ... Never let the blocks exit ... synchronize with each
- * other on the device": Hyperkernel teardown, "What a megakernel buys").
+ * operation to run next.  The blocks synchronise among themselves on the
+ * device instead of through kernel boundaries (Kittens VM summary page,
+ * "Method"; Hyperkernel teardown, "What a megakernel buys").
  * Dependencies between instructions are global-memory counters.  Weight tiles
  * stream through a multi-stage shared-memory ring fed by TMA bulk copies, with
  * an L2 prefetch of the following weights (epic-kernel README, "Pipelining for
@@ -100,8 +98,9 @@ typedef struct {
     int ring_stages;      /* shared-memory weight ring depth (default 3) */
     int stage_bytes;      /* bytes per ring stage, multiple of 1024 (default 65536) */
     int rows_per_instr;   /* cap on GEMV rows per instruction (default and max 1024) */
-    int kv_splits;        /* split-KV chunks per kv head (0 = default: about one split per 128 positions of
-                             max_seq, at most SMs / n_kv_heads; n_q_heads * kv_splits <= 2048) */
+    int kv_splits;        /* split-KV chunks per kv head (0 = default: about one split per 192 positions of
+                             max_seq at head_dim 64, per 128 at head_dim 128, at most SMs / n_kv_heads;
+                             n_q_heads * kv_splits <= 2048) */
     int l2_prefetch;      /* bytes kept prefetched into L2 ahead of the TMA stream (-1 default) */
     int trace;            /* 1: record per-instruction globaltimer stamps (mk_get_trace) */
     int snapshots;        /* 1: record the residual stream after every layer (mk_get_hidden) */

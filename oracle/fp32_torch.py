@@ -1,8 +1,9 @@
 """Second, independent CPU restatement of the decode step in fp32 (torch CPU ops).
 
 TEST INFRASTRUCTURE ONLY.  It exists to measure the fp32-vs-fp64 noise floor
-(the Hyperkernel teardown, "Which claims the repo backs": compare against an
-independent implementation next to its own noise floor) and to cross-check the
+(the Hyperkernel teardown, "Which claims the repo backs", judges agreement
+with an independent implementation against that implementation's own noise
+floor) and to cross-check the
 C oracle: it is written from the same plain decoder definition with torch
 tensor ops, sharing no code with oracle.c.
 """

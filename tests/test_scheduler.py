@@ -198,14 +198,17 @@ def test_fused_ffn_is_the_default_for_every_supported_hidden_size():
         assert OP["FFN"] not in ops(cfg, split_ffn=1) and {OP["UG"], OP["DOWN"]} <= ops(cfg, split_ffn=1)
 
 
-@pytest.mark.parametrize("cfg,expect", [(configs.LLAMA_1B, 9), (configs.LLAMA_3B, 17), (configs.TINY, 1),
-                                        (configs.llama1b_sweep(16384), 18)], ids=lambda x: getattr(x, "name", x))
+@pytest.mark.parametrize("cfg,expect", [(configs.LLAMA_1B, 6), (configs.LLAMA_3B, 17), (configs.TINY, 1),
+                                        (configs.llama1b_sweep(2048), 11), (configs.llama1b_sweep(16384), 18),
+                                        (configs.MIXTRAL_8L, 9)], ids=lambda x: getattr(x, "name", x))
 def test_default_kv_splits(cfg, expect):
-    # about one split per 128 positions of the longest context, at most one per SM per kv head
+    # about one split per 192 positions of the longest context at head_dim 64 (tensor-core
+    # attention) and per 128 at head_dim 128, at most one per SM per kv head
     words, n_instr, inc = dpb.plan(cfg, 148)
     attn = [w for _, _, w in instrs(words, n_instr) if w[W_OP] == OP["ATTN"]]
     s = int(attn[0][W_END]) if attn else 0
-    assert s == min(-(-cfg.max_seq // 128), 148 // cfg.n_kv_heads, 2048 // cfg.n_heads)
+    span = 192 if cfg.head_dim == 64 else 128
+    assert s == min(-(-cfg.max_seq // span), 148 // cfg.n_kv_heads, 2048 // cfg.n_heads)
     if expect is not None:
         assert s == expect
 
