@@ -177,6 +177,7 @@ void mk_default_options(mk_options* o) {
     std::memset(o, 0, sizeof(*o));
     o->l2_prefetch = -1;
     o->prefetch_ahead = -1;
+    o->l2_head_start = -1;
     o->mode = MK_MODE_MEGAKERNEL;
 }
 
@@ -244,6 +245,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     p.ring_stages = o.ring_stages;
     p.stage_bytes = o.stage_bytes;
     p.l2_prefetch = o.l2_prefetch;
+    p.l2_head_start = o.l2_head_start;
     p.prefetch_ahead = o.prefetch_ahead;
     p.prefetch_max_bytes = o.prefetch_max_bytes;
     p.spin_limit_ns = o.spin_limit_ns;

@@ -64,6 +64,7 @@ constexpr int kMaxGroup = 4;         // query heads per kv head
 constexpr int kMaxHeadDim = 128;
 constexpr int kMaxTopK = 2;
 constexpr int kMaxMergeSlots = 2048;  // query heads x kv splits merged in the O-projection prologue
+constexpr int kDefaultL2HeadStart = 0;  // ring stages of an FFN / LM-head stream prefetched into L2 past the ring
 
 // Counter ids: per layer [QKV, ATTN (one signal per split), OPROJ, FFN1, FFN2], then the LM head's
 // arrival counter.
@@ -184,11 +185,12 @@ struct DevParams {
     float* snap;       // [(L+1)][H] or null
     int32_t* router_idx;  // [L][kMaxTopK]
     float* router_w;      // [L][kMaxTopK]
-    unsigned long long* trace;  // [n_sm][max_instr][4] or null
+    unsigned long long* trace;  // [n_sm][max_instr][kTraceWords] or null
     // kernel knobs
     int ring_stages;
     int stage_bytes;
     int l2_prefetch;
+    int l2_head_start;
     int prefetch_ahead;
     int prefetch_max_bytes;
     unsigned long long spin_limit_ns;

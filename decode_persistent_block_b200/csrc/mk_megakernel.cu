@@ -470,6 +470,15 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                 break;
             }
             issue_stage<TC>(p, pl, st, ring + (size_t)slot * SB, &full[slot]);
+            // Head start of a long stream: the loader reaches the first stage of the
+            // dense FFN (or the LM head) while the consumers still wait on the small
+            // ops before it and HBM is mostly idle.  The stages that follow the
+            // ring's worth are prefetched into L2 now, so they are close when the
+            // consumers free the ring's slots.
+            if (st == 0 && p.l2_head_start > 0 && (w[W_OP] == OP_FFN || w[W_OP] == OP_LMHEAD_ARGMAX)) {
+                const int e = pl.n_stages < NS + p.l2_head_start ? pl.n_stages : NS + p.l2_head_start;
+                for (int s2 = NS; s2 < e; ++s2) prefetch_stage(pl, s2);
+            }
             if (tr && st == 0) tr[T_LD_FIRST] = globaltimer_ns();
             if (tr && st == pl.n_stages - 1) tr[T_LD_LAST] = globaltimer_ns();
             used |= 1u << slot;

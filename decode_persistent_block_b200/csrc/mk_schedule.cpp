@@ -153,6 +153,7 @@ void fill_defaults(mk_options* o) {
     if (o->rows_per_instr <= 0 || o->rows_per_instr > kMaxRows) o->rows_per_instr = kMaxRows;
     if (o->l2_prefetch < 0) o->l2_prefetch = 0;
     if (o->prefetch_ahead < 0) o->prefetch_ahead = 0;
+    if (o->l2_head_start < 0) o->l2_head_start = kDefaultL2HeadStart;
     if (o->prefetch_max_bytes <= 0) o->prefetch_max_bytes = 1 << 20;
     if (o->attn_sm_ffn_permille <= 0) o->attn_sm_ffn_permille = 1000;
     if (o->spin_limit_ns == 0) o->spin_limit_ns = 2000000000ull;
@@ -172,6 +173,7 @@ int check_options(const mk_config& c, const mk_options& o) {
     if (attn_stage_rows(o.stage_bytes, c.head_dim) < 16) return MK_ERR_UNSUPPORTED;  // 16-row attention tiles
     if (o.kv_splits < 0 || (long long)o.kv_splits * c.n_q_heads > kMaxMergeSlots) return MK_ERR_INVALID_ARG;
     if (o.attn_sm_ffn_permille < 0 || o.attn_sm_ffn_permille > 4000) return MK_ERR_INVALID_ARG;
+    if (o.l2_head_start < 0 || o.l2_head_start > 64) return MK_ERR_INVALID_ARG;
     if (o.mode < MK_MODE_MEGAKERNEL || o.mode > MK_MODE_MULTI_KERNEL_GRAPH) return MK_ERR_INVALID_ARG;
     // ring + barriers + partial-sum slots + misc must fit the 227 KB per-block opt-in limit
     if ((long long)o.ring_stages * o.stage_bytes + 16LL * o.ring_stages + 128 + 4LL * kRowSlots * 8 + 512 > 232448)

@@ -45,7 +45,7 @@ class MkOptions(ctypes.Structure):
                 ("l2_prefetch", _I), ("trace", _I), ("snapshots", _I), ("spin_limit_ns", ctypes.c_ulonglong),
                 ("mode", _I), ("n_sm", _I), ("prefetch_ahead", _I), ("prefetch_max_bytes", _I),
                 ("attn_sm_ffn_permille", _I), ("serve_idle_ns", ctypes.c_ulonglong), ("general_kernel", _I),
-                ("split_ffn", _I)]
+                ("split_ffn", _I), ("l2_head_start", _I)]
 
 
 class MkStatus(ctypes.Structure):

@@ -93,7 +93,7 @@ typedef struct {
 } mk_weights;
 
 /* Schedule and kernel knobs.  Zero selects the default for every field except
- * l2_prefetch and prefetch_ahead (-1 = default, 0 = off). */
+ * l2_prefetch, prefetch_ahead and l2_head_start (-1 = default, 0 = off). */
 typedef struct {
     int ring_stages;      /* shared-memory weight ring depth (default 3) */
     int stage_bytes;      /* bytes per ring stage, multiple of 1024 (default 65536) */
@@ -123,6 +123,10 @@ typedef struct {
                              varies between runs); 1: separate up/gate and down instructions, no copy,
                              bitwise reproducible.  The split form is also used whenever hidden > 8192
                              or 2 * hidden > stage_bytes */
+    int l2_head_start;    /* when the loader issues the first stage of a dense fused-FFN or LM-head
+                             instruction, it also prefetches into L2 this many ring stages of that
+                             instruction's weights past the ring (0..64; -1 default, 0 = off), so the
+                             stream is already moving when the instruction's dependency is met */
 } mk_options;
 
 /* Device status block, copied out by mk_get_status.  On a device-side error
