@@ -109,18 +109,31 @@ void split_rows(const std::vector<Segment>& segs, int n_sm, int cap, F emit,
 
 }  // namespace
 
-// Splits per kv head.  A split takes about `span` cached positions of the
-// longest context: 192 at head_dim 64, where the attention runs on tensor cores
-// and a split's fixed costs (prologue, partial write, its share of the merge)
-// outweigh its per-row work, and 128 at head_dim 128 (CUDA-core attention).
-// At most one split per SM per kv head, and few enough that the O-projection's
-// prologue can merge every head's splits (kMaxMergeSlots).
+// Splits per kv head: at most one split per SM per kv head, and few enough
+// that the O-projection's prologue can merge every head's splits
+// (kMaxMergeSlots).  Within that:
+//  - head_dim 64 (tensor-core attention): the count that minimises a model of
+//    one layer's attention plus merge time at the longest context,
+//      t(S) = t_row * max_seq / S + t_split * S + t_trip * ceil(S / 8),
+//    with t_row = 10 ns per cached row of a split, t_split = 0.3 us for each
+//    split's partials that every O-projection block reads, and t_trip = 1 us
+//    per merge round trip (8 splits each).  The constants come from per-op
+//    device traces of the Llama-1B shape.  The model orders its measured split
+//    sweep (4 to 16 splits at 1152 positions) almost exactly.
+//  - head_dim 128 (CUDA-core attention, about 5x the per-row cost): about one
+//    split per 128 positions.
 int default_kv_splits(const mk_config& c, int n_sm) {
-    const int span = c.head_dim == 64 ? 192 : 128;
     const int per_sm = std::max(1, n_sm / std::max(1, c.n_kv_heads));
-    const int by_len = std::max(1, (c.max_seq + span - 1) / span);
     const int by_merge = std::max(1, kMaxMergeSlots / std::max(1, c.n_q_heads));
-    return std::min(std::min(per_sm, by_len), by_merge);
+    const int cap = std::min(per_sm, by_merge);
+    if (c.head_dim != 64) return std::min(cap, std::max(1, (c.max_seq + 127) / 128));
+    int best = 1;
+    double best_t = 0;
+    for (int s = 1; s <= cap; ++s) {
+        const double t = 10.0 * c.max_seq / s + 300.0 * s + 1000.0 * ((s + 7) / 8);
+        if (s == 1 || t < best_t) best = s, best_t = t;
+    }
+    return best;
 }
 
 int check_config(const mk_config& c) {

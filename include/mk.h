@@ -98,9 +98,10 @@ typedef struct {
     int ring_stages;      /* shared-memory weight ring depth (default 3) */
     int stage_bytes;      /* bytes per ring stage, multiple of 1024 (default 65536) */
     int rows_per_instr;   /* cap on GEMV rows per instruction (default and max 1024) */
-    int kv_splits;        /* split-KV chunks per kv head (0 = default: about one split per 192 positions of
-                             max_seq at head_dim 64, per 128 at head_dim 128, at most SMs / n_kv_heads;
-                             n_q_heads * kv_splits <= 2048) */
+    int kv_splits;        /* split-KV chunks per kv head (0 = default, at most SMs / n_kv_heads: at
+                             head_dim 64 the count minimising a fitted model of attention plus merge
+                             time at max_seq, 6 for 1152 positions; at head_dim 128 about one split
+                             per 128 positions of max_seq; n_q_heads * kv_splits <= 2048) */
     int l2_prefetch;      /* bytes kept prefetched into L2 ahead of the TMA stream (-1 default) */
     int trace;            /* 1: record per-instruction globaltimer stamps (mk_get_trace) */
     int snapshots;        /* 1: record the residual stream after every layer (mk_get_hidden) */
