@@ -45,6 +45,14 @@ ROOFLINE_NOMINAL_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
 
+def byte_floor_us(n_bytes: float, gbs: float) -> float:
+    """Least time, in µs, to stream `n_bytes` from HBM at `gbs` GB/s.  At batch 1
+    every weight byte crosses HBM at least once per step, so bytes over
+    bandwidth bounds any kernel from below (Hyperkernel teardown, "Where the
+    numbers sit against the hardware")."""
+    return n_bytes / (gbs * 1e9) * 1e6
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -393,6 +401,7 @@ def run_ours(args, rank, world, local):
         "tokens_per_s": round(1e6 / us_per_token, 1),
         "hbm_gbs": round(achieved, 1),
         "frac_of_8tbs": round(achieved / ROOFLINE_NOMINAL_GBS, 4),
+        "floor_us_at_8tbs": round(byte_floor_us(bpt, ROOFLINE_NOMINAL_GBS), 1),
         "bytes_per_token": int(bpt),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",

@@ -217,9 +217,11 @@ int mk_reset(mk_handle *h);
  * serve_idle_ns without a request; the next mk_serve_step then returns
  * MK_ERR_STOPPED and mk_serve_start may be called again.  While serving, the
  * calls that touch the device (step, reset, getters, fault injection, schedule
- * rebuild) return MK_ERR_INVALID_ARG; mk_destroy stops the grid first.  Counters and KV positions continue across the serving
- * and per-launch paths (same epoch rule).  The paper's launch-once server loop;
- * errors: MK_ERR_INVALID_ARG, MK_ERR_STOPPED, MK_ERR_TIMEOUT, MK_ERR_BAD_INSTR,
+ * rebuild) return MK_ERR_INVALID_ARG; mk_destroy stops the grid first.
+ * Counters and KV positions continue across the serving and per-launch paths
+ * (same epoch rule).  This is the launch-once, ring-fed server loop of the
+ * Hyperkernel teardown ("A single kernel launch, read from the host").
+ * Errors: MK_ERR_INVALID_ARG, MK_ERR_STOPPED, MK_ERR_TIMEOUT, MK_ERR_BAD_INSTR,
  * MK_ERR_CUDA. */
 int mk_serve_start(mk_handle *h, float *logits_dev);
 int mk_serve_step(mk_handle *h, int32_t token, int32_t pos, int32_t *next_token_host);
@@ -271,7 +273,7 @@ int mk_attention_decode(const float *q, const void *k_cache, const void *v_cache
  * memory is owned by another allocator or pool, or a latency-critical decode
  * loop where an allocation (and the device synchronisation it can imply) is
  * not allowed.  This entry point calls no cudaMalloc, cudaFree or other
- * allocating routine.  The paper has no counterpart for it.
+ * allocating routine.  The pages describe no counterpart for it.
  *  - Its split partials live in one fixed device array of
  *    MK_ATTENTION_NOALLOC_SCRATCH_BYTES inside the library, present on every
  *    GPU that loads the library until the process exits; a call whose

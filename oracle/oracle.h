@@ -13,6 +13,10 @@
  * teardown, "What a megakernel buys": a megakernel evaluates the same forward
  * pass in one launch).  Weights and KV cache are bf16 bit patterns (uint16);
  * every product and sum is in double.
+ *
+ * Every building block and the whole step are pinned by the CPU tests to
+ * closed forms, brute force, special cases and an independent fp32
+ * restatement; none is parity unpinned.
  */
 #ifndef ORC_ORACLE_H
 #define ORC_ORACLE_H
