@@ -70,6 +70,8 @@ def parse():
     ap.add_argument("--no-baselines", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--calibrate", type=int, default=0,
+                    help="1: split the FFN and LM-head rows by per-SM speed measured on this GPU at start-up")
     return ap.parse_args()
 
 
@@ -275,6 +277,7 @@ def run_ours(args, rank, world, local):
 
     import synth
     from decode_persistent_block_b200 import Decoder, to_device
+    from decode_persistent_block_b200.calibrate import measure_sm_speed
     torch.cuda.set_device(local)
     cfg, p0, positions = workload(args)
     W = synth.make_model(cfg)
@@ -286,6 +289,12 @@ def run_ours(args, rank, world, local):
     mode = {"megakernel": 0, "multi_kernel": 1, "multi_kernel_graph": 2}[args.mode]
     opts = dict(mode=mode, l2_prefetch=args.l2_prefetch, ring_stages=args.ring_stages,
                 stage_bytes=args.stage_bytes, kv_splits=args.kv_splits, serve_idle_ns=2_000_000_000)
+    calib = None
+    if args.calibrate and args.mode == "megakernel":
+        # start-up calibration, outside the timed region: a few traced steps from p0
+        speed = measure_sm_speed(cfg, dW, dk, dv, first, positions[0], steps=8, **opts)
+        opts["sm_speed"] = speed
+        calib = {"steps": 8, "min": round(float(speed.min()), 3), "max": round(float(speed.max()), 3)}
     dec = Decoder(cfg, dW, dk, dv, **opts)
     K, Wm = args.steps, args.warmup
 
@@ -397,7 +406,8 @@ def run_ours(args, rank, world, local):
         "config": {"workload": f"{cfg.name}: batch-1 greedy decode, KV pre-filled to {cfg.prefill}, positions "
                                f"{p0}..{p0 + cfg.steps - 1}", "layers": cfg.n_layers, "hidden": cfg.hidden,
                    "vocab": cfg.vocab, "mode": args.mode, "parallelism": f"replicas x{world}",
-                   "l2": f"no flush: {bpt / 1e9:.2f} GB streamed per token > 126 MB L2"},
+                   "l2": f"no flush: {bpt / 1e9:.2f} GB streamed per token > 126 MB L2",
+                   "sm_speed": calib or "equal"},
         "tokens_per_s": round(1e6 / us_per_token, 1),
         "hbm_gbs": round(achieved, 1),
         "frac_of_8tbs": round(achieved / ROOFLINE_NOMINAL_GBS, 4),

@@ -46,6 +46,7 @@ struct mk_handle {
     bool down_t = false;  // transposed down-projection copies exist (fused FFN schedules)
     int last_cuda = 0;
     int last_error = MK_OK;
+    std::vector<float> sm_speed;  // copy of options.sm_speed (opt.sm_speed points here)
 };
 
 namespace {
@@ -227,6 +228,11 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, h->device);
     if (dev_sms <= 0) return fail(MK_ERR_CUDA);
     h->n_sm = (o.n_sm > 0 && o.n_sm < dev_sms) ? o.n_sm : dev_sms;
+    if (o.sm_speed) {
+        if (o.n_sm_speed != h->n_sm) return fail(MK_ERR_INVALID_ARG);
+        h->sm_speed.assign(o.sm_speed, o.sm_speed + o.n_sm_speed);
+        h->opt.sm_speed = h->sm_speed.data();
+    }
 
     const mk_config& c = *cfg;
     const int L = c.n_layers, H = c.hidden, d = c.head_dim, nq = c.n_q_heads, nkv = c.n_kv_heads;

@@ -18,6 +18,7 @@
 //    prediction", which notes the idle SMs during attention).
 #include <algorithm>
 #include <array>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <random>
@@ -187,6 +188,11 @@ int check_options(const mk_config& c, const mk_options& o) {
     if (o.kv_splits < 0 || (long long)o.kv_splits * c.n_q_heads > kMaxMergeSlots) return MK_ERR_INVALID_ARG;
     if (o.attn_sm_ffn_permille < 0 || o.attn_sm_ffn_permille > 4000) return MK_ERR_INVALID_ARG;
     if (o.l2_head_start < 0 || o.l2_head_start > 64) return MK_ERR_INVALID_ARG;
+    if (o.sm_speed) {
+        if (o.n_sm_speed <= 0) return MK_ERR_INVALID_ARG;
+        for (int i = 0; i < o.n_sm_speed; ++i)
+            if (!(o.sm_speed[i] > 0.f) || !std::isfinite(o.sm_speed[i])) return MK_ERR_INVALID_ARG;
+    }
     if (o.mode < MK_MODE_MEGAKERNEL || o.mode > MK_MODE_MULTI_KERNEL_GRAPH) return MK_ERR_INVALID_ARG;
     // ring + barriers + partial-sum slots + misc must fit the 227 KB per-block opt-in limit
     if ((long long)o.ring_stages * o.stage_bytes + 16LL * o.ring_stages + 128 + 4LL * kRowSlots * 8 + 512 > 232448)
@@ -206,6 +212,11 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     if (n_sm <= 0) return MK_ERR_INVALID_ARG;
     mk_options o = o_in;
     fill_defaults(&o);
+    if (o.sm_speed && o.n_sm_speed != n_sm) return MK_ERR_INVALID_ARG;
+    // relative streaming speed of every block: the dense FFN and LM head rows follow it
+    std::vector<double> speed(n_sm, 1.0);
+    if (o.sm_speed)
+        for (int i = 0; i < n_sm; ++i) speed[i] = o.sm_speed[i];
     const int L = c.n_layers, nkv = c.n_kv_heads, d = c.head_dim, H = c.hidden, F = c.ffn;
     const int S = o.kv_splits > 0 ? o.kv_splits : default_kv_splits(c, n_sm);
     const int cap = o.rows_per_instr;
@@ -243,7 +254,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
                 ctr_id(l, C_QKV));
         // attention: kv head g, split s -> instruction k = g * S + s, rotated per layer
         const int total = nkv * S;
-        std::vector<double> ffn_weight(n_sm, 1.0);  // blocks with an attention split take fewer FFN rows
+        std::vector<double> ffn_weight = speed;  // blocks with an attention split may take fewer FFN rows
         for (int k = 0; k < total; ++k) {
             Instr w = blank();
             w[W_OP] = OP_ATTN;
@@ -255,7 +266,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
             w[W_SIGNAL_CTR] = ctr_id(l, C_ATTN);
             int sm = (int)(((long long)k + (long long)l * total) % n_sm);
             add(sm, w);
-            ffn_weight[sm] = o.attn_sm_ffn_permille / 1000.0;
+            ffn_weight[sm] = speed[sm] * (o.attn_sm_ffn_permille / 1000.0);
         }
         gemv_op(OP_OPROJ_RES, l, {{0, H}}, ctr_id(l, C_ATTN), ctr_id(l, C_OPROJ));
         std::vector<Segment> slots;
@@ -285,7 +296,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
             w[W_AUX_CTR] = ctr_lm(L);
             w[W_SEQ] = seq++;
             add(sm, w);
-        });
+        }, o.sm_speed ? &speed : nullptr);
     }
     // fill wait increments and aux increments
     for (auto& qs : q)

@@ -45,7 +45,7 @@ class MkOptions(ctypes.Structure):
                 ("l2_prefetch", _I), ("trace", _I), ("snapshots", _I), ("spin_limit_ns", ctypes.c_ulonglong),
                 ("mode", _I), ("n_sm", _I), ("prefetch_ahead", _I), ("prefetch_max_bytes", _I),
                 ("attn_sm_ffn_permille", _I), ("serve_idle_ns", ctypes.c_ulonglong), ("general_kernel", _I),
-                ("split_ffn", _I), ("l2_head_start", _I)]
+                ("split_ffn", _I), ("l2_head_start", _I), ("sm_speed", ctypes.c_void_p), ("n_sm_speed", _I)]
 
 
 class MkStatus(ctypes.Structure):
@@ -134,11 +134,22 @@ def make_config(cfg) -> MkConfig:
 
 
 def make_options(**kw) -> MkOptions:
+    """mk_options with the library defaults, then the given fields.  `sm_speed`
+    takes a sequence of per-block speeds; the returned struct keeps the array
+    alive (the library copies it when it reads the options)."""
     o = MkOptions()
     load().mk_default_options(ctypes.byref(o))
     for k, v in kw.items():
         if not hasattr(o, k):
             raise KeyError(f"unknown option {k}")
+        if k == "sm_speed":
+            if v is None:
+                continue
+            arr = np.ascontiguousarray(v, dtype=np.float32)
+            o._sm_speed = arr
+            o.sm_speed = arr.ctypes.data
+            o.n_sm_speed = int(arr.size)
+            continue
         setattr(o, k, v)
     return o
 

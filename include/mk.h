@@ -128,6 +128,13 @@ typedef struct {
                              instruction, it also prefetches into L2 this many ring stages of that
                              instruction's weights past the ring (0..64; -1 default, 0 = off), so the
                              stream is already moving when the instruction's dependency is met */
+    const float *sm_speed; /* host array of n_sm_speed relative streaming speeds, one per block of the
+                             grid (NULL = all equal).  The dense fused FFN's rows and the LM head's rows
+                             are split in proportion, so blocks that stream slower on this GPU take fewer
+                             rows.  Each speed must be finite and > 0, and n_sm_speed must equal the
+                             grid's block count.  Read (copied) by mk_create and mk_plan; the caller may
+                             free it afterwards */
+    int n_sm_speed;
 } mk_options;
 
 /* Device status block, copied out by mk_get_status.  On a device-side error

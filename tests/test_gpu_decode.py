@@ -175,6 +175,24 @@ def test_llama1b(cuda):
     _full(configs.LLAMA_1B, 4)
 
 
+def test_llama1b_calibrated_sm_speed(cuda):
+    # FFN and LM-head rows split by the per-SM speed measured on this GPU: same bar
+    from decode_persistent_block_b200.calibrate import measure_sm_speed
+    cfg = configs.LLAMA_1B
+    s = parity.Setup(cfg)
+    p0 = cfg.prefill + cfg.prompt_len
+    speed = measure_sm_speed(cfg, s.dW, s.dk, s.dv, int(parity.synth.prompt_tokens(cfg)[0]), p0, steps=3)
+    assert np.all(np.isfinite(speed)) and abs(speed.mean() - 1.0) < 0.05 and speed.min() >= 0.5
+    reps = parity.run(s, steps=None if FULL else 3, sm_speed=speed)
+    parity.assert_parity(reps, cfg)
+
+
+def test_tiny_skewed_sm_speed(tiny):
+    import torch
+    n = torch.cuda.get_device_properties(0).multi_processor_count
+    parity.assert_parity(parity.run(tiny, sm_speed=np.linspace(0.5, 1.5, n)))
+
+
 def test_llama1b_split_ffn(cuda):
     _full(configs.LLAMA_1B, 2, split_ffn=1)
 

@@ -241,3 +241,57 @@ def test_attention_blocks_take_fewer_ffn_rows(permille):
         a = np.mean([rows[s] for s in attn_sms])
         b = np.mean([rows[s] for s in rows if s not in attn_sms])
         assert a / b == pytest.approx(permille / 1000, abs=0.03)
+
+
+def _rows_per_sm(words, n_instr, op, layer):
+    r = np.zeros(words.shape[0], dtype=np.int64)
+    for sm, _, w in instrs(words, n_instr):
+        if w[W_OP] == OP[op] and w[W_LAYER] == layer:
+            r[sm] += int(w[W_END]) - int(w[W_BEGIN])
+    return r
+
+
+@pytest.mark.parametrize("n_sm", [148, 13])
+def test_sm_speed_splits_ffn_and_lm_rows_in_proportion(n_sm):
+    cfg = configs.LLAMA_1B
+    speed = np.linspace(0.5, 1.5, n_sm)
+    words, n_instr, inc = dpb.plan(cfg, n_sm, sm_speed=speed)
+    for op, layer, total in (("FFN", 3, cfg.ffn), ("LM", cfg.n_layers, cfg.vocab)):
+        rows = _rows_per_sm(words, n_instr, op, layer)
+        assert rows.sum() == total
+        # each block's share is its speed's share of the total, to a row (the cut points round)
+        want = total * speed / speed.sum()
+        assert np.abs(rows - want).max() <= 1.0 + 1e-9
+    # every other op keeps the even split of the default schedule
+    w0, n0, inc0 = dpb.plan(cfg, n_sm)
+    for op in ("RMS_QKV", "OPROJ"):
+        np.testing.assert_array_equal(_rows_per_sm(words, n_instr, op, 3), _rows_per_sm(w0, n0, op, 3))
+    # QKV, attention and O-projection counters keep their increments; the FFN's and the LM head's
+    # count their instructions: one per started 512 FFN rows (two accumulator sets of 1024 slots)
+    # or 1024 LM rows of a block's share
+    L = cfg.n_layers
+    for slot in (0, 1, 2):
+        np.testing.assert_array_equal(inc[slot:5 * L:5], inc0[slot:5 * L:5])
+    ffn = _rows_per_sm(words, n_instr, "FFN", 3)
+    assert inc[5 * 3 + 4] == sum(-(-int(r) // 512) for r in ffn)
+    lm = _rows_per_sm(words, n_instr, "LM", L)
+    assert inc[-1] == sum(-(-int(r) // 1024) for r in lm)
+    rc, done = mk.simulate(words, n_instr, inc, steps=2, seed=3)
+    assert rc == 0 and done == 2 * int(n_instr.sum())
+
+
+def test_sm_speed_uniform_matches_default_and_bad_speeds_are_rejected():
+    # equal speeds give the default split (the LM head's cut points may round the other way: +-1 row)
+    cfg = configs.LLAMA_1B
+    w0, n0, _ = dpb.plan(cfg, 148)
+    w1, n1, _ = dpb.plan(cfg, 148, sm_speed=np.full(148, 2.5))
+    np.testing.assert_array_equal(n0, n1)
+    for layer in range(cfg.n_layers):
+        for op in ("RMS_QKV", "ATTN", "OPROJ", "FFN"):
+            np.testing.assert_array_equal(_rows_per_sm(w0, n0, op, layer), _rows_per_sm(w1, n1, op, layer))
+    d = _rows_per_sm(w0, n0, "LM", cfg.n_layers) - _rows_per_sm(w1, n1, "LM", cfg.n_layers)
+    assert np.abs(d).max() <= 1 and d.sum() == 0
+    for bad in (np.ones(147), np.r_[np.ones(147), 0.0], np.r_[np.ones(147), -1.0], np.r_[np.ones(147), np.nan],
+                np.r_[np.ones(147), np.inf]):
+        with pytest.raises(mk.MkError):
+            dpb.plan(cfg, 148, sm_speed=bad)
