@@ -1,0 +1,148 @@
+"""Per-instruction device trace (`mk_options.trace = 1`): per-op latency
+breakdown and per-SM spread.
+
+`Decoder.trace()` returns, for the last step, eight globaltimer stamps (ns, 0 =
+not reached) per instruction of the schedule [n_sm][max_instr]:
+  0 reached, 1 dependency met, 2 input vector ready, 3 first stage full,
+  4 main stages consumed, 5 done and signalled (consumer warps);
+  6 first stage issued, 7 last stage issued (loader warp).
+
+`op_breakdown` reduces them to the phases of each op, averaged over layers:
+  phase   previous op's last end -> this op's last end (the op's share of the step)
+  hop     previous op's last end -> dependency met (mean over blocks)
+  ready   dependency met -> input vector ready
+  first   -> first stage full
+  main    first stage -> main stages consumed
+  epi     -> done and signalled
+  spread  last end - first end across the op's blocks
+  ld_lead loader's first issue -> dependency met (how far the loader ran ahead)
+  ld_last dependency met -> loader's last issue
+
+Command line (on a GPU):
+  python -m decode_persistent_block_b200.trace llama1b [--steps 4] [--npz out.npz] [key=value options]
+"""
+from __future__ import annotations
+
+import numpy as np
+
+OP_NAMES = {1: "QKV", 2: "ATTN", 3: "OPROJ", 4: "UG", 5: "DOWN", 6: "LM", 7: "MOE_UG", 8: "MOE_DOWN", 9: "FFN",
+            10: "MOE_FFN"}
+ORDER = ["QKV", "ATTN", "OPROJ", "UG", "DOWN", "FFN", "MOE_UG", "MOE_DOWN", "MOE_FFN", "LM"]
+COLUMNS = ["phase", "hop", "ready", "first", "main", "epi", "spread", "ld_lead", "ld_last"]
+T_START, T_DEP, T_READY, T_FIRST, T_MAIN, T_END, T_LD_FIRST, T_LD_LAST = range(8)
+
+
+def _groups(schedule: np.ndarray, trace: np.ndarray):
+    """{(layer, op name): array [blocks, 8] of stamps in µs from the step's first stamp (nan = not reached)}."""
+    tr = trace.reshape(schedule.shape[0], schedule.shape[1], -1).astype(np.int64)
+    reached = tr[:, :, T_START][tr[:, :, T_START] > 0]
+    if reached.size == 0:
+        return {}
+    t0 = reached.min()
+    out = {}
+    for sm in range(schedule.shape[0]):
+        for i in range(schedule.shape[1]):
+            op = int(schedule[sm, i, 0])
+            if op == 0:
+                continue
+            out.setdefault((int(schedule[sm, i, 1]), OP_NAMES.get(op, str(op))), []).append(tr[sm, i])
+    return {k: np.where(np.array(v) > 0, (np.array(v) - t0) / 1000.0, np.nan) for k, v in out.items()}
+
+
+def op_breakdown(schedule: np.ndarray, trace: np.ndarray) -> dict:
+    """{op name: {column: mean µs over the layers}} in step order (see the module doc)."""
+    g = _groups(schedule, trace)
+    keys = sorted(g, key=lambda k: (k[0], np.nanmin(g[k][:, T_START])))
+    agg: dict = {}
+    prev_end = None
+    for key in keys:
+        a = g[key]
+        end_max = np.nanmax(a[:, T_END])
+        row = {
+            "phase": end_max - prev_end if prev_end is not None else np.nan,
+            "hop": np.nanmean(a[:, T_DEP] - prev_end) if prev_end is not None else np.nan,
+            "ready": np.nanmean(a[:, T_READY] - a[:, T_DEP]),
+            "first": np.nanmean(a[:, T_FIRST] - np.fmax(a[:, T_READY], a[:, T_DEP])),
+            "main": np.nanmean(a[:, T_MAIN] - a[:, T_FIRST]),
+            "epi": np.nanmean(a[:, T_END] - a[:, T_MAIN]),
+            "spread": end_max - np.nanmin(a[:, T_END]),
+            "ld_lead": np.nanmean(a[:, T_DEP] - a[:, T_LD_FIRST]),
+            "ld_last": np.nanmean(a[:, T_LD_LAST] - a[:, T_DEP]),
+        }
+        prev_end = end_max
+        agg.setdefault(key[1], []).append(row)
+    return {op: {c: _mean([r[c] for r in agg[op]]) for c in COLUMNS} for op in ORDER if op in agg}
+
+
+def _mean(xs) -> float:
+    a = np.asarray(xs, dtype=np.float64)
+    a = a[~np.isnan(a)]
+    return float(a.mean()) if a.size else float("nan")
+
+
+def per_sm_duration(schedule: np.ndarray, trace: np.ndarray, op_name: str, n_layers: int) -> np.ndarray:
+    """[n_sm, n_layers] dependency-met -> done µs of `op_name` (nan where the block has none)."""
+    tr = trace.reshape(schedule.shape[0], schedule.shape[1], -1).astype(np.int64)
+    out = np.full((schedule.shape[0], max(n_layers, 1)), np.nan)
+    for sm in range(schedule.shape[0]):
+        for i in range(schedule.shape[1]):
+            if OP_NAMES.get(int(schedule[sm, i, 0])) == op_name:
+                l = int(schedule[sm, i, 1])
+                if 0 <= l < out.shape[1] and tr[sm, i, T_DEP] > 0 and tr[sm, i, T_END] > 0:
+                    out[sm, l] = (tr[sm, i, T_END] - tr[sm, i, T_DEP]) / 1000.0
+    return out
+
+
+def format_breakdown(bd: dict) -> str:
+    lines = [f"{'op':8s} " + " ".join(f"{c:>8s}" for c in COLUMNS)]
+    for op, row in bd.items():
+        lines.append(f"{op:8s} " + " ".join(f"{row[c]:8.2f}" for c in COLUMNS))
+    return "\n".join(lines)
+
+
+def main(argv=None) -> None:
+    import argparse
+    import os
+    import sys
+
+    import torch
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import synth
+    from synth import configs
+
+    from .mk import Decoder, to_device
+
+    ap = argparse.ArgumentParser(description="per-op latency breakdown from the device trace")
+    ap.add_argument("config")
+    ap.add_argument("--steps", type=int, default=4)
+    ap.add_argument("--npz", default="")
+    ap.add_argument("options", nargs="*", help="mk_options fields as key=value (integers)")
+    args = ap.parse_args(argv)
+    cfg = configs.get(args.config)
+    opts = {k: int(v) for k, v in (kv.split("=") for kv in args.options)}
+    W = synth.make_model(cfg)
+    kc, vc = synth.make_kv_cache(cfg)
+    dk = torch.from_numpy(kc.view(np.int16)).cuda()
+    dv = torch.from_numpy(vc.view(np.int16)).cuda()
+    p0 = cfg.prefill + cfg.prompt_len
+    with Decoder(cfg, to_device(W), dk, dv, trace=1, **opts) as dec:
+        tok = dec.step(int(synth.prompt_tokens(cfg)[0]), p0)
+        for i in range(1, args.steps):
+            tok = dec.step(tok, p0 + i)
+        sched, tr = dec.schedule(), dec.trace()
+        print(f"{cfg.name}: last step {dec.last_step_ns() / 1000:.1f} us (traced)")
+    print(format_breakdown(op_breakdown(sched, tr)))
+    present = {OP_NAMES.get(int(o)) for o in np.unique(sched[:, :, 0])}
+    big = next((n for n in ("FFN", "MOE_FFN", "UG", "MOE_UG") if n in present), "LM")
+    d = per_sm_duration(sched, tr, big, cfg.n_layers)
+    mean = np.nanmean(d, axis=1)
+    print(f"{big} dependency->done per SM: mean {np.nanmean(mean):.2f} min {np.nanmin(mean):.2f} "
+          f"max {np.nanmax(mean):.2f} us; even/odd-layer correlation "
+          f"{np.corrcoef(np.nanmean(d[:, 0::2], 1), np.nanmean(d[:, 1::2], 1))[0, 1]:.2f}")
+    if args.npz:
+        np.savez(args.npz, schedule=sched, trace=tr.reshape(sched.shape[0], sched.shape[1], -1))
+
+
+if __name__ == "__main__":
+    main()
