@@ -18,6 +18,9 @@ Prints ONE JSON line (rank 0):
   cpu_baseline     the fp64 oracle on this host's cores, bounded sample
   baselines        the plain multi-kernel path of the same opcodes, stream
                    launches and a CUDA graph
+  per_config       the Llama-3B-shaped and Mixtral-shaped workloads timed the
+                   same way in the same run (value, roofline, e2e, clocks,
+                   baselines), beside the Llama-1B headline
 `--impl reference` times the fp64 oracle instead (rank 0 only).
 Multi-GPU (torchrun): independent replicas, one per GPU, no collective on the
 data path ("scaling": "weak").
@@ -66,10 +69,14 @@ def parse():
     ap.add_argument("--ring-stages", type=int, default=0)
     ap.add_argument("--stage-bytes", type=int, default=0)
     ap.add_argument("--kv-splits", type=int, default=0)
+    ap.add_argument("--claim-permille", type=int, default=0,
+                    help="fixed row share of the fused FFN and LM head per mille (0 = library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-baselines", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--per-config", type=int, default=1,
+                    help="1: with the default llama1b workload, also time llama3b and mixtral8l (per_config)")
     ap.add_argument("--calibrate", type=int, default=0,
                     help="1: split the FFN and LM-head rows by per-SM speed measured on this GPU at start-up")
     return ap.parse_args()
@@ -271,7 +278,10 @@ def bytes_per_token(cfg, positions):
 
 # ---- our arm --------------------------------------------------------------------------------------------
 
-def run_ours(args, rank, world, local):
+def measure(args, cfg, p0, positions, K, Wm, rank, world, local, with_extras=True):
+    """Device-timed steps of one workload through the megakernel (or the
+    multi-kernel path), plus the C-ABI end-to-end loops and the multi-kernel
+    baselines; returns the measured fields of one bench entry."""
     import numpy as np
     import torch
 
@@ -279,16 +289,18 @@ def run_ours(args, rank, world, local):
     from decode_persistent_block_b200 import Decoder, to_device
     from decode_persistent_block_b200.calibrate import measure_sm_speed
     torch.cuda.set_device(local)
-    cfg, p0, positions = workload(args)
     W = synth.make_model(cfg)
     kc, vc = synth.make_kv_cache(cfg)
     dW = to_device(W)
+    del W
     dk = torch.from_numpy(kc.view(np.int16)).cuda()
     dv = torch.from_numpy(vc.view(np.int16)).cuda()
+    del kc, vc
     first = int(synth.prompt_tokens(cfg)[0])
     mode = {"megakernel": 0, "multi_kernel": 1, "multi_kernel_graph": 2}[args.mode]
     opts = dict(mode=mode, l2_prefetch=args.l2_prefetch, ring_stages=args.ring_stages,
-                stage_bytes=args.stage_bytes, kv_splits=args.kv_splits, serve_idle_ns=2_000_000_000)
+                stage_bytes=args.stage_bytes, kv_splits=args.kv_splits, serve_idle_ns=2_000_000_000,
+                claim_permille=args.claim_permille)
     calib = None
     if args.calibrate and args.mode == "megakernel":
         # start-up calibration, outside the timed region: a few traced steps from p0
@@ -296,7 +308,6 @@ def run_ours(args, rank, world, local):
         opts["sm_speed"] = speed
         calib = {"steps": 8, "min": round(float(speed.min()), 3), "max": round(float(speed.max()), 3)}
     dec = Decoder(cfg, dW, dk, dv, **opts)
-    K, Wm = args.steps, args.warmup
 
     def timed(d, k, warm):
         d.step(first, positions[0])
@@ -351,7 +362,7 @@ def run_ours(args, rank, world, local):
     # (a profiler that runs each launch to completion before the host continues
     # cannot serve: the grid then leaves when idle and this measurement is skipped)
     e2e_serve = None
-    if not args.no_e2e and args.mode == "megakernel":
+    if with_extras and not args.no_e2e and args.mode == "megakernel":
         from decode_persistent_block_b200 import MkError
         torch.cuda.synchronize()
         dec.serve_start()
@@ -385,6 +396,48 @@ def run_ours(args, rank, world, local):
                 tms, _ = timed(b, kb, 3)
                 baselines[name] = round(reduce_max(tms, world) * 1000.0 / (kb * world), 3)
     dec.close()
+    del dW, dk, dv
+    torch.cuda.empty_cache()
+    return {
+        "value": round(us_per_token, 3), "tokens_per_s": round(1e6 / us_per_token, 1),
+        "hbm_gbs": round(achieved, 1), "frac_of_8tbs": round(achieved / ROOFLINE_NOMINAL_GBS, 4),
+        "floor_us_at_8tbs": round(byte_floor_us(bpt, ROOFLINE_NOMINAL_GBS), 1), "bytes_per_token": int(bpt),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+                     "traffic": committed_traffic(cfg.name, args.mode), "launch_us": round(launch_ms * 1000, 2)},
+        "e2e": e2e, "e2e_serve": e2e_serve, "baselines": baselines, "clocks": clk, "calib": calib,
+        "steps": K, "warmup": Wm,
+    }
+
+
+def workload_name(cfg, p0):
+    return (f"{cfg.name}: batch-1 greedy decode, KV pre-filled to {cfg.prefill}, positions "
+            f"{p0}..{p0 + cfg.steps - 1}")
+
+
+# The other target shape and the MoE shape, measured in the same run as the headline workload (fewer
+# timed steps each: their steps are 2-3x longer), so every target config has a number in one bench line.
+PER_CONFIG = (("llama3b", 384), ("mixtral8l", 256))
+
+
+def run_ours(args, rank, world, local):
+    from synth import configs
+    cfg, p0, positions = workload(args)
+    K, Wm = args.steps, args.warmup
+    r = measure(args, cfg, p0, positions, K, Wm, rank, world, local)
+
+    per_config = {}
+    if args.per_config and not args.layers and args.config == "llama1b":
+        for name, k in PER_CONFIG:
+            c2 = configs.get(name)
+            q0 = c2.prefill + c2.prompt_len
+            pos2 = [q0 + (i % c2.steps) for i in range(max(k, Wm) + 1)]
+            m = measure(args, c2, q0, pos2, min(k, K), Wm, rank, world, local, with_extras=False)
+            per_config[name] = {"workload": workload_name(c2, q0), "value": m["value"], "unit": UNIT,
+                                "tokens_per_s": m["tokens_per_s"], "roofline": m["roofline"],
+                                "frac_of_8tbs": m["frac_of_8tbs"], "bytes_per_token": m["bytes_per_token"],
+                                "e2e": m["e2e"], "baselines": m["baselines"], "clocks": m["clocks"],
+                                "steps": m["steps"], "warmup": m["warmup"]}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -399,29 +452,27 @@ def run_ours(args, rank, world, local):
     if rank != 0:
         return None
     line = {
-        "metric": METRIC, "value": round(us_per_token, 3), "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": Wm, "ms_per_step": round(us_per_token * world / 1000.0, 6), "higher_is_better": False,
+        "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": round(r["value"] * world / 1000.0, 6), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16 weights/KV, fp32 accumulate",
         "data": "synthetic random-init weights and KV prefill (seeded generator)",
-        "config": {"workload": f"{cfg.name}: batch-1 greedy decode, KV pre-filled to {cfg.prefill}, positions "
-                               f"{p0}..{p0 + cfg.steps - 1}", "layers": cfg.n_layers, "hidden": cfg.hidden,
+        "config": {"workload": workload_name(cfg, p0), "layers": cfg.n_layers, "hidden": cfg.hidden,
                    "vocab": cfg.vocab, "mode": args.mode, "parallelism": f"replicas x{world}",
-                   "l2": f"no flush: {bpt / 1e9:.2f} GB streamed per token > 126 MB L2",
-                   "sm_speed": calib or "equal"},
-        "tokens_per_s": round(1e6 / us_per_token, 1),
-        "hbm_gbs": round(achieved, 1),
-        "frac_of_8tbs": round(achieved / ROOFLINE_NOMINAL_GBS, 4),
-        "floor_us_at_8tbs": round(byte_floor_us(bpt, ROOFLINE_NOMINAL_GBS), 1),
-        "bytes_per_token": int(bpt),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
-                     "traffic": committed_traffic(cfg.name, args.mode), "launch_us": round(launch_ms * 1000, 2)},
-        "e2e": e2e,
-        "e2e_serve": e2e_serve,
+                   "l2": f"no flush: {r['bytes_per_token'] / 1e9:.2f} GB streamed per token > 126 MB L2",
+                   "sm_speed": r["calib"] or "equal"},
+        "tokens_per_s": r["tokens_per_s"],
+        "hbm_gbs": r["hbm_gbs"],
+        "frac_of_8tbs": r["frac_of_8tbs"],
+        "floor_us_at_8tbs": r["floor_us_at_8tbs"],
+        "bytes_per_token": r["bytes_per_token"],
+        "roofline": r["roofline"],
+        "e2e": r["e2e"],
+        "e2e_serve": r["e2e_serve"],
         "gpu_launches": K if args.mode == "megakernel" else None,
-        "baselines": baselines,
+        "baselines": r["baselines"],
+        "per_config": per_config or None,
         "cpu_baseline": cpu,
-        "clocks": clk,
+        "clocks": r["clocks"],
     }
     if args.mode != "megakernel":
         per_step = 6 * cfg.n_layers + 3 + (cfg.n_layers * cfg.top_k if cfg.n_experts else 0)

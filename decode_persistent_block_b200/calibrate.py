@@ -21,7 +21,7 @@ T_DEP, T_END = 1, 5
 
 def sm_speed_from_trace(schedule: np.ndarray, trace: np.ndarray, hidden: int):
     """(bytes, ns) per block from one step's schedule [n_sm, max_instr, 16] and
-    trace [n_sm, max_instr, 8]: each dense fused-FFN row streams 3 weight rows
+    trace [n_sm, max_instr, words]: each dense fused-FFN row streams 3 weight rows
     (up, gate, transposed down) of `hidden` bf16, and each LM-head row one."""
     n_sm = schedule.shape[0]
     nbytes = np.zeros(n_sm)

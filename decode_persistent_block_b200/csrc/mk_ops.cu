@@ -220,8 +220,27 @@ static __device__ __align__(256) float g_attn_noalloc_scratch[MK_ATTENTION_NOALL
 
 namespace {
 constexpr int kMaxDevices = 64;
-float* g_scratch_addr[kMaxDevices];  // device address of the array, per device ordinal (host-side cache)
+// Host-side cache of the array's device address, per device ordinal, with the
+// context it was looked up in: a device reset (cudaDeviceReset) gives the
+// device a new context and the module a new address, so the lookup is redone
+// whenever the current context differs from the cached one.
+float* g_scratch_addr[kMaxDevices];
+CUcontext g_scratch_ctx[kMaxDevices];
 std::mutex g_scratch_mu;
+
+CUresult current_context(CUcontext* ctx) {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    static GetCurrent fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !p)
+            return CUDA_ERROR_NOT_FOUND;
+        fn = reinterpret_cast<GetCurrent>(p);
+    }
+    return fn(ctx);
+}
 }  // namespace
 
 extern "C" int mk_attention_decode_noalloc(const float* q, const void* k_cache, const void* v_cache, int n_q_heads,
@@ -238,10 +257,13 @@ extern "C" int mk_attention_decode_noalloc(const float* q, const void* k_cache, 
         // Set-up, once per device, with that device current: the array's name is a
         // host-side stand-in, so its device address has to be looked up.
         std::lock_guard<std::mutex> lock(g_scratch_mu);
-        if (!g_scratch_addr[dev]) {
+        CUcontext ctx = nullptr;
+        if (!g_scratch_addr[dev] || current_context(&ctx) != CUDA_SUCCESS || ctx != g_scratch_ctx[dev]) {
             void* addr = nullptr;
             if (cudaGetSymbolAddress(&addr, g_attn_noalloc_scratch) != cudaSuccess || !addr) return MK_ERR_CUDA;
+            if (current_context(&ctx) != CUDA_SUCCESS) ctx = nullptr;
             g_scratch_addr[dev] = static_cast<float*>(addr);
+            g_scratch_ctx[dev] = ctx;
         }
         scratch = g_scratch_addr[dev];
     }

@@ -7,6 +7,10 @@ not reached) per instruction of the schedule [n_sm][max_instr]:
   4 main stages consumed, 5 done and signalled (consumer warps);
   6 first stage issued, 7 last stage issued (loader warp).
 
+Records of 32 words add, for each instruction's first 8 ring stages, consumer
+thread 0's full-barrier wait returned (8 + s), its share of the stage consumed
+(16 + s) and the loader's issue (24 + s); `stage_breakdown` reduces those.
+
 `op_breakdown` reduces them to the phases of each op, averaged over layers:
   phase   previous op's last end -> this op's last end (the op's share of the step)
   hop     previous op's last end -> dependency met (mean over blocks)
@@ -30,6 +34,8 @@ OP_NAMES = {1: "QKV", 2: "ATTN", 3: "OPROJ", 4: "UG", 5: "DOWN", 6: "LM", 7: "MO
 ORDER = ["QKV", "ATTN", "OPROJ", "UG", "DOWN", "FFN", "MOE_UG", "MOE_DOWN", "MOE_FFN", "LM"]
 COLUMNS = ["phase", "hop", "ready", "first", "main", "epi", "spread", "ld_lead", "ld_last"]
 T_START, T_DEP, T_READY, T_FIRST, T_MAIN, T_END, T_LD_FIRST, T_LD_LAST = range(8)
+N_STAGES = 8
+T_SREADY, T_SDONE, T_SISSUE = 8, 8 + N_STAGES, 8 + 2 * N_STAGES
 
 
 def _groups(schedule: np.ndarray, trace: np.ndarray):
@@ -72,6 +78,40 @@ def op_breakdown(schedule: np.ndarray, trace: np.ndarray) -> dict:
         prev_end = end_max
         agg.setdefault(key[1], []).append(row)
     return {op: {c: _mean([r[c] for r in agg[op]]) for c in COLUMNS} for op in ORDER if op in agg}
+
+
+def stage_breakdown(schedule: np.ndarray, trace: np.ndarray, n_stages: int = 4) -> dict:
+    """{op name: [n_stages][3] mean µs over blocks and layers} from the per-stage stamps:
+    wait (previous stage consumed, or the input vector ready, -> this stage's wait returned),
+    consume (wait returned -> consumed) and lead (loader issue -> wait returned)."""
+    g = _groups(schedule, trace)
+    acc: dict = {}
+    for (layer, op), a in g.items():
+        if a.shape[1] < T_SISSUE + N_STAGES:
+            return {}
+        rows = []
+        for s in range(n_stages):
+            prev = a[:, T_SDONE + s - 1] if s > 0 else np.fmax(a[:, T_READY], a[:, T_DEP])
+            rows.append([a[:, T_SREADY + s] - prev, a[:, T_SDONE + s] - a[:, T_SREADY + s],
+                         a[:, T_SREADY + s] - a[:, T_SISSUE + s]])
+        acc.setdefault(op, []).append(np.array(rows))  # [stages][3][blocks]
+    out = {}
+    for op in ORDER:
+        if op in acc:
+            cat = np.concatenate(acc[op], axis=2)
+            with np.errstate(all="ignore"):
+                out[op] = [[_mean(cat[s, k]) for k in range(3)] for s in range(n_stages)]
+    return out
+
+
+def format_stages(sb: dict) -> str:
+    if not sb:
+        return ""
+    n = len(next(iter(sb.values())))
+    lines = [f"{'op':8s} " + " ".join(f"{'s%d wait/cons/lead' % s:>20s}" for s in range(n))]
+    for op, st in sb.items():
+        lines.append(f"{op:8s} " + " ".join(f"{w:6.2f}/{c:5.2f}/{l:6.2f} " for w, c, l in st))
+    return "\n".join(lines)
 
 
 def _mean(xs) -> float:
@@ -133,6 +173,7 @@ def main(argv=None) -> None:
         sched, tr = dec.schedule(), dec.trace()
         print(f"{cfg.name}: last step {dec.last_step_ns() / 1000:.1f} us (traced)")
     print(format_breakdown(op_breakdown(sched, tr)))
+    print(format_stages(stage_breakdown(sched, tr)))
     present = {OP_NAMES.get(int(o)) for o in np.unique(sched[:, :, 0])}
     big = next((n for n in ("FFN", "MOE_FFN", "UG", "MOE_UG") if n in present), "LM")
     d = per_sm_duration(sched, tr, big, cfg.n_layers)

@@ -135,6 +135,10 @@ typedef struct {
                              grid's block count.  Read (copied) by mk_create and mk_plan; the caller may
                              free it afterwards */
     int n_sm_speed;
+    int claim_permille;   /* dense fused FFN and LM head: each block's fixed share of the rows, per mille of
+                             an even split (0 = default, 1..1000); the remaining rows are claimed at run time
+                             in stage-sized chunks from a per-op counter by whichever block is ready first,
+                             so the op ends together on every SM.  1000 = fixed shares only */
 } mk_options;
 
 /* Device status block, copied out by mk_get_status.  On a device-side error
@@ -157,18 +161,31 @@ void mk_default_options(mk_options *out);
 /* Create a handle: validates the config and pointers, allocates the library's
  * device buffers (instruction tensor, counters, fp32 activations, status) on
  * the current device and binds `cuda_stream` (a cudaStream_t, NULL = legacy
- * default stream).  Errors: MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_CUDA. */
+ * default stream).  Errors: MK_ERR_INVALID_ARG, MK_ERR_UNSUPPORTED, MK_ERR_CUDA.
+ * Source: the one-time host set-up before the persistent kernel's first launch
+ * -- weights placed at the addresses the plan names, the kernel's buffers and
+ * launch shape fixed (Hyperkernel teardown, "What is in the repository"); the
+ * shapes it accepts are the Llama and Mixtral decoders of the epic-kernel
+ * README ("3B model support", "Mixtral 8x7B MoE for batch-1 inference"). */
 int mk_create(const mk_config *cfg, const mk_weights *w, const mk_options *opt, void *cuda_stream,
               mk_handle **out);
 
 /* Build, validate and upload the instruction schedule (host work, done once).
  * Deterministic: the instruction words depend only on (config, options, SMs).
- * Errors: MK_ERR_SCHEDULE (validator), MK_ERR_CUDA. */
+ * Errors: MK_ERR_SCHEDULE (validator), MK_ERR_CUDA.
+ * Source: the instruction tensor each block reads at run time to learn which
+ * op it runs next (Kittens VM summary page, "Method"); a schedule whose
+ * grid-wide waits cannot deadlock and that keeps every SM busy across ops of
+ * different shapes is one of the hard parts the Hyperkernel teardown names
+ * ("What a megakernel buys"). */
 int mk_build_schedule(mk_handle *h);
 
 /* Copy the instruction tensor ([n_sm][max_instr][MK_INSTR_WORDS] int32, unused
- * slots zero) to host `buf` of `cap` words.  *n_words receives the size. */
-#define MK_INSTR_WORDS 16
+ * slots zero) to host `buf` of `cap` words.  *n_words receives the size.
+ * Errors: MK_ERR_NO_SCHEDULE, MK_ERR_CAPACITY (cap too small; *n_words is set).
+ * Source: the same instruction tensor (Kittens VM summary page, "Method"),
+ * exposed so that schedules can be checked on the host. */
+#define MK_INSTR_WORDS 24
 int mk_get_schedule(mk_handle *h, int32_t *buf, size_t cap, size_t *n_words, int *n_sm, int *max_instr);
 
 /* One decode step: embeds `token` (or, if token < 0, the previous step's
@@ -180,32 +197,52 @@ int mk_get_schedule(mk_handle *h, int32_t *buf, size_t cap, size_t *n_words, int
  * device-side errors surface at the next synchronous call or mk_get_status.
  * Positions must be stepped in order: pos reads cache entries 0..pos-1.
  * Errors: MK_ERR_INVALID_ARG, MK_ERR_NO_SCHEDULE, MK_ERR_TIMEOUT,
- * MK_ERR_BAD_INSTR, MK_ERR_STOPPED, MK_ERR_CUDA. */
+ * MK_ERR_BAD_INSTR, MK_ERR_STOPPED, MK_ERR_CUDA.
+ * Source: one megakernel launch per call, the whole forward pass inside it
+ * (Hyperkernel teardown, "A single kernel launch, read from the host": one
+ * launch per call); the forward is the batch-1 decode step of the epic-kernel
+ * README's models, the next-token choice the greedy argmax. */
 int mk_decode_step(mk_handle *h, int32_t token, int32_t pos, float *logits_dev, int32_t *next_token_host);
 
 /* Residual stream after layer `layer` of the last step (0 = embedding,
  * n_layers = after the last layer) as fp32 [hidden] into host `out_host`.
- * Needs options.snapshots = 1.  Synchronises the stream. */
+ * Needs options.snapshots = 1.  Synchronises the stream.
+ * Source: per-layer checks against a reference, the kind of correctness
+ * evidence the Hyperkernel teardown asks a megakernel release to ship ("What a
+ * megakernel buys": correctness checks good enough to trust the result). */
 int mk_get_hidden(mk_handle *h, int layer, float *out_host);
 
 /* MoE routing of `layer` in the last step: top_k expert ids and weights
- * (host arrays of top_k entries).  MK_ERR_INVALID_ARG for dense models. */
+ * (host arrays of top_k entries).  MK_ERR_INVALID_ARG for dense models.
+ * Source: the router scoring and expert selection the epic-kernel README fuses
+ * into its MoE instructions ("Mixtral 8x7B MoE for batch-1 inference"). */
 int mk_get_router(mk_handle *h, int layer, int32_t *idx, float *w);
 
-/* Dependency counters (uint32, monotone across steps) into host `out`. */
+/* Dependency counters (uint32, monotone across steps) into host `out`.
+ * Source: the blocks synchronise on the device instead of through kernel
+ * boundaries (Hyperkernel teardown, "What a megakernel buys"); these are the
+ * global-memory counters they synchronise on. */
 int mk_get_counters(mk_handle *h, uint32_t *out, size_t cap, size_t *n);
 
 /* Per-counter increment per step, as planned by the scheduler (host `out`). */
 int mk_get_counter_increments(mk_handle *h, uint32_t *out, size_t cap, size_t *n);
 
-/* Copy the device status block (synchronises the stream). */
+/* Copy the device status block (synchronises the stream).
+ * Source: the control block with a watchdog word, a stop word and bounds
+ * flags, and a host that reports a failed step instead of a number
+ * (Hyperkernel teardown, "Hardware fault detection and replanning"). */
 int mk_get_status(mk_handle *h, mk_status *out);
 
-/* Trace stamps of the last step: [n_sm][max_instr][8] uint64 globaltimer ns,
+/* Trace stamps of the last step: [n_sm][max_instr][32] uint64 globaltimer ns,
  * zero where not reached.  Consumer warps: 0 instruction reached, 1 dependency
  * satisfied, 2 input vector ready, 3 first stage full, 4 main stages consumed
  * (the fused FFN's up/gate rows), 5 done and signalled.  Loader warp: 6 first
- * stage issued, 7 last stage issued.  Needs options.trace = 1. */
+ * stage issued, 7 last stage issued.  Then for the instruction's first 8 ring
+ * stages s: 8 + s consumer thread 0's wait for the stage returned, 16 + s its
+ * share of the stage consumed, 24 + s the loader issued the stage.  Needs
+ * options.trace = 1.
+ * Source: the per-instruction timing trace the epic-kernel README records for
+ * its SM-occupancy and HBM-utilisation plots (its profiling instructions). */
 int mk_get_trace(mk_handle *h, uint64_t *out, size_t cap, size_t *n);
 
 /* Clear counters, epoch, status and stop word and re-upload the schedule
@@ -287,8 +324,9 @@ int mk_attention_decode(const float *q, const void *k_cache, const void *v_cache
  *    n_q_heads * splits * (head_dim + 2) floats exceed it returns
  *    MK_ERR_CAPACITY.
  *  - The first call on a device looks up the array's device address (once
- *    per device, with that device current); make that first call before any
- *    stream capture.
+ *    per device, with that device current, and again after the device's
+ *    context has changed, e.g. after cudaDeviceReset); make that first call
+ *    before any stream capture.
  *  - All calls share the array: calls that overlap on the GPU (for example on
  *    two streams at once) race and give wrong results; serialise them.  Each
  *    call writes every slot it reads, so no clearing is needed between calls. */

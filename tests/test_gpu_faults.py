@@ -92,7 +92,8 @@ def test_trace_stamps_are_ordered(tiny):
     with tiny.decoder(trace=1) as dec:
         dec.step(3, 0)
         sched = dec.schedule()
-        tr = dec.trace().reshape(sched.shape[0], -1, 8).astype(np.int64)
+        tr = dec.trace().reshape(sched.shape[0], sched.shape[1], -1).astype(np.int64)
+        assert tr.shape[2] == 32  # 8 instruction stamps, then 8 stages x (ready, consumed, issued)
         n = (sched[:, :, 0] != 0).sum(1)
         for sm in range(tr.shape[0]):
             t = tr[sm, :n[sm]]
@@ -105,3 +106,8 @@ def test_trace_stamps_are_ordered(tiny):
             # loader: the first stage of an instruction is issued before its consumers see it full
             hit = (t[:, 6] > 0) & (t[:, 3] > 0)
             assert np.all(t[hit, 3] >= t[hit, 6]) and np.all(t[t[:, 7] > 0, 7] >= t[t[:, 7] > 0, 6])
+            # per stage: issued <= the consumers' wait returned <= their share consumed
+            for s_ in range(8):
+                ready, done, issued = t[:, 8 + s_], t[:, 16 + s_], t[:, 24 + s_]
+                hit = (ready > 0) & (done > 0) & (issued > 0)
+                assert np.all(done[hit] >= ready[hit]) and np.all(ready[hit] >= issued[hit]), (sm, s_)

@@ -155,3 +155,53 @@ def test_idle_grid_leaves_by_itself(tiny):
         dec.step(-1, 1)  # the per-launch path works again
     finally:
         dec.close()
+
+
+def _served_vs_oracle(setup, steps=None, **opts):
+    """Teacher-forced launch-once serving against the fp64 oracle: every served
+    step's logits and token, then (after the grid has left) the last step's
+    per-layer hidden states."""
+    import torch
+    from decode_persistent_block_b200 import Decoder
+    cfg = setup.cfg
+    orc = setup.oracle()
+    setup.fresh_caches()
+    torch.cuda.synchronize()
+    lg = torch.empty(cfg.vocab, device="cuda")
+    s = torch.cuda.Stream()
+    reports = []
+    dec = Decoder(cfg, setup.dW, setup.dk, setup.dv, stream=s, serve_idle_ns=IDLE, snapshots=1, **opts)
+    try:
+        dec.serve_start(lg)
+        nxt = None
+        for pos, tok in parity.schedule(cfg, steps):
+            t = tok if tok is not None else nxt
+            got = dec.serve_step(t, pos)
+            o = orc.step(t, pos)
+            lo = o["logits"]
+            srt = np.sort(lo)
+            reports.append({"logit_err": float(np.max(np.abs(lg.cpu().numpy().astype(np.float64) - lo))),
+                            "margin": float(srt[-1] - srt[-2]), "next_orc": o["next"], "next_gpu": got, "pos": pos})
+            nxt = o["next"]
+        dec.serve_stop()
+        assert dec.status()["code"] == 0
+        hg = dec.hidden_all().astype(np.float64)
+        ho = o["hidden"]
+        reports[-1]["hidden_rel"] = (np.linalg.norm(hg - ho, axis=1) /
+                                     np.maximum(np.linalg.norm(ho, axis=1), 1e-30)).tolist()
+    finally:
+        dec.close()
+    return reports
+
+
+@pytest.mark.parametrize("split_ffn", [0, 1], ids=["fused_ffn", "split_ffn"])
+def test_served_steps_match_oracle_tiny(tiny, split_ffn):
+    reps = _served_vs_oracle(tiny, split_ffn=split_ffn)
+    assert len(reps) == configs.TINY.prompt_len + configs.TINY.steps
+    parity.assert_parity(reps)
+
+
+def test_served_steps_match_oracle_llama1b(cuda):
+    # the full-size shape in the benchmark's launch configuration (default options), 3 positions
+    reps = _served_vs_oracle(parity.Setup(configs.LLAMA_1B), steps=3)
+    parity.assert_parity(reps)

@@ -13,6 +13,7 @@ import ctypes
 import numpy as np
 import pytest
 
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -62,3 +63,28 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(cuda):
     mk.attention_decode_noalloc(q, kc, vc, 64, ok, out)
     torch.cuda.synchronize()
     assert np.max(np.abs(out.cpu().numpy() - ref.cpu().numpy())) <= 1e-5 * max(1.0, ref.abs().max().item())
+
+
+def _oracle_attention(q, kc, vc, n_pos):
+    """fp64 attention of every query head (the oracle's definition) on the bf16 caches."""
+    qh, k16, v16 = q.cpu().numpy(), kc.cpu().numpy().view(np.uint16), vc.cpu().numpy().view(np.uint16)
+    nq, nkv = qh.shape[0], k16.shape[0]
+    return np.stack([oracle.attend(qh[h].astype(np.float64), k16[h // (nq // nkv), :n_pos],
+                                   v16[h // (nq // nkv), :n_pos]) for h in range(nq)])
+
+
+def test_noalloc_matches_oracle_after_a_larger_call(cuda):
+    """A call with many splits and heads fills more of the shared scratch than
+    the call after it; the second call, with fewer splits and heads, must not
+    read any partial the first one left behind: both match the fp64 oracle."""
+    import torch
+    from decode_persistent_block_b200 import mk
+    rng = np.random.default_rng(7)
+    for nq, nkv, d, n_pos, splits in ((32, 8, 128, 3000, 40), (4, 2, 64, 37, 3)):
+        q, kc, vc = _inputs(rng, nq, nkv, d, n_pos, n_pos + 5)
+        got = torch.full_like(q, float("nan"))
+        mk.attention_decode_noalloc(q, kc, vc, n_pos, splits, got)
+        torch.cuda.synchronize()
+        ref = _oracle_attention(q, kc, vc, n_pos)
+        g = got.cpu().numpy().astype(np.float64)
+        assert np.max(np.abs(g - ref)) <= 1e-5 * max(1.0, np.max(np.abs(ref))), (nq, splits, np.max(np.abs(g - ref)))
