@@ -69,8 +69,6 @@ def parse():
     ap.add_argument("--ring-stages", type=int, default=0)
     ap.add_argument("--stage-bytes", type=int, default=0)
     ap.add_argument("--kv-splits", type=int, default=0)
-    ap.add_argument("--claim-permille", type=int, default=0,
-                    help="fixed row share of the fused FFN and LM head per mille (0 = library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-baselines", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -299,8 +297,7 @@ def measure(args, cfg, p0, positions, K, Wm, rank, world, local, with_extras=Tru
     first = int(synth.prompt_tokens(cfg)[0])
     mode = {"megakernel": 0, "multi_kernel": 1, "multi_kernel_graph": 2}[args.mode]
     opts = dict(mode=mode, l2_prefetch=args.l2_prefetch, ring_stages=args.ring_stages,
-                stage_bytes=args.stage_bytes, kv_splits=args.kv_splits, serve_idle_ns=2_000_000_000,
-                claim_permille=args.claim_permille)
+                stage_bytes=args.stage_bytes, kv_splits=args.kv_splits, serve_idle_ns=2_000_000_000)
     calib = None
     if args.calibrate and args.mode == "megakernel":
         # start-up calibration, outside the timed region: a few traced steps from p0

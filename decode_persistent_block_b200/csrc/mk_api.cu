@@ -242,7 +242,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     std::memset(&p, 0, sizeof(p));
     p.L = L; p.H = H; p.nq = nq; p.nkv = nkv; p.d = d; p.F = c.ffn; p.V = c.vocab; p.E = E;
     p.topk = E > 0 ? c.top_k : 0; p.max_seq = c.max_seq; p.eps = c.rms_eps; p.kv_splits = S;
-    p.n_ctr = mk::n_counters(L, nkv);
+    p.n_ctr = mk::n_counters(L);
     p.embed = static_cast<const uint16_t*>(w->embed);
     p.lm_head = static_cast<const uint16_t*>(w->lm_head);
     p.final_norm = static_cast<const uint16_t*>(w->final_norm);
@@ -315,25 +315,6 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
         e = cudaDeviceSynchronize();
         if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
         h->down_t = true;
-    }
-    // The O-projection runs per kv group over that group's columns of w_o: keep a group-major
-    // copy [n_kv][hidden][group * head_dim] of every w_o (library-owned), so that the rows a block
-    // streams are contiguous.
-    if (o.mode == MK_MODE_MEGAKERNEL && L > 0) {
-        const size_t gcols = (size_t)(nq / nkv) * d, qd = (size_t)nq * d;
-        for (int l = 0; l < L; ++l) {
-            const uint16_t** t = &h->wt_host[(size_t)l * stride];
-            uint16_t* og = nullptr;
-            if ((rc = dalloc(h, &og, (size_t)H * qd))) return fail(rc);
-            for (int g = 0; g < nkv; ++g) {
-                e = cudaMemcpy2D(og + (size_t)g * H * gcols, gcols * 2, t[mk::WT_O] + (size_t)g * gcols, qd * 2,
-                                 gcols * 2, (size_t)H, cudaMemcpyDeviceToDevice);
-                if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
-            }
-            t[mk::WT_O_G] = og;
-        }
-        e = cudaDeviceSynchronize();
-        if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
     }
     p.wt = wt_dev;
     p.rope = rope;

@@ -73,6 +73,22 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// The same with an L2 cache policy (make_evict_first_policy): the copy's lines are
+// the first candidates for eviction, so a stream read once per step does not push
+// the data that is reused across steps (KV cache, activations, counters) out of L2.
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+// L2 policy for the whole of a copy: evict first.
+__device__ __forceinline__ uint64_t make_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
 // 2-D tensor-map box load (coordinates: x = column, y = row) into shared
 // memory, completion as transaction bytes on `bar`.  x * 2 bytes is a
 // multiple of 16 at every call site.  Never the multicast form.

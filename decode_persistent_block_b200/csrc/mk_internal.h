@@ -26,7 +26,7 @@ enum Opcode : int32_t {
     OP_NOP = 0,
     OP_RMS_QKV = 1,          // xn = rmsnorm(x) * w_attn; rows of [Wq; Wk; Wv] xn (raw, pre-RoPE)
     OP_ATTN = 2,             // RoPE + KV append + one split of GQA decode attention (partial o, m, l)
-    OP_OPROJ_RES = 3,        // x[rows] += Wo[rows, cols of kv group g] attn_g (atomics; the QKV op set x to the residual)
+    OP_OPROJ_RES = 3,        // x[rows] = x[rows] + Wo[rows] attn   (layer 0: embed row + ...)
     OP_RMS_UPGATE_SILU = 4,  // h[rows] = silu(Wg[rows] xn) * (Wu[rows] xn), xn = rmsnorm(x) * w_ffn
     OP_DOWN_RES = 5,         // x[rows] += Wd[rows] h
     OP_LMHEAD_ARGMAX = 6,    // logits[rows] = Wlm[rows] rmsnorm(x) * w_final; last instruction reduces argmax
@@ -51,17 +51,6 @@ enum Word : int {
     W_AUX_CTR = 8,    // ATTN: per-head-group arrival counter; LMHEAD: arrival counter
     W_AUX_INC = 9,    // its per-step increment
     W_SEQ = 10,       // LMHEAD: slot of this instruction's partial argmax; ATTN: unused
-    W_INIT0 = 11,     // QKV: 8-element chunks [W_INIT0, W_INIT1) of the residual this block copies into the
-    W_INIT1 = 12,     //   O-projection's accumulator x (and x2 at layer 0); empty range: none
-    // Run-time row claiming (dense fused FFN, LM head): after its fixed rows [W_BEGIN, W_END), the
-    // instruction claims chunks of W_CLAIM_ROWS rows of the op's pool [W_POOL0, W_POOL0 + W_POOL_N)
-    // from counter W_CLAIM_CTR (-1: no claims) until a claim lands past the pool; every step adds
-    // exactly W_CLAIM_INC (= chunks + claiming instructions) to that counter.
-    W_CLAIM_CTR = 13,
-    W_CLAIM_INC = 14,
-    W_POOL0 = 15,
-    W_POOL_N = 16,
-    W_CLAIM_ROWS = 17,
     W_NWORDS = MK_INSTR_WORDS
 };
 
@@ -72,28 +61,17 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;  // + one loader warp
 constexpr int kMaxGroup = 4;         // query heads per kv head
-constexpr int kMaxKvHeads = 256;
-constexpr int kMaxRingStages = 32;
 constexpr int kMaxHeadDim = 128;
-constexpr int kMaxOprojCols = kMaxGroup * kMaxHeadDim;  // columns of one kv group's O-projection
 constexpr int kMaxTopK = 2;
 constexpr int kMaxMergeSlots = 2048;  // query heads x kv splits merged in the O-projection prologue
 constexpr int kDefaultL2HeadStart = 0;  // ring stages of an FFN / LM-head stream prefetched into L2 past the ring
-constexpr int kDefaultClaimPermille = 1000;  // fixed row share of the dense fused FFN and LM head (1000: no claims)
 
-// Counter ids: per layer [QKV, ATTN (unused: attention signals per kv group), OPROJ, FFN1, FFN2],
-// then the LM head's arrival counter, then one attention counter per (layer, kv group): the
-// splits of group g signal it and the O-projection blocks of group g wait on it.
+// Counter ids: per layer [QKV, ATTN (one signal per split), OPROJ, FFN1, FFN2], then the LM head's
+// arrival counter.
 enum CtrSlot : int { C_QKV = 0, C_ATTN = 1, C_OPROJ = 2, C_FFN1 = 3, C_FFN2 = 4, kCountersPerLayer = 5 };
 MK_HD inline int ctr_id(int layer, int slot) { return layer * kCountersPerLayer + slot; }
 MK_HD inline int ctr_lm(int n_layers) { return n_layers * kCountersPerLayer; }
-MK_HD inline int ctr_attn_group(int n_layers, int n_kv, int layer, int g) {
-    return n_layers * kCountersPerLayer + 1 + layer * n_kv + g;
-}
-// The last counter: the LM head's claim counter.  The fused FFN's claims use the layer's FFN1 slot
-// (the mid-FFN signal only split-FFN schedules use).
-MK_HD inline int n_counters(int n_layers, int n_kv) { return n_layers * (kCountersPerLayer + n_kv) + 2; }
-MK_HD inline int ctr_lm_claim(int n_layers, int n_kv) { return n_layers * (kCountersPerLayer + n_kv) + 1; }
+MK_HD inline int n_counters(int n_layers) { return n_layers * kCountersPerLayer + 1; }
 
 // Trace record of one instruction (options.trace): globaltimer stamps in ns,
 // zero where not reached.  Consumer side: reached, dependency satisfied,
@@ -111,11 +89,8 @@ enum TraceStamp : int {
 
 // Weight pointer table: per layer kLayerFixed entries, then gate/up/down per expert.
 // Slot wt_down_t holds the library's transposed copy [ffn][hidden] of w_down
-// (null unless the fused FFN is used).  WT_O_G holds the library's group-major
-// copy of w_o, [n_kv][hidden][group * head_dim]: the columns of kv group g
-// (its query heads' outputs) for every output row, contiguous per row
-// (megakernel mode only).
-enum WSlot : int { WT_ATTN_NORM = 0, WT_Q, WT_K, WT_V, WT_O, WT_FFN_NORM, WT_ROUTER, WT_O_G, kLayerFixed };
+// (null unless the fused FFN is used).
+enum WSlot : int { WT_ATTN_NORM = 0, WT_Q, WT_K, WT_V, WT_O, WT_FFN_NORM, WT_ROUTER, kLayerFixed };
 MK_HD inline int wt_stride(int n_experts) { return kLayerFixed + 4 * (n_experts > 0 ? n_experts : 1); }
 MK_HD inline int wt_gate(int e) { return kLayerFixed + e; }
 MK_HD inline int wt_up(int e, int n_experts) { return kLayerFixed + (n_experts > 0 ? n_experts : 1) + e; }
@@ -128,7 +103,7 @@ MK_HD inline int wt_down_t(int e, int n_experts) { return kLayerFixed + 3 * (n_e
 MK_HD inline int kparts_of(int K) { return (K + kMaxPartK - 1) / kMaxPartK; }
 MK_HD inline int acc_sets(int op, int H, int qd, int F, int topk) {
     switch (op) {
-        case OP_OPROJ_RES: return 1;  // whole rows per warp, no per-warp slots
+        case OP_OPROJ_RES: return kparts_of(qd);
         case OP_RMS_UPGATE_SILU:
         case OP_MOE_UPGATE:
         case OP_FFN:

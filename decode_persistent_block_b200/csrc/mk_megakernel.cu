@@ -64,11 +64,6 @@ struct Misc {
     // serving: the step block 0 published, as taken by this block's consumer thread 0
     int s_go, s_token, s_pos, s_seq;
     uint32_t s_epoch;
-    // run-time claims: the rows (first, count) the loader put in each ring slot's stage (count 0:
-    // the claim landed past the pool, no more stages), and consumer thread 0's reading of the
-    // current chunk (first, count, ok) broadcast to the block
-    int2 sinfo[kMaxRingStages];
-    int c_row0, c_rows, c_ok;
 };
 
 __host__ __device__ inline size_t smem_bars_off(int ns, int sb) { return (size_t)ns * sb; }
@@ -151,41 +146,6 @@ __device__ bool warp_wait_full(uint64_t* bar, uint32_t parity, const DevParams& 
     return ok != 0;
 }
 
-// Run-time claims, consumer side: thread 0 waits (bounded) for the next claimed
-// stage -- and, for a fused-FFN chunk, for its down-projection stage in the
-// following slot -- reads the stage table, and broadcasts (first row, rows, ok)
-// through shared memory; after the block barrier every thread takes the same
-// decision, so the block's barriers inside a claim loop always match up.
-// Returns rows (0: the claim past the pool) or -1 when a wait gave up.
-__device__ int claim_next(const DevParams& p, Misc& m, uint64_t* full, int slot, uint32_t phase, bool two, int ii,
-                          int op, int& row0) {
-    const int tid = threadIdx.x;
-    if (tid == 0) {
-        int ok = wait_mbar(&full[slot], phase, p, m, ii, op) ? 1 : 0;
-        const int2 info = ok ? make_int2(vload(&m.sinfo[slot].x), vload(&m.sinfo[slot].y)) : make_int2(0, 0);
-        if (ok && two && info.y > 0) {
-            const int s2 = slot + 1 == p.ring_stages ? 0 : slot + 1;
-            ok = wait_mbar(&full[s2], slot + 1 == p.ring_stages ? phase ^ 1u : phase, p, m, ii, op) ? 1 : 0;
-        }
-        m.c_row0 = info.x;
-        m.c_rows = info.y;
-        m.c_ok = ok;
-        if (!ok) vstore(&m.abort_flag, 1);
-    }
-    cbar();
-    if (!vload(&m.c_ok)) return -1;
-    for (int k = 0; k < 64 && !mbar_try_wait(&full[slot], phase); ++k) {  // this thread's own acquire
-    }
-    row0 = vload(&m.c_row0);
-    return vload(&m.c_rows);
-}
-
-// Sum of the 8 consumer warps' partials of one row, in a fixed order.
-__device__ __forceinline__ float sum_warps(const float* ps) {
-    const float4 x0 = reinterpret_cast<const float4*>(ps)[0], x1 = reinterpret_cast<const float4*>(ps)[1];
-    return ((x0.x + x0.y) + (x0.z + x0.w)) + ((x1.x + x1.y) + (x1.z + x1.w));
-}
-
 // ---------------------------------------------------------------------------
 // instruction checks and the stage plan shared by loader and consumers
 // ---------------------------------------------------------------------------
@@ -221,24 +181,10 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
         return w[W_SIGNAL_CTR] >= 0;
     }
     if (op == OP_RMS_QKV && (sub < 0 || sub > 2)) return false;
-    if (op == OP_OPROJ_RES && (sub < 0 || sub >= p.nkv || (p.nq / p.nkv) * p.d > kMaxOprojCols)) return false;
-    if (w[W_INIT0] != w[W_INIT1] &&
-        (op != OP_RMS_QKV || w[W_INIT0] < 0 || w[W_INIT0] > w[W_INIT1] || w[W_INIT1] > (p.H >> 3)))
-        return false;
     if ((op == OP_MOE_UPGATE || op == OP_MOE_FFN) && (sub < 0 || sub >= p.topk)) return false;
     if (op == OP_FFN && sub != 0) return false;
     if ((op == OP_FFN || op == OP_MOE_FFN) && (p.H > kMaxPartK || 2 * p.H > p.stage_bytes)) return false;
-    const bool claims = w[W_CLAIM_CTR] >= 0;
-    if (claims) {
-        if ((op != OP_FFN && op != OP_LMHEAD_ARGMAX) || w[W_CLAIM_CTR] >= p.n_ctr || w[W_CLAIM_INC] <= 0) return false;
-        const int R = op_rows(p, op, sub), cr = w[W_CLAIM_ROWS];
-        if (w[W_POOL0] < e || w[W_POOL_N] <= 0 || w[W_POOL0] + w[W_POOL_N] != R || cr <= 0 || cr > kMaxRows) return false;
-        // a chunk fits one stage: up/gate rows of both spans (FFN), or hidden-wide rows (LM head)
-        if ((long long)cr * p.H * 2 * (op == OP_FFN ? 2 : 1) > p.stage_bytes || p.H > kMaxPartK) return false;
-        if ((long long)cr * kConsumerWarps * (op == OP_FFN ? 2 : 1) + cr > (long long)kRowSlots * kConsumerWarps)
-            return false;
-    }
-    if (b < 0 || b > e || (b == e && !claims) || e > op_rows(p, op, sub) || e - b > kMaxRows) return false;
+    if (b < 0 || b >= e || e > op_rows(p, op, sub) || e - b > kMaxRows) return false;
     if ((e - b) * acc_sets(op, p.H, p.nq * p.d, p.F, p.topk) > kRowSlots) return false;
     if (op == OP_LMHEAD_ARGMAX) return w[W_AUX_CTR] >= 0 && w[W_AUX_INC] > 0 && w[W_SEQ] >= 0 && w[W_SEQ] < w[W_AUX_INC];
     return w[W_SIGNAL_CTR] >= 0;
@@ -319,10 +265,7 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
             return;
         }
         case OP_RMS_QKV: s0 = wt[WT_Q + sub]; break;
-        case OP_OPROJ_RES:  // kv group `sub`: its columns of every row, from the group-major copy
-            K = (p.nq / p.nkv) * p.d;
-            s0 = wt[WT_O_G] + (size_t)sub * p.H * K;
-            break;
+        case OP_OPROJ_RES: K = p.nq * p.d; s0 = wt[WT_O]; break;
         case OP_RMS_UPGATE_SILU: pl.nspan = 2; s0 = wt[wt_gate(0)]; s1 = wt[wt_up(0, p.E)]; break;
         case OP_DOWN_RES: K = p.F; s0 = wt[wt_down(0, p.E)]; break;
         case OP_LMHEAD_ARGMAX: s0 = p.lm_head; break;
@@ -352,17 +295,17 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
     }
     pl.kparts = kparts_of(K);
     pl.nphase = nslot * pl.kparts;
-    pl.rows = e - b;  // 0: an instruction with run-time claims only
+    pl.rows = e - b;
     pl.src_stride = (uint32_t)K * 2u;
     pl.row_bytes = pl.src_stride / (uint32_t)pl.kparts;
     const int rps = (int)(SB / ((uint32_t)pl.nspan * pl.row_bytes));
-    pl.rps = rps < pl.rows ? rps : (pl.rows > 0 ? pl.rows : rps);
+    pl.rps = rps < pl.rows ? rps : pl.rows;
     pl.spp = (pl.rows + pl.rps - 1) / pl.rps;
     pl.n_stages = pl.main_stages = pl.spp * pl.nphase;
     if (tail) {
         pl.tail_row_bytes = (uint32_t)p.H * 2u;
         const int trps = (int)(SB / pl.tail_row_bytes);
-        pl.tail_rps = trps < pl.rows ? trps : (pl.rows > 0 ? pl.rows : trps);
+        pl.tail_rps = trps < pl.rows ? trps : pl.rows;
         pl.tail_spp = (pl.rows + pl.tail_rps - 1) / pl.tail_rps;
         pl.tail_src = (const unsigned char*)(tail + (size_t)b * p.H);
         pl.n_stages += pl.tail_spp;
@@ -411,12 +354,17 @@ __device__ void issue_stage(const DevParams& p, const Plan& pl, int st, unsigned
             }
         return;
     }
+    // Weight rows are read once per step: they are loaded with the evict-first L2 policy, which
+    // leaves L2 to what is reused across steps (the KV cache, whose rows up to the position are
+    // read again by the next step, the activations and the counters).  K/V rows keep the normal
+    // policy.
+    const uint64_t pol = make_evict_first_policy();
     if (st >= pl.main_stages) {  // fused FFN: transposed down-projection rows
         const int r0 = (st - pl.main_stages) * pl.tail_rps;
         const int nr = (pl.rows - r0) < pl.tail_rps ? (pl.rows - r0) : pl.tail_rps;
         const uint32_t bytes = (uint32_t)nr * pl.tail_row_bytes;
         mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s(dst_stage, pl.tail_src + (size_t)r0 * pl.tail_row_bytes, bytes, bar);
+        bulk_g2s_hint(dst_stage, pl.tail_src + (size_t)r0 * pl.tail_row_bytes, bytes, bar, pol);
         return;
     }
     const int ph = st / pl.spp, sst = st % pl.spp;
@@ -428,11 +376,13 @@ __device__ void issue_stage(const DevParams& p, const Plan& pl, int st, unsigned
     for (int s = 0; s < pl.nspan; ++s) {
         const unsigned char* src = pl.src[slot][s] + (size_t)r0 * pl.src_stride + (size_t)part * pl.row_bytes;
         unsigned char* dst = dst_stage + (size_t)s * pl.rps * pl.row_bytes;
+        const bool kv = pl.tma_row0 >= 0;  // K/V rows of an attention split (contiguous-copy path)
         if (pl.kparts == 1) {
-            bulk_g2s(dst, src, bytes, bar);
+            if (kv) bulk_g2s(dst, src, bytes, bar);
+            else bulk_g2s_hint(dst, src, bytes, bar, pol);
         } else {
             for (int r = 0; r < nr; ++r)
-                bulk_g2s(dst + (size_t)r * pl.row_bytes, src + (size_t)r * pl.src_stride, pl.row_bytes, bar);
+                bulk_g2s_hint(dst + (size_t)r * pl.row_bytes, src + (size_t)r * pl.src_stride, pl.row_bytes, bar, pol);
         }
     }
 }
@@ -501,55 +451,6 @@ struct LoaderRing {
     uint32_t phase = 0;
     uint32_t used = 0, last_parity = 0;  // slots ever filled, parity of their last fill
 };
-
-// Run-time claims of an instruction (after its fixed stages): claim chunk c =
-// atomicAdd(counter) - (epoch - 1) * increment until c lands past the pool.  A
-// chunk is one stage of rows (LM head) or an up/gate stage and a down stage
-// (fused FFN); the rows go into the slot's stage table before the stage's
-// arrival, and the claim past the pool is a stage with no rows and no copy.
-// Every block makes exactly one claim past the pool, so each step adds exactly
-// chunks + claiming instructions to the counter.
-__device__ bool loader_claims(const DevParams& p, const StepArgs& a, const int32_t* w, const Plan& pl,
-                              unsigned char* ring, uint64_t* full, uint64_t* empty, Misc& m, LoaderRing& lr, int ii) {
-    const int op = w[W_OP], b = w[W_BEGIN], crows = w[W_CLAIM_ROWS], pool0 = w[W_POOL0], R = pool0 + w[W_POOL_N];
-    const int nchunks = (w[W_POOL_N] + crows - 1) / crows;
-    const uint32_t base = (a.epoch - 1u) * (uint32_t)w[W_CLAIM_INC];
-    uint32_t* ctr = p.counters + w[W_CLAIM_CTR];
-    const uint32_t SB = (uint32_t)p.stage_bytes;
-    for (;;) {
-        const int c = (int)(atomicAdd(ctr, 1u) - base);
-        const bool more = c >= 0 && c < nchunks;
-        const int row0 = more ? pool0 + c * crows : 0;
-        const int nr = more ? (R - row0 < crows ? R - row0 : crows) : 0;
-        const int nst = more && op == OP_FFN ? 2 : 1;
-        for (int k = 0; k < nst; ++k) {
-            if (!wait_mbar(&empty[lr.slot], lr.phase ^ 1u, p, m, ii, op)) return false;
-            unsigned char* dst = ring + (size_t)lr.slot * SB;
-            uint64_t* bar = &full[lr.slot];
-            m.sinfo[lr.slot] = make_int2(row0, nr);  // ordered before the arrival (release)
-            if (!more) {
-                mbar_arrive(bar);  // no copy: this arrival completes the phase
-            } else if (op == OP_FFN && k == 1) {  // transposed down-projection rows of the chunk
-                const uint32_t bytes = (uint32_t)nr * pl.tail_row_bytes;
-                mbar_arrive_expect_tx(bar, bytes);
-                bulk_g2s(dst, pl.tail_src + (size_t)(row0 - b) * pl.tail_row_bytes, bytes, bar);
-            } else {  // up/gate rows (one span each, crows rows apart) or LM-head rows
-                const uint32_t bytes = (uint32_t)nr * pl.row_bytes;
-                mbar_arrive_expect_tx(bar, bytes * (uint32_t)pl.nspan);
-                for (int s2 = 0; s2 < pl.nspan; ++s2)
-                    bulk_g2s(dst + (size_t)s2 * crows * pl.row_bytes,
-                             pl.src[0][s2] + (size_t)(row0 - b) * pl.src_stride, bytes, bar);
-            }
-            lr.used |= 1u << lr.slot;
-            lr.last_parity = (lr.last_parity & ~(1u << lr.slot)) | (lr.phase << lr.slot);
-            if (++lr.slot == p.ring_stages) {
-                lr.slot = 0;
-                lr.phase ^= 1u;
-            }
-        }
-        if (!more) return true;
-    }
-}
 
 // One step's queue; false if a wait gave up (the block is leaving).
 template <bool PF, bool TC>
@@ -627,9 +528,6 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
             }
         }
         if (!ok) return false;
-        if (w[W_CLAIM_CTR] >= 0 && pl.n_stages >= 0 && instr_ok(p, w) &&
-            !loader_claims(p, a, w, pl, ring, full, empty, m, lr, i))
-            return false;
     }
     return true;
 }
@@ -678,14 +576,77 @@ __device__ __forceinline__ void load_vec(const float* __restrict__ src, int K, f
     }
 }
 
+// Input of the O-projection, columns [col0, col0 + K): the attention output of
+// every query head, merged here from its kv splits' partials (unnormalised
+// o_s, running max m_s in the log2 domain, sum l_s):
+//   attn = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s,
+// taken B splits per round trip with an online rescale, in split order.
+template <int J, int B>
+__device__ __forceinline__ void load_attn_merged(const DevParams& p, int col0, int K, float (&v)[J][8]) {
+    const int tid = threadIdx.x, nch = K >> 3, S = p.kv_splits, D = p.d;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int c = tid + kConsumerThreads * j;
+        if (c >= nch) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
+            continue;
+        }
+        const int col = col0 + 8 * c, h = col / D, dc = col - h * D;
+        const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)h * S;
+        const float4* po = reinterpret_cast<const float4*>(p.part_o + (size_t)h * S * D + dc);
+        const int D4 = D >> 2;
+        float M = -CUDART_INF_F, den = 0.f, acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+        for (int s0 = 0; s0 < S; s0 += B) {
+            float2 t[B];
+            float4 o0[B], o1[B];
+#pragma unroll
+            for (int k = 0; k < B; ++k) {
+                if (s0 + k < S) {
+                    t[k] = __ldcg(ml + s0 + k);
+                    o0[k] = __ldcg(po + (size_t)(s0 + k) * D4);
+                    o1[k] = __ldcg(po + (size_t)(s0 + k) * D4 + 1);
+                } else {
+                    t[k] = make_float2(-CUDART_INF_F, 0.f);
+                    o0[k] = o1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            float bm = M;
+#pragma unroll
+            for (int k = 0; k < B; ++k) bm = fmaxf(bm, t[k].x);
+            if (bm == -CUDART_INF_F) continue;  // no position in these splits yet
+            const float r = exp2f(M - bm);
+            den *= r;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] *= r;
+#pragma unroll
+            for (int k = 0; k < B; ++k) {
+                const float f = exp2f(t[k].x - bm);
+                den = fmaf(f, t[k].y, den);
+                acc[0] = fmaf(f, o0[k].x, acc[0]);
+                acc[1] = fmaf(f, o0[k].y, acc[1]);
+                acc[2] = fmaf(f, o0[k].z, acc[2]);
+                acc[3] = fmaf(f, o0[k].w, acc[3]);
+                acc[4] = fmaf(f, o1[k].x, acc[4]);
+                acc[5] = fmaf(f, o1[k].y, acc[5]);
+                acc[6] = fmaf(f, o1[k].z, acc[6]);
+                acc[7] = fmaf(f, o1[k].w, acc[7]);
+            }
+            M = bm;
+        }
+        const float inv = 1.0f / den;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[j][k] = acc[k] * inv;
+    }
+}
+
 // v = rmsnorm(x) * w for x fp32 (or the bf16 embedding row), all threads.
 // The norm weights are loaded together with x so both round trips overlap.
-// copy / copy2 (optional): the chunks [c0, c1) of the un-normalised x are also
-// stored there (the residual copied into the O-projection's accumulators).
 template <int J>
 __device__ void load_rms(const DevParams& p, Misc& m, const float* x32, const uint16_t* x16, const uint16_t* nw,
-                         float (&v)[J][8], float* snap = nullptr, float* copy = nullptr, float* copy2 = nullptr,
-                         int c0 = 0, int c1 = 0) {
+                         float (&v)[J][8], float* snap = nullptr) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.H, nch = K >> 3;
     uint4 wraw[J];
 #pragma unroll
@@ -704,22 +665,6 @@ __device__ void load_rms(const DevParams& p, Misc& m, const float* x32, const ui
         } else {
 #pragma unroll
             for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
-        }
-    }
-    if (copy) {
-#pragma unroll
-        for (int j = 0; j < J; ++j) {
-            const int c = tid + kConsumerThreads * j;
-            if (c >= c0 && c < c1) {
-                const float4 a0 = make_float4(v[j][0], v[j][1], v[j][2], v[j][3]);
-                const float4 a1 = make_float4(v[j][4], v[j][5], v[j][6], v[j][7]);
-                reinterpret_cast<float4*>(copy)[2 * c] = a0;
-                reinterpret_cast<float4*>(copy)[2 * c + 1] = a1;
-                if (copy2) {
-                    reinterpret_cast<float4*>(copy2)[2 * c] = a0;
-                    reinterpret_cast<float4*>(copy2)[2 * c + 1] = a1;
-                }
-            }
         }
     }
     if (snap) {  // record the residual stream the op reads (hidden-state snapshot)
@@ -848,6 +793,34 @@ __device__ __forceinline__ void rows_block(const uint4* __restrict__ Ws, int row
     if (reduce_rows_writer<RG>(lane)) A[(rg + reduce_rows_lane_row<RG>(lane)) * kConsumerWarps + (tid >> 5)] = s_row;
 }
 
+// rows_block for rows [rg, rg + RG) of which those at or past nr read as zero
+// and are not stored: one copy of the block code covers every row count (a
+// smaller kernel; the stages of one-chunk-per-thread ops hold 8 or 16 rows, so
+// little work is spent on the padding).
+template <int J, int RG>
+__device__ __forceinline__ void rows_block_pred(const uint4* __restrict__ Ws, int row16, int rg, int nr,
+                                                const bool (&jv)[J], const float (&v)[J][8], float* A, int lane) {
+    const int tid = threadIdx.x;
+    uint4 wv[RG][J];
+#pragma unroll
+    for (int r = 0; r < RG; ++r)
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+            wv[r][j] = (jv[j] && rg + r < nr) ? Ws[(rg + r) * row16 + tid + kConsumerThreads * j]
+                                              : make_uint4(0u, 0u, 0u, 0u);
+    float part[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < J; ++j) dot8x2(wv[r][j], v[j], a0, a1);
+        part[r] = a0 + a1;
+    }
+    const float s_row = reduce_rows<RG>(part, lane);
+    const int row = rg + reduce_rows_lane_row<RG>(lane);
+    if (reduce_rows_writer<RG>(lane) && row < nr) A[row * kConsumerWarps + (tid >> 5)] = s_row;
+}
+
 // This thread's column slice of rows [0, nr) of one span of a ring stage (Ws:
 // the span in shared memory, row16 16-byte chunks per row) dotted with its
 // slice v of the input vector, into the warp slots of rows [0, nr) of A.  Rows go in blocks of
@@ -861,6 +834,10 @@ __device__ __forceinline__ void stage_rows(const uint4* __restrict__ Ws, int row
 #pragma unroll
     for (int j = 0; j < J; ++j) jv[j] = (int)threadIdx.x + kConsumerThreads * j < nch;
     int rg = 0;
+    if constexpr (J == 1) {  // one chunk per thread: 8-row blocks, the last one predicated
+        for (; rg < nr; rg += RG) rows_block_pred<J, RG>(Ws, row16, rg, nr, jv, v, A, lane);
+        return;
+    }
     for (; rg + RG <= nr; rg += RG) rows_block<J, RG>(Ws, row16, rg, jv, v, A, lane);
     if constexpr (RG >= 8) {
         if (rg + 4 <= nr) { rows_block<J, 4>(Ws, row16, rg, jv, v, A, lane); rg += 4; }
@@ -909,21 +886,21 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     const float* vsrc = nullptr;  // fp32 input for OPROJ / DOWN (all column parts)
     switch (op) {
         case OP_RMS_QKV:
-            // the residual after layer l-1 (x2; the embedding row at layer 0); one block records it as
-            // snapshot l, and each block copies its share of it into the O-projection's accumulator x
-            // (and, at layer 0, into x2 as well: the FFN adds into x2 after the O-projection)
+            // the residual after layer l-1 (x2); one block records it as snapshot l
             load_rms<J>(p, m, p.x2, l == 0 ? p.embed + (size_t)token * p.H : nullptr, wt[WT_ATTN_NORM], v,
-                        (p.snap && sub == 0 && b == 0) ? p.snap + (size_t)l * p.H : nullptr,
-                        w[W_INIT1] > w[W_INIT0] ? p.x : nullptr, l == 0 ? p.x2 : nullptr, w[W_INIT0], w[W_INIT1]);
+                        (p.snap && l > 0 && sub == 0 && b == 0) ? p.snap + (size_t)l * p.H : nullptr);
             break;
         case OP_RMS_UPGATE_SILU:
         case OP_MOE_UPGATE:
-            load_rms<J>(p, m, p.x, nullptr, wt[WT_FFN_NORM], v);
+            if constexpr (!HOIST) load_rms<J>(p, m, p.x, nullptr, wt[WT_FFN_NORM], v);
             break;
         case OP_LMHEAD_ARGMAX:
             // the residual after the last layer (or the embedding row without layers): snapshot L
             load_rms<J>(p, m, p.x2, p.L == 0 ? p.embed + (size_t)token * p.H : nullptr, p.final_norm, v,
                         (p.snap && w[W_SEQ] == 0) ? p.snap + (size_t)p.L * p.H : nullptr);
+            break;
+        case OP_OPROJ_RES:
+            K = p.nq * p.d;  // input: the attention output, merged from the kv splits below
             break;
         case OP_DOWN_RES:
         case OP_MOE_DOWN2_RES:
@@ -932,10 +909,13 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
             break;
     }
     const int kp = K / kparts_of(K);  // columns per part
+    if (op == OP_OPROJ_RES) load_attn_merged<J, HOIST ? 8 : 4>(p, 0, kp, v);
     if (vsrc) load_vec<J>(vsrc, kp, v);
     // 3. routing (once per layer per block; the loader waits for it)
-    if (op == OP_MOE_UPGATE && vload(&m.router_layer) != route_key(a.epoch, l, p.L))
-        route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v, a.epoch);
+    if constexpr (!HOIST) {
+        if (op == OP_MOE_UPGATE && vload(&m.router_layer) != route_key(a.epoch, l, p.L))
+            route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v, a.epoch);
+    }
     if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
     if (!early) {
         int eidx[kMaxTopK];
@@ -947,7 +927,8 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     const int nch = kp >> 3;
     for (int ph = 0; ph < pl.nphase; ++ph) {
         const int vslot = ph / pl.kparts, part = ph % pl.kparts;
-        if (ph > 0) load_vec<J>(vsrc + (size_t)vslot * p.F + (size_t)part * kp, kp, v);
+        if (ph > 0 && op == OP_OPROJ_RES) load_attn_merged<J, HOIST ? 8 : 4>(p, part * kp, kp, v);
+        else if (ph > 0) load_vec<J>(vsrc + (size_t)vslot * p.F + (size_t)part * kp, kp, v);
         for (int sst = 0; sst < pl.spp; ++sst) {
             const int r0 = sst * pl.rps;
             const int nr = (rows - r0) < pl.rps ? (rows - r0) : pl.rps;
@@ -996,24 +977,42 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
             for (int r = tid; r < rows; r += kConsumerThreads) p.qkv[off + b + r] = acc(0, r);
             break;
         }
-        case OP_RMS_UPGATE_SILU:
-        case OP_MOE_UPGATE: {
-            float* h = p.hbuf + (op == OP_MOE_UPGATE ? (size_t)sub * p.F : 0);
+        case OP_OPROJ_RES:
             for (int r = tid; r < rows; r += kConsumerThreads) {
-                const float g = acc(0, r), u = acc(1, r);
-                h[b + r] = g / (1.0f + expf(-g)) * u;
+                float base;
+                if (l == 0) {
+                    const uint16_t e = p.embed[(size_t)token * p.H + b + r];
+                    base = __uint_as_float((uint32_t)e << 16);
+                    if (p.snap) p.snap[b + r] = base;
+                } else {
+                    base = __ldcg(p.x2 + b + r);
+                }
+                const float nx = base + acc(0, r);
+                p.x[b + r] = nx;   // read by the FFN's RMSNorm
+                p.x2[b + r] = nx;  // the FFN adds its output here
             }
             break;
-        }
+        case OP_RMS_UPGATE_SILU:
+        case OP_MOE_UPGATE:
+            if constexpr (!HOIST) {  // split-FFN ops run in the general instantiation only
+                float* h = p.hbuf + (op == OP_MOE_UPGATE ? (size_t)sub * p.F : 0);
+                for (int r = tid; r < rows; r += kConsumerThreads) {
+                    const float g = acc(0, r), u = acc(1, r);
+                    h[b + r] = g / (1.0f + expf(-g)) * u;
+                }
+            }
+            break;
         case OP_DOWN_RES:
         case OP_MOE_DOWN2_RES:
-            for (int r = tid; r < rows; r += kConsumerThreads) {
-                float add = acc(0, r);
-                if (op == OP_MOE_DOWN2_RES) {
-                    add = m.ew[0] * add;
-                    if (p.topk > 1) add += m.ew[1] * acc(1, r);
+            if constexpr (!HOIST) {
+                for (int r = tid; r < rows; r += kConsumerThreads) {
+                    float add = acc(0, r);
+                    if (op == OP_MOE_DOWN2_RES) {
+                        add = m.ew[0] * add;
+                        if (p.topk > 1) add += m.ew[1] * acc(1, r);
+                    }
+                    p.x2[b + r] = __ldcg(p.x2 + b + r) + add;
                 }
-                p.x2[b + r] = __ldcg(p.x2 + b + r) + add;
             }
             break;
         case OP_LMHEAD_ARGMAX: {
@@ -1026,35 +1025,6 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
                     bv = val;
                     bi = b + r;
                 }
-            }
-            if (w[W_CLAIM_CTR] >= 0) {  // then rows claimed at run time, one stage per chunk
-                cbar();                 // every row sum of the fixed rows has been read: the scratch is free
-                for (;;) {
-                    int row0 = 0;
-                    const int nr = claim_next(p, m, full, slot, phase, false, ii, op, row0);
-                    if (nr < 0) break;
-                    if (nr > 0)
-                        stage_rows<J, RG>(reinterpret_cast<const uint4*>(ring + (size_t)slot * SB),
-                                          (int)(pl.row_bytes >> 4), nr, nch, v, part_sums, lane);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[slot]);
-                    if (++slot == p.ring_stages) {
-                        slot = 0;
-                        phase ^= 1u;
-                    }
-                    if (nr == 0) break;
-                    cbar();
-                    for (int r = tid; r < nr; r += kConsumerThreads) {
-                        const float val = sum_warps(part_sums + (size_t)r * kConsumerWarps);
-                        a.logits[row0 + r] = val;
-                        if (val > bv || (val == bv && row0 + r < bi)) {
-                            bv = val;
-                            bi = row0 + r;
-                        }
-                    }
-                }
-                cbar();
-                if (vload(&m.abort_flag)) return false;
             }
             warp_argmax(bv, bi);
             const int warp = tid >> 5;
@@ -1269,62 +1239,6 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     }
     cbar();
     if (vload(&m.abort_flag)) return false;
-
-    // then rows claimed at run time: per chunk an up/gate stage (crows rows of each span), its h
-    // rows, and a stage of the matching transposed down-projection rows
-    if (w[W_CLAIM_CTR] >= 0) {
-        const int crows = w[W_CLAIM_ROWS];
-        float* cps = scratch;                                  // [2 * crows][8 warps] gate / up row sums
-        float* ch = scratch + (size_t)2 * crows * kConsumerWarps;  // [crows] h of the chunk
-        for (;;) {
-            int row0 = 0;
-            const int nr = claim_next(p, m, full, slot, phase, true, ii, op, row0);
-            if (nr < 0) break;
-            if (nr > 0) {
-                const unsigned char* stage = ring + (size_t)slot * SB;
-                for (int s = 0; s < 2; ++s)
-                    stage_rows<J, RG>(reinterpret_cast<const uint4*>(stage + (size_t)s * crows * pl.row_bytes),
-                                      (int)(pl.row_bytes >> 4), nr, nch, v, cps + (size_t)s * crows * kConsumerWarps,
-                                      lane);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
-            if (++slot == p.ring_stages) {
-                slot = 0;
-                phase ^= 1u;
-            }
-            if (nr == 0) break;
-            cbar();
-            for (int r = tid; r < nr; r += kConsumerThreads) {
-                const float g = sum_warps(cps + (size_t)r * kConsumerWarps);
-                const float u = sum_warps(cps + (size_t)(crows + r) * kConsumerWarps);
-                ch[r] = wgt * (g / (1.0f + expf(-g)) * u);
-            }
-            cbar();
-            for (int k = 0; k < 64 && !mbar_try_wait(&full[slot], phase); ++k) {  // own acquire of the down stage
-            }
-            const uint4* Ws = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
-            for (int r = 0; r < nr; ++r) {
-                const float hk = ch[r];
-#pragma unroll
-                for (int j = 0; j < J; ++j) {
-                    if (!jv[j]) continue;
-                    float f[8];
-                    unpack8(Ws[r * nch + tid + kConsumerThreads * j], f);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) y[j][k] = fmaf(f[k], hk, y[j][k]);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
-            if (++slot == p.ring_stages) {
-                slot = 0;
-                phase ^= 1u;
-            }
-        }
-        cbar();
-        if (vload(&m.abort_flag)) return false;
-    }
 #pragma unroll
     for (int j = 0; j < J; ++j) {
         if (!jv[j]) continue;
@@ -1333,154 +1247,6 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
         atomicAdd(dst + 1, make_float4(y[j][4], y[j][5], y[j][6], y[j][7]));
     }
     cbar();
-    if (tid == 0) signal_release(p.counters + w[W_SIGNAL_CTR]);
-    return true;
-}
-
-// O-projection rows of one warp: rows r, r + 8, ..., r + 8 (RG - 1) of the
-// stage (row length nck 16-byte chunks; lane holds chunks lane and lane + 32 of
-// the input vector), reduced across the warp; the writer lanes add the row
-// results into both residual copies.
-template <int RG>
-__device__ __forceinline__ void orow_block(const uint4* __restrict__ Ws, int nck, int r, const float (&v)[2][8],
-                                           float* x, float* x2, int lane) {
-    const bool j0 = lane < nck, j1 = lane + 32 < nck;
-    uint4 wv[RG][2];
-#pragma unroll
-    for (int k = 0; k < RG; ++k) {
-        wv[k][0] = j0 ? Ws[(size_t)(r + 8 * k) * nck + lane] : make_uint4(0u, 0u, 0u, 0u);
-        wv[k][1] = j1 ? Ws[(size_t)(r + 8 * k) * nck + lane + 32] : make_uint4(0u, 0u, 0u, 0u);
-    }
-    float part[RG];
-#pragma unroll
-    for (int k = 0; k < RG; ++k) {
-        float a0 = 0.f, a1 = 0.f;
-        dot8x2(wv[k][0], v[0], a0, a1);
-        dot8x2(wv[k][1], v[1], a0, a1);
-        part[k] = a0 + a1;
-    }
-    const float s_row = reduce_rows<RG>(part, lane);
-    if (reduce_rows_writer<RG>(lane)) {
-        const int row = r + 8 * reduce_rows_lane_row<RG>(lane);
-        atomicAdd(x + row, s_row);
-        atomicAdd(x2 + row, s_row);
-    }
-}
-
-// O-projection of kv group g (OP_OPROJ_RES): rows [b, e) of w_o restricted to
-// the columns of group g's query heads, times the group's attention output,
-// added into the residual.  The output projection is linear in the attention
-// output, so x + Wo attn = x + sum_g Wo[:, cols_g] attn_g: each group's blocks
-// wait only for that group's attention splits, merge them, and add their
-// rows' share with fp32 atomics (the QKV op copied the residual into x before;
-// summation order across groups varies between runs).  Each warp takes whole
-// rows; lanes hold 8-column chunks of the group's attention output.
-template <bool HOIST>
-__device__ bool oproj_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
-                            uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = w[W_SUB], b = w[W_BEGIN], rows = w[W_END] - b;
-    const int G = p.nq / p.nkv, D = p.d, K = G * D, nck = K >> 3, S = p.kv_splits;
-    const uint32_t SB = (uint32_t)p.stage_bytes;
-    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
-    Plan pl;
-    if (HOIST) make_plan(p, a.pos, w, nullptr, pl);
-    else prefetch_plan_l1(p, w);
-    if (tid == 0) {
-        if (!wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, OP_OPROJ_RES))
-            vstore(&m.abort_flag, 1);
-        if (tr) tr[T_DEP] = globaltimer_ns();
-    }
-    cbar();
-    if (vload(&m.abort_flag)) return false;
-
-    // The group's attention output, merged from its splits' partials (unnormalised
-    // o_s, running max m_s in the log2 domain, sum l_s):
-    //   attn = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s,
-    // eight splits per round trip with an online rescale, in split order.  Thread t
-    // merges columns 2t, 2t + 1 into shared memory.
-    float* vs = scratch;  // [K]
-    if (2 * tid < K) {
-        const int col = 2 * tid, h = g * G + col / D, dc = col - (col / D) * D;
-        const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)h * S;
-        const float2* po = reinterpret_cast<const float2*>(p.part_o + (size_t)h * S * D + dc);
-        const int D2 = D >> 1;
-        float M = -CUDART_INF_F, den = 0.f, acc0 = 0.f, acc1 = 0.f;
-        for (int s0 = 0; s0 < S; s0 += 8) {
-            float2 t[8], o[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                if (s0 + k < S) {
-                    t[k] = __ldcg(ml + s0 + k);
-                    o[k] = __ldcg(po + (size_t)(s0 + k) * D2);
-                } else {
-                    t[k] = make_float2(-CUDART_INF_F, 0.f);
-                    o[k] = make_float2(0.f, 0.f);
-                }
-            }
-            float bm = M;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) bm = fmaxf(bm, t[k].x);
-            if (bm == -CUDART_INF_F) continue;  // no position in these splits yet
-            const float r = exp2f(M - bm);
-            den *= r;
-            acc0 *= r;
-            acc1 *= r;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const float f = exp2f(t[k].x - bm);
-                den = fmaf(f, t[k].y, den);
-                acc0 = fmaf(f, o[k].x, acc0);
-                acc1 = fmaf(f, o[k].y, acc1);
-            }
-            M = bm;
-        }
-        const float inv = 1.0f / den;
-        vs[col] = acc0 * inv;
-        vs[col + 1] = acc1 * inv;
-    }
-    cbar();
-    float v[2][8];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int c = lane + 32 * j;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) v[j][k] = c < nck ? vs[8 * c + k] : 0.f;
-    }
-    if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
-    if (!HOIST) make_plan(p, a.pos, w, nullptr, pl);
-
-    // stages: warp w takes rows w, w + 8, ... of each stage
-    float* xo = p.x + b;
-    float* x2o = p.x2 + b;
-    for (int sst = 0; sst < pl.spp; ++sst) {
-        const int r0 = sst * pl.rps;
-        const int nr = (rows - r0) < pl.rps ? (rows - r0) : pl.rps;
-        const bool ok = warp_wait_full(&full[slot], phase, p, m, ii, OP_OPROJ_RES);
-        if (tr && tid == 0 && sst == 0) tr[T_FIRST] = globaltimer_ns();
-        if (tid == 0) stage_stamp(tr, T_SREADY, sst);
-        if (ok) {
-            const uint4* Ws = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
-            const int mine = nr > warp ? (nr - warp + 7) >> 3 : 0;  // rows warp + 8 i of the stage
-            int i = 0;
-            for (; i + 8 <= mine; i += 8) orow_block<8>(Ws, nck, warp + 8 * i, v, xo + r0, x2o + r0, lane);
-            if (i + 4 <= mine) { orow_block<4>(Ws, nck, warp + 8 * i, v, xo + r0, x2o + r0, lane); i += 4; }
-            if (i + 2 <= mine) { orow_block<2>(Ws, nck, warp + 8 * i, v, xo + r0, x2o + r0, lane); i += 2; }
-            if (i < mine) orow_block<1>(Ws, nck, warp + 8 * i, v, xo + r0, x2o + r0, lane);
-            __syncwarp();
-            if (tid == 0) stage_stamp(tr, T_SDONE, sst);
-            if (lane == 0) mbar_arrive(&empty[slot]);
-        } else if (tid == 0) {
-            vstore(&m.abort_flag, 1);
-        }
-        if (++slot == p.ring_stages) {
-            slot = 0;
-            phase ^= 1u;
-        }
-    }
-    cbar();
-    if (vload(&m.abort_flag)) return false;
-    if (tr && tid == 0) tr[T_MAIN] = globaltimer_ns();
     if (tid == 0) signal_release(p.counters + w[W_SIGNAL_CTR]);
     return true;
 }
@@ -2105,6 +1871,7 @@ __device__ bool attn_tc(const DevParams& p, const StepArgs& a, const int32_t* w,
 
 __device__ __forceinline__ int gemv_k(const DevParams& p, int op) {
     switch (op) {
+        case OP_OPROJ_RES: return p.nq * p.d;
         case OP_DOWN_RES:
         case OP_MOE_DOWN2_RES: return p.F;
     }
@@ -2118,11 +1885,17 @@ template <int JF>
 __device__ bool gemv_dispatch(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                               uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase,
                               int token) {
-    if (w[W_OP] == OP_OPROJ_RES) return oproj_instr<JF != 0>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
     if constexpr (JF > 0) {
+        // the specialised instantiations run fused-FFN schedules only (chosen on the host)
         if (w[W_OP] == OP_FFN || w[W_OP] == OP_MOE_FFN)
             return ffn_instr<JF, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-        return gemv_instr<JF, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+        if (w[W_OP] == OP_RMS_QKV || w[W_OP] == OP_OPROJ_RES || w[W_OP] == OP_LMHEAD_ARGMAX)
+            return gemv_instr<JF, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+        if (threadIdx.x == 0) {
+            record_error(p.status, MK_ERR_BAD_INSTR, blockIdx.x, ii, w[W_OP], -1, 0, 0);
+            vstore(&m.abort_flag, 1);
+        }
+        return false;
     }
     const int K = gemv_k(p, w[W_OP]);
     const int kp = K / kparts_of(K);
@@ -2257,9 +2030,11 @@ __device__ void serve_respond(const DevParams& p, const StepArgs& a, int next_to
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
-// One instantiation per JF (see gemv_dispatch); the specialised ones leave out
-// the consumers' optional per-instruction L2 prefetch (prefetch_ahead).
-template <int JF, int DH>
+// One instantiation per JF (see gemv_dispatch).  PF: the loader's L2-prefetch
+// cursor (options.l2_prefetch) is compiled in; the specialised instantiations
+// exist with and without it, so the default ones carry no prefetch code.  The
+// consumers' per-instruction prefetch (prefetch_ahead) is in the general one only.
+template <int JF, int DH, bool PF>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ DevParams p, const StepArgs a) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int NS = p.ring_stages, SB = p.stage_bytes;
@@ -2291,7 +2066,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             for (uint32_t k = 0;; ++k) {
                 StepArgs sa = a;
                 if (a.serve && !serve_take(p, m, k, a, sa)) break;
-                if (!loader<true, DH == 64>(p, sa, q, n, smem, full, empty, m, lr) || !a.serve) break;
+                if (!loader<PF, DH == 64>(p, sa, q, n, smem, full, empty, m, lr) || !a.serve) break;
             }
             loader_drain(p, full, lr);
         }
@@ -2354,10 +2129,12 @@ namespace {
 using KernelFn = void (*)(DevParams, StepArgs);
 KernelFn kernel_of(int variant) {
     switch (variant) {
-        case 1: return megakernel<1, 64>;
-        case 2: return megakernel<2, 128>;
+        case 1: return megakernel<1, 64, false>;
+        case 2: return megakernel<2, 128, false>;
+        case 3: return megakernel<1, 64, true>;
+        case 4: return megakernel<2, 128, true>;
     }
-    return megakernel<0, 0>;
+    return megakernel<0, 0, true>;
 }
 // J of a GEMV over K columns (chunks of 8 per consumer thread, per column part)
 int j_of(int K) {
@@ -2366,13 +2143,13 @@ int j_of(int K) {
 }
 }  // namespace
 
+// 0: general; 1 / 2: specialised for one chunk (head_dim 64) / two chunks (head_dim 128) per
+// thread; 3 / 4: the same with the loader's L2-prefetch cursor (options.l2_prefetch > 0).
 int megakernel_variant(const DevParams& p, bool fused_ffn) {
-    // The loader's L2-prefetch cursor (l2_prefetch) is compiled into every instantiation; the
-    // consumers' per-instruction prefetch (prefetch_ahead) only into the general one.
     if (!fused_ffn || p.prefetch_ahead > 0) return 0;
-    const int jh = j_of(p.H);  // every GEMV but the O-projection (whole rows per warp) reads hidden-wide rows
-    if (jh == 1 && p.d == 64) return 1;
-    if (jh == 2 && p.d == 128) return 2;
+    const int jh = j_of(p.H), jo = j_of(p.nq * p.d), pf = p.l2_prefetch > 0 ? 2 : 0;
+    if (jh == 1 && jo == 1 && p.d == 64) return 1 + pf;
+    if (jh == 2 && jo == 2 && p.d == 128) return 2 + pf;
     return 0;
 }
 
@@ -2394,7 +2171,7 @@ cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, i
 cudaError_t prepare_megakernel(int ring_stages, int stage_bytes, int* max_blocks_per_sm) {
     const size_t smem = megakernel_smem_bytes(ring_stages, stage_bytes);
     *max_blocks_per_sm = 1 << 30;
-    for (int v = 0; v <= 2; ++v) {
+    for (int v = 0; v <= 4; ++v) {
         cudaError_t e = cudaFuncSetAttribute(kernel_of(v), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         int per_sm = 0;

@@ -39,7 +39,6 @@ Instr blank() {
     w[W_WAIT_CTR] = -1;
     w[W_SIGNAL_CTR] = -1;
     w[W_AUX_CTR] = -1;
-    w[W_CLAIM_CTR] = -1;
     return w;
 }
 
@@ -144,7 +143,7 @@ int check_config(const mk_config& c) {
         return MK_ERR_INVALID_ARG;
     if (!(c.rms_eps >= 0.f) || !(c.rope_theta > 0.f)) return MK_ERR_INVALID_ARG;
     if (c.head_dim != 64 && c.head_dim != 128) return MK_ERR_UNSUPPORTED;
-    if (c.n_q_heads % c.n_kv_heads || c.n_kv_heads > kMaxKvHeads) return MK_ERR_UNSUPPORTED;
+    if (c.n_q_heads % c.n_kv_heads) return MK_ERR_UNSUPPORTED;
     {
         const int g = c.n_q_heads / c.n_kv_heads;  // query heads per kv head (attention kernel instances)
         if (g < 1 || g > 4) return MK_ERR_UNSUPPORTED;  // attention kernel instances
@@ -173,7 +172,6 @@ void fill_defaults(mk_options* o) {
     if (o->attn_sm_ffn_permille <= 0) o->attn_sm_ffn_permille = 1000;
     if (o->spin_limit_ns == 0) o->spin_limit_ns = 2000000000ull;
     if (o->serve_idle_ns == 0) o->serve_idle_ns = 60000000000ull;
-    if (o->claim_permille <= 0) o->claim_permille = kDefaultClaimPermille;
 }
 
 int check_options(const mk_config& c, const mk_options& o) {
@@ -190,7 +188,6 @@ int check_options(const mk_config& c, const mk_options& o) {
     if (o.kv_splits < 0 || (long long)o.kv_splits * c.n_q_heads > kMaxMergeSlots) return MK_ERR_INVALID_ARG;
     if (o.attn_sm_ffn_permille < 0 || o.attn_sm_ffn_permille > 4000) return MK_ERR_INVALID_ARG;
     if (o.l2_head_start < 0 || o.l2_head_start > 64) return MK_ERR_INVALID_ARG;
-    if (o.claim_permille < 1 || o.claim_permille > 1000) return MK_ERR_INVALID_ARG;
     if (o.sm_speed) {
         if (o.n_sm_speed <= 0) return MK_ERR_INVALID_ARG;
         for (int i = 0; i < o.n_sm_speed; ++i)
@@ -227,7 +224,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     const bool fused = ffn_fused(c, o);
 
     std::vector<std::vector<Instr>> q(n_sm);
-    std::vector<uint32_t> inc(n_counters(L, nkv), 0);
+    std::vector<uint32_t> inc(n_counters(L), 0);
 
     auto add = [&](int sm, Instr w) {
         q[sm].push_back(w);
@@ -251,65 +248,10 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
         }, weight);
     };
 
-    const int nch = H / 8;  // 8-element chunks of the residual
-    // An op whose rows [0, pool0) are split into fixed shares (by `weight`) and whose rows [pool0, R)
-    // are claimed at run time in chunks of `crows` rows: every block gets an instruction (its fixed
-    // rows, possibly none), and the last one of each block claims until the pool is exhausted.  The
-    // claim counter's per-step increment is the chunk count plus one final (empty) claim per block.
-    // LM head: arrival counter `aux`, one partial-argmax slot per instruction.
-    auto claimed_op = [&](int op, int layer, int R, int pool0, int crows, int wait, int signal, int claim, int aux,
-                          const std::vector<double>& weight) {
-        std::vector<int> last(n_sm, -1);
-        int seq = 0;
-        auto emit = [&](int sm, int b, int e) {
-            Instr w = blank();
-            w[W_OP] = op;
-            w[W_LAYER] = layer;
-            w[W_BEGIN] = b;
-            w[W_END] = e;
-            w[W_WAIT_CTR] = wait;
-            w[W_SIGNAL_CTR] = signal;
-            w[W_AUX_CTR] = aux;
-            if (aux >= 0) w[W_SEQ] = seq++;
-            add(sm, w);
-            last[sm] = (int)q[sm].size() - 1;
-        };
-        if (pool0 > 0)
-            split_rows({{0, pool0}}, n_sm, op_cap(op), [&](int sm, int, int b, int e) { emit(sm, b, e); },
-                       o.sm_speed || op == OP_FFN ? &weight : nullptr);
-        for (int sm = 0; sm < n_sm; ++sm)
-            if (last[sm] < 0) emit(sm, pool0, pool0);  // no fixed rows: claims only
-        const int pool_n = R - pool0, chunks = (pool_n + crows - 1) / crows;
-        for (int sm = 0; sm < n_sm; ++sm) {
-            Instr& w = q[sm][last[sm]];
-            w[W_CLAIM_CTR] = claim;
-            w[W_POOL0] = pool0;
-            w[W_POOL_N] = pool_n;
-            w[W_CLAIM_ROWS] = crows;
-        }
-        inc[claim] += (uint32_t)(chunks + n_sm);
-    };
-
     for (int l = 0; l < L; ++l) {
         const int prev_down = l > 0 ? ctr_id(l - 1, C_FFN2) : -1;
-        std::vector<int> first_qkv(n_sm, -1);  // index in q[sm] of the block's first QKV instruction of the layer
-        for (int sm = 0; sm < n_sm; ++sm) first_qkv[sm] = (int)q[sm].size();
         gemv_op(OP_RMS_QKV, l, {{0, c.n_q_heads * d}, {1, nkv * d}, {2, nkv * d}}, prev_down,
                 ctr_id(l, C_QKV));
-        // The residual entering the layer is copied into the O-projection's accumulator x by the QKV
-        // blocks, which load it anyway: each block with a QKV instruction takes an even share of the
-        // chunks, so that every chunk is copied exactly once before the O-projection adds into it.
-        {
-            std::vector<int> holders;
-            for (int sm = 0; sm < n_sm; ++sm)
-                if (first_qkv[sm] < (int)q[sm].size()) holders.push_back(sm);
-            const int nh = (int)holders.size();
-            for (int k = 0; k < nh; ++k) {
-                Instr& w = q[holders[k]][first_qkv[holders[k]]];
-                w[W_INIT0] = (int32_t)((long long)nch * k / nh);
-                w[W_INIT1] = (int32_t)((long long)nch * (k + 1) / nh);
-            }
-        }
         // attention: kv head g, split s -> instruction k = g * S + s, rotated per layer
         const int total = nkv * S;
         std::vector<double> ffn_weight = speed;  // blocks with an attention split may take fewer FFN rows
@@ -321,52 +263,15 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
             w[W_BEGIN] = k % S;
             w[W_END] = S;
             w[W_WAIT_CTR] = ctr_id(l, C_QKV);
-            w[W_SIGNAL_CTR] = ctr_attn_group(L, nkv, l, k / S);
+            w[W_SIGNAL_CTR] = ctr_id(l, C_ATTN);
             int sm = (int)(((long long)k + (long long)l * total) % n_sm);
             add(sm, w);
             ffn_weight[sm] = speed[sm] * (o.attn_sm_ffn_permille / 1000.0);
         }
-        // O-projection by kv group: segment g is every output row restricted to the columns of
-        // group g's query heads.  Default: blocks are shared out between the groups and each block
-        // of group g waits only for group g's attention splits.  Split-FFN schedules (the bitwise
-        // reproducible form) instead give every block one row range and all groups for it, in
-        // group order: each row's group contributions then come from one thread in program order,
-        // so their fp32 sum has a fixed order.
-        {
-            auto emit = [&](int sm, int g, int b, int e) {
-                Instr w = blank();
-                w[W_OP] = OP_OPROJ_RES;
-                w[W_LAYER] = l;
-                w[W_SUB] = g;
-                w[W_BEGIN] = b;
-                w[W_END] = e;
-                w[W_WAIT_CTR] = ctr_attn_group(L, nkv, l, g);
-                w[W_SIGNAL_CTR] = ctr_id(l, C_OPROJ);
-                add(sm, w);
-            };
-            if (fused) {
-                std::vector<Segment> groups;
-                for (int g = 0; g < nkv; ++g) groups.push_back({g, H});
-                split_rows(groups, n_sm, op_cap(OP_OPROJ_RES), emit);
-            } else {
-                const int capo = op_cap(OP_OPROJ_RES);
-                for (int sm = 0; sm < n_sm; ++sm) {
-                    const int b = (int)((long long)H * sm / n_sm), e = (int)((long long)H * (sm + 1) / n_sm);
-                    for (int g = 0; g < nkv; ++g)
-                        for (int r = b; r < e; r += capo) emit(sm, g, r, std::min(e, r + capo));
-                }
-            }
-        }
+        gemv_op(OP_OPROJ_RES, l, {{0, H}}, ctr_id(l, C_ATTN), ctr_id(l, C_OPROJ));
         std::vector<Segment> slots;
         for (int s = 0; s < (moe ? c.top_k : 1); ++s) slots.push_back({s, F});
-        if (fused && !moe && o.claim_permille < 1000) {
-            // fixed shares of the first claim_permille / 1000 of the rows, then the rest claimed at run
-            // time in chunks of one up/gate stage (sb / (2 * 2 * hidden) rows each)
-            const int pool0 = (int)((long long)F * o.claim_permille / 1000);
-            const int crows = std::max(1, std::min(kMaxRows, o.stage_bytes / (4 * H)));
-            claimed_op(OP_FFN, l, F, pool0, crows, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN2), ctr_id(l, C_FFN1),
-                       -1, ffn_weight);
-        } else if (fused) {
+        if (fused) {
             // one instruction per block: its up/gate rows, then the matching down-projection columns
             gemv_op(moe ? OP_MOE_FFN : OP_FFN, l, slots, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN2), &ffn_weight);
         } else if (!moe) {
@@ -379,32 +284,25 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     }
     // LM head + argmax: partial slots numbered in emission order
     {
+        int seq = 0;
         const int wait = L > 0 ? ctr_id(L - 1, C_FFN2) : -1;
-        if (o.claim_permille < 1000) {
-            const int pool0 = (int)((long long)c.vocab * o.claim_permille / 1000);
-            const int crows = std::max(1, std::min(kMaxRows, o.stage_bytes / (2 * H)));
-            claimed_op(OP_LMHEAD_ARGMAX, L, c.vocab, pool0, crows, wait, -1, ctr_lm_claim(L, nkv), ctr_lm(L), speed);
-        } else {
-            int seq = 0;
-            split_rows({{0, c.vocab}}, n_sm, op_cap(OP_LMHEAD_ARGMAX), [&](int sm, int, int b, int e) {
-                Instr w = blank();
-                w[W_OP] = OP_LMHEAD_ARGMAX;
-                w[W_LAYER] = L;
-                w[W_BEGIN] = b;
-                w[W_END] = e;
-                w[W_WAIT_CTR] = wait;
-                w[W_AUX_CTR] = ctr_lm(L);
-                w[W_SEQ] = seq++;
-                add(sm, w);
-            }, o.sm_speed ? &speed : nullptr);
-        }
+        split_rows({{0, c.vocab}}, n_sm, op_cap(OP_LMHEAD_ARGMAX), [&](int sm, int, int b, int e) {
+            Instr w = blank();
+            w[W_OP] = OP_LMHEAD_ARGMAX;
+            w[W_LAYER] = L;
+            w[W_BEGIN] = b;
+            w[W_END] = e;
+            w[W_WAIT_CTR] = wait;
+            w[W_AUX_CTR] = ctr_lm(L);
+            w[W_SEQ] = seq++;
+            add(sm, w);
+        }, o.sm_speed ? &speed : nullptr);
     }
     // fill wait increments and aux increments
     for (auto& qs : q)
         for (auto& w : qs) {
             w[W_WAIT_INC] = w[W_WAIT_CTR] >= 0 ? (int32_t)inc[w[W_WAIT_CTR]] : 0;
             w[W_AUX_INC] = w[W_AUX_CTR] >= 0 ? (int32_t)inc[w[W_AUX_CTR]] : 0;
-            w[W_CLAIM_INC] = w[W_CLAIM_CTR] >= 0 ? (int32_t)inc[w[W_CLAIM_CTR]] : 0;
         }
 
     int max_instr = 1;
@@ -445,11 +343,9 @@ static int op_index(const int32_t* w) {
     return w[W_LAYER] * 5 + slot;
 }
 
-// Op index of the op that signals counter `ctr` (LM arrival counter: n_layers*5;
-// per-group attention counters: the layer's attention op).
-static int producer_op(int ctr, int L, int nkv) {
+// Op index of the op that signals counter `ctr` (LM arrival counter: n_layers*5).
+static int producer_op(int ctr, int L) {
     if (ctr == ctr_lm(L)) return L * 5;
-    if (ctr > ctr_lm(L)) return (ctr - ctr_lm(L) - 1) / nkv * 5 + 1;
     const int l = ctr / kCountersPerLayer, slot = ctr % kCountersPerLayer;
     switch (slot) {
         case C_QKV: return l * 5 + 0;
@@ -463,16 +359,13 @@ static int producer_op(int ctr, int L, int nkv) {
 
 int validate(const mk_config& c, const Planned& p) {
     const int L = c.n_layers, nkv = c.n_kv_heads, d = c.head_dim;
-    const int nctr = n_counters(L, nkv);
+    const int nctr = n_counters(L);
     if ((int)p.ctr_inc.size() != nctr) return MK_ERR_SCHEDULE;
     const bool moe = c.n_experts > 0;
     // coverage bitmaps: per (layer, op, sub) rows covered exactly once
     std::vector<std::vector<uint8_t>> cov;
-    auto cov_key = [&](int l, int op, int sub) { return ((size_t)l * OP_COUNT + op) * kMaxKvHeads + sub; };
-    cov.resize((size_t)(L + 1) * OP_COUNT * kMaxKvHeads);
-    // per layer: residual chunks copied into the O-projection's accumulator by the QKV blocks
-    const int nch = c.hidden / 8;
-    std::vector<std::vector<uint8_t>> init_hits((size_t)std::max(L, 1), std::vector<uint8_t>(nch, 0));
+    auto cov_key = [&](int l, int op, int sub) { return ((size_t)l * OP_COUNT + op) * 4 + sub; };
+    cov.resize((size_t)(L + 1) * OP_COUNT * 4);
     auto rows_of = [&](int op, int sub) -> int {
         switch (op) {
             case OP_RMS_QKV: return sub == 0 ? c.n_q_heads * d : nkv * d;
@@ -483,9 +376,6 @@ int validate(const mk_config& c, const Planned& p) {
         return -1;
     };
     std::vector<uint32_t> signals(nctr, 0);
-    // run-time claims: per claim counter, the pool (first row, rows, rows per chunk) and its claimers
-    struct Claim { int pool0 = 0, pool_n = 0, rows = 0, claimers = 0; };
-    std::vector<Claim> claims(nctr);
     std::vector<std::vector<uint8_t>> attn_seen((size_t)std::max(L, 1) * nkv, std::vector<uint8_t>(p.kv_splits, 0));
     std::vector<uint8_t> lm_seq(std::max(p.n_lm, 1), 0);
     for (int sm = 0; sm < p.n_sm; ++sm) {
@@ -507,7 +397,7 @@ int validate(const mk_config& c, const Planned& p) {
             // waits only on counters produced by strictly earlier ops, with the planned increment
             if (w[W_WAIT_CTR] >= 0) {
                 if (w[W_WAIT_CTR] >= nctr) return MK_ERR_SCHEDULE;
-                const int po = producer_op(w[W_WAIT_CTR], L, nkv);
+                const int po = producer_op(w[W_WAIT_CTR], L);
                 if (po < 0 || po >= oi) return MK_ERR_SCHEDULE;
                 if ((uint32_t)w[W_WAIT_INC] != p.ctr_inc[w[W_WAIT_CTR]] || w[W_WAIT_INC] <= 0) return MK_ERR_SCHEDULE;
             } else if (!(op == OP_RMS_QKV && l == 0) && !(op == OP_LMHEAD_ARGMAX && L == 0)) {
@@ -515,33 +405,10 @@ int validate(const mk_config& c, const Planned& p) {
             }
             if (w[W_SIGNAL_CTR] >= nctr || w[W_AUX_CTR] >= nctr) return MK_ERR_SCHEDULE;
             if (w[W_AUX_CTR] >= 0 && (uint32_t)w[W_AUX_INC] != p.ctr_inc[w[W_AUX_CTR]]) return MK_ERR_SCHEDULE;
-            const bool claimer = w[W_CLAIM_CTR] != -1;
-            if (claimer) {
-                const int cc = w[W_CLAIM_CTR];
-                if (op != OP_FFN && op != OP_LMHEAD_ARGMAX) return MK_ERR_SCHEDULE;
-                if (cc != (op == OP_FFN ? ctr_id(l, C_FFN1) : ctr_lm_claim(L, nkv))) return MK_ERR_SCHEDULE;
-                const int R = op == OP_FFN ? c.ffn : c.vocab;
-                if (w[W_CLAIM_ROWS] <= 0 || w[W_CLAIM_ROWS] > kMaxRows || w[W_POOL_N] <= 0 || w[W_POOL0] < 0 ||
-                    w[W_POOL0] + w[W_POOL_N] != R || (uint32_t)w[W_CLAIM_INC] != p.ctr_inc[cc])
-                    return MK_ERR_SCHEDULE;
-                Claim& cl = claims[cc];
-                if (cl.claimers == 0) {
-                    cl.pool0 = w[W_POOL0];
-                    cl.pool_n = w[W_POOL_N];
-                    cl.rows = w[W_CLAIM_ROWS];
-                    auto& hits = cov[cov_key(l, op, 0)];  // the pool's rows are covered by the claims
-                    if (hits.empty()) hits.assign(R, 0);
-                    for (int r = cl.pool0; r < R; ++r)
-                        if (hits[r]++) return MK_ERR_SCHEDULE;
-                } else if (cl.pool0 != w[W_POOL0] || cl.pool_n != w[W_POOL_N] || cl.rows != w[W_CLAIM_ROWS]) {
-                    return MK_ERR_SCHEDULE;
-                }
-                cl.claimers++;
-            }
             if (op == OP_ATTN) {
                 const int g = w[W_SUB], s = w[W_BEGIN];
                 if (g < 0 || g >= nkv || s < 0 || s >= p.kv_splits || w[W_END] != p.kv_splits) return MK_ERR_SCHEDULE;
-                if (w[W_AUX_CTR] != -1 || w[W_SIGNAL_CTR] != ctr_attn_group(L, nkv, l, g)) return MK_ERR_SCHEDULE;
+                if (w[W_AUX_CTR] != -1 || w[W_SIGNAL_CTR] != ctr_id(l, C_ATTN)) return MK_ERR_SCHEDULE;
                 if (attn_seen[(size_t)l * nkv + g][s]++) return MK_ERR_SCHEDULE;
                 signals[w[W_SIGNAL_CTR]]++;
                 continue;
@@ -552,20 +419,10 @@ int validate(const mk_config& c, const Planned& p) {
             const int R = rows_of(op, op == OP_RMS_QKV ? sub : 0);
             if (op == OP_RMS_QKV && (sub < 0 || sub > 2)) return MK_ERR_SCHEDULE;
             if ((op == OP_MOE_UPGATE || op == OP_MOE_FFN) && (sub < 0 || sub >= c.top_k)) return MK_ERR_SCHEDULE;
-            if (op == OP_OPROJ_RES && (sub < 0 || sub >= nkv || w[W_WAIT_CTR] != ctr_attn_group(L, nkv, l, sub)))
-                return MK_ERR_SCHEDULE;
-            if (op != OP_RMS_QKV && op != OP_MOE_UPGATE && op != OP_MOE_FFN && op != OP_OPROJ_RES && sub != 0)
-                return MK_ERR_SCHEDULE;
-            if (w[W_INIT0] != w[W_INIT1]) {  // residual copy: QKV only, chunks inside the row, each once
-                if (op != OP_RMS_QKV || w[W_INIT0] < 0 || w[W_INIT0] > w[W_INIT1] || w[W_INIT1] > nch)
-                    return MK_ERR_SCHEDULE;
-                for (int k = w[W_INIT0]; k < w[W_INIT1]; ++k)
-                    if (init_hits[l][k]++) return MK_ERR_SCHEDULE;
-            }
+            if (op != OP_RMS_QKV && op != OP_MOE_UPGATE && op != OP_MOE_FFN && sub != 0) return MK_ERR_SCHEDULE;
             const int b = w[W_BEGIN], e = w[W_END];
             const int sets = acc_sets(op, c.hidden, c.n_q_heads * d, c.ffn, c.top_k);
-            if (b < 0 || e > R || b > e || (b == e && !claimer) || e - b > kMaxRows || (e - b) * sets > kRowSlots)
-                return MK_ERR_SCHEDULE;
+            if (b < 0 || e > R || b >= e || e - b > kMaxRows || (e - b) * sets > kRowSlots) return MK_ERR_SCHEDULE;
             auto& hits = cov[cov_key(l, op, sub)];
             if (hits.empty()) hits.assign(R, 0);
             for (int r = b; r < e; ++r)
@@ -598,21 +455,13 @@ int validate(const mk_config& c, const Planned& p) {
                                moe ? OP_MOE_DOWN2_RES : OP_DOWN_RES};
         for (int op : need)
             if (cov[cov_key(l, op, 0)].empty()) return MK_ERR_SCHEDULE;
-        for (int g = 1; g < nkv; ++g)  // every kv group's O-projection columns
-            if (cov[cov_key(l, OP_OPROJ_RES, g)].empty()) return MK_ERR_SCHEDULE;
-        for (int k = 0; k < nch; ++k)  // the whole residual copied once
-            if (init_hits[l][k] != 1) return MK_ERR_SCHEDULE;
         if (moe)  // every routed slot's rows are covered
             for (int sl = 1; sl < c.top_k; ++sl)
                 if (cov[cov_key(l, p.fused_ffn ? OP_MOE_FFN : OP_MOE_UPGATE, sl)].empty()) return MK_ERR_SCHEDULE;
     }
     if (cov[cov_key(L, OP_LMHEAD_ARGMAX, 0)].empty()) return MK_ERR_SCHEDULE;
-    for (int i = 0; i < nctr; ++i) {
-        const Claim& cl = claims[i];
-        const uint32_t claim_inc = cl.claimers ? (uint32_t)((cl.pool_n + cl.rows - 1) / cl.rows + cl.claimers) : 0;
-        if (signals[i] + claim_inc != p.ctr_inc[i]) return MK_ERR_SCHEDULE;
-        if (cl.claimers && signals[i]) return MK_ERR_SCHEDULE;  // a claim counter is never a signal counter
-    }
+    for (int i = 0; i < nctr; ++i)
+        if (signals[i] != p.ctr_inc[i]) return MK_ERR_SCHEDULE;
     return MK_OK;
 }
 
@@ -623,7 +472,6 @@ int simulate(const int32_t* words, int n_sm, int max_instr, const int32_t* n_ins
     long long done = 0;
     for (int e = 1; e <= steps; ++e) {
         std::vector<int> pc(n_sm, 0);
-        std::vector<uint8_t> pool_taken(nctr, 0);  // run-time claims: the first claimer of a step takes the pool
         long long remaining = 0;
         for (int sm = 0; sm < n_sm; ++sm) remaining += n_instr[sm];
         std::vector<int> ready;
@@ -643,14 +491,6 @@ int simulate(const int32_t* words, int n_sm, int max_instr, const int32_t* n_ins
             const int32_t* w = words + ((size_t)sm * max_instr + pc[sm]) * W_NWORDS;
             if (w[W_AUX_CTR] >= 0) ctr[w[W_AUX_CTR]]++;
             if (w[W_SIGNAL_CTR] >= 0) ctr[w[W_SIGNAL_CTR]]++;
-            if (w[W_CLAIM_CTR] >= 0) {  // its chunks (if the pool is still there), then the claim past it
-                const int cc = w[W_CLAIM_CTR];
-                if (!pool_taken[cc] && w[W_CLAIM_ROWS] > 0) {
-                    ctr[cc] += (uint64_t)((w[W_POOL_N] + w[W_CLAIM_ROWS] - 1) / w[W_CLAIM_ROWS]);
-                    pool_taken[cc] = 1;
-                }
-                ctr[cc]++;
-            }
             pc[sm]++;
             remaining--;
             done++;
@@ -695,7 +535,7 @@ extern "C" int mk_simulate(const int32_t* buf, int n_sm, int max_instr, const in
         if (n_instr[sm] < 0 || n_instr[sm] > max_instr) return MK_ERR_INVALID_ARG;
         for (int i = 0; i < n_instr[sm]; ++i) {
             const int32_t* w = buf + ((size_t)sm * max_instr + i) * mk::W_NWORDS;
-            for (int k : {mk::W_WAIT_CTR, mk::W_SIGNAL_CTR, mk::W_AUX_CTR, mk::W_CLAIM_CTR})
+            for (int k : {mk::W_WAIT_CTR, mk::W_SIGNAL_CTR, mk::W_AUX_CTR})
                 if (w[k] >= n_counters || w[k] < -1) return MK_ERR_INVALID_ARG;
         }
     }

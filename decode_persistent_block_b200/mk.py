@@ -23,7 +23,7 @@ ERRORS = {
 CODES = {v: k for k, v in ERRORS.items()}
 MODE_MEGAKERNEL, MODE_MULTI_KERNEL, MODE_MULTI_KERNEL_GRAPH = 0, 1, 2
 FAULT_NONE, FAULT_UNREACHABLE_WAIT, FAULT_BAD_OPCODE, FAULT_PRESET_STOP = 0, 1, 2, 3
-INSTR_WORDS = 24
+INSTR_WORDS = 16
 
 _I, _F, _P = ctypes.c_int, ctypes.c_float, ctypes.c_void_p
 
@@ -45,8 +45,7 @@ class MkOptions(ctypes.Structure):
                 ("l2_prefetch", _I), ("trace", _I), ("snapshots", _I), ("spin_limit_ns", ctypes.c_ulonglong),
                 ("mode", _I), ("n_sm", _I), ("prefetch_ahead", _I), ("prefetch_max_bytes", _I),
                 ("attn_sm_ffn_permille", _I), ("serve_idle_ns", ctypes.c_ulonglong), ("general_kernel", _I),
-                ("split_ffn", _I), ("l2_head_start", _I), ("sm_speed", ctypes.c_void_p), ("n_sm_speed", _I),
-                ("claim_permille", _I)]
+                ("split_ffn", _I), ("l2_head_start", _I), ("sm_speed", ctypes.c_void_p), ("n_sm_speed", _I)]
 
 
 class MkStatus(ctypes.Structure):

@@ -133,6 +133,24 @@ def per_sm_duration(schedule: np.ndarray, trace: np.ndarray, op_name: str, n_lay
     return out
 
 
+def layer_timeline(schedule: np.ndarray, trace: np.ndarray, layer: int) -> str:
+    """Per op of one layer, µs from the layer's first QKV dependency: first start, first and last
+    dependency met, first and last end (the op's blocks)."""
+    g = _groups(schedule, trace)
+    keys = [k for k in g if k[0] == layer]
+    if not keys:
+        return ""
+    q = g.get((layer, "QKV"))
+    t0 = np.nanmin(q[:, T_DEP]) if q is not None else min(np.nanmin(g[k][:, T_START]) for k in keys)
+    lines = [f"layer {layer}: {'op':8s} {'start0':>8s} {'dep0':>8s} {'dep1':>8s} {'end0':>8s} {'end1':>8s} {'blocks':>6s}"]
+    for k in sorted(keys, key=lambda k: np.nanmin(g[k][:, T_START])):
+        a = g[k]
+        lines.append(f"         {k[1]:8s} " + " ".join(f"{v - t0:8.2f}" for v in (
+            np.nanmin(a[:, T_START]), np.nanmin(a[:, T_DEP]), np.nanmax(a[:, T_DEP]), np.nanmin(a[:, T_END]),
+            np.nanmax(a[:, T_END]))) + f" {a.shape[0]:6d}")
+    return "\n".join(lines)
+
+
 def format_breakdown(bd: dict) -> str:
     lines = [f"{'op':8s} " + " ".join(f"{c:>8s}" for c in COLUMNS)]
     for op, row in bd.items():
@@ -158,7 +176,7 @@ def main(argv=None) -> None:
     ap.add_argument("--steps", type=int, default=4)
     ap.add_argument("--npz", default="")
     ap.add_argument("options", nargs="*", help="mk_options fields as key=value (integers)")
-    args = ap.parse_args(argv)
+    args = ap.parse_intermixed_args(argv)
     cfg = configs.get(args.config)
     opts = {k: int(v) for k, v in (kv.split("=") for kv in args.options)}
     W = synth.make_model(cfg)
@@ -174,6 +192,9 @@ def main(argv=None) -> None:
         print(f"{cfg.name}: last step {dec.last_step_ns() / 1000:.1f} us (traced)")
     print(format_breakdown(op_breakdown(sched, tr)))
     print(format_stages(stage_breakdown(sched, tr)))
+    for layer in sorted({0, cfg.n_layers // 2, cfg.n_layers - 1}):
+        if cfg.n_layers:
+            print(layer_timeline(sched, tr, layer))
     present = {OP_NAMES.get(int(o)) for o in np.unique(sched[:, :, 0])}
     big = next((n for n in ("FFN", "MOE_FFN", "UG", "MOE_UG") if n in present), "LM")
     d = per_sm_duration(sched, tr, big, cfg.n_layers)

@@ -135,10 +135,6 @@ typedef struct {
                              grid's block count.  Read (copied) by mk_create and mk_plan; the caller may
                              free it afterwards */
     int n_sm_speed;
-    int claim_permille;   /* dense fused FFN and LM head: each block's fixed share of the rows, per mille of
-                             an even split (0 = default, 1..1000); the remaining rows are claimed at run time
-                             in stage-sized chunks from a per-op counter by whichever block is ready first,
-                             so the op ends together on every SM.  1000 = fixed shares only */
 } mk_options;
 
 /* Device status block, copied out by mk_get_status.  On a device-side error
@@ -185,7 +181,7 @@ int mk_build_schedule(mk_handle *h);
  * Errors: MK_ERR_NO_SCHEDULE, MK_ERR_CAPACITY (cap too small; *n_words is set).
  * Source: the same instruction tensor (Kittens VM summary page, "Method"),
  * exposed so that schedules can be checked on the host. */
-#define MK_INSTR_WORDS 24
+#define MK_INSTR_WORDS 16
 int mk_get_schedule(mk_handle *h, int32_t *buf, size_t cap, size_t *n_words, int *n_sm, int *max_instr);
 
 /* One decode step: embeds `token` (or, if token < 0, the previous step's

@@ -36,8 +36,6 @@ def test_tiny_all_steps(tiny, mode):
     dict(n_sm=7), dict(n_sm=1), dict(kv_splits=1), dict(kv_splits=40), dict(ring_stages=2),
     dict(stage_bytes=4096), dict(stage_bytes=4096, ring_stages=3, l2_prefetch=16384), dict(rows_per_instr=3),
     dict(l2_prefetch=65536), dict(split_ffn=1), dict(split_ffn=1, n_sm=7),
-    dict(claim_permille=800), dict(claim_permille=1), dict(claim_permille=500, n_sm=7),
-    dict(claim_permille=800, stage_bytes=4096, ring_stages=2), dict(claim_permille=800, general_kernel=1),
 ], ids=lambda o: ",".join(f"{k}={v}" for k, v in o.items()))
 def test_tiny_schedule_options(tiny, opts):
     parity.assert_parity(parity.run(tiny, **opts))
@@ -193,25 +191,6 @@ def test_tiny_skewed_sm_speed(tiny):
     import torch
     n = torch.cuda.get_device_properties(0).multi_processor_count
     parity.assert_parity(parity.run(tiny, sm_speed=np.linspace(0.5, 1.5, n)))
-
-
-@pytest.mark.parametrize("permille", [800, 950])
-def test_llama1b_claimed_rows(cuda, permille):
-    # fused FFN and LM head with run-time row claims, in the benchmark's launch configuration
-    _full(configs.LLAMA_1B, 3, claim_permille=permille)
-
-
-def test_llama3b_claimed_rows(cuda):
-    _full(configs.LLAMA_3B, 2, claim_permille=800)
-
-
-def test_claim_counters_are_exact_multiples_after_steps(tiny):
-    tiny.fresh_caches()
-    with tiny.decoder(claim_permille=700) as dec:
-        inc = dec.counter_increments()
-        for s, (pos, tok) in enumerate(parity.schedule(configs.TINY, 6)):
-            dec.step(tok if tok is not None else 1, pos)
-            assert np.array_equal(dec.counters(), (s + 1) * inc.astype(np.uint64)), s
 
 
 def test_llama1b_split_ffn(cuda):

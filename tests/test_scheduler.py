@@ -15,7 +15,7 @@ from decode_persistent_block_b200 import mk
 from synth import configs
 
 OP = dict(RMS_QKV=1, ATTN=2, OPROJ=3, UG=4, DOWN=5, LM=6, MOE_UG=7, MOE_DOWN=8, FFN=9, MOE_FFN=10)
-W_OP, W_LAYER, W_SUB, W_BEGIN, W_END, W_WAIT, W_WINC, W_SIG, W_AUX, W_AINC, W_SEQ, W_INIT0, W_INIT1 = range(13)
+W_OP, W_LAYER, W_SUB, W_BEGIN, W_END, W_WAIT, W_WINC, W_SIG, W_AUX, W_AINC, W_SEQ = range(11)
 
 CFGS = [configs.TINY, configs.LLAMA_1B, configs.LLAMA_3B, configs.MIXTRAL_8L, configs.llama1b_sweep(16384),
         configs.TINY.with_(name="tiny_moe", n_experts=4, top_k=2),
@@ -35,12 +35,7 @@ def instrs(words, n_instr):
 
 
 def n_ctr_per_layer(cfg):
-    return 5  # QKV, ATTN (unused), OPROJ, FFN1, FFN2
-
-
-def attn_group_ctr(cfg, layer, g):
-    # after the per-layer counters and the LM head's: one attention counter per (layer, kv group)
-    return cfg.n_layers * 5 + 1 + layer * cfg.n_kv_heads + g
+    return 5  # QKV, ATTN, OPROJ, FFN1, FFN2
 
 
 @pytest.mark.parametrize("split_ffn", [0, 1], ids=["fused_ffn", "split_ffn"])
@@ -50,9 +45,8 @@ def test_plan_covers_rows_and_counts_signals(cfg, n_sm, split_ffn):
     words, n_instr, inc = dpb.plan(cfg, n_sm, split_ffn=split_ffn)
     L, nkv, d = cfg.n_layers, cfg.n_kv_heads, cfg.head_dim
     per = n_ctr_per_layer(cfg)
-    assert inc.size == L * per + 2 + L * nkv  # + the LM head's claim counter (last)
-    rows = {OP["RMS_QKV"]: {0: cfg.n_heads * d, 1: nkv * d, 2: nkv * d},
-            OP["OPROJ"]: {g: cfg.hidden for g in range(nkv)},
+    assert inc.size == L * per + 1
+    rows = {OP["RMS_QKV"]: {0: cfg.n_heads * d, 1: nkv * d, 2: nkv * d}, OP["OPROJ"]: {0: cfg.hidden},
             OP["UG"]: {0: cfg.ffn}, OP["DOWN"]: {0: cfg.hidden}, OP["LM"]: {0: cfg.vocab},
             OP["MOE_UG"]: {s: cfg.ffn for s in range(max(cfg.top_k, 1))}, OP["MOE_DOWN"]: {0: cfg.hidden},
             OP["FFN"]: {0: cfg.ffn}, OP["MOE_FFN"]: {s: cfg.ffn for s in range(max(cfg.top_k, 1))}}
@@ -67,15 +61,9 @@ def test_plan_covers_rows_and_counts_signals(cfg, n_sm, split_ffn):
             key = (l, int(w[W_SUB]), int(w[W_BEGIN]))
             assert key not in attn_seen
             attn_seen.add(key)
-            assert w[W_AUX] == -1 and w[W_SIG] == attn_group_ctr(cfg, l, int(w[W_SUB])) and w[W_WAIT] == l * per + 0
+            assert w[W_AUX] == -1 and w[W_SIG] == l * per + 1 and w[W_WAIT] == l * per + 0
             signals[w[W_SIG]] += 1
             continue
-        if op == OP["OPROJ"]:  # group g's columns: waits for group g's attention splits only
-            assert w[W_WAIT] == attn_group_ctr(cfg, l, int(w[W_SUB])) and w[W_SIG] == l * per + 2
-        if w[W_INIT1] != w[W_INIT0]:  # residual chunks copied by this QKV instruction
-            assert op == OP["RMS_QKV"] and 0 <= w[W_INIT0] < w[W_INIT1] <= cfg.hidden // 8
-            init = cover.setdefault((l, "init"), np.zeros(cfg.hidden // 8, dtype=np.int32))
-            init[w[W_INIT0]:w[W_INIT1]] += 1
         key = (l, op, int(w[W_SUB]))
         hit = cover.setdefault(key, np.zeros(rows[op][int(w[W_SUB])], dtype=np.int32))
         hit[w[W_BEGIN]:w[W_END]] += 1
@@ -93,18 +81,13 @@ def test_plan_covers_rows_and_counts_signals(cfg, n_sm, split_ffn):
     for l in range(L):
         for op in (OP["RMS_QKV"], OP["OPROJ"]) + ffn_ops:
             assert (l, op, 0) in cover
-        for g in range(nkv):
-            assert (l, OP["OPROJ"], g) in cover
-        assert (l, "init") in cover  # every residual chunk copied exactly once (checked above)
     assert (L, OP["LM"], 0) in cover
     assert np.array_equal(signals, inc)
     if L:
         assert len(attn_seen) == L * nkv * splits
-        # closed form: every split of kv group g signals g's counter, which g's O-projection waits for
+        # closed form: every split of every kv head signals; the O-projection waits for all
         for l in range(L):
-            assert inc[l * per + 1] == 0
-            for g in range(nkv):
-                assert inc[attn_group_ctr(cfg, l, g)] == splits
+            assert inc[l * per + 1] == nkv * splits
 
 
 def _ranges(total, n_sm):
@@ -120,14 +103,10 @@ def test_increment_closed_forms_llama1b(n_sm, split_ffn):
     lm = sum(-(-(b - a) // 1024) for a, b in _ranges(cfg.vocab, n_sm))
     for l in range(cfg.n_layers):
         assert inc[l * per + 0] == n_sm      # QKV: every block holds rows of exactly one of q, k, v
-        # O-proj: one instruction per block (default, blocks shared out between the kv groups), or one
-        # per block and kv group (split FFN: each block takes all groups of its row range, in order)
-        assert inc[l * per + 2] == (n_sm * cfg.n_kv_heads if split_ffn else n_sm)
+        assert inc[l * per + 2] == n_sm      # O-proj: hidden >= n_sm rows, <= 1024 per block
         assert inc[l * per + 3] == (n_sm if split_ffn else 0)  # up/gate (split FFN only)
         assert inc[l * per + 4] == n_sm      # down, or the fused FFN slice
-    assert inc[cfg.n_layers * per] == lm  # the LM head's arrival counter
-    for l in range(cfg.n_layers):  # 6 splits of every kv group, 18 or 19 O-projection blocks per group
-        assert all(inc[attn_group_ctr(cfg, l, g)] == 6 for g in range(cfg.n_kv_heads))
+    assert inc[-1] == lm
     # every block's queue is sorted by (layer, op slot)
     order = {OP["RMS_QKV"]: 0, OP["ATTN"]: 1, OP["OPROJ"]: 2, OP["UG"]: 3, OP["FFN"]: 3, OP["DOWN"]: 4,
              OP["LM"]: 0}
@@ -146,16 +125,6 @@ def test_segments_get_blocks_in_proportion_to_rows(cfg):
     rows = [int(w[W_END] - w[W_BEGIN]) for _, _, w in instrs(words, n_instr) if w[W_OP] == op and w[W_LAYER] == 0]
     assert len(rows) == n_sm
     assert max(rows) <= -(-cfg.qkv_rows // n_sm) + 1
-
-
-def test_split_ffn_oproj_gives_each_block_all_groups_of_its_rows():
-    # the bitwise-reproducible form: every row's group contributions come from one block, in group order
-    cfg = configs.LLAMA_1B
-    words, n_instr, _ = dpb.plan(cfg, 148, split_ffn=1)
-    for sm in (0, 77, 147):
-        o = [w for w in words[sm, :n_instr[sm]] if w[W_OP] == OP["OPROJ"] and w[W_LAYER] == 2]
-        assert [int(w[W_SUB]) for w in o] == list(range(cfg.n_kv_heads))
-        assert len({(int(w[W_BEGIN]), int(w[W_END])) for w in o}) == 1
 
 
 def test_plan_is_deterministic():
@@ -303,11 +272,10 @@ def test_sm_speed_splits_ffn_and_lm_rows_in_proportion(n_sm):
     L = cfg.n_layers
     for slot in (0, 1, 2):
         np.testing.assert_array_equal(inc[slot:5 * L:5], inc0[slot:5 * L:5])
-    np.testing.assert_array_equal(inc[5 * L + 1:], inc0[5 * L + 1:])  # per-group attention and claim counters
     ffn = _rows_per_sm(words, n_instr, "FFN", 3)
     assert inc[5 * 3 + 4] == sum(-(-int(r) // 512) for r in ffn)
     lm = _rows_per_sm(words, n_instr, "LM", L)
-    assert inc[5 * L] == sum(-(-int(r) // 1024) for r in lm)
+    assert inc[-1] == sum(-(-int(r) // 1024) for r in lm)
     rc, done = mk.simulate(words, n_instr, inc, steps=2, seed=3)
     assert rc == 0 and done == 2 * int(n_instr.sum())
 
@@ -327,48 +295,3 @@ def test_sm_speed_uniform_matches_default_and_bad_speeds_are_rejected():
                 np.r_[np.ones(147), np.inf]):
         with pytest.raises(mk.MkError):
             dpb.plan(cfg, 148, sm_speed=bad)
-
-
-W_CLAIM_CTR, W_CLAIM_INC, W_POOL0, W_POOL_N, W_CLAIM_ROWS = 13, 14, 15, 16, 17
-
-
-@pytest.mark.parametrize("permille", [800, 950, 1])
-@pytest.mark.parametrize("cfg", [configs.LLAMA_1B, configs.LLAMA_3B, configs.TINY], ids=lambda c: c.name)
-@pytest.mark.parametrize("n_sm", [148, 7])
-def test_claimed_rows_cover_the_op_and_count_exactly(cfg, n_sm, permille):
-    """Run-time row claiming: fixed shares of the first permille/1000 of the rows, the rest a pool of
-    stage-sized chunks; each block's last instruction of the op claims until it draws past the pool,
-    so the claim counter gains exactly chunks + blocks per step."""
-    words, n_instr, inc = dpb.plan(cfg, n_sm, claim_permille=permille)
-    L, nkv = cfg.n_layers, cfg.n_kv_heads
-    sb = 65536
-    for op, layer, R, crows, cc in (("FFN", 1, cfg.ffn, sb // (4 * cfg.hidden), 1 * 5 + 3),
-                                    ("LM", L, cfg.vocab, sb // (2 * cfg.hidden), L * (5 + nkv) + 1)):
-        ins = [(sm, i, w) for sm, i, w in instrs(words, n_instr) if w[W_OP] == OP[op] and w[W_LAYER] == layer]
-        pool0 = R * permille // 1000
-        hit = np.zeros(R, dtype=np.int32)
-        claimers = 0
-        for sm in range(n_sm):
-            mine = [w for s, _, w in ins if s == sm]
-            assert mine, (op, sm)  # every block takes part
-            for k, w in enumerate(mine):
-                hit[w[W_BEGIN]:w[W_END]] += 1
-                if k == len(mine) - 1:  # the block's last instruction of the op claims
-                    assert w[W_CLAIM_CTR] == cc and w[W_POOL0] == pool0 and w[W_POOL_N] == R - pool0
-                    assert w[W_CLAIM_ROWS] == crows and w[W_CLAIM_INC] == inc[cc]
-                    claimers += 1
-                else:
-                    assert w[W_CLAIM_CTR] == -1
-        assert np.all(hit[:pool0] == 1) and np.all(hit[pool0:] == 0)
-        assert claimers == n_sm
-        assert inc[cc] == -(-(R - pool0) // crows) + n_sm
-    rc, done = dpb.simulate(words, n_instr, inc, steps=3, seed=5)
-    assert rc == mk.MK_OK and done == 3 * int(n_instr.sum())
-
-
-def test_claims_off_by_default_and_bad_permille_rejected():
-    words, n_instr, inc = dpb.plan(configs.LLAMA_1B, 148)
-    assert all(w[W_CLAIM_CTR] == -1 for _, _, w in instrs(words, n_instr))
-    for bad in (1001, 5000):  # (0 or negative selects the default)
-        with pytest.raises(mk.MkError):
-            dpb.plan(configs.LLAMA_1B, 148, claim_permille=bad)
