@@ -409,14 +409,16 @@ __device__ void prefetch_stage(const Plan& pl, int st) {
 }
 
 // Plan instruction i for the loader; for MoE ops wait (bounded) until the
-// consumers have routed the layer, unless `block` is false.
+// consumers have routed the layer, unless `block` is false.  MOE: the
+// instantiation runs MoE schedules (dense ones carry no routing code).
+template <bool MOE>
 __device__ bool loader_plan(const DevParams& p, const StepArgs& a, const int32_t* w, Misc& m, Plan& pl, bool block,
                             int ii) {
     if (!instr_ok(p, w)) {
         pl.n_stages = 0;
         return true;
     }
-    if (needs_routing(w[W_OP])) {
+    if (MOE && needs_routing(w[W_OP])) {
         const int l = w[W_LAYER];
         if (vload(&m.router_layer) != route_key(a.epoch, l, p.L)) {
             if (!block) return false;
@@ -453,7 +455,7 @@ struct LoaderRing {
 };
 
 // One step's queue; false if a wait gave up (the block is leaving).
-template <bool PF, bool TC>
+template <bool PF, bool TC, bool MOE>
 __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, int n, unsigned char* ring,
                        uint64_t* full, uint64_t* empty, Misc& m, LoaderRing& lr) {
     const int NS = p.ring_stages;
@@ -473,7 +475,7 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
     for (int i = 0; i < n; ++i) {
         const int32_t* w = q + (size_t)i * W_NWORDS;
         Plan pl;
-        if (!loader_plan(p, a, w, m, pl, true, i)) break;
+        if (!loader_plan<MOE>(p, a, w, m, pl, true, i)) break;
         bool ok = true;
         unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + i) * kTraceWords : nullptr;
         for (int st = 0; st < pl.n_stages; ++st, ++g) {
@@ -515,7 +517,7 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                             break;
                         }
                         Plan np;
-                        if (!loader_plan(p, a, q + (size_t)(pf_i + 1) * W_NWORDS, m, np, false, pf_i + 1)) break;
+                        if (!loader_plan<MOE>(p, a, q + (size_t)(pf_i + 1) * W_NWORDS, m, np, false, pf_i + 1)) break;
                         pf_i++;
                         pf_plan = np;
                         pf_st = 0;
@@ -1092,7 +1094,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
 // added into the post-FFN residual x2 with float4 atomics.  One instruction,
 // one continuous weight stream per block: the up/gate -> down dependency stays
 // inside the block.
-template <int J, bool HOIST>
+template <int J, bool HOIST, bool MOE>
 __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                           uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
     constexpr int RG = J == 1 ? 8 : J == 2 ? 4 : J == 3 ? 2 : 1;
@@ -1102,7 +1104,7 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     float* part_sums = scratch;  // [2 * rows][8 warps] gate / up row sums, then h[rows]
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
     Plan pl;
-    const bool early = HOIST && op == OP_FFN;  // dense: planned before the wait
+    const bool early = HOIST && (!MOE || op == OP_FFN);  // dense: planned before the wait
     if (early) make_plan(p, a.pos, w, nullptr, pl);
     else prefetch_plan_l1(p, w);  // weight-pointer table entries, while the dependency is pending
 
@@ -1116,8 +1118,10 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     float v[J][8];
     const uint16_t* const* wt = p.wt + (size_t)l * wt_stride(p.E);
     load_rms<J>(p, m, p.x, nullptr, wt[WT_FFN_NORM], v);
-    if (op == OP_MOE_FFN && vload(&m.router_layer) != route_key(a.epoch, l, p.L))
-        route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v, a.epoch);
+    if constexpr (MOE) {
+        if (op == OP_MOE_FFN && vload(&m.router_layer) != route_key(a.epoch, l, p.L))
+            route<J>(p, m, scratch, wt[WT_ROUTER], l, sub == 0 && b == 0, v, a.epoch);
+    }
     if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
     if (!early) {
         int eidx[kMaxTopK];
@@ -1156,7 +1160,7 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     if (tr && tid == 0) tr[T_MAIN] = globaltimer_ns();
 
     // h = silu(g) * u (times the router weight), then kept at the start of the scratch
-    const float wgt = op == OP_MOE_FFN ? m.ew[sub] : 1.0f;
+    const float wgt = MOE && op == OP_MOE_FFN ? m.ew[sub] : 1.0f;
     float hv[2] = {0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -1881,14 +1885,14 @@ __device__ __forceinline__ int gemv_k(const DevParams& p, int op) {
 // JF > 0: every GEMV-type instruction of the schedule has J == JF (checked on
 // the host), so only that instantiation is compiled into the kernel; JF == 0:
 // dispatch on the instruction's J at run time.
-template <int JF>
+template <int JF, bool MOE>
 __device__ bool gemv_dispatch(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                               uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase,
                               int token) {
     if constexpr (JF > 0) {
         // the specialised instantiations run fused-FFN schedules only (chosen on the host)
-        if (w[W_OP] == OP_FFN || w[W_OP] == OP_MOE_FFN)
-            return ffn_instr<JF, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+        if (w[W_OP] == OP_FFN || (MOE && w[W_OP] == OP_MOE_FFN))
+            return ffn_instr<JF, true, MOE>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
         if (w[W_OP] == OP_RMS_QKV || w[W_OP] == OP_OPROJ_RES || w[W_OP] == OP_LMHEAD_ARGMAX)
             return gemv_instr<JF, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
         if (threadIdx.x == 0) {
@@ -1902,10 +1906,10 @@ __device__ bool gemv_dispatch(const DevParams& p, const StepArgs& a, const int32
     const int J = ((kp >> 3) + kConsumerThreads - 1) / kConsumerThreads;
     if (w[W_OP] == OP_FFN || w[W_OP] == OP_MOE_FFN) {
         switch (J) {
-            case 1: return ffn_instr<1, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-            case 2: return ffn_instr<2, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-            case 3: return ffn_instr<3, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
-            case 4: return ffn_instr<4, false>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 1: return ffn_instr<1, false, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 2: return ffn_instr<2, false, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 3: return ffn_instr<3, false, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
+            case 4: return ffn_instr<4, false, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
         }
         return false;
     }
@@ -2034,7 +2038,8 @@ __device__ void serve_respond(const DevParams& p, const StepArgs& a, int next_to
 // cursor (options.l2_prefetch) is compiled in; the specialised instantiations
 // exist with and without it, so the default ones carry no prefetch code.  The
 // consumers' per-instruction prefetch (prefetch_ahead) is in the general one only.
-template <int JF, int DH, bool PF>
+// MOE: MoE routing is compiled in (dense models run instantiations without it).
+template <int JF, int DH, bool PF, bool MOE>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ DevParams p, const StepArgs a) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int NS = p.ring_stages, SB = p.stage_bytes;
@@ -2066,7 +2071,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             for (uint32_t k = 0;; ++k) {
                 StepArgs sa = a;
                 if (a.serve && !serve_take(p, m, k, a, sa)) break;
-                if (!loader<PF, DH == 64>(p, sa, q, n, smem, full, empty, m, lr) || !a.serve) break;
+                if (!loader<PF, DH == 64, MOE>(p, sa, q, n, smem, full, empty, m, lr) || !a.serve) break;
             }
             loader_drain(p, full, lr);
         }
@@ -2114,7 +2119,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
                 else
                     ok = attn_cc(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
             } else {
-                ok = gemv_dispatch<JF>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase, token);
+                ok = gemv_dispatch<JF, MOE>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase, token);
             }
             if (p.trace && tid == 0) p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_END] = globaltimer_ns();
             if (!ok) break;
@@ -2129,12 +2134,14 @@ namespace {
 using KernelFn = void (*)(DevParams, StepArgs);
 KernelFn kernel_of(int variant) {
     switch (variant) {
-        case 1: return megakernel<1, 64, false>;
-        case 2: return megakernel<2, 128, false>;
-        case 3: return megakernel<1, 64, true>;
-        case 4: return megakernel<2, 128, true>;
+        case 1: return megakernel<1, 64, false, false>;
+        case 2: return megakernel<2, 128, false, false>;
+        case 3: return megakernel<1, 64, true, false>;
+        case 4: return megakernel<2, 128, true, false>;
+        case 5: return megakernel<1, 64, false, true>;
+        case 6: return megakernel<2, 128, false, true>;
     }
-    return megakernel<0, 0, true>;
+    return megakernel<0, 0, true, true>;
 }
 // J of a GEMV over K columns (chunks of 8 per consumer thread, per column part)
 int j_of(int K) {
@@ -2143,14 +2150,16 @@ int j_of(int K) {
 }
 }  // namespace
 
-// 0: general; 1 / 2: specialised for one chunk (head_dim 64) / two chunks (head_dim 128) per
-// thread; 3 / 4: the same with the loader's L2-prefetch cursor (options.l2_prefetch > 0).
+// 0: general; 1 / 2: dense, specialised for one chunk (head_dim 64) / two chunks (head_dim 128)
+// per thread; 3 / 4: the same with the loader's L2-prefetch cursor (options.l2_prefetch > 0);
+// 5 / 6: MoE, specialised (without the prefetch cursor; MoE with it runs the general kernel).
 int megakernel_variant(const DevParams& p, bool fused_ffn) {
     if (!fused_ffn || p.prefetch_ahead > 0) return 0;
-    const int jh = j_of(p.H), jo = j_of(p.nq * p.d), pf = p.l2_prefetch > 0 ? 2 : 0;
-    if (jh == 1 && jo == 1 && p.d == 64) return 1 + pf;
-    if (jh == 2 && jo == 2 && p.d == 128) return 2 + pf;
-    return 0;
+    const int jh = j_of(p.H), jo = j_of(p.nq * p.d);
+    const int base = (jh == 1 && jo == 1 && p.d == 64) ? 1 : (jh == 2 && jo == 2 && p.d == 128) ? 2 : 0;
+    if (base == 0) return 0;
+    if (p.E > 0) return p.l2_prefetch > 0 ? 0 : base + 4;
+    return p.l2_prefetch > 0 ? base + 2 : base;
 }
 
 cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, int variant, cudaStream_t stream) {
@@ -2171,7 +2180,7 @@ cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, i
 cudaError_t prepare_megakernel(int ring_stages, int stage_bytes, int* max_blocks_per_sm) {
     const size_t smem = megakernel_smem_bytes(ring_stages, stage_bytes);
     *max_blocks_per_sm = 1 << 30;
-    for (int v = 0; v <= 4; ++v) {
+    for (int v = 0; v <= 6; ++v) {
         cudaError_t e = cudaFuncSetAttribute(kernel_of(v), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         int per_sm = 0;
