@@ -69,6 +69,9 @@ def parse():
     ap.add_argument("--ring-stages", type=int, default=0)
     ap.add_argument("--stage-bytes", type=int, default=0)
     ap.add_argument("--kv-splits", type=int, default=0)
+    ap.add_argument("--spec-experts", type=int, default=-1,
+                    help="MoE configs: speculative expert prediction (0 off, 1 on, 2 mispredict; -1: the "
+                         "library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-baselines", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -298,6 +301,8 @@ def measure(args, cfg, p0, positions, K, Wm, rank, world, local, with_extras=Tru
     mode = {"megakernel": 0, "multi_kernel": 1, "multi_kernel_graph": 2}[args.mode]
     opts = dict(mode=mode, l2_prefetch=args.l2_prefetch, ring_stages=args.ring_stages,
                 stage_bytes=args.stage_bytes, kv_splits=args.kv_splits, serve_idle_ns=2_000_000_000)
+    if cfg.n_experts and args.spec_experts >= 0:
+        opts["spec_experts"] = args.spec_experts
     calib = None
     if args.calibrate and args.mode == "megakernel":
         # start-up calibration, outside the timed region: a few traced steps from p0
@@ -385,6 +390,26 @@ def measure(args, cfg, p0, positions, K, Wm, rank, world, local, with_extras=Tru
                          "h2d_bytes_per_step": 16, "d2h_bytes_per_step": 12,
                          "path": "mk_serve_step (resident grid, pinned mailbox)"}
 
+    # speculative expert prediction (MoE): how many of the fused FFN's expert slots the prediction
+    # named, over a few untimed steps (the getters synchronise)
+    prediction = None
+    if cfg.n_experts and args.mode == "megakernel" and dec.options.spec_experts:
+        from decode_persistent_block_b200 import MkError
+        try:
+            hit = slots = 0
+            tok = dec.step(first, positions[0])
+            n = min(16, len(positions))
+            for i in range(1, n):
+                tok = dec.step(tok, positions[i])
+                for l in range(cfg.n_layers):
+                    pe, re_ = sorted(dec.predicted_experts(l).tolist()), sorted(dec.router(l)[0].tolist())
+                    hit += sum(a == b for a, b in zip(pe, re_))
+                    slots += len(pe)
+            prediction = {"option": int(dec.options.spec_experts), "slots_hit": hit, "slots": slots,
+                          "hit_rate": round(hit / max(slots, 1), 4), "steps": n - 1}
+        except MkError:  # the kernel chosen for these options does not predict
+            prediction = {"option": int(dec.options.spec_experts), "active": False}
+
     baselines = {}
     if not args.no_baselines and args.mode == "megakernel":
         for name, m in (("multi_kernel", 1), ("multi_kernel_graph", 2)):
@@ -403,7 +428,7 @@ def measure(args, cfg, p0, positions, K, Wm, rank, world, local, with_extras=Tru
                      "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
                      "traffic": committed_traffic(cfg.name, args.mode), "launch_us": round(launch_ms * 1000, 2)},
         "e2e": e2e, "e2e_serve": e2e_serve, "baselines": baselines, "clocks": clk, "calib": calib,
-        "steps": K, "warmup": Wm,
+        "steps": K, "warmup": Wm, "expert_prediction": prediction,
     }
 
 
@@ -435,6 +460,8 @@ def run_ours(args, rank, world, local):
                                 "frac_of_8tbs": m["frac_of_8tbs"], "bytes_per_token": m["bytes_per_token"],
                                 "e2e": m["e2e"], "baselines": m["baselines"], "clocks": m["clocks"],
                                 "steps": m["steps"], "warmup": m["warmup"]}
+            if m["expert_prediction"] is not None:
+                per_config[name]["expert_prediction"] = m["expert_prediction"]
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -468,6 +495,7 @@ def run_ours(args, rank, world, local):
         "gpu_launches": K if args.mode == "megakernel" else None,
         "baselines": r["baselines"],
         "per_config": per_config or None,
+        "expert_prediction": r["expert_prediction"],
         "cpu_baseline": cpu,
         "clocks": r["clocks"],
     }

@@ -293,6 +293,10 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     if ((rc = dalloc(h, &p.lm_part, (size_t)lm_slots * 2))) return fail(rc);
     if ((rc = dalloc(h, &p.router_idx, (size_t)std::max(L, 1) * mk::kMaxTopK))) return fail(rc);
     if ((rc = dalloc(h, &p.router_w, (size_t)std::max(L, 1) * mk::kMaxTopK))) return fail(rc);
+    if ((rc = dalloc(h, &p.pred_idx, (size_t)std::max(L, 1) * mk::kMaxTopK))) return fail(rc);
+    e = cudaMemset(p.pred_idx, 0xFF, sizeof(int32_t) * (size_t)std::max(L, 1) * mk::kMaxTopK);  // -1: none
+    if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
+    p.spec_experts = E > 0 ? o.spec_experts : 0;
     if (o.snapshots && (rc = dalloc(h, &p.snap, (size_t)(L + 1) * H))) return fail(rc);
     float2* rope = nullptr;
     if ((rc = dalloc(h, &rope, (size_t)c.max_seq * (d / 2)))) return fail(rc);
@@ -365,6 +369,8 @@ int mk_build_schedule(mk_handle* h) {
     if (plan.fused_ffn && h->cfg.n_layers > 0 && !h->down_t) return MK_ERR_SCHEDULE;
     h->plan = plan;
     h->variant = h->opt.general_kernel ? 0 : mk::megakernel_variant(h->p, plan.fused_ffn);
+    // the prediction runs in the specialised MoE kernels (the general one keeps the prefetch cursor)
+    h->p.spec_experts = h->variant != 0 && plan.fused_ffn && h->cfg.n_experts > 0 ? h->opt.spec_experts : 0;
     int32_t* words = nullptr;
     int32_t* n_instr = nullptr;
     if ((rc = dalloc(h, &words, plan.words.size()))) return rc;
@@ -461,6 +467,16 @@ int mk_get_router(mk_handle* h, int layer, int32_t* idx, float* wts) {
     CK(cudaMemcpy(idx, h->p.router_idx + (size_t)layer * mk::kMaxTopK, sizeof(int32_t) * h->cfg.top_k,
                   cudaMemcpyDeviceToHost));
     CK(cudaMemcpy(wts, h->p.router_w + (size_t)layer * mk::kMaxTopK, sizeof(float) * h->cfg.top_k,
+                  cudaMemcpyDeviceToHost));
+    return MK_OK;
+}
+
+int mk_get_predicted_experts(mk_handle* h, int layer, int32_t* idx) {
+    if (!h || h->serving || !idx || h->cfg.n_experts <= 0 || !h->p.spec_experts || layer < 0 ||
+        layer >= h->cfg.n_layers)
+        return MK_ERR_INVALID_ARG;
+    CK(cudaStreamSynchronize(h->stream));
+    CK(cudaMemcpy(idx, h->p.pred_idx + (size_t)layer * mk::kMaxTopK, sizeof(int32_t) * h->cfg.top_k,
                   cudaMemcpyDeviceToHost));
     return MK_OK;
 }

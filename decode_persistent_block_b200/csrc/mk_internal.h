@@ -51,6 +51,10 @@ enum Word : int {
     W_AUX_CTR = 8,    // ATTN: per-head-group arrival counter; LMHEAD: arrival counter
     W_AUX_INC = 9,    // its per-step increment
     W_SEQ = 10,       // LMHEAD: slot of this instruction's partial argmax; ATTN: unused
+    W_SPEC = 11,      // speculative expert prediction.  QKV: 1 = after it, this block predicts the layer's
+                      //   experts (its last QKV instruction of the layer), 2 = the same and it publishes the
+                      //   prediction; MOE_FFN: 1 = the block's loader streams the predicted expert's first
+                      //   stages before the routing is known (the block predicted this layer).  0: none
     W_NWORDS = MK_INSTR_WORDS
 };
 
@@ -193,6 +197,7 @@ struct DevParams {
     float* snap;       // [(L+1)][H] or null
     int32_t* router_idx;  // [L][kMaxTopK]
     float* router_w;      // [L][kMaxTopK]
+    int32_t* pred_idx;    // [L][kMaxTopK] predicted experts (spec_experts)
     unsigned long long* trace;  // [n_sm][max_instr][kTraceWords] or null
     // kernel knobs
     int ring_stages;
@@ -201,6 +206,7 @@ struct DevParams {
     int l2_head_start;
     int prefetch_ahead;
     int prefetch_max_bytes;
+    int spec_experts;  // MoE: speculative expert prediction (see mk_options)
     unsigned long long spin_limit_ns;
     // serving (only read when the launch's StepArgs.serve is set)
     ServeBox* serve_box;     // device view of the pinned host mailbox

@@ -59,6 +59,8 @@ struct Misc {
     int router_layer;  // route_key(epoch, layer) of the routing in eidx/ew (-1: none)
     int eidx[kMaxTopK];
     float ew[kMaxTopK];
+    int pred_layer;    // route_key(epoch, layer) of the predicted experts in pred_eidx (-1: none)
+    int pred_eidx[kMaxTopK];
     int is_last;
     int pad[3];
     // serving: the step block 0 published, as taken by this block's consumer thread 0
@@ -230,7 +232,15 @@ __device__ __forceinline__ AttnRange attn_range(int pos, int split, int S) {
     return r;
 }
 
-// eidx: the routed experts of the instruction's layer (MoE ops only).
+// Slot k of a fused MoE FFN instruction takes the k-th smallest of the top-k
+// experts in e (the layer's output sums over the routed experts, so the order
+// does not change it).  A prediction of the routed set in another order then
+// still names every slot's expert.  Returns the index into e.
+__device__ __forceinline__ int ffn_slot(const int* e, int topk, int sub) {
+    return (topk == 2 && e[1] < e[0]) ? 1 - sub : sub;
+}
+
+// eidx: the routed (or predicted) experts of the instruction's layer (MoE ops only).
 __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const int* eidx, Plan& pl) {
     const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], e = w[W_END];
     const uint16_t* const* wt = p.wt + (size_t)(l < p.L ? l : 0) * wt_stride(p.E);
@@ -286,12 +296,14 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
             s1 = wt[wt_up(0, p.E)];
             tail = wt[wt_down_t(0, p.E)];
             break;
-        case OP_MOE_FFN:
+        case OP_MOE_FFN: {
+            const int x = eidx[ffn_slot(eidx, p.topk, sub)];
             pl.nspan = 2;
-            s0 = wt[wt_gate(eidx[sub])];
-            s1 = wt[wt_up(eidx[sub], p.E)];
-            tail = wt[wt_down_t(eidx[sub], p.E)];
+            s0 = wt[wt_gate(x)];
+            s1 = wt[wt_up(x, p.E)];
+            tail = wt[wt_down_t(x, p.E)];
             break;
+        }
     }
     pl.kparts = kparts_of(K);
     pl.nphase = nslot * pl.kparts;
@@ -408,6 +420,37 @@ __device__ void prefetch_stage(const Plan& pl, int st) {
     }
 }
 
+// Loader: wait (bounded) until the consumers have set *field to key (a
+// route_key of the routing or of the prediction); false on stop, abort or
+// timeout (recorded).
+__device__ bool wait_misc_key(const DevParams& p, Misc& m, const int* field, int key, int ii, int op) {
+    const uint64_t t0 = globaltimer_ns();
+    uint64_t next = t0 + kStopPollNs;
+    while (vload(field) != key) {
+        const uint64_t now = globaltimer_ns();
+        if (now >= next) {
+            if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
+            if (now - t0 > p.spin_limit_ns) {
+                record_error(p.status, MK_ERR_TIMEOUT, blockIdx.x, ii, op, -1, 0, 0);
+                return false;
+            }
+            next = now + kStopPollNs;
+        }
+    }
+    return true;
+}
+
+// A fused MoE FFN slice's speculative stages hold the routed expert's rows:
+// the predicted and the routed experts of its slot are the same (both known).
+__device__ __forceinline__ bool spec_hit(const DevParams& p, const Misc& m, int sub) {
+    int e[kMaxTopK], q[kMaxTopK];
+    for (int k = 0; k < kMaxTopK; ++k) {
+        e[k] = vload(&m.eidx[k]);
+        q[k] = vload(&m.pred_eidx[k]);
+    }
+    return e[ffn_slot(e, p.topk, sub)] == q[ffn_slot(q, p.topk, sub)];
+}
+
 // Plan instruction i for the loader; for MoE ops wait (bounded) until the
 // consumers have routed the layer, unless `block` is false.  MOE: the
 // instantiation runs MoE schedules (dense ones carry no routing code).
@@ -419,22 +462,10 @@ __device__ bool loader_plan(const DevParams& p, const StepArgs& a, const int32_t
         return true;
     }
     if (MOE && needs_routing(w[W_OP])) {
-        const int l = w[W_LAYER];
-        if (vload(&m.router_layer) != route_key(a.epoch, l, p.L)) {
+        const int key = route_key(a.epoch, w[W_LAYER], p.L);
+        if (vload(&m.router_layer) != key) {
             if (!block) return false;
-            const uint64_t t0 = globaltimer_ns();
-            uint64_t next = t0 + kStopPollNs;
-            while (vload(&m.router_layer) != route_key(a.epoch, l, p.L)) {
-                const uint64_t now = globaltimer_ns();
-                if (now >= next) {
-                    if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
-                    if (now - t0 > p.spin_limit_ns) {
-                        record_error(p.status, MK_ERR_TIMEOUT, blockIdx.x, ii, w[W_OP], -1, 0, 0);
-                        return false;
-                    }
-                    next = now + kStopPollNs;
-                }
-            }
+            if (!wait_misc_key(p, m, &m.router_layer, key, ii, w[W_OP])) return false;
         }
         __threadfence_block();
         int eidx[kMaxTopK];
@@ -475,10 +506,48 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
     for (int i = 0; i < n; ++i) {
         const int32_t* w = q + (size_t)i * W_NWORDS;
         Plan pl;
-        if (!loader_plan<MOE>(p, a, w, m, pl, true, i)) break;
+        int st0 = 0;  // first stage of pl issued below
+        if constexpr (MOE && !PF) {
+            // Speculative expert prediction: the slice's first ring stages come from the expert that
+            // this block predicted after its QKV instruction, issued before the routing is known.
+            // Once it is: on a hit the stream goes on from there, on a miss it restarts with the
+            // routed expert and the consumers drop the speculative stages.
+            if (w[W_OP] == OP_MOE_FFN && w[W_SPEC] != 0 && p.spec_experts) {
+                if (!wait_misc_key(p, m, &m.pred_layer, route_key(a.epoch, w[W_LAYER], p.L), i, w[W_OP])) break;
+                __threadfence_block();
+                int pe[kMaxTopK];
+                for (int k = 0; k < kMaxTopK; ++k) pe[k] = vload(&m.pred_eidx[k]);
+                Plan sp;
+                make_plan(p, a.pos, w, pe, sp);
+                const int ns = sp.n_stages < NS ? sp.n_stages : NS;
+                bool sok = true;
+                for (int st = 0; st < ns; ++st) {
+                    if (!wait_mbar(&empty[slot], phase ^ 1u, p, m, i, w[W_OP])) {
+                        sok = false;
+                        break;
+                    }
+                    issue_stage<TC>(p, sp, st, ring + (size_t)slot * SB, &full[slot]);
+                    if (st == 0 && p.trace)
+                        p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_LD_FIRST] = globaltimer_ns();
+                    used |= 1u << slot;
+                    last_parity = (last_parity & ~(1u << slot)) | (phase << slot);
+                    if (++slot == NS) {
+                        slot = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!sok) return false;
+                if (!loader_plan<MOE>(p, a, w, m, pl, true, i)) break;
+                if (spec_hit(p, m, w[W_SUB])) st0 = ns;
+            } else if (!loader_plan<MOE>(p, a, w, m, pl, true, i)) {
+                break;
+            }
+        } else {
+            if (!loader_plan<MOE>(p, a, w, m, pl, true, i)) break;
+        }
         bool ok = true;
         unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + i) * kTraceWords : nullptr;
-        for (int st = 0; st < pl.n_stages; ++st, ++g) {
+        for (int st = st0; st < pl.n_stages; ++st, ++g) {
             if (!wait_mbar(&empty[slot], phase ^ 1u, p, m, i, w[W_OP])) {
                 ok = false;
                 break;
@@ -715,54 +784,93 @@ __device__ __forceinline__ void dot8x2(const uint4 w, const float* v, float& a0,
 
 // Router of a MoE layer from xn (this thread's slice in v): logits of all
 // experts, top-k (ties to the lower index), softmax over the selected.
-template <int J>
+// PRED: the speculative prediction (into pred_eidx / pred_idx / pred_layer)
+// instead of the routing.  The expert rows are read in batches of RB whose
+// loads are all issued before their FMAs (one L2 round trip per batch), each
+// batch's dot products are reduced across the warp together, and warp 0 adds
+// the 8 warps' partials (in warp order) and selects the top k by shuffles.
+template <int J, bool PRED = false>
 __device__ void route(const DevParams& p, Misc& m, float* scratch, const uint16_t* wr, int layer, bool publish,
                       float (&v)[J][8], uint32_t epoch) {
+    constexpr int RB = J <= 2 ? 8 : 2;  // expert rows per batch: RB * J live 128-bit loads
+    constexpr int LPR = 32 / RB;        // lanes that hold each row's sum after the reduction
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.H, nch = K >> 3, E = p.E;
-    for (int e = 0; e < E; ++e) {  // one expert row at a time: few live registers
-        float a0 = 0.f, a1 = 0.f;
+    for (int e0 = 0; e0 < E; e0 += RB) {
+        uint4 wv[RB][J];
 #pragma unroll
-        for (int j = 0; j < J; ++j) {
-            const int c = tid + kConsumerThreads * j;
-            if (c < nch) dot8x2(__ldg(reinterpret_cast<const uint4*>(wr + (size_t)e * K) + c), v[j], a0, a1);
+        for (int k = 0; k < RB; ++k)
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int c = tid + kConsumerThreads * j;
+                wv[k][j] = (e0 + k < E && c < nch) ? __ldg(reinterpret_cast<const uint4*>(wr + (size_t)(e0 + k) * K) + c)
+                                                   : make_uint4(0u, 0u, 0u, 0u);
+            }
+        float a[RB];
+#pragma unroll
+        for (int k = 0; k < RB; ++k) {
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < J; ++j)
+                if (tid + kConsumerThreads * j < nch) dot8x2(wv[k][j], v[j], a0, a1);
+            a[k] = a0 + a1;
         }
-        const float s_e = warp_sum(a0 + a1);
-        if (lane == 0) scratch[warp * 64 + e] = s_e;
+        const float s_e = reduce_rows<RB>(a, lane);
+        const int e = e0 + lane / LPR;
+        if (lane % LPR == 0 && e < E) scratch[warp * 64 + e] = s_e;
     }
     cbar();
-    if (tid == 0) {
-        float logit[64];
-        for (int e = 0; e < E; ++e) {
-            float t = 0.f;
-            for (int w = 0; w < kConsumerWarps; ++w) t += scratch[w * 64 + e];
-            logit[e] = t;
+    if (warp == 0) {
+        // lane holds experts lane and lane + 32; the prediction's check mode (spec_experts == 2)
+        // takes the lowest scores instead
+        const float sgn = PRED && p.spec_experts == 2 ? -1.0f : 1.0f;
+        float lg[2] = {0.f, 0.f};
+        bool open[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int e = lane + 32 * h;
+            open[h] = e < E;
+            if (open[h])
+                for (int w = 0; w < kConsumerWarps; ++w) lg[h] += scratch[w * 64 + e];
         }
         int idx[kMaxTopK];
-        unsigned long long taken = 0;
+        float sel[kMaxTopK];
         for (int k = 0; k < p.topk; ++k) {
-            int best = -1;
-            for (int e = 0; e < E; ++e) {
-                if ((taken >> e) & 1ull) continue;
-                if (best < 0 || logit[e] > logit[best]) best = e;
+            float bv = -CUDART_INF_F;
+            int bi = 0x7FFFFFFF;
+            if (open[0]) { bv = sgn * lg[0]; bi = lane; }
+            if (open[1] && (bi == 0x7FFFFFFF || sgn * lg[1] > bv)) { bv = sgn * lg[1]; bi = lane + 32; }
+            warp_argmax(bv, bi);
+            idx[k] = bi;
+            sel[k] = sgn * bv;
+            if (bi == lane) open[0] = false;
+            if (bi == lane + 32) open[1] = false;
+        }
+        if (lane == 0) {
+            if constexpr (PRED) {
+                for (int k = 0; k < p.topk; ++k) {
+                    m.pred_eidx[k] = idx[k];
+                    if (publish) p.pred_idx[layer * kMaxTopK + k] = idx[k];
+                }
+                __threadfence_block();
+                vstore(&m.pred_layer, route_key(epoch, layer, p.L));
+            } else {
+                float z = 0.f, ex[kMaxTopK];
+                for (int k = 0; k < p.topk; ++k) {
+                    ex[k] = expf(sel[k] - sel[0]);
+                    z += ex[k];
+                }
+                for (int k = 0; k < p.topk; ++k) {
+                    m.eidx[k] = idx[k];
+                    m.ew[k] = ex[k] / z;
+                    if (publish) {
+                        p.router_idx[layer * kMaxTopK + k] = idx[k];
+                        p.router_w[layer * kMaxTopK + k] = ex[k] / z;
+                    }
+                }
+                __threadfence_block();
+                vstore(&m.router_layer, route_key(epoch, layer, p.L));
             }
-            taken |= 1ull << best;
-            idx[k] = best;
         }
-        float mx = logit[idx[0]], z = 0.f, ex[kMaxTopK];
-        for (int k = 0; k < p.topk; ++k) {
-            ex[k] = expf(logit[idx[k]] - mx);
-            z += ex[k];
-        }
-        for (int k = 0; k < p.topk; ++k) {
-            m.eidx[k] = idx[k];
-            m.ew[k] = ex[k] / z;
-            if (publish) {
-                p.router_idx[layer * kMaxTopK + k] = idx[k];
-                p.router_w[layer * kMaxTopK + k] = ex[k] / z;
-            }
-        }
-        __threadfence_block();
-        vstore(&m.router_layer, route_key(epoch, layer, p.L));
     }
     cbar();
 }
@@ -854,7 +962,9 @@ __device__ __forceinline__ void stage_rows(const uint4* __restrict__ Ws, int row
 
 // HOIST: dense instructions make their stage plan before the dependency wait
 // (costs registers across the wait; used by the specialised kernels).
-template <int J, bool HOIST>
+// SPEC: a QKV instruction marked for it predicts the layer's experts after it
+// signals (MoE instantiations).
+template <int J, bool HOIST, bool SPEC = false>
 __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                            uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase,
                            int token) {
@@ -1083,6 +1193,13 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     }
     cbar();
     if (tid == 0 && w[W_SIGNAL_CTR] >= 0 && op != OP_LMHEAD_ARGMAX) signal_release(p.counters + w[W_SIGNAL_CTR]);
+    if constexpr (SPEC) {
+        // Speculative expert prediction: the router applied to this instruction's input (the
+        // attention input of the layer), off the critical path: the QKV outputs are already
+        // signalled, and the loader streams the predicted experts' first FFN stages meanwhile.
+        if (op == OP_RMS_QKV && w[W_SPEC] != 0 && p.spec_experts)
+            route<J, true>(p, m, scratch, wt[WT_ROUTER], l, w[W_SPEC] == 2, v, a.epoch);
+    }
     return true;
 }
 
@@ -1128,6 +1245,25 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
         for (int k = 0; k < kMaxTopK; ++k) eidx[k] = m.eidx[k];
         make_plan(p, a.pos, w, eidx, pl);
     }
+    if constexpr (MOE) {
+        // speculative stages of a mispredicted expert: released unread (the loader streams the
+        // routed expert's rows after them)
+        if (op == OP_MOE_FFN && w[W_SPEC] != 0 && p.spec_experts && !spec_hit(p, m, sub)) {
+            const int ns = pl.n_stages < p.ring_stages ? pl.n_stages : p.ring_stages;
+            for (int st = 0; st < ns; ++st) {
+                if (warp_wait_full(&full[slot], phase, p, m, ii, op)) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[slot]);
+                } else if (tid == 0) {
+                    vstore(&m.abort_flag, 1);
+                }
+                if (++slot == p.ring_stages) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    }
     const int nch = p.H >> 3;
 
     // up/gate rows
@@ -1160,7 +1296,7 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
     if (tr && tid == 0) tr[T_MAIN] = globaltimer_ns();
 
     // h = silu(g) * u (times the router weight), then kept at the start of the scratch
-    const float wgt = MOE && op == OP_MOE_FFN ? m.ew[sub] : 1.0f;
+    const float wgt = MOE && op == OP_MOE_FFN ? m.ew[ffn_slot(m.eidx, p.topk, sub)] : 1.0f;
     float hv[2] = {0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -1894,7 +2030,7 @@ __device__ bool gemv_dispatch(const DevParams& p, const StepArgs& a, const int32
         if (w[W_OP] == OP_FFN || (MOE && w[W_OP] == OP_MOE_FFN))
             return ffn_instr<JF, true, MOE>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase);
         if (w[W_OP] == OP_RMS_QKV || w[W_OP] == OP_OPROJ_RES || w[W_OP] == OP_LMHEAD_ARGMAX)
-            return gemv_instr<JF, true>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
+            return gemv_instr<JF, true, MOE>(p, a, w, ii, ring, full, empty, scratch, m, slot, phase, token);
         if (threadIdx.x == 0) {
             record_error(p.status, MK_ERR_BAD_INSTR, blockIdx.x, ii, w[W_OP], -1, 0, 0);
             vstore(&m.abort_flag, 1);
@@ -2055,6 +2191,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             mbar_init(&empty[s], kConsumerWarps);
         }
         m.router_layer = -1;
+        m.pred_layer = -1;
         m.is_last = 0;
         m.abort_flag = ld_relaxed_s32(&p.status->stop) ? 1 : 0;
         if (m.abort_flag && atomicCAS(&p.status->code, 0, MK_ERR_STOPPED) == 0) p.status->sm = blockIdx.x;

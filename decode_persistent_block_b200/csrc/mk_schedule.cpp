@@ -194,6 +194,7 @@ int check_options(const mk_config& c, const mk_options& o) {
             if (!(o.sm_speed[i] > 0.f) || !std::isfinite(o.sm_speed[i])) return MK_ERR_INVALID_ARG;
     }
     if (o.mode < MK_MODE_MEGAKERNEL || o.mode > MK_MODE_MULTI_KERNEL_GRAPH) return MK_ERR_INVALID_ARG;
+    if (o.spec_experts < 0 || o.spec_experts > 2) return MK_ERR_INVALID_ARG;
     // ring + barriers + partial-sum slots + misc must fit the 227 KB per-block opt-in limit
     if ((long long)o.ring_stages * o.stage_bytes + 16LL * o.ring_stages + 128 + 4LL * kRowSlots * 8 + 512 > 232448)
         return MK_ERR_INVALID_ARG;
@@ -280,6 +281,29 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
         } else {
             gemv_op(OP_MOE_UPGATE, l, slots, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN1));
             gemv_op(OP_MOE_DOWN2_RES, l, {{0, H}}, ctr_id(l, C_FFN1), ctr_id(l, C_FFN2));
+        }
+    }
+    // Speculative expert prediction: in every block that runs both a QKV instruction and a slice of
+    // the fused MoE FFN of a layer, the last QKV instruction of the layer predicts the experts and
+    // the FFN slices stream the predicted expert's first stages early; the first such block (lowest
+    // index) publishes the layer's prediction.
+    if (moe && fused && o.spec_experts > 0) {
+        std::vector<int> publisher(L, -1);
+        for (int sm = 0; sm < n_sm; ++sm) {
+            auto& qs = q[sm];
+            std::vector<int> last_qkv(L, -1);
+            for (size_t i = 0; i < qs.size(); ++i)
+                if (qs[i][W_OP] == OP_RMS_QKV) last_qkv[qs[i][W_LAYER]] = (int)i;
+            for (size_t i = 0; i < qs.size(); ++i) {
+                const int l = qs[i][W_LAYER];
+                if (qs[i][W_OP] != OP_MOE_FFN || last_qkv[l] < 0) continue;
+                qs[i][W_SPEC] = 1;
+                if (qs[last_qkv[l]][W_SPEC] == 0) qs[last_qkv[l]][W_SPEC] = 1;
+                if (publisher[l] < 0) {
+                    publisher[l] = sm;
+                    qs[last_qkv[l]][W_SPEC] = 2;
+                }
+            }
         }
     }
     // LM head + argmax: partial slots numbered in emission order
@@ -378,8 +402,10 @@ int validate(const mk_config& c, const Planned& p) {
     std::vector<uint32_t> signals(nctr, 0);
     std::vector<std::vector<uint8_t>> attn_seen((size_t)std::max(L, 1) * nkv, std::vector<uint8_t>(p.kv_splits, 0));
     std::vector<uint8_t> lm_seq(std::max(p.n_lm, 1), 0);
+    std::vector<int> spec_publishers(std::max(L, 1), 0), spec_predictors(std::max(L, 1), 0);
     for (int sm = 0; sm < p.n_sm; ++sm) {
         int last_op = -1;
+        int predicted_layer = -1;  // layer predicted by this block's last QKV instruction with W_SPEC
         std::vector<uint8_t> had_moe_ug(std::max(L, 1), 0);
         if (p.n_instr[sm] < 0 || p.n_instr[sm] > p.max_instr) return MK_ERR_SCHEDULE;
         for (int i = 0; i < p.n_instr[sm]; ++i) {
@@ -404,6 +430,22 @@ int validate(const mk_config& c, const Planned& p) {
                 return MK_ERR_SCHEDULE;  // everything but the first op depends on something
             }
             if (w[W_SIGNAL_CTR] >= nctr || w[W_AUX_CTR] >= nctr) return MK_ERR_SCHEDULE;
+            // speculative expert prediction: a predicting QKV instruction is the block's last QKV of
+            // its layer, and an FFN slice streams predicted stages only after its block predicted
+            if (w[W_SPEC] != 0) {
+                const bool qkv = op == OP_RMS_QKV && (w[W_SPEC] == 1 || w[W_SPEC] == 2);
+                const bool ffn = op == OP_MOE_FFN && w[W_SPEC] == 1;
+                if (!(moe && p.fused_ffn) || !(qkv || ffn)) return MK_ERR_SCHEDULE;
+                if (qkv) {
+                    if (predicted_layer == l) return MK_ERR_SCHEDULE;  // one predicting QKV per layer
+                    predicted_layer = l;
+                    spec_predictors[l]++;
+                    if (w[W_SPEC] == 2) spec_publishers[l]++;
+                }
+                if (ffn && predicted_layer != l) return MK_ERR_SCHEDULE;
+            } else if (op == OP_RMS_QKV && predicted_layer == l) {
+                return MK_ERR_SCHEDULE;  // a QKV instruction after the predicting one
+            }
             if (w[W_AUX_CTR] >= 0 && (uint32_t)w[W_AUX_INC] != p.ctr_inc[w[W_AUX_CTR]]) return MK_ERR_SCHEDULE;
             if (op == OP_ATTN) {
                 const int g = w[W_SUB], s = w[W_BEGIN];
@@ -460,6 +502,8 @@ int validate(const mk_config& c, const Planned& p) {
                 if (cov[cov_key(l, p.fused_ffn ? OP_MOE_FFN : OP_MOE_UPGATE, sl)].empty()) return MK_ERR_SCHEDULE;
     }
     if (cov[cov_key(L, OP_LMHEAD_ARGMAX, 0)].empty()) return MK_ERR_SCHEDULE;
+    for (int l = 0; l < L; ++l)  // a predicted layer has exactly one publisher
+        if (spec_publishers[l] != (spec_predictors[l] > 0 ? 1 : 0)) return MK_ERR_SCHEDULE;
     for (int i = 0; i < nctr; ++i)
         if (signals[i] != p.ctr_inc[i]) return MK_ERR_SCHEDULE;
     return MK_OK;

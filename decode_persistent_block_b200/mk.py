@@ -45,7 +45,8 @@ class MkOptions(ctypes.Structure):
                 ("l2_prefetch", _I), ("trace", _I), ("snapshots", _I), ("spin_limit_ns", ctypes.c_ulonglong),
                 ("mode", _I), ("n_sm", _I), ("prefetch_ahead", _I), ("prefetch_max_bytes", _I),
                 ("attn_sm_ffn_permille", _I), ("serve_idle_ns", ctypes.c_ulonglong), ("general_kernel", _I),
-                ("split_ffn", _I), ("l2_head_start", _I), ("sm_speed", ctypes.c_void_p), ("n_sm_speed", _I)]
+                ("split_ffn", _I), ("l2_head_start", _I), ("sm_speed", ctypes.c_void_p), ("n_sm_speed", _I),
+                ("spec_experts", _I)]
 
 
 class MkStatus(ctypes.Structure):
@@ -67,6 +68,7 @@ SIGNATURES = {
     "mk_decode_step": (_I, [_P, ctypes.c_int32, ctypes.c_int32, _P, _P]),
     "mk_get_hidden": (_I, [_P, _I, _P]),
     "mk_get_router": (_I, [_P, _I, _P, _P]),
+    "mk_get_predicted_experts": (_I, [_P, _I, _P]),
     "mk_get_counters": (_I, [_P, _P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)]),
     "mk_get_counter_increments": (_I, [_P, _P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)]),
     "mk_get_status": (_I, [_P, ctypes.POINTER(MkStatus)]),
@@ -293,6 +295,12 @@ class Decoder:
 
     def hidden_all(self) -> np.ndarray:
         return np.stack([self.hidden(l) for l in range(self.config.n_layers + 1)])
+
+    def predicted_experts(self, layer: int) -> np.ndarray:
+        """The experts predicted for `layer` in the last step (options.spec_experts = 1)."""
+        idx = np.empty(self.config.top_k, dtype=np.int32)
+        check(self.lib.mk_get_predicted_experts(self.h, layer, idx.ctypes.data), "mk_get_predicted_experts")
+        return idx
 
     def router(self, layer: int):
         k = self.config.top_k

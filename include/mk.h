@@ -135,6 +135,15 @@ typedef struct {
                              grid's block count.  Read (copied) by mk_create and mk_plan; the caller may
                              free it afterwards */
     int n_sm_speed;
+    int spec_experts;     /* MoE models with the fused FFN: 1 = speculative expert prediction.  After its
+                             last QKV instruction of a layer each block applies the layer's router to the
+                             attention input (the RMSNorm of the residual entering the layer, with the
+                             attention norm weights, already in registers), and its loader streams the
+                             first ring stages of its FFN slice of the predicted experts before the real
+                             routing is known; on a miss those stages are dropped and the routed expert's
+                             rows are streamed instead.  The result is the same either way.  2 = predict
+                             the experts with the lowest scores instead (every prediction misses unless
+                             all experts are selected; exercises the miss path).  0 (default) = off */
 } mk_options;
 
 /* Device status block, copied out by mk_get_status.  On a device-side error
@@ -213,6 +222,19 @@ int mk_get_hidden(mk_handle *h, int layer, float *out_host);
  * Source: the router scoring and expert selection the epic-kernel README fuses
  * into its MoE instructions ("Mixtral 8x7B MoE for batch-1 inference"). */
 int mk_get_router(mk_handle *h, int layer, int32_t *idx, float *w);
+
+/* Speculative expert prediction (options.spec_experts > 0): the top_k experts
+ * predicted for `layer` in the last step from the residual entering the layer
+ * (host array of top_k entries, best first), to compare with mk_get_router.
+ * Synchronises.  Entries are -1 for a layer that no block predicted (the
+ * schedule gives the prediction to blocks that run a QKV instruction and an
+ * FFN slice of the layer; with every block doing so, every layer is predicted).
+ * MK_ERR_INVALID_ARG for dense models or with the option off.
+ * Source: the instruction that predicts the top-2 experts from the
+ * pre-attention residual while attention runs, so that the predicted experts'
+ * weights are on their way before the router confirms them (epic-kernel README,
+ * "Speculative expert prediction"). */
+int mk_get_predicted_experts(mk_handle *h, int layer, int32_t *idx);
 
 /* Dependency counters (uint32, monotone across steps) into host `out`.
  * Source: the blocks synchronise on the device instead of through kernel

@@ -72,6 +72,8 @@ def lib():
                                       _P]
         L.orc_decode_step.restype = _I
         L.orc_num_threads.restype = _I
+        L.orc_predict_experts.argtypes = [ctypes.POINTER(Shape), ctypes.POINTER(Weights), _I, _P, _P]
+        L.orc_predict_experts.restype = _I
         _lib = L
     return _lib
 
@@ -211,4 +213,18 @@ class Model:
                                     rw.ctypes.data if cfg.n_experts else None)
         if nxt < 0:
             raise ValueError(f"oracle rejected token={token} pos={pos}")
-        return {"logits": logits, "hidden": hidden, "next": nxt, "router_idx": ridx, "router_w": rw}
+        pred = None
+        if cfg.n_experts and hidden is not None:
+            pred = np.stack([self.predicted_experts(hidden[l], l) for l in range(cfg.n_layers)]) \
+                if cfg.n_layers else np.zeros((0, K), dtype=np.int32)
+        return {"logits": logits, "hidden": hidden, "next": nxt, "router_idx": ridx, "router_w": rw,
+                "pred_idx": pred}
+
+    def predicted_experts(self, x, layer: int) -> np.ndarray:
+        """Speculative expert prediction of `layer` from the residual x entering it (orc_predict_experts)."""
+        x = _f64(x)
+        idx = np.empty(self.cfg.top_k, dtype=np.int32)
+        if lib().orc_predict_experts(ctypes.byref(self.shape), ctypes.byref(self.weights), int(layer),
+                                     x.ctypes.data, idx.ctypes.data) != 0:
+            raise ValueError(f"oracle rejected the prediction of layer {layer}")
+        return idx

@@ -175,6 +175,18 @@ static void ffn(const uint16_t *wg, const uint16_t *wu, const uint16_t *wd, int 
     free(u);
 }
 
+int orc_predict_experts(const orc_shape *s, const orc_weights *w, int layer, const double *x, int *idx) {
+    const int H = s->hidden, E = s->n_experts, K = s->top_k;
+    if (E <= 0 || K < 1 || K > E || E > 64 || layer < 0 || layer >= s->n_layers) return -1;
+    double *xn = (double *)malloc(sizeof(double) * (size_t)H);
+    double r[64], wt[64];
+    orc_rmsnorm(x, w->attn_norm[layer], H, s->rms_eps, xn);
+    orc_gemv(w->router[layer], E, H, xn, r);
+    orc_topk(r, E, K, idx, wt);
+    free(xn);
+    return 0;
+}
+
 int orc_decode_step(const orc_shape *s, const orc_weights *w, uint16_t *kcache, uint16_t *vcache, int token,
                     int pos, double *logits, double *hidden, int *router_idx, double *router_w) {
     const int L = s->n_layers, H = s->hidden, nq = s->n_heads, nkv = s->n_kv_heads, d = s->head_dim;

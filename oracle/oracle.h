@@ -67,6 +67,18 @@ int orc_argmax(const double *v, int n);
 int orc_decode_step(const orc_shape *s, const orc_weights *w, uint16_t *kcache, uint16_t *vcache, int token,
                     int pos, double *logits, double *hidden, int *router_idx, double *router_w);
 
+/* Speculative expert prediction for MoE layer `layer`: the top_k experts
+ * (best first) that the layer's router gives the layer's attention input,
+ * rmsnorm(x) with the attention norm weights, where x is the residual entering
+ * the layer (hidden[layer] of orc_decode_step).  The expert choice that the
+ * FFN of the layer makes applies the same router to the residual after
+ * attention, normalised with the FFN norm weights; the prediction reads the
+ * residual before attention (epic-kernel README, "Speculative expert
+ * prediction").  The pages do not give the predictor's form: this is the
+ * plainest reading, the layer's own router on the pre-attention normalised
+ * residual.  Returns 0, or -1 on bad arguments. */
+int orc_predict_experts(const orc_shape *s, const orc_weights *w, int layer, const double *x, int *idx);
+
 int orc_num_threads(void);
 
 #ifdef __cplusplus

@@ -18,6 +18,9 @@ HIDDEN_RTOL = 1e-2
 LOGIT_ATOL = 5e-2
 MARGIN = 0.1
 ROUTER_MARGIN = 1e-2
+# The prediction's router scores come from the kernel's own fp32 residual (within HIDDEN_RTOL of the
+# oracle's): below this gap between the k-th and (k+1)-th score the two may pick differently.
+PRED_MARGIN = 1e-2
 
 
 def schedule(cfg, steps: int | None = None):
@@ -61,7 +64,36 @@ class Setup:
         return Decoder(self.cfg, self.dW, self.dk, self.dv, **opts)
 
 
-def compare_step(cfg, dec, logits_gpu, o, gpu_next) -> dict:
+def prediction_scores(cfg, weights: dict, hidden_l, layer: int) -> np.ndarray:
+    """Router scores of the attention input of `layer` (from the oracle's building blocks)."""
+    L = weights["layers"][layer]
+    return oracle.gemv(L["router"], oracle.rmsnorm(hidden_l, L["attn_norm"], cfg.rms_eps))
+
+
+def _slots(e):
+    """Experts of the fused MoE FFN's slots: the routed (or predicted) experts in ascending order."""
+    return sorted(int(x) for x in e)
+
+
+def prediction_report(cfg, dec, o, weights: dict) -> list:
+    """Per layer: (GPU prediction, expected prediction, score margin at the cut, slots hit).
+
+    spec_experts 1 predicts the top_k router scores of the attention input; 2 the bottom top_k."""
+    sgn = -1.0 if dec.options.spec_experts == 2 else 1.0
+    out = []
+    for l in range(cfg.n_layers):
+        s = sgn * prediction_scores(cfg, weights, o["hidden"][l], l)
+        want = oracle.topk(s, cfg.top_k)[0]
+        srt = np.sort(s)[::-1]
+        margin = float(srt[cfg.top_k - 1] - srt[cfg.top_k]) if cfg.n_experts > cfg.top_k else np.inf
+        got = dec.predicted_experts(l)
+        routed = dec.router(l)[0]
+        hits = sum(a == b for a, b in zip(_slots(got), _slots(routed)))
+        out.append((got.tolist(), want.tolist(), margin, hits))
+    return out
+
+
+def compare_step(cfg, dec, logits_gpu, o, gpu_next, weights: dict | None = None) -> dict:
     lo = o["logits"]
     lg = logits_gpu.astype(np.float64)
     srt = np.sort(lo)
@@ -76,6 +108,8 @@ def compare_step(cfg, dec, logits_gpu, o, gpu_next) -> dict:
         for l in range(cfg.n_layers):
             gi, gw = dec.router(l)
             r["router"].append((gi.tolist(), o["router_idx"][l].tolist(), gw.tolist(), o["router_w"][l].tolist()))
+        if dec.options.spec_experts and weights is not None:
+            r["pred"] = prediction_report(cfg, dec, o, weights)
     return r
 
 
@@ -93,7 +127,7 @@ def run(setup: Setup, steps: int | None = None, orc=None, **opts) -> list[dict]:
             t = tok if tok is not None else nxt
             gpu_next = dec.step(t, pos, logits=logits)
             o = orc.step(t, pos)
-            r = compare_step(cfg, dec, logits.cpu().numpy(), o, gpu_next)
+            r = compare_step(cfg, dec, logits.cpu().numpy(), o, gpu_next, setup.W)
             r["pos"] = pos
             reports.append(r)
             nxt = o["next"]
@@ -111,4 +145,7 @@ def assert_parity(reports: list[dict], cfg=None):
         for gi, oi, gw, ow in r.get("router", []):
             assert gi == oi, (r["pos"], gi, oi)
             assert np.allclose(gw, ow, atol=1e-4), (gw, ow)
+        for got, want, margin, _ in r.get("pred", []):
+            if margin > PRED_MARGIN:
+                assert got == want, (r["pos"], got, want, margin)
     return worst_h, worst_l

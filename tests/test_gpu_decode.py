@@ -217,3 +217,66 @@ def test_llama1b_kv_sweep(cuda, prefill):
 
 def test_mixtral8l(cuda):
     _full(configs.MIXTRAL_8L, 3)
+
+
+# ---- speculative expert prediction ------------------------------------------------
+
+def _pred_stats(reports):
+    """(layers predicted as the oracle predicts where the margin allows, slots hit, slots)."""
+    hits = slots = 0
+    for r in reports:
+        for got, want, margin, h in r["pred"]:
+            hits += h
+            slots += len(got)
+    return hits, slots
+
+
+@pytest.mark.parametrize("spec", [1, 2], ids=["predict", "mispredict"])
+@pytest.mark.parametrize("E,k", [(4, 2), (2, 1), (8, 2)])
+def test_tiny_moe_speculative_experts(cuda, E, k, spec):
+    # spec 1 streams the predicted experts' first FFN stages before the routing; spec 2 predicts the
+    # lowest-scoring experts, so most slots miss and their speculative stages are dropped
+    cfg = configs.TINY.with_(name=f"tiny_moe{E}_{k}", n_experts=E, top_k=k)
+    reps = parity.run(parity.Setup(cfg), spec_experts=spec)
+    parity.assert_parity(reps, cfg)
+    assert all("pred" in r for r in reps)
+
+
+def _no_attention_mixing(W):
+    for L in W["layers"]:
+        L["wo"] = np.zeros_like(L["wo"])
+        L["ffn_norm"] = L["attn_norm"].copy()
+
+
+@pytest.mark.parametrize("spec", [1, 2], ids=["all_hit", "all_miss"])
+def test_tiny_moe_speculative_experts_all_hit_or_all_miss(cuda, spec):
+    # With W_o = 0 and one set of norm weights the router sees the attention input itself: the
+    # prediction is the routing (every slot hits), and its inverse (bottom-2 of 4) misses every slot.
+    cfg = configs.TINY.with_(name="tiny_moe4_2", n_experts=4, top_k=2)
+    W = parity.synth.make_model(cfg)
+    _no_attention_mixing(W)
+    reps = parity.run(parity.Setup(cfg, W), spec_experts=spec)
+    parity.assert_parity(reps, cfg)
+    hits, slots = _pred_stats(reps)
+    assert slots == len(reps) * cfg.n_layers * cfg.top_k
+    assert hits == (slots if spec == 1 else 0), (hits, slots)
+
+
+def test_tiny_moe_speculative_experts_off_is_rejected_by_the_getter(cuda):
+    from decode_persistent_block_b200 import MkError
+    cfg = configs.TINY.with_(name="tiny_moe4_2", n_experts=4, top_k=2)
+    s = parity.Setup(cfg)
+    with s.decoder() as dec:
+        dec.step(1, 0)
+        with pytest.raises(MkError):
+            dec.predicted_experts(0)
+    with s.decoder(spec_experts=1, l2_prefetch=65536) as dec:  # the general kernel does not predict
+        dec.step(1, 0)
+        with pytest.raises(MkError):
+            dec.predicted_experts(0)
+
+
+def test_mixtral8l_speculative_experts(cuda):
+    reps = _full(configs.MIXTRAL_8L, 3, spec_experts=1)
+    hits, slots = _pred_stats(reps)
+    print(f"mixtral8l speculative experts: {hits}/{slots} slots hit")

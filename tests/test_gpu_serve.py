@@ -81,14 +81,16 @@ def test_served_steps_default_options(tiny):
         np.testing.assert_allclose(a, b, rtol=1e-4, atol=1e-4)
 
 
-def test_serve_moe(cuda):
+@pytest.mark.parametrize("spec", [0, 1, 2], ids=["no_spec", "spec", "spec_miss"])
+def test_serve_moe(cuda, spec):
+    # the resident grid carries the speculative expert prediction across its served steps
     cfg = configs.TINY.with_(name="tiny_moe4_2", n_experts=4, top_k=2)
     setup = parity.Setup(cfg)
     import torch
     from decode_persistent_block_b200 import Decoder
     ref = []
     setup.fresh_caches()
-    with setup.decoder() as dec:
+    with setup.decoder(spec_experts=spec) as dec:
         nxt = None
         for pos, tok in parity.schedule(cfg):
             nxt = dec.step(tok if tok is not None else nxt, pos)
@@ -96,7 +98,7 @@ def test_serve_moe(cuda):
     setup.fresh_caches()
     torch.cuda.synchronize()
     s = torch.cuda.Stream()
-    dec = Decoder(cfg, setup.dW, setup.dk, setup.dv, stream=s, serve_idle_ns=IDLE)
+    dec = Decoder(cfg, setup.dW, setup.dk, setup.dv, stream=s, serve_idle_ns=IDLE, spec_experts=spec)
     try:
         dec.serve_start()
         got, nxt = [], None

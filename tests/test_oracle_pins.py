@@ -372,6 +372,55 @@ def test_moe_router_choice_is_exhaustive_top2_of_router_scores():
         np.testing.assert_allclose(out["hidden"][1], expect, atol=1e-12)
 
 
+def _no_attention_mixing(W):
+    """Attention adds nothing to the residual (W_o = 0) and the FFN norm weights are the attention
+    norm weights: the FFN's router then sees exactly the attention input of its layer."""
+    for L in W["layers"]:
+        L["wo"] = _zero_like(L["wo"])
+        L["ffn_norm"] = L["attn_norm"].copy()
+
+
+def test_prediction_is_the_routing_when_attention_adds_nothing():
+    # Speculative expert prediction reads the residual entering the layer; the router reads it after
+    # attention.  With nothing added by attention (and one set of norm weights) the two agree in every
+    # layer, which fixes the prediction's input to the layer's own entering residual.
+    cfg = TINY.with_(name="tiny_moe", n_layers=3, n_experts=8, top_k=2)
+    W = synth.make_model(cfg)
+    _no_attention_mixing(W)
+    kc, vc = synth.make_kv_cache(cfg)
+    m = oracle.Model(cfg, W, kc, vc)
+    for pos, tok in enumerate((5, 600, 3000, 77)):
+        out = m.step(tok, pos)
+        np.testing.assert_array_equal(out["pred_idx"], out["router_idx"])
+    # top-1 of 4 experts too
+    cfg1 = cfg.with_(n_experts=4, top_k=1)
+    W1 = synth.make_model(cfg1)
+    _no_attention_mixing(W1)
+    kc, vc = synth.make_kv_cache(cfg1)
+    out = oracle.Model(cfg1, W1, kc, vc).step(42, 0)
+    np.testing.assert_array_equal(out["pred_idx"], out["router_idx"])
+
+
+def test_prediction_ignores_the_ffn_norm_weights():
+    # The prediction of layer 0 is made from the embedding row with the attention norm weights: changing
+    # the FFN norm weights changes the routing but never the prediction.
+    cfg = TINY.with_(name="tiny_moe", n_layers=1, n_experts=8, top_k=2)
+    W = synth.make_model(cfg)
+    _no_attention_mixing(W)
+    kc, vc = synth.make_kv_cache(cfg)
+    preds, routes = [], []
+    for seed in range(6):
+        W["layers"][0]["ffn_norm"] = synth.normal_bf16((cfg.hidden,), 0, f"fn{seed}", 1.0)
+        out = oracle.Model(cfg, W, kc.copy(), vc.copy()).step(321, 0)
+        preds.append(tuple(out["pred_idx"][0]))
+        routes.append(tuple(out["router_idx"][0]))
+    assert len(set(preds)) == 1
+    assert len(set(routes)) > 1  # the FFN norm weights did change the routing
+    W["layers"][0]["ffn_norm"] = W["layers"][0]["attn_norm"].copy()
+    out = oracle.Model(cfg, W, kc.copy(), vc.copy()).step(321, 0)
+    assert tuple(out["router_idx"][0]) == preds[0]
+
+
 def test_rejects_bad_token_and_position():
     cfg = TINY
     W = synth.make_model(cfg)

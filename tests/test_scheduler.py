@@ -295,3 +295,57 @@ def test_sm_speed_uniform_matches_default_and_bad_speeds_are_rejected():
                 np.r_[np.ones(147), np.inf]):
         with pytest.raises(mk.MkError):
             dpb.plan(cfg, 148, sm_speed=bad)
+
+
+W_SPEC = 11
+
+
+@pytest.mark.parametrize("n_sm", [148, 37, 600, 1])
+@pytest.mark.parametrize("cfg", [configs.MIXTRAL_8L, configs.TINY.with_(name="tiny_moe", n_experts=4, top_k=2),
+                                 configs.TINY.with_(name="tiny_moe1", n_experts=2, top_k=1)], ids=lambda c: c.name)
+def test_speculative_prediction_marks(cfg, n_sm):
+    # Every block that runs a QKV instruction and a fused MoE FFN slice of a layer predicts the layer's
+    # experts after its last QKV instruction of the layer; those FFN slices stream the prediction; the
+    # lowest such block publishes.  Nothing else carries the mark.
+    words, n_instr, _ = dpb.plan(cfg, n_sm, spec_experts=1)
+    L = cfg.n_layers
+    expect = np.zeros_like(words[:, :, W_SPEC])
+    publisher = [None] * L
+    for sm in range(n_sm):
+        q = words[sm, :n_instr[sm]]
+        for l in range(L):
+            qkv = [i for i in range(len(q)) if q[i, W_OP] == OP["RMS_QKV"] and q[i, W_LAYER] == l]
+            ffn = [i for i in range(len(q)) if q[i, W_OP] == OP["MOE_FFN"] and q[i, W_LAYER] == l]
+            if qkv and ffn:
+                assert max(qkv) < min(ffn)
+                expect[sm, max(qkv)] = 1
+                expect[sm, ffn] = 1
+                if publisher[l] is None:
+                    publisher[l] = sm
+                    expect[sm, max(qkv)] = 2
+    np.testing.assert_array_equal(words[:, :, W_SPEC], expect)
+    if (cfg.n_heads + 2 * cfg.n_kv_heads) * cfg.head_dim >= n_sm:
+        # every block holds QKV rows of every layer: every FFN slice streams a prediction
+        ffn = words[:, :, W_OP] == OP["MOE_FFN"]
+        assert np.all(words[:, :, W_SPEC][ffn] == 1)
+    else:  # more blocks than QKV rows: the blocks without QKV rows stream no prediction
+        assert np.any(expect[words[:, :, W_OP] == OP["MOE_FFN"]] == 0)
+    # the mark changes nothing else
+    base, n0, inc0 = dpb.plan(cfg, n_sm)
+    assert np.all(base[:, :, W_SPEC] == 0)
+    w2 = words.copy()
+    w2[:, :, W_SPEC] = 0
+    np.testing.assert_array_equal(w2, base)
+
+
+@pytest.mark.parametrize("cfg,opts", [(configs.LLAMA_1B, {}), (configs.MIXTRAL_8L, dict(split_ffn=1))],
+                         ids=["dense", "moe_split_ffn"])
+def test_speculative_prediction_needs_the_fused_moe_ffn(cfg, opts):
+    words, _, _ = dpb.plan(cfg, 148, spec_experts=1, **opts)
+    assert np.all(words[:, :, W_SPEC] == 0)
+
+
+def test_speculative_prediction_option_range():
+    for bad in (-1, 3):
+        with pytest.raises(mk.MkError):
+            dpb.plan(configs.MIXTRAL_8L, 148, spec_experts=bad)
