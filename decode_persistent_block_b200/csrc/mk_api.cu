@@ -121,7 +121,7 @@ int make_kv_maps(mk_handle* h, const mk_config& c, const mk_options& o, void* kc
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
     const int d = c.head_dim;
-    const cuuint64_t rows = (cuuint64_t)std::max(c.n_layers, 1) * c.n_kv_heads * c.max_seq;
+    const cuuint64_t rows = (cuuint64_t)std::max(o.batch, 1) * std::max(c.n_layers, 1) * c.n_kv_heads * c.max_seq;
     const cuuint64_t dims[2] = {(cuuint64_t)d, rows};
     const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
     const cuuint32_t box[2] = {64u, (cuuint32_t)mk::attn_box_rows(o.stage_bytes, d)};
@@ -236,13 +236,16 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
 
     const mk_config& c = *cfg;
     const int L = c.n_layers, H = c.hidden, d = c.head_dim, nq = c.n_q_heads, nkv = c.n_kv_heads;
-    const int S = o.kv_splits > 0 ? o.kv_splits : mk::default_kv_splits(c, h->n_sm);
+    const int NB = o.batch;
+    const int S = o.kv_splits > 0 ? o.kv_splits : mk::default_kv_splits(c, h->n_sm, NB);
     const int E = c.n_experts, topk = E > 0 ? c.top_k : 1;
     mk::DevParams& p = h->p;
     std::memset(&p, 0, sizeof(p));
     p.L = L; p.H = H; p.nq = nq; p.nkv = nkv; p.d = d; p.F = c.ffn; p.V = c.vocab; p.E = E;
     p.topk = E > 0 ? c.top_k : 0; p.max_seq = c.max_seq; p.eps = c.rms_eps; p.kv_splits = S;
     p.n_ctr = mk::n_counters(L);
+    p.nb = NB;
+    p.kv_seq_stride = (size_t)L * nkv * c.max_seq * d;
     p.embed = static_cast<const uint16_t*>(w->embed);
     p.lm_head = static_cast<const uint16_t*>(w->lm_head);
     p.final_norm = static_cast<const uint16_t*>(w->final_norm);
@@ -277,27 +280,30 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
         }
     }
     const uint16_t** wt_dev = nullptr;
-    const int lm_slots = std::max(h->n_sm + c.vocab / o.rows_per_instr + 1, mk::baseline_lm_blocks(p, h->n_sm));
+    const int lm_rows = std::min(o.rows_per_instr, mk::kRowSlots / NB);  // LM-head rows per instruction, at most
+    const int lm_slots = std::max(h->n_sm + c.vocab / lm_rows + 1, mk::baseline_lm_blocks(p, h->n_sm));
     h->lm_slots = lm_slots;
     if ((rc = dalloc(h, &wt_dev, h->wt_host.size()))) return fail(rc);
     if ((rc = dalloc(h, &p.counters, (size_t)p.n_ctr))) return fail(rc);
     if ((rc = dalloc(h, &p.status, 1))) return fail(rc);
-    if ((rc = dalloc(h, &p.x, (size_t)H))) return fail(rc);
-    if ((rc = dalloc(h, &p.x2, (size_t)H))) return fail(rc);
-    if ((rc = dalloc(h, &p.qkv, (size_t)(nq + 2 * nkv) * d))) return fail(rc);
+    // per-sequence activations: NB copies one after the other
+    if ((rc = dalloc(h, &p.x, (size_t)NB * H))) return fail(rc);
+    if ((rc = dalloc(h, &p.x2, (size_t)NB * H))) return fail(rc);
+    if ((rc = dalloc(h, &p.qkv, (size_t)NB * (nq + 2 * nkv) * d))) return fail(rc);
     if ((rc = dalloc(h, &p.attn, (size_t)nq * d))) return fail(rc);
-    if ((rc = dalloc(h, &p.part_o, (size_t)nq * S * d))) return fail(rc);
-    if ((rc = dalloc(h, &p.part_ml, (size_t)nq * S * 2))) return fail(rc);
+    if ((rc = dalloc(h, &p.part_o, (size_t)NB * nq * S * d))) return fail(rc);
+    if ((rc = dalloc(h, &p.part_ml, (size_t)NB * nq * S * 2))) return fail(rc);
     if ((rc = dalloc(h, &p.hbuf, (size_t)topk * c.ffn))) return fail(rc);
-    if ((rc = dalloc(h, &p.logits, (size_t)c.vocab))) return fail(rc);
-    if ((rc = dalloc(h, &p.lm_part, (size_t)lm_slots * 2))) return fail(rc);
+    if ((rc = dalloc(h, &p.logits, (size_t)NB * c.vocab))) return fail(rc);
+    if ((rc = dalloc(h, &p.lm_part, (size_t)lm_slots * NB * 2))) return fail(rc);
+    if ((rc = dalloc(h, &p.next_tok, (size_t)mk::kMaxBatch))) return fail(rc);
     if ((rc = dalloc(h, &p.router_idx, (size_t)std::max(L, 1) * mk::kMaxTopK))) return fail(rc);
     if ((rc = dalloc(h, &p.router_w, (size_t)std::max(L, 1) * mk::kMaxTopK))) return fail(rc);
     if ((rc = dalloc(h, &p.pred_idx, (size_t)std::max(L, 1) * mk::kMaxTopK))) return fail(rc);
     e = cudaMemset(p.pred_idx, 0xFF, sizeof(int32_t) * (size_t)std::max(L, 1) * mk::kMaxTopK);  // -1: none
     if (e != cudaSuccess) { h->last_cuda = e; return fail(MK_ERR_CUDA); }
     p.spec_experts = E > 0 ? o.spec_experts : 0;
-    if (o.snapshots && (rc = dalloc(h, &p.snap, (size_t)(L + 1) * H))) return fail(rc);
+    if (o.snapshots && (rc = dalloc(h, &p.snap, (size_t)NB * (L + 1) * H))) return fail(rc);
     float2* rope = nullptr;
     if ((rc = dalloc(h, &rope, (size_t)c.max_seq * (d / 2)))) return fail(rc);
     if ((rc = dalloc(h, &h->stepbuf, 1))) return fail(rc);
@@ -369,6 +375,7 @@ int mk_build_schedule(mk_handle* h) {
     if (plan.fused_ffn && h->cfg.n_layers > 0 && !h->down_t) return MK_ERR_SCHEDULE;
     h->plan = plan;
     h->variant = h->opt.general_kernel ? 0 : mk::megakernel_variant(h->p, plan.fused_ffn);
+    if (h->variant < 0) return MK_ERR_UNSUPPORTED;  // no kernel instantiation for this batch
     // the prediction runs in the specialised MoE kernels (the general one keeps the prefetch cursor)
     h->p.spec_experts = h->variant != 0 && plan.fused_ffn && h->cfg.n_experts > 0 ? h->opt.spec_experts : 0;
     int32_t* words = nullptr;
@@ -401,7 +408,7 @@ int mk_get_schedule(mk_handle* h, int32_t* buf, size_t cap, size_t* n_words, int
 }
 
 int mk_decode_step(mk_handle* h, int32_t token, int32_t pos, float* logits_dev, int32_t* next_token_host) {
-    if (!h || h->serving) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving || h->p.nb > 1) return MK_ERR_INVALID_ARG;  // batched handles: mk_decode_step_batch
     if (token >= h->cfg.vocab || pos < 0 || pos >= h->cfg.max_seq) return MK_ERR_INVALID_ARG;
     if (!h->scheduled) return MK_ERR_NO_SCHEDULE;
     if (token < 0) token = -1;
@@ -452,11 +459,49 @@ int mk_decode_step(mk_handle* h, int32_t token, int32_t pos, float* logits_dev, 
     return MK_OK;
 }
 
+int mk_decode_step_batch(mk_handle* h, const int32_t* tokens, const int32_t* pos, float* logits_dev,
+                         int32_t* next_host) {
+    if (!h || h->serving || !tokens || !pos) return MK_ERR_INVALID_ARG;
+    const int nb = h->p.nb;
+    if (nb == 1) {
+        int32_t nxt = 0;
+        const int rc = mk_decode_step(h, tokens[0], pos[0], logits_dev, next_host ? &nxt : nullptr);
+        if (rc == MK_OK && next_host) next_host[0] = nxt;
+        return rc;
+    }
+    for (int b = 0; b < nb; ++b)
+        if (tokens[b] >= h->cfg.vocab || pos[b] < 0 || pos[b] >= h->cfg.max_seq) return MK_ERR_INVALID_ARG;
+    if (!h->scheduled) return MK_ERR_NO_SCHEDULE;
+    h->epoch++;
+    mk::DevParams& p = h->p;
+    mk::StepArgs a;
+    for (int b = 0; b < nb; ++b) {
+        a.btok[b] = tokens[b] < 0 ? -1 : tokens[b];
+        a.bpos[b] = pos[b];
+    }
+    a.token = a.btok[0];
+    a.pos = a.bpos[0];
+    a.epoch = h->epoch;
+    a.logits = logits_dev ? logits_dev : p.logits;
+    CK(cudaEventRecord(h->ev0, h->stream));
+    CK(mk::launch_megakernel(p, a, h->n_sm, h->variant, h->stream));
+    CK(cudaEventRecord(h->ev1, h->stream));
+    if (next_host) {
+        mk::DevStatus st;
+        int rc = read_status(h, &st);
+        if (rc) return rc;
+        if (st.code != MK_OK) return st.code;
+        CK(cudaMemcpy(next_host, p.next_tok, sizeof(int32_t) * nb, cudaMemcpyDeviceToHost));
+    }
+    return MK_OK;
+}
+
 int mk_get_hidden(mk_handle* h, int layer, float* out_host) {
     if (!h || h->serving || !out_host || layer < 0 || layer > h->cfg.n_layers || !h->p.snap) return MK_ERR_INVALID_ARG;
     CK(cudaStreamSynchronize(h->stream));
-    CK(cudaMemcpy(out_host, h->p.snap + (size_t)layer * h->cfg.hidden, sizeof(float) * h->cfg.hidden,
-                  cudaMemcpyDeviceToHost));
+    const size_t H = (size_t)h->cfg.hidden, per_seq = (size_t)(h->cfg.n_layers + 1) * H;
+    CK(cudaMemcpy2D(out_host, sizeof(float) * H, h->p.snap + (size_t)layer * H, sizeof(float) * per_seq,
+                    sizeof(float) * H, (size_t)h->p.nb, cudaMemcpyDeviceToHost));
     return MK_OK;
 }
 
@@ -604,7 +649,7 @@ int serve_ended(mk_handle* h) {
 }  // namespace
 
 int mk_serve_start(mk_handle* h, float* logits_dev) {
-    if (!h || h->serving || h->opt.mode != MK_MODE_MEGAKERNEL) return MK_ERR_INVALID_ARG;
+    if (!h || h->serving || h->opt.mode != MK_MODE_MEGAKERNEL || h->p.nb > 1) return MK_ERR_INVALID_ARG;
     if (!h->scheduled) return MK_ERR_NO_SCHEDULE;
     if (!h->box_host) {
         void* ptr = nullptr;

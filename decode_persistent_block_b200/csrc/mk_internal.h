@@ -50,7 +50,7 @@ enum Word : int {
     W_SIGNAL_CTR = 7, // counter incremented once when the instruction's outputs are visible (-1: none)
     W_AUX_CTR = 8,    // ATTN: per-head-group arrival counter; LMHEAD: arrival counter
     W_AUX_INC = 9,    // its per-step increment
-    W_SEQ = 10,       // LMHEAD: slot of this instruction's partial argmax; ATTN: unused
+    W_SEQ = 10,       // LMHEAD: slot of this instruction's partial argmax; ATTN: sequence of the batch
     W_SPEC = 11,      // speculative expert prediction.  QKV: 1 = after it, this block predicts the layer's
                       //   experts (its last QKV instruction of the layer), 2 = the same and it publishes the
                       //   prediction; MOE_FFN: 1 = the block's loader streams the predicted expert's first
@@ -67,6 +67,8 @@ constexpr int kThreads = kConsumerThreads + 32;  // + one loader warp
 constexpr int kMaxGroup = 4;         // query heads per kv head
 constexpr int kMaxHeadDim = 128;
 constexpr int kMaxTopK = 2;
+constexpr int kMaxBatch = 8;         // sequences of one batched decode step
+constexpr int kMiscBytes = 1024;     // shared-memory budget of the kernel's per-block bookkeeping
 constexpr int kMaxMergeSlots = 2048;  // query heads x kv splits merged in the O-projection prologue
 constexpr int kDefaultL2HeadStart = 0;  // ring stages of an FFN / LM-head stream prefetched into L2 past the ring
 
@@ -184,6 +186,11 @@ struct DevParams {
     uint16_t* kcache;
     uint16_t* vcache;
     const float2* rope;      // [max_seq][d/2] (cos, sin)
+    // batched decode: nb sequences per step; every activation below, the logits, the snapshots and
+    // the KV caches hold nb per-sequence copies one after the other (strides in elements below)
+    int nb;
+    size_t kv_seq_stride;   // L * nkv * max_seq * d
+    int32_t* next_tok;      // [kMaxBatch] each sequence's argmax of the last step
     // activations (fp32)
     float* x;          // [H] residual stream read by the FFN (written by O-proj)
     float* x2;         // [H] residual stream after the FFN (O-proj writes it too; the FFN adds into it)
@@ -224,6 +231,10 @@ struct StepArgs {
     int serve = 0;    // 1: launch-once serving; the step fields come from the mailbox, epoch is the
                       // base (request k, counted from 1, runs epoch + k)
     int seq = 0;      // serving: number of this step's request
+    // batched decode (DevParams.nb > 1): token (< 0: the sequence's previous argmax) and position of
+    // every sequence; sequence 0 is also in token / pos
+    int btok[kMaxBatch] = {0, 0, 0, 0, 0, 0, 0, 0};
+    int bpos[kMaxBatch] = {0, 0, 0, 0, 0, 0, 0, 0};
 };
 
 }  // namespace mk

@@ -63,10 +63,18 @@ struct Misc {
     int pred_eidx[kMaxTopK];
     int is_last;
     int pad[3];
+    // batched decode: every sequence's position and token of this step (token resolved: < 0 read
+    // from the previous step's argmax)
+    int bpos[kMaxBatch];
+    int btok[kMaxBatch];
+    float bred[kMaxBatch * kConsumerWarps];  // per-sequence, per-warp argmax partials
+    int bredi[kMaxBatch * kConsumerWarps];
     // serving: the step block 0 published, as taken by this block's consumer thread 0
     int s_go, s_token, s_pos, s_seq;
     uint32_t s_epoch;
 };
+
+static_assert(sizeof(Misc) <= kMiscBytes, "per-block bookkeeping outgrew its shared-memory budget");
 
 __host__ __device__ inline size_t smem_bars_off(int ns, int sb) { return (size_t)ns * sb; }
 __host__ __device__ inline size_t smem_scratch_off(int ns, int sb) {
@@ -180,6 +188,7 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
     if (w[W_WAIT_CTR] >= 0 && w[W_WAIT_INC] <= 0) return false;
     if (op == OP_ATTN) {
         if (sub < 0 || sub >= p.nkv || e != p.kv_splits || b < 0 || b >= e) return false;
+        if (w[W_SEQ] < 0 || w[W_SEQ] >= p.nb) return false;
         return w[W_SIGNAL_CTR] >= 0;
     }
     if (op == OP_RMS_QKV && (sub < 0 || sub > 2)) return false;
@@ -187,7 +196,7 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
     if (op == OP_FFN && sub != 0) return false;
     if ((op == OP_FFN || op == OP_MOE_FFN) && (p.H > kMaxPartK || 2 * p.H > p.stage_bytes)) return false;
     if (b < 0 || b >= e || e > op_rows(p, op, sub) || e - b > kMaxRows) return false;
-    if ((e - b) * acc_sets(op, p.H, p.nq * p.d, p.F, p.topk) > kRowSlots) return false;
+    if ((e - b) * acc_sets(op, p.H, p.nq * p.d, p.F, p.topk) * p.nb > kRowSlots) return false;
     if (op == OP_LMHEAD_ARGMAX) return w[W_AUX_CTR] >= 0 && w[W_AUX_INC] > 0 && w[W_SEQ] >= 0 && w[W_SEQ] < w[W_AUX_INC];
     return w[W_SIGNAL_CTR] >= 0;
 }
@@ -269,7 +278,8 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
             pl.rps = attn_stage_rows((int)SB, p.d);
             pl.spp = (pl.rows + pl.rps - 1) / pl.rps;
             pl.n_stages = pl.main_stages = pl.spp;
-            pl.tma_row0 = (int)(((size_t)l * p.nkv + sub) * (size_t)p.max_seq + (size_t)r.jb);
+            // (batched decode: the sequence's cache follows the previous sequences' caches)
+            pl.tma_row0 = (int)((((size_t)w[W_SEQ] * p.L + l) * p.nkv + sub) * (size_t)p.max_seq + (size_t)r.jb);
             pl.src[0][0] = (const unsigned char*)(p.kcache + (size_t)pl.tma_row0 * p.d);
             pl.src[0][1] = (const unsigned char*)(p.vcache + (size_t)pl.tma_row0 * p.d);
             return;
@@ -454,7 +464,7 @@ __device__ __forceinline__ bool spec_hit(const DevParams& p, const Misc& m, int 
 // Plan instruction i for the loader; for MoE ops wait (bounded) until the
 // consumers have routed the layer, unless `block` is false.  MOE: the
 // instantiation runs MoE schedules (dense ones carry no routing code).
-template <bool MOE>
+template <bool MOE, int NB>
 __device__ bool loader_plan(const DevParams& p, const StepArgs& a, const int32_t* w, Misc& m, Plan& pl, bool block,
                             int ii) {
     if (!instr_ok(p, w)) {
@@ -473,7 +483,7 @@ __device__ bool loader_plan(const DevParams& p, const StepArgs& a, const int32_t
         make_plan(p, a.pos, w, eidx, pl);
         return true;
     }
-    make_plan(p, a.pos, w, nullptr, pl);
+    make_plan(p, NB > 1 && w[W_OP] == OP_ATTN ? m.bpos[w[W_SEQ]] : a.pos, w, nullptr, pl);
     return true;
 }
 
@@ -486,7 +496,7 @@ struct LoaderRing {
 };
 
 // One step's queue; false if a wait gave up (the block is leaving).
-template <bool PF, bool TC, bool MOE>
+template <bool PF, bool TC, bool MOE, int NB>
 __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, int n, unsigned char* ring,
                        uint64_t* full, uint64_t* empty, Misc& m, LoaderRing& lr) {
     const int NS = p.ring_stages;
@@ -537,13 +547,13 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                     }
                 }
                 if (!sok) return false;
-                if (!loader_plan<MOE>(p, a, w, m, pl, true, i)) break;
+                if (!loader_plan<MOE, NB>(p, a, w, m, pl, true, i)) break;
                 if (spec_hit(p, m, w[W_SUB])) st0 = ns;
-            } else if (!loader_plan<MOE>(p, a, w, m, pl, true, i)) {
+            } else if (!loader_plan<MOE, NB>(p, a, w, m, pl, true, i)) {
                 break;
             }
         } else {
-            if (!loader_plan<MOE>(p, a, w, m, pl, true, i)) break;
+            if (!loader_plan<MOE, NB>(p, a, w, m, pl, true, i)) break;
         }
         bool ok = true;
         unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + i) * kTraceWords : nullptr;
@@ -586,7 +596,7 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                             break;
                         }
                         Plan np;
-                        if (!loader_plan<MOE>(p, a, q + (size_t)(pf_i + 1) * W_NWORDS, m, np, false, pf_i + 1)) break;
+                        if (!loader_plan<MOE, NB>(p, a, q + (size_t)(pf_i + 1) * W_NWORDS, m, np, false, pf_i + 1)) break;
                         pf_i++;
                         pf_plan = np;
                         pf_st = 0;
@@ -652,9 +662,12 @@ __device__ __forceinline__ void load_vec(const float* __restrict__ src, int K, f
 // o_s, running max m_s in the log2 domain, sum l_s):
 //   attn = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s,
 // taken B splits per round trip with an online rescale, in split order.
+// sq: the sequence of a batched decode step.
 template <int J, int B>
-__device__ __forceinline__ void load_attn_merged(const DevParams& p, int col0, int K, float (&v)[J][8]) {
+__device__ __forceinline__ void load_attn_merged(const DevParams& p, int col0, int K, float (&v)[J][8], int sq = 0) {
     const int tid = threadIdx.x, nch = K >> 3, S = p.kv_splits, D = p.d;
+    const float* part_ml = p.part_ml + (size_t)sq * p.nq * S * 2;
+    const float* part_o = p.part_o + (size_t)sq * p.nq * S * D;
 #pragma unroll
     for (int j = 0; j < J; ++j) {
         const int c = tid + kConsumerThreads * j;
@@ -664,8 +677,8 @@ __device__ __forceinline__ void load_attn_merged(const DevParams& p, int col0, i
             continue;
         }
         const int col = col0 + 8 * c, h = col / D, dc = col - h * D;
-        const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)h * S;
-        const float4* po = reinterpret_cast<const float4*>(p.part_o + (size_t)h * S * D + dc);
+        const float2* ml = reinterpret_cast<const float2*>(part_ml) + (size_t)h * S;
+        const float4* po = reinterpret_cast<const float4*>(part_o + (size_t)h * S * D + dc);
         const int D4 = D >> 2;
         float M = -CUDART_INF_F, den = 0.f, acc[8];
 #pragma unroll
@@ -1392,6 +1405,547 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
 }
 
 // ---------------------------------------------------------------------------
+// consumers: batched decode (NB > 1 sequences per step, nb of them in use)
+// ---------------------------------------------------------------------------
+// RG rows [rg, rg + RG) of a stage against the sequences' input vectors: the
+// rows' weights are loaded and widened to fp32 once, then every sequence's dot
+// products reuse them; each sequence's row sums are reduced across the warp
+// and stored in that sequence's accumulator set (A + q * aset, one slot per
+// row and warp, added in warp order by the epilogue).  Rows at or past nr are
+// predicated off.
+template <int J, int RG, int NB>
+__device__ __forceinline__ void rows_block_b(const uint4* __restrict__ Ws, int row16, int rg, int nr,
+                                             const bool (&jv)[J], const float (&v)[NB][J][8], float* A, int aset,
+                                             int nb, int lane) {
+    const int tid = threadIdx.x;
+    float wf[RG][J][8];
+#pragma unroll
+    for (int r = 0; r < RG; ++r)
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+            unpack8((jv[j] && rg + r < nr) ? Ws[(rg + r) * row16 + tid + kConsumerThreads * j]
+                                           : make_uint4(0u, 0u, 0u, 0u),
+                    wf[r][j]);
+    const int row = rg + reduce_rows_lane_row<RG>(lane);
+    const bool writer = reduce_rows_writer<RG>(lane) && row < nr;
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        if (q >= nb) break;
+        float part[RG];
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < J; ++j)
+#pragma unroll
+                for (int k = 0; k < 8; k += 2) {
+                    a0 = fmaf(wf[r][j][k], v[q][j][k], a0);
+                    a1 = fmaf(wf[r][j][k + 1], v[q][j][k + 1], a1);
+                }
+            part[r] = a0 + a1;
+        }
+        const float s_row = reduce_rows<RG>(part, lane);
+        if (writer) A[(size_t)q * aset + row * kConsumerWarps + (tid >> 5)] = s_row;
+    }
+}
+
+template <int J, int RG, int NB>
+__device__ __forceinline__ void stage_rows_b(const uint4* __restrict__ Ws, int row16, int nr, int nch,
+                                             const float (&v)[NB][J][8], float* A, int aset, int nb, int lane) {
+    bool jv[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) jv[j] = (int)threadIdx.x + kConsumerThreads * j < nch;
+    for (int rg = 0; rg < nr; rg += RG) rows_block_b<J, RG, NB>(Ws, row16, rg, nr, jv, v, A, aset, nb, lane);
+}
+
+// Row sum r of accumulator set k (one per sequence and span): the 8 warps'
+// partial sums in fixed order.
+__device__ __forceinline__ float acc_row(const float* part_sums, int aset, int k, int r) {
+    const float4* ps = reinterpret_cast<const float4*>(part_sums + (size_t)k * aset + (size_t)r * kConsumerWarps);
+    const float4 x0 = ps[0], x1 = ps[1];
+    return ((x0.x + x0.y) + (x0.z + x0.w)) + ((x1.x + x1.y) + (x1.z + x1.w));
+}
+
+// v[q] = rmsnorm(x_q) * w for the nb sequences of a batched step (x_q fp32 at
+// x32 + q * H, or the bf16 embedding row of the sequence's token when
+// from_embed): every sequence's slice and the norm weights are loaded before
+// any is used, and the sequences' sums of squares share one block reduction.
+// snap (optional): sequence q's un-normalised input is stored at snap + q * snap_stride.
+template <int J, int NB>
+__device__ void load_rms_b(const DevParams& p, Misc& m, const float* x32, bool from_embed, const uint16_t* nw,
+                           float (&v)[NB][J][8], float* snap = nullptr, size_t snap_stride = 0) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, K = p.H, nch = K >> 3, nb = p.nb;
+    uint4 wraw[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int c = tid + kConsumerThreads * j;
+        wraw[j] = c < nch ? __ldg(reinterpret_cast<const uint4*>(nw) + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int q = 0; q < NB; ++q)
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int c = tid + kConsumerThreads * j;
+            if (q < nb && c < nch) {
+                if (from_embed) {
+                    unpack8(__ldg(reinterpret_cast<const uint4*>(p.embed + (size_t)m.btok[q] * K) + c), v[q][j]);
+                } else {
+                    const float4* src = reinterpret_cast<const float4*>(x32 + (size_t)q * K);
+                    const float4 a0 = __ldcg(src + 2 * c), a1 = __ldcg(src + 2 * c + 1);
+                    v[q][j][0] = a0.x; v[q][j][1] = a0.y; v[q][j][2] = a0.z; v[q][j][3] = a0.w;
+                    v[q][j][4] = a1.x; v[q][j][5] = a1.y; v[q][j][6] = a1.z; v[q][j][7] = a1.w;
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[q][j][k] = 0.f;
+            }
+        }
+    if (snap) {
+#pragma unroll
+        for (int q = 0; q < NB; ++q)
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int c = tid + kConsumerThreads * j;
+                if (q < nb && c < nch) {
+                    float4* dst = reinterpret_cast<float4*>(snap + (size_t)q * snap_stride);
+                    dst[2 * c] = make_float4(v[q][j][0], v[q][j][1], v[q][j][2], v[q][j][3]);
+                    dst[2 * c + 1] = make_float4(v[q][j][4], v[q][j][5], v[q][j][6], v[q][j][7]);
+                }
+            }
+    }
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) ss = fmaf(v[q][j][k], v[q][j][k], ss);
+        ss = warp_sum(ss);
+        if (lane == 0) m.bred[q * kConsumerWarps + warp] = ss;
+    }
+    cbar();
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) tot += m.bred[q * kConsumerWarps + w];
+        const float rs = 1.0f / sqrtf(tot / (float)K + p.eps);
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            float wf[8];
+            unpack8(wraw[j], wf);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[q][j][k] = v[q][j][k] * rs * wf[k];
+        }
+    }
+    cbar();  // m.bred free again
+}
+
+// The O-projection's input for the nb sequences of a batched step: the
+// attention output of every query head, merged from its kv splits as in
+// load_attn_merged, with the loads of QG sequences x SG splits issued together
+// per round trip.
+template <int J, int NB>
+__device__ void load_attn_merged_b(const DevParams& p, int K, float (&v)[NB][J][8]) {
+    constexpr int QG = NB < 4 ? NB : 4;  // sequences per round
+    constexpr int SG = 8 / QG;           // splits per round
+    const int tid = threadIdx.x, nch = K >> 3, S = p.kv_splits, D = p.d, D4 = D >> 2, nb = p.nb;
+    const size_t seq_ml = (size_t)p.nq * S * 2, seq_o = (size_t)p.nq * S * D;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+        const int c = tid + kConsumerThreads * j;
+        const int col = 8 * c, h = col / D, dc = col - h * D;
+#pragma unroll
+        for (int q0 = 0; q0 < NB; q0 += QG) {
+            float M[QG], den[QG], acc[QG][8];
+#pragma unroll
+            for (int g = 0; g < QG; ++g) {
+                M[g] = -CUDART_INF_F;
+                den[g] = 0.f;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) acc[g][k] = 0.f;
+            }
+            const bool live = c < nch && q0 < nb;
+            for (int s0 = 0; live && s0 < S; s0 += SG) {
+                float2 t[QG][SG];
+                float4 o0[QG][SG], o1[QG][SG];
+#pragma unroll
+                for (int g = 0; g < QG; ++g)
+#pragma unroll
+                    for (int k = 0; k < SG; ++k) {
+                        if (q0 + g < nb && s0 + k < S) {
+                            const float2* ml = reinterpret_cast<const float2*>(p.part_ml + (q0 + g) * seq_ml) +
+                                               (size_t)h * S + s0 + k;
+                            const float4* po = reinterpret_cast<const float4*>(
+                                p.part_o + (q0 + g) * seq_o + ((size_t)h * S + s0 + k) * D + dc);
+                            t[g][k] = __ldcg(ml);
+                            o0[g][k] = __ldcg(po);
+                            o1[g][k] = __ldcg(po + 1);
+                        } else {
+                            t[g][k] = make_float2(-CUDART_INF_F, 0.f);
+                            o0[g][k] = o1[g][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                    }
+#pragma unroll
+                for (int g = 0; g < QG; ++g) {
+                    float bm = M[g];
+#pragma unroll
+                    for (int k = 0; k < SG; ++k) bm = fmaxf(bm, t[g][k].x);
+                    if (bm == -CUDART_INF_F) continue;  // no position in these splits yet
+                    const float r = exp2f(M[g] - bm);
+                    den[g] *= r;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) acc[g][k] *= r;
+#pragma unroll
+                    for (int k = 0; k < SG; ++k) {
+                        const float f = exp2f(t[g][k].x - bm);
+                        den[g] = fmaf(f, t[g][k].y, den[g]);
+                        acc[g][0] = fmaf(f, o0[g][k].x, acc[g][0]);
+                        acc[g][1] = fmaf(f, o0[g][k].y, acc[g][1]);
+                        acc[g][2] = fmaf(f, o0[g][k].z, acc[g][2]);
+                        acc[g][3] = fmaf(f, o0[g][k].w, acc[g][3]);
+                        acc[g][4] = fmaf(f, o1[g][k].x, acc[g][4]);
+                        acc[g][5] = fmaf(f, o1[g][k].y, acc[g][5]);
+                        acc[g][6] = fmaf(f, o1[g][k].z, acc[g][6]);
+                        acc[g][7] = fmaf(f, o1[g][k].w, acc[g][7]);
+                    }
+                    M[g] = bm;
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < QG; ++g) {
+                const bool ok = live && q0 + g < nb;
+                const float inv = ok ? 1.0f / den[g] : 0.f;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[q0 + g][j][k] = ok ? acc[g][k] * inv : 0.f;
+            }
+        }
+    }
+}
+
+// Batched QKV, O-projection and LM head (one column part, one span): each
+// stage of weights is applied to the nb sequences' input vectors before its
+// slot is freed, and the epilogue writes every sequence's outputs.
+template <int J, int NB>
+__device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
+                             uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
+    constexpr int RG = J == 1 ? 4 : 2;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nb = p.nb;
+    const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], rows = w[W_END] - b;
+    const uint32_t SB = (uint32_t)p.stage_bytes;
+    const size_t H = (size_t)p.H;
+    float* part_sums = scratch;  // [sequence][row][8 warps]
+    const int aset = rows * kConsumerWarps;
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
+    Plan pl;
+    make_plan(p, a.pos, w, nullptr, pl);
+    if (tid == 0 && w[W_WAIT_CTR] >= 0 &&
+        !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op))
+        vstore(&m.abort_flag, 1);
+    if (tr && tid == 0) tr[T_DEP] = globaltimer_ns();
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+
+    // input vectors of the sequences
+    float v[NB][J][8];
+    const uint16_t* const* wt = p.wt + (size_t)(l < p.L ? l : 0) * wt_stride(p.E);
+    const int K = op == OP_OPROJ_RES ? p.nq * p.d : p.H;
+    const size_t snap_stride = (size_t)(p.L + 1) * H;
+    if (op == OP_RMS_QKV)
+        load_rms_b<J, NB>(p, m, p.x2, l == 0, wt[WT_ATTN_NORM], v,
+                          (p.snap && l > 0 && sub == 0 && b == 0) ? p.snap + (size_t)l * H : nullptr, snap_stride);
+    else if (op == OP_LMHEAD_ARGMAX)
+        load_rms_b<J, NB>(p, m, p.x2, p.L == 0, p.final_norm, v,
+                          (p.snap && w[W_SEQ] == 0) ? p.snap + (size_t)p.L * H : nullptr, snap_stride);
+    else
+        load_attn_merged_b<J, NB>(p, K, v);
+    if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
+
+    // stages
+    const int nch = K >> 3;
+    for (int sst = 0; sst < pl.spp; ++sst) {
+        const int r0 = sst * pl.rps;
+        const int nr = (rows - r0) < pl.rps ? (rows - r0) : pl.rps;
+        if (warp_wait_full(&full[slot], phase, p, m, ii, op)) {
+            if (tid == 0) {
+                if (tr && sst == 0) tr[T_FIRST] = globaltimer_ns();
+                stage_stamp(tr, T_SREADY, sst);
+            }
+            const uint4* Ws = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
+            stage_rows_b<J, RG, NB>(Ws, (int)(pl.row_bytes >> 4), nr, nch, v,
+                                    part_sums + (size_t)r0 * kConsumerWarps, aset, nb, lane);
+            __syncwarp();
+            if (tid == 0) stage_stamp(tr, T_SDONE, sst);
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        } else if (tid == 0) {
+            vstore(&m.abort_flag, 1);
+        }
+        if (++slot == p.ring_stages) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+    if (tr && tid == 0) tr[T_MAIN] = globaltimer_ns();
+
+    // epilogue
+    if (op == OP_RMS_QKV) {
+        const int qkvn = (p.nq + 2 * p.nkv) * p.d;
+        const int off = sub == 0 ? 0 : (sub == 1 ? p.nq * p.d : (p.nq + p.nkv) * p.d);
+        for (int q = 0; q < nb; ++q)
+            for (int r = tid; r < rows; r += kConsumerThreads)
+                p.qkv[(size_t)q * qkvn + off + b + r] = acc_row(part_sums, aset, q, r);
+    } else if (op == OP_OPROJ_RES) {
+        for (int q = 0; q < nb; ++q)
+            for (int r = tid; r < rows; r += kConsumerThreads) {
+                const size_t i = q * H + b + r;
+                float base;
+                if (l == 0) {
+                    const uint16_t e = p.embed[(size_t)m.btok[q] * H + b + r];
+                    base = __uint_as_float((uint32_t)e << 16);
+                    if (p.snap) p.snap[(size_t)q * (p.L + 1) * H + b + r] = base;
+                } else {
+                    base = __ldcg(p.x2 + i);
+                }
+                const float nx = base + acc_row(part_sums, aset, q, r);
+                p.x[i] = nx;
+                p.x2[i] = nx;
+            }
+    } else {  // LM head: logits, then each sequence's argmax over this instruction's rows
+        float bv[NB];
+        int bi[NB];
+#pragma unroll
+        for (int q = 0; q < NB; ++q) {
+            bv[q] = -CUDART_INF_F;
+            bi[q] = 0x7FFFFFFF;
+            if (q >= nb) continue;
+            for (int r = tid; r < rows; r += kConsumerThreads) {
+                const float val = acc_row(part_sums, aset, q, r);
+                a.logits[(size_t)q * p.V + b + r] = val;
+                if (val > bv[q] || (val == bv[q] && b + r < bi[q])) {
+                    bv[q] = val;
+                    bi[q] = b + r;
+                }
+            }
+            warp_argmax(bv[q], bi[q]);
+            if (lane == 0) {
+                m.bred[q * kConsumerWarps + warp] = bv[q];
+                m.bredi[q * kConsumerWarps + warp] = bi[q];
+            }
+        }
+        cbar();
+        if (tid == 0) {
+            for (int q = 0; q < nb; ++q) {
+                float cv = m.bred[q * kConsumerWarps];
+                int ci = m.bredi[q * kConsumerWarps];
+                for (int k = 1; k < kConsumerWarps; ++k) {
+                    const float ov = m.bred[q * kConsumerWarps + k];
+                    const int oi = m.bredi[q * kConsumerWarps + k];
+                    if (ov > cv || (ov == cv && oi < ci)) {
+                        cv = ov;
+                        ci = oi;
+                    }
+                }
+                const size_t slot_q = ((size_t)w[W_SEQ] * nb + q) * 2;
+                p.lm_part[slot_q] = cv;
+                p.lm_part[slot_q + 1] = __int_as_float(ci);
+            }
+            const uint32_t old = arrive_release(p.counters + w[W_AUX_CTR]);
+            m.is_last = (old + 1u == a.epoch * (uint32_t)w[W_AUX_INC]) ? 1 : 0;
+        }
+        cbar();
+        if (m.is_last) {  // the last LM-head instruction to finish picks every sequence's token
+            fence_acquire();
+            const int n_lm = w[W_AUX_INC];
+            for (int q = 0; q < nb; ++q) {
+                float cv = -CUDART_INF_F;
+                int ci = 0x7FFFFFFF;
+                for (int k = tid; k < n_lm; k += kConsumerThreads) {
+                    const float val = __ldcg(p.lm_part + ((size_t)k * nb + q) * 2);
+                    const int idx = __float_as_int(__ldcg(p.lm_part + ((size_t)k * nb + q) * 2 + 1));
+                    if (val > cv || (val == cv && idx < ci)) {
+                        cv = val;
+                        ci = idx;
+                    }
+                }
+                warp_argmax(cv, ci);
+                if (lane == 0) {
+                    m.bred[q * kConsumerWarps + warp] = cv;
+                    m.bredi[q * kConsumerWarps + warp] = ci;
+                }
+            }
+            cbar();
+            if (tid == 0) {
+                for (int q = 0; q < nb; ++q) {
+                    float cv = m.bred[q * kConsumerWarps];
+                    int ci = m.bredi[q * kConsumerWarps];
+                    for (int k = 1; k < kConsumerWarps; ++k) {
+                        const float ov = m.bred[q * kConsumerWarps + k];
+                        const int oi = m.bredi[q * kConsumerWarps + k];
+                        if (ov > cv || (ov == cv && oi < ci)) {
+                            cv = ov;
+                            ci = oi;
+                        }
+                    }
+                    p.next_tok[q] = ci;
+                    if (q == 0) p.status->next_token = ci;
+                }
+            }
+        }
+    }
+    cbar();
+    if (tid == 0 && w[W_SIGNAL_CTR] >= 0 && op != OP_LMHEAD_ARGMAX) signal_release(p.counters + w[W_SIGNAL_CTR]);
+    return true;
+}
+
+// Batched fused FFN slice (OP_FFN): rows [b, e) of the up/gate projections for
+// every sequence (each stage applied to the nb input vectors), h per sequence
+// and row, then the same rows of the transposed down-projection: each weight
+// chunk is widened once and accumulated into every sequence's column chunks,
+// which are added into the sequences' residuals with float4 atomics.
+template <int J, int NB>
+__device__ bool ffn_instr_b(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
+                            uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
+    constexpr int RG = J == 1 ? 4 : 2;
+    const int tid = threadIdx.x, lane = tid & 31, nb = p.nb;
+    const int op = w[W_OP], l = w[W_LAYER], b = w[W_BEGIN], rows = w[W_END] - b;
+    const uint32_t SB = (uint32_t)p.stage_bytes;
+    const size_t H = (size_t)p.H;
+    float* part_sums = scratch;  // [span][sequence < nb][row][8 warps]
+    const int aset = rows * kConsumerWarps;
+    unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
+    Plan pl;
+    make_plan(p, a.pos, w, nullptr, pl);
+    if (tid == 0 && !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op))
+        vstore(&m.abort_flag, 1);
+    if (tr && tid == 0) tr[T_DEP] = globaltimer_ns();
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+
+    float v[NB][J][8];
+    const uint16_t* const* wt = p.wt + (size_t)l * wt_stride(p.E);
+    load_rms_b<J, NB>(p, m, p.x, false, wt[WT_FFN_NORM], v);
+    if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
+    const int nch = p.H >> 3;
+
+    // up/gate rows (gate span, then up span, of each stage)
+    for (int sst = 0; sst < pl.spp; ++sst) {
+        const int r0 = sst * pl.rps;
+        const int nr = (rows - r0) < pl.rps ? (rows - r0) : pl.rps;
+        if (warp_wait_full(&full[slot], phase, p, m, ii, op)) {
+            if (tid == 0) {
+                if (tr && sst == 0) tr[T_FIRST] = globaltimer_ns();
+                stage_stamp(tr, T_SREADY, sst);
+            }
+            const unsigned char* stage = ring + (size_t)slot * SB;
+            for (int s = 0; s < 2; ++s) {
+                const uint4* Ws = reinterpret_cast<const uint4*>(stage + (size_t)s * pl.rps * pl.row_bytes);
+                stage_rows_b<J, RG, NB>(Ws, (int)(pl.row_bytes >> 4), nr, nch, v,
+                                        part_sums + ((size_t)s * nb * rows + r0) * kConsumerWarps, aset, nb, lane);
+            }
+            __syncwarp();
+            if (tid == 0) stage_stamp(tr, T_SDONE, sst);
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        } else if (tid == 0) {
+            vstore(&m.abort_flag, 1);
+        }
+        if (++slot == p.ring_stages) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+    if (tr && tid == 0) tr[T_MAIN] = globaltimer_ns();
+
+    // h[q][r] = silu(g) * u, kept at the start of the scratch (after every thread read its sums)
+    constexpr int HR = 2;  // rows per thread (rows <= 512)
+    float hv[NB][HR];
+#pragma unroll
+    for (int q = 0; q < NB; ++q)
+#pragma unroll
+        for (int k = 0; k < HR; ++k) {
+            const int r = tid + kConsumerThreads * k;
+            hv[q][k] = 0.f;
+            if (q < nb && r < rows) {
+                const float g = acc_row(part_sums, aset, q, r);
+                const float u = acc_row(part_sums, aset, nb + q, r);
+                hv[q][k] = g / (1.0f + expf(-g)) * u;
+            }
+        }
+    cbar();
+#pragma unroll
+    for (int q = 0; q < NB; ++q)
+#pragma unroll
+        for (int k = 0; k < HR; ++k) {
+            const int r = tid + kConsumerThreads * k;
+            if (q < nb && r < rows) scratch[(size_t)r * NB + q] = hv[q][k];
+        }
+    cbar();
+
+    // transposed down-projection rows: this thread's column chunks of Wd[:, rows] h_q, every q
+    float y[NB][J][8];
+    bool jv[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) jv[j] = tid + kConsumerThreads * j < nch;
+#pragma unroll
+    for (int q = 0; q < NB; ++q)
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) y[q][j][k] = 0.f;
+    for (int tst = 0; tst < pl.tail_spp; ++tst) {
+        const int r0 = tst * pl.tail_rps;
+        const int nr = (rows - r0) < pl.tail_rps ? (rows - r0) : pl.tail_rps;
+        if (warp_wait_full(&full[slot], phase, p, m, ii, op)) {
+            if (tid == 0) stage_stamp(tr, T_SREADY, pl.spp + tst);
+            const uint4* Ws = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
+            for (int r = 0; r < nr; ++r) {
+                float f[J][8];
+#pragma unroll
+                for (int j = 0; j < J; ++j)
+                    unpack8(jv[j] ? Ws[r * nch + tid + kConsumerThreads * j] : make_uint4(0u, 0u, 0u, 0u), f[j]);
+                const float* hr = scratch + (size_t)(r0 + r) * NB;
+#pragma unroll
+                for (int q = 0; q < NB; ++q) {
+                    if (q >= nb) break;
+                    const float hk = hr[q];
+#pragma unroll
+                    for (int j = 0; j < J; ++j)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) y[q][j][k] = fmaf(f[j][k], hk, y[q][j][k]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        } else if (tid == 0) {
+            vstore(&m.abort_flag, 1);
+        }
+        if (++slot == p.ring_stages) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    cbar();
+    if (vload(&m.abort_flag)) return false;
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        if (q >= nb) break;
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            if (!jv[j]) continue;
+            float4* dst = reinterpret_cast<float4*>(p.x2 + q * H) + 2 * (tid + kConsumerThreads * j);
+            atomicAdd(dst, make_float4(y[q][j][0], y[q][j][1], y[q][j][2], y[q][j][3]));
+            atomicAdd(dst + 1, make_float4(y[q][j][4], y[q][j][5], y[q][j][6], y[q][j][7]));
+        }
+    }
+    cbar();
+    if (tid == 0) signal_release(p.counters + w[W_SIGNAL_CTR]);
+    return true;
+}
+
+// ---------------------------------------------------------------------------
 // consumers: attention (RoPE + append + one split of GQA decode attention)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void ml_combine(float& m, float& l, float* o, float m2, float l2, const float* o2) {
@@ -1413,6 +1967,7 @@ __device__ __forceinline__ void ml_combine(float& m, float& l, float* o, float m
 // at most 2 of the kv head's query heads and streams every K/V row of the stage
 // for them), which keeps the per-thread q and output accumulators to 2 x 8 +
 // 2 x 8 registers.  The stage holds K then V rows, contiguous (bulk copies).
+template <int NB>
 __device__ bool attn_cc(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                            uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
     const int D = p.d;                                  // head_dim, 64 or 128
@@ -1427,7 +1982,15 @@ __device__ bool attn_cc(const DevParams& p, const StepArgs& a, const int32_t* w,
     const int set = warp / SET_WARPS;
     const int stid = tid - set * SET_THREADS;
     const int h0 = set * GW;                            // first query head (within the group) of this set
-    const int l = w[W_LAYER], g = w[W_SUB], c = w[W_BEGIN], S = w[W_END], pos = a.pos;
+    const int l = w[W_LAYER], g = w[W_SUB], c = w[W_BEGIN], S = w[W_END];
+    // batched decode: the instruction's sequence (its position, projections, cache and partials)
+    const int sq = NB > 1 ? w[W_SEQ] : 0;
+    const int pos = NB > 1 ? m.bpos[sq] : a.pos;
+    const float* qkv_s = p.qkv + (size_t)sq * (p.nq + 2 * p.nkv) * p.d;
+    uint16_t* kc_s = p.kcache + (size_t)sq * p.kv_seq_stride;
+    uint16_t* vc_s = p.vcache + (size_t)sq * p.kv_seq_stride;
+    float* part_o_s = p.part_o + (size_t)sq * p.nq * p.kv_splits * p.d;
+    float* part_ml_s = p.part_ml + (size_t)sq * p.nq * p.kv_splits * 2;
     const uint32_t SB = (uint32_t)p.stage_bytes;
     const AttnRange rg = attn_range(pos, c, S);
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
@@ -1450,13 +2013,13 @@ __device__ bool attn_cc(const DevParams& p, const StepArgs& a, const int32_t* w,
     const bool first_half = col0 < D / 2;
     const float qscale = 1.4426950408889634f / sqrtf((float)D);
     const float4* rp4 = reinterpret_cast<const float4*>(p.rope + (size_t)pos * (D / 2) + (col0 & (D / 2 - 1)));
-    const float* ks = p.qkv + (size_t)p.nq * D + (size_t)g * D;
-    const float* vs = p.qkv + (size_t)(p.nq + p.nkv) * D + (size_t)g * D;
+    const float* ks = qkv_s + (size_t)p.nq * D + (size_t)g * D;
+    const float* vs = qkv_s + (size_t)(p.nq + p.nkv) * D + (size_t)g * D;
     float4 qx[GW][2], qy[GW][2], rc[4], kx[2], ky[2], vx[2];
 #pragma unroll
     for (int hh = 0; hh < GW; ++hh) {
         const int h = h0 + hh < G ? h0 + hh : G - 1;  // spare head slots compute a copy that is never stored
-        const float4* src = reinterpret_cast<const float4*>(p.qkv + (size_t)(g * G + h) * D);
+        const float4* src = reinterpret_cast<const float4*>(qkv_s + (size_t)(g * G + h) * D);
         qx[hh][0] = __ldcg(src + col0 / 4);
         qx[hh][1] = __ldcg(src + col0 / 4 + 1);
         qy[hh][0] = __ldcg(src + pcol / 4);
@@ -1511,8 +2074,8 @@ __device__ bool attn_cc(const DevParams& p, const StepArgs& a, const int32_t* w,
             uint4 ku, vu;
             ku.x = kb[0] | (kb[1] << 16); ku.y = kb[2] | (kb[3] << 16); ku.z = kb[4] | (kb[5] << 16); ku.w = kb[6] | (kb[7] << 16);
             vu.x = vb[0] | (vb[1] << 16); vu.y = vb[2] | (vb[3] << 16); vu.z = vb[4] | (vb[5] << 16); vu.w = vb[6] | (vb[7] << 16);
-            *reinterpret_cast<uint4*>(p.kcache + off) = ku;
-            *reinterpret_cast<uint4*>(p.vcache + off) = vu;
+            *reinterpret_cast<uint4*>(kc_s + off) = ku;
+            *reinterpret_cast<uint4*>(vc_s + off) = vu;
         }
     }
 
@@ -1685,10 +2248,10 @@ __device__ bool attn_cc(const DevParams& p, const StepArgs& a, const int32_t* w,
             }
         }
         const size_t part = (size_t)(g * G + h) * S + c;
-        p.part_o[part * D + col] = O;
+        part_o_s[part * D + col] = O;
         if (col == 0) {
-            p.part_ml[part * 2] = M;
-            p.part_ml[part * 2 + 1] = Ls;
+            part_ml_s[part * 2] = M;
+            part_ml_s[part * 2 + 1] = Ls;
         }
     }
     cbar();
@@ -1699,7 +2262,7 @@ __device__ bool attn_cc(const DevParams& p, const StepArgs& a, const int32_t* w,
 // Tensor-core split attention (the head_dim-64 kernel).  DH: head_dim fixed at
 // compile time.  The stage holds K then V rows in 128-byte-swizzled tensor-map
 // boxes.
-template <int DH>
+template <int DH, int NB>
 __device__ bool attn_tc(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                            uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
     constexpr int DMAX = DH > 0 ? DH : kMaxHeadDim;
@@ -1713,7 +2276,15 @@ __device__ bool attn_tc(const DevParams& p, const StepArgs& a, const int32_t* w,
     const int set = warp / SET_WARPS;
     const int stid = tid - set * SET_THREADS;
     const int h0 = set * GW;                            // first query head (within the group) of this set
-    const int l = w[W_LAYER], g = w[W_SUB], c = w[W_BEGIN], S = w[W_END], pos = a.pos;
+    const int l = w[W_LAYER], g = w[W_SUB], c = w[W_BEGIN], S = w[W_END];
+    // batched decode: the instruction's sequence (its position, projections, cache and partials)
+    const int sq = NB > 1 ? w[W_SEQ] : 0;
+    const int pos = NB > 1 ? m.bpos[sq] : a.pos;
+    const float* qkv_s = p.qkv + (size_t)sq * (p.nq + 2 * p.nkv) * p.d;
+    uint16_t* kc_s = p.kcache + (size_t)sq * p.kv_seq_stride;
+    uint16_t* vc_s = p.vcache + (size_t)sq * p.kv_seq_stride;
+    float* part_o_s = p.part_o + (size_t)sq * p.nq * p.kv_splits * p.d;
+    float* part_ml_s = p.part_ml + (size_t)sq * p.nq * p.kv_splits * 2;
     const uint32_t SB = (uint32_t)p.stage_bytes;
     const AttnRange rg = attn_range(pos, c, S);
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
@@ -1736,13 +2307,13 @@ __device__ bool attn_tc(const DevParams& p, const StepArgs& a, const int32_t* w,
     const bool first_half = col0 < D / 2;
     const float qscale = 1.4426950408889634f / sqrtf((float)D);
     const float4* rp4 = reinterpret_cast<const float4*>(p.rope + (size_t)pos * (D / 2) + (col0 & (D / 2 - 1)));
-    const float* ks = p.qkv + (size_t)p.nq * D + (size_t)g * D;
-    const float* vs = p.qkv + (size_t)(p.nq + p.nkv) * D + (size_t)g * D;
+    const float* ks = qkv_s + (size_t)p.nq * D + (size_t)g * D;
+    const float* vs = qkv_s + (size_t)(p.nq + p.nkv) * D + (size_t)g * D;
     float4 qx[GW][2], qy[GW][2], rc[4], kx[2], ky[2], vx[2];
 #pragma unroll
     for (int hh = 0; hh < GW; ++hh) {
         const int h = h0 + hh < G ? h0 + hh : G - 1;  // spare head slots compute a copy that is never stored
-        const float4* src = reinterpret_cast<const float4*>(p.qkv + (size_t)(g * G + h) * D);
+        const float4* src = reinterpret_cast<const float4*>(qkv_s + (size_t)(g * G + h) * D);
         qx[hh][0] = __ldcg(src + col0 / 4);
         qx[hh][1] = __ldcg(src + col0 / 4 + 1);
         qy[hh][0] = __ldcg(src + pcol / 4);
@@ -1797,8 +2368,8 @@ __device__ bool attn_tc(const DevParams& p, const StepArgs& a, const int32_t* w,
             uint4 ku, vu;
             ku.x = kb[0] | (kb[1] << 16); ku.y = kb[2] | (kb[3] << 16); ku.z = kb[4] | (kb[5] << 16); ku.w = kb[6] | (kb[7] << 16);
             vu.x = vb[0] | (vb[1] << 16); vu.y = vb[2] | (vb[3] << 16); vu.z = vb[4] | (vb[5] << 16); vu.w = vb[6] | (vb[7] << 16);
-            *reinterpret_cast<uint4*>(p.kcache + off) = ku;
-            *reinterpret_cast<uint4*>(p.vcache + off) = vu;
+            *reinterpret_cast<uint4*>(kc_s + off) = ku;
+            *reinterpret_cast<uint4*>(vc_s + off) = vu;
         }
     }
 
@@ -1998,10 +2569,10 @@ __device__ bool attn_tc(const DevParams& p, const StepArgs& a, const int32_t* w,
             }
         }
         const size_t part = (size_t)(g * G + h) * S + c;
-        p.part_o[part * D + col] = O;
+        part_o_s[part * D + col] = O;
         if (col == 0) {
-            p.part_ml[part * 2] = M;
-            p.part_ml[part * 2 + 1] = Ls;
+            part_ml_s[part * 2] = M;
+            part_ml_s[part * 2 + 1] = Ls;
         }
     }
     cbar();
@@ -2175,7 +2746,8 @@ __device__ void serve_respond(const DevParams& p, const StepArgs& a, int next_to
 // exist with and without it, so the default ones carry no prefetch code.  The
 // consumers' per-instruction prefetch (prefetch_ahead) is in the general one only.
 // MOE: MoE routing is compiled in (dense models run instantiations without it).
-template <int JF, int DH, bool PF, bool MOE>
+// NB > 1: batched decode of up to NB sequences per step (p.nb of them).
+template <int JF, int DH, bool PF, bool MOE, int NB = 1>
 __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant__ DevParams p, const StepArgs a) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int NS = p.ring_stages, SB = p.stage_bytes;
@@ -2195,6 +2767,13 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         m.is_last = 0;
         m.abort_flag = ld_relaxed_s32(&p.status->stop) ? 1 : 0;
         if (m.abort_flag && atomicCAS(&p.status->code, 0, MK_ERR_STOPPED) == 0) p.status->sm = blockIdx.x;
+        if constexpr (NB > 1) {  // every sequence's position and token (< 0: its previous argmax)
+#pragma unroll
+            for (int q = 0; q < NB; ++q) {
+                m.bpos[q] = a.bpos[q];
+                m.btok[q] = q < p.nb ? (a.btok[q] >= 0 ? a.btok[q] : __ldcg(p.next_tok + q)) : 0;
+            }
+        }
         fence_mbar_init();
     }
     __syncthreads();
@@ -2208,7 +2787,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             for (uint32_t k = 0;; ++k) {
                 StepArgs sa = a;
                 if (a.serve && !serve_take(p, m, k, a, sa)) break;
-                if (!loader<PF, DH == 64, MOE>(p, sa, q, n, smem, full, empty, m, lr) || !a.serve) break;
+                if (!loader<PF, DH == 64, MOE, NB>(p, sa, q, n, smem, full, empty, m, lr) || !a.serve) break;
             }
             loader_drain(p, full, lr);
         }
@@ -2237,7 +2816,11 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
             sa.seq = m.s_seq;
             sa.epoch = m.s_epoch;
         }
-        const int token = sa.token >= 0 ? sa.token : __ldcg(&p.status->next_token);
+        int token = sa.token >= 0 ? sa.token : __ldcg(&p.status->next_token);
+        if constexpr (NB > 1) {  // any sequence's token out of range fails the step
+            for (int q = 0; q < p.nb; ++q)
+                if (m.btok[q] < 0 || m.btok[q] >= p.V) token = -1;
+        }
         bool ok = true;
         for (int i = 0; i < n; ++i) {
             const int32_t* w = q + (size_t)i * W_NWORDS;
@@ -2252,9 +2835,21 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
                 ok = false;
             } else if (w[W_OP] == OP_ATTN) {
                 if constexpr (DH == 64)
-                    ok = attn_tc<64>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
+                    ok = attn_tc<64, NB>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
                 else
-                    ok = attn_cc(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
+                    ok = attn_cc<NB>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
+            } else if constexpr (NB > 1) {
+                if (w[W_OP] == OP_FFN) {
+                    ok = ffn_instr_b<JF, NB>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
+                } else if (w[W_OP] == OP_RMS_QKV || w[W_OP] == OP_OPROJ_RES || w[W_OP] == OP_LMHEAD_ARGMAX) {
+                    ok = gemv_instr_b<JF, NB>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase);
+                } else {
+                    if (tid == 0) {
+                        record_error(p.status, MK_ERR_BAD_INSTR, blockIdx.x, i, w[W_OP], -1, 0, 0);
+                        vstore(&m.abort_flag, 1);
+                    }
+                    ok = false;
+                }
             } else {
                 ok = gemv_dispatch<JF, MOE>(p, sa, w, i, smem, full, empty, scratch, m, slot, phase, token);
             }
@@ -2277,6 +2872,11 @@ KernelFn kernel_of(int variant) {
         case 4: return megakernel<2, 128, true, false>;
         case 5: return megakernel<1, 64, false, true>;
         case 6: return megakernel<2, 128, false, true>;
+        case 7: return megakernel<1, 64, false, false, 2>;
+        case 8: return megakernel<1, 64, false, false, 4>;
+        case 9: return megakernel<1, 64, false, false, 8>;
+        case 10: return megakernel<2, 128, false, false, 2>;
+        case 11: return megakernel<2, 128, false, false, 4>;
     }
     return megakernel<0, 0, true, true>;
 }
@@ -2289,11 +2889,19 @@ int j_of(int K) {
 
 // 0: general; 1 / 2: dense, specialised for one chunk (head_dim 64) / two chunks (head_dim 128)
 // per thread; 3 / 4: the same with the loader's L2-prefetch cursor (options.l2_prefetch > 0);
-// 5 / 6: MoE, specialised (without the prefetch cursor; MoE with it runs the general kernel).
+// 5 / 6: MoE, specialised (without the prefetch cursor; MoE with it runs the general kernel);
+// 7 / 8 / 9: batched decode of up to 2 / 4 / 8 sequences, one chunk per thread (head_dim 64);
+// 10 / 11: up to 2 / 4 sequences, two chunks (head_dim 128).  -1: no kernel for the batch.
 int megakernel_variant(const DevParams& p, bool fused_ffn) {
-    if (!fused_ffn || p.prefetch_ahead > 0) return 0;
     const int jh = j_of(p.H), jo = j_of(p.nq * p.d);
     const int base = (jh == 1 && jo == 1 && p.d == 64) ? 1 : (jh == 2 && jo == 2 && p.d == 128) ? 2 : 0;
+    if (p.nb > 1) {
+        if (!fused_ffn || p.E > 0 || p.prefetch_ahead > 0 || p.l2_prefetch > 0) return -1;
+        if (base == 1) return p.nb <= 2 ? 7 : p.nb <= 4 ? 8 : p.nb <= 8 ? 9 : -1;
+        if (base == 2) return p.nb <= 2 ? 10 : p.nb <= 4 ? 11 : -1;
+        return -1;
+    }
+    if (!fused_ffn || p.prefetch_ahead > 0) return 0;
     if (base == 0) return 0;
     if (p.E > 0) return p.l2_prefetch > 0 ? 0 : base + 4;
     return p.l2_prefetch > 0 ? base + 2 : base;
@@ -2317,7 +2925,7 @@ cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, i
 cudaError_t prepare_megakernel(int ring_stages, int stage_bytes, int* max_blocks_per_sm) {
     const size_t smem = megakernel_smem_bytes(ring_stages, stage_bytes);
     *max_blocks_per_sm = 1 << 30;
-    for (int v = 0; v <= 6; ++v) {
+    for (int v = 0; v <= 11; ++v) {
         cudaError_t e = cudaFuncSetAttribute(kernel_of(v), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         int per_sm = 0;

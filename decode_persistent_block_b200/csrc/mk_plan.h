@@ -13,6 +13,7 @@ struct Planned {
     int kv_splits = 1;
     int n_lm = 0;                  // LM-head instructions (partial argmax slots)
     bool fused_ffn = true;         // one OP_FFN / OP_MOE_FFN per layer instead of up/gate + down
+    int nb = 1;                    // sequences per step (batched decode)
     std::vector<int32_t> words;    // [n_sm][max_instr][W_NWORDS]
     std::vector<int32_t> n_instr;  // [n_sm]
     std::vector<uint32_t> ctr_inc; // per-step increment of every counter
@@ -21,7 +22,9 @@ struct Planned {
 int check_config(const mk_config& c);
 int check_options(const mk_config& c, const mk_options& o);
 void fill_defaults(mk_options* o);
-int default_kv_splits(const mk_config& c, int n_sm);
+int default_kv_splits(const mk_config& c, int n_sm, int nb = 1);
+// Largest options.batch the kernels support for this shape (1: no batched decode).
+int max_batch(const mk_config& c);
 // Whether the schedule fuses each layer's FFN into one instruction per block:
 // asked for (split_ffn == 0), the up/gate rows need no column parts, and one
 // transposed down-projection row (hidden bf16 values) fits a ring stage.

@@ -123,8 +123,9 @@ void split_rows(const std::vector<Segment>& segs, int n_sm, int cap, F emit,
 //    sweep (4 to 16 splits at 1152 positions) almost exactly.
 //  - head_dim 128 (CUDA-core attention, about 5x the per-row cost): about one
 //    split per 128 positions.
-int default_kv_splits(const mk_config& c, int n_sm) {
-    const int per_sm = std::max(1, n_sm / std::max(1, c.n_kv_heads));
+int default_kv_splits(const mk_config& c, int n_sm, int nb) {
+    // at most one split per block across the batch's sequences and kv heads
+    const int per_sm = std::max(1, n_sm / std::max(1, c.n_kv_heads * std::max(1, nb)));
     const int by_merge = std::max(1, kMaxMergeSlots / std::max(1, c.n_q_heads));
     const int cap = std::min(per_sm, by_merge);
     if (c.head_dim != 64) return std::min(cap, std::max(1, (c.max_seq + 127) / 128));
@@ -172,6 +173,20 @@ void fill_defaults(mk_options* o) {
     if (o->attn_sm_ffn_permille <= 0) o->attn_sm_ffn_permille = 1000;
     if (o->spin_limit_ns == 0) o->spin_limit_ns = 2000000000ull;
     if (o->serve_idle_ns == 0) o->serve_idle_ns = 60000000000ull;
+    if (o->batch == 0) o->batch = 1;
+}
+
+// Chunks of 8 elements per consumer thread for a GEMV over k columns (per column part).
+static int chunks_per_thread(int k) {
+    const int parts = (k + 8191) / 8192;
+    return ((k / parts) / 8 + kConsumerThreads - 1) / kConsumerThreads;
+}
+
+int max_batch(const mk_config& c) {
+    const int jh = chunks_per_thread(c.hidden), jo = chunks_per_thread(c.n_q_heads * c.head_dim);
+    if (c.n_experts == 0 && jh == 1 && jo == 1 && c.head_dim == 64) return kMaxBatch;
+    if (c.n_experts == 0 && jh == 2 && jo == 2 && c.head_dim == 128) return kMaxBatch / 2;
+    return 1;
 }
 
 int check_options(const mk_config& c, const mk_options& o) {
@@ -195,8 +210,14 @@ int check_options(const mk_config& c, const mk_options& o) {
     }
     if (o.mode < MK_MODE_MEGAKERNEL || o.mode > MK_MODE_MULTI_KERNEL_GRAPH) return MK_ERR_INVALID_ARG;
     if (o.spec_experts < 0 || o.spec_experts > 2) return MK_ERR_INVALID_ARG;
+    if (o.batch < 1 || o.batch > kMaxBatch) return MK_ERR_INVALID_ARG;
+    if (o.batch > 1) {  // batched decode: the specialised dense kernels with the fused FFN only
+        if (o.batch > max_batch(c) || o.mode != MK_MODE_MEGAKERNEL || !ffn_fused(c, o) || o.spec_experts ||
+            o.general_kernel || o.l2_prefetch > 0 || o.prefetch_ahead > 0)
+            return MK_ERR_UNSUPPORTED;
+    }
     // ring + barriers + partial-sum slots + misc must fit the 227 KB per-block opt-in limit
-    if ((long long)o.ring_stages * o.stage_bytes + 16LL * o.ring_stages + 128 + 4LL * kRowSlots * 8 + 512 > 232448)
+    if ((long long)o.ring_stages * o.stage_bytes + 16LL * o.ring_stages + 128 + 4LL * kRowSlots * 8 + kMiscBytes > 232448)
         return MK_ERR_INVALID_ARG;
     return MK_OK;
 }
@@ -219,7 +240,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     if (o.sm_speed)
         for (int i = 0; i < n_sm; ++i) speed[i] = o.sm_speed[i];
     const int L = c.n_layers, nkv = c.n_kv_heads, d = c.head_dim, H = c.hidden, F = c.ffn;
-    const int S = o.kv_splits > 0 ? o.kv_splits : default_kv_splits(c, n_sm);
+    const int S = o.kv_splits > 0 ? o.kv_splits : default_kv_splits(c, n_sm, o.batch);
     const int cap = o.rows_per_instr;
     const bool moe = c.n_experts > 0;
     const bool fused = ffn_fused(c, o);
@@ -233,7 +254,8 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
         if (w[W_AUX_CTR] >= 0) inc[w[W_AUX_CTR]]++;
     };
     const int qd = c.n_q_heads * d;
-    auto op_cap = [&](int op) { return std::min(cap, kRowSlots / acc_sets(op, H, qd, F, c.top_k)); };
+    const int nb = o.batch;  // every GEMV row keeps nb accumulator sets (one per sequence)
+    auto op_cap = [&](int op) { return std::min(cap, kRowSlots / (acc_sets(op, H, qd, F, c.top_k) * nb)); };
     auto gemv_op = [&](int op, int layer, const std::vector<Segment>& segs, int wait, int signal,
                        const std::vector<double>* weight = nullptr) {
         split_rows(segs, n_sm, op_cap(op), [&](int sm, int sub, int b, int e) {
@@ -253,16 +275,17 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
         const int prev_down = l > 0 ? ctr_id(l - 1, C_FFN2) : -1;
         gemv_op(OP_RMS_QKV, l, {{0, c.n_q_heads * d}, {1, nkv * d}, {2, nkv * d}}, prev_down,
                 ctr_id(l, C_QKV));
-        // attention: kv head g, split s -> instruction k = g * S + s, rotated per layer
-        const int total = nkv * S;
+        // attention: sequence q, kv head g, split s -> instruction k = (q * nkv + g) * S + s, rotated per layer
+        const int total = nb * nkv * S;
         std::vector<double> ffn_weight = speed;  // blocks with an attention split may take fewer FFN rows
         for (int k = 0; k < total; ++k) {
             Instr w = blank();
             w[W_OP] = OP_ATTN;
             w[W_LAYER] = l;
-            w[W_SUB] = k / S;
+            w[W_SUB] = (k / S) % nkv;
             w[W_BEGIN] = k % S;
             w[W_END] = S;
+            w[W_SEQ] = k / (S * nkv);
             w[W_WAIT_CTR] = ctr_id(l, C_QKV);
             w[W_SIGNAL_CTR] = ctr_id(l, C_ATTN);
             int sm = (int)(((long long)k + (long long)l * total) % n_sm);
@@ -336,6 +359,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     out->kv_splits = S;
     out->n_lm = (int)inc[ctr_lm(L)];
     out->fused_ffn = fused;
+    out->nb = nb;
     out->words.assign((size_t)n_sm * max_instr * W_NWORDS, 0);
     out->n_instr.assign(n_sm, 0);
     for (int sm = 0; sm < n_sm; ++sm) {
@@ -400,7 +424,10 @@ int validate(const mk_config& c, const Planned& p) {
         return -1;
     };
     std::vector<uint32_t> signals(nctr, 0);
-    std::vector<std::vector<uint8_t>> attn_seen((size_t)std::max(L, 1) * nkv, std::vector<uint8_t>(p.kv_splits, 0));
+    const int nb = p.nb;
+    if (nb < 1 || nb > kMaxBatch || (nb > 1 && (moe || !p.fused_ffn))) return MK_ERR_SCHEDULE;
+    std::vector<std::vector<uint8_t>> attn_seen((size_t)std::max(L, 1) * nb * nkv,
+                                                std::vector<uint8_t>(p.kv_splits, 0));
     std::vector<uint8_t> lm_seq(std::max(p.n_lm, 1), 0);
     std::vector<int> spec_publishers(std::max(L, 1), 0), spec_predictors(std::max(L, 1), 0);
     for (int sm = 0; sm < p.n_sm; ++sm) {
@@ -448,10 +475,11 @@ int validate(const mk_config& c, const Planned& p) {
             }
             if (w[W_AUX_CTR] >= 0 && (uint32_t)w[W_AUX_INC] != p.ctr_inc[w[W_AUX_CTR]]) return MK_ERR_SCHEDULE;
             if (op == OP_ATTN) {
-                const int g = w[W_SUB], s = w[W_BEGIN];
+                const int g = w[W_SUB], s = w[W_BEGIN], sq = w[W_SEQ];
                 if (g < 0 || g >= nkv || s < 0 || s >= p.kv_splits || w[W_END] != p.kv_splits) return MK_ERR_SCHEDULE;
+                if (sq < 0 || sq >= nb) return MK_ERR_SCHEDULE;
                 if (w[W_AUX_CTR] != -1 || w[W_SIGNAL_CTR] != ctr_id(l, C_ATTN)) return MK_ERR_SCHEDULE;
-                if (attn_seen[(size_t)l * nkv + g][s]++) return MK_ERR_SCHEDULE;
+                if (attn_seen[((size_t)l * nb + sq) * nkv + g][s]++) return MK_ERR_SCHEDULE;
                 signals[w[W_SIGNAL_CTR]]++;
                 continue;
             }
@@ -464,7 +492,7 @@ int validate(const mk_config& c, const Planned& p) {
             if (op != OP_RMS_QKV && op != OP_MOE_UPGATE && op != OP_MOE_FFN && sub != 0) return MK_ERR_SCHEDULE;
             const int b = w[W_BEGIN], e = w[W_END];
             const int sets = acc_sets(op, c.hidden, c.n_q_heads * d, c.ffn, c.top_k);
-            if (b < 0 || e > R || b >= e || e - b > kMaxRows || (e - b) * sets > kRowSlots) return MK_ERR_SCHEDULE;
+            if (b < 0 || e > R || b >= e || e - b > kMaxRows || (e - b) * sets * nb > kRowSlots) return MK_ERR_SCHEDULE;
             auto& hits = cov[cov_key(l, op, sub)];
             if (hits.empty()) hits.assign(R, 0);
             for (int r = b; r < e; ++r)
@@ -488,9 +516,9 @@ int validate(const mk_config& c, const Planned& p) {
                     if (h != 1) return MK_ERR_SCHEDULE;
             }
     for (int l = 0; l < L; ++l) {
-        for (int g = 0; g < nkv; ++g)
+        for (int g = 0; g < nb * nkv; ++g)
             for (int s = 0; s < p.kv_splits; ++s)
-                if (attn_seen[(size_t)l * nkv + g][s] != 1) return MK_ERR_SCHEDULE;
+                if (attn_seen[(size_t)l * nb * nkv + g][s] != 1) return MK_ERR_SCHEDULE;
         const std::vector<int> need = p.fused_ffn
             ? std::vector<int>{OP_RMS_QKV, OP_OPROJ_RES, moe ? OP_MOE_FFN : OP_FFN}
             : std::vector<int>{OP_RMS_QKV, OP_OPROJ_RES, moe ? OP_MOE_UPGATE : OP_RMS_UPGATE_SILU,

@@ -46,7 +46,7 @@ class MkOptions(ctypes.Structure):
                 ("mode", _I), ("n_sm", _I), ("prefetch_ahead", _I), ("prefetch_max_bytes", _I),
                 ("attn_sm_ffn_permille", _I), ("serve_idle_ns", ctypes.c_ulonglong), ("general_kernel", _I),
                 ("split_ffn", _I), ("l2_head_start", _I), ("sm_speed", ctypes.c_void_p), ("n_sm_speed", _I),
-                ("spec_experts", _I)]
+                ("spec_experts", _I), ("batch", _I)]
 
 
 class MkStatus(ctypes.Structure):
@@ -66,6 +66,7 @@ SIGNATURES = {
     "mk_get_schedule": (_I, [_P, _P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(_I),
                              ctypes.POINTER(_I)]),
     "mk_decode_step": (_I, [_P, ctypes.c_int32, ctypes.c_int32, _P, _P]),
+    "mk_decode_step_batch": (_I, [_P, _P, _P, _P, _P]),
     "mk_get_hidden": (_I, [_P, _I, _P]),
     "mk_get_router": (_I, [_P, _I, _P, _P]),
     "mk_get_predicted_experts": (_I, [_P, _I, _P]),
@@ -197,8 +198,9 @@ class Decoder:
     dicts with attn_norm, wq, wk, wv, wo, ffn_norm, w_gate, w_up, w_down and,
     for MoE, router plus per-expert lists for w_gate/w_up/w_down), each a CUDA
     tensor holding bf16 bits (any 2-byte dtype).  kcache/vcache: CUDA tensors
-    [L, n_kv, max_seq, d] of bf16 bits.  The tensors must stay alive as long as
-    the decoder.  `stream`: a torch.cuda.Stream or None (current stream)."""
+    [L, n_kv, max_seq, d] of bf16 bits ([batch, L, n_kv, max_seq, d] with the
+    option batch > 1).  The tensors must stay alive as long as the decoder.
+    `stream`: a torch.cuda.Stream or None (current stream)."""
 
     def __init__(self, cfg, weights: dict, kcache, vcache, stream=None, build_schedule: bool = True, **options):
         import torch
@@ -206,7 +208,11 @@ class Decoder:
         self.cfg = cfg
         self._keep = [weights, kcache, vcache]
         self.config = make_config(cfg)
-        self.config.max_seq = int(kcache.shape[2])
+        self.config.max_seq = int(kcache.shape[-2])
+        nb = max(1, int(options.get("batch", 1) or 1))
+        if (kcache.dim() == 5) != (nb > 1) or (nb > 1 and kcache.shape[0] != nb):
+            raise ValueError(f"KV cache shape {tuple(kcache.shape)} does not match batch={nb}")
+        self.batch = nb
         L = self.config.n_layers
         E = self.config.n_experts
         layers = weights["layers"]
@@ -287,11 +293,27 @@ class Decoder:
         return self.lib.mk_decode_step(self.h, int(token), int(pos), _ptr(logits) if logits is not None else None,
                                        ctypes.byref(out) if sync else None)
 
+    def step_batch(self, tokens, pos, logits=None, sync: bool = True):
+        """One decode step of every sequence of the batch: tokens and pos are sequences of `batch`
+        ints (token < 0: that sequence's previous argmax).  logits: optional CUDA fp32 tensor
+        [batch, vocab].  With sync=True returns the next tokens (int32 array); else only enqueues."""
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        ps = np.ascontiguousarray(pos, dtype=np.int32)
+        if t.size != self.batch or ps.size != self.batch:
+            raise ValueError(f"expected {self.batch} tokens and positions")
+        out = np.full(self.batch, -1, dtype=np.int32)
+        rc = self.lib.mk_decode_step_batch(self.h, t.ctypes.data, ps.ctypes.data,
+                                           _ptr(logits) if logits is not None else None,
+                                           out.ctypes.data if sync else None)
+        check(rc, "mk_decode_step_batch")
+        return out if sync else None
+
     # -- debug getters ------------------------------------------------------------------
     def hidden(self, layer: int) -> np.ndarray:
-        out = np.empty(self.config.hidden, dtype=np.float32)
+        """Residual stream after `layer`: [hidden], or [batch, hidden] with batch > 1."""
+        out = np.empty((self.batch, self.config.hidden), dtype=np.float32)
         check(self.lib.mk_get_hidden(self.h, layer, out.ctypes.data), "mk_get_hidden")
-        return out
+        return out[0] if self.batch == 1 else out
 
     def hidden_all(self) -> np.ndarray:
         return np.stack([self.hidden(l) for l in range(self.config.n_layers + 1)])

@@ -175,19 +175,29 @@ def main(argv=None) -> None:
     ap.add_argument("config")
     ap.add_argument("--steps", type=int, default=4)
     ap.add_argument("--npz", default="")
+    ap.add_argument("--batch", type=int, default=1, help="sequences per step (batched decode)")
     ap.add_argument("options", nargs="*", help="mk_options fields as key=value (integers)")
     args = ap.parse_intermixed_args(argv)
     cfg = configs.get(args.config)
     opts = {k: int(v) for k, v in (kv.split("=") for kv in args.options)}
     W = synth.make_model(cfg)
-    kc, vc = synth.make_kv_cache(cfg)
-    dk = torch.from_numpy(kc.view(np.int16)).cuda()
-    dv = torch.from_numpy(vc.view(np.int16)).cuda()
+    B = args.batch
+    caches = [synth.make_kv_cache(cfg, stream=f".{b}" if b else "") for b in range(B)]
+    stack = (lambda a: a[0]) if B == 1 else np.stack
+    dk = torch.from_numpy(stack([c[0] for c in caches]).view(np.int16)).cuda()
+    dv = torch.from_numpy(stack([c[1] for c in caches]).view(np.int16)).cuda()
     p0 = cfg.prefill + cfg.prompt_len
+    if B > 1:
+        opts["batch"] = B
     with Decoder(cfg, to_device(W), dk, dv, trace=1, **opts) as dec:
-        tok = dec.step(int(synth.prompt_tokens(cfg)[0]), p0)
-        for i in range(1, args.steps):
-            tok = dec.step(tok, p0 + i)
+        if B == 1:
+            tok = dec.step(int(synth.prompt_tokens(cfg)[0]), p0)
+            for i in range(1, args.steps):
+                tok = dec.step(tok, p0 + i)
+        else:
+            toks = dec.step_batch([int(synth.prompt_tokens(cfg, stream=f".{b}")[0]) for b in range(B)], [p0] * B)
+            for i in range(1, args.steps):
+                toks = dec.step_batch(toks, [p0 + i] * B)
         sched, tr = dec.schedule(), dec.trace()
         print(f"{cfg.name}: last step {dec.last_step_ns() / 1000:.1f} us (traced)")
     print(format_breakdown(op_breakdown(sched, tr)))

@@ -83,7 +83,9 @@ typedef struct {
  * n_layers device pointers; for MoE, w_gate/w_up/w_down have
  * n_layers * n_experts entries ([layer * n_experts + expert]) and router has
  * n_layers entries.  router may be NULL for dense models; the KV caches may
- * be NULL when n_layers == 0.  All device pointers must be 16-byte aligned. */
+ * be NULL when n_layers == 0.  All device pointers must be 16-byte aligned.
+ * With options.batch = B > 1 each cache holds B sequences' caches one after
+ * the other ([B][n_layers][n_kv][max_seq][head_dim]). */
 typedef struct {
     const void *embed, *lm_head, *final_norm;
     const void *const *attn_norm, *const *wq, *const *wk, *const *wv, *const *wo, *const *ffn_norm;
@@ -144,6 +146,16 @@ typedef struct {
                              rows are streamed instead.  The result is the same either way.  2 = predict
                              the experts with the lowest scores instead (every prediction misses unless
                              all experts are selected; exercises the miss path).  0 (default) = off */
+    int batch;            /* sequences decoded together per step (1..8; 0 = 1).  With batch B > 1 every
+                             weight stage that reaches shared memory is applied to the B sequences' input
+                             vectors before its slot is freed, so the weights cross HBM once per step for
+                             all of them; attention, RoPE, the KV append and the argmax run per sequence.
+                             Each sequence has its own KV cache (the caches are [B][n_layers][n_kv]
+                             [max_seq][head_dim], sequence-major), token and position, stepped by
+                             mk_decode_step_batch.  B > 1 needs a dense model with the fused FFN in
+                             megakernel mode, hidden and n_q_heads*head_dim at most 2048 (B <= 8) or 4096
+                             (B <= 4), and no serving or speculative prediction; otherwise
+                             mk_create returns MK_ERR_UNSUPPORTED */
 } mk_options;
 
 /* Device status block, copied out by mk_get_status.  On a device-side error
@@ -209,8 +221,26 @@ int mk_get_schedule(mk_handle *h, int32_t *buf, size_t cap, size_t *n_words, int
  * README's models, the next-token choice the greedy argmax. */
 int mk_decode_step(mk_handle *h, int32_t token, int32_t pos, float *logits_dev, int32_t *next_token_host);
 
+/* One decode step of the options.batch sequences of the handle in one launch:
+ * sequence b embeds tokens[b] (token < 0: its previous on-device argmax), runs
+ * every layer at position pos[b] against its own KV cache (appending at pos[b],
+ * attending over 0..pos[b]); positions may differ between sequences.  tokens
+ * and pos are host arrays of batch entries (read before the call returns).
+ * logits_dev: device [batch][vocab] fp32, may be NULL.  next_host: host array
+ * of batch entries, or NULL to only enqueue (as mk_decode_step).  A batch-1
+ * handle accepts this call too (the same step as mk_decode_step).
+ * Errors: as mk_decode_step; MK_ERR_INVALID_ARG for a null array or a bad
+ * token or position.
+ * Source: a megakernel removes the launch gaps that dominate batch-1 decode,
+ * while at larger batch the matrix products grow to hide them (Hyperkernel
+ * teardown, "What a megakernel buys"); this is the small-batch variant of the
+ * same step, each weight read from HBM once for every sequence of the batch. */
+int mk_decode_step_batch(mk_handle *h, const int32_t *tokens, const int32_t *pos, float *logits_dev,
+                         int32_t *next_host);
+
 /* Residual stream after layer `layer` of the last step (0 = embedding,
- * n_layers = after the last layer) as fp32 [hidden] into host `out_host`.
+ * n_layers = after the last layer) as fp32 [batch][hidden] into host
+ * `out_host` (batch = options.batch, 1 by default).
  * Needs options.snapshots = 1.  Synchronises the stream.
  * Source: per-layer checks against a reference, the kind of correctness
  * evidence the Hyperkernel teardown asks a megakernel release to ship ("What a

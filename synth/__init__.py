@@ -114,13 +114,14 @@ def make_model(cfg: ModelConfig) -> dict:
     return m
 
 
-def make_kv_cache(cfg: ModelConfig, max_seq: int | None = None):
+def make_kv_cache(cfg: ModelConfig, max_seq: int | None = None, stream: str = ""):
     """(K, V) bf16 caches [L][nkv][max_seq][d]; positions < cfg.prefill hold
-    N(0, kv_sigma^2) draws (taken as already rotated), the rest zero."""
+    N(0, kv_sigma^2) draws (taken as already rotated), the rest zero.  `stream`
+    names an independent draw (the caches of the sequences of a batch)."""
     ms = cfg.max_seq if max_seq is None else max_seq
     shape = (cfg.n_layers, cfg.n_kv_heads, ms, cfg.head_dim)
     out = []
-    for prefix in ("kcache", "vcache"):
+    for prefix in ("kcache" + stream, "vcache" + stream):
         c = np.empty(shape, dtype=np.uint16)
         lib().synth_kv_prefill(c.ctypes.data, cfg.n_layers, cfg.n_kv_heads, ms, cfg.head_dim, cfg.prefill,
                                cfg.seed, prefix.encode(), cfg.kv_sigma)
@@ -128,11 +129,12 @@ def make_kv_cache(cfg: ModelConfig, max_seq: int | None = None):
     return out[0], out[1]
 
 
-def prompt_tokens(cfg: ModelConfig) -> np.ndarray:
+def prompt_tokens(cfg: ModelConfig, stream: str = "") -> np.ndarray:
     """Random prompt (tiny model: 16 tokens) or, for pre-filled caches, the one
-    random token fed at the first decode position."""
+    random token fed at the first decode position.  `stream` names an
+    independent draw (the prompts of the sequences of a batch)."""
     n = cfg.prompt_len if cfg.prompt_len else 1
-    return tokens(n, cfg.seed, "prompt", cfg.vocab)
+    return tokens(n, cfg.seed, "prompt" + stream, cfg.vocab)
 
 
 __all__ = ["configs", "ModelConfig", "build", "normal_bf16", "const_bf16", "tokens", "bf16_to_f32", "f32_to_bf16",

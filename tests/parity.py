@@ -149,3 +149,45 @@ def assert_parity(reports: list[dict], cfg=None):
             if margin > PRED_MARGIN:
                 assert got == want, (r["pos"], got, want, margin)
     return worst_h, worst_l
+
+
+def run_batch(cfg, prefills, steps: int, weights: dict | None = None, **opts) -> list[dict]:
+    """Teacher-forced batched decode of len(prefills) sequences in one handle: sequence b has its own
+    KV cache (pre-filled with its own draws below prefills[b]) and prompt, starts at position
+    prefills[b], feeds its prompt tokens, then its oracle's greedy tokens.  One report per sequence
+    and step, each checked against that sequence's own fp64 oracle."""
+    import torch
+    from decode_persistent_block_b200 import Decoder, to_device
+    B = len(prefills)
+    run_cfg = cfg.with_(prefill=max(prefills), prompt_len=0, steps=steps)
+    W = weights if weights is not None else synth.make_model(cfg)
+    dW = to_device(W)
+    caches = [synth.make_kv_cache(cfg.with_(prefill=pf), max_seq=run_cfg.max_seq, stream=f".{b}")
+              for b, pf in enumerate(prefills)]
+    dk = torch.from_numpy(np.stack([c[0] for c in caches]).view(np.int16)).cuda()
+    dv = torch.from_numpy(np.stack([c[1] for c in caches]).view(np.int16)).cuda()
+    orcs = [oracle.Model(run_cfg, W, c[0].copy(), c[1].copy()) for c in caches]
+    prompts = [synth.prompt_tokens(cfg, stream=f".{b}") for b in range(B)]
+    logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    reports, nxt = [], [None] * B
+    opts.setdefault("snapshots", 1)
+    with Decoder(run_cfg, dW, dk, dv, batch=B, **opts) as dec:
+        for i in range(steps):
+            toks = [int(prompts[b][i]) if i < len(prompts[b]) else nxt[b] for b in range(B)]
+            pos = [pf + i for pf in prefills]
+            got = dec.step_batch(toks, pos, logits=logits)
+            lg = logits.cpu().numpy().astype(np.float64)
+            hid = dec.hidden_all().astype(np.float64) if dec.options.snapshots else None  # [L+1][B][H]
+            for b in range(B):
+                o = orcs[b].step(toks[b], pos[b])
+                lo = o["logits"]
+                srt = np.sort(lo)
+                r = {"logit_err": float(np.max(np.abs(lg[b] - lo))), "margin": float(srt[-1] - srt[-2]),
+                     "next_orc": o["next"], "next_gpu": int(got[b]), "pos": pos[b], "seq": b}
+                if hid is not None:
+                    hb, ho = hid[:, b], o["hidden"]
+                    r["hidden_rel"] = (np.linalg.norm(hb - ho, axis=1) /
+                                       np.maximum(np.linalg.norm(ho, axis=1), 1e-30)).tolist()
+                reports.append(r)
+                nxt[b] = o["next"]
+    return reports

@@ -280,3 +280,63 @@ def test_mixtral8l_speculative_experts(cuda):
     reps = _full(configs.MIXTRAL_8L, 3, spec_experts=1)
     hits, slots = _pred_stats(reps)
     print(f"mixtral8l speculative experts: {hits}/{slots} slots hit")
+
+
+# ---- batched decode ------------------------------------------------------------------
+
+# head_dim 128, two chunks per thread (the Llama-3B kernel's widths) at small depth and vocabulary
+H3K_SMALL = configs.TINY.with_(name="tiny_h3072", hidden=3072, n_heads=24, n_kv_heads=8, head_dim=128, ffn=1024)
+
+
+@pytest.mark.parametrize("B", [2, 3, 4, 5, 8])
+def test_tiny_batch(cuda, B):
+    # ragged positions: sequence b starts 3 b positions later, with its own cache, prompt and tokens
+    parity.assert_parity(parity.run_batch(configs.TINY, [3 * b for b in range(B)], steps=20), configs.TINY)
+
+
+@pytest.mark.parametrize("B", [2, 4])
+def test_head_dim_128_batch(cuda, B):
+    parity.assert_parity(parity.run_batch(H3K_SMALL, [5 * b + 1 for b in range(B)], steps=6), H3K_SMALL)
+
+
+def test_tiny_batch_ring_and_split_options(cuda):
+    for opts in (dict(ring_stages=2), dict(kv_splits=3), dict(stage_bytes=32768), dict(n_sm=7)):
+        parity.assert_parity(parity.run_batch(configs.TINY, [0, 4, 9, 2], steps=8, **opts), configs.TINY)
+
+
+def test_batch_handle_rejects_single_steps_and_bad_arguments(cuda):
+    import torch
+    from decode_persistent_block_b200 import Decoder, MkError, to_device
+    cfg = configs.TINY
+    W = to_device(parity.synth.make_model(cfg))
+    kc, vc = parity.synth.make_kv_cache(cfg)
+    dk = torch.from_numpy(np.stack([kc, kc]).view(np.int16)).cuda()
+    dv = torch.from_numpy(np.stack([vc, vc]).view(np.int16)).cuda()
+    with Decoder(cfg, W, dk, dv, batch=2) as dec:
+        with pytest.raises(MkError) as e:
+            dec.step(1, 0)
+        assert e.value.name == "MK_ERR_INVALID_ARG"
+        for toks, pos in (([1, cfg.vocab], [0, 0]), ([1, 2], [0, cfg.max_seq]), ([1, 2], [-1, 0])):
+            with pytest.raises(MkError) as e:
+                dec.step_batch(toks, pos)
+            assert e.value.name == "MK_ERR_INVALID_ARG"
+        with pytest.raises(MkError) as e:
+            dec.serve_start()
+        assert e.value.name == "MK_ERR_INVALID_ARG"
+        out = dec.step_batch([1, 2], [0, 0])  # still usable
+        assert out.shape == (2,) and dec.status()["code"] == 0
+    moe = cfg.with_(name="tiny_moe", n_experts=4, top_k=2)
+    Wm = to_device(parity.synth.make_model(moe))
+    with pytest.raises(MkError) as e:
+        Decoder(moe, Wm, dk, dv, batch=2)
+    assert e.value.name == "MK_ERR_UNSUPPORTED"
+
+
+def test_llama1b_batch8(cuda):
+    cfg = configs.LLAMA_1B
+    parity.assert_parity(parity.run_batch(cfg, [cfg.prefill - 37 * b for b in range(8)], steps=3), cfg)
+
+
+def test_llama3b_batch4(cuda):
+    cfg = configs.LLAMA_3B
+    parity.assert_parity(parity.run_batch(cfg, [cfg.prefill - 101 * b for b in range(4)], steps=2), cfg)

@@ -349,3 +349,43 @@ def test_speculative_prediction_option_range():
     for bad in (-1, 3):
         with pytest.raises(mk.MkError):
             dpb.plan(configs.MIXTRAL_8L, 148, spec_experts=bad)
+
+
+@pytest.mark.parametrize("B", [2, 5, 8])
+@pytest.mark.parametrize("n_sm", [148, 37])
+def test_batch_schedule(B, n_sm):
+    # every (sequence, kv head, split) attention instruction once per layer; every GEMV instruction keeps
+    # B accumulator sets per row within the shared-memory slots; counters count the batch's signals
+    cfg = configs.LLAMA_1B
+    words, n_instr, inc = dpb.plan(cfg, n_sm, batch=B)
+    S = None
+    seen = set()
+    for sm, i, w in instrs(words, n_instr):
+        op = int(w[W_OP])
+        if op == OP["ATTN"]:
+            S = int(w[W_END])
+            key = (int(w[W_LAYER]), int(w[W_SEQ]), int(w[W_SUB]), int(w[W_BEGIN]))
+            assert key not in seen and 0 <= key[1] < B
+            seen.add(key)
+        else:
+            sets = 2 if op == OP["FFN"] else 1
+            if op != OP["LM"]:
+                assert (w[W_END] - w[W_BEGIN]) * sets * B <= 1024
+    assert len(seen) == cfg.n_layers * B * cfg.n_kv_heads * S
+    assert inc[1] == B * cfg.n_kv_heads * S  # layer 0's attention counter
+    assert B * cfg.n_kv_heads * S <= max(n_sm, B * cfg.n_kv_heads)
+    rc, done = dpb.simulate(words, n_instr, inc, steps=2, seed=B)
+    assert rc == 0 and done == 2 * int(n_instr.sum())
+
+
+def test_batch_options_are_checked():
+    with pytest.raises(mk.MkError) as e:
+        dpb.plan(configs.LLAMA_1B, 148, batch=9)
+    assert e.value.name == "MK_ERR_INVALID_ARG"
+    for cfg, opts in ((configs.LLAMA_3B, dict(batch=8)), (configs.MIXTRAL_8L, dict(batch=2)),
+                      (configs.LLAMA_1B, dict(batch=2, split_ffn=1)), (configs.LLAMA_1B, dict(batch=2, mode=1)),
+                      (configs.LLAMA_1B, dict(batch=2, l2_prefetch=65536))):
+        with pytest.raises(mk.MkError) as e:
+            dpb.plan(cfg, 148, **opts)
+        assert e.value.name == "MK_ERR_UNSUPPORTED", (cfg.name, opts)
+    dpb.plan(configs.LLAMA_3B, 148, batch=4)
