@@ -69,6 +69,8 @@ def parse():
     ap.add_argument("--ring-stages", type=int, default=0)
     ap.add_argument("--stage-bytes", type=int, default=0)
     ap.add_argument("--kv-splits", type=int, default=0)
+    ap.add_argument("--batch-sizes", default="2,4,8",
+                    help="batched-decode sizes measured after the headline (comma list; empty: none)")
     ap.add_argument("--spec-experts", type=int, default=-1,
                     help="MoE configs: speculative expert prediction (0 off, 1 on, 2 mispredict; -1: the "
                          "library default)")
@@ -432,6 +434,50 @@ def measure(args, cfg, p0, positions, K, Wm, rank, world, local, with_extras=Tru
     }
 
 
+def measure_batch(args, cfg, p0, B, K, Wm, world, local):
+    """Device-timed batched decode steps (B sequences per launch, each with its own cache and
+    token, all at the same positions as the batch-1 workload); returns one `batch` entry."""
+    import numpy as np
+    import torch
+
+    import synth
+    from decode_persistent_block_b200 import Decoder, to_device
+    torch.cuda.set_device(local)
+    dW = to_device(synth.make_model(cfg))
+    caches = [synth.make_kv_cache(cfg, stream=f".{b}") for b in range(B)]
+    dk = torch.from_numpy(np.stack([c[0] for c in caches]).view(np.int16)).cuda()
+    dv = torch.from_numpy(np.stack([c[1] for c in caches]).view(np.int16)).cuda()
+    del caches
+    first = [int(synth.prompt_tokens(cfg, stream=f".{b}")[0]) for b in range(B)]
+    pos = [p0 + (i % cfg.steps) for i in range(max(K, Wm) + 1)]
+    with Decoder(cfg, dW, dk, dv, batch=B) as dec:
+        dec.step_batch(first, [pos[0]] * B)
+        for i in range(1, Wm):
+            dec.step_batch([-1] * B, [pos[i]] * B, sync=False)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(K):
+            dec.step_batch([-1] * B, [pos[i % len(pos)]] * B, sync=False)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        st = dec.status()
+        if st["code"] != 0:
+            raise RuntimeError(f"device status after batched steps: {st}")
+    step_us = reduce_max(e0.elapsed_time(e1), world) * 1000.0 / K
+    bpt = cfg.weight_bytes_per_token() + B * statistics.fmean(cfg.kv_bytes_per_token(q) for q in pos[:K])
+    del dW, dk, dv
+    torch.cuda.empty_cache()
+    return {"batch": B, "us_per_step": round(step_us, 1), "us_per_token": round(step_us / B, 2),
+            "tokens_per_s": round(B * world * 1e6 / step_us, 1), "gb_per_step": round(bpt / 1e9, 4),
+            "hbm_gbs": round(bpt / (step_us * 1e-6) / 1e9, 1), "steps": K, "warmup": Wm,
+            "workload": f"{cfg.name}: {B} sequences per step, each with its own KV cache pre-filled to "
+                        f"{cfg.prefill} and its own tokens, positions {p0}..{p0 + cfg.steps - 1}"}
+
+
 def workload_name(cfg, p0):
     return (f"{cfg.name}: batch-1 greedy decode, KV pre-filled to {cfg.prefill}, positions "
             f"{p0}..{p0 + cfg.steps - 1}")
@@ -462,6 +508,15 @@ def run_ours(args, rank, world, local):
                                 "steps": m["steps"], "warmup": m["warmup"]}
             if m["expert_prediction"] is not None:
                 per_config[name]["expert_prediction"] = m["expert_prediction"]
+
+    batched = []
+    if args.batch_sizes and not args.layers and args.mode == "megakernel" and not cfg.n_experts:
+        from decode_persistent_block_b200 import MkError
+        for B in (int(x) for x in args.batch_sizes.split(",") if x):
+            try:
+                batched.append(measure_batch(args, cfg, p0, B, min(K, 256), Wm, world, local))
+            except MkError as e:  # no kernel for this batch size on this shape
+                batched.append({"batch": B, "unsupported": e.name})
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -495,6 +550,7 @@ def run_ours(args, rank, world, local):
         "gpu_launches": K if args.mode == "megakernel" else None,
         "baselines": r["baselines"],
         "per_config": per_config or None,
+        "batched": batched or None,
         "expert_prediction": r["expert_prediction"],
         "cpu_baseline": cpu,
         "clocks": r["clocks"],

@@ -217,10 +217,10 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
         if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
     }
 }
-// Transpose-reduce of RG per-lane partials (one per row, RG in {1,2,4,8})
-// across the warp: log2(RG) halving rounds exchange half of the values, then
-// 5 - log2(RG) butterfly rounds finish the sum (RG - 1 + 5 - log2(RG) shuffles
-// instead of 5 * RG).  On return every lane holds the full sum of row
+// Transpose-reduce of RG per-lane partials (one per row, RG a power of two up
+// to 32) across the warp: log2(RG) halving rounds exchange half of the values,
+// then 5 - log2(RG) butterfly rounds finish the sum (RG - 1 + 5 - log2(RG)
+// shuffles instead of 5 * RG).  On return every lane holds the full sum of row
 // lane >> (5 - log2(RG)).
 template <int RG>
 __device__ __forceinline__ float reduce_rows(float (&a)[RG], int lane) {
@@ -234,7 +234,7 @@ __device__ __forceinline__ float reduce_rows(float (&a)[RG], int lane) {
             a[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
         }
     }
-    constexpr int first = RG == 8 ? 2 : RG == 4 ? 4 : RG == 2 ? 8 : 16;
+    constexpr int first = RG == 32 ? 0 : RG == 16 ? 1 : RG == 8 ? 2 : RG == 4 ? 4 : RG == 2 ? 8 : 16;
     float e = a[0];
 #pragma unroll
     for (int off = first; off > 0; off >>= 1) e += __shfl_xor_sync(0xFFFFFFFFu, e, off);
@@ -242,7 +242,7 @@ __device__ __forceinline__ float reduce_rows(float (&a)[RG], int lane) {
 }
 template <int RG>
 __device__ __forceinline__ int reduce_rows_lane_row(int lane) {
-    return RG == 8 ? lane >> 2 : RG == 4 ? lane >> 3 : RG == 2 ? lane >> 4 : 0;
+    return RG == 32 ? lane : RG == 16 ? lane >> 1 : RG == 8 ? lane >> 2 : RG == 4 ? lane >> 3 : RG == 2 ? lane >> 4 : 0;
 }
 template <int RG>
 __device__ __forceinline__ bool reduce_rows_writer(int lane) {

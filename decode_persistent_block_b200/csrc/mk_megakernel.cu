@@ -1409,10 +1409,11 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
 // ---------------------------------------------------------------------------
 // RG rows [rg, rg + RG) of a stage against the sequences' input vectors: the
 // rows' weights are loaded and widened to fp32 once, then every sequence's dot
-// products reuse them; each sequence's row sums are reduced across the warp
-// and stored in that sequence's accumulator set (A + q * aset, one slot per
-// row and warp, added in warp order by the epilogue).  Rows at or past nr are
-// predicated off.
+// products reuse them (all NB, the unused ones against zero vectors, so the
+// chains interleave); the NB x RG row sums are reduced across the warp in one
+// transpose-reduce and stored in each sequence's accumulator set (A + q *
+// aset, one slot per row and warp, added in warp order by the epilogue).  Rows
+// at or past nr are predicated off.
 template <int J, int RG, int NB>
 __device__ __forceinline__ void rows_block_b(const uint4* __restrict__ Ws, int row16, int rg, int nr,
                                              const bool (&jv)[J], const float (&v)[NB][J][8], float* A, int aset,
@@ -1426,12 +1427,10 @@ __device__ __forceinline__ void rows_block_b(const uint4* __restrict__ Ws, int r
             unpack8((jv[j] && rg + r < nr) ? Ws[(rg + r) * row16 + tid + kConsumerThreads * j]
                                            : make_uint4(0u, 0u, 0u, 0u),
                     wf[r][j]);
-    const int row = rg + reduce_rows_lane_row<RG>(lane);
-    const bool writer = reduce_rows_writer<RG>(lane) && row < nr;
+    constexpr int N = NB * RG;  // index q * RG + r
+    float part[N];
 #pragma unroll
-    for (int q = 0; q < NB; ++q) {
-        if (q >= nb) break;
-        float part[RG];
+    for (int q = 0; q < NB; ++q)
 #pragma unroll
         for (int r = 0; r < RG; ++r) {
             float a0 = 0.f, a1 = 0.f;
@@ -1442,11 +1441,12 @@ __device__ __forceinline__ void rows_block_b(const uint4* __restrict__ Ws, int r
                     a0 = fmaf(wf[r][j][k], v[q][j][k], a0);
                     a1 = fmaf(wf[r][j][k + 1], v[q][j][k + 1], a1);
                 }
-            part[r] = a0 + a1;
+            part[q * RG + r] = a0 + a1;
         }
-        const float s_row = reduce_rows<RG>(part, lane);
-        if (writer) A[(size_t)q * aset + row * kConsumerWarps + (tid >> 5)] = s_row;
-    }
+    const float s = reduce_rows<N>(part, lane);
+    const int idx = reduce_rows_lane_row<N>(lane), q = idx / RG, row = rg + idx % RG;
+    if (reduce_rows_writer<N>(lane) && q < nb && row < nr)
+        A[(size_t)q * aset + row * kConsumerWarps + (tid >> 5)] = s;
 }
 
 template <int J, int RG, int NB>
@@ -1547,8 +1547,8 @@ __device__ void load_rms_b(const DevParams& p, Misc& m, const float* x32, bool f
 // per round trip.
 template <int J, int NB>
 __device__ void load_attn_merged_b(const DevParams& p, int K, float (&v)[NB][J][8]) {
-    constexpr int QG = NB < 4 ? NB : 4;  // sequences per round
-    constexpr int SG = 8 / QG;           // splits per round
+    constexpr int QG = NB < 4 ? NB : 4;        // sequences per round
+    constexpr int SG = NB >= 8 ? 1 : 8 / QG;   // splits per round (QG x SG x 10 live floats)
     const int tid = threadIdx.x, nch = K >> 3, S = p.kv_splits, D = p.d, D4 = D >> 2, nb = p.nb;
     const size_t seq_ml = (size_t)p.nq * S * 2, seq_o = (size_t)p.nq * S * D;
 #pragma unroll
@@ -1697,21 +1697,28 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
             for (int r = tid; r < rows; r += kConsumerThreads)
                 p.qkv[(size_t)q * qkvn + off + b + r] = acc_row(part_sums, aset, q, r);
     } else if (op == OP_OPROJ_RES) {
-        for (int q = 0; q < nb; ++q)
-            for (int r = tid; r < rows; r += kConsumerThreads) {
-                const size_t i = q * H + b + r;
-                float base;
-                if (l == 0) {
-                    const uint16_t e = p.embed[(size_t)m.btok[q] * H + b + r];
-                    base = __uint_as_float((uint32_t)e << 16);
-                    if (p.snap) p.snap[(size_t)q * (p.L + 1) * H + b + r] = base;
-                } else {
-                    base = __ldcg(p.x2 + i);
+        for (int r = tid; r < rows; r += kConsumerThreads) {
+            float base[NB];
+#pragma unroll
+            for (int q = 0; q < NB; ++q) {  // every sequence's residual load first (one round trip)
+                base[q] = 0.f;
+                if (q < nb) {
+                    if (l == 0)
+                        base[q] = __uint_as_float((uint32_t)p.embed[(size_t)m.btok[q] * H + b + r] << 16);
+                    else
+                        base[q] = __ldcg(p.x2 + q * H + b + r);
                 }
-                const float nx = base + acc_row(part_sums, aset, q, r);
+            }
+#pragma unroll
+            for (int q = 0; q < NB; ++q) {
+                if (q >= nb) break;
+                const size_t i = q * H + b + r;
+                if (l == 0 && p.snap) p.snap[(size_t)q * (p.L + 1) * H + b + r] = base[q];
+                const float nx = base[q] + acc_row(part_sums, aset, q, r);
                 p.x[i] = nx;
                 p.x2[i] = nx;
             }
+        }
     } else {  // LM head: logits, then each sequence's argmax over this instruction's rows
         float bv[NB];
         int bi[NB];
@@ -1880,7 +1887,7 @@ __device__ bool ffn_instr_b(const DevParams& p, const StepArgs& a, const int32_t
 #pragma unroll
         for (int k = 0; k < HR; ++k) {
             const int r = tid + kConsumerThreads * k;
-            if (q < nb && r < rows) scratch[(size_t)r * NB + q] = hv[q][k];
+            if (r < rows) scratch[(size_t)r * NB + q] = hv[q][k];  // 0 for unused sequences
         }
     cbar();
 
@@ -1901,21 +1908,28 @@ __device__ bool ffn_instr_b(const DevParams& p, const StepArgs& a, const int32_t
         if (warp_wait_full(&full[slot], phase, p, m, ii, op)) {
             if (tid == 0) stage_stamp(tr, T_SREADY, pl.spp + tst);
             const uint4* Ws = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
-            for (int r = 0; r < nr; ++r) {
-                float f[J][8];
+            // two rows per iteration (the unused sequences' h are zero)
+            for (int r = 0; r < nr; r += 2) {
+                float f[2][J][8], hk[2][NB];
 #pragma unroll
-                for (int j = 0; j < J; ++j)
-                    unpack8(jv[j] ? Ws[r * nch + tid + kConsumerThreads * j] : make_uint4(0u, 0u, 0u, 0u), f[j]);
-                const float* hr = scratch + (size_t)(r0 + r) * NB;
-#pragma unroll
-                for (int q = 0; q < NB; ++q) {
-                    if (q >= nb) break;
-                    const float hk = hr[q];
+                for (int u = 0; u < 2; ++u) {
+                    const bool live = r + u < nr;
 #pragma unroll
                     for (int j = 0; j < J; ++j)
+                        unpack8((live && jv[j]) ? Ws[(r + u) * nch + tid + kConsumerThreads * j]
+                                                : make_uint4(0u, 0u, 0u, 0u),
+                                f[u][j]);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) y[q][j][k] = fmaf(f[j][k], hk, y[q][j][k]);
+                    for (int q = 0; q < NB; ++q) hk[u][q] = live ? scratch[(size_t)(r0 + r + u) * NB + q] : 0.f;
                 }
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int q = 0; q < NB; ++q)
+#pragma unroll
+                        for (int j = 0; j < J; ++j)
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) y[q][j][k] = fmaf(f[u][j][k], hk[u][q], y[q][j][k]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
