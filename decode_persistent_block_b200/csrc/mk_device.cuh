@@ -217,6 +217,18 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
         if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
     }
 }
+// Two fp32 FMAs in one instruction (sm_100 packed f32x2):
+// (a.x * b.x + c.x, a.y * b.y + c.y), each rounded to nearest like fmaf.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
 // Transpose-reduce of RG per-lane partials (one per row, RG a power of two up
 // to 32) across the warp: log2(RG) halving rounds exchange half of the values,
 // then 5 - log2(RG) butterfly rounds finish the sum (RG - 1 + 5 - log2(RG)

@@ -107,6 +107,18 @@ MK_HD inline int wt_down_t(int e, int n_experts) { return kLayerFixed + 3 * (n_e
 // row (spans x expert slots x column parts); rows per instruction are capped at
 // kRowSlots / sets so that every (set, row) has a slot per consumer warp.
 MK_HD inline int kparts_of(int K) { return (K + kMaxPartK - 1) / kMaxPartK; }
+// Accumulator slots (rows x sets x sequences) an instruction of `rows` rows keeps in shared
+// memory.  A batched LM-head instruction goes through its rows in chunks (lm_chunk_rows), so
+// only one chunk's slots count.
+MK_HD inline int lm_chunk_rows(int nb, int rps) {
+    const int c = kRowSlots / (nb > 0 ? nb : 1) / rps * rps;  // whole ring stages of rps rows
+    return c > rps ? c : rps;
+}
+
+MK_HD inline int row_slots(int op, int rows, int sets, int nb) {
+    return op == OP_LMHEAD_ARGMAX && nb > 1 ? 0 : rows * sets * nb;
+}
+
 MK_HD inline int acc_sets(int op, int H, int qd, int F, int topk) {
     switch (op) {
         case OP_OPROJ_RES: return kparts_of(qd);

@@ -196,7 +196,7 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
     if (op == OP_FFN && sub != 0) return false;
     if ((op == OP_FFN || op == OP_MOE_FFN) && (p.H > kMaxPartK || 2 * p.H > p.stage_bytes)) return false;
     if (b < 0 || b >= e || e > op_rows(p, op, sub) || e - b > kMaxRows) return false;
-    if ((e - b) * acc_sets(op, p.H, p.nq * p.d, p.F, p.topk) * p.nb > kRowSlots) return false;
+    if (row_slots(op, e - b, acc_sets(op, p.H, p.nq * p.d, p.F, p.topk), p.nb) > kRowSlots) return false;
     if (op == OP_LMHEAD_ARGMAX) return w[W_AUX_CTR] >= 0 && w[W_AUX_INC] > 0 && w[W_SEQ] >= 0 && w[W_SEQ] < w[W_AUX_INC];
     return w[W_SIGNAL_CTR] >= 0;
 }
@@ -1433,15 +1433,13 @@ __device__ __forceinline__ void rows_block_b(const uint4* __restrict__ Ws, int r
     for (int q = 0; q < NB; ++q)
 #pragma unroll
         for (int r = 0; r < RG; ++r) {
-            float a0 = 0.f, a1 = 0.f;
+            float2 a = make_float2(0.f, 0.f);  // even / odd elements, two FMAs per instruction
 #pragma unroll
             for (int j = 0; j < J; ++j)
 #pragma unroll
-                for (int k = 0; k < 8; k += 2) {
-                    a0 = fmaf(wf[r][j][k], v[q][j][k], a0);
-                    a1 = fmaf(wf[r][j][k + 1], v[q][j][k + 1], a1);
-                }
-            part[q * RG + r] = a0 + a1;
+                for (int k = 0; k < 8; k += 2)
+                    a = fma2(make_float2(wf[r][j][k], wf[r][j][k + 1]), make_float2(v[q][j][k], v[q][j][k + 1]), a);
+            part[q * RG + r] = a.x + a.y;
         }
     const float s = reduce_rows<N>(part, lane);
     const int idx = reduce_rows_lane_row<N>(lane), q = idx / RG, row = rg + idx % RG;
@@ -1634,11 +1632,22 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
     const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], rows = w[W_END] - b;
     const uint32_t SB = (uint32_t)p.stage_bytes;
     const size_t H = (size_t)p.H;
-    float* part_sums = scratch;  // [sequence][row][8 warps]
-    const int aset = rows * kConsumerWarps;
+    float* part_sums = scratch;  // [sequence][row of the chunk][8 warps]
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
     Plan pl;
     make_plan(p, a.pos, w, nullptr, pl);
+    // The LM head's rows go through in chunks of whole stages whose partial sums fit the scratch
+    // (its logits and argmax need no other rows); the other ops' rows fit in one chunk.
+    const bool lm = op == OP_LMHEAD_ARGMAX;
+    const int chunk = lm ? lm_chunk_rows(nb, pl.rps) : rows;
+    const int aset = chunk * kConsumerWarps;
+    float bv[NB];  // LM head: each sequence's best logit and its row over the chunks so far
+    int bi[NB];
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        bv[q] = -CUDART_INF_F;
+        bi[q] = 0x7FFFFFFF;
+    }
     if (tid == 0 && w[W_WAIT_CTR] >= 0 &&
         !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op))
         vstore(&m.abort_flag, 1);
@@ -1673,7 +1682,7 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
             }
             const uint4* Ws = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
             stage_rows_b<J, RG, NB>(Ws, (int)(pl.row_bytes >> 4), nr, nch, v,
-                                    part_sums + (size_t)r0 * kConsumerWarps, aset, nb, lane);
+                                    part_sums + (size_t)(r0 % chunk) * kConsumerWarps, aset, nb, lane);
             __syncwarp();
             if (tid == 0) stage_stamp(tr, T_SDONE, sst);
             if (lane == 0) mbar_arrive(&empty[slot]);
@@ -1683,6 +1692,26 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
         if (++slot == p.ring_stages) {
             slot = 0;
             phase ^= 1u;
+        }
+        const int done = r0 + nr;
+        if (lm && (done == rows || done % chunk == 0)) {  // a chunk of the LM head is complete
+            const int c0 = (done - 1) / chunk * chunk, cn = done - c0;
+            cbar();
+            if (vload(&m.abort_flag)) return false;
+#pragma unroll
+            for (int q = 0; q < NB; ++q) {
+                if (q >= nb) break;
+                for (int r = tid; r < cn; r += kConsumerThreads) {
+                    const float val = acc_row(part_sums, aset, q, r);
+                    const int row = b + c0 + r;
+                    a.logits[(size_t)q * p.V + row] = val;
+                    if (val > bv[q]) {  // rows ascend for every thread: ties keep the lower row
+                        bv[q] = val;
+                        bi[q] = row;
+                    }
+                }
+            }
+            cbar();  // the scratch takes the next chunk
         }
     }
     cbar();
@@ -1719,22 +1748,10 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
                 p.x2[i] = nx;
             }
         }
-    } else {  // LM head: logits, then each sequence's argmax over this instruction's rows
-        float bv[NB];
-        int bi[NB];
+    } else {  // LM head: each sequence's argmax over this instruction's rows (logits written per chunk)
 #pragma unroll
         for (int q = 0; q < NB; ++q) {
-            bv[q] = -CUDART_INF_F;
-            bi[q] = 0x7FFFFFFF;
             if (q >= nb) continue;
-            for (int r = tid; r < rows; r += kConsumerThreads) {
-                const float val = acc_row(part_sums, aset, q, r);
-                a.logits[(size_t)q * p.V + b + r] = val;
-                if (val > bv[q] || (val == bv[q] && b + r < bi[q])) {
-                    bv[q] = val;
-                    bi[q] = b + r;
-                }
-            }
             warp_argmax(bv[q], bi[q]);
             if (lane == 0) {
                 m.bred[q * kConsumerWarps + warp] = bv[q];
@@ -1929,7 +1946,13 @@ __device__ bool ffn_instr_b(const DevParams& p, const StepArgs& a, const int32_t
 #pragma unroll
                         for (int j = 0; j < J; ++j)
 #pragma unroll
-                            for (int k = 0; k < 8; ++k) y[q][j][k] = fmaf(f[u][j][k], hk[u][q], y[q][j][k]);
+                            for (int k = 0; k < 8; k += 2) {
+                                const float2 t = fma2(make_float2(f[u][j][k], f[u][j][k + 1]),
+                                                      make_float2(hk[u][q], hk[u][q]),
+                                                      make_float2(y[q][j][k], y[q][j][k + 1]));
+                                y[q][j][k] = t.x;
+                                y[q][j][k + 1] = t.y;
+                            }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);

@@ -255,7 +255,10 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     };
     const int qd = c.n_q_heads * d;
     const int nb = o.batch;  // every GEMV row keeps nb accumulator sets (one per sequence)
-    auto op_cap = [&](int op) { return std::min(cap, kRowSlots / (acc_sets(op, H, qd, F, c.top_k) * nb)); };
+    auto op_cap = [&](int op) {
+        const int need = row_slots(op, 1, acc_sets(op, H, qd, F, c.top_k), nb);  // slots per row
+        return need > 0 ? std::min(cap, kRowSlots / need) : cap;
+    };
     auto gemv_op = [&](int op, int layer, const std::vector<Segment>& segs, int wait, int signal,
                        const std::vector<double>* weight = nullptr) {
         split_rows(segs, n_sm, op_cap(op), [&](int sm, int sub, int b, int e) {
@@ -492,7 +495,8 @@ int validate(const mk_config& c, const Planned& p) {
             if (op != OP_RMS_QKV && op != OP_MOE_UPGATE && op != OP_MOE_FFN && sub != 0) return MK_ERR_SCHEDULE;
             const int b = w[W_BEGIN], e = w[W_END];
             const int sets = acc_sets(op, c.hidden, c.n_q_heads * d, c.ffn, c.top_k);
-            if (b < 0 || e > R || b >= e || e - b > kMaxRows || (e - b) * sets * nb > kRowSlots) return MK_ERR_SCHEDULE;
+            if (b < 0 || e > R || b >= e || e - b > kMaxRows || row_slots(op, e - b, sets, nb) > kRowSlots)
+                return MK_ERR_SCHEDULE;
             auto& hits = cov[cov_key(l, op, sub)];
             if (hits.empty()) hits.assign(R, 0);
             for (int r = b; r < e; ++r)

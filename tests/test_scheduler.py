@@ -369,7 +369,7 @@ def test_batch_schedule(B, n_sm):
             seen.add(key)
         else:
             sets = 2 if op == OP["FFN"] else 1
-            if op != OP["LM"]:
+            if op != OP["LM"]:  # the LM head goes through its rows in chunks
                 assert (w[W_END] - w[W_BEGIN]) * sets * B <= 1024
     assert len(seen) == cfg.n_layers * B * cfg.n_kv_heads * S
     assert inc[1] == B * cfg.n_kv_heads * S  # layer 0's attention counter
