@@ -69,6 +69,8 @@ def parse():
     ap.add_argument("--ring-stages", type=int, default=0)
     ap.add_argument("--stage-bytes", type=int, default=0)
     ap.add_argument("--kv-splits", type=int, default=0)
+    ap.add_argument("--batch-only", type=int, default=0,
+                    help="profiling: time only batched decode of this many sequences (no headline line)")
     ap.add_argument("--batch-sizes", default="2,4,8",
                     help="batched-decode sizes measured after the headline (comma list; empty: none)")
     ap.add_argument("--spec-experts", type=int, default=-1,
@@ -492,6 +494,9 @@ def run_ours(args, rank, world, local):
     from synth import configs
     cfg, p0, positions = workload(args)
     K, Wm = args.steps, args.warmup
+    if args.batch_only > 1:  # a profiling run of the batched kernel alone
+        b = measure_batch(args, cfg, p0, args.batch_only, K, Wm, world, local)
+        return {"impl": "ours", "batched_only": b} if rank == 0 else None
     r = measure(args, cfg, p0, positions, K, Wm, rank, world, local)
 
     per_config = {}
