@@ -376,6 +376,7 @@ int mk_build_schedule(mk_handle* h) {
     h->plan = plan;
     h->variant = h->opt.general_kernel ? 0 : mk::megakernel_variant(h->p, plan.fused_ffn);
     if (h->variant < 0) return MK_ERR_UNSUPPORTED;  // no kernel instantiation for this batch
+    h->p.row_pad = mk::megakernel_row_pad(h->variant);
     // the prediction runs in the specialised MoE kernels (the general one keeps the prefetch cursor)
     h->p.spec_experts = h->variant != 0 && plan.fused_ffn && h->cfg.n_experts > 0 ? h->opt.spec_experts : 0;
     int32_t* words = nullptr;

@@ -194,6 +194,12 @@ __device__ __forceinline__ float dot8(const uint4 w, const float* v, float acc) 
     acc = fmaf(bf_hi(w.w), v[7], acc);
     return acc;
 }
+// Two fp32 values as bf16x2 (x0 in the low half), each rounded to nearest even: one cvt.
+__device__ __forceinline__ uint32_t pack_bf16x2(float x0, float x1) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(x1), "f"(x0));
+    return d;
+}
 // fp32 -> bf16 bits, round to nearest even
 __device__ __forceinline__ uint32_t f2bf(float f) {
     uint32_t u = __float_as_uint(f);

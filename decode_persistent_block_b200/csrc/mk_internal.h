@@ -115,6 +115,11 @@ MK_HD inline int lm_chunk_rows(int nb, int rps) {
     return c > rps ? c : rps;
 }
 
+// Batched decode: the one-chunk kernel with 8 sequence slots runs its GEMVs on the tensor cores
+// (stages of padded rows); the other batched kernels keep the CUDA-core form, which measured
+// faster there (the tensor-core form's per-instruction prologues cost more than it saves).
+MK_HD constexpr bool batch_on_tensor_cores(int J, int NB) { return J == 1 && NB == 8; }
+
 MK_HD inline int row_slots(int op, int rows, int sets, int nb) {
     return op == OP_LMHEAD_ARGMAX && nb > 1 ? 0 : rows * sets * nb;
 }
@@ -201,6 +206,7 @@ struct DevParams {
     // batched decode: nb sequences per step; every activation below, the logits, the snapshots and
     // the KV caches hold nb per-sequence copies one after the other (strides in elements below)
     int nb;
+    int row_pad;            // bytes between weight rows in a stage beyond the row (tensor-core batched kernel: 16)
     size_t kv_seq_stride;   // L * nkv * max_seq * d
     int32_t* next_tok;      // [kMaxBatch] each sequence's argmax of the last step
     // activations (fp32)

@@ -25,6 +25,8 @@ cudaError_t prepare_megakernel(int ring_stages, int stage_bytes, int* max_blocks
 // has that many 8-column chunks per consumer thread (fused FFN, no optional L2
 // prefetch), else 0 (the general kernel).
 int megakernel_variant(const DevParams& p, bool fused_ffn);
+// Bytes between the weight rows of a ring stage beyond the row, for instantiation `variant`.
+int megakernel_row_pad(int variant);
 cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, int variant, cudaStream_t stream);
 
 // dst[c][r] = src[r][c] for a row-major bf16 matrix of rows x cols (one-time,

@@ -215,13 +215,15 @@ struct Plan {
     int rps;        // rows per stage
     int spp;        // stages per phase
     uint32_t row_bytes;   // bytes of one row part in shared memory
+    uint32_t pitch;       // bytes between consecutive rows in the stage (batched decode: row_bytes + 16,
+                          // so that the 8 rows of an ldmatrix tile fall in different banks)
     uint32_t src_stride;  // bytes between consecutive rows in global memory
     const unsigned char* src[kMaxTopK][2];  // [slot][span]: row 0 of the instruction, column 0
     // fused FFN: after the main stages, `tail_spp` stages of the transposed
     // down-projection rows (one span, whole rows of tail_row_bytes)
     int main_stages;
     int tail_rps, tail_spp;
-    uint32_t tail_row_bytes;
+    uint32_t tail_row_bytes, tail_pitch;
     const unsigned char* tail_src;
     int tma_row0;  // attention: first cache row of the split in the tensor maps' row space (-1: not attention)
 };
@@ -259,7 +261,7 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
     pl.kparts = 1;
     pl.src[0][1] = pl.src[1][0] = pl.src[1][1] = nullptr;
     pl.tail_rps = pl.tail_spp = 0;
-    pl.tail_row_bytes = 0;
+    pl.tail_row_bytes = pl.tail_pitch = 0;
     pl.tail_src = nullptr;
     pl.tma_row0 = -1;
     const uint16_t* tail = nullptr;  // transposed down-projection rows of a fused FFN
@@ -274,7 +276,7 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
             pl.nphase = 1;
             pl.nspan = 2;
             pl.rows = r.ncached;
-            pl.row_bytes = pl.src_stride = (uint32_t)p.d * 2u;
+            pl.row_bytes = pl.src_stride = pl.pitch = (uint32_t)p.d * 2u;
             pl.rps = attn_stage_rows((int)SB, p.d);
             pl.spp = (pl.rows + pl.rps - 1) / pl.rps;
             pl.n_stages = pl.main_stages = pl.spp;
@@ -320,13 +322,16 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
     pl.rows = e - b;
     pl.src_stride = (uint32_t)K * 2u;
     pl.row_bytes = pl.src_stride / (uint32_t)pl.kparts;
-    const int rps = (int)(SB / ((uint32_t)pl.nspan * pl.row_bytes));
+    const uint32_t pad = (uint32_t)p.row_pad;  // tensor-core batched kernel: padded rows
+    pl.pitch = pl.row_bytes + pad;
+    const int rps = (int)(SB / ((uint32_t)pl.nspan * pl.pitch));
     pl.rps = rps < pl.rows ? rps : pl.rows;
     pl.spp = (pl.rows + pl.rps - 1) / pl.rps;
     pl.n_stages = pl.main_stages = pl.spp * pl.nphase;
     if (tail) {
         pl.tail_row_bytes = (uint32_t)p.H * 2u;
-        const int trps = (int)(SB / pl.tail_row_bytes);
+        pl.tail_pitch = pl.tail_row_bytes + pad;
+        const int trps = (int)(SB / pl.tail_pitch);
         pl.tail_rps = trps < pl.rows ? trps : pl.rows;
         pl.tail_spp = (pl.rows + pl.tail_rps - 1) / pl.tail_rps;
         pl.tail_src = (const unsigned char*)(tail + (size_t)b * p.H);
@@ -359,7 +364,7 @@ __device__ __forceinline__ bool needs_routing(int op) {
 // ---------------------------------------------------------------------------
 // TC: attention stages are tensor-map boxes (for attn_tc); otherwise contiguous
 // K and V spans (for attn_cc).
-template <bool TC>
+template <bool TC, int NB = 1>
 __device__ void issue_stage(const DevParams& p, const Plan& pl, int st, unsigned char* dst_stage, uint64_t* bar) {
     if (TC && pl.tma_row0 >= 0) {  // attention: K and V in boxes of attn_box_rows rows (past the split: masked)
         const int halves = p.d / 64, y = pl.tma_row0 + st * pl.rps;
@@ -386,7 +391,13 @@ __device__ void issue_stage(const DevParams& p, const Plan& pl, int st, unsigned
         const int nr = (pl.rows - r0) < pl.tail_rps ? (pl.rows - r0) : pl.tail_rps;
         const uint32_t bytes = (uint32_t)nr * pl.tail_row_bytes;
         mbar_arrive_expect_tx(bar, bytes);
-        bulk_g2s_hint(dst_stage, pl.tail_src + (size_t)r0 * pl.tail_row_bytes, bytes, bar, pol);
+        if (NB > 1 && pl.tail_pitch != pl.tail_row_bytes) {  // padded rows
+            for (int r = 0; r < nr; ++r)
+                bulk_g2s_hint(dst_stage + (size_t)r * pl.tail_pitch, pl.tail_src + (size_t)(r0 + r) * pl.tail_row_bytes,
+                              pl.tail_row_bytes, bar, pol);
+        } else {
+            bulk_g2s_hint(dst_stage, pl.tail_src + (size_t)r0 * pl.tail_row_bytes, bytes, bar, pol);
+        }
         return;
     }
     const int ph = st / pl.spp, sst = st % pl.spp;
@@ -397,9 +408,12 @@ __device__ void issue_stage(const DevParams& p, const Plan& pl, int st, unsigned
     mbar_arrive_expect_tx(bar, bytes * (uint32_t)pl.nspan);
     for (int s = 0; s < pl.nspan; ++s) {
         const unsigned char* src = pl.src[slot][s] + (size_t)r0 * pl.src_stride + (size_t)part * pl.row_bytes;
-        unsigned char* dst = dst_stage + (size_t)s * pl.rps * pl.row_bytes;
+        unsigned char* dst = dst_stage + (size_t)s * pl.rps * pl.pitch;
         const bool kv = pl.tma_row0 >= 0;  // K/V rows of an attention split (contiguous-copy path)
-        if (pl.kparts == 1) {
+        if (NB > 1 && !kv && pl.pitch != pl.row_bytes) {  // tensor-core batched kernel: padded rows
+            for (int r = 0; r < nr; ++r)
+                bulk_g2s_hint(dst + (size_t)r * pl.pitch, src + (size_t)r * pl.src_stride, pl.row_bytes, bar, pol);
+        } else if (pl.kparts == 1) {
             if (kv) bulk_g2s(dst, src, bytes, bar);
             else bulk_g2s_hint(dst, src, bytes, bar, pol);
         } else {
@@ -536,7 +550,7 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                         sok = false;
                         break;
                     }
-                    issue_stage<TC>(p, sp, st, ring + (size_t)slot * SB, &full[slot]);
+                    issue_stage<TC, NB>(p, sp, st, ring + (size_t)slot * SB, &full[slot]);
                     if (st == 0 && p.trace)
                         p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_LD_FIRST] = globaltimer_ns();
                     used |= 1u << slot;
@@ -562,7 +576,7 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                 ok = false;
                 break;
             }
-            issue_stage<TC>(p, pl, st, ring + (size_t)slot * SB, &full[slot]);
+            issue_stage<TC, NB>(p, pl, st, ring + (size_t)slot * SB, &full[slot]);
             // Head start of a long stream: the loader reaches the first stage of the
             // dense FFN (or the LM head) while the consumers still wait on the small
             // ops before it and HBM is mostly idle.  The stages that follow the
@@ -1407,6 +1421,221 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
 // ---------------------------------------------------------------------------
 // consumers: batched decode (NB > 1 sequences per step, nb of them in use)
 // ---------------------------------------------------------------------------
+// A batched GEMV is a skinny GEMM, y[row][q] = sum_k W[row][k] x_q[k], so it
+// runs on the tensor cores: each ring stage's rows (stored at a pitch of
+// row_bytes + 16, so the 8 rows of an ldmatrix tile fall in different banks)
+// are the A operand of m16n8k16 bf16 MMAs whose N dimension is the 8 sequence
+// slots (unused slots hold zeros).  Warp w takes columns [w K/8, (w + 1) K/8)
+// of every row.  The fp32 activations enter as bf16 high and low parts (x = hi
+// + lo to about 16 mantissa bits), two MMAs per k-step, fp32 accumulation.
+
+// x0, x1 as bf16x2 high parts (rounded to nearest) and the bf16x2 of what the
+// high parts leave (x0 in the low half of each word).
+__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    hi = pack_bf16x2(x0, x1);
+    lo = pack_bf16x2(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xFFFF0000u));
+}
+
+// B fragments of one warp's k-range for the 8 sequence slots: lane (g, t) =
+// (lane / 4, lane % 4) holds sequence g's columns kb + 2t, 2t + 1 (word 0) and
+// kb + 2t + 8, 2t + 9 (word 1) of every k-step of 16 columns, high and low parts.
+template <int KS>
+struct BFrag {
+    uint32_t hi[KS][2], lo[KS][2];
+};
+
+// The sequences' input vectors, held in the CUDA-core layout (thread tid: the
+// 8-column chunks tid + 256 j), rearranged into B fragments through the
+// scratch, as many sequences per pass as fit.
+template <int J, int NB, int KS>
+__device__ __forceinline__ void to_bfrag(const float (&v)[NB][J][8], int K, float* scratch, BFrag<KS>& bf, int lane,
+                                         int warp) {
+    const int tid = threadIdx.x, g = lane >> 2, t = lane & 3, nch = K >> 3;
+    const int SP = kRowSlots * kConsumerWarps / K;  // sequences per pass
+    const int kw = K / kConsumerWarps, ksr = kw / 16;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) bf.hi[ks][0] = bf.hi[ks][1] = bf.lo[ks][0] = bf.lo[ks][1] = 0u;
+    for (int p0 = 0; p0 < NB; p0 += SP) {
+#pragma unroll
+        for (int q = 0; q < NB; ++q) {
+            if (q < p0 || q >= p0 + SP) continue;
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int c = tid + kConsumerThreads * j;
+                if (c < nch) {
+                    float4* dst = reinterpret_cast<float4*>(scratch + (size_t)(q - p0) * K) + 2 * c;
+                    dst[0] = make_float4(v[q][j][0], v[q][j][1], v[q][j][2], v[q][j][3]);
+                    dst[1] = make_float4(v[q][j][4], v[q][j][5], v[q][j][6], v[q][j][7]);
+                }
+            }
+        }
+        cbar();
+        if (g >= p0 && g < p0 + SP) {
+            const float* src = scratch + (size_t)(g - p0) * K + warp * kw + 2 * t;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                if (ks >= ksr) continue;  // (not break: the unrolled loop keeps static indices)
+                const float2 x = *reinterpret_cast<const float2*>(src + 16 * ks);
+                const float2 y = *reinterpret_cast<const float2*>(src + 16 * ks + 8);
+                split_pack(x.x, x.y, bf.hi[ks][0], bf.lo[ks][0]);
+                split_pack(y.x, y.y, bf.hi[ks][1], bf.lo[ks][1]);
+            }
+        }
+        cbar();
+    }
+}
+
+// The nb sequences' RMSNorm-ed inputs straight into B fragments (no detour
+// through the CUDA-core layout): lane (g, t) of warp w loads sequence g's
+// columns of its k-steps (x fp32 at x32 + g H, or the bf16 embedding row of
+// the sequence's token when from_embed) and the norm weights there; the
+// sums of squares of each sequence meet in one block reduction; the scaled
+// values are split into bf16 high and low parts.  snap (optional): sequence
+// g's un-normalised input is stored at snap + g * snap_stride.
+template <int KS>
+__device__ __forceinline__ void rms_bfrag(const DevParams& p, Misc& m, const float* x32, bool from_embed,
+                                          const uint16_t* nw, BFrag<KS>& bf, float* snap, size_t snap_stride,
+                                          int lane, int warp) {
+    const int K = p.H, g = lane >> 2, t = lane & 3, ksr = K / (16 * kConsumerWarps);
+    const int c0 = warp * (K / kConsumerWarps) + 2 * t;
+    const bool live = g < p.nb;
+    float x[KS][4];
+    uint32_t wn[KS][2];
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+        x[ks][0] = x[ks][1] = x[ks][2] = x[ks][3] = 0.f;
+        wn[ks][0] = wn[ks][1] = 0u;
+        if (ks >= ksr) continue;
+        const int c = c0 + 16 * ks;
+        wn[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(nw + c));
+        wn[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(nw + c + 8));
+        if (!live) continue;
+        if (from_embed) {
+            const uint16_t* e = p.embed + (size_t)m.btok[g] * K + c;
+            const uint32_t e0 = __ldg(reinterpret_cast<const uint32_t*>(e));
+            const uint32_t e1 = __ldg(reinterpret_cast<const uint32_t*>(e + 8));
+            x[ks][0] = __uint_as_float(e0 << 16);
+            x[ks][1] = __uint_as_float(e0 & 0xFFFF0000u);
+            x[ks][2] = __uint_as_float(e1 << 16);
+            x[ks][3] = __uint_as_float(e1 & 0xFFFF0000u);
+        } else {
+            const float* src = x32 + (size_t)g * K + c;
+            const float2 a = __ldcg(reinterpret_cast<const float2*>(src));
+            const float2 b = __ldcg(reinterpret_cast<const float2*>(src + 8));
+            x[ks][0] = a.x;
+            x[ks][1] = a.y;
+            x[ks][2] = b.x;
+            x[ks][3] = b.y;
+        }
+    }
+    if (snap && live) {
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            if (ks >= ksr) continue;
+            float* dst = snap + (size_t)g * snap_stride + c0 + 16 * ks;
+            *reinterpret_cast<float2*>(dst) = make_float2(x[ks][0], x[ks][1]);
+            *reinterpret_cast<float2*>(dst + 8) = make_float2(x[ks][2], x[ks][3]);
+        }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ss = fmaf(x[ks][e], x[ks][e], ss);
+    ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 1);  // the 4 lanes of sequence g in this warp
+    ss += __shfl_xor_sync(0xFFFFFFFFu, ss, 2);
+    if (t == 0) m.bred[g * kConsumerWarps + warp] = ss;
+    cbar();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) tot += m.bred[g * kConsumerWarps + w];
+    const float rs = live ? 1.0f / sqrtf(tot / (float)K + p.eps) : 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+        const float w0 = __uint_as_float(wn[ks][0] << 16), w1 = __uint_as_float(wn[ks][0] & 0xFFFF0000u);
+        const float w2 = __uint_as_float(wn[ks][1] << 16), w3 = __uint_as_float(wn[ks][1] & 0xFFFF0000u);
+        split_pack(x[ks][0] * rs * w0, x[ks][1] * rs * w1, bf.hi[ks][0], bf.lo[ks][0]);
+        split_pack(x[ks][2] * rs * w2, x[ks][3] * rs * w3, bf.hi[ks][1], bf.lo[ks][1]);
+    }
+    cbar();  // m.bred free again
+}
+
+// Rows [0, nr) of one span of a stage (pitch bytes apart) against the 8
+// sequence slots, 16 rows per MMA tile: this warp's k-range in k-steps of two
+// MMAs (high and low activation parts).  The warp's row sums land in each
+// sequence's accumulator set, A + q * aset at [row][warp], as the CUDA-core
+// consumers' do (the epilogue adds the 8 warps in order).
+template <int KS>
+__device__ __forceinline__ void stage_rows_tc(const unsigned char* Ws, uint32_t pitch, int nr, int K,
+                                              const BFrag<KS>& bf, float* A, int aset, int nb, int lane, int warp) {
+    const int g = lane >> 2, t = lane & 3, ksr = K / (16 * kConsumerWarps);
+    const uint32_t col = (uint32_t)(warp * (K / kConsumerWarps) + (lane >> 4) * 8) * 2u;
+    for (int m0 = 0; m0 < nr; m0 += 16) {
+        // ldmatrix x4: matrices (rows m0..m0+7 | m0+8..m0+15) x (k 0..7 | 8..15); lane l gives row l % 16
+        // (rows past nr read the last row; their sums are dropped)
+        const int ar = m0 + (lane & 15) < nr ? m0 + (lane & 15) : nr - 1;
+        const uint32_t base = smem_u32(Ws) + (uint32_t)ar * pitch + col;
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            if (ks >= ksr) continue;  // (not break: the unrolled loop keeps static indices)
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(base + 32u * ks, a0, a1, a2, a3);
+            mma_bf16(c, a0, a1, a2, a3, bf.hi[ks][0], bf.hi[ks][1]);
+            mma_bf16(c, a0, a1, a2, a3, bf.lo[ks][0], bf.lo[ks][1]);
+        }
+        // c0, c1: row m0 + g, sequences 2t, 2t + 1; c2, c3: row m0 + g + 8
+        const int q = 2 * t, w = warp;
+        if (m0 + g < nr) {
+            if (q < nb) A[(size_t)q * aset + (m0 + g) * kConsumerWarps + w] = c[0];
+            if (q + 1 < nb) A[(size_t)(q + 1) * aset + (m0 + g) * kConsumerWarps + w] = c[1];
+        }
+        if (m0 + g + 8 < nr) {
+            if (q < nb) A[(size_t)q * aset + (m0 + g + 8) * kConsumerWarps + w] = c[2];
+            if (q + 1 < nb) A[(size_t)(q + 1) * aset + (m0 + g + 8) * kConsumerWarps + w] = c[3];
+        }
+    }
+}
+
+// Transposed down-projection rows [0, nr) of one stage (pitch bytes apart)
+// into this warp's output columns: y[col][q] += sum_r Wt[r][col] h[r][q] for
+// the warp's H/8 columns in MT tiles of 16 (A = Wt^T through ldmatrix.trans,
+// B = h of 16 rows for the 8 sequence slots, high and low parts).  h holds the
+// stage's rows at h[r * hstride + q], zero for unused sequences.
+template <int MT>
+__device__ __forceinline__ void down_rows_tc(const unsigned char* Ws, uint32_t pitch, int nr, int H, const float* h,
+                                             int hstride, int nb, float (&y)[MT][4], int lane, int warp) {
+    const int g = lane >> 2, t = lane & 3, mtr = H / (16 * kConsumerWarps);
+    const uint32_t col = (uint32_t)(warp * (H / kConsumerWarps) + 8 * ((lane >> 3) & 1)) * 2u;
+    for (int k0 = 0; k0 < nr; k0 += 16) {
+        auto hv = [&](int r) { return (k0 + r < nr && g < nb) ? h[(size_t)(k0 + r) * hstride + g] : 0.f; };
+        uint32_t bh0, bl0, bh1, bl1;
+        split_pack(hv(2 * t), hv(2 * t + 1), bh0, bl0);
+        split_pack(hv(2 * t + 8), hv(2 * t + 9), bh1, bl1);
+        // ldmatrix.trans x4: matrices (cols 0..7 | 8..15) x (rows k0..k0+7 | k0+8..k0+15) of the stage;
+        // lane l gives stage row k0 + l % 8 + 8 (l / 16) at column block 8 ((l / 8) % 2)
+        const int r = k0 + (lane & 7) + 8 * (lane >> 4);
+        const uint32_t base = smem_u32(Ws) + (uint32_t)(r < nr ? r : nr - 1) * pitch + col;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            if (mt >= mtr) continue;  // (not break: the unrolled loop keeps static indices)
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_trans(base + 32u * mt, a0, a1, a2, a3);
+            mma_bf16(y[mt], a0, a1, a2, a3, bh0, bh1);
+            mma_bf16(y[mt], a0, a1, a2, a3, bl0, bl1);
+        }
+    }
+}
+
+// Row sum r of accumulator set k (one per sequence and span): the 8 warps'
+// partial sums in fixed order.
+__device__ __forceinline__ float acc_row(const float* part_sums, int aset, int k, int r) {
+    const float4* ps = reinterpret_cast<const float4*>(part_sums + (size_t)k * aset + (size_t)r * kConsumerWarps);
+    const float4 x0 = ps[0], x1 = ps[1];
+    return ((x0.x + x0.y) + (x0.z + x0.w)) + ((x1.x + x1.y) + (x1.z + x1.w));
+}
+
+// CUDA-core form of the batched GEMV (small batches, and the two-chunk kernels):
 // RG rows [rg, rg + RG) of a stage against the sequences' input vectors: the
 // rows' weights are loaded and widened to fp32 once, then every sequence's dot
 // products reuse them (all NB, the unused ones against zero vectors, so the
@@ -1454,14 +1683,6 @@ __device__ __forceinline__ void stage_rows_b(const uint4* __restrict__ Ws, int r
 #pragma unroll
     for (int j = 0; j < J; ++j) jv[j] = (int)threadIdx.x + kConsumerThreads * j < nch;
     for (int rg = 0; rg < nr; rg += RG) rows_block_b<J, RG, NB>(Ws, row16, rg, nr, jv, v, A, aset, nb, lane);
-}
-
-// Row sum r of accumulator set k (one per sequence and span): the 8 warps'
-// partial sums in fixed order.
-__device__ __forceinline__ float acc_row(const float* part_sums, int aset, int k, int r) {
-    const float4* ps = reinterpret_cast<const float4*>(part_sums + (size_t)k * aset + (size_t)r * kConsumerWarps);
-    const float4 x0 = ps[0], x1 = ps[1];
-    return ((x0.x + x0.y) + (x0.z + x0.w)) + ((x1.x + x1.y) + (x1.z + x1.w));
 }
 
 // v[q] = rmsnorm(x_q) * w for the nb sequences of a batched step (x_q fp32 at
@@ -1627,7 +1848,9 @@ __device__ void load_attn_merged_b(const DevParams& p, int K, float (&v)[NB][J][
 template <int J, int NB>
 __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                              uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
-    constexpr int RG = J == 1 ? 4 : 2;
+    constexpr int KS = J == 1 ? 16 : 24;  // k-steps of 16 columns per warp at the widest row (2048 or 3072)
+    constexpr bool TCP = batch_on_tensor_cores(J, NB);
+    constexpr int RG = J == 1 ? 4 : 2;    // CUDA-core form: rows per block
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nb = p.nb;
     const int op = w[W_OP], l = w[W_LAYER], sub = w[W_SUB], b = w[W_BEGIN], rows = w[W_END] - b;
     const uint32_t SB = (uint32_t)p.stage_bytes;
@@ -1655,23 +1878,36 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
     cbar();
     if (vload(&m.abort_flag)) return false;
 
-    // input vectors of the sequences
+    // input vectors of the sequences: as the MMAs' B operand (tensor cores), or per thread chunk
+    BFrag<KS> bf;
     float v[NB][J][8];
     const uint16_t* const* wt = p.wt + (size_t)(l < p.L ? l : 0) * wt_stride(p.E);
     const int K = op == OP_OPROJ_RES ? p.nq * p.d : p.H;
     const size_t snap_stride = (size_t)(p.L + 1) * H;
-    if (op == OP_RMS_QKV)
-        load_rms_b<J, NB>(p, m, p.x2, l == 0, wt[WT_ATTN_NORM], v,
-                          (p.snap && l > 0 && sub == 0 && b == 0) ? p.snap + (size_t)l * H : nullptr, snap_stride);
-    else if (op == OP_LMHEAD_ARGMAX)
-        load_rms_b<J, NB>(p, m, p.x2, p.L == 0, p.final_norm, v,
-                          (p.snap && w[W_SEQ] == 0) ? p.snap + (size_t)p.L * H : nullptr, snap_stride);
-    else
+    if constexpr (!TCP) {
+        if (op == OP_RMS_QKV)
+            load_rms_b<J, NB>(p, m, p.x2, l == 0, wt[WT_ATTN_NORM], v,
+                              (p.snap && l > 0 && sub == 0 && b == 0) ? p.snap + (size_t)l * H : nullptr,
+                              snap_stride);
+        else if (op == OP_LMHEAD_ARGMAX)
+            load_rms_b<J, NB>(p, m, p.x2, p.L == 0, p.final_norm, v,
+                              (p.snap && w[W_SEQ] == 0) ? p.snap + (size_t)p.L * H : nullptr, snap_stride);
+        else
+            load_attn_merged_b<J, NB>(p, K, v);
+    } else if (op == OP_RMS_QKV) {
+        rms_bfrag<KS>(p, m, p.x2, l == 0, wt[WT_ATTN_NORM], bf,
+                      (p.snap && l > 0 && sub == 0 && b == 0) ? p.snap + (size_t)l * H : nullptr, snap_stride, lane,
+                      warp);
+    } else if (op == OP_LMHEAD_ARGMAX) {
+        rms_bfrag<KS>(p, m, p.x2, p.L == 0, p.final_norm, bf,
+                      (p.snap && w[W_SEQ] == 0) ? p.snap + (size_t)p.L * H : nullptr, snap_stride, lane, warp);
+    } else {  // the merged attention output, through the CUDA-core layout
         load_attn_merged_b<J, NB>(p, K, v);
+        to_bfrag<J, NB, KS>(v, K, scratch, bf, lane, warp);
+    }
     if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
 
     // stages
-    const int nch = K >> 3;
     for (int sst = 0; sst < pl.spp; ++sst) {
         const int r0 = sst * pl.rps;
         const int nr = (rows - r0) < pl.rps ? (rows - r0) : pl.rps;
@@ -1680,9 +1916,13 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
                 if (tr && sst == 0) tr[T_FIRST] = globaltimer_ns();
                 stage_stamp(tr, T_SREADY, sst);
             }
-            const uint4* Ws = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
-            stage_rows_b<J, RG, NB>(Ws, (int)(pl.row_bytes >> 4), nr, nch, v,
-                                    part_sums + (size_t)(r0 % chunk) * kConsumerWarps, aset, nb, lane);
+            if constexpr (TCP)
+                stage_rows_tc<KS>(ring + (size_t)slot * SB, pl.pitch, nr, K, bf,
+                                  part_sums + (size_t)(r0 % chunk) * kConsumerWarps, aset, nb, lane, warp);
+            else
+                stage_rows_b<J, RG, NB>(reinterpret_cast<const uint4*>(ring + (size_t)slot * SB), (int)(pl.pitch >> 4),
+                                        nr, K >> 3, v, part_sums + (size_t)(r0 % chunk) * kConsumerWarps, aset, nb,
+                                        lane);
             __syncwarp();
             if (tid == 0) stage_stamp(tr, T_SDONE, sst);
             if (lane == 0) mbar_arrive(&empty[slot]);
@@ -1700,7 +1940,7 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
             if (vload(&m.abort_flag)) return false;
 #pragma unroll
             for (int q = 0; q < NB; ++q) {
-                if (q >= nb) break;
+                if (q >= nb) continue;  // (not break: the unrolled loop keeps static indices)
                 for (int r = tid; r < cn; r += kConsumerThreads) {
                     const float val = acc_row(part_sums, aset, q, r);
                     const int row = b + c0 + r;
@@ -1740,7 +1980,7 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
             }
 #pragma unroll
             for (int q = 0; q < NB; ++q) {
-                if (q >= nb) break;
+                if (q >= nb) continue;  // (not break: the unrolled loop keeps static indices)
                 const size_t i = q * H + b + r;
                 if (l == 0 && p.snap) p.snap[(size_t)q * (p.L + 1) * H + b + r] = base[q];
                 const float nx = base[q] + acc_row(part_sums, aset, q, r);
@@ -1831,8 +2071,10 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
 template <int J, int NB>
 __device__ bool ffn_instr_b(const DevParams& p, const StepArgs& a, const int32_t* w, int ii, unsigned char* ring,
                             uint64_t* full, uint64_t* empty, float* scratch, Misc& m, int& slot, uint32_t& phase) {
-    constexpr int RG = J == 1 ? 4 : 2;
-    const int tid = threadIdx.x, lane = tid & 31, nb = p.nb;
+    constexpr int KS = J == 1 ? 16 : 24;  // k-steps per warp (up/gate) and column tiles per warp (down) at the widest row
+    constexpr bool TCP = batch_on_tensor_cores(J, NB);
+    constexpr int RG = J == 1 ? 4 : 2;    // CUDA-core form: rows per block
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nb = p.nb;
     const int op = w[W_OP], l = w[W_LAYER], b = w[W_BEGIN], rows = w[W_END] - b;
     const uint32_t SB = (uint32_t)p.stage_bytes;
     const size_t H = (size_t)p.H;
@@ -1847,11 +2089,15 @@ __device__ bool ffn_instr_b(const DevParams& p, const StepArgs& a, const int32_t
     cbar();
     if (vload(&m.abort_flag)) return false;
 
-    float v[NB][J][8];
     const uint16_t* const* wt = p.wt + (size_t)l * wt_stride(p.E);
-    load_rms_b<J, NB>(p, m, p.x, false, wt[WT_FFN_NORM], v);
-    if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
+    BFrag<KS> bf;
+    float v[NB][J][8];
+    if constexpr (TCP)
+        rms_bfrag<KS>(p, m, p.x, false, wt[WT_FFN_NORM], bf, nullptr, 0, lane, warp);
+    else
+        load_rms_b<J, NB>(p, m, p.x, false, wt[WT_FFN_NORM], v);
     const int nch = p.H >> 3;
+    if (tr && tid == 0) tr[T_READY] = globaltimer_ns();
 
     // up/gate rows (gate span, then up span, of each stage)
     for (int sst = 0; sst < pl.spp; ++sst) {
@@ -1864,9 +2110,13 @@ __device__ bool ffn_instr_b(const DevParams& p, const StepArgs& a, const int32_t
             }
             const unsigned char* stage = ring + (size_t)slot * SB;
             for (int s = 0; s < 2; ++s) {
-                const uint4* Ws = reinterpret_cast<const uint4*>(stage + (size_t)s * pl.rps * pl.row_bytes);
-                stage_rows_b<J, RG, NB>(Ws, (int)(pl.row_bytes >> 4), nr, nch, v,
-                                        part_sums + ((size_t)s * nb * rows + r0) * kConsumerWarps, aset, nb, lane);
+                float* A = part_sums + ((size_t)s * nb * rows + r0) * kConsumerWarps;
+                if constexpr (TCP)
+                    stage_rows_tc<KS>(stage + (size_t)s * pl.rps * pl.pitch, pl.pitch, nr, p.H, bf, A, aset, nb, lane,
+                                      warp);
+                else
+                    stage_rows_b<J, RG, NB>(reinterpret_cast<const uint4*>(stage + (size_t)s * pl.rps * pl.pitch),
+                                            (int)(pl.pitch >> 4), nr, nch, v, A, aset, nb, lane);
             }
             __syncwarp();
             if (tid == 0) stage_stamp(tr, T_SDONE, sst);
@@ -1908,73 +2158,127 @@ __device__ bool ffn_instr_b(const DevParams& p, const StepArgs& a, const int32_t
         }
     cbar();
 
-    // transposed down-projection rows: this thread's column chunks of Wd[:, rows] h_q, every q
-    float y[NB][J][8];
-    bool jv[J];
-#pragma unroll
-    for (int j = 0; j < J; ++j) jv[j] = tid + kConsumerThreads * j < nch;
-#pragma unroll
-    for (int q = 0; q < NB; ++q)
-#pragma unroll
-        for (int j = 0; j < J; ++j)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) y[q][j][k] = 0.f;
-    for (int tst = 0; tst < pl.tail_spp; ++tst) {
-        const int r0 = tst * pl.tail_rps;
-        const int nr = (rows - r0) < pl.tail_rps ? (rows - r0) : pl.tail_rps;
-        if (warp_wait_full(&full[slot], phase, p, m, ii, op)) {
-            if (tid == 0) stage_stamp(tr, T_SREADY, pl.spp + tst);
-            const uint4* Ws = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
-            // two rows per iteration (the unused sequences' h are zero)
-            for (int r = 0; r < nr; r += 2) {
-                float f[2][J][8], hk[2][NB];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const bool live = r + u < nr;
-#pragma unroll
-                    for (int j = 0; j < J; ++j)
-                        unpack8((live && jv[j]) ? Ws[(r + u) * nch + tid + kConsumerThreads * j]
-                                                : make_uint4(0u, 0u, 0u, 0u),
-                                f[u][j]);
-#pragma unroll
-                    for (int q = 0; q < NB; ++q) hk[u][q] = live ? scratch[(size_t)(r0 + r + u) * NB + q] : 0.f;
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-#pragma unroll
-                    for (int q = 0; q < NB; ++q)
-#pragma unroll
-                        for (int j = 0; j < J; ++j)
-#pragma unroll
-                            for (int k = 0; k < 8; k += 2) {
-                                const float2 t = fma2(make_float2(f[u][j][k], f[u][j][k + 1]),
-                                                      make_float2(hk[u][q], hk[u][q]),
-                                                      make_float2(y[q][j][k], y[q][j][k + 1]));
-                                y[q][j][k] = t.x;
-                                y[q][j][k + 1] = t.y;
-                            }
+    if constexpr (TCP) {
+        // transposed down-projection rows on the tensor cores: this warp's columns of Wd[:, rows] h_q
+        float y[KS][4];
+    #pragma unroll
+        for (int mt = 0; mt < KS; ++mt) y[mt][0] = y[mt][1] = y[mt][2] = y[mt][3] = 0.f;
+        for (int tst = 0; tst < pl.tail_spp; ++tst) {
+            const int r0 = tst * pl.tail_rps;
+            const int nr = (rows - r0) < pl.tail_rps ? (rows - r0) : pl.tail_rps;
+            if (warp_wait_full(&full[slot], phase, p, m, ii, op)) {
+                if (tid == 0) stage_stamp(tr, T_SREADY, pl.spp + tst);
+                down_rows_tc<KS>(ring + (size_t)slot * SB, pl.tail_pitch, nr, p.H, scratch + (size_t)r0 * NB, NB, nb, y,
+                                 lane, warp);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[slot]);
+            } else if (tid == 0) {
+                vstore(&m.abort_flag, 1);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
-        } else if (tid == 0) {
-            vstore(&m.abort_flag, 1);
+            if (++slot == p.ring_stages) {
+                slot = 0;
+                phase ^= 1u;
+            }
         }
-        if (++slot == p.ring_stages) {
-            slot = 0;
-            phase ^= 1u;
+        cbar();
+        if (vload(&m.abort_flag)) return false;
+        // Into the residuals: the warps' tiles go through the scratch, as many sequences per pass as
+        // fit, and leave as float4 atomics over contiguous columns.  Lane (g, t) holds, per tile mt,
+        // columns c = 16 mt + g and c + 8 for sequences 2t and 2t + 1.
+        {
+            const int g = lane >> 2, t = lane & 3, mtr = p.H / (16 * kConsumerWarps);
+            const int SP = kRowSlots * kConsumerWarps / p.H, H4 = p.H / 4;
+            for (int p0 = 0; p0 < nb; p0 += SP) {
+    #pragma unroll
+                for (int mt = 0; mt < KS; ++mt) {
+                    if (mt >= mtr) continue;  // (not break: the unrolled loop keeps static indices)
+                    const int c = warp * (p.H / kConsumerWarps) + 16 * mt + g;
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q = 2 * t + (e & 1) - p0;
+                        if (q >= 0 && q < SP) scratch[(size_t)q * H + c + 8 * (e >> 1)] = y[mt][e];
+                    }
+                }
+                cbar();
+                const int n4 = (nb - p0 < SP ? nb - p0 : SP) * H4;
+                for (int i = tid; i < n4; i += kConsumerThreads) {
+                    const int q = i / H4;
+                    atomicAdd(reinterpret_cast<float4*>(p.x2 + (p0 + q) * H) + (i - q * H4),
+                              reinterpret_cast<const float4*>(scratch)[i]);
+                }
+                cbar();
+            }
         }
-    }
-    cbar();
-    if (vload(&m.abort_flag)) return false;
-#pragma unroll
-    for (int q = 0; q < NB; ++q) {
-        if (q >= nb) break;
-#pragma unroll
-        for (int j = 0; j < J; ++j) {
-            if (!jv[j]) continue;
-            float4* dst = reinterpret_cast<float4*>(p.x2 + q * H) + 2 * (tid + kConsumerThreads * j);
-            atomicAdd(dst, make_float4(y[q][j][0], y[q][j][1], y[q][j][2], y[q][j][3]));
-            atomicAdd(dst + 1, make_float4(y[q][j][4], y[q][j][5], y[q][j][6], y[q][j][7]));
+    } else {
+        // transposed down-projection rows: this thread's column chunks of Wd[:, rows] h_q, every q
+        float y[NB][J][8];
+        bool jv[J];
+    #pragma unroll
+        for (int j = 0; j < J; ++j) jv[j] = tid + kConsumerThreads * j < nch;
+    #pragma unroll
+        for (int q = 0; q < NB; ++q)
+    #pragma unroll
+            for (int j = 0; j < J; ++j)
+    #pragma unroll
+                for (int k = 0; k < 8; ++k) y[q][j][k] = 0.f;
+        for (int tst = 0; tst < pl.tail_spp; ++tst) {
+            const int r0 = tst * pl.tail_rps;
+            const int nr = (rows - r0) < pl.tail_rps ? (rows - r0) : pl.tail_rps;
+            if (warp_wait_full(&full[slot], phase, p, m, ii, op)) {
+                if (tid == 0) stage_stamp(tr, T_SREADY, pl.spp + tst);
+                const uint4* Ws = reinterpret_cast<const uint4*>(ring + (size_t)slot * SB);
+                const int tpitch16 = (int)(pl.tail_pitch >> 4);
+                // two rows per iteration (the unused sequences' h are zero)
+                for (int r = 0; r < nr; r += 2) {
+                    float f[2][J][8], hk[2][NB];
+    #pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const bool live = r + u < nr;
+    #pragma unroll
+                        for (int j = 0; j < J; ++j)
+                            unpack8((live && jv[j]) ? Ws[(r + u) * tpitch16 + tid + kConsumerThreads * j]
+                                                    : make_uint4(0u, 0u, 0u, 0u),
+                                    f[u][j]);
+    #pragma unroll
+                        for (int q = 0; q < NB; ++q) hk[u][q] = live ? scratch[(size_t)(r0 + r + u) * NB + q] : 0.f;
+                    }
+    #pragma unroll
+                    for (int u = 0; u < 2; ++u)
+    #pragma unroll
+                        for (int q = 0; q < NB; ++q)
+    #pragma unroll
+                            for (int j = 0; j < J; ++j)
+    #pragma unroll
+                                for (int k = 0; k < 8; k += 2) {
+                                    const float2 t = fma2(make_float2(f[u][j][k], f[u][j][k + 1]),
+                                                          make_float2(hk[u][q], hk[u][q]),
+                                                          make_float2(y[q][j][k], y[q][j][k + 1]));
+                                    y[q][j][k] = t.x;
+                                    y[q][j][k + 1] = t.y;
+                                }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[slot]);
+            } else if (tid == 0) {
+                vstore(&m.abort_flag, 1);
+            }
+            if (++slot == p.ring_stages) {
+                slot = 0;
+                phase ^= 1u;
+            }
+        }
+        cbar();
+        if (vload(&m.abort_flag)) return false;
+    #pragma unroll
+        for (int q = 0; q < NB; ++q) {
+            if (q >= nb) continue;
+    #pragma unroll
+            for (int j = 0; j < J; ++j) {
+                if (!jv[j]) continue;
+                float4* dst = reinterpret_cast<float4*>(p.x2 + q * H) + 2 * (tid + kConsumerThreads * j);
+                atomicAdd(dst, make_float4(y[q][j][0], y[q][j][1], y[q][j][2], y[q][j][3]));
+                atomicAdd(dst + 1, make_float4(y[q][j][4], y[q][j][5], y[q][j][6], y[q][j][7]));
+            }
         }
     }
     cbar();
@@ -2943,6 +3247,10 @@ int megakernel_variant(const DevParams& p, bool fused_ffn) {
     if (p.E > 0) return p.l2_prefetch > 0 ? 0 : base + 4;
     return p.l2_prefetch > 0 ? base + 2 : base;
 }
+
+// Bytes between the weight rows of a stage beyond the row itself, for an instantiation (its
+// tensor-core batched GEMVs read the stage with ldmatrix: 16 keeps each 8-row tile in distinct banks).
+int megakernel_row_pad(int variant) { return variant == 9 ? 16 : 0; }
 
 cudaError_t launch_megakernel(const DevParams& p, const StepArgs& a, int n_sm, int variant, cudaStream_t stream) {
     const size_t smem = megakernel_smem_bytes(p.ring_stages, p.stage_bytes);

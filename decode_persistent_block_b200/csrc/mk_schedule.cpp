@@ -183,9 +183,13 @@ static int chunks_per_thread(int k) {
 }
 
 int max_batch(const mk_config& c) {
-    const int jh = chunks_per_thread(c.hidden), jo = chunks_per_thread(c.n_q_heads * c.head_dim);
-    if (c.n_experts == 0 && jh == 1 && jo == 1 && c.head_dim == 64) return kMaxBatch;
-    if (c.n_experts == 0 && jh == 2 && jo == 2 && c.head_dim == 128) return kMaxBatch / 2;
+    // the 8-sequence kernel's tensor-core GEMVs split every row into 8 warp ranges of whole
+    // 16-column k-steps (rows a multiple of 128 columns)
+    const int qd = c.n_q_heads * c.head_dim;
+    if (c.n_experts != 0) return 1;
+    const int jh = chunks_per_thread(c.hidden), jo = chunks_per_thread(qd);
+    if (jh == 1 && jo == 1 && c.head_dim == 64) return c.hidden % 128 == 0 && qd % 128 == 0 ? kMaxBatch : kMaxBatch / 2;
+    if (jh == 2 && jo == 2 && c.head_dim == 128) return kMaxBatch / 2;
     return 1;
 }
 
