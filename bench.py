@@ -436,16 +436,18 @@ def measure(args, cfg, p0, positions, K, Wm, rank, world, local, with_extras=Tru
     }
 
 
-def measure_batch(args, cfg, p0, B, K, Wm, world, local):
+def measure_batch(args, cfg, p0, B, K, Wm, world, local, dW=None):
     """Device-timed batched decode steps (B sequences per launch, each with its own cache and
-    token, all at the same positions as the batch-1 workload); returns one `batch` entry."""
+    token, all at the same positions as the batch-1 workload); returns one `batch` entry.
+    dW: the model's device weights, if already made."""
     import numpy as np
     import torch
 
     import synth
     from decode_persistent_block_b200 import Decoder, to_device
     torch.cuda.set_device(local)
-    dW = to_device(synth.make_model(cfg))
+    if dW is None:
+        dW = to_device(synth.make_model(cfg))
     caches = [synth.make_kv_cache(cfg, stream=f".{b}") for b in range(B)]
     dk = torch.from_numpy(np.stack([c[0] for c in caches]).view(np.int16)).cuda()
     dv = torch.from_numpy(np.stack([c[1] for c in caches]).view(np.int16)).cuda()
@@ -471,7 +473,7 @@ def measure_batch(args, cfg, p0, B, K, Wm, world, local):
             raise RuntimeError(f"device status after batched steps: {st}")
     step_us = reduce_max(e0.elapsed_time(e1), world) * 1000.0 / K
     bpt = cfg.weight_bytes_per_token() + B * statistics.fmean(cfg.kv_bytes_per_token(q) for q in pos[:K])
-    del dW, dk, dv
+    del dk, dv
     torch.cuda.empty_cache()
     return {"batch": B, "us_per_step": round(step_us, 1), "us_per_token": round(step_us / B, 2),
             "tokens_per_s": round(B * world * 1e6 / step_us, 1), "gb_per_step": round(bpt / 1e9, 4),
@@ -516,12 +518,18 @@ def run_ours(args, rank, world, local):
 
     batched = []
     if args.batch_sizes and not args.layers and args.mode == "megakernel" and not cfg.n_experts:
-        from decode_persistent_block_b200 import MkError
+        import synth
+        import torch
+        from decode_persistent_block_b200 import MkError, to_device
+        torch.cuda.set_device(local)
+        dW = to_device(synth.make_model(cfg))  # one copy of the weights for every batch size
         for B in (int(x) for x in args.batch_sizes.split(",") if x):
             try:
-                batched.append(measure_batch(args, cfg, p0, B, min(K, 256), Wm, world, local))
+                batched.append(measure_batch(args, cfg, p0, B, min(K, 256), Wm, world, local, dW))
             except MkError as e:  # no kernel for this batch size on this shape
                 batched.append({"batch": B, "unsupported": e.name})
+        del dW
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:

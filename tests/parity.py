@@ -18,6 +18,11 @@ HIDDEN_RTOL = 1e-2
 LOGIT_ATOL = 5e-2
 MARGIN = 0.1
 ROUTER_MARGIN = 1e-2
+# Router weights: a softmax over the top-k router scores, whose slope is at most 1/4 for top-2, so a
+# weight error of ROUTER_W_ATOL is a score-gap error of 4 x that.  The scores are dot products of
+# the kernel's own fp32 residual, which may differ from the oracle's fp64 one by HIDDEN_RTOL
+# relative; over 128-step chains on the Mixtral shape the weights differed by up to 1.5e-4.
+ROUTER_W_ATOL = 1e-3
 # The prediction's router scores come from the kernel's own fp32 residual (within HIDDEN_RTOL of the
 # oracle's): below this gap between the k-th and (k+1)-th score the two may pick differently.
 PRED_MARGIN = 1e-2
@@ -144,7 +149,7 @@ def assert_parity(reports: list[dict], cfg=None):
             assert r["next_gpu"] == r["next_orc"], r
         for gi, oi, gw, ow in r.get("router", []):
             assert gi == oi, (r["pos"], gi, oi)
-            assert np.allclose(gw, ow, atol=1e-4), (gw, ow)
+            assert np.allclose(gw, ow, atol=ROUTER_W_ATOL), (gw, ow)
         for got, want, margin, _ in r.get("pred", []):
             if margin > PRED_MARGIN:
                 assert got == want, (r["pos"], got, want, margin)
