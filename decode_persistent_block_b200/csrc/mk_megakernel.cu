@@ -2299,10 +2299,6 @@ __device__ __forceinline__ void ml_combine(float& m, float& l, float* o, float m
     m = M;
 }
 
-// Query heads are split between the two halves of the consumer warps (each
-// half owns at most 2 of the kv head's query heads and streams every K/V row of
-// the stage for them), which keeps the per-thread q and output accumulators to
-// 2 x 8 + 2 x 8 registers.
 // CUDA-core split attention (the general and head_dim-128 kernels): query
 // heads are split between the two halves of the consumer warps (each half owns
 // at most 2 of the kv head's query heads and streams every K/V row of the stage
