@@ -208,7 +208,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     if (rc) return rc;
     mk_options o;
     if (opt) o = *opt; else mk_default_options(&o);
-    mk::fill_defaults(&o);
+    mk::fill_defaults(*cfg, &o);
     rc = mk::check_options(*cfg, o);
     if (rc) return rc;
     if (o.mode != MK_MODE_MEGAKERNEL) o.split_ffn = 1;  // the schedule of the plain launches is never fused

@@ -21,7 +21,7 @@ struct Planned {
 
 int check_config(const mk_config& c);
 int check_options(const mk_config& c, const mk_options& o);
-void fill_defaults(mk_options* o);
+void fill_defaults(const mk_config& c, mk_options* o);
 int default_kv_splits(const mk_config& c, int n_sm, int nb = 1);
 // Largest options.batch the kernels support for this shape (1: no batched decode).
 int max_batch(const mk_config& c);
