@@ -110,6 +110,7 @@ MK_HD inline int kparts_of(int K) { return (K + kMaxPartK - 1) / kMaxPartK; }
 // Accumulator slots (rows x sets x sequences) an instruction of `rows` rows keeps in shared
 // memory.  A batched LM-head instruction goes through its rows in chunks (lm_chunk_rows), so
 // only one chunk's slots count.
+// (rps <= kRowSlots / nb: the stage plan caps a batched LM head's rows per stage.)
 MK_HD inline int lm_chunk_rows(int nb, int rps) {
     const int c = kRowSlots / (nb > 0 ? nb : 1) / rps * rps;  // whole ring stages of rps rows
     return c > rps ? c : rps;

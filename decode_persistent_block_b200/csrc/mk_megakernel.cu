@@ -324,7 +324,9 @@ __device__ void make_plan(const DevParams& p, int pos, const int32_t* w, const i
     pl.row_bytes = pl.src_stride / (uint32_t)pl.kparts;
     const uint32_t pad = (uint32_t)p.row_pad;  // tensor-core batched kernel: padded rows
     pl.pitch = pl.row_bytes + pad;
-    const int rps = (int)(SB / ((uint32_t)pl.nspan * pl.pitch));
+    int rps = (int)(SB / ((uint32_t)pl.nspan * pl.pitch));
+    // a batched LM head keeps every sequence's sums of a stage's rows at once (lm_chunk_rows)
+    if (p.nb > 1 && op == OP_LMHEAD_ARGMAX && rps > kRowSlots / p.nb) rps = kRowSlots / p.nb;
     pl.rps = rps < pl.rows ? rps : pl.rows;
     pl.spp = (pl.rows + pl.rps - 1) / pl.rps;
     pl.n_stages = pl.main_stages = pl.spp * pl.nphase;
