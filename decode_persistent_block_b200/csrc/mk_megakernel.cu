@@ -1423,8 +1423,10 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
 // ---------------------------------------------------------------------------
 // consumers: batched decode (NB > 1 sequences per step, nb of them in use)
 // ---------------------------------------------------------------------------
-// A batched GEMV is a skinny GEMM, y[row][q] = sum_k W[row][k] x_q[k], so it
-// runs on the tensor cores: each ring stage's rows (stored at a pitch of
+// A batched GEMV is a skinny GEMM, y[row][q] = sum_k W[row][k] x_q[k].  The
+// one-chunk kernel with 8 sequence slots (batch_on_tensor_cores) runs it on the
+// tensor cores; the other batched kernels use the CUDA-core form further down.
+// On the tensor cores each ring stage's rows (stored at a pitch of
 // row_bytes + 16, so the 8 rows of an ldmatrix tile fall in different banks)
 // are the A operand of m16n8k16 bf16 MMAs whose N dimension is the 8 sequence
 // slots (unused slots hold zeros).  Warp w takes columns [w K/8, (w + 1) K/8)
