@@ -165,10 +165,10 @@ int check_config(const mk_config& c) {
 void fill_defaults(const mk_config& c, mk_options* o) {
     // The ring's shape: 3 stages of 64 KB, or 2 stages of 96 KB for dense head_dim-128 models
     // (the two-chunk kernels: each block's slices of their 3072-wide rows are larger) and for
-    // batches of 4 or more sequences (each stage carries more work per byte).  Measured: 3-4%
-    // faster on the Llama-3B shape, 3-5% on the Llama-1B shape at 4 and 8 sequences; slower at
-    // batch 1 on the Llama-1B and Mixtral shapes.
-    const bool big = c.n_experts == 0 && (c.head_dim == 128 || o->batch >= 4);
+    // batched decode (each stage carries more work per byte).  Measured: 3-4% faster on the
+    // Llama-3B shape, 1-5% on the Llama-1B shape at 2 to 8 sequences; slower at batch 1 on the
+    // Llama-1B and Mixtral shapes.
+    const bool big = c.n_experts == 0 && (c.head_dim == 128 || o->batch >= 2);
     if (o->ring_stages <= 0 && o->stage_bytes <= 0 && big) {
         o->ring_stages = 2;
         o->stage_bytes = 98304;

@@ -98,9 +98,9 @@ typedef struct {
  * l2_prefetch, prefetch_ahead and l2_head_start (-1 = default, 0 = off). */
 typedef struct {
     int ring_stages;      /* shared-memory weight ring depth (default 3; 2 for dense head_dim-128 models
-                             and for batch >= 4) */
+                             and for batch > 1) */
     int stage_bytes;      /* bytes per ring stage, multiple of 1024 (default 65536; 98304 for dense
-                             head_dim-128 models and for batch >= 4, when ring_stages is left at 0 too) */
+                             head_dim-128 models and for batch > 1, when ring_stages is left at 0 too) */
     int rows_per_instr;   /* cap on GEMV rows per instruction (default and max 1024) */
     int kv_splits;        /* split-KV chunks per kv head (0 = default, at most SMs / n_kv_heads: at
                              head_dim 64 the count minimising a fitted model of attention plus merge
