@@ -76,6 +76,9 @@ def parse():
     ap.add_argument("--spec-experts", type=int, default=-1,
                     help="MoE configs: speculative expert prediction (0 off, 1 on, 2 mispredict; -1: the "
                          "library default)")
+    ap.add_argument("--attn-merge", type=int, default=0,
+                    help="merge of the attention splits: 1 in every O-projection block, 2 once per kv head "
+                         "(0: the library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-baselines", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -307,6 +310,8 @@ def measure(args, cfg, p0, positions, K, Wm, rank, world, local, with_extras=Tru
                 stage_bytes=args.stage_bytes, kv_splits=args.kv_splits, serve_idle_ns=2_000_000_000)
     if cfg.n_experts and args.spec_experts >= 0:
         opts["spec_experts"] = args.spec_experts
+    if args.attn_merge:
+        opts["attn_merge"] = args.attn_merge
     calib = None
     if args.calibrate and args.mode == "megakernel":
         # start-up calibration, outside the timed region: a few traced steps from p0

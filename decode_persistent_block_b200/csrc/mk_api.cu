@@ -290,7 +290,8 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
     if ((rc = dalloc(h, &p.x, (size_t)NB * H))) return fail(rc);
     if ((rc = dalloc(h, &p.x2, (size_t)NB * H))) return fail(rc);
     if ((rc = dalloc(h, &p.qkv, (size_t)NB * (nq + 2 * nkv) * d))) return fail(rc);
-    if ((rc = dalloc(h, &p.attn, (size_t)nq * d))) return fail(rc);
+    if ((rc = dalloc(h, &p.attn, (size_t)NB * nq * d))) return fail(rc);
+    if ((rc = dalloc(h, &p.attn_arrive, (size_t)NB * std::max(L, 1) * nkv))) return fail(rc);
     if ((rc = dalloc(h, &p.part_o, (size_t)NB * nq * S * d))) return fail(rc);
     if ((rc = dalloc(h, &p.part_ml, (size_t)NB * nq * S * 2))) return fail(rc);
     if ((rc = dalloc(h, &p.hbuf, (size_t)topk * c.ffn))) return fail(rc);
@@ -578,6 +579,7 @@ int mk_reset(mk_handle* h) {
     if (!h || h->serving) return MK_ERR_INVALID_ARG;
     CK(cudaStreamSynchronize(h->stream));
     CK(cudaMemset(h->p.counters, 0, sizeof(uint32_t) * h->p.n_ctr));
+    CK(cudaMemset(h->p.attn_arrive, 0, sizeof(uint32_t) * h->p.nb * std::max(h->p.L, 1) * h->p.nkv));
     CK(cudaMemset(h->p.status, 0, sizeof(mk::DevStatus)));
     if (h->p.trace) CK(cudaMemset(h->p.trace, 0, sizeof(uint64_t) * h->plan.n_sm * h->plan.max_instr * mk::kTraceWords));
     h->epoch = 0;

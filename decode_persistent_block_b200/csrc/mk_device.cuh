@@ -162,6 +162,11 @@ __device__ __forceinline__ uint32_t arrive_release(uint32_t* ctr) {
     return old;
 }
 __device__ __forceinline__ void fence_acquire() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+// Arrival on a dependency counter whose ordering a fence of the same thread
+// already provided (after arrive_release, for example).
+__device__ __forceinline__ void signal_relaxed(uint32_t* ctr) {
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+}
 __device__ __forceinline__ int ld_relaxed_s32(const int* p) {
     int v;
     asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

@@ -55,6 +55,9 @@ enum Word : int {
                       //   experts (its last QKV instruction of the layer), 2 = the same and it publishes the
                       //   prediction; MOE_FFN: 1 = the block's loader streams the predicted expert's first
                       //   stages before the routing is known (the block predicted this layer).  0: none
+    W_MERGE = 12,     // ATTN: 1 = the kv head's last split to arrive merges the S splits of its query heads
+                      //   into DevParams.attn before it signals; OPROJ: 1 = the input is that merged
+                      //   output.  0 (both): every O-projection block merges the splits itself
     W_NWORDS = MK_INSTR_WORDS
 };
 
@@ -70,6 +73,9 @@ constexpr int kMaxTopK = 2;
 constexpr int kMaxBatch = 8;         // sequences of one batched decode step
 constexpr int kMiscBytes = 1024;     // shared-memory budget of the kernel's per-block bookkeeping
 constexpr int kMaxMergeSlots = 2048;  // query heads x kv splits merged in the O-projection prologue
+// Above this many bytes of split partials (n_q_heads x kv_splits x head_dim fp32), which every
+// O-projection block would read from L2 to merge, one split per kv head merges them instead (W_MERGE).
+constexpr long long kMergeOnceBytes = 96 * 1024;
 constexpr int kDefaultL2HeadStart = 0;  // ring stages of an FFN / LM-head stream prefetched into L2 past the ring
 
 // Counter ids: per layer [QKV, ATTN (one signal per split), OPROJ, FFN1, FFN2], then the LM head's
@@ -214,7 +220,8 @@ struct DevParams {
     float* x;          // [H] residual stream read by the FFN (written by O-proj)
     float* x2;         // [H] residual stream after the FFN (O-proj writes it too; the FFN adds into it)
     float* qkv;        // [(nq + 2 nkv) d]  raw projections, pre-RoPE
-    float* attn;       // [nq d]
+    float* attn;       // [nb][nq d] attention output, merged once per kv head (W_MERGE)
+    uint32_t* attn_arrive;  // [nb][L][nkv] arrivals of the kv splits (W_MERGE), epoch x kv_splits after a step
     float* part_o;     // [nq][kv_splits][d]
     float* part_ml;    // [nq][kv_splits][2]
     float* hbuf;       // [max(topk,1)][F]

@@ -186,6 +186,7 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
         w[W_AUX_CTR] < -1 || w[W_AUX_CTR] >= p.n_ctr)
         return false;
     if (w[W_WAIT_CTR] >= 0 && w[W_WAIT_INC] <= 0) return false;
+    if (w[W_MERGE] != 0 && (w[W_MERGE] != 1 || (op != OP_ATTN && op != OP_OPROJ_RES) || p.nb > 1)) return false;
     if (op == OP_ATTN) {
         if (sub < 0 || sub >= p.nkv || e != p.kv_splits || b < 0 || b >= e) return false;
         if (w[W_SEQ] < 0 || w[W_SEQ] >= p.nb) return false;
@@ -1041,7 +1042,8 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
                         (p.snap && w[W_SEQ] == 0) ? p.snap + (size_t)p.L * p.H : nullptr);
             break;
         case OP_OPROJ_RES:
-            K = p.nq * p.d;  // input: the attention output, merged from the kv splits below
+            K = p.nq * p.d;  // input: the attention output, merged once (W_MERGE) or from the kv splits below
+            if (w[W_MERGE]) vsrc = p.attn;
             break;
         case OP_DOWN_RES:
         case OP_MOE_DOWN2_RES:
@@ -1050,7 +1052,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
             break;
     }
     const int kp = K / kparts_of(K);  // columns per part
-    if (op == OP_OPROJ_RES) load_attn_merged<J, HOIST ? 8 : 4>(p, 0, kp, v);
+    if (op == OP_OPROJ_RES && !vsrc) load_attn_merged<J, HOIST ? 8 : 4>(p, 0, kp, v);
     if (vsrc) load_vec<J>(vsrc, kp, v);
     // 3. routing (once per layer per block; the loader waits for it)
     if constexpr (!HOIST) {
@@ -1068,7 +1070,7 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
     const int nch = kp >> 3;
     for (int ph = 0; ph < pl.nphase; ++ph) {
         const int vslot = ph / pl.kparts, part = ph % pl.kparts;
-        if (ph > 0 && op == OP_OPROJ_RES) load_attn_merged<J, HOIST ? 8 : 4>(p, part * kp, kp, v);
+        if (ph > 0 && op == OP_OPROJ_RES && !vsrc) load_attn_merged<J, HOIST ? 8 : 4>(p, part * kp, kp, v);
         else if (ph > 0) load_vec<J>(vsrc + (size_t)vslot * p.F + (size_t)part * kp, kp, v);
         for (int sst = 0; sst < pl.spp; ++sst) {
             const int r0 = sst * pl.rps;
@@ -1772,7 +1774,7 @@ template <int J, int NB>
 __device__ void load_attn_merged_b(const DevParams& p, int K, float (&v)[NB][J][8]) {
     constexpr int QG = NB < 4 ? NB : 4;        // sequences per round
     constexpr int SG = NB >= 8 ? 1 : 8 / QG;   // splits per round (QG x SG x 10 live floats)
-    const int tid = threadIdx.x, nch = K >> 3, S = p.kv_splits, D = p.d, D4 = D >> 2, nb = p.nb;
+    const int tid = threadIdx.x, nch = K >> 3, S = p.kv_splits, D = p.d, nb = p.nb;
     const size_t seq_ml = (size_t)p.nq * S * 2, seq_o = (size_t)p.nq * S * D;
 #pragma unroll
     for (int j = 0; j < J; ++j) {
@@ -2303,6 +2305,77 @@ __device__ __forceinline__ void ml_combine(float& m, float& l, float* o, float m
     m = M;
 }
 
+// End of an attention split whose partials are written: signal the attention
+// counter.  With W_MERGE the split also counts itself on its kv head's arrival
+// counter; the last of the S splits to arrive merges the S partials of each of
+// the kv head's G query heads (the rescaled combination that load_attn_merged
+// computes in the O-projection otherwise) and writes the attention output to
+// p.attn before it signals.  The other splits signal at once, so the counter
+// still completes only once every head's output is final.  One thread per two
+// adjacent columns (G * head_dim / 2 <= 256), 16 splits per round trip.
+__device__ void attn_finish(const DevParams& p, const StepArgs& a, const int32_t* w, Misc& m, int sq, int l,
+                            int g, int G, int S, int D) {
+    const int tid = threadIdx.x;
+    uint32_t* ctr = p.counters + w[W_SIGNAL_CTR];
+    cbar();
+    if (!w[W_MERGE]) {
+        if (tid == 0) signal_release(ctr);
+        return;
+    }
+    if (tid == 0) {
+        const uint32_t old = arrive_release(p.attn_arrive + ((size_t)sq * p.L + l) * p.nkv + g);
+        const int last = old + 1u == a.epoch * (uint32_t)S;
+        if (last) fence_acquire();  // the other splits' partials, before the block reads them
+        else signal_relaxed(ctr);   // ordered by the fence in arrive_release
+        m.is_last = last;
+    }
+    cbar();
+    if (!m.is_last) return;
+    constexpr int B = 16;
+    if (tid < G * D / 2) {
+        const int h = (2 * tid) / D, col = 2 * tid - h * D;
+        const size_t base = (size_t)sq * p.nq * S + (size_t)(g * G + h) * S;  // partial slot of split 0
+        const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + base;
+        const float2* po = reinterpret_cast<const float2*>(p.part_o + base * D + col);
+        const int D2 = D >> 1;
+        float M = -CUDART_INF_F, den = 0.f, acc0 = 0.f, acc1 = 0.f;
+        for (int s0 = 0; s0 < S; s0 += B) {
+            float2 t[B], o[B];
+#pragma unroll
+            for (int k = 0; k < B; ++k) {
+                if (s0 + k < S) {
+                    t[k] = __ldcg(ml + s0 + k);
+                    o[k] = __ldcg(po + (size_t)(s0 + k) * D2);
+                } else {
+                    t[k] = make_float2(-CUDART_INF_F, 0.f);
+                    o[k] = make_float2(0.f, 0.f);
+                }
+            }
+            float bm = M;
+#pragma unroll
+            for (int k = 0; k < B; ++k) bm = fmaxf(bm, t[k].x);
+            if (bm == -CUDART_INF_F) continue;  // no position in these splits
+            const float r = exp2f(M - bm);
+            den *= r;
+            acc0 *= r;
+            acc1 *= r;
+#pragma unroll
+            for (int k = 0; k < B; ++k) {
+                const float f = exp2f(t[k].x - bm);
+                den = fmaf(f, t[k].y, den);
+                acc0 = fmaf(f, o[k].x, acc0);
+                acc1 = fmaf(f, o[k].y, acc1);
+            }
+            M = bm;
+        }
+        const float inv = 1.0f / den;
+        *reinterpret_cast<float2*>(p.attn + (size_t)sq * p.nq * D + (size_t)(g * G + h) * D + col) =
+            make_float2(acc0 * inv, acc1 * inv);
+    }
+    cbar();
+    if (tid == 0) signal_release(ctr);
+}
+
 // CUDA-core split attention (the general and head_dim-128 kernels): query
 // heads are split between the two halves of the consumer warps (each half owns
 // at most 2 of the kv head's query heads and streams every K/V row of the stage
@@ -2595,8 +2668,7 @@ __device__ bool attn_cc(const DevParams& p, const StepArgs& a, const int32_t* w,
             part_ml_s[part * 2 + 1] = Ls;
         }
     }
-    cbar();
-    if (tid == 0) signal_release(p.counters + w[W_SIGNAL_CTR]);
+    attn_finish(p, a, w, m, sq, l, g, G, S, D);
     return true;
 }
 
@@ -2916,8 +2988,7 @@ __device__ bool attn_tc(const DevParams& p, const StepArgs& a, const int32_t* w,
             part_ml_s[part * 2 + 1] = Ls;
         }
     }
-    cbar();
-    if (tid == 0) signal_release(p.counters + w[W_SIGNAL_CTR]);
+    attn_finish(p, a, w, m, sq, l, g, G, S, D);
     return true;
 }
 

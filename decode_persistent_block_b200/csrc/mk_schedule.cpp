@@ -225,6 +225,8 @@ int check_options(const mk_config& c, const mk_options& o) {
     if (o.mode < MK_MODE_MEGAKERNEL || o.mode > MK_MODE_MULTI_KERNEL_GRAPH) return MK_ERR_INVALID_ARG;
     if (o.spec_experts < 0 || o.spec_experts > 2) return MK_ERR_INVALID_ARG;
     if (o.batch < 1 || o.batch > kMaxBatch) return MK_ERR_INVALID_ARG;
+    if (o.attn_merge < 0 || o.attn_merge > 2) return MK_ERR_INVALID_ARG;
+    if (o.attn_merge == 2 && o.batch > 1) return MK_ERR_UNSUPPORTED;
     if (o.batch > 1) {  // batched decode: the specialised dense kernels with the fused FFN only
         if (o.batch > max_batch(c) || o.mode != MK_MODE_MEGAKERNEL || !ffn_fused(c, o) || o.spec_experts ||
             o.general_kernel || o.l2_prefetch > 0 || o.prefetch_ahead > 0)
@@ -269,6 +271,10 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     };
     const int qd = c.n_q_heads * d;
     const int nb = o.batch;  // every GEMV row keeps nb accumulator sets (one per sequence)
+    // Merge the attention splits once per kv head (the last split to arrive) instead of in every
+    // O-projection block, when the partials that each of those blocks would read from L2 are large.
+    const int merge_once = o.attn_merge == 2 ||
+                           (o.attn_merge == 0 && nb == 1 && 4LL * qd * S > kMergeOnceBytes);
     auto op_cap = [&](int op) {
         const int need = row_slots(op, 1, acc_sets(op, H, qd, F, c.top_k), nb);  // slots per row
         return need > 0 ? std::min(cap, kRowSlots / need) : cap;
@@ -305,11 +311,16 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
             w[W_SEQ] = k / (S * nkv);
             w[W_WAIT_CTR] = ctr_id(l, C_QKV);
             w[W_SIGNAL_CTR] = ctr_id(l, C_ATTN);
+            w[W_MERGE] = merge_once;
             int sm = (int)(((long long)k + (long long)l * total) % n_sm);
             add(sm, w);
             ffn_weight[sm] = speed[sm] * (o.attn_sm_ffn_permille / 1000.0);
         }
         gemv_op(OP_OPROJ_RES, l, {{0, H}}, ctr_id(l, C_ATTN), ctr_id(l, C_OPROJ));
+        if (merge_once)
+            for (auto& qs : q)
+                for (auto& w : qs)
+                    if (w[W_OP] == OP_OPROJ_RES && w[W_LAYER] == l) w[W_MERGE] = 1;
         std::vector<Segment> slots;
         for (int s = 0; s < (moe ? c.top_k : 1); ++s) slots.push_back({s, F});
         if (fused) {
@@ -377,6 +388,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     out->n_lm = (int)inc[ctr_lm(L)];
     out->fused_ffn = fused;
     out->nb = nb;
+    out->merge_once = merge_once;
     out->words.assign((size_t)n_sm * max_instr * W_NWORDS, 0);
     out->n_instr.assign(n_sm, 0);
     for (int sm = 0; sm < n_sm; ++sm) {
@@ -443,6 +455,7 @@ int validate(const mk_config& c, const Planned& p) {
     std::vector<uint32_t> signals(nctr, 0);
     const int nb = p.nb;
     if (nb < 1 || nb > kMaxBatch || (nb > 1 && (moe || !p.fused_ffn))) return MK_ERR_SCHEDULE;
+    if (p.merge_once != 0 && (p.merge_once != 1 || nb > 1)) return MK_ERR_SCHEDULE;
     std::vector<std::vector<uint8_t>> attn_seen((size_t)std::max(L, 1) * nb * nkv,
                                                 std::vector<uint8_t>(p.kv_splits, 0));
     std::vector<uint8_t> lm_seq(std::max(p.n_lm, 1), 0);
@@ -474,6 +487,8 @@ int validate(const mk_config& c, const Planned& p) {
                 return MK_ERR_SCHEDULE;  // everything but the first op depends on something
             }
             if (w[W_SIGNAL_CTR] >= nctr || w[W_AUX_CTR] >= nctr) return MK_ERR_SCHEDULE;
+            // the merge of the attention splits: once per kv head (ATTN and OPROJ agree) or in every block
+            if (w[W_MERGE] != ((op == OP_ATTN || op == OP_OPROJ_RES) ? p.merge_once : 0)) return MK_ERR_SCHEDULE;
             // speculative expert prediction: a predicting QKV instruction is the block's last QKV of
             // its layer, and an FFN slice streams predicted stages only after its block predicted
             if (w[W_SPEC] != 0) {

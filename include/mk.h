@@ -158,6 +158,16 @@ typedef struct {
                              megakernel mode, hidden and n_q_heads*head_dim at most 2048 (B <= 8) or 4096
                              (B <= 4), and no serving or speculative prediction; otherwise
                              mk_create returns MK_ERR_UNSUPPORTED */
+    int attn_merge;       /* where the kv splits of the split attention are merged (the combine step of
+                             split-KV decoding: each split's partial output rescaled by its running max).
+                             1 = every O-projection block merges all splits of every head while loading
+                             its input, so the partials are read from L2 once per block; 2 = the last split
+                             of each kv head to finish merges that head's splits once and writes the
+                             attention output, which the O-projection blocks read as a plain vector (one
+                             atomic arrival per split, one extra L2 round trip for the last one).  0
+                             (default) = 2 when the partials that every block would read exceed 96 KB
+                             (n_q_heads * kv_splits * head_dim * 4 bytes) and batch is 1, else 1.  2 with
+                             batch > 1 returns MK_ERR_UNSUPPORTED */
 } mk_options;
 
 /* Device status block, copied out by mk_get_status.  On a device-side error

@@ -36,6 +36,8 @@ def test_tiny_all_steps(tiny, mode):
     dict(n_sm=7), dict(n_sm=1), dict(kv_splits=1), dict(kv_splits=40), dict(ring_stages=2),
     dict(stage_bytes=4096), dict(stage_bytes=4096, ring_stages=3, l2_prefetch=16384), dict(rows_per_instr=3),
     dict(l2_prefetch=65536), dict(split_ffn=1), dict(split_ffn=1, n_sm=7),
+    dict(attn_merge=2), dict(attn_merge=2, n_sm=7), dict(attn_merge=2, n_sm=1), dict(attn_merge=2, kv_splits=1),
+    dict(attn_merge=2, kv_splits=40), dict(attn_merge=2, split_ffn=1), dict(attn_merge=2, general_kernel=1),
 ], ids=lambda o: ",".join(f"{k}={v}" for k, v in o.items()))
 def test_tiny_schedule_options(tiny, opts):
     parity.assert_parity(parity.run(tiny, **opts))
@@ -55,9 +57,10 @@ def test_no_layers_is_lm_head_of_embedding(cuda):
     parity.assert_parity(parity.run(parity.Setup(cfg)))
 
 
-def test_head_dim_128_group_3(cuda):
+@pytest.mark.parametrize("attn_merge", [1, 2], ids=["merge_in_oproj", "merge_once"])
+def test_head_dim_128_group_3(cuda, attn_merge):
     cfg = configs.TINY.with_(name="tiny_d128", n_heads=6, n_kv_heads=2, head_dim=128, hidden=384, ffn=1024)
-    parity.assert_parity(parity.run(parity.Setup(cfg)))
+    parity.assert_parity(parity.run(parity.Setup(cfg), attn_merge=attn_merge))
 
 
 def test_group_1_and_wide_rows(cuda):
@@ -68,9 +71,10 @@ def test_group_1_and_wide_rows(cuda):
         parity.assert_parity(parity.run(setup, mode=mode, split_ffn=split))
 
 
-def test_counters_are_exact_multiples_after_steps(tiny):
+@pytest.mark.parametrize("attn_merge", [1, 2], ids=["merge_in_oproj", "merge_once"])
+def test_counters_are_exact_multiples_after_steps(tiny, attn_merge):
     tiny.fresh_caches()
-    with tiny.decoder() as dec:
+    with tiny.decoder(attn_merge=attn_merge) as dec:
         inc = dec.counter_increments()
         for s, (pos, tok) in enumerate(parity.schedule(configs.TINY)):
             dec.step(tok if tok is not None else 1, pos)
@@ -92,9 +96,11 @@ def _repeat(tiny, n, **opts):
     return outs
 
 
-def test_determinism_bitwise(tiny):
-    # split FFN: every sum has a fixed order, so repeated runs agree bit for bit
-    outs = _repeat(tiny, 2, split_ffn=1)
+@pytest.mark.parametrize("attn_merge", [1, 2], ids=["merge_in_oproj", "merge_once"])
+def test_determinism_bitwise(tiny, attn_merge):
+    # split FFN: every sum has a fixed order (the once-per-head merge reads the splits in order,
+    # whichever split runs it), so repeated runs agree bit for bit
+    outs = _repeat(tiny, 2, split_ffn=1, attn_merge=attn_merge)
     assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
 
 
@@ -202,7 +208,16 @@ def test_llama1b_multi_kernel(cuda):
 
 
 def test_llama3b(cuda):
-    _full(configs.LLAMA_3B, 3)
+    _full(configs.LLAMA_3B, 3)  # the attention splits merged once per kv head (204 KB of partials)
+
+
+def test_llama3b_merge_in_oproj(cuda):
+    _full(configs.LLAMA_3B, 2, attn_merge=1)
+
+
+def test_llama1b_merge_once(cuda):
+    # the head_dim-64 tensor-core attention with the once-per-head merge
+    _full(configs.LLAMA_1B, 2, attn_merge=2)
 
 
 @pytest.mark.parametrize("prefill", configs.LONG_PREFILLS)

@@ -64,10 +64,12 @@ def _served(tiny, **opts):
     return toks, logits
 
 
-def test_served_steps_equal_per_launch_steps_bitwise(tiny):
-    # split FFN: every sum has a fixed order, so the two paths agree bit for bit
-    t1, l1 = _per_launch(tiny, split_ffn=1)
-    t2, l2 = _served(tiny, split_ffn=1)
+@pytest.mark.parametrize("attn_merge", [1, 2], ids=["merge_in_oproj", "merge_once"])
+def test_served_steps_equal_per_launch_steps_bitwise(tiny, attn_merge):
+    # split FFN: every sum has a fixed order (the once-per-head merge too, whichever split does it),
+    # so the two paths agree bit for bit
+    t1, l1 = _per_launch(tiny, split_ffn=1, attn_merge=attn_merge)
+    t2, l2 = _served(tiny, split_ffn=1, attn_merge=attn_merge)
     assert t1 == t2
     for a, b in zip(l1, l2):
         assert np.array_equal(a, b)
@@ -196,9 +198,10 @@ def _served_vs_oracle(setup, steps=None, **opts):
     return reports
 
 
-@pytest.mark.parametrize("split_ffn", [0, 1], ids=["fused_ffn", "split_ffn"])
-def test_served_steps_match_oracle_tiny(tiny, split_ffn):
-    reps = _served_vs_oracle(tiny, split_ffn=split_ffn)
+@pytest.mark.parametrize("opts", [dict(split_ffn=0), dict(split_ffn=1), dict(attn_merge=2)],
+                         ids=["fused_ffn", "split_ffn", "merge_once"])
+def test_served_steps_match_oracle_tiny(tiny, opts):
+    reps = _served_vs_oracle(tiny, **opts)
     assert len(reps) == configs.TINY.prompt_len + configs.TINY.steps
     parity.assert_parity(reps)
 

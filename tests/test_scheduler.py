@@ -389,3 +389,57 @@ def test_batch_options_are_checked():
             dpb.plan(cfg, 148, **opts)
         assert e.value.name == "MK_ERR_UNSUPPORTED", (cfg.name, opts)
     dpb.plan(configs.LLAMA_3B, 148, batch=4)
+
+
+W_MERGE = 12
+
+
+@pytest.mark.parametrize("cfg,opts", [
+    (configs.LLAMA_1B, {}),                  # 148 blocks: 32 heads x 6 splits x 64 x 4 B = 48 KB of partials
+    (configs.LLAMA_3B, {}),                  # 24 x 17 x 128 x 4 B = 204 KB
+    (configs.MIXTRAL_8L, {}),                # 32 x 9 x 128 x 4 B = 144 KB
+    (configs.llama1b_sweep(16384), {}),      # 32 x 16 x 64 x 4 B = 128 KB
+    (configs.LLAMA_1B, dict(kv_splits=12)),  # exactly 96 KB: not above the bound
+    (configs.LLAMA_1B, dict(kv_splits=13)),
+    (configs.LLAMA_1B, dict(attn_merge=2)),
+    (configs.LLAMA_3B, dict(attn_merge=1)),
+    (configs.LLAMA_3B, dict(batch=2)),       # batched decode merges in the O-projection
+    (configs.TINY, dict(attn_merge=2)),
+], ids=lambda x: getattr(x, "name", str(x)))
+@pytest.mark.parametrize("n_sm", [148, 37])
+def test_attention_merge_marks(cfg, opts, n_sm):
+    # Every attention split and O-projection instruction of every layer carries the same merge mark:
+    # forced by attn_merge, else set when the partials every O-projection block would read
+    # (n_q_heads x splits x head_dim fp32) exceed 96 KB at batch 1.  Nothing else carries it, and it
+    # changes no other word and no counter increment.
+    words, n_instr, inc = dpb.plan(cfg, n_sm, **opts)
+    ops = words[:, :, W_OP]
+    marked = (ops == OP["ATTN"]) | (ops == OP["OPROJ"])
+    S = int(words[:, :, W_END][ops == OP["ATTN"]][0])
+    forced = opts.get("attn_merge", 0)
+    auto = opts.get("batch", 1) == 1 and cfg.n_heads * S * cfg.head_dim * 4 > 96 * 1024
+    expect = 1 if forced == 2 or (forced == 0 and auto) else 0
+    if cfg is configs.LLAMA_3B and n_sm == 148 and not opts:
+        assert S == 17 and expect == 1
+    if cfg is configs.LLAMA_1B and n_sm == 148 and not opts:
+        assert S == 6 and expect == 0
+    assert marked.any()
+    assert np.all(words[:, :, W_MERGE][marked] == expect)
+    assert np.all(words[:, :, W_MERGE][~marked] == 0)
+    base, _, inc0 = dpb.plan(cfg, n_sm, **{**opts, "attn_merge": 1})
+    w2 = words.copy()
+    w2[:, :, W_MERGE] = 0
+    np.testing.assert_array_equal(w2, base)
+    np.testing.assert_array_equal(inc, inc0)
+    rc, done = dpb.simulate(words, n_instr, inc, steps=2, seed=n_sm)
+    assert rc == 0 and done == 2 * int(n_instr.sum())
+
+
+def test_attention_merge_option_is_checked():
+    for bad in (-1, 3):
+        with pytest.raises(mk.MkError) as e:
+            dpb.plan(configs.LLAMA_1B, 148, attn_merge=bad)
+        assert e.value.name == "MK_ERR_INVALID_ARG"
+    with pytest.raises(mk.MkError) as e:
+        dpb.plan(configs.LLAMA_1B, 148, attn_merge=2, batch=2)
+    assert e.value.name == "MK_ERR_UNSUPPORTED"
