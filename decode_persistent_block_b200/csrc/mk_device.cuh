@@ -146,12 +146,12 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-// Publish one arrival on a dependency counter: the fence orders every write
-// this block made before the preceding block barrier (cumulatively, at gpu
-// scope) ahead of the increment, which itself needs no ordering.
+// Publish one arrival on a dependency counter: a release reduction, which
+// orders every write this block made before the preceding block barrier
+// (cumulatively, at gpu scope) ahead of the increment.  Measured a little
+// faster than a separate fence.acq_rel followed by a relaxed reduction.
 __device__ __forceinline__ void signal_release(uint32_t* ctr) {
-    asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
 // Arrival that also returns the previous count (last-arriver detection); the
 // caller fences again (acquire) before reading what the other arrivals wrote.

@@ -44,10 +44,15 @@ def _recovers(tiny, dec):
     parity.assert_parity(reps)
 
 
+@pytest.mark.parametrize("attn_merge", [1, 2], ids=["merge_in_oproj", "merge_once"])
 @pytest.mark.parametrize("block", [0, 3, 147])
-def test_unreachable_wait_times_out_and_recovers(tiny, block):
+def test_unreachable_wait_times_out_and_recovers(tiny, block, attn_merge):
+    # With 4 splits, block 0's first waiting instruction is split 0 of kv head 0 in layer 0: with the
+    # once-per-head merge the other 3 splits of that head have counted themselves when the step gives
+    # up, and the reset must clear those arrivals too, or the next step would take the wrong split
+    # for the last one.
     tiny.fresh_caches()
-    with tiny.decoder(spin_limit_ns=LIMIT_NS) as dec:
+    with tiny.decoder(spin_limit_ns=LIMIT_NS, attn_merge=attn_merge, kv_splits=4) as dec:
         dec.step(1, 0)
         dec.inject_fault(mk.FAULT_UNREACHABLE_WAIT, block)
         t0 = time.perf_counter()
