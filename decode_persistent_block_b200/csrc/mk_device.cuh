@@ -153,19 +153,16 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 __device__ __forceinline__ void signal_release(uint32_t* ctr) {
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
-// Arrival that also returns the previous count (last-arriver detection); the
-// caller fences again (acquire) before reading what the other arrivals wrote.
+// Arrival that also returns the previous count (last-arriver detection): an
+// acquire-release atomic, so the block's earlier writes (ordered by the
+// preceding block barrier) are visible before the count moves, and the last
+// arrival sees every other arrival's writes once the caller's next block
+// barrier has passed.  Measured faster than a fence, a relaxed atomic and a
+// second fence in the last arrival.
 __device__ __forceinline__ uint32_t arrive_release(uint32_t* ctr) {
     uint32_t old;
-    asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(ctr) : "memory");
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(ctr) : "memory");
     return old;
-}
-__device__ __forceinline__ void fence_acquire() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-// Arrival on a dependency counter whose ordering a fence of the same thread
-// already provided (after arrive_release, for example).
-__device__ __forceinline__ void signal_relaxed(uint32_t* ctr) {
-    asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
 }
 __device__ __forceinline__ int ld_relaxed_s32(const int* p) {
     int v;

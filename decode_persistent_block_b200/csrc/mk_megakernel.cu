@@ -1190,7 +1190,6 @@ __device__ bool gemv_instr(const DevParams& p, const StepArgs& a, const int32_t*
             }
             cbar();
             if (m.is_last) {
-                fence_acquire();
                 const int n_lm = w[W_AUX_INC];
                 float cv = -CUDART_INF_F;
                 int ci = 0x7FFFFFFF;
@@ -2026,7 +2025,6 @@ __device__ bool gemv_instr_b(const DevParams& p, const StepArgs& a, const int32_
         }
         cbar();
         if (m.is_last) {  // the last LM-head instruction to finish picks every sequence's token
-            fence_acquire();
             const int n_lm = w[W_AUX_INC];
             for (int q = 0; q < nb; ++q) {
                 float cv = -CUDART_INF_F;
@@ -2325,8 +2323,7 @@ __device__ void attn_finish(const DevParams& p, const StepArgs& a, const int32_t
     if (tid == 0) {
         const uint32_t old = arrive_release(p.attn_arrive + ((size_t)sq * p.L + l) * p.nkv + g);
         const int last = old + 1u == a.epoch * (uint32_t)S;
-        if (last) fence_acquire();  // the other splits' partials, before the block reads them
-        else signal_relaxed(ctr);   // ordered by the fence in arrive_release
+        if (!last) signal_release(ctr);
         m.is_last = last;
     }
     cbar();
