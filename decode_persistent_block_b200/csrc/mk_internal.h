@@ -58,6 +58,9 @@ enum Word : int {
     W_MERGE = 12,     // ATTN: 1 = the kv head's last split to arrive merges the S splits of its query heads
                       //   into DevParams.attn before it signals; OPROJ: 1 = the input is that merged
                       //   output.  0 (both): every O-projection block merges the splits itself
+    W_GATE = 13,      // FFN (dense, fused): > 0 = the loader issues the slice's stages from this index on only
+                      //   once the FFN's dependency is met (the earlier ones stream during the small ops
+                      //   before it); 0: no gate
     W_NWORDS = MK_INSTR_WORDS
 };
 

@@ -187,6 +187,7 @@ __device__ bool instr_ok(const DevParams& p, const int32_t* w) {
         return false;
     if (w[W_WAIT_CTR] >= 0 && w[W_WAIT_INC] <= 0) return false;
     if (w[W_MERGE] != 0 && (w[W_MERGE] != 1 || (op != OP_ATTN && op != OP_OPROJ_RES) || p.nb > 1)) return false;
+    if (w[W_GATE] < 0 || (w[W_GATE] != 0 && op != OP_FFN)) return false;
     if (op == OP_ATTN) {
         if (sub < 0 || sub >= p.nkv || e != p.kv_splits || b < 0 || b >= e) return false;
         if (w[W_SEQ] < 0 || w[W_SEQ] >= p.nb) return false;
@@ -553,9 +554,9 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                         sok = false;
                         break;
                     }
-                    issue_stage<TC, NB>(p, sp, st, ring + (size_t)slot * SB, &full[slot]);
-                    if (st == 0 && p.trace)
+                    if (st == 0 && p.trace)  // stamped before the copy is issued: it cannot land earlier
                         p.trace[((size_t)blockIdx.x * p.max_instr + i) * kTraceWords + T_LD_FIRST] = globaltimer_ns();
+                    issue_stage<TC, NB>(p, sp, st, ring + (size_t)slot * SB, &full[slot]);
                     used |= 1u << slot;
                     last_parity = (last_parity & ~(1u << slot)) | (phase << slot);
                     if (++slot == NS) {
@@ -575,10 +576,20 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
         bool ok = true;
         unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + i) * kTraceWords : nullptr;
         for (int st = st0; st < pl.n_stages; ++st, ++g) {
+            // gated FFN slice: the stages from W_GATE on wait for the FFN's own dependency
+            if (st == w[W_GATE] && st > 0 &&
+                !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], i, w[W_OP])) {
+                ok = false;
+                break;
+            }
             if (!wait_mbar(&empty[slot], phase ^ 1u, p, m, i, w[W_OP])) {
                 ok = false;
                 break;
             }
+            // issue stamps are taken before the copy is issued, so a copy never lands before its stamp
+            if (tr && st == 0) tr[T_LD_FIRST] = globaltimer_ns();
+            stage_stamp(tr, T_SISSUE, st);
+            if (tr && st == pl.n_stages - 1) tr[T_LD_LAST] = globaltimer_ns();
             issue_stage<TC, NB>(p, pl, st, ring + (size_t)slot * SB, &full[slot]);
             // Head start of a long stream: the loader reaches the first stage of the
             // dense FFN (or the LM head) while the consumers still wait on the small
@@ -589,9 +600,6 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
                 const int e = pl.n_stages < NS + p.l2_head_start ? pl.n_stages : NS + p.l2_head_start;
                 for (int s2 = NS; s2 < e; ++s2) prefetch_stage(pl, s2);
             }
-            if (tr && st == 0) tr[T_LD_FIRST] = globaltimer_ns();
-            stage_stamp(tr, T_SISSUE, st);
-            if (tr && st == pl.n_stages - 1) tr[T_LD_LAST] = globaltimer_ns();
             used |= 1u << slot;
             last_parity = (last_parity & ~(1u << slot)) | (phase << slot);
             if (++slot == NS) {

@@ -15,6 +15,7 @@ struct Planned {
     bool fused_ffn = true;         // one OP_FFN / OP_MOE_FFN per layer instead of up/gate + down
     int nb = 1;                    // sequences per step (batched decode)
     int merge_once = 0;            // W_MERGE on every ATTN and OPROJ instruction
+    int ffn_gate = 0;              // W_GATE on every dense fused FFN instruction
     std::vector<int32_t> words;    // [n_sm][max_instr][W_NWORDS]
     std::vector<int32_t> n_instr;  // [n_sm]
     std::vector<uint32_t> ctr_inc; // per-step increment of every counter

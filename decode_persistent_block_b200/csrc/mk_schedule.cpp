@@ -227,6 +227,7 @@ int check_options(const mk_config& c, const mk_options& o) {
     if (o.batch < 1 || o.batch > kMaxBatch) return MK_ERR_INVALID_ARG;
     if (o.attn_merge < 0 || o.attn_merge > 2) return MK_ERR_INVALID_ARG;
     if (o.attn_merge == 2 && o.batch > 1) return MK_ERR_UNSUPPORTED;
+    if (o.ffn_early_stages < -1 || o.ffn_early_stages > 64) return MK_ERR_INVALID_ARG;
     if (o.batch > 1) {  // batched decode: the specialised dense kernels with the fused FFN only
         if (o.batch > max_batch(c) || o.mode != MK_MODE_MEGAKERNEL || !ffn_fused(c, o) || o.spec_experts ||
             o.general_kernel || o.l2_prefetch > 0 || o.prefetch_ahead > 0)
@@ -275,6 +276,17 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     // O-projection block, when the partials that each of those blocks would read from L2 are large.
     const int merge_once = o.attn_merge == 2 ||
                            (o.attn_merge == 0 && nb == 1 && 4LL * qd * S > kMergeOnceBytes);
+    // The loader streams a dense fused FFN's first stage during the small ops before it and the rest
+    // only once the FFN's dependency is met, so that the weight stream leaves HBM and L2 quiet for
+    // those ops' latency chain.  Default: on for one-chunk models (hidden <= 2048) at batch 1 or 2
+    // whose FFN slice spans at least 4 ring stages (measured faster there; slower for a 2-stage slice,
+    // for hidden 3072 at batch 4 and for hidden 2048 at batch 8).
+    int ffn_gate = 0;
+    if (fused && !moe) {
+        const long long slice = 3LL * F * H * 2 / n_sm;
+        if (o.ffn_early_stages > 0) ffn_gate = o.ffn_early_stages;
+        else if (o.ffn_early_stages == 0 && nb <= 2 && H <= 2048 && slice >= 4LL * o.stage_bytes) ffn_gate = 1;
+    }
     auto op_cap = [&](int op) {
         const int need = row_slots(op, 1, acc_sets(op, H, qd, F, c.top_k), nb);  // slots per row
         return need > 0 ? std::min(cap, kRowSlots / need) : cap;
@@ -326,6 +338,10 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
         if (fused) {
             // one instruction per block: its up/gate rows, then the matching down-projection columns
             gemv_op(moe ? OP_MOE_FFN : OP_FFN, l, slots, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN2), &ffn_weight);
+            if (ffn_gate)
+                for (auto& qs : q)
+                    for (auto& w : qs)
+                        if (w[W_OP] == OP_FFN && w[W_LAYER] == l) w[W_GATE] = ffn_gate;
         } else if (!moe) {
             gemv_op(OP_RMS_UPGATE_SILU, l, slots, ctr_id(l, C_OPROJ), ctr_id(l, C_FFN1));
             gemv_op(OP_DOWN_RES, l, {{0, H}}, ctr_id(l, C_FFN1), ctr_id(l, C_FFN2));
@@ -389,6 +405,7 @@ int plan_schedule(const mk_config& c, const mk_options& o_in, int n_sm, Planned*
     out->fused_ffn = fused;
     out->nb = nb;
     out->merge_once = merge_once;
+    out->ffn_gate = ffn_gate;
     out->words.assign((size_t)n_sm * max_instr * W_NWORDS, 0);
     out->n_instr.assign(n_sm, 0);
     for (int sm = 0; sm < n_sm; ++sm) {
@@ -456,6 +473,7 @@ int validate(const mk_config& c, const Planned& p) {
     const int nb = p.nb;
     if (nb < 1 || nb > kMaxBatch || (nb > 1 && (moe || !p.fused_ffn))) return MK_ERR_SCHEDULE;
     if (p.merge_once != 0 && (p.merge_once != 1 || nb > 1)) return MK_ERR_SCHEDULE;
+    if (p.ffn_gate < 0 || p.ffn_gate > 64 || (p.ffn_gate && (moe || !p.fused_ffn))) return MK_ERR_SCHEDULE;
     std::vector<std::vector<uint8_t>> attn_seen((size_t)std::max(L, 1) * nb * nkv,
                                                 std::vector<uint8_t>(p.kv_splits, 0));
     std::vector<uint8_t> lm_seq(std::max(p.n_lm, 1), 0);
@@ -489,6 +507,7 @@ int validate(const mk_config& c, const Planned& p) {
             if (w[W_SIGNAL_CTR] >= nctr || w[W_AUX_CTR] >= nctr) return MK_ERR_SCHEDULE;
             // the merge of the attention splits: once per kv head (ATTN and OPROJ agree) or in every block
             if (w[W_MERGE] != ((op == OP_ATTN || op == OP_OPROJ_RES) ? p.merge_once : 0)) return MK_ERR_SCHEDULE;
+            if (w[W_GATE] != (op == OP_FFN ? p.ffn_gate : 0)) return MK_ERR_SCHEDULE;
             // speculative expert prediction: a predicting QKV instruction is the block's last QKV of
             // its layer, and an FFN slice streams predicted stages only after its block predicted
             if (w[W_SPEC] != 0) {

@@ -46,7 +46,8 @@ class MkOptions(ctypes.Structure):
                 ("mode", _I), ("n_sm", _I), ("prefetch_ahead", _I), ("prefetch_max_bytes", _I),
                 ("attn_sm_ffn_permille", _I), ("serve_idle_ns", ctypes.c_ulonglong), ("general_kernel", _I),
                 ("split_ffn", _I), ("l2_head_start", _I), ("sm_speed", ctypes.c_void_p), ("n_sm_speed", _I),
-                ("spec_experts", _I), ("batch", _I), ("attn_merge", _I)]
+                ("spec_experts", _I), ("batch", _I), ("attn_merge", _I),
+                ("ffn_early_stages", _I)]
 
 
 class MkStatus(ctypes.Structure):

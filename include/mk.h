@@ -168,6 +168,12 @@ typedef struct {
                              (default) = 2 when the partials that every block would read exceed 96 KB
                              (n_q_heads * kv_splits * head_dim * 4 bytes) and batch is 1, else 1.  2 with
                              batch > 1 returns MK_ERR_UNSUPPORTED */
+    int ffn_early_stages; /* dense models with the fused FFN: the loader issues at most this many of a
+                             block's FFN stages before the FFN's dependency is met (the rest wait for it),
+                             so that the weight stream leaves HBM and L2 quiet while the small ops before
+                             the FFN run their latency chain.  -1 = no limit; 0 (default) = 1 for hidden
+                             <= 2048 at batch 1 or 2 when the block's FFN slice spans at least 4 ring
+                             stages, else no limit; 1..64 = that many */
 } mk_options;
 
 /* Device status block, copied out by mk_get_status.  On a device-side error

@@ -38,6 +38,8 @@ def test_tiny_all_steps(tiny, mode):
     dict(l2_prefetch=65536), dict(split_ffn=1), dict(split_ffn=1, n_sm=7),
     dict(attn_merge=2), dict(attn_merge=2, n_sm=7), dict(attn_merge=2, n_sm=1), dict(attn_merge=2, kv_splits=1),
     dict(attn_merge=2, kv_splits=40), dict(attn_merge=2, split_ffn=1), dict(attn_merge=2, general_kernel=1),
+    dict(ffn_early_stages=1, n_sm=7), dict(ffn_early_stages=1, stage_bytes=4096),
+    dict(ffn_early_stages=3, stage_bytes=4096, ring_stages=4), dict(ffn_early_stages=1, n_sm=7, general_kernel=1),
 ], ids=lambda o: ",".join(f"{k}={v}" for k, v in o.items()))
 def test_tiny_schedule_options(tiny, opts):
     parity.assert_parity(parity.run(tiny, **opts))
@@ -345,6 +347,12 @@ def test_batch_handle_rejects_single_steps_and_bad_arguments(cuda):
     with pytest.raises(MkError) as e:
         Decoder(moe, Wm, dk, dv, batch=2)
     assert e.value.name == "MK_ERR_UNSUPPORTED"
+
+
+def test_llama1b_batch2(cuda):
+    # two sequences: the FFN stage gate is on by default here, as at batch 1
+    cfg = configs.LLAMA_1B
+    parity.assert_parity(parity.run_batch(cfg, [cfg.prefill, cfg.prefill - 101], steps=2), cfg)
 
 
 def test_llama1b_batch8(cuda):

@@ -198,8 +198,9 @@ def _served_vs_oracle(setup, steps=None, **opts):
     return reports
 
 
-@pytest.mark.parametrize("opts", [dict(split_ffn=0), dict(split_ffn=1), dict(attn_merge=2)],
-                         ids=["fused_ffn", "split_ffn", "merge_once"])
+@pytest.mark.parametrize("opts", [dict(split_ffn=0), dict(split_ffn=1), dict(attn_merge=2),
+                                  dict(ffn_early_stages=1, n_sm=7)],
+                         ids=["fused_ffn", "split_ffn", "merge_once", "ffn_gate"])
 def test_served_steps_match_oracle_tiny(tiny, opts):
     reps = _served_vs_oracle(tiny, **opts)
     assert len(reps) == configs.TINY.prompt_len + configs.TINY.steps

@@ -443,3 +443,40 @@ def test_attention_merge_option_is_checked():
     with pytest.raises(mk.MkError) as e:
         dpb.plan(configs.LLAMA_1B, 148, attn_merge=2, batch=2)
     assert e.value.name == "MK_ERR_UNSUPPORTED"
+
+
+W_GATE = 13
+
+
+@pytest.mark.parametrize("cfg,opts,expect", [
+    (configs.LLAMA_1B, {}, 1),                         # 680 KB of FFN per block: 10.6 stages of 64 KB
+    (configs.LLAMA_1B, dict(batch=2), 1),              # 7 stages of 96 KB
+    (configs.LLAMA_1B, dict(batch=8), 0),
+    (configs.LLAMA_3B, {}, 0),                         # hidden 3072
+    (configs.TINY, {}, 0),                             # 8 KB of FFN per block
+    (configs.TINY, dict(ffn_early_stages=2), 2),
+    (configs.LLAMA_1B, dict(ffn_early_stages=-1), 0),
+    (configs.LLAMA_1B, dict(split_ffn=1), 0),          # no fused FFN instruction
+    (configs.MIXTRAL_8L, {}, 0),                       # MoE: the routing gates the expert stream already
+    (configs.MIXTRAL_8L, dict(ffn_early_stages=1), 0),
+], ids=lambda x: getattr(x, "name", str(x)))
+def test_ffn_gate_marks(cfg, opts, expect):
+    # Every dense fused FFN instruction carries the gate (the stage from which the loader waits for the
+    # FFN's dependency); nothing else does, and it changes no other word and no counter increment.
+    words, n_instr, inc = dpb.plan(cfg, 148, **opts)
+    ops = words[:, :, W_OP]
+    ffn = ops == OP["FFN"]
+    assert np.all(words[:, :, W_GATE][ffn] == expect)
+    assert np.all(words[:, :, W_GATE][~ffn] == 0)
+    base, _, inc0 = dpb.plan(cfg, 148, **{**opts, "ffn_early_stages": -1})
+    w2 = words.copy()
+    w2[:, :, W_GATE] = 0
+    np.testing.assert_array_equal(w2, base)
+    np.testing.assert_array_equal(inc, inc0)
+
+
+def test_ffn_gate_option_is_checked():
+    for bad in (-2, 65):
+        with pytest.raises(mk.MkError) as e:
+            dpb.plan(configs.LLAMA_1B, 148, ffn_early_stages=bad)
+        assert e.value.name == "MK_ERR_INVALID_ARG"
