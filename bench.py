@@ -79,6 +79,9 @@ def parse():
     ap.add_argument("--attn-merge", type=int, default=0,
                     help="merge of the attention splits: 1 in every O-projection block, 2 once per kv head "
                          "(0: the library default)")
+    ap.add_argument("--ffn-early-stages", type=int, default=0,
+                    help="dense FFN stages the loader issues before the FFN's dependency is met (-1: no limit; "
+                         "0: the library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-baselines", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -312,6 +315,8 @@ def measure(args, cfg, p0, positions, K, Wm, rank, world, local, with_extras=Tru
         opts["spec_experts"] = args.spec_experts
     if args.attn_merge:
         opts["attn_merge"] = args.attn_merge
+    if args.ffn_early_stages:
+        opts["ffn_early_stages"] = args.ffn_early_stages
     calib = None
     if args.calibrate and args.mode == "megakernel":
         # start-up calibration, outside the timed region: a few traced steps from p0
