@@ -62,7 +62,8 @@ struct Misc {
     int pred_layer;    // route_key(epoch, layer) of the predicted experts in pred_eidx (-1: none)
     int pred_eidx[kMaxTopK];
     int is_last;
-    int pad[3];
+    int ffn_go;        // route_key(epoch, layer) of the last dense FFN whose dependency the consumers passed
+    int pad[2];
     // batched decode: every sequence's position and token of this step (token resolved: < 0 read
     // from the previous step's argmax)
     int bpos[kMaxBatch];
@@ -468,6 +469,29 @@ __device__ bool wait_misc_key(const DevParams& p, Misc& m, const int* field, int
     return true;
 }
 
+// Loader side of the FFN stage gate: wait (bounded) until this block's
+// consumers have passed the dense FFN's dependency and published its key.  The
+// loader polls shared memory, with a short sleep, instead of the global
+// counter: a second poller per block on the counter's line slowed the
+// consumers' own dependency polls on the neighbouring counters.
+__device__ bool wait_ffn_go(const DevParams& p, Misc& m, int key, int ii, int op) {
+    const uint64_t t0 = globaltimer_ns();
+    uint64_t next = t0 + kStopPollNs;
+    while (vload(&m.ffn_go) != key) {
+        __nanosleep(64);
+        const uint64_t now = globaltimer_ns();
+        if (now >= next) {
+            if (ld_relaxed_s32(&p.status->stop) || vload(&m.abort_flag)) return false;
+            if (now - t0 > p.spin_limit_ns) {
+                record_error(p.status, MK_ERR_TIMEOUT, blockIdx.x, ii, op, -1, 0, 0);
+                return false;
+            }
+            next = now + kStopPollNs;
+        }
+    }
+    return true;
+}
+
 // A fused MoE FFN slice's speculative stages hold the routed expert's rows:
 // the predicted and the routed experts of its slot are the same (both known).
 __device__ __forceinline__ bool spec_hit(const DevParams& p, const Misc& m, int sub) {
@@ -576,9 +600,8 @@ __device__ bool loader(const DevParams& p, const StepArgs& a, const int32_t* q, 
         bool ok = true;
         unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + i) * kTraceWords : nullptr;
         for (int st = st0; st < pl.n_stages; ++st, ++g) {
-            // gated FFN slice: the stages from W_GATE on wait for the FFN's own dependency
-            if (st == w[W_GATE] && st > 0 &&
-                !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], i, w[W_OP])) {
+            // gated FFN slice: the stages from W_GATE on wait until the consumers pass the FFN's dependency
+            if (st == w[W_GATE] && st > 0 && !wait_ffn_go(p, m, route_key(a.epoch, w[W_LAYER], p.L), i, w[W_OP])) {
                 ok = false;
                 break;
             }
@@ -1265,6 +1288,7 @@ __device__ bool ffn_instr(const DevParams& p, const StepArgs& a, const int32_t* 
 
     if (tid == 0) {
         if (!wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op)) vstore(&m.abort_flag, 1);
+        else if (op == OP_FFN) vstore(&m.ffn_go, route_key(a.epoch, l, p.L));  // the loader's gate
         if (tr) tr[T_DEP] = globaltimer_ns();
     }
     cbar();
@@ -2095,8 +2119,10 @@ __device__ bool ffn_instr_b(const DevParams& p, const StepArgs& a, const int32_t
     unsigned long long* tr = p.trace ? p.trace + ((size_t)blockIdx.x * p.max_instr + ii) * kTraceWords : nullptr;
     Plan pl;
     make_plan(p, a.pos, w, nullptr, pl);
-    if (tid == 0 && !wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op))
-        vstore(&m.abort_flag, 1);
+    if (tid == 0) {
+        if (!wait_counter(p, m, w[W_WAIT_CTR], a.epoch * (uint32_t)w[W_WAIT_INC], ii, op)) vstore(&m.abort_flag, 1);
+        else vstore(&m.ffn_go, route_key(a.epoch, l, p.L));  // the loader's gate
+    }
     if (tr && tid == 0) tr[T_DEP] = globaltimer_ns();
     cbar();
     if (vload(&m.abort_flag)) return false;
@@ -3182,6 +3208,7 @@ __global__ void __launch_bounds__(kThreads, 1) megakernel(const __grid_constant_
         m.router_layer = -1;
         m.pred_layer = -1;
         m.is_last = 0;
+        m.ffn_go = -1;
         m.abort_flag = ld_relaxed_s32(&p.status->stop) ? 1 : 0;
         if (m.abort_flag && atomicCAS(&p.status->code, 0, MK_ERR_STOPPED) == 0) p.status->sm = blockIdx.x;
         if constexpr (NB > 1) {  // every sequence's position and token (< 0: its previous argmax)
