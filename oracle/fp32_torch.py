@@ -1,10 +1,9 @@
 """Second, independent CPU restatement of the decode step in fp32 (torch CPU ops).
 
 TEST INFRASTRUCTURE ONLY.  It exists to measure the fp32-vs-fp64 noise floor
-(the Hyperkernel teardown, "Which claims the repo backs", judges agreement
+(the Hyperkernel teardown, "Which claims the repo backs", weighs agreement
 with an independent implementation against that implementation's own noise
-floor) and to cross-check the
-C oracle: it is written from the same plain decoder definition with torch
+floor) and to cross-check the C oracle: it is written from the same plain decoder definition with torch
 tensor ops, sharing no code with oracle.c.
 """
 from __future__ import annotations
